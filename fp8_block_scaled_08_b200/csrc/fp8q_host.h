@@ -1,0 +1,41 @@
+// Host-side helpers shared by the libfp8q translation units: argument checks,
+// device queries, TMA descriptor encoding and the device error word.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fp8q.h"
+
+namespace fp8q {
+
+// Address of the device error word on the current device (set up once per device).
+unsigned* device_error_word();
+
+// Streaming multiprocessor count of the current device; 0 if it is not sm_100.
+int sm100_sm_count();
+
+// 2D tiled tensor map (no multicast, no interleave). `inner`/`outer` are the tensor's
+// extents in elements, `row_bytes` the byte stride between rows. Returns false if
+// the driver entry point is missing or the encoding is rejected.
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                    uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                    uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Remembers the text of a failure for fp8q_last_error_message (thread-local).
+void set_last_error(const char* where, cudaError_t e);
+
+inline fp8q_status launch_status(const char* where = "launch") {
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return FP8Q_OK;
+  set_last_error(where, e);
+  return FP8Q_ERR_CUDA;
+}
+
+// Bounded waits inside the kernels give up after this long (nanoseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+}  // namespace fp8q

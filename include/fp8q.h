@@ -1,0 +1,172 @@
+/*
+ * fp8q.h — C ABI of libfp8q.so: the block-scaled FP8 linear layer on B200 (sm_100a).
+ *
+ * The operations are those of the quantization scheme in "Resumen Técnico: Jet-RL"
+ * (gist.science, paper 2601.14243), section "Esquema de Cuantización":
+ * activations quantized per 1x128 group, weights per 128x128 block, FP8
+ * activations saved for backward and produced by the preceding (fused) operator,
+ * BF16 gradients between operators, FP8 DGrad and WGrad (WGrad with 1x128 and
+ * 128x1 grouping). Section "Arquitectura Central" requires the forward GEMM to be
+ * the same for rollout and for the training forward pass.
+ *
+ * Number formats
+ *   FP8    OCP E4M3 "fn" (bias 7, max finite 448, no infinities), one byte per code.
+ *   scale  fp32. A group's scale is s = amax/448 (IEEE division); an all-zero group
+ *          has s = 1. A code is the E4M3 value nearest to x/s (IEEE division),
+ *          ties to even, saturating at +-448, sign kept (so -0 encodes as 0x80).
+ *   BF16   passed as uint16_t bit patterns.
+ *
+ * Layouts (row-major; "ld" is a row stride in elements)
+ *   codes         uint8_t [rows][cols], dense (row stride = cols).
+ *   1x128 scales  float [cols/128][lds]: scale of (row m, group g) at s[g*lds + m].
+ *                 lds >= rows, lds % 4 == 0 (the GEMMs load 128 row scales of one
+ *                 group as one contiguous 512-byte run).
+ *   128x128       float [N/128][K/128].
+ *   128x1 scales  float [rows/128][cols]: scale of (row group mb, column c) at
+ *                 s[mb*cols + c]; the codes of such groups are stored transposed.
+ *
+ * Conventions
+ *   - Every pointer is a DEVICE pointer owned by the caller; the library allocates
+ *     no device memory, keeps no per-call state and never synchronises the host.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Each call validates
+ *     its arguments synchronously, then enqueues one kernel on `stream`.
+ *   - Shapes: K (the grouped / reduction dimension) % 128 == 0 everywhere;
+ *     weight N % 128 == 0; M % 128 == 0 on the 128x1 paths; otherwise M >= 1.
+ *   - Alignment: every pointer 16-byte aligned; BF16 row strides % 8 == 0.
+ *   - No call aborts or throws; each returns an fp8q_status.
+ *   - Thread safety: re-entrant; calls on different streams may overlap.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int fp8q_status;
+#define FP8Q_OK 0
+#define FP8Q_ERR_NULL 1        /* a required pointer is NULL                        */
+#define FP8Q_ERR_SHAPE 2       /* a size is <= 0, not a multiple of 128 where
+                                  required, or a leading dimension is too small      */
+#define FP8Q_ERR_ALIGN 3       /* a pointer or row stride breaks 16-byte alignment   */
+#define FP8Q_ERR_CUDA 4        /* the launch failed (cudaGetLastError)               */
+#define FP8Q_ERR_TIMEOUT 5     /* a kernel gave up a bounded wait (device error word) */
+#define FP8Q_ERR_UNSUPPORTED 6 /* no sm_100 device / driver entry point missing     */
+
+/* Human-readable name of a status code (static storage). */
+const char* fp8q_status_string(fp8q_status status);
+
+/* Text of the last CUDA error seen by a call on this host thread (FP8Q_ERR_CUDA or
+ * FP8Q_ERR_UNSUPPORTED), or "" if none. Static thread-local storage. */
+const char* fp8q_last_error_message(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int fp8q_version(void);
+
+/* Synchronises `stream`, then reads the device error word that kernels set when a
+ * bounded wait gives up (FP8Q_ERR_TIMEOUT) and, if `clear` != 0, resets it.
+ * Returns FP8Q_OK when no kernel reported an error. For tests and diagnostics. */
+fp8q_status fp8q_device_error(void* stream, int clear);
+
+/* a1. Activation quantization per 1x128 group ("Esquema de Cuantización",
+ * activations bullet).
+ *   x  [M][K] BF16, row stride ldx (>= K, % 8 == 0)
+ *   q  [M][K] FP8 codes (dense)        s [K/128][lds] fp32 (1x128 layout)
+ * Requires M >= 1, K % 128 == 0. */
+fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                 uint8_t* q, float* s, int64_t lds, void* stream);
+
+/* a2. Weight quantization per 128x128 block ("Esquema de Cuantización", weights
+ * bullet). Run once per optimizer step from the BF16 master weights
+ * ("Arquitectura Central", master weights bullet).
+ *   w  [N][K] BF16, row stride ldw     q [N][K] codes   s [N/128][K/128] fp32
+ *   qT [K][N] codes: the same codes transposed (the DGrad operand); may be NULL.
+ * Requires N % 128 == 0, K % 128 == 0. */
+fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                                      uint8_t* q, float* s, uint8_t* qT, void* stream);
+
+/* a3. RMSNorm fused with 1x128 quantization: the FP8 saved activation produced by
+ * the preceding operator ("Esquema de Cuantización", saved-activations bullet;
+ * "Implementación", fused RMSNorm kernels).
+ *   y_i = bf16( fl32( fl32(x_i * r) * gamma_i ) ),
+ *   r   = (float)(1 / sqrt(sum_i x_i^2 / H + eps)) computed in fp64,
+ * then the 1x128 quantization of y.
+ *   x [M][H] BF16 (row stride ldx), gamma [H] BF16, q [M][H], s [H/128][lds].
+ * Requires H % 128 == 0 and H <= 16384. */
+fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, int64_t M,
+                               int64_t H, int64_t ldx, float eps, uint8_t* q, float* s,
+                               int64_t lds, void* stream);
+
+/* a4. SwiGLU fused with 1x128 quantization ("Implementación", fused activation
+ * kernels). gu [M][2I] BF16 holds the gate in columns 0..I-1 and the up projection
+ * in I..2I-1 (row stride ldgu >= 2I):
+ *   h = bf16( fl32( fl32(g / fl32(1 + E(-g))) * u ) ),
+ * with E the library's fixed fp32 exponential (Cody-Waite range reduction and a
+ * degree-7 Taylor polynomial, argument clamped to [-80, 88]), then the 1x128
+ * quantization of h:  q [M][I], s [I/128][lds].   Requires I % 128 == 0. */
+fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t I, int64_t ldgu,
+                              uint8_t* q, float* s, int64_t lds, void* stream);
+
+/* a6. The BF16 gradient dY quantized for both backward GEMMs in one pass
+ * ("Esquema de Cuantización", backward bullets; "Implementación", transposition):
+ *   row-wise 1x128 for DGrad:  q_row [M][N], s_row [N/128][lds_row]  (may be NULL)
+ *   column-wise 128x1 for WGrad, stored transposed: q_colT [N][M], s_col [M/128][N].
+ *   dy [M][N] BF16, row stride lddy.  Requires M % 128 == 0, N % 128 == 0. */
+fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, int64_t N,
+                                      int64_t lddy, uint8_t* q_row, float* s_row,
+                                      int64_t lds_row, uint8_t* q_colT, float* s_col,
+                                      void* stream);
+
+/* a8. The saved FP8 activation (1x128 groups) re-grouped 128x1 for WGrad:
+ * xhat = fl32(s * dec(q)), then 128x1 quantization along M, stored transposed.
+ *   q [M][K] codes, s [K/128][lds]  ->  qT [K][M] codes, sT [M/128][K].
+ * Requires M % 128 == 0, K % 128 == 0. */
+fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s, int64_t M,
+                                     int64_t K, int64_t lds, uint8_t* qT, float* sT,
+                                     void* stream);
+
+/* a5. Forward GEMM, shared by rollout and the training forward pass
+ * ("Arquitectura Central"; "Esquema de Cuantización"):
+ *   Y[m,n] = sum_kb  sa[kb][m] * sw[n/128][kb] * sum_{k in kb} qa[m,k] * qw[n,k]
+ * accumulated in fp32 one 128-wide K slice at a time, in increasing kb, then
+ * rounded to BF16. Row m of Y does not depend on M (batch invariant).
+ *   qa [M][K], sa [K/128][ldsa], qw [N][K], sw [N/128][K/128], y [M][N] BF16 (ldy).
+ * Requires N % 128 == 0, K % 128 == 0, M >= 1. */
+fp8q_status fp8q_linear_fwd(const uint8_t* qa, const float* sa, int64_t ldsa,
+                            const uint8_t* qw, const float* sw, int64_t M, int64_t N,
+                            int64_t K, uint16_t* y, int64_t ldy, void* stream);
+
+/* a7. DGrad in FP8 ("Esquema de Cuantización", backward GEMMs):
+ *   dX[m,k] = sum_nb sdy[nb][m] * sw[nb][k/128] * sum_{n in nb} qdy[m,n] * qw[n,k]
+ * with the row-wise dY codes of fp8q_transpose_quant_bf16 and the transposed
+ * weight codes qwT [K][N] of fp8q_quant_weight_128x128.
+ *   qdy [M][N], sdy [N/128][ldsdy], qwT [K][N], sw [N/128][K/128], dx [M][K] (lddx).
+ * Requires N % 128 == 0, K % 128 == 0, M >= 1. */
+fp8q_status fp8q_linear_dgrad(const uint8_t* qdy, const float* sdy, int64_t ldsdy,
+                              const uint8_t* qwT, const float* sw, int64_t M, int64_t N,
+                              int64_t K, uint16_t* dx, int64_t lddx, void* stream);
+
+/* a9. WGrad in FP8 with 1x128 / 128x1 grouping ("Esquema de Cuantización"): both
+ * operands grouped along the reduction dimension M (tokens):
+ *   dW[n,k] = sum_mb sdy_c[mb][n] * sx_c[mb][k] * sum_{m in mb} qdyT[n,m] * qxT[k,m]
+ *   qdyT [N][M], sdy_c [M/128][N] (from fp8q_transpose_quant_bf16),
+ *   qxT [K][M], sx_c [M/128][K] (from fp8q_transpose_quant_fp8), dw [N][K] BF16 (lddw).
+ * Requires M % 128 == 0, N % 128 == 0, K % 128 == 0. */
+fp8q_status fp8q_linear_wgrad(const uint8_t* qdyT, const float* sdy_c, const uint8_t* qxT,
+                              const float* sx_c, int64_t M, int64_t N, int64_t K,
+                              uint16_t* dw, int64_t lddw, void* stream);
+
+/* Diagnostic: launches one CTA that waits on a barrier nothing completes, with a
+ * wait limit of `limit_ns` nanoseconds, exactly as the GEMM's bounded waits do.
+ * The kernel gives up, records FP8Q_ERR_TIMEOUT in the device error word and
+ * returns; the caller reads it with fp8q_device_error. Used by the tests of the
+ * failure path; it faults nothing and leaves the context usable. */
+fp8q_status fp8q_debug_wait_timeout(int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */
