@@ -387,6 +387,70 @@ def run_reference(args, rank, world):
 
 
 # --------------------------------------------------------------------------
+# Single-kernel cases (for profilers): one kernel of the layer on its real shape,
+# with only the buffers it needs on the device.
+# --------------------------------------------------------------------------
+
+CASES = ("gemm_fwd", "gemm_dgrad", "gemm_wgrad", "quantizers")
+
+
+def run_case(name, reps):
+    import fp8_block_scaled_08_b200 as fq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = WORKLOAD
+    M = wl.tokens
+    lin = wl.layer.linears[2]  # gate/up: N = 28672, K = 4096 (the largest linear)
+    N, K = lin.n, lin.k
+    w = workloads.normal_bf16((N, K), wl.w_std, wl.seed, workloads.TID_W[lin.name], dev)
+    if name == "gemm_fwd":
+        x = workloads.activations_bf16((M, K), wl.seed, workloads.TID_X_MLP, dev,
+                                       outlier_frac=wl.act_outlier_frac,
+                                       outlier_scale=wl.act_outlier_scale)
+        qx, sx = fq.quant_act_1x128_alloc(x)
+        qw, sw, _ = fq.quant_weight_alloc(w, want_t=False)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.linear_fwd(qx, sx, qw, sw, y)  # noqa: E731
+    elif name == "gemm_dgrad":
+        dy = workloads.gradients_bf16((M, N), wl.dy_std, wl.seed, workloads.TID_DY[lin.name], dev)
+        qdy, sdy = fq.quant_act_1x128_alloc(dy)
+        _, sw, qwT = fq.quant_weight_alloc(w)
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.linear_dgrad(qdy, sdy, qwT, sw, dx)  # noqa: E731
+    elif name == "gemm_wgrad":
+        x = workloads.activations_bf16((M, K), wl.seed, workloads.TID_X_MLP, dev)
+        dy = workloads.gradients_bf16((M, N), wl.dy_std, wl.seed, workloads.TID_DY[lin.name], dev)
+        qx, sx = fq.quant_act_1x128_alloc(x)
+        qxT, sxT = fq.transpose_quant_fp8_alloc(qx, sx)
+        _, _, qdyT, sdyc = fq.transpose_quant_bf16_alloc(dy, want_row=False)
+        dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.linear_wgrad(qdyT, sdyc, qxT, sxT, dw)  # noqa: E731
+    elif name == "quantizers":
+        x = workloads.activations_bf16((M, K), wl.seed, workloads.TID_X_MLP, dev)
+        g = workloads.gamma_bf16(K, wl.seed, workloads.TID_GAMMA2, dev)
+        dy = workloads.gradients_bf16((M, N), wl.dy_std, wl.seed, workloads.TID_DY[lin.name], dev)
+        q, s = fq.quant_act_1x128_alloc(x)
+
+        def fn():
+            fq.quant_act_1x128_alloc(x)
+            fq.rmsnorm_quant_alloc(x, g, wl.eps)
+            fq.swiglu_quant_alloc(dy)
+            fq.quant_weight_alloc(w)
+            fq.transpose_quant_bf16_alloc(dy)
+            fq.transpose_quant_fp8_alloc(q, s)
+    else:
+        raise SystemExit("unknown case %r (choose from %s)" % (name, ", ".join(CASES)))
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        fn()
+    torch.cuda.synchronize()
+    if fq.device_error() != fq.FP8Q_OK:
+        raise RuntimeError("device error in case %s" % name)
+    print("case %s: %d repetitions OK" % (name, reps))
+    return 0
+
+
+# --------------------------------------------------------------------------
 # Our arm
 # --------------------------------------------------------------------------
 
@@ -398,7 +462,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="run one kernel of the layer on its real shape (for profilers)")
+    ap.add_argument("--case-reps", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        return run_case(args.case, args.case_reps)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

@@ -19,21 +19,30 @@
 // is the same whatever M is (the rollout and the training forward share numerics,
 // "Arquitectura Central").
 //
-// Kernel structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
-//   warp 0      TMA producer: A/B tiles into a 4-stage shared-memory ring (128-byte
-//               swizzle) and the scale vectors into an 8-slot ring.
-//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (kind::f8f6f4, 128x256x32, 4 per slice) into TMEM buffer r%2 and
-//               commits to mbarriers that free the smem stage / publish the slice.
+// Kernel structure. CTAs run in pairs (a cluster of 2 on neighbouring SMs) that share
+// one 256x256 output tile: each CTA loads its own 128 rows of A and its own 128 rows
+// of B (no multicast), and the leader CTA issues tcgen05.mma.cta_group::2 (M = 256,
+// N = 256, K = 32; 4 per slice) that reads both CTAs' shared memory and writes
+// 128 x 256 fp32 into each CTA's TMEM. Per 128-wide slice each SM therefore moves
+// 32 KB in (TMA) and 32 KB out (tensor-core reads) of shared memory instead of 48 + 48
+// KB with single-CTA 128x256 tiles, which keeps shared-memory bandwidth below the
+// tensor core's demand. 384 threads per CTA:
+//   warp 0      TMA producer: its A/B halves into a 4-stage ring (128-byte swizzle),
+//               completing on the leader's barrier; its scale vectors into an 8-slot
+//               ring.
+//   warp 1      allocates 512 TMEM columns (both CTAs); in the leader, one thread
+//               issues the pair MMAs into TMEM buffer r%2 and commits to barriers in
+//               both CTAs that free the smem stage / publish the slice.
 //   warps 2, 3  idle. Warpgroup 0 (warps 0-3) hands registers to the others.
-//   warps 4..11 two warpgroups; warpgroup h promotes columns 128h..128h+127 of the
-//               128x256 tile: tcgen05.ld, packed fp32 FMA into 128 registers per
-//               thread, release the TMEM buffer; after the last slice they round to
-//               BF16 and store the tile.
+//   warps 4..11 two warpgroups; warpgroup h promotes columns 128h..128h+127 of this
+//               CTA's 128 x 256 part: tcgen05.ld, packed fp32 FMA into 128 registers
+//               per thread, release the TMEM buffer (the peer's warps arrive on the
+//               leader's barrier); after the last slice they round to BF16, stage the
+//               rows in shared memory (128-byte swizzle) and store them with TMA.
 // Registers: the block launches with 168 per thread (168 x 384 = 64512); warpgroup
 // 0 drops to 40 and the promotion warpgroups rise to 232 (40*128 + 232*256 = 64512).
 // Every mbarrier wait is bounded (kWaitLimitNs): a wait that gives up records
-// FP8Q_ERR_TIMEOUT in the device error word and the CTA winds down cleanly.
+// FP8Q_ERR_TIMEOUT in the device error word and both CTAs wind down.
 #include <algorithm>
 
 #include "fp8q_device.cuh"
@@ -42,7 +51,10 @@
 namespace fp8q {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int BM = 128;        // rows of the tile per CTA (the pair covers 256)
+constexpr int BN = 256;        // columns of the tile (each CTA loads 128 rows of B)
+constexpr int BK = 128;        // one scale slice
+constexpr int kPairM = 2 * BM;
 constexpr int kStages = 4;
 constexpr int kScStages = 8;
 constexpr int kThreads = 384;
@@ -53,22 +65,28 @@ static_assert(kRegsControl * 128 + kRegsPromote * 256 <= kRegsLaunch * kThreads,
               "register hand-over exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;  // two 128x256 fp32 accumulators
 constexpr uint32_t kABytes = BM * BK;
-constexpr uint32_t kBBytes = BN * BK;
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kBBytes = (BN / 2) * BK;
+constexpr uint32_t kStageBytes = kABytes + kBBytes;  // per CTA
 constexpr uint32_t kScABytes = BM * 4;
 constexpr uint32_t kScBBytes = BN * 4;
 constexpr uint32_t kScSlot = kScABytes + kScBBytes;
+constexpr uint32_t kStageOutBytes = 32 * 64 * 2;  // one 32-row x 64-column BF16 box
 
 __host__ __device__ constexpr uint32_t kOffA(int s) { return s * kStageBytes; }
 __host__ __device__ constexpr uint32_t kOffB(int s) { return s * kStageBytes + kABytes; }
 __host__ __device__ constexpr uint32_t kOffScA(int i) { return kStages * kStageBytes + i * kScSlot; }
 __host__ __device__ constexpr uint32_t kOffScB(int i) { return kOffScA(i) + kScABytes; }
-constexpr uint32_t kOffBars = kStages * kStageBytes + kScStages * kScSlot;
+constexpr uint32_t kOffOut = kStages * kStageBytes + kScStages * kScSlot;  // 8 warps x 2 boxes
+__host__ __device__ constexpr uint32_t kOffOutBox(int w, int j) {
+  return kOffOut + (2 * w + j) * kStageOutBytes;
+}
+constexpr uint32_t kOffBars = kOffOut + 16 * kStageOutBytes;
 constexpr uint32_t kNumBars = 2 * kStages + 4 + 2 * kScStages + 1;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
 static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+static_assert(kOffOut % 1024 == 0, "TMA store boxes need 1024-byte alignment");
 
 struct GemmParams {
   int32_t M, N, K;
@@ -102,19 +120,19 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 }
 
 template <bool kColScaleB>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                const GemmParams p) {
+                const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
-  uint64_t* full = bars;
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* sfull = tempty + 2;
+  uint64_t* full = bars;              // leader: both CTAs' A/B bytes of a stage
+  uint64_t* empty = full + kStages;   // both: stage consumed by the pair MMAs
+  uint64_t* tfull = empty + kStages;  // both: slice accumulator ready in TMEM
+  uint64_t* tempty = tfull + 2;       // leader: both CTAs' promotion warps done with it
+  uint64_t* sfull = tempty + 2;       // local scale ring
   uint64_t* sempty = sfull + kScStages;
   uint64_t* done = sempty + kScStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -122,6 +140,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -130,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, 8);  // the 8 promotion warps
+      mbar_init(tempty + b, 16);  // 8 promotion warps in each CTA of the pair
     }
     for (int i = 0; i < kScStages; ++i) {
       mbar_init(sfull + i, 1);
@@ -144,11 +165,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmSA);
+    prefetch_tensormap(&tmY);
     if (kColScaleB) prefetch_tensormap(&tmSB);
   }
-  if (warp == 1) tmem_alloc<kTmemCols>(tmem_slot);
+  if (warp == 1) tmem_alloc_pair<kTmemCols>(tmem_slot);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.err, p.wait_limit_ns};
@@ -165,19 +187,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // bit s of issued/par: stage s has a load in flight or done, and its phase parity
       uint32_t issued = 0, par = 0, sc_issued = 0, sc_par = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int t = pair; ok && t < num_tiles; t += npairs) {
         int mb, nb;
         tile_coords(t, p, mb, nb);
+        const int row0 = mb * kPairM + static_cast<int>(rank) * BM;
+        const int brow0 = nb * BN + static_cast<int>(rank) * (BN / 2);
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1, ctl)) { ok = false; break; }
-          mbar_arrive_expect_tx(full + stage, kStageBytes);
-          tma_load_2d(smem + kOffA(stage), &tmA, kb * BK, mb * BM, full + stage);
-          tma_load_2d(smem + kOffB(stage), &tmB, kb * BK, nb * BN, full + stage);
+          if (rank == 0) mbar_arrive_expect_tx(full + stage, 2 * kStageBytes);
+          const uint32_t leader_full = cluster_addr(full + stage, 0);
+          tma_load_2d_pair(smem + kOffA(stage), &tmA, kb * BK, row0, leader_full);
+          tma_load_2d_pair(smem + kOffB(stage), &tmB, kb * BK, brow0, leader_full);
           issued |= 1u << stage;
           par = (par & ~(1u << stage)) | (phase << stage);
           if (!mbar_wait(sempty + sci, scph ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(sfull + sci, kScABytes + (kColScaleB ? kScBBytes : 0u));
-          tma_load_2d(smem + kOffScA(sci), &tmSA, mb * BM, kb, sfull + sci);
+          tma_load_2d(smem + kOffScA(sci), &tmSA, row0, kb, sfull + sci);
           if (kColScaleB) tma_load_2d(smem + kOffScB(sci), &tmSB, nb * BN, kb, sfull + sci);
           sc_issued |= 1u << sci;
           sc_par = (sc_par & ~(1u << sci)) | (scph << sci);
@@ -186,20 +211,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {  // let every copy already issued land before the CTA exits
-        for (int s = 0; s < kStages; ++s)
-          if ((issued >> s) & 1u) mbar_wait_drain(full + s, (par >> s) & 1u, p.wait_limit_ns);
+        if (rank == 0)
+          for (int s = 0; s < kStages; ++s)
+            if ((issued >> s) & 1u) mbar_wait_drain(full + s, (par >> s) & 1u, p.wait_limit_ns);
         for (int i = 0; i < kScStages; ++i)
           if ((sc_issued >> i) & 1u) mbar_wait_drain(sfull + i, (sc_par >> i) & 1u, p.wait_limit_ns);
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_e4m3_f32(BM, BN);
+   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_e4m3_f32(kPairM, BN);
       uint32_t stage = 0, phase = 0, it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int t = pair; ok && t < num_tiles; t += npairs) {
         for (int kb = 0; kb < p.kblocks; ++kb) {
           const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
           if (!mbar_wait(tempty + buf, tph ^ 1u, ctl)) { ok = false; break; }
@@ -210,16 +236,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t d = tmem_base + buf * BN;
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)
-            mma_f8f6f4(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc,
-                       k > 0 ? 1u : 0u);
-          mma_commit(empty + stage);
-          mma_commit(tfull + buf);
+            mma_f8f6f4_pair(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k),
+                            idesc, k > 0 ? 1u : 0u);
+          mma_commit_pair_multicast(empty + stage, 0x3);
+          mma_commit_pair_multicast(tfull + buf, 0x3);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
           ++it;
         }
       }
-      // wait for every MMA this thread issued (they read smem and write TMEM)
-      mma_commit(done);
+      // wait for every MMA issued (they read both CTAs' smem and write both TMEMs)
+      mma_commit_pair_multicast(done, 0x1);
       mbar_wait_drain(done, 0, p.wait_limit_ns);
     }
     __syncwarp();
@@ -230,104 +256,134 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;           // TMEM lane quarter this warp may access
     const int half = (warp - 4) >> 2;  // column half of the 256-wide tile
     const int row = wq * 32 + lane;
+    const uint32_t tempty_leader0 = cluster_addr(tempty, 0);
+    uint8_t* out0 = smem + kOffOutBox(warp - 4, 0);
+    uint8_t* out1 = smem + kOffOutBox(warp - 4, 1);
     uint32_t it = 0, sci = 0, scph = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+    bool ok = true, stored = false;
+    for (int t = pair; ok && t < num_tiles; t += npairs) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
-      const int ncol0 = nb * BN + half * BM;
+      const int row0 = mb * kPairM + static_cast<int>(rank) * BM;
+      const int ncol0 = nb * BN + half * 128;
       const bool col_ok = ncol0 < p.N;
       const float* sbp = kColScaleB ? nullptr : p.sb + static_cast<int64_t>(ncol0 / 128) * p.sb_sj;
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      // block scale of the next slice, loaded one slice ahead
+      float sb_next = (!kColScaleB && col_ok) ? __ldg(sbp) : 0.0f;
       for (int kb = 0; kb < p.kblocks; ++kb) {
-        float sbv = 0.0f;
-        if (!kColScaleB && col_ok) sbv = __ldg(sbp + kb * p.sb_sr);
+        const float sbv = sb_next;
+        if (!kColScaleB && col_ok && kb + 1 < p.kblocks) sb_next = __ldg(sbp + (kb + 1) * p.sb_sr);
         if (!mbar_wait_warp(sfull + sci, scph, ctl)) { ok = false; break; }
         const float sa = reinterpret_cast<const float*>(smem + kOffScA(sci))[row];
+        const float4* scb4 =
+            reinterpret_cast<const float4*>(smem + kOffScB(sci)) + half * 32;  // col scales
         const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
         if (!mbar_wait_warp(tfull + buf, tph, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr =
-            tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + buf * BN + half * BM;
-        if (!kColScaleB) {
-          const float s = __fmul_rn(sa, sbv);
+            tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + buf * BN + half * 128;
+        const float s = __fmul_rn(sa, sbv);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {  // two 64-column halves, two loads in flight
-            uint32_t r[64];
-            tmem_ld32(taddr + c * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-            tmem_ld32(taddr + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-            tmem_wait_ld();
+        for (int c = 0; c < 2; ++c) {  // two 64-column halves, two loads in flight
+          uint32_t r[64];
+          tmem_ld32(taddr + c * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(taddr + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_wait_ld();
+          if (!kColScaleB) {
 #pragma unroll
             for (int i = 0; i < 64; i += 2)
               fma2(acc[c * 64 + i], acc[c * 64 + i + 1], __uint_as_float(r[i]),
                    __uint_as_float(r[i + 1]), s, s);
-          }
-        } else {
-          const float* scb = reinterpret_cast<const float*>(smem + kOffScB(sci)) + half * BM;
+          } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {  // four 32-column quarters, one load in flight
-            uint32_t r[32];
-            tmem_ld32(taddr + c * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const float2 sb2 = *reinterpret_cast<const float2*>(scb + c * 32 + i);
-              float s0, s1;
-              mul2(s0, s1, sa, sa, sb2.x, sb2.y);
-              fma2(acc[c * 32 + i], acc[c * 32 + i + 1], __uint_as_float(r[i]),
+            for (int i = 0; i < 64; i += 4) {
+              const float4 sb4 = scb4[c * 16 + i / 4];
+              float s0, s1, s2, s3;
+              mul2(s0, s1, sa, sa, sb4.x, sb4.y);
+              mul2(s2, s3, sa, sa, sb4.z, sb4.w);
+              fma2(acc[c * 64 + i], acc[c * 64 + i + 1], __uint_as_float(r[i]),
                    __uint_as_float(r[i + 1]), s0, s1);
+              fma2(acc[c * 64 + i + 2], acc[c * 64 + i + 3], __uint_as_float(r[i + 2]),
+                   __uint_as_float(r[i + 3]), s2, s3);
             }
           }
         }
+        // hand the TMEM buffer and the scale slot back (measured: releasing the buffer
+        // between the two halves instead is slower, it keeps the loads from being
+        // scheduled ahead of the first half's FMAs)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(tempty + buf);
+          if (rank == 0) mbar_arrive(tempty + buf);
+          else mbar_arrive_cluster(tempty_leader0 + buf * 8);
           mbar_arrive(sempty + sci);
         }
         ++it;
         if (++sci == kScStages) { sci = 0; scph ^= 1; }
       }
       if (!ok) break;
-      const int64_t m = static_cast<int64_t>(mb) * BM + row;
-      if (m < p.M && col_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(p.y + m * p.ldy + ncol0);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          uint4 v;
-          v.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
-          v.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
-          v.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
-          v.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
-          dst[c] = v;
+      // epilogue: BF16 rows into this warp's two swizzled 32 x 64 boxes, then TMA stores
+      const int wrow0 = row0 + wq * 32;
+      if (col_ok && wrow0 < p.M) {
+        if (stored) {  // the previous tile's stores must have read the boxes
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
         }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          uint8_t* box = j ? out1 : out0;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float* a = acc + j * 64 + c * 8;
+            uint4 v;
+            v.x = pack_bf16x2(a[0], a[1]);
+            v.y = pack_bf16x2(a[2], a[3]);
+            v.z = pack_bf16x2(a[4], a[5]);
+            v.w = pack_bf16x2(a[6], a[7]);
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, out0, ncol0, wrow0);
+          tma_store_2d(&tmY, out1, ncol0 + 64, wrow0);
+          tma_store_commit();
+        }
+        stored = true;
       }
     }
+    if (stored && lane == 0) tma_store_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 1) {
-    __syncwarp();
     tc_fence_after();
-    tmem_dealloc<kTmemCols>(tmem_base);
+    tmem_dealloc_pair<kTmemCols>(tmem_base);
   }
 }
 
+// Per device and kernel variant: opt in to the shared memory, check the register
+// budget of the hand-over, and find how many CTA pairs can be resident at once (pairs
+// are placed within one GPC, so this can be below half the SM count). Returns that
+// number, or 0 on failure (the reason is in fp8q_last_error_message).
 template <bool kCol>
-bool ensure_smem_attr() {
-  static int done_for_device[64] = {0};
+int kernel_setup() {
+  static int pairs_for_device[64] = {0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (done_for_device[dev]) return true;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (pairs_for_device[dev]) return pairs_for_device[dev];
   const cudaError_t e = cudaFuncSetAttribute(
       gemm_kernel<kCol>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) {
     set_last_error("cudaFuncSetAttribute(gemm max dynamic smem)", e);
     cudaGetLastError();
-    return false;
+    return 0;
   }
   // The register hand-over inside the kernel waits until the block's launch allocation
   // covers the new budgets; refuse to launch a build whose allocation would not.
@@ -336,15 +392,33 @@ bool ensure_smem_attr() {
   if (ea != cudaSuccess) {
     set_last_error("cudaFuncGetAttributes(gemm)", ea);
     cudaGetLastError();
-    return false;
+    return 0;
   }
   if (static_cast<uint32_t>(attr.numRegs) * kThreads < kRegsControl * 128 + kRegsPromote * 256 ||
       attr.maxThreadsPerBlock < kThreads) {
     set_last_error("gemm register budget check", cudaErrorLaunchOutOfResources);
-    return false;
+    return 0;
   }
-  done_for_device[dev] = 1;
-  return true;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 74, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  const cudaError_t eo = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<kCol>, &cfg);
+  if (eo != cudaSuccess || clusters <= 0) {
+    set_last_error("cudaOccupancyMaxActiveClusters(gemm)", eo != cudaSuccess ? eo : cudaErrorInvalidConfiguration);
+    cudaGetLastError();
+    return 0;
+  }
+  pairs_for_device[dev] = clusters;
+  return clusters;
 }
 
 // out [Mg][Ng] = A [Mg][Kg] x B [Ng][Kg]^T with the scales described above.
@@ -356,10 +430,12 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   const int sms = sm100_sm_count();
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
   if (Mg > 0x7FFFFFFF || Ng > 0x7FFFFFFF || Kg > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  CUtensorMap tmA, tmB, tmSA, tmSB;
+  CUtensorMap tmA, tmB, tmSA, tmSB, tmY;
   bool ok = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, Kg, Mg, Kg, BK, BM,
                            CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, Kg, Ng, Kg, BK, BN,
+            encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, Kg, Ng, Kg, BK, BN / 2,
+                           CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, Ng, Mg, ldy * 2, 64, 32,
                            CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_tmap_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, Mg, Kg / BK, ldsa * 4, BM,
                            1, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -369,13 +445,14 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   else
     tmSB = tmSA;
   if (!ok) return FP8Q_ERR_UNSUPPORTED;
-  if (!ensure_smem_attr<kCol>()) return FP8Q_ERR_CUDA;
+  const int max_pairs = kernel_setup<kCol>();
+  if (max_pairs <= 0) return FP8Q_ERR_CUDA;
 
   GemmParams p;
   p.M = static_cast<int32_t>(Mg);
   p.N = static_cast<int32_t>(Ng);
   p.K = static_cast<int32_t>(Kg);
-  p.mblocks = static_cast<int32_t>((Mg + BM - 1) / BM);
+  p.mblocks = static_cast<int32_t>((Mg + kPairM - 1) / kPairM);
   p.nblocks = static_cast<int32_t>((Ng + BN - 1) / BN);
   p.kblocks = static_cast<int32_t>(Kg / BK);
   p.n_fastest = Ng <= Mg ? 1 : 0;
@@ -389,8 +466,8 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   if (!p.err) return FP8Q_ERR_CUDA;
   const int64_t tiles = static_cast<int64_t>(p.mblocks) * p.nblocks;
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
-  gemm_kernel<kCol><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmSA, tmSB, p);
+  const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, max_pairs));
+  gemm_kernel<kCol><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmSA, tmSB, tmY, p);
   return launch_status("gemm_kernel launch");
 }
 

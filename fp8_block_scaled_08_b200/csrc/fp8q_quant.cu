@@ -3,11 +3,16 @@
 // dual (row 1x128 + transposed column 128x1) quantizer of BF16 gradients and the
 // transposed 128x1 requantizer of saved FP8 activations.
 //
-// All of them are HBM-bound: BF16 is read with 16-byte loads that a warp issues
-// as contiguous 512-byte runs, group maxima are taken with warp shuffles, and the
-// codes come from the hardware E4M3 conversion (round to nearest even, saturate).
-// Scale and quotient use IEEE division (div.rn) so that codes are a function of the
-// inputs alone: s = amax/448 (s = 1 for an all-zero group), code = E4M3(x/s).
+// All of them are HBM-bound: BF16 is read with 16-byte loads that a warp issues as
+// contiguous runs, group maxima are taken with warp shuffles, and the codes come from
+// the hardware E4M3 conversion (round to nearest even, saturate). A group's scale is
+// s = amax/448 by IEEE division (s = 1 for an all-zero group); each code is the E4M3
+// value nearest to the IEEE quotient x/s. Where x is a BF16 value (every quantizer
+// but the FP8 requantizer) the quotient is formed from the correctly rounded
+// reciprocal r = 1/s with one residual correction (q = x*r; e = fma(-q, s, x);
+// q = fma(e, r, q); sign of x), which yields the same E4M3 code as the IEEE quotient
+// for every BF16 x and every BF16 amax >= |x| with s >= 2^-80 (checked exhaustively by
+// the test suite); groups with smaller s use the IEEE division itself.
 //
 // Method: "Resumen Técnico: Jet-RL" (gist.science, paper 2601.14243), section
 // "Esquema de Cuantización" (1x128 activation groups, 128x128 weight blocks,
@@ -24,25 +29,65 @@ namespace fp8q {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr float kSmallScale = 0x1p-80f;  // below it the quotient uses IEEE division
 
 // ---------------------------------------------------------------------------
-// One 1x128 group held by a half-warp: 16 lanes x 8 values.
-// Returns the group scale; writes the 8 codes of this lane to `codes`.
-// All 32 lanes must call it (the shuffles use the full mask).
+// Group scale and quotient
 // ---------------------------------------------------------------------------
+struct GroupScale {
+  float s, rs;
+  bool small;
+};
+
+__device__ __forceinline__ GroupScale group_scale(float amax) {
+  GroupScale g;
+  g.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+  g.rs = __frcp_rn(g.s);
+  g.small = g.s < kSmallScale;
+  return g;
+}
+
+__device__ __forceinline__ float copy_sign(float v, float sgn) {
+  return __uint_as_float((__float_as_uint(v) & 0x7FFFFFFFu) | (__float_as_uint(sgn) & 0x80000000u));
+}
+
+// Two quotients x/s of BF16-valued x (see the file header for why this equals the
+// IEEE quotient's code).
+__device__ __forceinline__ void quotient2(float x0, float x1, const GroupScale& g, float& t0,
+                                          float& t1) {
+  if (g.small) {
+    t0 = __fdiv_rn(x0, g.s);
+    t1 = __fdiv_rn(x1, g.s);
+    return;
+  }
+  float q0, q1;
+  mul2(q0, q1, x0, x1, g.rs, g.rs);      // q = x * r
+  float e0 = x0, e1 = x1;
+  fma2(e0, e1, -q0, -q1, g.s, g.s);      // e = fma(-q, s, x), exact
+  fma2(q0, q1, e0, e1, g.rs, g.rs);      // q = fma(e, r, q)
+  t0 = copy_sign(q0, x0);
+  t1 = copy_sign(q1, x1);
+}
+
+// Eight codes of BF16-valued x (packed little-endian into two words).
+__device__ __forceinline__ uint2 codes8(const float (&v)[8], const GroupScale& g) {
+  float t[8];
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) quotient2(v[i], v[i + 1], g, t[i], t[i + 1]);
+  return make_uint2(cvt_e4m3x4(t[0], t[1], t[2], t[3]), cvt_e4m3x4(t[4], t[5], t[6], t[7]));
+}
+
+// One 1x128 group held by a half-warp: 16 lanes x 8 values. Returns the group scale;
+// writes the 8 codes of this lane. All 32 lanes must call it (full-mask shuffles).
 __device__ __forceinline__ float quant_half_warp(const float (&v)[8], uint2& codes) {
   float a = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
 #pragma unroll
   for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
-  const float s = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 448.0f);
-  float t[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = __fdiv_rn(v[i], s);
-  codes.x = cvt_e4m3x4(t[0], t[1], t[2], t[3]);
-  codes.y = cvt_e4m3x4(t[4], t[5], t[6], t[7]);
-  return s;
+  const GroupScale g = group_scale(a);
+  codes = codes8(v, g);
+  return g.s;
 }
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4& r, float (&v)[8]) {
@@ -67,33 +112,56 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 // e^r in Horner form with fused multiply-adds, scaled by 2^n. The argument is
 // clamped to [-80, 88], where 2^n stays a normal number; below -80, 1 + e^x is 1 in
 // fp32 anyway. Every step is an IEEE-rounded operation, so the result is a fixed
-// function of x.
+// function of x. Two arguments at a time (packed fp32 pairs).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float exp_cw(float x) {
+__device__ __forceinline__ void exp_cw2(float x0, float x1, float& e0, float& e1) {
   const float kLog2e = 0x1.715476p+0f;
   const float kLn2Hi = 0x1.62ep-1f;
   const float kLn2Lo = 0x1.0bfbe8p-15f;
-  x = fminf(fmaxf(x, -80.0f), 88.0f);
-  const float n = rintf(__fmul_rn(x, kLog2e));
-  float r = __fmaf_rn(-n, kLn2Hi, x);
-  r = __fmaf_rn(-n, kLn2Lo, r);
-  float p = 0x1.a01a02p-13f;            // 1/7!
-  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);  // 1/6!
-  p = __fmaf_rn(p, r, 0x1.111112p-7f);   // 1/5!
-  p = __fmaf_rn(p, r, 0x1.555556p-5f);   // 1/4!
-  p = __fmaf_rn(p, r, 0x1.555556p-3f);   // 1/3!
-  p = __fmaf_rn(p, r, 0.5f);
-  p = __fmaf_rn(p, r, 1.0f);
-  p = __fmaf_rn(p, r, 1.0f);
-  const float two_n = __int_as_float((static_cast<int>(n) + 127) << 23);
-  return __fmul_rn(p, two_n);
+  x0 = fminf(fmaxf(x0, -80.0f), 88.0f);
+  x1 = fminf(fmaxf(x1, -80.0f), 88.0f);
+  float l0, l1;
+  mul2(l0, l1, x0, x1, kLog2e, kLog2e);
+  const float n0 = rintf(l0), n1 = rintf(l1);
+  float r0 = x0, r1 = x1;
+  fma2(r0, r1, -n0, -n1, kLn2Hi, kLn2Hi);
+  fma2(r0, r1, -n0, -n1, kLn2Lo, kLn2Lo);
+  // Horner: p = ((((((c7 r + c6) r + c5) r + c4) r + c3) r + c2) r + 1) r + 1
+  float p0 = 0x1.6c16c2p-10f, p1 = 0x1.6c16c2p-10f;  // starts as c6, then c7*r + c6
+  fma2(p0, p1, r0, r1, 0x1.a01a02p-13f, 0x1.a01a02p-13f);
+  float c0 = 0x1.111112p-7f, c1 = 0x1.111112p-7f;
+  fma2(c0, c1, p0, p1, r0, r1);
+  p0 = c0; p1 = c1;
+  c0 = 0x1.555556p-5f; c1 = 0x1.555556p-5f;
+  fma2(c0, c1, p0, p1, r0, r1);
+  p0 = c0; p1 = c1;
+  c0 = 0x1.555556p-3f; c1 = 0x1.555556p-3f;
+  fma2(c0, c1, p0, p1, r0, r1);
+  p0 = c0; p1 = c1;
+  c0 = 0.5f; c1 = 0.5f;
+  fma2(c0, c1, p0, p1, r0, r1);
+  p0 = c0; p1 = c1;
+  c0 = 1.0f; c1 = 1.0f;
+  fma2(c0, c1, p0, p1, r0, r1);
+  p0 = c0; p1 = c1;
+  c0 = 1.0f; c1 = 1.0f;
+  fma2(c0, c1, p0, p1, r0, r1);
+  const float s0 = __int_as_float((static_cast<int>(n0) + 127) << 23);
+  const float s1 = __int_as_float((static_cast<int>(n1) + 127) << 23);
+  mul2(e0, e1, c0, c1, s0, s1);
 }
 
-__device__ __forceinline__ float swiglu1(float g, float u) {
-  const float e = exp_cw(-g);
-  const float d = __fadd_rn(1.0f, e);
-  const float silu = __fdiv_rn(g, d);
-  return round_bf16(__fmul_rn(silu, u));
+// h = bf16( fl32( fl32(g / fl32(1 + E(-g))) * u ) ), two at a time.
+__device__ __forceinline__ void swiglu2(float g0, float g1, float u0, float u1, float& h0,
+                                        float& h1) {
+  float e0, e1;
+  exp_cw2(-g0, -g1, e0, e1);
+  const float d0 = __fadd_rn(1.0f, e0), d1 = __fadd_rn(1.0f, e1);
+  const float s0 = __fdiv_rn(g0, d0), s1 = __fdiv_rn(g1, d1);
+  float m0, m1;
+  mul2(m0, m1, s0, s1, u0, u1);
+  h0 = round_bf16(m0);
+  h1 = round_bf16(m1);
 }
 
 // ---------------------------------------------------------------------------
@@ -127,7 +195,7 @@ struct SwigluSrc {
     unpack_bf16x8(r.g, g);
     unpack_bf16x8(r.u, u);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = swiglu1(g[i], u[i]);
+    for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[i], v[i + 1]);
   }
 };
 
@@ -178,13 +246,96 @@ __global__ void __launch_bounds__(256) rowgroup_quant_kernel(Src src, int64_t M,
 }
 
 // ---------------------------------------------------------------------------
-// a3: RMSNorm + 1x128 quantization. One CTA (256 threads) per row; thread t owns
-// 8-element chunks t, t+256, ... so that each half-warp covers one 128-group.
+// a3: RMSNorm + 1x128 quantization.
+// Rows of up to kWarpRowChunks*256 elements: one warp per row (the row stays in
+// registers, the sum of squares is a warp reduction), 8 rows per CTA.
+// Longer rows: one CTA (256 threads) per row.
+// Thread t of the row owns 8-element chunks t, t+T, ... (T = threads per row), so
+// that each half-warp covers one 128-group.
 // ---------------------------------------------------------------------------
-constexpr int kNormThreads = 256;
-constexpr int kNormMaxChunks = 8;  // H <= 8 * 8 * 256 = 16384
+__device__ __forceinline__ float rstd_from_ss(double ss, int64_t H, float eps) {
+  const double ms = __ddiv_rn(ss, static_cast<double>(H));
+  const double rr = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, static_cast<double>(eps))));
+  return __double2float_rn(rr);
+}
 
-__global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_kernel(
+// y = bf16(fl32(fl32(x r) g)) for one chunk, then the half-warp group quantization.
+__device__ __forceinline__ void norm_quant_chunk(const uint4& xr, const uint16_t* gamma, int64_t c,
+                                                 bool act, float r, uint8_t* qrow, float* s,
+                                                 int64_t lds, int64_t m, int lane) {
+  float v[8];
+  if (act) {
+    float xv[8], gv[8];
+    unpack_bf16x8(xr, xv);
+    unpack_bf16x8(ld_nc_v4(gamma + c * 8), gv);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float a0, a1, b0, b1;
+      mul2(a0, a1, xv[i], xv[i + 1], r, r);
+      mul2(b0, b1, a0, a1, gv[i], gv[i + 1]);
+      v[i] = round_bf16(b0);
+      v[i + 1] = round_bf16(b1);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+  }
+  uint2 codes;
+  const float sc = quant_half_warp(v, codes);
+  if (act) {
+    *reinterpret_cast<uint2*>(qrow + c * 8) = codes;
+    if ((lane & 15) == 0) s[(c >> 4) * lds + m] = sc;
+  }
+}
+
+constexpr int kWarpRowChunks = 24;  // warp-per-row path: H <= 24 * 256 = 6144
+
+template <int kChunks>
+__global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma, int64_t M, int64_t H,
+    int64_t ldx, float eps, uint8_t* __restrict__ q, float* __restrict__ s, int64_t lds) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nch = H >> 3;
+  const int64_t wglobal = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t m = wglobal; m < M; m += nw) {
+    const uint16_t* row = x + m * ldx;
+    uint4 raw[kChunks];
+    double ss = 0.0;
+#pragma unroll
+    for (int j = 0; j < kChunks; ++j) {
+      const int64_t c = lane + 32 * j;
+      if (c < nch) raw[j] = ld_nc_v4(row + c * 8);
+    }
+#pragma unroll
+    for (int j = 0; j < kChunks; ++j) {
+      const int64_t c = lane + 32 * j;
+      if (c < nch) {
+        float v[8];
+        unpack_bf16x8(raw[j], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const double d = static_cast<double>(v[i]);
+          ss = __fma_rn(d, d, ss);  // the square is exact, so this is the fp64 sum
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, off));
+    const float r = rstd_from_ss(ss, H, eps);
+#pragma unroll
+    for (int j = 0; j < kChunks; ++j) {
+      if (32 * j >= nch) break;  // warp-uniform; nch is a multiple of 16
+      const int64_t c = lane + 32 * j;
+      norm_quant_chunk(raw[j], gamma, c, c < nch, r, q + m * H, s, lds, m, lane);
+    }
+  }
+}
+
+constexpr int kNormThreads = 256;
+constexpr int kNormMaxChunks = 8;  // CTA-per-row path: H <= 8 * 8 * 256 = 16384
+
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_cta_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma, int64_t M, int64_t H,
     int64_t ldx, float eps, uint8_t* __restrict__ q, float* __restrict__ s, int64_t lds) {
   __shared__ double red[kNormThreads / 32];
@@ -210,7 +361,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_kernel(
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const double d = static_cast<double>(v[i]);
-          ss = __dadd_rn(ss, __dmul_rn(d, d));  // each square is exact in fp64
+          ss = __fma_rn(d, d, ss);
         }
       }
     }
@@ -221,9 +372,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_kernel(
     if (tid == 0) {
       double tot = 0.0;
       for (int w = 0; w < kNormThreads / 32; ++w) tot = __dadd_rn(tot, red[w]);
-      const double ms = __ddiv_rn(tot, static_cast<double>(H));
-      const double rr = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, static_cast<double>(eps))));
-      r_sh = __double2float_rn(rr);
+      r_sh = rstd_from_ss(tot, H, eps);
     }
     __syncthreads();
     const float r = r_sh;
@@ -232,98 +381,70 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_kernel(
       const int64_t c0 = static_cast<int64_t>(j) * kNormThreads + (tid & ~31);
       if (c0 >= nch) break;  // warp-uniform: nch is a multiple of 16
       const int64_t c = tid + j * kNormThreads;
-      const bool act = c < nch;
-      float v[8];
-      if (act) {
-        float xv[8], gv[8];
-        unpack_bf16x8(raw[j], xv);
-        unpack_bf16x8(ld_nc_v4(gamma + c * 8), gv);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = round_bf16(__fmul_rn(__fmul_rn(xv[i], r), gv[i]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      }
-      uint2 codes;
-      const float sc = quant_half_warp(v, codes);
-      if (act) {
-        *reinterpret_cast<uint2*>(q + m * H + c * 8) = codes;
-        if ((tid & 15) == 0) s[(c >> 4) * lds + m] = sc;
-      }
+      norm_quant_chunk(raw[j], gamma, c, c < nch, r, q + m * H, s, lds, m, lane);
     }
     __syncthreads();  // red / r_sh are reused by the next row
   }
 }
 
 // ---------------------------------------------------------------------------
-// 128x128 tile kernels (a2, a6, a8). 256 threads; thread t owns rows
-// t/16 + 16j (j = 0..7) and the 8 columns 8*(t%16) .. +7 of the tile, so each
-// row is read by one half-warp as a contiguous 256-byte (BF16) run. Codes that
-// must be stored transposed go through a shared byte tile with an odd row pitch
-// (129), which spreads a warp's byte stores over the banks.
+// 128x128 tile kernels (a2, a6, a8). 256 threads.
+// Row pass: thread t owns rows t/16 + 16j (j = 0..7) and the 8 columns
+// 8*(t%16) .. +7, so each tile row is read by one half-warp as one contiguous run and
+// each row is one 1x128 group.
+// Column pass: the tile is staged in shared memory; thread t owns the column pair
+// 2*(t%64), +1 and the 32 rows 32*(t/64) .. +31. A warp reads 32 consecutive column
+// pairs of one row per load (no bank conflicts); each thread produces 2 x 32
+// consecutive codes of the transposed output, stored as two 32-byte runs.
 // ---------------------------------------------------------------------------
-constexpr int kTilePitch = 129;
+constexpr int kTP = 136;  // row pitch of a staged BF16 tile, in elements (272 bytes)
 
-// Column maxima over the 128 rows of the tile: v[j][i] is (row t/16+16j, col 8*(t%16)+i).
-// Result: colmax[c] for c in 0..127 in shared memory.
-__device__ __forceinline__ void tile_column_max(const float (&v)[8][8], float* colmax_part,
-                                                float* colmax) {
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  float cm[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float a = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j][i]));
-    a = fmaxf(a, __shfl_xor_sync(kFull, a, 16));
-    cm[i] = a;
-  }
-  if (lane < 16) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) colmax_part[wid * 128 + lane * 8 + i] = cm[i];
-  }
-  __syncthreads();
-  if (tid < 128) {
-    float a = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) a = fmaxf(a, colmax_part[w * 128 + tid]);
-    colmax[tid] = a;
-  }
-  __syncthreads();
-}
-
-// Quantize the tile by columns (scale sc[col]) into the transposed byte tile
-// T[col][row], then store T's rows to dst[(col0 + c) * ldd + row0 .. +127].
-__device__ __forceinline__ void tile_quant_cols_store_T(const float (&v)[8][8], const float* sc,
-                                                        uint8_t* T, uint8_t* __restrict__ dst,
-                                                        int64_t ldd) {
+// Column pass over a staged BF16 tile Ts[128][kTP]. Column scales: computed per
+// column (per_col) or the given block scale. Codes go to dst[(c)*ldd + r] for
+// tile column c and tile row r; per-column scales to scol[c] (if not null).
+__device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, bool per_col,
+                                               const GroupScale& blk, uint8_t* __restrict__ dst,
+                                               int64_t ldd, float* __restrict__ scol) {
   const int tid = threadIdx.x;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
+  const int cp = tid & 63, rq = tid >> 6;
+  uint32_t w[32];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float s = sc[c8 + i];
+  for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(Ts + (32 * rq + r) * kTP + 2 * cp);
+  GroupScale g0 = blk, g1 = blk;
+  if (per_col) {
+    float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      const uint32_t two = cvt_e4m3x2(__fdiv_rn(v[j][i], s), __fdiv_rn(v[j + 1][i], s));
-      T[(c8 + i) * kTilePitch + rr + 16 * j] = static_cast<uint8_t>(two & 0xFF);
-      T[(c8 + i) * kTilePitch + rr + 16 * (j + 1)] = static_cast<uint8_t>(two >> 8);
+    for (int r = 0; r < 32; ++r) {
+      a0 = fmaxf(a0, fabsf(bf16_lo(w[r])));
+      a1 = fmaxf(a1, fabsf(bf16_hi(w[r])));
     }
+    red[rq * 128 + 2 * cp] = a0;
+    red[rq * 128 + 2 * cp + 1] = a1;
+    __syncthreads();
+    a0 = fmaxf(fmaxf(red[2 * cp], red[128 + 2 * cp]), fmaxf(red[256 + 2 * cp], red[384 + 2 * cp]));
+    a1 = fmaxf(fmaxf(red[2 * cp + 1], red[128 + 2 * cp + 1]),
+               fmaxf(red[256 + 2 * cp + 1], red[384 + 2 * cp + 1]));
+    g0 = group_scale(a0);
+    g1 = group_scale(a1);
+    if (rq == 0 && scol) *reinterpret_cast<float2*>(scol + 2 * cp) = make_float2(g0.s, g1.s);
   }
-  __syncthreads();
-  // 128 rows x 8 chunks of 16 bytes; 4 chunks per thread
+  uint32_t o0[8], o1[8];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int idx = tid + k * 256;
-    const int row = idx >> 3, ch = idx & 7;
-    const uint8_t* src = T + row * kTilePitch + ch * 16;
-    uint32_t w[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-      w[b] = static_cast<uint32_t>(src[4 * b]) | (static_cast<uint32_t>(src[4 * b + 1]) << 8) |
-             (static_cast<uint32_t>(src[4 * b + 2]) << 16) |
-             (static_cast<uint32_t>(src[4 * b + 3]) << 24);
-    *reinterpret_cast<uint4*>(dst + row * ldd + ch * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  for (int k = 0; k < 8; ++k) {
+    float t0[4], t1[4];
+    quotient2(bf16_lo(w[4 * k]), bf16_lo(w[4 * k + 1]), g0, t0[0], t0[1]);
+    quotient2(bf16_lo(w[4 * k + 2]), bf16_lo(w[4 * k + 3]), g0, t0[2], t0[3]);
+    quotient2(bf16_hi(w[4 * k]), bf16_hi(w[4 * k + 1]), g1, t1[0], t1[1]);
+    quotient2(bf16_hi(w[4 * k + 2]), bf16_hi(w[4 * k + 3]), g1, t1[2], t1[3]);
+    o0[k] = cvt_e4m3x4(t0[0], t0[1], t0[2], t0[3]);
+    o1[k] = cvt_e4m3x4(t1[0], t1[1], t1[2], t1[3]);
   }
+  uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * ldd + 32 * rq);
+  uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * ldd + 32 * rq);
+  d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+  d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
+  d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+  d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
 }
 
 // a2: 128x128 weight blocks. grid = (N/128) * (K/128).
@@ -333,7 +454,7 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
                                                            float* __restrict__ s,
                                                            uint8_t* __restrict__ qT) {
   __shared__ float red[8];
-  __shared__ __align__(16) uint8_t T[128 * kTilePitch];
+  __shared__ __align__(16) uint16_t Ts[128 * kTP];
   const int64_t KB = K >> 7;
   const int64_t nb = blockIdx.x / KB, kb = blockIdx.x % KB;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -342,13 +463,14 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
   uint4 raw[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) raw[j] = ld_nc_v4(base + (rr + 16 * j) * ldw);
-  float v[8][8];
   float a = 0.0f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    unpack_bf16x8(raw[j], v[j]);
+    float v[8];
+    unpack_bf16x8(raw[j], v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[j][i]));
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    if (qT) *reinterpret_cast<uint4*>(Ts + (rr + 16 * j) * kTP + c8) = raw[j];
   }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
@@ -357,52 +479,26 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
   float amax = red[0];
 #pragma unroll
   for (int k = 1; k < 8; ++k) amax = fmaxf(amax, red[k]);
-  const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-  if (tid == 0) s[nb * KB + kb] = sc;
+  const GroupScale g = group_scale(amax);
+  if (tid == 0) s[nb * KB + kb] = g.s;
   uint8_t* qb = q + (nb * 128) * K + kb * 128 + c8;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    float t[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) t[i] = __fdiv_rn(v[j][i], sc);
-    uint2 codes;
-    codes.x = cvt_e4m3x4(t[0], t[1], t[2], t[3]);
-    codes.y = cvt_e4m3x4(t[4], t[5], t[6], t[7]);
-    *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes;
-    if (qT) {
-      const uint8_t* cb = reinterpret_cast<const uint8_t*>(&codes);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) T[(c8 + i) * kTilePitch + rr + 16 * j] = cb[i];
-    }
+    float v[8];
+    unpack_bf16x8(raw[j], v);
+    *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes8(v, g);
   }
-  if (qT) {
-    __syncthreads();
-    uint8_t* dst = qT + (kb * 128) * N + nb * 128;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int idx = tid + k * 256;
-      const int row = idx >> 3, ch = idx & 7;
-      const uint8_t* src = T + row * kTilePitch + ch * 16;
-      uint32_t wv[4];
-#pragma unroll
-      for (int b = 0; b < 4; ++b)
-        wv[b] = static_cast<uint32_t>(src[4 * b]) | (static_cast<uint32_t>(src[4 * b + 1]) << 8) |
-                (static_cast<uint32_t>(src[4 * b + 2]) << 16) |
-                (static_cast<uint32_t>(src[4 * b + 3]) << 24);
-      *reinterpret_cast<uint4*>(dst + row * N + ch * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-    }
-  }
+  if (qT) tile_cols_bf16(Ts, nullptr, false, g, qT + (kb * 128) * N + nb * 128, N, nullptr);
 }
 
-// a6: BF16 dY tile -> row-wise 1x128 codes (direct) + column-wise 128x1 codes
-// (transposed). grid = (M/128) * (N/128).
+// a6: BF16 dY tile -> row-wise 1x128 codes (row pass) + column-wise 128x1 codes
+// (column pass, transposed). grid = (M/128) * (N/128).
 __global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
     const uint16_t* __restrict__ dy, int64_t M, int64_t N, int64_t lddy,
     uint8_t* __restrict__ q_row, float* __restrict__ s_row, int64_t lds_row,
     uint8_t* __restrict__ q_colT, float* __restrict__ s_col) {
-  __shared__ float colmax_part[8 * 128];
-  __shared__ float colsc[128];
-  __shared__ __align__(16) uint8_t T[128 * kTilePitch];
+  __shared__ float red[4 * 128];
+  __shared__ __align__(16) uint16_t Ts[128 * kTP];
   const int64_t NB = N >> 7;
   const int64_t mb = blockIdx.x / NB, nb = blockIdx.x % NB;
   const int tid = threadIdx.x;
@@ -411,74 +507,93 @@ __global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
   uint4 raw[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) raw[j] = ld_nc_v4(base + (rr + 16 * j) * lddy);
-  float v[8][8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) unpack_bf16x8(raw[j], v[j]);
-
-  if (q_row) {  // row-wise: each tile row is one 1x128 group, held by a half-warp
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < 8; ++j) {
+    *reinterpret_cast<uint4*>(Ts + (rr + 16 * j) * kTP + c8) = raw[j];
+    if (q_row) {  // each tile row is one 1x128 group, held by a half-warp
+      float v[8];
+      unpack_bf16x8(raw[j], v);
       uint2 codes;
-      const float sc = quant_half_warp(v[j], codes);
+      const float sc = quant_half_warp(v, codes);
       const int64_t m = mb * 128 + rr + 16 * j;
       *reinterpret_cast<uint2*>(q_row + m * N + nb * 128 + c8) = codes;
       if ((tid & 15) == 0) s_row[nb * lds_row + m] = sc;
     }
   }
-  tile_column_max(v, colmax_part, colsc);
-  if (tid < 128) {
-    const float a = colsc[tid];
-    const float sc = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 448.0f);
-    colsc[tid] = sc;
-    s_col[mb * N + nb * 128 + tid] = sc;
-  }
   __syncthreads();
-  tile_quant_cols_store_T(v, colsc, T, q_colT + (nb * 128) * M + mb * 128, M);
+  const GroupScale unused{1.0f, 1.0f, false};
+  tile_cols_bf16(Ts, red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
+                 s_col + mb * N + nb * 128);
 }
 
 // a8: saved FP8 activation tile (1x128 groups) -> xhat = fl32(s * dec(q)) ->
 // 128x1 groups along M, stored transposed. grid = (M/128) * (K/128).
+// The codes and row scales are staged in shared memory; the column pass decodes two
+// codes per load. xhat is an arbitrary fp32 value here, so quotients use IEEE
+// division.
+constexpr int kQP = 144;  // row pitch of a staged code tile, in bytes
+
 __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
     const uint8_t* __restrict__ qin, const float* __restrict__ sin, int64_t M, int64_t K,
     int64_t lds, uint8_t* __restrict__ qT, float* __restrict__ sT) {
-  __shared__ float colmax_part[8 * 128];
-  __shared__ float colsc[128];
-  __shared__ __align__(16) uint8_t T[128 * kTilePitch];
+  __shared__ float red[4 * 128];
+  __shared__ float rsc[128];
+  __shared__ __align__(16) uint8_t Tq[128 * kQP];
   const int64_t KB = K >> 7;
   const int64_t mb = blockIdx.x / KB, kb = blockIdx.x % KB;
   const int tid = threadIdx.x;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  const uint8_t* base = qin + (mb * 128) * K + kb * 128 + c8;
-  uint2 raw[8];
-  float rs[8];
+  {
+    const int rr = tid >> 3, c16 = (tid & 7) * 16;  // 32 rows x 8 chunks of 16 bytes per pass
+    const uint8_t* base = qin + (mb * 128) * K + kb * 128 + c16;
+    uint4 raw[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    raw[j] = *reinterpret_cast<const uint2*>(base + (rr + 16 * j) * K);
-    rs[j] = sin[kb * lds + mb * 128 + rr + 16 * j];
-  }
-  float v[8][8];
+    for (int j = 0; j < 4; ++j) raw[j] = ld_nc_v4(base + (rr + 32 * j) * K);
+    if (tid < 128) rsc[tid] = sin[kb * lds + mb * 128 + tid];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t w[2] = {raw[j].x, raw[j].y};
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const float2 lo = e4m3x2_to_f32(static_cast<uint16_t>(w[h] & 0xFFFF));
-      const float2 hi = e4m3x2_to_f32(static_cast<uint16_t>(w[h] >> 16));
-      v[j][4 * h + 0] = __fmul_rn(rs[j], lo.x);
-      v[j][4 * h + 1] = __fmul_rn(rs[j], lo.y);
-      v[j][4 * h + 2] = __fmul_rn(rs[j], hi.x);
-      v[j][4 * h + 3] = __fmul_rn(rs[j], hi.y);
-    }
-  }
-  tile_column_max(v, colmax_part, colsc);
-  if (tid < 128) {
-    const float a = colsc[tid];
-    const float sc = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 448.0f);
-    colsc[tid] = sc;
-    sT[mb * K + kb * 128 + tid] = sc;
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(Tq + (rr + 32 * j) * kQP + c16) = raw[j];
   }
   __syncthreads();
-  tile_quant_cols_store_T(v, colsc, T, qT + (kb * 128) * M + mb * 128, M);
+  const int cp = tid & 63, rq = tid >> 6;
+  float x0[32], x1[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    const int row = 32 * rq + r;
+    const uint16_t two = *reinterpret_cast<const uint16_t*>(Tq + row * kQP + 2 * cp);
+    const float2 d = e4m3x2_to_f32(two);
+    const float sr = rsc[row];
+    x0[r] = __fmul_rn(sr, d.x);
+    x1[r] = __fmul_rn(sr, d.y);
+  }
+  float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    a0 = fmaxf(a0, fabsf(x0[r]));
+    a1 = fmaxf(a1, fabsf(x1[r]));
+  }
+  red[rq * 128 + 2 * cp] = a0;
+  red[rq * 128 + 2 * cp + 1] = a1;
+  __syncthreads();
+  a0 = fmaxf(fmaxf(red[2 * cp], red[128 + 2 * cp]), fmaxf(red[256 + 2 * cp], red[384 + 2 * cp]));
+  a1 = fmaxf(fmaxf(red[2 * cp + 1], red[128 + 2 * cp + 1]),
+             fmaxf(red[256 + 2 * cp + 1], red[384 + 2 * cp + 1]));
+  const float s0 = (a0 == 0.0f) ? 1.0f : __fdiv_rn(a0, 448.0f);
+  const float s1 = (a1 == 0.0f) ? 1.0f : __fdiv_rn(a1, 448.0f);
+  if (rq == 0) *reinterpret_cast<float2*>(sT + mb * K + kb * 128 + 2 * cp) = make_float2(s0, s1);
+  uint32_t o0[8], o1[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    o0[k] = cvt_e4m3x4(__fdiv_rn(x0[4 * k], s0), __fdiv_rn(x0[4 * k + 1], s0),
+                       __fdiv_rn(x0[4 * k + 2], s0), __fdiv_rn(x0[4 * k + 3], s0));
+    o1[k] = cvt_e4m3x4(__fdiv_rn(x1[4 * k], s1), __fdiv_rn(x1[4 * k + 1], s1),
+                       __fdiv_rn(x1[4 * k + 2], s1), __fdiv_rn(x1[4 * k + 3], s1));
+  }
+  uint8_t* dst = qT + (kb * 128) * M + mb * 128;
+  uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * M + 32 * rq);
+  uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * M + 32 * rq);
+  d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+  d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
+  d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+  d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
 }
 
 int grid_for_units(int64_t warps_needed) {
@@ -502,10 +617,10 @@ extern "C" fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   const int64_t G = K / 128;
   const int64_t units = M * ((G + 1) / 2);
-  rowgroup_quant_kernel<ActSrc, 2><<<grid_for_units((units + 1) / 2), 256, 0,
+  rowgroup_quant_kernel<ActSrc, 4><<<grid_for_units((units + 3) / 4), 256, 0,
                                      static_cast<cudaStream_t>(stream)>>>(ActSrc{x, ldx}, M, G, q,
                                                                           K, s, lds);
-  return launch_status();
+  return launch_status("quant_act_1x128 launch");
 }
 
 extern "C" fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t I, int64_t ldgu,
@@ -519,7 +634,7 @@ extern "C" fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t 
   rowgroup_quant_kernel<SwigluSrc, 2><<<grid_for_units((units + 1) / 2), 256, 0,
                                         static_cast<cudaStream_t>(stream)>>>(
       SwigluSrc{gu, ldgu, I}, M, G, q, I, s, lds);
-  return launch_status();
+  return launch_status("swiglu_quant launch");
 }
 
 extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, int64_t M,
@@ -533,10 +648,22 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
     return FP8Q_ERR_ALIGN;
   const int sms = sm100_sm_count();
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
-  const int64_t grid = M < static_cast<int64_t>(sms) * 64 ? M : static_cast<int64_t>(sms) * 64;
-  rmsnorm_quant_kernel<<<static_cast<int>(grid), kNormThreads, 0,
-                         static_cast<cudaStream_t>(stream)>>>(x, gamma, M, H, ldx, eps, q, s, lds);
-  return launch_status();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (H <= 8 * 32 * kWarpRowChunks) {
+    const int64_t ctas = (M + 7) / 8;
+    const int64_t grid = ctas < static_cast<int64_t>(sms) * 8 ? ctas : static_cast<int64_t>(sms) * 8;
+    if (H <= 8 * 32 * 16)
+      rmsnorm_quant_warp_kernel<16><<<static_cast<int>(grid), 256, 0, st>>>(x, gamma, M, H, ldx,
+                                                                            eps, q, s, lds);
+    else
+      rmsnorm_quant_warp_kernel<kWarpRowChunks><<<static_cast<int>(grid), 256, 0, st>>>(
+          x, gamma, M, H, ldx, eps, q, s, lds);
+  } else {
+    const int64_t grid = M < static_cast<int64_t>(sms) * 64 ? M : static_cast<int64_t>(sms) * 64;
+    rmsnorm_quant_cta_kernel<<<static_cast<int>(grid), kNormThreads, 0, st>>>(x, gamma, M, H, ldx,
+                                                                              eps, q, s, lds);
+  }
+  return launch_status("rmsnorm_quant launch");
 }
 
 extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, int64_t K,
@@ -551,7 +678,7 @@ extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, i
   if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   quant_weight_kernel<<<static_cast<unsigned>(blocks), 256, 0,
                         static_cast<cudaStream_t>(stream)>>>(w, N, K, ldw, q, s, qT);
-  return launch_status();
+  return launch_status("quant_weight_128x128 launch");
 }
 
 extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, int64_t N,
@@ -570,7 +697,7 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
   transpose_quant_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0,
                                 static_cast<cudaStream_t>(stream)>>>(dy, M, N, lddy, q_row, s_row,
                                                                      lds_row, q_colT, s_col);
-  return launch_status();
+  return launch_status("transpose_quant_bf16 launch");
 }
 
 extern "C" fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s, int64_t M,
@@ -585,5 +712,5 @@ extern "C" fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s
   if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   transpose_quant_fp8_kernel<<<static_cast<unsigned>(blocks), 256, 0,
                                static_cast<cudaStream_t>(stream)>>>(q, s, M, K, lds, qT, sT);
-  return launch_status();
+  return launch_status("transpose_quant_fp8 launch");
 }

@@ -91,6 +91,51 @@ def test_special_groups(fq, oracle_mod):
     assert_scales_equal(s, rs, "special scales", cols=6)
 
 
+def test_quotient_dense_sweep(fq, oracle_mod):
+    """Groups whose amax is a chosen BF16 value and whose other 127 elements sweep the
+    BF16 values below it: the kernel's quotient path against the oracle's IEEE
+    division, across every binade of amax (including fp32-subnormal scales)."""
+    rng = np.random.default_rng(5)
+    amax_bits = np.concatenate([rng.integers(0x0001, 0x7F80, 1500), [0x0001, 0x0080, 0x43E0, 0x7F7F]])
+    rows = []
+    for ab in amax_bits:
+        xs = rng.integers(0, int(ab) + 1, 127 * 8).astype(np.uint16)
+        xs |= (rng.integers(0, 2, xs.size) << 15).astype(np.uint16)  # random signs
+        for k in range(8):
+            row = np.empty(128, np.uint16)
+            row[0] = ab
+            row[1:] = xs[127 * k: 127 * (k + 1)]
+            rows.append(row)
+    arr = np.stack(rows)
+    x = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16).to(DEV)
+    q, s = run_act(fq, x)
+    rq, rs = oracle_mod.quant_act_1x128(arr)
+    assert_codes_equal(q, rq, "dense quotient sweep")
+    assert_scales_equal(s, rs, "dense quotient sweep scales", cols=arr.shape[0])
+
+
+def test_swiglu_exhaustive_gate(fq, oracle_mod):
+    """Every BF16 gate value g with |g| <= 1e37, with up-projections u in {1, -0.5, 3.25}: SwiGLU
+    depends on g only through the fixed exponential and an IEEE division, so this
+    covers the kernel's whole silu path."""
+    pat = np.arange(65536, dtype=np.uint32)
+    vals = (pat << 16).view(np.float32)
+    gates = pat[np.isfinite(vals) & (np.abs(vals) <= 1e37)].astype(np.uint16)  # h stays finite
+    n = -(-len(gates) // 128) * 128
+    g = np.zeros(n, np.uint16)
+    g[: len(gates)] = gates
+    g = g.reshape(-1, 128)
+    for u in (1.0, -0.5, 3.25):
+        ub = np.full_like(g, np.float32(u).view(np.uint32) >> 16)
+        arr = np.concatenate([g, ub], axis=1)                     # [rows, 2I] with I = 128
+        x = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16).to(DEV)
+        q, s = fq.swiglu_quant_alloc(x)
+        torch.cuda.synchronize()
+        rq, rs = oracle_mod.swiglu_quant(arr)
+        assert_codes_equal(q, rq, "swiglu exhaustive u=%g" % u)
+        assert_scales_equal(s, rs, "swiglu exhaustive scales u=%g" % u, cols=arr.shape[0])
+
+
 # ---------------------------------------------------------------- a2
 @pytest.mark.parametrize("N,K", [(512, 512), (128, 128), (384, 256)])
 def test_weight_quant_matches_oracle(fq, oracle_mod, N, K):
