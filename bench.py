@@ -61,6 +61,28 @@ def read_peaks():
 
 
 # --------------------------------------------------------------------------
+# Multi-rank host logic (weak scaling: one independent token batch per rank)
+# --------------------------------------------------------------------------
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own token batch (and weights): sub-stream seed offset."""
+    return rank
+
+
+def max_over_ranks(value_ms: float, dist=None, device="cpu") -> float:
+    """The slowest rank's device-timed duration (all ranks take the same collective)."""
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, max_ms_per_step: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time."""
+    return flops_per_rank * world / (max_ms_per_step * 1e-3) / 1e12
+
+
+# --------------------------------------------------------------------------
 # The layer step on the GPU
 # --------------------------------------------------------------------------
 
@@ -489,7 +511,7 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    step = LayerStep(fq, WORKLOAD, dev, seed_offset=rank)
+    step = LayerStep(fq, WORKLOAD, dev, seed_offset=rank_seed_offset(rank))
     torch.cuda.synchronize()
     for _ in range(args.warmup):
         step.run()
@@ -516,12 +538,9 @@ def main():
     elapsed_ms = start.elapsed_time(end)
     if fq.device_error() != fq.FP8Q_OK:
         raise RuntimeError("a kernel reported a device error in the timed region")
-    t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, pg, dev)
     ms_per_step = max_ms / args.steps
-    value = step.flops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(step.flops, world, ms_per_step)
 
     # ---- per-kernel breakdown (same timed steps)
     peaks = read_peaks()
@@ -564,11 +583,8 @@ def main():
         step.run_e2e(bufs)
     e1.record()
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if pg:
-        pg.all_reduce(te, op=pg.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / args.e2e_steps
-    e2e_value = step.flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev) / args.e2e_steps
+    e2e_value = whole_job_tflops(step.flops, world, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
