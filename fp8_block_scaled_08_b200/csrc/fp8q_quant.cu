@@ -35,15 +35,93 @@ constexpr float kSmallScale = 0x1p-80f;  // below it the quotient uses IEEE divi
 // Group scale and quotient
 // ---------------------------------------------------------------------------
 struct GroupScale {
-  float s, rs;
-  bool small;
+  float s, rs, ns;  // scale, its correctly rounded reciprocal, -scale
+  bool small;       // s < 2^-80 (or a tiny amax): quotients by IEEE division
 };
 
+// Scale of a group with an arbitrary fp32 amax: s = amax/448 (IEEE), s = 1 if amax = 0.
 __device__ __forceinline__ GroupScale group_scale(float amax) {
   GroupScale g;
   g.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
   g.rs = __frcp_rn(g.s);
+  g.ns = -g.s;
   g.small = g.s < kSmallScale;
+  return g;
+}
+
+// For amax = (1 + i/128) * 2^E, a normal BF16 value: amax/448 = ((1 + i/128)/7) * 2^(E-6),
+// and scaling by a power of two commutes with rounding while the result stays a normal
+// float, so fl32(amax/448) = kScaleMant[i] * 2^(E-6) and fl32(1/s) = kRecipMant[i] *
+// 2^(6-E), with kScaleMant[i] = fl32((1 + i/128)/7) and kRecipMant[i] =
+// fl32(1/kScaleMant[i]) (values below; the test suite re-derives them and checks the
+// identity for every BF16 amax with E >= -71).
+__constant__ float kScaleMant[128] = {
+    0x1.24924ap-3f, 0x1.26db6ep-3f, 0x1.292492p-3f, 0x1.2b6db6p-3f, 0x1.2db6dcp-3f, 0x1.3p-3f,
+    0x1.324924p-3f, 0x1.34924ap-3f, 0x1.36db6ep-3f, 0x1.392492p-3f, 0x1.3b6db6p-3f, 0x1.3db6dcp-3f,
+    0x1.4p-3f, 0x1.424924p-3f, 0x1.44924ap-3f, 0x1.46db6ep-3f, 0x1.492492p-3f, 0x1.4b6db6p-3f,
+    0x1.4db6dcp-3f, 0x1.5p-3f, 0x1.524924p-3f, 0x1.54924ap-3f, 0x1.56db6ep-3f, 0x1.592492p-3f,
+    0x1.5b6db6p-3f, 0x1.5db6dcp-3f, 0x1.6p-3f, 0x1.624924p-3f, 0x1.64924ap-3f, 0x1.66db6ep-3f,
+    0x1.692492p-3f, 0x1.6b6db6p-3f, 0x1.6db6dcp-3f, 0x1.7p-3f, 0x1.724924p-3f, 0x1.74924ap-3f,
+    0x1.76db6ep-3f, 0x1.792492p-3f, 0x1.7b6db6p-3f, 0x1.7db6dcp-3f, 0x1.8p-3f, 0x1.824924p-3f,
+    0x1.84924ap-3f, 0x1.86db6ep-3f, 0x1.892492p-3f, 0x1.8b6db6p-3f, 0x1.8db6dcp-3f, 0x1.9p-3f,
+    0x1.924924p-3f, 0x1.94924ap-3f, 0x1.96db6ep-3f, 0x1.992492p-3f, 0x1.9b6db6p-3f, 0x1.9db6dcp-3f,
+    0x1.ap-3f, 0x1.a24924p-3f, 0x1.a4924ap-3f, 0x1.a6db6ep-3f, 0x1.a92492p-3f, 0x1.ab6db6p-3f,
+    0x1.adb6dcp-3f, 0x1.bp-3f, 0x1.b24924p-3f, 0x1.b4924ap-3f, 0x1.b6db6ep-3f, 0x1.b92492p-3f,
+    0x1.bb6db6p-3f, 0x1.bdb6dcp-3f, 0x1.cp-3f, 0x1.c24924p-3f, 0x1.c4924ap-3f, 0x1.c6db6ep-3f,
+    0x1.c92492p-3f, 0x1.cb6db6p-3f, 0x1.cdb6dcp-3f, 0x1.dp-3f, 0x1.d24924p-3f, 0x1.d4924ap-3f,
+    0x1.d6db6ep-3f, 0x1.d92492p-3f, 0x1.db6db6p-3f, 0x1.ddb6dcp-3f, 0x1.ep-3f, 0x1.e24924p-3f,
+    0x1.e4924ap-3f, 0x1.e6db6ep-3f, 0x1.e92492p-3f, 0x1.eb6db6p-3f, 0x1.edb6dcp-3f, 0x1.fp-3f,
+    0x1.f24924p-3f, 0x1.f4924ap-3f, 0x1.f6db6ep-3f, 0x1.f92492p-3f, 0x1.fb6db6p-3f, 0x1.fdb6dcp-3f,
+    0x1p-2f, 0x1.012492p-2f, 0x1.024924p-2f, 0x1.036db6p-2f, 0x1.04924ap-2f, 0x1.05b6dcp-2f,
+    0x1.06db6ep-2f, 0x1.08p-2f, 0x1.092492p-2f, 0x1.0a4924p-2f, 0x1.0b6db6p-2f, 0x1.0c924ap-2f,
+    0x1.0db6dcp-2f, 0x1.0edb6ep-2f, 0x1.1p-2f, 0x1.112492p-2f, 0x1.124924p-2f, 0x1.136db6p-2f,
+    0x1.14924ap-2f, 0x1.15b6dcp-2f, 0x1.16db6ep-2f, 0x1.18p-2f, 0x1.192492p-2f, 0x1.1a4924p-2f,
+    0x1.1b6db6p-2f, 0x1.1c924ap-2f, 0x1.1db6dcp-2f, 0x1.1edb6ep-2f, 0x1.2p-2f, 0x1.212492p-2f,
+    0x1.224924p-2f, 0x1.236db6p-2f,
+};
+__constant__ float kRecipMant[128] = {
+    0x1.bffffep+2f, 0x1.bc86f2p+2f, 0x1.b91b92p+2f, 0x1.b5bd9p+2f, 0x1.b26c9ap+2f, 0x1.af286cp+2f,
+    0x1.abf0b8p+2f, 0x1.a8c536p+2f, 0x1.a5a5a6p+2f, 0x1.a291cp+2f, 0x1.9f8948p+2f, 0x1.9c8bf8p+2f,
+    0x1.99999ap+2f, 0x1.96b1eep+2f, 0x1.93d4bap+2f, 0x1.9101cap+2f, 0x1.8e38e4p+2f, 0x1.8b79d4p+2f,
+    0x1.88c462p+2f, 0x1.861862p+2f, 0x1.8375ap+2f, 0x1.80dbeap+2f, 0x1.7e4b18p+2f, 0x1.7bc2f8p+2f,
+    0x1.79436p+2f, 0x1.76cc2p+2f, 0x1.745d18p+2f, 0x1.71f618p+2f, 0x1.6f96f8p+2f, 0x1.6d3f98p+2f,
+    0x1.6aefccp+2f, 0x1.68a774p+2f, 0x1.666666p+2f, 0x1.642c86p+2f, 0x1.61f9aep+2f, 0x1.5fcdbep+2f,
+    0x1.5da896p+2f, 0x1.5b8a16p+2f, 0x1.59722p+2f, 0x1.576092p+2f, 0x1.555556p+2f, 0x1.53504ap+2f,
+    0x1.51515p+2f, 0x1.4f5854p+2f, 0x1.4d6536p+2f, 0x1.4b77dep+2f, 0x1.49902ep+2f, 0x1.47ae14p+2f,
+    0x1.45d174p+2f, 0x1.43fa36p+2f, 0x1.422844p+2f, 0x1.405b88p+2f, 0x1.3e93eap+2f, 0x1.3cd154p+2f,
+    0x1.3b13b2p+2f, 0x1.395aeep+2f, 0x1.37a6f4p+2f, 0x1.35f7b2p+2f, 0x1.344d14p+2f, 0x1.32a704p+2f,
+    0x1.310572p+2f, 0x1.2f684cp+2f, 0x1.2dcf8p+2f, 0x1.2c3af8p+2f, 0x1.2aaaaap+2f, 0x1.291e82p+2f,
+    0x1.27967p+2f, 0x1.26126p+2f, 0x1.24924ap+2f, 0x1.231618p+2f, 0x1.219dbcp+2f, 0x1.20292ap+2f,
+    0x1.1eb852p+2f, 0x1.1d4b26p+2f, 0x1.1be196p+2f, 0x1.1a7b96p+2f, 0x1.19191ap+2f, 0x1.17ba1p+2f,
+    0x1.165e72p+2f, 0x1.15063p+2f, 0x1.13b13cp+2f, 0x1.125f8ap+2f, 0x1.111112p+2f, 0x1.0fc5c4p+2f,
+    0x1.0e7d96p+2f, 0x1.0d387cp+2f, 0x1.0bf66ep+2f, 0x1.0ab75ep+2f, 0x1.097b42p+2f, 0x1.08421p+2f,
+    0x1.070bbep+2f, 0x1.05d842p+2f, 0x1.04a79p+2f, 0x1.0379a2p+2f, 0x1.024e6ap+2f, 0x1.0125e2p+2f,
+    0x1p+2f, 0x1.fdb976p+1f, 0x1.fb7814p+1f, 0x1.f93bc8p+1f, 0x1.f7047cp+1f, 0x1.f4d22ap+1f,
+    0x1.f2a4bap+1f, 0x1.f07c2p+1f, 0x1.ee5848p+1f, 0x1.ec3924p+1f, 0x1.ea1ea4p+1f, 0x1.e808b6p+1f,
+    0x1.e5f752p+1f, 0x1.e3ea66p+1f, 0x1.e1e1e2p+1f, 0x1.dfddbap+1f, 0x1.dddddep+1f, 0x1.dbe244p+1f,
+    0x1.d9ead6p+1f, 0x1.d7f792p+1f, 0x1.d60864p+1f, 0x1.d41d42p+1f, 0x1.d2361ep+1f, 0x1.d052ecp+1f,
+    0x1.ce739ep+1f, 0x1.cc9828p+1f, 0x1.cac082p+1f, 0x1.c8ec9ep+1f, 0x1.c71c72p+1f, 0x1.c54ffp+1f,
+    0x1.c3870ep+1f, 0x1.c1c1c4p+1f,
+};
+
+// Same result as group_scale for every amax that is a BF16 value (the maximum of BF16
+// values is one). amax < 2^-71 (s below about 2^-80), and non-finite amax (outside the
+// contract), take the division path.
+__device__ __forceinline__ GroupScale group_scale_bf16(float amax) {
+  GroupScale g;
+  const uint32_t b = __float_as_uint(amax);
+  const int ebias = static_cast<int>(b >> 23);  // biased exponent (amax >= 0)
+  if (ebias < 127 - 71 || ebias == 255) {
+    g = group_scale(amax);
+    g.small = true;
+    return g;
+  }
+  const int e = ebias - 127;
+  const uint32_t i = (b >> 16) & 0x7Fu;
+  g.s = __uint_as_float(__float_as_uint(kScaleMant[i]) + static_cast<uint32_t>((e - 6) << 23));
+  g.rs = __uint_as_float(__float_as_uint(kRecipMant[i]) + static_cast<uint32_t>((6 - e) << 23));
+  g.ns = -g.s;
+  g.small = false;
   return g;
 }
 
@@ -63,7 +141,7 @@ __device__ __forceinline__ void quotient2(float x0, float x1, const GroupScale& 
   float q0, q1;
   mul2(q0, q1, x0, x1, g.rs, g.rs);      // q = x * r
   float e0 = x0, e1 = x1;
-  fma2(e0, e1, -q0, -q1, g.s, g.s);      // e = fma(-q, s, x), exact
+  fma2(e0, e1, q0, q1, g.ns, g.ns);      // e = fma(q, -s, x), exact
   fma2(q0, q1, e0, e1, g.rs, g.rs);      // q = fma(e, r, q)
   t0 = copy_sign(q0, x0);
   t1 = copy_sign(q1, x1);
@@ -77,15 +155,15 @@ __device__ __forceinline__ uint2 codes8(const float (&v)[8], const GroupScale& g
   return make_uint2(cvt_e4m3x4(t[0], t[1], t[2], t[3]), cvt_e4m3x4(t[4], t[5], t[6], t[7]));
 }
 
-// One 1x128 group held by a half-warp: 16 lanes x 8 values. Returns the group scale;
-// writes the 8 codes of this lane. All 32 lanes must call it (full-mask shuffles).
+// One 1x128 group of BF16 values held by a half-warp: 16 lanes x 8 values. Returns the
+// group scale; writes the 8 codes of this lane. All 32 lanes must call it.
 __device__ __forceinline__ float quant_half_warp(const float (&v)[8], uint2& codes) {
   float a = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
 #pragma unroll
   for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
-  const GroupScale g = group_scale(a);
+  const GroupScale g = group_scale_bf16(a);
   codes = codes8(v, g);
   return g.s;
 }
@@ -204,30 +282,35 @@ __global__ void __launch_bounds__(256) rowgroup_quant_kernel(Src src, int64_t M,
                                                              uint8_t* __restrict__ q, int64_t ldq,
                                                              float* __restrict__ s, int64_t lds) {
   const int64_t pairs = (G + 1) >> 1;
-  const int64_t units = M * pairs;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;
   const int sub = lane & 15;
-
-  for (int64_t base = warp; base < units; base += kUnroll * nwarps) {
+  // Unit u = m * pairs + pair. Slot j of this warp visits u = warp + j*nwarps + k*stride;
+  // (m, pair) of each slot advance by the quotient/remainder of `stride` (divisions
+  // only here, once).
+  const int64_t stride = kUnroll * nwarps;
+  const int64_t qs = stride / pairs, rs = stride % pairs;
+  int64_t mm[kUnroll], pp[kUnroll];
+#pragma unroll
+  for (int j = 0; j < kUnroll; ++j) {
+    const int64_t u = warp + j * nwarps;
+    mm[j] = u / pairs;
+    pp[j] = u - mm[j] * pairs;
+  }
+  while (mm[0] < M) {
     typename Src::Raw raw[kUnroll];
     bool act[kUnroll];
-    int64_t mm[kUnroll], gg[kUnroll];
 #pragma unroll
     for (int j = 0; j < kUnroll; ++j) {
-      const int64_t u = base + j * nwarps;
-      const int64_t m = u / pairs;
-      const int64_t g = 2 * (u - m * pairs) + half;
-      mm[j] = m;
-      gg[j] = g;
-      act[j] = (u < units) && (g < G);
-      if (act[j]) raw[j] = src.fetch(m, g * 128 + sub * 8);
+      const int64_t g = 2 * pp[j] + half;
+      act[j] = (mm[j] < M) && (g < G);
+      if (act[j]) raw[j] = src.fetch(mm[j], g * 128 + sub * 8);
     }
 #pragma unroll
     for (int j = 0; j < kUnroll; ++j) {
-      if (base + j * nwarps >= units) break;  // warp-uniform
+      if (mm[j] >= M) break;  // warp-uniform (later slots have larger u)
       float v[8];
       if (act[j]) {
         src.values(raw[j], v);
@@ -238,8 +321,18 @@ __global__ void __launch_bounds__(256) rowgroup_quant_kernel(Src src, int64_t M,
       uint2 codes;
       const float sc = quant_half_warp(v, codes);
       if (act[j]) {
-        *reinterpret_cast<uint2*>(q + mm[j] * ldq + gg[j] * 128 + sub * 8) = codes;
-        if (sub == 0) s[gg[j] * lds + mm[j]] = sc;
+        const int64_t g = 2 * pp[j] + half;
+        *reinterpret_cast<uint2*>(q + mm[j] * ldq + g * 128 + sub * 8) = codes;
+        if (sub == 0) s[g * lds + mm[j]] = sc;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kUnroll; ++j) {
+      pp[j] += rs;
+      mm[j] += qs;
+      if (pp[j] >= pairs) {
+        pp[j] -= pairs;
+        ++mm[j];
       }
     }
   }
@@ -388,20 +481,40 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_cta_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// 128x128 tile kernels (a2, a6, a8). 256 threads.
-// Row pass: thread t owns rows t/16 + 16j (j = 0..7) and the 8 columns
-// 8*(t%16) .. +7, so each tile row is read by one half-warp as one contiguous run and
-// each row is one 1x128 group.
-// Column pass: the tile is staged in shared memory; thread t owns the column pair
-// 2*(t%64), +1 and the 32 rows 32*(t/64) .. +31. A warp reads 32 consecutive column
-// pairs of one row per load (no bank conflicts); each thread produces 2 x 32
-// consecutive codes of the transposed output, stored as two 32-byte runs.
+// 128x128 tile kernels (a2, a6, a8): persistent CTAs of 256 threads. Tiles arrive in
+// shared memory by TMA into a double buffer, so the next tile loads while this one is
+// processed; a tile's arrival is an mbarrier that thread 0 waits on with the bounded
+// wait (the CTA stops if it gives up, after letting issued copies land).
+// Row pass: thread t owns rows t/16 + 16j (j = 0..7) and the 8 columns 8*(t%16) .. +7
+// of the staged tile (a half-warp reads one 256-byte row), so each row is one 1x128
+// group. Column pass: thread t owns the column pair 2*(t%64), +1 and the 32 rows
+// 32*(t/64) .. +31; a warp reads 32 consecutive column pairs of one row per load (no
+// bank conflicts) and each thread writes 2 x 32 consecutive codes of the transposed
+// output as two 32-byte runs.
 // ---------------------------------------------------------------------------
-constexpr int kTP = 136;  // row pitch of a staged BF16 tile, in elements (272 bytes)
+constexpr int kTileElems = 128 * 128;
 
-// Column pass over a staged BF16 tile Ts[128][kTP]. Column scales: computed per
-// column (per_col) or the given block scale. Codes go to dst[(c)*ldd + r] for
-// tile column c and tile row r; per-column scales to scol[c] (if not null).
+struct TileSmem {
+  uint8_t* buf[2];
+  uint64_t* bar;  // [2]
+  float* red;     // [4 * 128]
+  int* flag;
+};
+
+// Thread 0 waits for tile buffer b (bounded); every thread then acquires it. Returns
+// false, uniformly across the CTA, if the wait gave up.
+__device__ __forceinline__ bool tile_acquire(const TileSmem& sm, int b, uint32_t parity,
+                                             const WaitCtl& ctl) {
+  if (threadIdx.x == 0) *sm.flag = mbar_wait(sm.bar + b, parity, ctl) ? 1 : 0;
+  __syncthreads();
+  if (!*sm.flag) return false;
+  mbar_try_wait(smem_u32(sm.bar + b), parity);  // completed: acquires the TMA writes
+  return true;
+}
+
+// Column pass over a staged BF16 tile Ts[128][128] (dense rows). Column scales:
+// computed per column (per_col) or the given block scale. Codes go to
+// dst[c * ldd + r] for tile column c and tile row r; per-column scales to scol[c].
 __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, bool per_col,
                                                const GroupScale& blk, uint8_t* __restrict__ dst,
                                                int64_t ldd, float* __restrict__ scol) {
@@ -409,7 +522,7 @@ __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, b
   const int cp = tid & 63, rq = tid >> 6;
   uint32_t w[32];
 #pragma unroll
-  for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(Ts + (32 * rq + r) * kTP + 2 * cp);
+  for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(Ts + (32 * rq + r) * 128 + 2 * cp);
   GroupScale g0 = blk, g1 = blk;
   if (per_col) {
     float a0 = 0.0f, a1 = 0.0f;
@@ -424,8 +537,8 @@ __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, b
     a0 = fmaxf(fmaxf(red[2 * cp], red[128 + 2 * cp]), fmaxf(red[256 + 2 * cp], red[384 + 2 * cp]));
     a1 = fmaxf(fmaxf(red[2 * cp + 1], red[128 + 2 * cp + 1]),
                fmaxf(red[256 + 2 * cp + 1], red[384 + 2 * cp + 1]));
-    g0 = group_scale(a0);
-    g1 = group_scale(a1);
+    g0 = group_scale_bf16(a0);
+    g1 = group_scale_bf16(a1);
     if (rq == 0 && scol) *reinterpret_cast<float2*>(scol + 2 * cp) = make_float2(g0.s, g1.s);
   }
   uint32_t o0[8], o1[8];
@@ -447,161 +560,268 @@ __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, b
   d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
 }
 
-// a2: 128x128 weight blocks. grid = (N/128) * (K/128).
-__global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __restrict__ w,
-                                                           int64_t N, int64_t K, int64_t ldw,
-                                                           uint8_t* __restrict__ q,
-                                                           float* __restrict__ s,
-                                                           uint8_t* __restrict__ qT) {
-  __shared__ float red[8];
-  __shared__ __align__(16) uint16_t Ts[128 * kTP];
-  const int64_t KB = K >> 7;
-  const int64_t nb = blockIdx.x / KB, kb = blockIdx.x % KB;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  const uint16_t* base = w + (nb * 128) * ldw + kb * 128 + c8;
-  uint4 raw[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) raw[j] = ld_nc_v4(base + (rr + 16 * j) * ldw);
-  float a = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    float v[8];
-    unpack_bf16x8(raw[j], v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
-    if (qT) *reinterpret_cast<uint4*>(Ts + (rr + 16 * j) * kTP + c8) = raw[j];
-  }
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
-  if (lane == 0) red[wid] = a;
-  __syncthreads();
-  float amax = red[0];
-#pragma unroll
-  for (int k = 1; k < 8; ++k) amax = fmaxf(amax, red[k]);
-  const GroupScale g = group_scale(amax);
-  if (tid == 0) s[nb * KB + kb] = g.s;
-  uint8_t* qb = q + (nb * 128) * K + kb * 128 + c8;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    float v[8];
-    unpack_bf16x8(raw[j], v);
-    *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes8(v, g);
-  }
-  if (qT) tile_cols_bf16(Ts, nullptr, false, g, qT + (kb * 128) * N + nb * 128, N, nullptr);
+// Shared memory of the BF16 tile kernels: two 32 KB tiles, the column reduction, bars.
+constexpr size_t kTileSmemBF16 = 1024 + 2 * kTileElems * 2 + 4 * 128 * 4 + 64;
+// ... of the FP8 tile kernel: two (16 KB codes + 512 B row scales) buffers.
+constexpr size_t kTileSmemFP8 = 1024 + 2 * (kTileElems + 512) + 4 * 128 * 4 + 64;
+
+__device__ __forceinline__ TileSmem carve_tiles(uint8_t* raw, int buf_bytes) {
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  TileSmem sm;
+  sm.buf[0] = base;
+  sm.buf[1] = base + buf_bytes;
+  sm.red = reinterpret_cast<float*>(base + 2 * buf_bytes);
+  sm.bar = reinterpret_cast<uint64_t*>(base + 2 * buf_bytes + 4 * 128 * 4);
+  sm.flag = reinterpret_cast<int*>(sm.bar + 2);
+  return sm;
 }
 
-// a6: BF16 dY tile -> row-wise 1x128 codes (row pass) + column-wise 128x1 codes
-// (column pass, transposed). grid = (M/128) * (N/128).
-__global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
-    const uint16_t* __restrict__ dy, int64_t M, int64_t N, int64_t lddy,
-    uint8_t* __restrict__ q_row, float* __restrict__ s_row, int64_t lds_row,
-    uint8_t* __restrict__ q_colT, float* __restrict__ s_col) {
-  __shared__ float red[4 * 128];
-  __shared__ __align__(16) uint16_t Ts[128 * kTP];
-  const int64_t NB = N >> 7;
-  const int64_t mb = blockIdx.x / NB, nb = blockIdx.x % NB;
-  const int tid = threadIdx.x;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  const uint16_t* base = dy + (mb * 128) * lddy + nb * 128 + c8;
-  uint4 raw[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) raw[j] = ld_nc_v4(base + (rr + 16 * j) * lddy);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    *reinterpret_cast<uint4*>(Ts + (rr + 16 * j) * kTP + c8) = raw[j];
-    if (q_row) {  // each tile row is one 1x128 group, held by a half-warp
-      float v[8];
-      unpack_bf16x8(raw[j], v);
-      uint2 codes;
-      const float sc = quant_half_warp(v, codes);
-      const int64_t m = mb * 128 + rr + 16 * j;
-      *reinterpret_cast<uint2*>(q_row + m * N + nb * 128 + c8) = codes;
-      if ((tid & 15) == 0) s_row[nb * lds_row + m] = sc;
+// Shared prologue / epilogue of the persistent tile loops. `issue(b, t)` starts the
+// copies of tile t into buffer b (thread 0 only).
+template <class Issue>
+__device__ __forceinline__ void tiles_prologue(const TileSmem& sm, int64_t tiles, Issue issue) {
+  if (threadIdx.x == 0) {
+    mbar_init(sm.bar, 1);
+    mbar_init(sm.bar + 1, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < 2; ++j) {
+      const int64_t t = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
+      if (t < tiles) issue(j, t);
     }
   }
-  __syncthreads();
-  const GroupScale unused{1.0f, 1.0f, false};
-  tile_cols_bf16(Ts, red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
-                 s_col + mb * N + nb * 128);
 }
 
-// a8: saved FP8 activation tile (1x128 groups) -> xhat = fl32(s * dec(q)) ->
-// 128x1 groups along M, stored transposed. grid = (M/128) * (K/128).
-// The codes and row scales are staged in shared memory; the column pass decodes two
-// codes per load. xhat is an arbitrary fp32 value here, so quotients use IEEE
-// division.
-constexpr int kQP = 144;  // row pitch of a staged code tile, in bytes
+// After processing tile number i (buffer i & 1): refill it with the tile two ahead.
+template <class Issue>
+__device__ __forceinline__ void tiles_advance(const TileSmem& sm, int64_t t, int64_t tiles,
+                                              int i, Issue issue) {
+  __syncthreads();  // every thread is done reading the buffer
+  const int64_t tn = t + 2 * static_cast<int64_t>(gridDim.x);
+  if (threadIdx.x == 0 && tn < tiles) issue(i & 1, tn);
+}
 
-__global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
-    const uint8_t* __restrict__ qin, const float* __restrict__ sin, int64_t M, int64_t K,
-    int64_t lds, uint8_t* __restrict__ qT, float* __restrict__ sT) {
-  __shared__ float red[4 * 128];
-  __shared__ float rsc[128];
-  __shared__ __align__(16) uint8_t Tq[128 * kQP];
+// If the loop stopped early, let the copies still in flight land before exiting.
+__device__ __forceinline__ void tiles_drain(const TileSmem& sm, int64_t t_stop, int64_t tiles,
+                                            int i_stop, uint64_t limit_ns) {
+  if (threadIdx.x != 0) return;
+  for (int j = 0; j < 2; ++j) {
+    const int i = i_stop + j;  // tile numbers i_stop, i_stop + 1 may be in flight
+    const int64_t t = t_stop + static_cast<int64_t>(j) * gridDim.x;
+    if (t < tiles) {
+      const uint32_t a = smem_u32(sm.bar + (i & 1));
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(a, (i >> 1) & 1)) {
+        if (global_timer_ns() - t0 > limit_ns) break;
+      }
+    }
+  }
+}
+
+// a2: 128x128 weight blocks, persistent over the (N/128) x (K/128) tiles.
+__global__ void __launch_bounds__(256) quant_weight_kernel(
+    const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t K, uint8_t* __restrict__ q,
+    float* __restrict__ s, uint8_t* __restrict__ qT, unsigned* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  const TileSmem sm = carve_tiles(smem_raw, kTileElems * 2);
+  __shared__ int abort_flag;
+  const WaitCtl ctl{&abort_flag, err, limit_ns};
+  if (threadIdx.x == 0) abort_flag = 0;
   const int64_t KB = K >> 7;
-  const int64_t mb = blockIdx.x / KB, kb = blockIdx.x % KB;
-  const int tid = threadIdx.x;
-  {
-    const int rr = tid >> 3, c16 = (tid & 7) * 16;  // 32 rows x 8 chunks of 16 bytes per pass
-    const uint8_t* base = qin + (mb * 128) * K + kb * 128 + c16;
-    uint4 raw[4];
+  const int64_t tiles = (N >> 7) * KB;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int rr = tid >> 4, c8 = (tid & 15) * 8;
+  auto issue = [&](int b, int64_t t) {
+    mbar_arrive_expect_tx(sm.bar + b, kTileElems * 2);
+    tma_load_2d(sm.buf[b], &tmW, static_cast<int32_t>((t % KB) * 128),
+                static_cast<int32_t>((t / KB) * 128), sm.bar + b);
+  };
+  tiles_prologue(sm, tiles, issue);
+  int i = 0;
+  int64_t t = blockIdx.x;
+  for (; t < tiles; t += gridDim.x, ++i) {
+    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    const uint16_t* Ts = reinterpret_cast<const uint16_t*>(sm.buf[i & 1]);
+    const int64_t nb = t / KB, kb = t % KB;
+    uint4 raw[8];
+    float a = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) raw[j] = ld_nc_v4(base + (rr + 32 * j) * K);
-    if (tid < 128) rsc[tid] = sin[kb * lds + mb * 128 + tid];
+    for (int j = 0; j < 8; ++j) {
+      raw[j] = *reinterpret_cast<const uint4*>(Ts + (rr + 16 * j) * 128 + c8);
+      float v[8];
+      unpack_bf16x8(raw[j], v);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(Tq + (rr + 32 * j) * kQP + c16) = raw[j];
+      for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(v[k]));
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
+    if (lane == 0) sm.red[wid] = a;
+    __syncthreads();
+    float amax = sm.red[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) amax = fmaxf(amax, sm.red[k]);
+    const GroupScale g = group_scale_bf16(amax);
+    if (tid == 0) s[nb * KB + kb] = g.s;
+    uint8_t* qb = q + (nb * 128) * K + kb * 128 + c8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float v[8];
+      unpack_bf16x8(raw[j], v);
+      *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes8(v, g);
+    }
+    if (qT) tile_cols_bf16(Ts, nullptr, false, g, qT + (kb * 128) * N + nb * 128, N, nullptr);
+    tiles_advance(sm, t, tiles, i, issue);
   }
-  __syncthreads();
-  const int cp = tid & 63, rq = tid >> 6;
-  float x0[32], x1[32];
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    const int row = 32 * rq + r;
-    const uint16_t two = *reinterpret_cast<const uint16_t*>(Tq + row * kQP + 2 * cp);
-    const float2 d = e4m3x2_to_f32(two);
-    const float sr = rsc[row];
-    x0[r] = __fmul_rn(sr, d.x);
-    x1[r] = __fmul_rn(sr, d.y);
-  }
-  float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    a0 = fmaxf(a0, fabsf(x0[r]));
-    a1 = fmaxf(a1, fabsf(x1[r]));
-  }
-  red[rq * 128 + 2 * cp] = a0;
-  red[rq * 128 + 2 * cp + 1] = a1;
-  __syncthreads();
-  a0 = fmaxf(fmaxf(red[2 * cp], red[128 + 2 * cp]), fmaxf(red[256 + 2 * cp], red[384 + 2 * cp]));
-  a1 = fmaxf(fmaxf(red[2 * cp + 1], red[128 + 2 * cp + 1]),
-             fmaxf(red[256 + 2 * cp + 1], red[384 + 2 * cp + 1]));
-  const float s0 = (a0 == 0.0f) ? 1.0f : __fdiv_rn(a0, 448.0f);
-  const float s1 = (a1 == 0.0f) ? 1.0f : __fdiv_rn(a1, 448.0f);
-  if (rq == 0) *reinterpret_cast<float2*>(sT + mb * K + kb * 128 + 2 * cp) = make_float2(s0, s1);
-  uint32_t o0[8], o1[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    o0[k] = cvt_e4m3x4(__fdiv_rn(x0[4 * k], s0), __fdiv_rn(x0[4 * k + 1], s0),
-                       __fdiv_rn(x0[4 * k + 2], s0), __fdiv_rn(x0[4 * k + 3], s0));
-    o1[k] = cvt_e4m3x4(__fdiv_rn(x1[4 * k], s1), __fdiv_rn(x1[4 * k + 1], s1),
-                       __fdiv_rn(x1[4 * k + 2], s1), __fdiv_rn(x1[4 * k + 3], s1));
-  }
-  uint8_t* dst = qT + (kb * 128) * M + mb * 128;
-  uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * M + 32 * rq);
-  uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * M + 32 * rq);
-  d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-  d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
-  d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-  d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
 
-int grid_for_units(int64_t warps_needed) {
-  const int sms = sm100_sm_count();
-  int64_t ctas = (warps_needed + 7) / 8;
-  const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 CTAs x 256 threads = 2048 per SM
-  if (ctas > cap) ctas = cap;
-  return static_cast<int>(ctas < 1 ? 1 : ctas);
+// a6: BF16 dY tiles -> row-wise 1x128 codes (row pass) + column-wise 128x1 codes
+// (column pass, transposed), persistent over the (M/128) x (N/128) tiles.
+__global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
+    const __grid_constant__ CUtensorMap tmDY, int64_t M, int64_t N, uint8_t* __restrict__ q_row,
+    float* __restrict__ s_row, int64_t lds_row, uint8_t* __restrict__ q_colT,
+    float* __restrict__ s_col, unsigned* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  const TileSmem sm = carve_tiles(smem_raw, kTileElems * 2);
+  __shared__ int abort_flag;
+  const WaitCtl ctl{&abort_flag, err, limit_ns};
+  if (threadIdx.x == 0) abort_flag = 0;
+  const int64_t NB = N >> 7;
+  const int64_t tiles = (M >> 7) * NB;
+  const int tid = threadIdx.x;
+  const int rr = tid >> 4, c8 = (tid & 15) * 8;
+  auto issue = [&](int b, int64_t t) {
+    mbar_arrive_expect_tx(sm.bar + b, kTileElems * 2);
+    tma_load_2d(sm.buf[b], &tmDY, static_cast<int32_t>((t % NB) * 128),
+                static_cast<int32_t>((t / NB) * 128), sm.bar + b);
+  };
+  tiles_prologue(sm, tiles, issue);
+  const GroupScale unused{1.0f, 1.0f, -1.0f, false};
+  int i = 0;
+  int64_t t = blockIdx.x;
+  for (; t < tiles; t += gridDim.x, ++i) {
+    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    const uint16_t* Ts = reinterpret_cast<const uint16_t*>(sm.buf[i & 1]);
+    const int64_t mb = t / NB, nb = t % NB;
+    if (q_row) {  // each tile row is one 1x128 group, held by a half-warp
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v[8];
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(Ts + (rr + 16 * j) * 128 + c8), v);
+        uint2 codes;
+        const float sc = quant_half_warp(v, codes);
+        const int64_t m = mb * 128 + rr + 16 * j;
+        *reinterpret_cast<uint2*>(q_row + m * N + nb * 128 + c8) = codes;
+        if ((tid & 15) == 0) s_row[nb * lds_row + m] = sc;
+      }
+    }
+    tile_cols_bf16(Ts, sm.red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
+                   s_col + mb * N + nb * 128);
+    tiles_advance(sm, t, tiles, i, issue);
+  }
+  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
+}
+
+// a8: saved FP8 activation tiles (1x128 groups) -> xhat = fl32(s * dec(q)) -> 128x1
+// groups along M, stored transposed; persistent over the (M/128) x (K/128) tiles.
+// Each buffer holds the 16 KB code tile and its 128 row scales. xhat is an arbitrary
+// fp32 value here, so the quotients use IEEE division.
+__global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS, int64_t M,
+    int64_t K, uint8_t* __restrict__ qT, float* __restrict__ sT, unsigned* err,
+    uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  const TileSmem sm = carve_tiles(smem_raw, kTileElems + 512);
+  __shared__ int abort_flag;
+  const WaitCtl ctl{&abort_flag, err, limit_ns};
+  if (threadIdx.x == 0) abort_flag = 0;
+  const int64_t KB = K >> 7;
+  const int64_t tiles = (M >> 7) * KB;
+  const int tid = threadIdx.x;
+  auto issue = [&](int b, int64_t t) {
+    const int32_t mx = static_cast<int32_t>((t / KB) * 128), kx = static_cast<int32_t>(t % KB);
+    mbar_arrive_expect_tx(sm.bar + b, kTileElems + 512);
+    tma_load_2d(sm.buf[b], &tmQ, kx * 128, mx, sm.bar + b);
+    tma_load_2d(sm.buf[b] + kTileElems, &tmS, mx, kx, sm.bar + b);
+  };
+  tiles_prologue(sm, tiles, issue);
+  const int cp = tid & 63, rq = tid >> 6;
+  int i = 0;
+  int64_t t = blockIdx.x;
+  for (; t < tiles; t += gridDim.x, ++i) {
+    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    const uint8_t* Tq = sm.buf[i & 1];
+    const float* rsc = reinterpret_cast<const float*>(Tq + kTileElems);
+    const int64_t mb = t / KB, kb = t % KB;
+    float x0[32], x1[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const int row = 32 * rq + r;
+      const uint16_t two = *reinterpret_cast<const uint16_t*>(Tq + row * 128 + 2 * cp);
+      const float2 d = e4m3x2_to_f32(two);
+      const float sr = rsc[row];
+      x0[r] = __fmul_rn(sr, d.x);
+      x1[r] = __fmul_rn(sr, d.y);
+    }
+    float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      a0 = fmaxf(a0, fabsf(x0[r]));
+      a1 = fmaxf(a1, fabsf(x1[r]));
+    }
+    sm.red[rq * 128 + 2 * cp] = a0;
+    sm.red[rq * 128 + 2 * cp + 1] = a1;
+    __syncthreads();
+    a0 = fmaxf(fmaxf(sm.red[2 * cp], sm.red[128 + 2 * cp]),
+               fmaxf(sm.red[256 + 2 * cp], sm.red[384 + 2 * cp]));
+    a1 = fmaxf(fmaxf(sm.red[2 * cp + 1], sm.red[128 + 2 * cp + 1]),
+               fmaxf(sm.red[256 + 2 * cp + 1], sm.red[384 + 2 * cp + 1]));
+    const float s0 = (a0 == 0.0f) ? 1.0f : __fdiv_rn(a0, 448.0f);
+    const float s1 = (a1 == 0.0f) ? 1.0f : __fdiv_rn(a1, 448.0f);
+    if (rq == 0) *reinterpret_cast<float2*>(sT + mb * K + kb * 128 + 2 * cp) = make_float2(s0, s1);
+    uint32_t o0[8], o1[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      o0[k] = cvt_e4m3x4(__fdiv_rn(x0[4 * k], s0), __fdiv_rn(x0[4 * k + 1], s0),
+                         __fdiv_rn(x0[4 * k + 2], s0), __fdiv_rn(x0[4 * k + 3], s0));
+      o1[k] = cvt_e4m3x4(__fdiv_rn(x1[4 * k], s1), __fdiv_rn(x1[4 * k + 1], s1),
+                         __fdiv_rn(x1[4 * k + 2], s1), __fdiv_rn(x1[4 * k + 3], s1));
+    }
+    uint8_t* dst = qT + (kb * 128) * M + mb * 128;
+    uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * M + 32 * rq);
+    uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * M + 32 * rq);
+    d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+    d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
+    d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+    d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+    tiles_advance(sm, t, tiles, i, issue);
+  }
+  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
+}
+
+// Resident CTAs per SM of a kernel (cached per device), for grid-stride/persistent grids.
+template <class Kernel>
+int resident_ctas(Kernel k, int threads, size_t dyn_smem, int* cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  if (cache[dev]) return cache[dev];
+  if (dyn_smem > 48 * 1024)
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn_smem));
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, dyn_smem) != cudaSuccess || n < 1)
+    n = 1;
+  cudaGetLastError();
+  cache[dev] = n;
+  return n;
+}
+
+int grid_for(int64_t ctas_needed, int per_sm) {
+  const int64_t cap = static_cast<int64_t>(sm100_sm_count()) * per_sm;
+  const int64_t g = ctas_needed < cap ? ctas_needed : cap;
+  return static_cast<int>(g < 1 ? 1 : g);
 }
 
 }  // namespace
@@ -617,7 +837,9 @@ extern "C" fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   const int64_t G = K / 128;
   const int64_t units = M * ((G + 1) / 2);
-  rowgroup_quant_kernel<ActSrc, 4><<<grid_for_units((units + 3) / 4), 256, 0,
+  static int occ[64];
+  const int per_sm = resident_ctas(rowgroup_quant_kernel<ActSrc, 4>, 256, 0, occ);
+  rowgroup_quant_kernel<ActSrc, 4><<<grid_for((units + 31) / 32, per_sm), 256, 0,
                                      static_cast<cudaStream_t>(stream)>>>(ActSrc{x, ldx}, M, G, q,
                                                                           K, s, lds);
   return launch_status("quant_act_1x128 launch");
@@ -631,7 +853,9 @@ extern "C" fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t 
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   const int64_t G = I / 128;
   const int64_t units = M * ((G + 1) / 2);
-  rowgroup_quant_kernel<SwigluSrc, 2><<<grid_for_units((units + 1) / 2), 256, 0,
+  static int occ[64];
+  const int per_sm = resident_ctas(rowgroup_quant_kernel<SwigluSrc, 2>, 256, 0, occ);
+  rowgroup_quant_kernel<SwigluSrc, 2><<<grid_for((units + 15) / 16, per_sm), 256, 0,
                                         static_cast<cudaStream_t>(stream)>>>(
       SwigluSrc{gu, ldgu, I}, M, G, q, I, s, lds);
   return launch_status("swiglu_quant launch");
@@ -650,14 +874,18 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (H <= 8 * 32 * kWarpRowChunks) {
-    const int64_t ctas = (M + 7) / 8;
-    const int64_t grid = ctas < static_cast<int64_t>(sms) * 8 ? ctas : static_cast<int64_t>(sms) * 8;
-    if (H <= 8 * 32 * 16)
-      rmsnorm_quant_warp_kernel<16><<<static_cast<int>(grid), 256, 0, st>>>(x, gamma, M, H, ldx,
+    const int64_t ctas = (M + 7) / 8;  // one warp per row
+    if (H <= 8 * 32 * 16) {
+      static int occ[64];
+      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<16>, 256, 0, occ);
+      rmsnorm_quant_warp_kernel<16><<<grid_for(ctas, per_sm), 256, 0, st>>>(x, gamma, M, H, ldx,
                                                                             eps, q, s, lds);
-    else
-      rmsnorm_quant_warp_kernel<kWarpRowChunks><<<static_cast<int>(grid), 256, 0, st>>>(
+    } else {
+      static int occ[64];
+      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<kWarpRowChunks>, 256, 0, occ);
+      rmsnorm_quant_warp_kernel<kWarpRowChunks><<<grid_for(ctas, per_sm), 256, 0, st>>>(
           x, gamma, M, H, ldx, eps, q, s, lds);
+    }
   } else {
     const int64_t grid = M < static_cast<int64_t>(sms) * 64 ? M : static_cast<int64_t>(sms) * 64;
     rmsnorm_quant_cta_kernel<<<static_cast<int>(grid), kNormThreads, 0, st>>>(x, gamma, M, H, ldx,
@@ -674,10 +902,16 @@ extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, i
   if (!aligned16(w) || !aligned16(q) || !aligned16(s) || (qT && !aligned16(qT)) || ldw % 8)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  const int64_t blocks = (N / 128) * (K / 128);
-  if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  quant_weight_kernel<<<static_cast<unsigned>(blocks), 256, 0,
-                        static_cast<cudaStream_t>(stream)>>>(w, N, K, ldw, q, s, qT);
+  CUtensorMap tm;
+  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, ldw * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  static int occ[64];
+  const int per_sm = resident_ctas(quant_weight_kernel, 256, kTileSmemBF16, occ);
+  quant_weight_kernel<<<grid_for((N / 128) * (K / 128), per_sm), 256, kTileSmemBF16,
+                        static_cast<cudaStream_t>(stream)>>>(tm, N, K, q, s, qT, err, kWaitLimitNs);
   return launch_status("quant_weight_128x128 launch");
 }
 
@@ -692,11 +926,17 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
       (q_row && (!aligned16(q_row) || !aligned16(s_row))))
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  const int64_t blocks = (M / 128) * (N / 128);
-  if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  transpose_quant_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0,
-                                static_cast<cudaStream_t>(stream)>>>(dy, M, N, lddy, q_row, s_row,
-                                                                     lds_row, q_colT, s_col);
+  CUtensorMap tm;
+  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, N, M, lddy * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  static int occ[64];
+  const int per_sm = resident_ctas(transpose_quant_bf16_kernel, 256, kTileSmemBF16, occ);
+  transpose_quant_bf16_kernel<<<grid_for((M / 128) * (N / 128), per_sm), 256, kTileSmemBF16,
+                                static_cast<cudaStream_t>(stream)>>>(
+      tm, M, N, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
   return launch_status("transpose_quant_bf16 launch");
 }
 
@@ -708,9 +948,18 @@ extern "C" fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s
   if (!aligned16(q) || !aligned16(s) || !aligned16(qT) || !aligned16(sT) || lds % 4)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  const int64_t blocks = (M / 128) * (K / 128);
-  if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  transpose_quant_fp8_kernel<<<static_cast<unsigned>(blocks), 256, 0,
-                               static_cast<cudaStream_t>(stream)>>>(q, s, M, K, lds, qT, sT);
+  CUtensorMap tmq, tms;
+  if (!encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, M, K, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, s, M, K / 128, lds * 4, 128, 1,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  static int occ[64];
+  const int per_sm = resident_ctas(transpose_quant_fp8_kernel, 256, kTileSmemFP8, occ);
+  transpose_quant_fp8_kernel<<<grid_for((M / 128) * (K / 128), per_sm), 256, kTileSmemFP8,
+                               static_cast<cudaStream_t>(stream)>>>(tmq, tms, M, K, qT, sT, err,
+                                                                    kWaitLimitNs);
   return launch_status("transpose_quant_fp8 launch");
 }

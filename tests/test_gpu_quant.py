@@ -82,7 +82,7 @@ def test_special_groups(fq, oracle_mod):
     xv[2, :128] = 0x0001         # smallest BF16 subnormal everywhere
     xv[2, 7] = -32765            # 0x8003: -3 x 2^-133
     x[3, 128] = -1e-30
-    x[4, :] = torch.linspace(-3e38, 3e38, 256)
+    x[4, :] = torch.linspace(-3e38, 3e38, 256, dtype=torch.float64)  # finite (fp64 steps)
     x[5, 130] = 3.0
     x[5, 131] = -0.0
     q, s = run_act(fq, x.to(DEV))
