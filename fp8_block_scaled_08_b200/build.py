@@ -24,7 +24,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libfp8q.so")
-SOURCES = ["fp8q_api.cu", "fp8q_quant.cu", "fp8q_gemm.cu"]
+SOURCES = ["fp8q_api.cu", "fp8q_quant.cu", "fp8q_gemm.cu", "fp8q_gemm_skinny.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [

@@ -523,6 +523,9 @@ extern "C" fp8q_status fp8q_linear_fwd(const uint8_t* qa, const float* sa, int64
       ldsa % 4 || ldy % 8)
     return FP8Q_ERR_ALIGN;
   // B = W [N][K]; block scale of (n, slice r) = sw[(n/128)*(K/128) + r]
+  if (M <= kSkinnyMaxM)
+    return launch_skinny_gemm(qa, qw, M, N, K, sa, ldsa, sw, K / 128, 1, y, ldy,
+                              static_cast<cudaStream_t>(stream));
   return launch_gemm<false, true>(qa, qw, M, N, K, sa, ldsa, sw, K / 128, 1, nullptr, y, ldy,
                             static_cast<cudaStream_t>(stream));
 }
@@ -539,6 +542,9 @@ extern "C" fp8q_status fp8q_linear_dgrad(const uint8_t* qdy, const float* sdy, i
     return FP8Q_ERR_ALIGN;
   // GEMM rows = M, columns = K, reduction = N. B = W^T [K][N];
   // block scale of (k, slice r over n) = sw[r*(K/128) + k/128]
+  if (M <= kSkinnyMaxM)
+    return launch_skinny_gemm(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, K / 128, dx, lddx,
+                              static_cast<cudaStream_t>(stream));
   return launch_gemm<false, true>(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, K / 128, nullptr, dx, lddx,
                             static_cast<cudaStream_t>(stream));
 }

@@ -1,0 +1,331 @@
+// Skinny-M block-scaled FP8 GEMM for sm_100a: the forward (and DGrad) of the linear
+// layer when the token batch is small (decode, M <= 256).
+//
+//   out[i, j] = sum_r  sA(i, r) * sB(j / 128, r) * sum_{l in slice r} qA[i, l] * qB[j, l]
+//
+// with the same operands, scales and promotion order as the large-tile kernel
+// ("Resumen Técnico: Jet-RL", section "Esquema de Cuantización": 1x128 activation
+// groups, 128x128 weight blocks). At these sizes the layer is bound by reading the
+// FP8 weights (about 2M flops per weight byte, far below the tensor-core ridge), so the
+// design goal is many SMs streaming weights at once with enough bytes in flight:
+//
+//  * Each CTA owns a narrow strip of kBN (16, 32 or 64) weight rows and at most 128
+//    token rows, over the whole K. Strips are independent: no split-K, so every output
+//    element is promoted slice after slice in increasing r, exactly as in the
+//    large-tile kernel (acc = fma(P_r, sA*sB, acc) from +0), and a row of the output has
+//    the same bits whatever M is ("Arquitectura Central": the rollout graph is a
+//    subgraph of the training graph).
+//  * tcgen05.mma.cta_group::1, M = 128 (token rows; rows past the batch are left as
+//    whatever the shared-memory tile holds and their accumulator lanes are never read),
+//    N = kBN, K = 32, four per 128-wide slice, into one of up to 8 TMEM accumulator
+//    buffers, so the tensor core runs ahead of the promotion by several slices.
+//  * A TMA ring of up to 16 stages (token rows of A, weight strip of B), sized to about
+//    96 KB of shared memory so that two CTAs fit on an SM.
+//  * 192 threads: warp 0 TMA producer, warp 1 TMEM allocation + MMA issue, warps 2-5
+//    promotion (warp w reads TMEM lanes 32*(w%4) .. +31; only the quarters that hold
+//    token rows work). Promotion adds each slice into kBN fp32 registers per thread;
+//    the epilogue rounds to BF16 and stores each token row's kBN outputs directly.
+// Every mbarrier wait is bounded; a wait that gives up records FP8Q_ERR_TIMEOUT in the
+// device error word and the CTA winds down.
+#include <algorithm>
+
+#include "fp8q_device.cuh"
+#include "fp8q_host.h"
+
+namespace fp8q {
+namespace {
+
+constexpr int kSkThreads = 192;
+constexpr int kSkBK = 128;
+constexpr int kSkMaxStages = 16;
+constexpr uint32_t kSkSmemTarget = 96 * 1024;
+constexpr uint32_t kSkATileRead = 128 * kSkBK;  // the MMA reads 128 rows of A
+
+struct SkinnyParams {
+  int32_t M, N, kblocks;
+  int32_t mtiles;
+  int32_t stages;
+  uint32_t a_stage, b_stage;  // bytes per stage (1024-aligned)
+  uint32_t a_rows;            // rows per A box
+  uint32_t off_bars;
+  const float* sa;
+  int64_t ldsa;
+  const float* sb;
+  int64_t sb_sj, sb_sr;
+  uint16_t* y;
+  int64_t ldy;
+  unsigned* err;
+  uint64_t wait_limit_ns;
+};
+
+template <int kBN>
+struct SkinnyShape {
+  static constexpr int kBufs = (kBN * 8 <= 256) ? 8 : 256 / kBN;  // accumulator buffers
+  static constexpr uint32_t kTmemCols = kBufs * kBN < 32 ? 32 : kBufs * kBN;
+  static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 64, "N of a cta_group::1 M=128 MMA");
+  static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM allocations are powers of two");
+};
+
+__device__ __forceinline__ void sk_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return;
+  }
+}
+
+template <int kBN>
+__device__ __forceinline__ void sk_tmem_load(uint32_t taddr, uint32_t (&r)[kBN]) {
+  if constexpr (kBN == 16) {
+    tmem_ld16(taddr, r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < kBN / 32; ++c)
+      tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+  }
+  tmem_wait_ld();
+}
+
+template <int kBN>
+__global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const SkinnyParams p) {
+  using Shape = SkinnyShape<kBN>;
+  constexpr int kBufs = Shape::kBufs;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int S = p.stages;
+  uint8_t* a_ring = smem;
+  uint8_t* b_ring = smem + S * p.a_stage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bars);
+  uint64_t* empty = full + kSkMaxStages;
+  uint64_t* tfull = empty + kSkMaxStages;
+  uint64_t* tempty = tfull + kBufs;
+  uint64_t* done = tempty + kBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int mt = blockIdx.x % p.mtiles;
+  const int nt = blockIdx.x / p.mtiles;
+  const int m0 = mt * 128;
+  const int n0 = nt * kBN;
+  const int rows = min(128, p.M - m0);       // token rows of this tile
+  const int quarters = (rows + 31) >> 5;     // TMEM lane quarters that hold them
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < kBufs; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, quarters);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) tmem_alloc<Shape::kTmemCols>(tmem_slot);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.err, p.wait_limit_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t stage_tx = p.a_rows * kSkBK + kBN * kSkBK;
+      int issued = 0;
+      bool ok = true;
+      for (int kb = 0; kb < p.kblocks; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = static_cast<uint32_t>(kb / S) & 1u;
+        if (!mbar_wait(empty + s, ph ^ 1u, ctl)) { ok = false; break; }
+        mbar_arrive_expect_tx(full + s, stage_tx);
+        tma_load_2d(a_ring + s * p.a_stage, &tmA, kb * kSkBK, m0, full + s);
+        tma_load_2d(b_ring + s * p.b_stage, &tmB, kb * kSkBK, n0, full + s);
+        issued = kb + 1;
+      }
+      if (!ok)  // let the copies still in flight land before the CTA exits
+        for (int kb = max(0, issued - S); kb < issued; ++kb)
+          sk_wait_drain(full + kb % S, static_cast<uint32_t>(kb / S) & 1u, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_e4m3_f32(128, kBN);
+      bool ok = true;
+      for (int kb = 0; kb < p.kblocks; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = static_cast<uint32_t>(kb / S) & 1u;
+        const int buf = kb % kBufs;
+        const uint32_t tph = static_cast<uint32_t>(kb / kBufs) & 1u;
+        if (!mbar_wait(full + s, ph, ctl)) { ok = false; break; }
+        if (!mbar_wait(tempty + buf, tph ^ 1u, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(a_ring + s * p.a_stage);
+        const uint32_t b0 = smem_u32(b_ring + s * p.b_stage);
+        const uint32_t d = tmem_base + buf * kBN;
+#pragma unroll
+        for (int k = 0; k < kSkBK / 32; ++k)
+          mma_f8f6f4(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc,
+                     k > 0 ? 1u : 0u);
+        mma_commit(empty + s);
+        mma_commit(tfull + buf);
+      }
+      (void)ok;
+      // every MMA issued so far has finished reading shared memory and writing TMEM
+      mma_commit(done);
+      sk_wait_drain(done, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ promotion + epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    if (q < quarters) {
+      const int row = q * 32 + lane;
+      const int m = m0 + row;
+      const bool row_ok = m < p.M;
+      const float* sap = p.sa + (row_ok ? m : 0);
+      const float* sbp = p.sb + static_cast<int64_t>(n0 / 128) * p.sb_sj;
+      float acc[kBN];
+#pragma unroll
+      for (int i = 0; i < kBN; ++i) acc[i] = 0.0f;
+      float san = __ldg(sap), sbn = __ldg(sbp);
+      bool ok = true;
+      for (int kb = 0; kb < p.kblocks; ++kb) {
+        const float sa = san, sb = sbn;
+        if (kb + 1 < p.kblocks) {  // next slice's scales, one slice ahead
+          san = __ldg(sap + static_cast<int64_t>(kb + 1) * p.ldsa);
+          sbn = __ldg(sbp + static_cast<int64_t>(kb + 1) * p.sb_sr);
+        }
+        const int buf = kb % kBufs;
+        const uint32_t tph = static_cast<uint32_t>(kb / kBufs) & 1u;
+        if (!mbar_wait_warp(tfull + buf, tph, ctl)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[kBN];
+        sk_tmem_load<kBN>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN, r);
+        const float s = __fmul_rn(sa, sb);
+#pragma unroll
+        for (int i = 0; i < kBN; i += 2)
+          fma2(acc[i], acc[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), s, s);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty + buf);
+      }
+      if (ok && row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m) * p.ldy + n0);
+#pragma unroll
+        for (int c = 0; c < kBN / 8; ++c) {
+          const float* a = acc + 8 * c;
+          dst[c] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                              pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<Shape::kTmemCols>(tmem_base);
+  }
+}
+
+// Per device and strip width: opt in to the shared memory the launch asks for.
+template <int kBN>
+bool skinny_setup(size_t smem_bytes) {
+  static size_t opted[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (opted[dev] >= smem_bytes) return true;
+  const cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel<kBN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem_bytes));
+  if (e != cudaSuccess) {
+    set_last_error("cudaFuncSetAttribute(skinny_gemm)", e);
+    cudaGetLastError();
+    return false;
+  }
+  opted[dev] = smem_bytes;
+  return true;
+}
+
+template <int kBN>
+fp8q_status launch_skinny(const CUtensorMap& tmA, const uint8_t* B, int64_t Ng, int64_t Kg,
+                          SkinnyParams p, cudaStream_t stream) {
+  using Shape = SkinnyShape<kBN>;
+  CUtensorMap tmB;
+  if (!encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, Kg, Ng, Kg, kSkBK, kBN,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8Q_ERR_UNSUPPORTED;
+  p.b_stage = kBN * kSkBK;  // 16 rows x 128 B = 2 KB: a multiple of the 1024-byte atom
+  const uint32_t per_stage = p.a_stage + p.b_stage;
+  p.stages = static_cast<int32_t>(
+      std::clamp<uint32_t>(kSkSmemTarget / per_stage, 2u, static_cast<uint32_t>(kSkMaxStages)));
+  uint32_t data = p.stages * per_stage;
+  // the MMA reads 128 rows from the last A stage: keep that inside the allocation
+  data = std::max<uint32_t>(data, (p.stages - 1) * p.a_stage + kSkATileRead);
+  p.off_bars = (data + 7u) & ~7u;
+  const uint32_t bars = (2 * kSkMaxStages + 2 * Shape::kBufs + 1) * 8 + 16;
+  const size_t smem = p.off_bars + bars + 1024;
+  if (smem > 232448) return FP8Q_ERR_UNSUPPORTED;
+  if (!skinny_setup<kBN>(smem)) return FP8Q_ERR_CUDA;
+  const int64_t grid = static_cast<int64_t>(p.mtiles) * (Ng / kBN);
+  if (grid > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  skinny_gemm_kernel<kBN><<<static_cast<unsigned>(grid), kSkThreads, smem, stream>>>(tmA, tmB, p);
+  return launch_status("skinny_gemm_kernel launch");
+}
+
+}  // namespace
+
+fp8q_status launch_skinny_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t Ng,
+                               int64_t Kg, const float* sa, int64_t ldsa, const float* sb,
+                               int64_t sb_sj, int64_t sb_sr, uint16_t* y, int64_t ldy,
+                               cudaStream_t stream) {
+  const int sms = sm100_sm_count();
+  if (!sms) return FP8Q_ERR_UNSUPPORTED;
+  if (Mg <= 0 || Mg > kSkinnyMaxM || Ng % 128 || Kg % 128 || Ng > 0x7FFFFFFF ||
+      Kg > 0x7FFFFFFF)
+    return FP8Q_ERR_SHAPE;
+  SkinnyParams p;
+  p.M = static_cast<int32_t>(Mg);
+  p.N = static_cast<int32_t>(Ng);
+  p.kblocks = static_cast<int32_t>(Kg / kSkBK);
+  p.mtiles = static_cast<int32_t>((Mg + 127) / 128);
+  // A box: the token rows (a multiple of 8, at most 128); rows past M read as zeros
+  p.a_rows = static_cast<uint32_t>(std::min<int64_t>(128, (Mg + 7) / 8 * 8));
+  p.a_stage = (p.a_rows * kSkBK + 1023u) & ~1023u;
+  p.sa = sa;
+  p.ldsa = ldsa;
+  p.sb = sb;
+  p.sb_sj = sb_sj;
+  p.sb_sr = sb_sr;
+  p.y = y;
+  p.ldy = ldy;
+  p.err = device_error_word();
+  p.wait_limit_ns = kWaitLimitNs;
+  if (!p.err) return FP8Q_ERR_CUDA;
+  CUtensorMap tmA;
+  if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, Kg, Mg, Kg, kSkBK, p.a_rows,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8Q_ERR_UNSUPPORTED;
+  // Strip width: the widest strip that still gives every SM at least one CTA (wider
+  // strips re-read the token rows from L2 fewer times); 16 if none does.
+  const int64_t mt = p.mtiles;
+  if (mt * (Ng / 64) >= sms) return launch_skinny<64>(tmA, B, Ng, Kg, p, stream);
+  if (mt * (Ng / 32) >= sms) return launch_skinny<32>(tmA, B, Ng, Kg, p, stream);
+  return launch_skinny<16>(tmA, B, Ng, Kg, p, stream);
+}
+
+}  // namespace fp8q

@@ -38,4 +38,15 @@ inline fp8q_status launch_status(const char* where = "launch") {
 // Bounded waits inside the kernels give up after this long (nanoseconds).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Token batches up to this many rows take the skinny-M GEMM (forward and DGrad).
+constexpr int64_t kSkinnyMaxM = 256;
+
+// out [Mg][Ng] = A [Mg][Kg] x B [Ng][Kg]^T with per-row A scales sa[r*ldsa + i] and
+// per-128x128-block B scales sb[(j/128)*sb_sj + r*sb_sr], for Mg <= kSkinnyMaxM.
+// Same arithmetic, in the same order, as the large-tile kernel.
+fp8q_status launch_skinny_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t Ng,
+                               int64_t Kg, const float* sa, int64_t ldsa, const float* sb,
+                               int64_t sb_sj, int64_t sb_sr, uint16_t* y, int64_t ldy,
+                               cudaStream_t stream);
+
 }  // namespace fp8q
