@@ -10,7 +10,8 @@
 // value nearest to the IEEE quotient x/s. Where x is a BF16 value (every quantizer
 // but the FP8 requantizer) the quotient is formed from the correctly rounded
 // reciprocal r = 1/s with one residual correction (q = x*r; e = fma(-q, s, x);
-// q = fma(e, r, q); sign of x), which yields the same E4M3 code as the IEEE quotient
+// q = fma(e, r, q); sign of x; the kernels evaluate it as q - (q*s - x)*r, which keeps
+// the sign of -0 by itself), which yields the same E4M3 code as the IEEE quotient
 // for every BF16 x and every BF16 amax >= |x| with s >= 2^-80 (checked exhaustively by
 // the test suite); groups with smaller s use the IEEE division itself.
 //
@@ -106,61 +107,69 @@ __constant__ float kRecipMant[128] = {
 
 // Same result as group_scale for every amax that is a BF16 value (the maximum of BF16
 // values is one). amax < 2^-71 (s below about 2^-80), and non-finite amax (outside the
-// contract), take the division path.
+// contract), take the division path; the branch is taken per warp, only when one of its
+// lanes needs it.
 __device__ __forceinline__ GroupScale group_scale_bf16(float amax) {
-  GroupScale g;
   const uint32_t b = __float_as_uint(amax);
   const int ebias = static_cast<int>(b >> 23);  // biased exponent (amax >= 0)
-  if (ebias < 127 - 71 || ebias == 255) {
-    g = group_scale(amax);
-    g.small = true;
-    return g;
-  }
+  const bool tiny = ebias < 127 - 71 || ebias == 255;
   const int e = ebias - 127;
   const uint32_t i = (b >> 16) & 0x7Fu;
+  GroupScale g;
   g.s = __uint_as_float(__float_as_uint(kScaleMant[i]) + static_cast<uint32_t>((e - 6) << 23));
   g.rs = __uint_as_float(__float_as_uint(kRecipMant[i]) + static_cast<uint32_t>((6 - e) << 23));
-  g.ns = -g.s;
   g.small = false;
+  if (__any_sync(kFull, tiny)) {
+    if (tiny) {
+      g = group_scale(amax);
+      g.small = true;
+    }
+  }
+  g.ns = -g.s;
   return g;
 }
 
-__device__ __forceinline__ float copy_sign(float v, float sgn) {
-  return __uint_as_float((__float_as_uint(v) & 0x7FFFFFFFu) | (__float_as_uint(sgn) & 0x80000000u));
+// x/s for a BF16-valued x (see the file header for why this has the IEEE quotient's
+// code): q = x*r, then q - (q*s - x)*r. Written this way the sign of x = -0 survives
+// without a separate copy-sign (q*s - x is +0 and q - (+0)*r is -0 + -0).
+__device__ __forceinline__ float quot(float x, const GroupScale& g) {
+  const float q = __fmul_rn(x, g.rs);
+  const float en = __fmaf_rn(q, g.s, -x);
+  return __fmaf_rn(en, -g.rs, q);
 }
 
-// Two quotients x/s of BF16-valued x (see the file header for why this equals the
-// IEEE quotient's code).
-__device__ __forceinline__ void quotient2(float x0, float x1, const GroupScale& g, float& t0,
-                                          float& t1) {
-  if (g.small) {
-    t0 = __fdiv_rn(x0, g.s);
-    t1 = __fdiv_rn(x1, g.s);
-    return;
-  }
-  float q0, q1;
-  mul2(q0, q1, x0, x1, g.rs, g.rs);      // q = x * r
-  float e0 = x0, e1 = x1;
-  fma2(e0, e1, q0, q1, g.ns, g.ns);      // e = fma(q, -s, x), exact
-  fma2(q0, q1, e0, e1, g.rs, g.rs);      // q = fma(e, r, q)
-  t0 = copy_sign(q0, x0);
-  t1 = copy_sign(q1, x1);
-}
-
-// Eight codes of BF16-valued x (packed little-endian into two words).
+// Eight codes of BF16-valued x (packed little-endian into two words). Groups with a
+// tiny scale divide; the branch is per warp and only taken when a lane needs it.
 __device__ __forceinline__ uint2 codes8(const float (&v)[8], const GroupScale& g) {
   float t[8];
+  if (__any_sync(kFull, g.small)) {
 #pragma unroll
-  for (int i = 0; i < 8; i += 2) quotient2(v[i], v[i + 1], g, t[i], t[i + 1]);
+    for (int i = 0; i < 8; ++i) t[i] = g.small ? __fdiv_rn(v[i], g.s) : quot(v[i], g);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = quot(v[i], g);
+  }
   return make_uint2(cvt_e4m3x4(t[0], t[1], t[2], t[3]), cvt_e4m3x4(t[4], t[5], t[6], t[7]));
+}
+
+// Lane-wise max of the magnitudes of two packed BF16 pairs (finite inputs).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  return r;
+}
+
+// Largest magnitude of eight values (balanced tree).
+__device__ __forceinline__ float absmax8(const float (&v)[8]) {
+  const float a = fmaxf(fabsf(v[0]), fabsf(v[1])), b = fmaxf(fabsf(v[2]), fabsf(v[3]));
+  const float c = fmaxf(fabsf(v[4]), fabsf(v[5])), d = fmaxf(fabsf(v[6]), fabsf(v[7]));
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
 // One 1x128 group of BF16 values held by a half-warp: 16 lanes x 8 values. Returns the
 // group scale; writes the 8 codes of this lane. All 32 lanes must call it.
 __device__ __forceinline__ float quant_half_warp(const float (&v)[8], uint2& codes) {
-  float a = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  float a = absmax8(v);
 #pragma unroll
   for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
   const GroupScale g = group_scale_bf16(a);
@@ -352,6 +361,30 @@ __device__ __forceinline__ float rstd_from_ss(double ss, int64_t H, float eps) {
   return __double2float_rn(rr);
 }
 
+// Sum of squares of this thread's chunks c = first + stride*j (c < nch) in fp64. Each
+// square of a BF16 value is exact in fp64; eight partial sums (one per position in the
+// chunk) keep the dependent chains short. The order differs from a sequential sum only
+// in the last bits of the fp64 result.
+template <int kChunks>
+__device__ __forceinline__ double sum_squares(const uint4 (&raw)[kChunks], int64_t first,
+                                              int64_t stride, int64_t nch) {
+  double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+  for (int j = 0; j < kChunks; ++j) {
+    if (first + stride * j < nch) {
+      float v[8];
+      unpack_bf16x8(raw[j], v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const double d = static_cast<double>(v[i]);
+        acc[i] = __fma_rn(d, d, acc[i]);
+      }
+    }
+  }
+  return __dadd_rn(__dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3])),
+                   __dadd_rn(__dadd_rn(acc[4], acc[5]), __dadd_rn(acc[6], acc[7])));
+}
+
 // y = bf16(fl32(fl32(x r) g)) for one chunk, then the half-warp group quantization.
 __device__ __forceinline__ void norm_quant_chunk(const uint4& xr, const uint16_t* gamma, int64_t c,
                                                  bool act, float r, uint8_t* qrow, float* s,
@@ -394,25 +427,12 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(
   for (int64_t m = wglobal; m < M; m += nw) {
     const uint16_t* row = x + m * ldx;
     uint4 raw[kChunks];
-    double ss = 0.0;
 #pragma unroll
     for (int j = 0; j < kChunks; ++j) {
       const int64_t c = lane + 32 * j;
       if (c < nch) raw[j] = ld_nc_v4(row + c * 8);
     }
-#pragma unroll
-    for (int j = 0; j < kChunks; ++j) {
-      const int64_t c = lane + 32 * j;
-      if (c < nch) {
-        float v[8];
-        unpack_bf16x8(raw[j], v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const double d = static_cast<double>(v[i]);
-          ss = __fma_rn(d, d, ss);  // the square is exact, so this is the fp64 sum
-        }
-      }
-    }
+    double ss = sum_squares<kChunks>(raw, lane, 32, nch);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, off));
     const float r = rstd_from_ss(ss, H, eps);
@@ -439,25 +459,12 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_cta_kernel(
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint16_t* row = x + m * ldx;
     uint4 raw[kNormMaxChunks];
-    double ss = 0.0;
 #pragma unroll
     for (int j = 0; j < kNormMaxChunks; ++j) {
       const int64_t c = tid + j * kNormThreads;
       if (c < nch) raw[j] = ld_nc_v4(row + c * 8);
     }
-#pragma unroll
-    for (int j = 0; j < kNormMaxChunks; ++j) {
-      const int64_t c = tid + j * kNormThreads;
-      if (c < nch) {
-        float v[8];
-        unpack_bf16x8(raw[j], v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const double d = static_cast<double>(v[i]);
-          ss = __fma_rn(d, d, ss);
-        }
-      }
-    }
+    double ss = sum_squares<kNormMaxChunks>(raw, tid, kNormThreads, nch);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, off));
     if (lane == 0) red[wid] = ss;
@@ -512,6 +519,30 @@ __device__ __forceinline__ bool tile_acquire(const TileSmem& sm, int b, uint32_t
   return true;
 }
 
+// Codes of a column pair's 32 values (lo / hi halves of w[]), four per word.
+template <bool kMaybeSmall>
+__device__ __forceinline__ void col_codes(const uint32_t (&w)[32], const GroupScale& g0,
+                                          const GroupScale& g1, uint32_t (&o0)[8],
+                                          uint32_t (&o1)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float t0[4], t1[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float x0 = bf16_lo(w[4 * k + i]), x1 = bf16_hi(w[4 * k + i]);
+      if (kMaybeSmall) {
+        t0[i] = g0.small ? __fdiv_rn(x0, g0.s) : quot(x0, g0);
+        t1[i] = g1.small ? __fdiv_rn(x1, g1.s) : quot(x1, g1);
+      } else {
+        t0[i] = quot(x0, g0);
+        t1[i] = quot(x1, g1);
+      }
+    }
+    o0[k] = cvt_e4m3x4(t0[0], t0[1], t0[2], t0[3]);
+    o1[k] = cvt_e4m3x4(t1[0], t1[1], t1[2], t1[3]);
+  }
+}
+
 // Column pass over a staged BF16 tile Ts[128][128] (dense rows). Column scales:
 // computed per column (per_col) or the given block scale. Codes go to
 // dst[c * ldd + r] for tile column c and tile row r; per-column scales to scol[c].
@@ -525,33 +556,26 @@ __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, b
   for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(Ts + (32 * rq + r) * 128 + 2 * cp);
   GroupScale g0 = blk, g1 = blk;
   if (per_col) {
-    float a0 = 0.0f, a1 = 0.0f;
+    // column maxima of the 32 rows on packed pairs (four interleaved chains)
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      a0 = fmaxf(a0, fabsf(bf16_lo(w[r])));
-      a1 = fmaxf(a1, fabsf(bf16_hi(w[r])));
-    }
-    red[rq * 128 + 2 * cp] = a0;
-    red[rq * 128 + 2 * cp + 1] = a1;
+    for (int r = 0; r < 32; ++r) m[r & 3] = bf16x2_absmax(m[r & 3], w[r]);
+    const uint32_t mm = bf16x2_absmax(bf16x2_absmax(m[0], m[1]), bf16x2_absmax(m[2], m[3]));
+    red[rq * 128 + 2 * cp] = bf16_lo(mm);
+    red[rq * 128 + 2 * cp + 1] = bf16_hi(mm);
     __syncthreads();
-    a0 = fmaxf(fmaxf(red[2 * cp], red[128 + 2 * cp]), fmaxf(red[256 + 2 * cp], red[384 + 2 * cp]));
-    a1 = fmaxf(fmaxf(red[2 * cp + 1], red[128 + 2 * cp + 1]),
-               fmaxf(red[256 + 2 * cp + 1], red[384 + 2 * cp + 1]));
-    g0 = group_scale_bf16(a0);
-    g1 = group_scale_bf16(a1);
+    const float c0 = fmaxf(fmaxf(red[2 * cp], red[128 + 2 * cp]), fmaxf(red[256 + 2 * cp], red[384 + 2 * cp]));
+    const float c1 = fmaxf(fmaxf(red[2 * cp + 1], red[128 + 2 * cp + 1]),
+                           fmaxf(red[256 + 2 * cp + 1], red[384 + 2 * cp + 1]));
+    g0 = group_scale_bf16(c0);
+    g1 = group_scale_bf16(c1);
     if (rq == 0 && scol) *reinterpret_cast<float2*>(scol + 2 * cp) = make_float2(g0.s, g1.s);
   }
   uint32_t o0[8], o1[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    float t0[4], t1[4];
-    quotient2(bf16_lo(w[4 * k]), bf16_lo(w[4 * k + 1]), g0, t0[0], t0[1]);
-    quotient2(bf16_lo(w[4 * k + 2]), bf16_lo(w[4 * k + 3]), g0, t0[2], t0[3]);
-    quotient2(bf16_hi(w[4 * k]), bf16_hi(w[4 * k + 1]), g1, t1[0], t1[1]);
-    quotient2(bf16_hi(w[4 * k + 2]), bf16_hi(w[4 * k + 3]), g1, t1[2], t1[3]);
-    o0[k] = cvt_e4m3x4(t0[0], t0[1], t0[2], t0[3]);
-    o1[k] = cvt_e4m3x4(t1[0], t1[1], t1[2], t1[3]);
-  }
+  if (__any_sync(kFull, g0.small || g1.small))
+    col_codes<true>(w, g0, g1, o0, o1);
+  else
+    col_codes<false>(w, g0, g1, o0, o1);
   uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * ldd + 32 * rq);
   uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * ldd + 32 * rq);
   d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
@@ -653,8 +677,7 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(
       raw[j] = *reinterpret_cast<const uint4*>(Ts + (rr + 16 * j) * 128 + c8);
       float v[8];
       unpack_bf16x8(raw[j], v);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(v[k]));
+      a = fmaxf(a, absmax8(v));
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
@@ -766,12 +789,14 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
       x0[r] = __fmul_rn(sr, d.x);
       x1[r] = __fmul_rn(sr, d.y);
     }
-    float a0 = 0.0f, a1 = 0.0f;
+    float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
-      a0 = fmaxf(a0, fabsf(x0[r]));
-      a1 = fmaxf(a1, fabsf(x1[r]));
+      c0[r & 3] = fmaxf(c0[r & 3], fabsf(x0[r]));
+      c1[r & 3] = fmaxf(c1[r & 3], fabsf(x1[r]));
     }
+    float a0 = fmaxf(fmaxf(c0[0], c0[1]), fmaxf(c0[2], c0[3]));
+    float a1 = fmaxf(fmaxf(c1[0], c1[1]), fmaxf(c1[2], c1[3]));
     sm.red[rq * 128 + 2 * cp] = a0;
     sm.red[rq * 128 + 2 * cp + 1] = a1;
     __syncthreads();

@@ -1,6 +1,7 @@
 """The quantizer kernels form x/s for BF16-valued x from the correctly rounded
 reciprocal r = 1/s with one residual correction: q = x*r; e = fma(-q, s, x);
-q = fma(e, r, q); sign of x. This test proves, by exhaustive enumeration on the CPU,
+q = fma(e, r, q); sign of x (computed as q = fma(fma(q, s, -x), -r, q), which keeps the
+sign of -0 by itself; the test checks the two forms agree bit for bit). This test proves, by exhaustive enumeration on the CPU,
 that the E4M3 code of that quotient equals the code of the IEEE quotient x/s for every
 BF16 amax (with s = fl32(amax/448) >= 2^-80; the kernels divide below that) and every
 BF16 x with |x| <= amax. It checks the kernels' arithmetic identity only: it uses its
@@ -48,6 +49,11 @@ int main(void) {
       float q = x * r;
       float e = fmaf(-q, s, x);
       float q2 = copysignf(fmaf(e, r, q), x);
+      /* the kernels' sign-preserving form: q*s - x and q - (q*s - x)*r keep the sign of
+         x = -0 without a copy-sign; it must equal q2 bit for bit */
+      float en = fmaf(q, s, -x);
+      float q3 = fmaf(en, -r, q);
+      if (u_of(q3) != u_of(q2)) bad++;
       total++;
       if (u_of(q2) != u_of(t)) {
         if (fabsf(t) >= 0x1p-11f || fabsf(q2) >= 0x1p-11f) {
@@ -75,3 +81,4 @@ def test_reciprocal_quotient_gives_ieee_codes_exhaustively():
         total, bad = map(int, out.stdout.split())
         assert total > 10 ** 9
         assert bad == 0 and out.returncode == 0
+
