@@ -36,6 +36,16 @@ import workloads  # noqa: E402
 
 METRIC = "FP8 linear fwd+dgrad+wgrad TFLOP/s and % of FP8 peak; quantizer HBM GB/s"
 WORKLOAD = workloads.LLAMA_LAYER
+# Other layer shapes of the pages, selectable with --workload (secondary measurements;
+# the decode shapes run the serving forward pass only, weights quantized once up front).
+WORKLOADS = {w.name: w for w in [workloads.LLAMA_LAYER, workloads.QWEN25_LONG,
+                                 workloads.DENSE32_TRAIN, workloads.DENSE32_DECODE]
+             + list(workloads.QWEN3_DECODE)}
+
+
+def is_decode(wl) -> bool:
+    """Decode-sized token batches run the forward pass only."""
+    return wl.tokens < 1024
 
 # Algorithmic bytes per element of each quantizer (reads + writes, scales included).
 BYTES_PER_ELEM = {
@@ -89,14 +99,15 @@ def whole_job_tflops(flops_per_rank: float, world: int, max_ms_per_step: float) 
 class LayerStep:
     """Device buffers of one layer pass and the launch sequence (all through the C ABI)."""
 
-    def __init__(self, fq, wl, device, seed_offset=0):
+    def __init__(self, fq, wl, device, seed_offset=0, forward_only=False):
         self.fq = fq
         L = wl.layer
         self.M = M = wl.tokens
         self.L = L
         self.eps = wl.eps
+        self.forward_only = forward_only
         wl_seeded = workloads.Workload(**{**wl.__dict__, "seed": wl.seed + seed_offset})
-        self.inp = inp = workloads.layer_inputs(wl_seeded, device)
+        self.inp = inp = workloads.layer_inputs(wl_seeded, device, with_grads=not forward_only)
         lds = fq.lds_for(M)
         H, I = L.hidden, L.intermediate
         e = lambda *s, dt=torch.uint8: torch.empty(s, dtype=dt, device=device)  # noqa: E731
@@ -105,30 +116,37 @@ class LayerStep:
         self.lin = {}
         for lin in L.linears:
             N, K = lin.n, lin.k
-            self.lin[lin.name] = dict(
-                N=N, K=K,
-                qw=e(N, K), sw=e(N // 128, K // 128, dt=f32), qwT=e(K, N),
-                y=e(M, N, dt=bf), dx=e(M, K, dt=bf), dw=e(N, K, dt=bf),
-                q_in=e(M, K), s_in=e(K // 128, lds, dt=f32),
-                q_inT=e(K, M), s_inT=e(M // 128, K, dt=f32),
-                q_dy=e(M, N), s_dy=e(N // 128, lds, dt=f32),
-                q_dyT=e(N, M), s_dyc=e(M // 128, N, dt=f32),
-            )
-        self.flops = workloads.layer_gemm_flops(L, M)
-        self.kernel_names = []
+            d = dict(N=N, K=K, qw=e(N, K), sw=e(N // 128, K // 128, dt=f32),
+                     y=e(M, N, dt=bf), q_in=e(M, K), s_in=e(K // 128, lds, dt=f32))
+            if not forward_only:
+                d.update(qwT=e(K, N), dx=e(M, K, dt=bf), dw=e(N, K, dt=bf),
+                         q_inT=e(K, M), s_inT=e(M // 128, K, dt=f32),
+                         q_dy=e(M, N), s_dy=e(N // 128, lds, dt=f32),
+                         q_dyT=e(N, M), s_dyc=e(M // 128, N, dt=f32))
+            self.lin[lin.name] = d
+        self.flops = workloads.layer_gemm_flops(L, M, passes=1 if forward_only else 3)
+        if forward_only:
+            # serving: the weights are quantized once (at weight sync), not per step
+            for name, d in self.lin.items():
+                fq.quant_weight_128x128(inp["w"][name], d["qw"], d["sw"], None)
 
     def _k(self, name, fn, timer):
+        if self.only is not None and name not in self.only:
+            return
         if timer is not None:
             timer.start(name)
         fn()
         if timer is not None:
             timer.stop(name)
 
-    def run(self, timer=None, stream=None):
+    only = None  # when set: launch only the kernels of these kinds (per-kind graphs)
+
+    def run(self, timer=None, stream=None, only=None):
         fq, inp, lin, M = self.fq, self.inp, self.lin, self.M
+        self.only = only
         k = self._k
         # weights: 128x128 quantization of the BF16 masters, with the transposed codes
-        for name, d in lin.items():
+        for name, d in (() if self.forward_only else lin.items()):
             k("quant_weight_128x128",
               lambda d=d, name=name: fq.quant_weight_128x128(inp["w"][name], d["qw"], d["sw"],
                                                              d["qwT"], stream), timer)
@@ -150,7 +168,7 @@ class LayerStep:
         k("gemm_fwd", lambda: fq.linear_fwd(dn["q_in"], dn["s_in"], dn["qw"], dn["sw"], dn["y"],
                                             stream), timer)
         # backward of each linear (BF16 upstream gradients)
-        for name in ("down", "gate_up", "o", "qkv"):
+        for name in (() if self.forward_only else ("down", "gate_up", "o", "qkv")):
             d = lin[name]
             k("transpose_quant_bf16",
               lambda d=d, name=name: fq.transpose_quant_bf16(inp["dy"][name], d["q_dy"], d["s_dy"],
@@ -163,12 +181,23 @@ class LayerStep:
             k("gemm_wgrad", lambda d=d: fq.linear_wgrad(d["q_dyT"], d["s_dyc"], d["q_inT"],
                                                         d["s_inT"], d["dw"], stream), timer)
 
-    launches_per_step = 28
+    @property
+    def launches_per_step(self):
+        return 8 if self.forward_only else 28
 
     def gemm_flops_by_kind(self):
         M = self.M
         tot = sum(2.0 * M * d["N"] * d["K"] for d in self.lin.values())
+        if self.forward_only:
+            return {"gemm_fwd": tot}
         return {"gemm_fwd": tot, "gemm_dgrad": tot, "gemm_wgrad": tot}
+
+    def fwd_gemm_bytes(self):
+        """Algorithmic HBM bytes of the forward GEMMs of one step: FP8 weight codes and
+        128x128 scales, FP8 activation codes and 1x128 scales, BF16 outputs."""
+        M = self.M
+        return sum(d["N"] * d["K"] * (1 + 4 / 16384) + M * d["K"] * (1 + 4 / 128) +
+                   2 * M * d["N"] for d in self.lin.values())
 
     def quant_bytes_by_kind(self):
         M = self.M
@@ -178,42 +207,98 @@ class LayerStep:
         w_elems = sum(d["N"] * d["K"] for d in self.lin.values())
         dy_elems = sum(M * d["N"] for d in self.lin.values())
         in_elems = sum(M * d["K"] for d in self.lin.values())
-        e = {
+        e = {} if self.forward_only else {
             "quant_weight_128x128": w_elems,
-            "rmsnorm_quant": 2 * M * H,
-            "quant_act_1x128": M * qo,
-            "swiglu_quant": M * I,
             "transpose_quant_bf16": dy_elems,
             "transpose_quant_fp8": in_elems,
         }
+        e.update({
+            "rmsnorm_quant": 2 * M * H,
+            "quant_act_1x128": M * qo,
+            "swiglu_quant": M * I,
+        })
         return {k: v * BYTES_PER_ELEM[k] for k, v in e.items()}
 
     # end-to-end: the per-step batch comes from pinned host memory, the results go back
-    def e2e_buffers(self):
-        inp = self.inp
-        names = ["x_attn", "x_mlp", "attn_out"]
-        host_in = {n: torch.empty_like(inp[n], device="cpu").pin_memory() for n in names}
-        for n in names:
-            host_in[n].copy_(inp[n])
-        host_dy = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in inp["dy"].items()}
-        for n, t in inp["dy"].items():
-            host_dy[n].copy_(t)
-        outs = [self.lin["down"]["y"], self.lin["qkv"]["dx"]]
-        host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + \
-            sum(t.numel() * t.element_size() for t in host_dy.values())
-        d2h = sum(t.numel() * t.element_size() for t in host_out)
-        return host_in, host_dy, outs, host_out, h2d, d2h
+    def e2e_pipeline(self):
+        return E2EPipeline(self)
 
-    def run_e2e(self, bufs, stream=None):
-        host_in, host_dy, outs, host_out, _, _ = bufs
-        for n, h in host_in.items():
-            self.inp[n].copy_(h, non_blocking=True)
-        for n, h in host_dy.items():
-            self.inp["dy"][n].copy_(h, non_blocking=True)
-        self.run(stream=stream)
-        for h, t in zip(host_out, outs):
-            h.copy_(t, non_blocking=True)
+
+class E2EPipeline:
+    """Each step uploads its inputs (activations and, for training, the upstream BF16
+    gradients) from pinned host memory and reads its results back (the down projection's
+    output and, for training, the QKV input gradient). Two device sets of inputs and of
+    results let step i+1's upload and step i-1's read-back run on their own streams
+    while step i computes."""
+
+    def __init__(self, step):
+        self.step = step
+        inp = step.inp
+        names = ["x_attn", "x_mlp", "attn_out"]
+        self.keys = [(n, None) for n in names] + [("dy", n) for n in inp["dy"]]
+        get = lambda d, k: d[k[0]] if k[1] is None else d[k[0]][k[1]]  # noqa: E731
+        self.get = get
+        self.host = {}
+        for k in self.keys:
+            t = get(inp, k)
+            self.host[k] = torch.empty(t.shape, dtype=t.dtype, device="cpu").pin_memory()
+            self.host[k].copy_(t)
+        self.dev = [{k: get(inp, k) for k in self.keys},
+                    {k: torch.empty_like(get(inp, k)) for k in self.keys}]
+        self.out_slots = [("down", "y")] + ([] if step.forward_only else [("qkv", "dx")])
+        self.outs = [[step.lin[a][b] for a, b in self.out_slots],
+                     [torch.empty_like(step.lin[a][b]) for a, b in self.out_slots]]
+        self.host_out = [[torch.empty(t.shape, dtype=t.dtype, device="cpu").pin_memory()
+                          for t in self.outs[0]] for _ in range(2)]
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host.values())
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.outs[0])
+        self.up = torch.cuda.Stream()
+        self.down = torch.cuda.Stream()
+        ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]  # noqa: E731
+        self.ev_in, self.ev_done, self.ev_out = ev(), ev(), ev()
+        self.i = 0
+
+    def _use(self, s):
+        st = self.step
+        for k in self.keys:
+            if k[1] is None:
+                st.inp[k[0]] = self.dev[s][k]
+            else:
+                st.inp[k[0]][k[1]] = self.dev[s][k]
+        for (a, b), t in zip(self.out_slots, self.outs[s]):
+            st.lin[a][b] = t
+
+    def run(self):
+        s = self.i & 1
+        cur = torch.cuda.current_stream()
+        first_use = self.i < 2
+        with torch.cuda.stream(self.up):
+            if not first_use:
+                self.up.wait_event(self.ev_done[s])  # set s's inputs were consumed
+            for k in self.keys:
+                self.dev[s][k].copy_(self.host[k], non_blocking=True)
+            self.ev_in[s].record(self.up)
+        cur.wait_event(self.ev_in[s])
+        if not first_use:
+            cur.wait_event(self.ev_out[s])  # set s's results were read back
+        self._use(s)
+        self.step.run()
+        self.ev_done[s].record(cur)
+        with torch.cuda.stream(self.down):
+            self.down.wait_event(self.ev_done[s])
+            for h, t in zip(self.host_out[s], self.outs[s]):
+                h.copy_(t, non_blocking=True)
+            self.ev_out[s].record(self.down)
+        self.i += 1
+
+    def finish(self):
+        """Make the current stream wait for the last uploads and read-backs."""
+        cur = torch.cuda.current_stream()
+        for s in range(2):
+            cur.wait_event(self.ev_out[s])
+
+    def restore(self):
+        self._use(0)
 
 
 class KernelTimer:
@@ -242,6 +327,59 @@ class KernelTimer:
             t[0] += ms
             t[1] += 1
         return out
+
+
+def capture_graphs(step, reps_per_kind=10):
+    """CUDA graphs of one step and, per kernel kind, of `reps_per_kind` steps' launches of
+    that kind only (for device-side per-kernel times without host launch gaps)."""
+    graphs = {}
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # one eager pass on the capture stream first
+        step.run()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step.run()
+    graphs["step"] = g
+    counter = KernelTimer()
+    step.run(counter)
+    torch.cuda.synchronize()
+    per_step = {name: n for name, (_, n) in counter.totals().items()}
+    graphs["kinds"] = {}
+    for name, n in per_step.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps_per_kind):
+                step.run(only={name})
+        step.only = None
+        graphs["kinds"][name] = (g, n, reps_per_kind)
+    torch.cuda.synchronize()
+    return graphs
+
+
+class GraphKindTimer:
+    """Per-kind device time from replays of the per-kind graphs, scaled to `steps` steps
+    (same interface as KernelTimer.totals)."""
+
+    def __init__(self, graphs, steps, replays=5):
+        self.out = {}
+        for name, (g, n_step, reps) in graphs["kinds"].items():
+            g.replay()
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(replays):
+                g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            per_launch = a.elapsed_time(b) / (replays * reps * n_step)
+            self.out[name] = [per_launch * n_step * steps, n_step * steps]
+
+    def totals(self):
+        return self.out
 
 
 class ClockSampler:
@@ -356,15 +494,15 @@ def oracle_host_inputs(wl):
     return {"bits": bits}
 
 
-def oracle_timing(min_seconds=10.0, max_steps=1000):
+def oracle_timing(wl=WORKLOAD, min_seconds=10.0, max_steps=1000):
     import oracle as orc
     orc.build()
-    host = oracle_host_inputs(WORKLOAD)
-    oracle_sample_step(orc, host, WORKLOAD)  # warm
+    host = oracle_host_inputs(wl)
+    oracle_sample_step(orc, host, wl)  # warm
     t0 = time.perf_counter()
     flops, steps = 0.0, 0
     while steps < max_steps:
-        flops += oracle_sample_step(orc, host, WORKLOAD)
+        flops += oracle_sample_step(orc, host, wl)
         steps += 1
         if time.perf_counter() - t0 >= min_seconds:
             break
@@ -373,7 +511,7 @@ def oracle_timing(min_seconds=10.0, max_steps=1000):
             "kind": "oracle",
             "sample": "%d repetitions of one 128-token block of the %s layer: every quantizer "
                       "on the rows it needs, a 128x128 output tile of each linear's forward, "
-                      "DGrad and WGrad (fp64 dot products); %.1f s" % (steps, WORKLOAD.name, dt)}
+                      "DGrad and WGrad (fp64 dot products); %.1f s" % (steps, wl.name, dt)}
 
 
 def run_reference(args, rank, world):
@@ -487,7 +625,10 @@ def main():
     ap.add_argument("--case", choices=CASES, default=None,
                     help="run one kernel of the layer on its real shape (for profilers)")
     ap.add_argument("--case-reps", type=int, default=3)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=WORKLOAD.name,
+                    help="layer shape (default: the Llama-3.1-8B layer at M = 8192)")
     args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
     if args.case:
         return run_case(args.case, args.case_reps)
     if args.warmup < 3:
@@ -511,7 +652,7 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    step = LayerStep(fq, WORKLOAD, dev, seed_offset=rank_seed_offset(rank))
+    step = LayerStep(fq, wl, dev, seed_offset=rank_seed_offset(rank), forward_only=is_decode(wl))
     torch.cuda.synchronize()
     for _ in range(args.warmup):
         step.run()
@@ -519,9 +660,14 @@ def main():
     if fq.device_error() != fq.FP8Q_OK:
         raise RuntimeError("a kernel reported a device error during warm-up")
 
-    # ---- timed region: K steps, per-kernel events on the launching stream
+    # ---- timed region: K steps, per-kernel events on the launching stream. Decode-sized
+    # steps launch kernels faster than the host can issue them one by one, so they are
+    # captured once into a CUDA graph (the same launches) and the graph is replayed.
     timer = KernelTimer()
     sampler = ClockSampler(local_rank)
+    graphs = None
+    if step.forward_only:
+        graphs = capture_graphs(step)
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
@@ -530,12 +676,17 @@ def main():
         end = torch.cuda.Event(enable_timing=True)
         start.record()
         for _ in range(args.steps):
-            step.run(timer)
+            if graphs:
+                graphs["step"].replay()
+            else:
+                step.run(timer)
         end.record()
         torch.cuda.synchronize()
     if pg:
         pg.barrier()
     elapsed_ms = start.elapsed_time(end)
+    if graphs:
+        timer = GraphKindTimer(graphs, args.steps)
     if fq.device_error() != fq.FP8Q_OK:
         raise RuntimeError("a kernel reported a device error in the timed region")
     max_ms = max_over_ranks(elapsed_ms, pg, dev)
@@ -546,19 +697,37 @@ def main():
     peaks = read_peaks()
     fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]  # fp8 dense = 2x bf16 (nominal ratio)
     kt = timer.totals()
+    roofline = None
     gflops = step.gemm_flops_by_kind()
     gemm_ms = sum(kt[k][0] for k in gflops)
     gemm_launches = sum(kt[k][1] for k in gflops)
     gemm_flops = sum(gflops.values()) * args.steps
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    if step.forward_only:
+        # below the ridge: the forward GEMMs are bound by reading the FP8 weights
+        gemm_gbs = step.fwd_gemm_bytes() * args.steps / (gemm_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": None,
+                    "kernel": "gemm_fwd (decode, weight-bytes bound)",
+                    "launches": gemm_launches // args.steps,
+                    "bytes_per_step": step.fwd_gemm_bytes(),
+                    "peak_source": "%s HBM copy bandwidth" % peaks["source"]}
     traffic = None
     prof = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if os.path.exists(prof):
         with open(prof) as f:
             traffic = json.load(f).get("bytes_per_launch")
+    if roofline is None:
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak,
+                    "unit": "TFLOP/s", "frac": achieved / fp8_peak, "traffic": traffic,
+                    "kernel": "gemm (fwd+dgrad+wgrad launches)",
+                    "launches": gemm_launches // args.steps,
+                    "peak_source": "%s bf16 sustained x2 (fp8/bf16 nominal ratio)" % peaks["source"]}
     kernels = {}
     for kname, fl in gflops.items():
         ms, n = kt[kname]
+        if n == 0:
+            continue
         kernels[kname] = {"ms_per_step": ms / args.steps, "launches_per_step": n // args.steps,
                           "tflops": fl * args.steps / (ms * 1e-3) / 1e12,
                           "frac_of_fp8_peak": fl * args.steps / (ms * 1e-3) / 1e12 / fp8_peak}
@@ -569,10 +738,12 @@ def main():
         kernels[kname] = {"ms_per_step": ms / args.steps, "launches_per_step": n // args.steps,
                           "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
 
-    # ---- end to end through the C ABI with host buffers
-    bufs = step.e2e_buffers()
+    # ---- end to end through the C ABI with host buffers (uploads and read-backs inside
+    # the timed region, overlapped with compute on their own streams)
+    pipe = step.e2e_pipeline()
     for _ in range(2):
-        step.run_e2e(bufs)
+        pipe.run()
+    pipe.finish()
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
@@ -580,15 +751,17 @@ def main():
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.e2e_steps):
-        step.run_e2e(bufs)
+        pipe.run()
+    pipe.finish()
     e1.record()
     torch.cuda.synchronize()
+    pipe.restore()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev) / args.e2e_steps
     e2e_value = whole_job_tflops(step.flops, world, e2e_ms)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_timing()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not step.forward_only:
+        cpu = oracle_timing(wl)
 
     if rank == 0:
         line = {
@@ -596,24 +769,22 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8_e4m3", "data": "synthetic",
-            "config": {"workload": WORKLOAD.name, "tokens_per_gpu": WORKLOAD.tokens,
-                       "hidden": WORKLOAD.layer.hidden,
-                       "intermediate": WORKLOAD.layer.intermediate,
+            "config": {"workload": wl.name, "tokens_per_gpu": wl.tokens,
+                       "hidden": wl.layer.hidden,
+                       "intermediate": wl.layer.intermediate,
+                       "pass": "forward (serving)" if step.forward_only else "forward+backward",
                        "gemm_tflop_per_step_per_gpu": step.flops / 1e12,
-                       "launches_per_step": LayerStep.launches_per_step,
+                       "launches_per_step": step.launches_per_step,
                        "l2": "inputs larger than L2: %.1f GB touched per step" % (
                            sum(qb.values()) / 1e9),
                        "parallelism": "replicas" if world > 1 else "single"},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak,
-                         "unit": "TFLOP/s", "frac": achieved / fp8_peak, "traffic": traffic,
-                         "kernel": "gemm (fwd+dgrad+wgrad launches)",
-                         "launches": gemm_launches // args.steps,
-                         "peak_source": "%s bf16 sustained x2 (fp8/bf16 nominal ratio)" % peaks["source"]},
+            "roofline": roofline,
             "kernels": kernels,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": bufs[4],
-                    "d2h_bytes_per_step": bufs[5], "ms_per_step": e2e_ms},
-            "gpu_launches": LayerStep.launches_per_step * args.steps,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": pipe.h2d_bytes,
+                    "d2h_bytes_per_step": pipe.d2h_bytes, "ms_per_step": e2e_ms,
+                    "overlap": "uploads and read-backs on their own streams, double-buffered"},
+            "gpu_launches": step.launches_per_step * args.steps,
             "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -121,7 +121,9 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled tensor loads, no multicast)
+// TMA (tiled tensor loads, no multicast). The shared-memory destination (or source of
+// a store) must start on a 128-byte boundary (1024 with the 128-byte swizzle), and the
+// innermost coordinate times the element size must be a multiple of 16 bytes.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
                                             int32_t y, uint64_t* bar) {
@@ -129,6 +131,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int32_t x,
+                                            int32_t y, int32_t z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -273,6 +284,24 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uin
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// One 128-wide K slice as four K = 32 steps into a fresh accumulator, in one block: the
+// descriptors of steps 1..3 are the step-0 descriptors advanced by 32 bytes (2 in the
+// 16-byte start-address field), and the accumulate predicates are set once.
+__device__ __forceinline__ void mma_f8f6f4_slice(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred fresh, acc;\n\t"
+      "setp.ne.b32 fresh, 0, 0;\n\t"
+      "setp.eq.b32 acc, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, fresh;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %5, %3, acc;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %6, %7, %3, acc;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %8, %9, %3, acc;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "l"(a_desc + 2), "l"(b_desc + 2), "l"(a_desc + 4),
+      "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
       : "memory");
 }
 

@@ -19,12 +19,23 @@
 //    whatever the shared-memory tile holds and their accumulator lanes are never read),
 //    N = kBN, K = 32, four per 128-wide slice, into one of up to 8 TMEM accumulator
 //    buffers, so the tensor core runs ahead of the promotion by several slices.
-//  * A TMA ring of up to 16 stages (token rows of A, weight strip of B), sized to about
-//    96 KB of shared memory so that two CTAs fit on an SM.
-//  * 192 threads: warp 0 TMA producer, warp 1 TMEM allocation + MMA issue, warps 2-5
-//    promotion (warp w reads TMEM lanes 32*(w%4) .. +31; only the quarters that hold
-//    token rows work). Promotion adds each slice into kBN fp32 registers per thread;
-//    the epilogue rounds to BF16 and stores each token row's kBN outputs directly.
+//  * A TMA ring of "super-stages" of G consecutive K-slices, about 96 KB of shared
+//    memory so that two CTAs fit on an SM. One 3D tensor copy per operand brings G
+//    slices at once (dimensions: 128 bytes of a slice, rows, slice index; the slice
+//    stride is 128 bytes), so each row of the strip is read as one G*128-byte run: with
+//    one 128-byte piece per row and slice, the weight stream is scattered over DRAM
+//    pages and ran below a third of the HBM bandwidth. The row scales of a super-stage
+//    arrive by TMA in a ring of their own (released by the promotion warps, since they
+//    outlive the stage), and the strip's KB block scales are read into shared memory
+//    once, so the promotion loop never waits on a global load.
+//  * 224 threads: warp 0 TMA producer; warps 1 and 2 issue the MMAs, alternating
+//    slices (warp 1 also allocates TMEM); warps 3-6 promotion (warp w reads TMEM lanes
+//    32*(w%4) .. +31; only the quarters that hold token rows work). One issuing thread
+//    needs ~70 cycles per MMA instruction and ~700 per slice in all (measured), which
+//    with narrow strips would cap the weight stream at N*128 bytes per 700 cycles; each
+//    slice is an independent 4-MMA group into its own TMEM buffer, so two threads can
+//    issue alternate slices. Promotion adds each slice into kBN fp32 registers per
+//    thread; the epilogue rounds to BF16 and stores each token row's kBN outputs.
 // Every mbarrier wait is bounded; a wait that gives up records FP8Q_ERR_TIMEOUT in the
 // device error word and the CTA winds down.
 #include <algorithm>
@@ -35,21 +46,27 @@
 namespace fp8q {
 namespace {
 
-constexpr int kSkThreads = 192;
+constexpr int kSkIssuers = 2;                      // MMA-issuing warps
+constexpr int kSkThreads = 32 * (1 + kSkIssuers + 4);
 constexpr int kSkBK = 128;
-constexpr int kSkMaxStages = 16;
+constexpr int kSkMaxStages = 8;
+constexpr int kSkMaxG = 8;
 constexpr uint32_t kSkSmemTarget = 96 * 1024;
 constexpr uint32_t kSkATileRead = 128 * kSkBK;  // the MMA reads 128 rows of A
+constexpr int kSkScRing = 8;                     // row-scale slots (one per super-stage)
 
 struct SkinnyParams {
   int32_t M, N, kblocks;
   int32_t mtiles;
-  int32_t stages;
-  uint32_t a_stage, b_stage;  // bytes per stage (1024-aligned)
-  uint32_t a_rows;            // rows per A box
+  int32_t stages;             // super-stages in the ring
+  int32_t G;                  // K-slices per super-stage
+  uint32_t a_slice, b_slice;  // bytes of one slice of A / B (1024-aligned)
+  uint32_t a_rows;            // token rows per A box
+  uint32_t off_b;             // start of the B ring
+  uint32_t off_sa;            // row-scale ring: kSkScRing slots of sa_slot bytes
+  uint32_t sa_slot;           // G * a_rows * 4 rounded up to 128 (TMA destination alignment)
+  uint32_t off_sb;            // block scales of the strip: kblocks fp32
   uint32_t off_bars;
-  const float* sa;
-  int64_t ldsa;
   const float* sb;
   int64_t sb_sj, sb_sr;
   uint16_t* y;
@@ -89,22 +106,26 @@ __device__ __forceinline__ void sk_tmem_load(uint32_t taddr, uint32_t (&r)[kBN])
 template <int kBN>
 __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-    const SkinnyParams p) {
+    const __grid_constant__ CUtensorMap tmSA, const SkinnyParams p) {
   using Shape = SkinnyShape<kBN>;
   constexpr int kBufs = Shape::kBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int S = p.stages;
+  const int S = p.stages, G = p.G, KB = p.kblocks;
+  const uint32_t a_stage = G * p.a_slice, b_stage = G * p.b_slice;
   uint8_t* a_ring = smem;
-  uint8_t* b_ring = smem + S * p.a_stage;
+  uint8_t* b_ring = smem + p.off_b;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bars);
   uint64_t* empty = full + kSkMaxStages;
   uint64_t* tfull = empty + kSkMaxStages;
   uint64_t* tempty = tfull + kBufs;
-  uint64_t* done = tempty + kBufs;
+  uint64_t* sfull = tempty + kBufs;
+  uint64_t* sempty = sfull + kSkScRing;
+  uint64_t* done = sempty + kSkScRing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sb_s = reinterpret_cast<float*>(smem + p.off_sb);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -114,25 +135,36 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
   const int n0 = nt * kBN;
   const int rows = min(128, p.M - m0);       // token rows of this tile
   const int quarters = (rows + 31) >> 5;     // TMEM lane quarters that hold them
+  const int nst = (KB + G - 1) / G;          // super-stages over K
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
+      mbar_init(empty + s, kSkIssuers);  // each issuer commits once per super-stage
     }
     for (int b = 0; b < kBufs; ++b) {
       mbar_init(tfull + b, 1);
       mbar_init(tempty + b, quarters);
     }
-    mbar_init(done, 1);
+    for (int i = 0; i < kSkScRing; ++i) {
+      mbar_init(sfull + i, 1);
+      mbar_init(sempty + i, quarters);
+    }
+    mbar_init(done, kSkIssuers);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmSA);
   }
   if (warp == 1) tmem_alloc<Shape::kTmemCols>(tmem_slot);
+  {  // block scales of this strip, one per slice
+    const float* sbp = p.sb + static_cast<int64_t>(n0 / 128) * p.sb_sj;
+    for (int kb = threadIdx.x; kb < KB; kb += kSkThreads)
+      sb_s[kb] = __ldg(sbp + static_cast<int64_t>(kb) * p.sb_sr);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -142,48 +174,63 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint32_t stage_tx = p.a_rows * kSkBK + kBN * kSkBK;
-      int issued = 0;
+      // slices past K (the last super-stage may be partial) read as zeros, and the
+      // transaction count is the full box either way
+      const uint32_t stage_tx = G * (p.a_rows * kSkBK + kBN * kSkBK);
+      int issued = 0, sc_issued = 0;
       bool ok = true;
-      for (int kb = 0; kb < p.kblocks; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = static_cast<uint32_t>(kb / S) & 1u;
-        if (!mbar_wait(empty + s, ph ^ 1u, ctl)) { ok = false; break; }
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % S;
+        if (!mbar_wait(empty + s, (static_cast<uint32_t>(st / S) & 1u) ^ 1u, ctl)) { ok = false; break; }
         mbar_arrive_expect_tx(full + s, stage_tx);
-        tma_load_2d(a_ring + s * p.a_stage, &tmA, kb * kSkBK, m0, full + s);
-        tma_load_2d(b_ring + s * p.b_stage, &tmB, kb * kSkBK, n0, full + s);
-        issued = kb + 1;
+        tma_load_3d(a_ring + s * a_stage, &tmA, 0, m0, st * G, full + s);
+        tma_load_3d(b_ring + s * b_stage, &tmB, 0, n0, st * G, full + s);
+        issued = st + 1;
+        const int si = st % kSkScRing;
+        if (!mbar_wait(sempty + si, (static_cast<uint32_t>(st / kSkScRing) & 1u) ^ 1u, ctl)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(sfull + si, G * p.a_rows * 4u);
+        tma_load_2d(smem + p.off_sa + si * p.sa_slot, &tmSA, m0, st * G, sfull + si);
+        sc_issued = st + 1;
       }
-      if (!ok)  // let the copies still in flight land before the CTA exits
-        for (int kb = max(0, issued - S); kb < issued; ++kb)
-          sk_wait_drain(full + kb % S, static_cast<uint32_t>(kb / S) & 1u, p.wait_limit_ns);
+      if (!ok) {  // let the copies still in flight land before the CTA exits
+        for (int st = max(0, issued - S); st < issued; ++st)
+          sk_wait_drain(full + st % S, static_cast<uint32_t>(st / S) & 1u, p.wait_limit_ns);
+        for (int st = max(0, sc_issued - kSkScRing); st < sc_issued; ++st)
+          sk_wait_drain(sfull + st % kSkScRing, static_cast<uint32_t>(st / kSkScRing) & 1u,
+                        p.wait_limit_ns);
+      }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp <= kSkIssuers) {
+    // ------------------------------------------------------------ MMA issuers
+    // issuer i = warp - 1 takes the slices kb with kb % kSkIssuers == i
     if (lane == 0) {
+      const int issuer = warp - 1;
       const uint32_t idesc = idesc_e4m3_f32(128, kBN);
       bool ok = true;
-      for (int kb = 0; kb < p.kblocks; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = static_cast<uint32_t>(kb / S) & 1u;
-        const int buf = kb % kBufs;
-        const uint32_t tph = static_cast<uint32_t>(kb / kBufs) & 1u;
-        if (!mbar_wait(full + s, ph, ctl)) { ok = false; break; }
-        if (!mbar_wait(tempty + buf, tph ^ 1u, ctl)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t a0 = smem_u32(a_ring + s * p.a_stage);
-        const uint32_t b0 = smem_u32(b_ring + s * p.b_stage);
-        const uint32_t d = tmem_base + buf * kBN;
-#pragma unroll
-        for (int k = 0; k < kSkBK / 32; ++k)
-          mma_f8f6f4(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc,
-                     k > 0 ? 1u : 0u);
-        mma_commit(empty + s);
-        mma_commit(tfull + buf);
+      for (int st = 0; ok && st < nst; ++st) {
+        const int s = st % S;
+        if (!mbar_wait(full + s, static_cast<uint32_t>(st / S) & 1u, ctl)) { ok = false; break; }
+        for (int j = 0; j < G; ++j) {
+          const int kb = st * G + j;
+          if (kb >= KB) break;
+          if (kb % kSkIssuers != issuer) continue;
+          const int buf = kb % kBufs;
+          const uint32_t tph = static_cast<uint32_t>(kb / kBufs) & 1u;
+          if (!mbar_wait(tempty + buf, tph ^ 1u, ctl)) { ok = false; break; }
+          tc_fence_after();
+          mma_f8f6f4_slice(tmem_base + buf * kBN,
+                           smem_desc_k_sw128(smem_u32(a_ring + s * a_stage + j * p.a_slice)),
+                           smem_desc_k_sw128(smem_u32(b_ring + s * b_stage + j * p.b_slice)), idesc);
+          mma_commit(tfull + buf);
+        }
+        // this issuer's reads of the super-stage are done when its MMAs are
+        if (ok) mma_commit(empty + s);
       }
-      (void)ok;
-      // every MMA issued so far has finished reading shared memory and writing TMEM
+      // every MMA this thread issued has finished reading shared memory and writing TMEM
       mma_commit(done);
       sk_wait_drain(done, 0, p.wait_limit_ns);
     }
@@ -195,18 +242,25 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
       const int row = q * 32 + lane;
       const int m = m0 + row;
       const bool row_ok = m < p.M;
-      const float* sap = p.sa + (row_ok ? m : 0);
-      const float* sbp = p.sb + static_cast<int64_t>(n0 / 128) * p.sb_sj;
+      const int srow = row < static_cast<int>(p.a_rows) ? row : 0;
       float acc[kBN];
 #pragma unroll
       for (int i = 0; i < kBN; ++i) acc[i] = 0.0f;
-      float san = __ldg(sap), sbn = __ldg(sbp);
       bool ok = true;
-      for (int kb = 0; kb < p.kblocks; ++kb) {
-        const float sa = san, sb = sbn;
-        if (kb + 1 < p.kblocks) {  // next slice's scales, one slice ahead
-          san = __ldg(sap + static_cast<int64_t>(kb + 1) * p.ldsa);
-          sbn = __ldg(sbp + static_cast<int64_t>(kb + 1) * p.sb_sr);
+      for (int kb = 0; kb < KB; ++kb) {
+        const int st = kb / G, j = kb - st * G;
+        const int si = st % kSkScRing;
+        if (j == 0 &&
+            !mbar_wait_warp(sfull + si, static_cast<uint32_t>(st / kSkScRing) & 1u, ctl)) {
+          ok = false;
+          break;
+        }
+        const float sa =
+            reinterpret_cast<const float*>(smem + p.off_sa + si * p.sa_slot)[j * p.a_rows + srow];
+        const float s = __fmul_rn(sa, sb_s[kb]);
+        if (j == G - 1 || kb == KB - 1) {  // last use of this super-stage's scales
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sempty + si);
         }
         const int buf = kb % kBufs;
         const uint32_t tph = static_cast<uint32_t>(kb / kBufs) & 1u;
@@ -214,7 +268,6 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
         tc_fence_after();
         uint32_t r[kBN];
         sk_tmem_load<kBN>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN, r);
-        const float s = __fmul_rn(sa, sb);
 #pragma unroll
         for (int i = 0; i < kBN; i += 2)
           fma2(acc[i], acc[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), s, s);
@@ -262,28 +315,55 @@ bool skinny_setup(size_t smem_bytes) {
 }
 
 template <int kBN>
-fp8q_status launch_skinny(const CUtensorMap& tmA, const uint8_t* B, int64_t Ng, int64_t Kg,
-                          SkinnyParams p, cudaStream_t stream) {
+fp8q_status launch_skinny(const uint8_t* A, int64_t Mg, const float* sa, int64_t ldsa,
+                          const uint8_t* B, int64_t Ng, int64_t Kg, SkinnyParams p,
+                          cudaStream_t stream) {
   using Shape = SkinnyShape<kBN>;
-  CUtensorMap tmB;
-  if (!encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, Kg, Ng, Kg, kSkBK, kBN,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
+  p.b_slice = kBN * kSkBK;  // 16 rows x 128 B = 2 KB: a multiple of the 1024-byte atom
+  const uint32_t per_slice = p.a_slice + p.b_slice;
+  // G slices per super-stage: up to 8, and at least two super-stages in the ring
+  p.G = static_cast<int32_t>(std::clamp<uint32_t>(kSkSmemTarget / 2 / per_slice, 1u,
+                                                  static_cast<uint32_t>(kSkMaxG)));
+  p.stages = static_cast<int32_t>(std::clamp<uint32_t>(kSkSmemTarget / (p.G * per_slice), 2u,
+                                                       static_cast<uint32_t>(kSkMaxStages)));
+  const uint32_t a_stage = p.G * p.a_slice, b_stage = p.G * p.b_slice;
+  p.off_b = p.stages * a_stage;
+  uint32_t data = p.off_b + p.stages * b_stage;
+  // the MMA reads 128 rows from the last A slice: keep that inside the allocation
+  data = std::max<uint32_t>(data, (p.stages - 1) * a_stage + (p.G - 1) * p.a_slice + kSkATileRead);
+  // every TMA destination in shared memory starts on a 128-byte boundary
+  p.sa_slot = (p.G * p.a_rows * 4u + 127u) & ~127u;
+  p.off_sa = (data + 127u) & ~127u;
+  p.off_sb = p.off_sa + kSkScRing * p.sa_slot;
+  p.off_bars = (p.off_sb + static_cast<uint32_t>(p.kblocks) * 4u + 7u) & ~7u;
+  if (p.a_slice % 1024u || p.b_slice % 1024u || p.off_b % 1024u || p.off_sa % 128u ||
+      p.sa_slot % 128u)
     return FP8Q_ERR_UNSUPPORTED;
-  p.b_stage = kBN * kSkBK;  // 16 rows x 128 B = 2 KB: a multiple of the 1024-byte atom
-  const uint32_t per_stage = p.a_stage + p.b_stage;
-  p.stages = static_cast<int32_t>(
-      std::clamp<uint32_t>(kSkSmemTarget / per_stage, 2u, static_cast<uint32_t>(kSkMaxStages)));
-  uint32_t data = p.stages * per_stage;
-  // the MMA reads 128 rows from the last A stage: keep that inside the allocation
-  data = std::max<uint32_t>(data, (p.stages - 1) * p.a_stage + kSkATileRead);
-  p.off_bars = (data + 7u) & ~7u;
-  const uint32_t bars = (2 * kSkMaxStages + 2 * Shape::kBufs + 1) * 8 + 16;
+  const uint32_t bars = (2 * kSkMaxStages + 2 * Shape::kBufs + 2 * kSkScRing + 1) * 8 + 16;
   const size_t smem = p.off_bars + bars + 1024;
   if (smem > 232448) return FP8Q_ERR_UNSUPPORTED;
+  // A and W as (128 bytes of a slice, rows, slice index): one copy brings G slices of
+  // a row block; the row-scale box covers the same G slices
+  CUtensorMap tmA, tmB, tmSA;
+  const uint64_t kslices = static_cast<uint64_t>(Kg / kSkBK);
+  const uint64_t strides[2] = {static_cast<uint64_t>(Kg), static_cast<uint64_t>(kSkBK)};
+  const uint64_t dims_a[3] = {static_cast<uint64_t>(kSkBK), static_cast<uint64_t>(Mg), kslices};
+  const uint64_t dims_b[3] = {static_cast<uint64_t>(kSkBK), static_cast<uint64_t>(Ng), kslices};
+  const uint32_t box_a[3] = {static_cast<uint32_t>(kSkBK), p.a_rows, static_cast<uint32_t>(p.G)};
+  const uint32_t box_b[3] = {static_cast<uint32_t>(kSkBK), static_cast<uint32_t>(kBN),
+                             static_cast<uint32_t>(p.G)};
+  if (!encode_tmap_3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, dims_a, strides, box_a,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, dims_b, strides, box_b,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, Mg, kslices, ldsa * 4, p.a_rows,
+                      static_cast<uint32_t>(p.G), CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
   if (!skinny_setup<kBN>(smem)) return FP8Q_ERR_CUDA;
   const int64_t grid = static_cast<int64_t>(p.mtiles) * (Ng / kBN);
   if (grid > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  skinny_gemm_kernel<kBN><<<static_cast<unsigned>(grid), kSkThreads, smem, stream>>>(tmA, tmB, p);
+  skinny_gemm_kernel<kBN><<<static_cast<unsigned>(grid), kSkThreads, smem, stream>>>(tmA, tmB, tmSA,
+                                                                                   p);
   return launch_status("skinny_gemm_kernel launch");
 }
 
@@ -305,9 +385,7 @@ fp8q_status launch_skinny_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, i
   p.mtiles = static_cast<int32_t>((Mg + 127) / 128);
   // A box: the token rows (a multiple of 8, at most 128); rows past M read as zeros
   p.a_rows = static_cast<uint32_t>(std::min<int64_t>(128, (Mg + 7) / 8 * 8));
-  p.a_stage = (p.a_rows * kSkBK + 1023u) & ~1023u;
-  p.sa = sa;
-  p.ldsa = ldsa;
+  p.a_slice = p.a_rows * kSkBK;  // a multiple of 1024 since a_rows is a multiple of 8
   p.sb = sb;
   p.sb_sj = sb_sj;
   p.sb_sr = sb_sr;
@@ -316,16 +394,12 @@ fp8q_status launch_skinny_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, i
   p.err = device_error_word();
   p.wait_limit_ns = kWaitLimitNs;
   if (!p.err) return FP8Q_ERR_CUDA;
-  CUtensorMap tmA;
-  if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, Kg, Mg, Kg, kSkBK, p.a_rows,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-    return FP8Q_ERR_UNSUPPORTED;
   // Strip width: the widest strip that still gives every SM at least one CTA (wider
   // strips re-read the token rows from L2 fewer times); 16 if none does.
   const int64_t mt = p.mtiles;
-  if (mt * (Ng / 64) >= sms) return launch_skinny<64>(tmA, B, Ng, Kg, p, stream);
-  if (mt * (Ng / 32) >= sms) return launch_skinny<32>(tmA, B, Ng, Kg, p, stream);
-  return launch_skinny<16>(tmA, B, Ng, Kg, p, stream);
+  if (mt * (Ng / 64) >= sms) return launch_skinny<64>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
+  if (mt * (Ng / 32) >= sms) return launch_skinny<32>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
+  return launch_skinny<16>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
 }
 
 }  // namespace fp8q

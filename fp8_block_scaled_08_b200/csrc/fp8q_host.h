@@ -23,6 +23,12 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
                     uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                     uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// 3D tiled tensor map with explicit byte strides for dimensions 1 and 2 (dimension 0
+// is contiguous); the strides need not increase with the dimension.
+bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                    const uint64_t (&dims)[3], const uint64_t (&strides_bytes)[2],
+                    const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Remembers the text of a failure for fp8q_last_error_message (thread-local).

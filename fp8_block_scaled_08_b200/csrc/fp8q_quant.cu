@@ -385,7 +385,8 @@ __device__ __forceinline__ double sum_squares(const uint4 (&raw)[kChunks], int64
                    __dadd_rn(__dadd_rn(acc[4], acc[5]), __dadd_rn(acc[6], acc[7])));
 }
 
-// y = bf16(fl32(fl32(x r) g)) for one chunk, then the half-warp group quantization.
+// y = bf16(fl32(fl32(x r) g)) for one chunk (gamma staged in shared memory), then the
+// half-warp group quantization.
 __device__ __forceinline__ void norm_quant_chunk(const uint4& xr, const uint16_t* gamma, int64_t c,
                                                  bool act, float r, uint8_t* qrow, float* s,
                                                  int64_t lds, int64_t m, int lane) {
@@ -393,7 +394,7 @@ __device__ __forceinline__ void norm_quant_chunk(const uint4& xr, const uint16_t
   if (act) {
     float xv[8], gv[8];
     unpack_bf16x8(xr, xv);
-    unpack_bf16x8(ld_nc_v4(gamma + c * 8), gv);
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(gamma + c * 8), gv);  // shared memory
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       float a0, a1, b0, b1;
@@ -420,8 +421,11 @@ template <int kChunks>
 __global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma, int64_t M, int64_t H,
     int64_t ldx, float eps, uint8_t* __restrict__ q, float* __restrict__ s, int64_t lds) {
+  extern __shared__ uint4 gamma_sm[];  // H BF16 values, shared by every row
   const int lane = threadIdx.x & 31;
   const int64_t nch = H >> 3;
+  for (int64_t i = threadIdx.x; i < nch; i += blockDim.x) gamma_sm[i] = ld_nc_v4(gamma + i * 8);
+  __syncthreads();
   const int64_t wglobal = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t m = wglobal; m < M; m += nw) {
@@ -440,7 +444,8 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(
     for (int j = 0; j < kChunks; ++j) {
       if (32 * j >= nch) break;  // warp-uniform; nch is a multiple of 16
       const int64_t c = lane + 32 * j;
-      norm_quant_chunk(raw[j], gamma, c, c < nch, r, q + m * H, s, lds, m, lane);
+      norm_quant_chunk(raw[j], reinterpret_cast<const uint16_t*>(gamma_sm), c, c < nch, r,
+                       q + m * H, s, lds, m, lane);
     }
   }
 }
@@ -453,9 +458,12 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_cta_kernel(
     int64_t ldx, float eps, uint8_t* __restrict__ q, float* __restrict__ s, int64_t lds) {
   __shared__ double red[kNormThreads / 32];
   __shared__ float r_sh;
+  extern __shared__ uint4 gamma_sm[];  // H BF16 values, shared by every row
   const int tid = threadIdx.x;
   const int lane = tid & 31, wid = tid >> 5;
   const int64_t nch = H >> 3;
+  for (int64_t i = tid; i < nch; i += kNormThreads) gamma_sm[i] = ld_nc_v4(gamma + i * 8);
+  __syncthreads();
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint16_t* row = x + m * ldx;
     uint4 raw[kNormMaxChunks];
@@ -481,7 +489,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_cta_kernel(
       const int64_t c0 = static_cast<int64_t>(j) * kNormThreads + (tid & ~31);
       if (c0 >= nch) break;  // warp-uniform: nch is a multiple of 16
       const int64_t c = tid + j * kNormThreads;
-      norm_quant_chunk(raw[j], gamma, c, c < nch, r, q + m * H, s, lds, m, lane);
+      norm_quant_chunk(raw[j], reinterpret_cast<const uint16_t*>(gamma_sm), c, c < nch, r,
+                       q + m * H, s, lds, m, lane);
     }
     __syncthreads();  // red / r_sh are reused by the next row
   }
@@ -898,23 +907,25 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   const int sms = sm100_sm_count();
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t gsm = static_cast<size_t>(H) * 2;  // gamma in shared memory
   if (H <= 8 * 32 * kWarpRowChunks) {
     const int64_t ctas = (M + 7) / 8;  // one warp per row
     if (H <= 8 * 32 * 16) {
       static int occ[64];
-      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<16>, 256, 0, occ);
-      rmsnorm_quant_warp_kernel<16><<<grid_for(ctas, per_sm), 256, 0, st>>>(x, gamma, M, H, ldx,
-                                                                            eps, q, s, lds);
+      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<16>, 256, 8 * 32 * 16 * 2, occ);
+      rmsnorm_quant_warp_kernel<16><<<grid_for(ctas, per_sm), 256, gsm, st>>>(x, gamma, M, H, ldx,
+                                                                              eps, q, s, lds);
     } else {
       static int occ[64];
-      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<kWarpRowChunks>, 256, 0, occ);
-      rmsnorm_quant_warp_kernel<kWarpRowChunks><<<grid_for(ctas, per_sm), 256, 0, st>>>(
+      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<kWarpRowChunks>, 256,
+                                       8 * 32 * kWarpRowChunks * 2, occ);
+      rmsnorm_quant_warp_kernel<kWarpRowChunks><<<grid_for(ctas, per_sm), 256, gsm, st>>>(
           x, gamma, M, H, ldx, eps, q, s, lds);
     }
   } else {
     const int64_t grid = M < static_cast<int64_t>(sms) * 64 ? M : static_cast<int64_t>(sms) * 64;
-    rmsnorm_quant_cta_kernel<<<static_cast<int>(grid), kNormThreads, 0, st>>>(x, gamma, M, H, ldx,
-                                                                              eps, q, s, lds);
+    rmsnorm_quant_cta_kernel<<<static_cast<int>(grid), kNormThreads, gsm, st>>>(x, gamma, M, H,
+                                                                                ldx, eps, q, s, lds);
   }
   return launch_status("rmsnorm_quant launch");
 }
