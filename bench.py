@@ -551,7 +551,7 @@ def run_reference(args, rank, world):
 # with only the buffers it needs on the device.
 # --------------------------------------------------------------------------
 
-CASES = ("gemm_fwd", "gemm_dgrad", "gemm_wgrad", "quantizers")
+CASES = ("gemm_fwd", "gemm_dgrad", "gemm_wgrad", "quantizers", "gemm_decode")
 
 
 def run_case(name, reps):
@@ -585,6 +585,17 @@ def run_case(name, reps):
         _, _, qdyT, sdyc = fq.transpose_quant_bf16_alloc(dy, want_row=False)
         dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.linear_wgrad(qdyT, sdyc, qxT, sxT, dw)  # noqa: E731
+    elif name == "gemm_decode":
+        # Qwen3-8B gate/up projection at a 16-token decode batch (skinny-M kernel)
+        dwl = workloads.QWEN3_DECODE[0]
+        dlin = dwl.layer.linears[2]
+        Nd, Kd = dlin.n, dlin.k
+        wd = workloads.normal_bf16((Nd, Kd), dwl.w_std, dwl.seed, workloads.TID_W[dlin.name], dev)
+        xd = workloads.activations_bf16((dwl.tokens, Kd), dwl.seed, workloads.TID_X_MLP, dev)
+        qx, sx = fq.quant_act_1x128_alloc(xd)
+        qw, sw, _ = fq.quant_weight_alloc(wd, want_t=False)
+        y = torch.empty((dwl.tokens, Nd), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.linear_fwd(qx, sx, qw, sw, y)  # noqa: E731
     elif name == "quantizers":
         x = workloads.activations_bf16((M, K), wl.seed, workloads.TID_X_MLP, dev)
         g = workloads.gamma_bf16(K, wl.seed, workloads.TID_GAMMA2, dev)
