@@ -58,6 +58,11 @@ constexpr int kPairM = 2 * BM;
 constexpr int kStages = 4;
 constexpr int kScStages = 8;
 constexpr int kThreads = 384;
+// Leader threads issuing MMAs (alternate slices, warps 1 and 2) when each slice is 8 MMAs
+// (N split in two halves); one for 4 MMAs a slice, where a second issuer measured slower.
+template <bool kSplitN>
+__host__ __device__ constexpr int issuers() { return kSplitN ? 2 : 1; }
+static_assert(kStages % 2 == 0, "each ring stage is always used by the same issuer");
 constexpr uint32_t kRegsLaunch = 168;   // what ptxas allots under __launch_bounds__(384, 1)
 constexpr uint32_t kRegsControl = 40;   // warpgroup 0 after the hand-over
 constexpr uint32_t kRegsPromote = 232;  // warpgroups 1 and 2 after the hand-over
@@ -160,7 +165,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(sfull + i, 1);
       mbar_init(sempty + i, 8);
     }
-    mbar_init(done, 1);
+    mbar_init(done, issuers<kSplitN>());
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -222,9 +227,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader)
+   } else if (warp <= issuers<kSplitN>()) {
+    // ------------------------------------------------------------ MMA issuers (leader)
+    // With two issuers, issuer i = warp - 1 takes the slices that use TMEM buffer i (slice
+    // parity): each slice is an independent group of MMAs into its own buffer, and one
+    // thread needs ~70 cycles to issue each MMA (measured), which for 8 MMAs a slice
+    // approaches the tensor core's own time per slice.
     if (lane == 0 && rank == 0) {
+      const uint32_t issuer = static_cast<uint32_t>(warp - 1);
       // kSplitN: each slice is issued as two N = 128 halves into separate TMEM
       // half-buffers with their own barriers, so a promotion warpgroup starts on its half
       // as soon as that half is done and the MMAs can run half a slice further ahead.
@@ -237,6 +247,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int t = pair; ok && t < num_tiles; t += npairs) {
         for (int kb = 0; ok && kb < p.kblocks; ++kb) {
           const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
+          if (issuers<kSplitN>() == 2 && buf != issuer) {  // the other issuer's slice
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+            ++it;
+            continue;
+          }
           if (!mbar_wait(full + stage, phase, ctl)) { ok = false; break; }
           const uint32_t a0 = smem_u32(smem + kOffA(stage));
           const uint32_t b0 = smem_u32(smem + kOffB(stage));
@@ -270,7 +285,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ++it;
         }
       }
-      // wait for every MMA issued (they read both CTAs' smem and write both TMEMs)
+      // wait for every MMA issued by both issuers (they read both CTAs' smem and write
+      // both TMEMs); `done` completes after each issuer's commit
       mma_commit_pair_multicast(done, 0x1);
       mbar_wait_drain(done, 0, p.wait_limit_ns);
     }

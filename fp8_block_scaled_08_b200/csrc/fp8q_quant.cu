@@ -205,11 +205,17 @@ __device__ __forceinline__ void exp_cw2(float x0, float x1, float& e0, float& e1
   const float kLog2e = 0x1.715476p+0f;
   const float kLn2Hi = 0x1.62ep-1f;
   const float kLn2Lo = 0x1.0bfbe8p-15f;
+  // Adding 1.5 * 2^23 to |v| < 2^22 leaves a float whose unit in the last place is 1, so
+  // the addition itself rounds v to the nearest integer, ties to even (= rint(v)), and
+  // that integer sits in the low mantissa bits: n = bits(t) - bits(1.5 * 2^23). This
+  // keeps the rounding and the 2^n exponent on the FMA/ALU pipes.
+  const float kShift = 0x1.8p+23f;
   x0 = fminf(fmaxf(x0, -80.0f), 88.0f);
   x1 = fminf(fmaxf(x1, -80.0f), 88.0f);
   float l0, l1;
   mul2(l0, l1, x0, x1, kLog2e, kLog2e);
-  const float n0 = rintf(l0), n1 = rintf(l1);
+  const float t0 = __fadd_rn(l0, kShift), t1 = __fadd_rn(l1, kShift);
+  const float n0 = __fsub_rn(t0, kShift), n1 = __fsub_rn(t1, kShift);  // rint(l), exact
   float r0 = x0, r1 = x1;
   fma2(r0, r1, -n0, -n1, kLn2Hi, kLn2Hi);
   fma2(r0, r1, -n0, -n1, kLn2Lo, kLn2Lo);
@@ -233,8 +239,10 @@ __device__ __forceinline__ void exp_cw2(float x0, float x1, float& e0, float& e1
   p0 = c0; p1 = c1;
   c0 = 1.0f; c1 = 1.0f;
   fma2(c0, c1, p0, p1, r0, r1);
-  const float s0 = __int_as_float((static_cast<int>(n0) + 127) << 23);
-  const float s1 = __int_as_float((static_cast<int>(n1) + 127) << 23);
+  const int k0 = __float_as_int(t0) - __float_as_int(kShift);
+  const int k1 = __float_as_int(t1) - __float_as_int(kShift);
+  const float s0 = __int_as_float((k0 + 127) << 23);
+  const float s1 = __int_as_float((k1 + 127) << 23);
   mul2(e0, e1, c0, c1, s0, s1);
 }
 
@@ -628,21 +636,24 @@ __device__ __forceinline__ void tiles_prologue(const TileSmem& sm, int64_t tiles
   }
 }
 
-// After processing tile number i (buffer i & 1): refill it with the tile two ahead.
+// At the start of tile number i >= 1, right after its acquire barrier (so every thread
+// has finished tile i - 1): refill buffer (i + 1) & 1, which held tile i - 1, with tile
+// i + 1. The prologue already issued tiles 0 and 1. One load stays in flight while a
+// tile is processed, and no barrier is needed at the end of a tile.
 template <class Issue>
-__device__ __forceinline__ void tiles_advance(const TileSmem& sm, int64_t t, int64_t tiles,
-                                              int i, Issue issue) {
-  __syncthreads();  // every thread is done reading the buffer
-  const int64_t tn = t + 2 * static_cast<int64_t>(gridDim.x);
-  if (threadIdx.x == 0 && tn < tiles) issue(i & 1, tn);
+__device__ __forceinline__ void tiles_refill(int64_t t, int64_t tiles, int i, Issue issue) {
+  if (i == 0) return;
+  const int64_t tn = t + static_cast<int64_t>(gridDim.x);
+  if (threadIdx.x == 0 && tn < tiles) issue((i + 1) & 1, tn);
 }
 
-// If the loop stopped early, let the copies still in flight land before exiting.
+// If the loop stopped at tile number i_stop (its wait gave up), let the copies still in
+// flight land before exiting: tile i_stop, and tile 1 as well if i_stop is 0.
 __device__ __forceinline__ void tiles_drain(const TileSmem& sm, int64_t t_stop, int64_t tiles,
                                             int i_stop, uint64_t limit_ns) {
   if (threadIdx.x != 0) return;
-  for (int j = 0; j < 2; ++j) {
-    const int i = i_stop + j;  // tile numbers i_stop, i_stop + 1 may be in flight
+  for (int j = 0; j < (i_stop == 0 ? 2 : 1); ++j) {
+    const int i = i_stop + j;
     const int64_t t = t_stop + static_cast<int64_t>(j) * gridDim.x;
     if (t < tiles) {
       const uint32_t a = smem_u32(sm.bar + (i & 1));
@@ -677,6 +688,7 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(
   int64_t t = blockIdx.x;
   for (; t < tiles; t += gridDim.x, ++i) {
     if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    tiles_refill(t, tiles, i, issue);
     const uint16_t* Ts = reinterpret_cast<const uint16_t*>(sm.buf[i & 1]);
     const int64_t nb = t / KB, kb = t % KB;
     uint4 raw[8];
@@ -705,7 +717,6 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(
       *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes8(v, g);
     }
     if (qT) tile_cols_bf16(Ts, nullptr, false, g, qT + (kb * 128) * N + nb * 128, N, nullptr);
-    tiles_advance(sm, t, tiles, i, issue);
   }
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
@@ -736,6 +747,7 @@ __global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
   int64_t t = blockIdx.x;
   for (; t < tiles; t += gridDim.x, ++i) {
     if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    tiles_refill(t, tiles, i, issue);
     const uint16_t* Ts = reinterpret_cast<const uint16_t*>(sm.buf[i & 1]);
     const int64_t mb = t / NB, nb = t % NB;
     if (q_row) {  // each tile row is one 1x128 group, held by a half-warp
@@ -752,7 +764,6 @@ __global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
     }
     tile_cols_bf16(Ts, sm.red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
                    s_col + mb * N + nb * 128);
-    tiles_advance(sm, t, tiles, i, issue);
   }
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
@@ -785,6 +796,7 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
   int64_t t = blockIdx.x;
   for (; t < tiles; t += gridDim.x, ++i) {
     if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    tiles_refill(t, tiles, i, issue);
     const uint8_t* Tq = sm.buf[i & 1];
     const float* rsc = reinterpret_cast<const float*>(Tq + kTileElems);
     const int64_t mb = t / KB, kb = t % KB;
@@ -831,7 +843,6 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
     d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
     d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
     d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
-    tiles_advance(sm, t, tiles, i, issue);
   }
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
