@@ -49,6 +49,10 @@ _SIGS = {
     "fp8q_transpose_quant_bf16": ([_P, _I, _I, _I, _P, _P, _I, _P, _P, _P], ctypes.c_int),
     "fp8q_transpose_quant_fp8": ([_P, _P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
     "fp8q_linear_fwd": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
+    "fp8q_linear_fwd_splitk_workspace": ([_I, _I, _I], ctypes.c_int64),
+    "fp8q_linear_fwd_splitk_counter_bytes": ([_I, _I], ctypes.c_int64),
+    "fp8q_linear_fwd_splitk": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P],
+                               ctypes.c_int),
     "fp8q_linear_dgrad": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_linear_wgrad": ([_P, _P, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_debug_wait_timeout": ([_I, _P], ctypes.c_int),
@@ -215,6 +219,35 @@ def linear_fwd(qa, sa, qw, sw, y, stream=None):
     N = qw.shape[0]
     _check(_lib.fp8q_linear_fwd(_ptr(qa), _ptr(sa), sa.shape[1], _ptr(qw), _ptr(sw), M, N, K,
                                 _ptr(y), _rows_dense(y, "y"), _stream(stream)), "fp8q_linear_fwd")
+
+
+def linear_fwd_splitk_workspace_bytes(M, N, K):
+    """Bytes of workspace fp8q_linear_fwd_splitk needs for this shape (0 if unsupported)."""
+    return int(_lib.fp8q_linear_fwd_splitk_workspace(M, N, K))
+
+
+def splitk_workspace(M, N, K, device):
+    """A workspace for fp8q_linear_fwd_splitk, zero-filled (its counters must start at
+    zero; the kernel leaves them at zero)."""
+    n = linear_fwd_splitk_workspace_bytes(M, N, K)
+    if n <= 0:
+        raise ValueError("no split-K workspace for M=%d N=%d K=%d" % (M, N, K))
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def linear_fwd_splitk(qa, sa, qw, sw, y, workspace, stream=None):
+    """a5 at decode sizes with K split over CTAs (same bits as linear_fwd); `workspace`
+    is a uint8 device tensor from splitk_workspace (not shared by concurrent calls)."""
+    for t, n in ((qa, "qa"), (sa, "sa"), (qw, "qw"), (sw, "sw")):
+        _dense(t, n)
+    _want(y, torch.bfloat16, 2, "y")
+    _want(workspace, torch.uint8, 1, "workspace")
+    M, K = qa.shape
+    N = qw.shape[0]
+    _check(_lib.fp8q_linear_fwd_splitk(_ptr(qa), _ptr(sa), sa.shape[1], _ptr(qw), _ptr(sw), M, N,
+                                       K, _ptr(y), _rows_dense(y, "y"), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)),
+           "fp8q_linear_fwd_splitk")
 
 
 def linear_dgrad(qdy, sdy, qwT, sw, dx, stream=None):

@@ -67,10 +67,15 @@ struct SkinnyParams {
   uint32_t sa_slot;           // G * a_rows * 4 rounded up to 128 (TMA destination alignment)
   uint32_t off_sb;            // block scales of the strip: kblocks fp32
   uint32_t off_bars;
+  const float* sa;
+  int64_t ldsa;
   const float* sb;
   int64_t sb_sj, sb_sr;
   uint16_t* y;
   int64_t ldy;
+  int32_t splits;         // CTAs per output strip along K (split variant)
+  float* ws_partials;     // [strip][kb][M][kBN] raw slice products (split variant)
+  unsigned* ws_counters;  // [strip] finished CTAs (split variant; zero between calls)
   unsigned* err;
   uint64_t wait_limit_ns;
 };
@@ -103,13 +108,14 @@ __device__ __forceinline__ void sk_tmem_load(uint32_t taddr, uint32_t (&r)[kBN])
   tmem_wait_ld();
 }
 
-template <int kBN>
+template <int kBN, bool kSplit>
 __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const __grid_constant__ CUtensorMap tmSA, const SkinnyParams p) {
   using Shape = SkinnyShape<kBN>;
   constexpr int kBufs = Shape::kBufs;
   extern __shared__ uint8_t smem_raw[];
+  __shared__ int last_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int S = p.stages, G = p.G, KB = p.kblocks;
@@ -129,13 +135,18 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mt = blockIdx.x % p.mtiles;
-  const int nt = blockIdx.x / p.mtiles;
+  // CTA -> (output strip, part of K); the CTAs of one strip are adjacent
+  const int tile = kSplit ? static_cast<int>(blockIdx.x) / p.splits : static_cast<int>(blockIdx.x);
+  const int part = kSplit ? static_cast<int>(blockIdx.x) % p.splits : 0;
+  const int mt = tile % p.mtiles;
+  const int nt = tile / p.mtiles;
   const int m0 = mt * 128;
   const int n0 = nt * kBN;
   const int rows = min(128, p.M - m0);       // token rows of this tile
   const int quarters = (rows + 31) >> 5;     // TMEM lane quarters that hold them
-  const int nst = (KB + G - 1) / G;          // super-stages over K
+  const int kb_begin = kSplit ? (part * KB) / p.splits : 0;
+  const int nsl = (kSplit ? ((part + 1) * KB) / p.splits : KB) - kb_begin;  // slices here
+  const int nst = (nsl + G - 1) / G;         // super-stages
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -157,10 +168,10 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
-    prefetch_tensormap(&tmSA);
+    if (!kSplit) prefetch_tensormap(&tmSA);
   }
   if (warp == 1) tmem_alloc<Shape::kTmemCols>(tmem_slot);
-  {  // block scales of this strip, one per slice
+  if (!kSplit) {  // block scales of this strip, one per slice
     const float* sbp = p.sb + static_cast<int64_t>(n0 / 128) * p.sb_sj;
     for (int kb = threadIdx.x; kb < KB; kb += kSkThreads)
       sb_s[kb] = __ldg(sbp + static_cast<int64_t>(kb) * p.sb_sr);
@@ -181,18 +192,20 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
       bool ok = true;
       for (int st = 0; st < nst; ++st) {
         const int s = st % S;
+        const int z = kb_begin + st * G;
         if (!mbar_wait(empty + s, (static_cast<uint32_t>(st / S) & 1u) ^ 1u, ctl)) { ok = false; break; }
         mbar_arrive_expect_tx(full + s, stage_tx);
-        tma_load_3d(a_ring + s * a_stage, &tmA, 0, m0, st * G, full + s);
-        tma_load_3d(b_ring + s * b_stage, &tmB, 0, n0, st * G, full + s);
+        tma_load_3d(a_ring + s * a_stage, &tmA, 0, m0, z, full + s);
+        tma_load_3d(b_ring + s * b_stage, &tmB, 0, n0, z, full + s);
         issued = st + 1;
+        if (kSplit) continue;  // raw products: no scales here
         const int si = st % kSkScRing;
         if (!mbar_wait(sempty + si, (static_cast<uint32_t>(st / kSkScRing) & 1u) ^ 1u, ctl)) {
           ok = false;
           break;
         }
         mbar_arrive_expect_tx(sfull + si, G * p.a_rows * 4u);
-        tma_load_2d(smem + p.off_sa + si * p.sa_slot, &tmSA, m0, st * G, sfull + si);
+        tma_load_2d(smem + p.off_sa + si * p.sa_slot, &tmSA, m0, z, sfull + si);
         sc_issued = st + 1;
       }
       if (!ok) {  // let the copies still in flight land before the CTA exits
@@ -206,7 +219,7 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
     __syncwarp();
   } else if (warp <= kSkIssuers) {
     // ------------------------------------------------------------ MMA issuers
-    // issuer i = warp - 1 takes the slices kb with kb % kSkIssuers == i
+    // issuer i = warp - 1 takes the slices i, i + kSkIssuers, ... of this CTA
     if (lane == 0) {
       const int issuer = warp - 1;
       const uint32_t idesc = idesc_e4m3_f32(128, kBN);
@@ -215,11 +228,11 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
         const int s = st % S;
         if (!mbar_wait(full + s, static_cast<uint32_t>(st / S) & 1u, ctl)) { ok = false; break; }
         for (int j = 0; j < G; ++j) {
-          const int kb = st * G + j;
-          if (kb >= KB) break;
-          if (kb % kSkIssuers != issuer) continue;
-          const int buf = kb % kBufs;
-          const uint32_t tph = static_cast<uint32_t>(kb / kBufs) & 1u;
+          const int i = st * G + j;  // slice number within this CTA
+          if (i >= nsl) break;
+          if (i % kSkIssuers != issuer) continue;
+          const int buf = i % kBufs;
+          const uint32_t tph = static_cast<uint32_t>(i / kBufs) & 1u;
           if (!mbar_wait(tempty + buf, tph ^ 1u, ctl)) { ok = false; break; }
           tc_fence_after();
           mma_f8f6f4_slice(tmem_base + buf * kBN,
@@ -245,37 +258,50 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
       const int srow = row < static_cast<int>(p.a_rows) ? row : 0;
       float acc[kBN];
 #pragma unroll
-      for (int i = 0; i < kBN; ++i) acc[i] = 0.0f;
+      for (int c = 0; c < kBN; ++c) acc[c] = 0.0f;
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int st = kb / G, j = kb - st * G;
-        const int si = st % kSkScRing;
-        if (j == 0 &&
-            !mbar_wait_warp(sfull + si, static_cast<uint32_t>(st / kSkScRing) & 1u, ctl)) {
-          ok = false;
-          break;
+      for (int i = 0; i < nsl; ++i) {
+        float s = 0.0f;
+        if (!kSplit) {
+          const int st = i / G, j = i - st * G;
+          const int si = st % kSkScRing;
+          if (j == 0 &&
+              !mbar_wait_warp(sfull + si, static_cast<uint32_t>(st / kSkScRing) & 1u, ctl)) {
+            ok = false;
+            break;
+          }
+          const float sa =
+              reinterpret_cast<const float*>(smem + p.off_sa + si * p.sa_slot)[j * p.a_rows + srow];
+          s = __fmul_rn(sa, sb_s[i]);
+          if (j == G - 1 || i == nsl - 1) {  // last use of this super-stage's scales
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sempty + si);
+          }
         }
-        const float sa =
-            reinterpret_cast<const float*>(smem + p.off_sa + si * p.sa_slot)[j * p.a_rows + srow];
-        const float s = __fmul_rn(sa, sb_s[kb]);
-        if (j == G - 1 || kb == KB - 1) {  // last use of this super-stage's scales
-          __syncwarp();
-          if (lane == 0) mbar_arrive(sempty + si);
-        }
-        const int buf = kb % kBufs;
-        const uint32_t tph = static_cast<uint32_t>(kb / kBufs) & 1u;
+        const int buf = i % kBufs;
+        const uint32_t tph = static_cast<uint32_t>(i / kBufs) & 1u;
         if (!mbar_wait_warp(tfull + buf, tph, ctl)) { ok = false; break; }
         tc_fence_after();
         uint32_t r[kBN];
         sk_tmem_load<kBN>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN, r);
+        if (kSplit) {
+          if (row_ok) {  // raw products of slice kb_begin + i, row m: kBN fp32
+            uint4* dst = reinterpret_cast<uint4*>(
+                p.ws_partials + ((static_cast<int64_t>(tile) * KB + kb_begin + i) * p.M + m) * kBN);
 #pragma unroll
-        for (int i = 0; i < kBN; i += 2)
-          fma2(acc[i], acc[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), s, s);
+            for (int c = 0; c < kBN / 4; ++c)
+              dst[c] = make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kBN; c += 2)
+            fma2(acc[c], acc[c + 1], __uint_as_float(r[c]), __uint_as_float(r[c + 1]), s, s);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty + buf);
       }
-      if (ok && row_ok) {
+      if (!kSplit && ok && row_ok) {
         uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m) * p.ldy + n0);
 #pragma unroll
         for (int c = 0; c < kBN / 8; ++c) {
@@ -293,16 +319,59 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
     tc_fence_after();
     tmem_dealloc<Shape::kTmemCols>(tmem_base);
   }
+  if (kSplit) {
+    // Every thread of this CTA has written its partials (barrier above). The CTA that
+    // completes the strip's count promotes all its slices in order and resets the count.
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const unsigned prev = atomicAdd(p.ws_counters + tile, 1u);
+      last_flag = (prev == static_cast<unsigned>(p.splits - 1)) ? 1 : 0;
+      if (last_flag) atomicExch(p.ws_counters + tile, 0u);
+    }
+    __syncthreads();
+    if (last_flag) {
+      __threadfence();
+      // scale products sa * sb of every (slice, row) of the strip, in the shared memory
+      // the stages no longer use (the launch checks it fits: KB * M floats)
+      float* sc = reinterpret_cast<float*>(smem);
+      const float* sbp = p.sb + static_cast<int64_t>(n0 / 128) * p.sb_sj;
+      for (int idx = threadIdx.x; idx < KB * rows; idx += kSkThreads) {
+        const int kb = idx / rows, mr = idx - kb * rows;
+        sc[idx] = __fmul_rn(__ldg(p.sa + static_cast<int64_t>(kb) * p.ldsa + m0 + mr),
+                            __ldg(sbp + static_cast<int64_t>(kb) * p.sb_sr));
+      }
+      __syncthreads();
+      // each output: the partials of all slices in increasing kb, 16 loads in flight
+      constexpr int kBatch = 16;
+      const int64_t pstride = static_cast<int64_t>(p.M) * kBN;
+      for (int idx = threadIdx.x; idx < rows * kBN; idx += kSkThreads) {
+        const int mr = idx / kBN, c = idx % kBN;
+        const float* pp = p.ws_partials + (static_cast<int64_t>(tile) * KB * p.M + m0 + mr) * kBN + c;
+        float acc = 0.0f;
+        for (int kb0 = 0; kb0 < KB; kb0 += kBatch) {
+          float part[kBatch];
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j)
+            part[j] = (kb0 + j < KB) ? __ldcg(pp + (kb0 + j) * pstride) : 0.0f;
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j)
+            if (kb0 + j < KB) acc = __fmaf_rn(part[j], sc[(kb0 + j) * rows + mr], acc);
+        }
+        p.y[static_cast<int64_t>(m0 + mr) * p.ldy + n0 + c] =
+            static_cast<uint16_t>(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+      }
+    }
+  }
 }
 
-// Per device and strip width: opt in to the shared memory the launch asks for.
-template <int kBN>
+// Per device and kernel variant: opt in to the shared memory the launch asks for.
+template <int kBN, bool kSplit>
 bool skinny_setup(size_t smem_bytes) {
   static size_t opted[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (opted[dev] >= smem_bytes) return true;
-  const cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel<kBN>,
+  const cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel<kBN, kSplit>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem_bytes));
   if (e != cudaSuccess) {
@@ -314,16 +383,22 @@ bool skinny_setup(size_t smem_bytes) {
   return true;
 }
 
-template <int kBN>
+template <int kBN, bool kSplit>
 fp8q_status launch_skinny(const uint8_t* A, int64_t Mg, const float* sa, int64_t ldsa,
                           const uint8_t* B, int64_t Ng, int64_t Kg, SkinnyParams p,
                           cudaStream_t stream) {
   using Shape = SkinnyShape<kBN>;
   p.b_slice = kBN * kSkBK;  // 16 rows x 128 B = 2 KB: a multiple of the 1024-byte atom
   const uint32_t per_slice = p.a_slice + p.b_slice;
-  // G slices per super-stage: up to 8, and at least two super-stages in the ring
+  // G slices per super-stage: up to 8 and at least two super-stages in the ring; when K
+  // is split, G divides each CTA's share (the splits divide the slice count), so no
+  // copy reaches into the next CTA's slices
   p.G = static_cast<int32_t>(std::clamp<uint32_t>(kSkSmemTarget / 2 / per_slice, 1u,
                                                   static_cast<uint32_t>(kSkMaxG)));
+  if (kSplit) {
+    const int32_t share = p.kblocks / p.splits;
+    while (share % p.G) --p.G;
+  }
   p.stages = static_cast<int32_t>(std::clamp<uint32_t>(kSkSmemTarget / (p.G * per_slice), 2u,
                                                        static_cast<uint32_t>(kSkMaxStages)));
   const uint32_t a_stage = p.G * p.a_slice, b_stage = p.G * p.b_slice;
@@ -339,6 +414,15 @@ fp8q_status launch_skinny(const uint8_t* A, int64_t Mg, const float* sa, int64_t
   if (p.a_slice % 1024u || p.b_slice % 1024u || p.off_b % 1024u || p.off_sa % 128u ||
       p.sa_slot % 128u)
     return FP8Q_ERR_UNSUPPORTED;
+  if (kSplit) {  // the last CTA's scale table reuses the stage memory: make it fit
+    const uint64_t table = static_cast<uint64_t>(p.kblocks) * static_cast<uint64_t>(Mg) * 4u;
+    if (table > p.off_sa) {
+      if (table > 200u * 1024u) return FP8Q_ERR_UNSUPPORTED;
+      p.off_sa = static_cast<uint32_t>((table + 127u) & ~127ull);
+      p.off_sb = p.off_sa + kSkScRing * p.sa_slot;
+      p.off_bars = (p.off_sb + static_cast<uint32_t>(p.kblocks) * 4u + 7u) & ~7u;
+    }
+  }
   const uint32_t bars = (2 * kSkMaxStages + 2 * Shape::kBufs + 2 * kSkScRing + 1) * 8 + 16;
   const size_t smem = p.off_bars + bars + 1024;
   if (smem > 232448) return FP8Q_ERR_UNSUPPORTED;
@@ -359,11 +443,11 @@ fp8q_status launch_skinny(const uint8_t* A, int64_t Mg, const float* sa, int64_t
       !encode_tmap_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, Mg, kslices, ldsa * 4, p.a_rows,
                       static_cast<uint32_t>(p.G), CU_TENSOR_MAP_SWIZZLE_NONE))
     return FP8Q_ERR_UNSUPPORTED;
-  if (!skinny_setup<kBN>(smem)) return FP8Q_ERR_CUDA;
-  const int64_t grid = static_cast<int64_t>(p.mtiles) * (Ng / kBN);
+  if (!skinny_setup<kBN, kSplit>(smem)) return FP8Q_ERR_CUDA;
+  const int64_t grid = static_cast<int64_t>(p.mtiles) * (Ng / kBN) * (kSplit ? p.splits : 1);
   if (grid > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  skinny_gemm_kernel<kBN><<<static_cast<unsigned>(grid), kSkThreads, smem, stream>>>(tmA, tmB, tmSA,
-                                                                                   p);
+  skinny_gemm_kernel<kBN, kSplit><<<static_cast<unsigned>(grid), kSkThreads, smem, stream>>>(
+      tmA, tmB, tmSA, p);
   return launch_status("skinny_gemm_kernel launch");
 }
 
@@ -386,6 +470,11 @@ fp8q_status launch_skinny_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, i
   // A box: the token rows (a multiple of 8, at most 128); rows past M read as zeros
   p.a_rows = static_cast<uint32_t>(std::min<int64_t>(128, (Mg + 7) / 8 * 8));
   p.a_slice = p.a_rows * kSkBK;  // a multiple of 1024 since a_rows is a multiple of 8
+  p.sa = sa;
+  p.ldsa = ldsa;
+  p.splits = 1;
+  p.ws_partials = nullptr;
+  p.ws_counters = nullptr;
   p.sb = sb;
   p.sb_sj = sb_sj;
   p.sb_sr = sb_sr;
@@ -397,9 +486,95 @@ fp8q_status launch_skinny_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, i
   // Strip width: the widest strip that still gives every SM at least one CTA (wider
   // strips re-read the token rows from L2 fewer times); 16 if none does.
   const int64_t mt = p.mtiles;
-  if (mt * (Ng / 64) >= sms) return launch_skinny<64>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
-  if (mt * (Ng / 32) >= sms) return launch_skinny<32>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
-  return launch_skinny<16>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
+  if (mt * (Ng / 64) >= sms) return launch_skinny<64, false>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
+  if (mt * (Ng / 32) >= sms) return launch_skinny<32, false>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
+  return launch_skinny<16, false>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
+}
+
+// Split variant: 64-column strips, K divided over `splits` CTAs per strip so that the
+// grid covers about two CTAs per SM.
+constexpr int kSplitBN = 64;
+
+int64_t splitk_counter_bytes(int64_t N) { return (4 * (N / kSplitBN) + 255) / 256 * 256; }
+
+int64_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return splitk_counter_bytes(N) + N * (K / kSkBK) * M * 4;
+}
+
+fp8q_status launch_skinny_gemm_splitk(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t Ng,
+                                      int64_t Kg, const float* sa, int64_t ldsa, const float* sb,
+                                      int64_t sb_sj, int64_t sb_sr, uint16_t* y, int64_t ldy,
+                                      void* workspace, int64_t workspace_bytes,
+                                      cudaStream_t stream) {
+  const int sms = sm100_sm_count();
+  if (!sms) return FP8Q_ERR_UNSUPPORTED;
+  if (Mg <= 0 || Mg > 128 || Ng % 128 || Kg % 128 || Ng > 0x7FFFFFFF || Kg > 0x7FFFFFFF)
+    return FP8Q_ERR_SHAPE;
+  const int64_t strips = Ng / kSplitBN;
+  const int64_t kblocks = Kg / kSkBK;
+  // the smallest divisor of the slice count that gives about two CTAs per SM
+  const int64_t target = (2 * sms + strips - 1) / strips;
+  int64_t splits = 1;
+  if (target > 1) {
+    splits = kblocks;
+    for (int64_t d = target; d < kblocks; ++d)
+      if (kblocks % d == 0) { splits = d; break; }
+  }
+  if (splits <= 1)  // the strips alone fill the GPU
+    return launch_skinny_gemm(A, B, Mg, Ng, Kg, sa, ldsa, sb, sb_sj, sb_sr, y, ldy, stream);
+  if (!workspace || !aligned16(workspace)) return workspace ? FP8Q_ERR_ALIGN : FP8Q_ERR_NULL;
+  if (workspace_bytes < splitk_workspace_bytes(Mg, Ng, Kg)) return FP8Q_ERR_SHAPE;
+  SkinnyParams p;
+  p.M = static_cast<int32_t>(Mg);
+  p.N = static_cast<int32_t>(Ng);
+  p.kblocks = static_cast<int32_t>(kblocks);
+  p.mtiles = 1;
+  p.a_rows = static_cast<uint32_t>((Mg + 7) / 8 * 8);
+  p.a_slice = p.a_rows * kSkBK;
+  p.sa = sa;
+  p.ldsa = ldsa;
+  p.sb = sb;
+  p.sb_sj = sb_sj;
+  p.sb_sr = sb_sr;
+  p.y = y;
+  p.ldy = ldy;
+  p.splits = static_cast<int32_t>(splits);
+  p.ws_counters = static_cast<unsigned*>(workspace);
+  p.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           splitk_counter_bytes(Ng));
+  p.err = device_error_word();
+  p.wait_limit_ns = kWaitLimitNs;
+  if (!p.err) return FP8Q_ERR_CUDA;
+  return launch_skinny<kSplitBN, true>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
 }
 
 }  // namespace fp8q
+
+using namespace fp8q;
+
+extern "C" int64_t fp8q_linear_fwd_splitk_workspace(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || M > 128 || N <= 0 || K <= 0 || N % 128 || K % 128) return 0;
+  return splitk_workspace_bytes(M, N, K);
+}
+
+extern "C" int64_t fp8q_linear_fwd_splitk_counter_bytes(int64_t M, int64_t N) {
+  if (M <= 0 || M > 128 || N <= 0 || N % 128) return 0;
+  return splitk_counter_bytes(N);
+}
+
+extern "C" fp8q_status fp8q_linear_fwd_splitk(const uint8_t* qa, const float* sa, int64_t ldsa,
+                                              const uint8_t* qw, const float* sw, int64_t M,
+                                              int64_t N, int64_t K, uint16_t* y, int64_t ldy,
+                                              void* workspace, int64_t workspace_bytes,
+                                              void* stream) {
+  if (!qa || !sa || !qw || !sw || !y) return FP8Q_ERR_NULL;
+  if (M <= 0 || M > 128 || N <= 0 || K <= 0 || N % 128 || K % 128 || ldsa < M || ldy < N)
+    return FP8Q_ERR_SHAPE;
+  if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y) ||
+      ldsa % 4 || ldy % 8)
+    return FP8Q_ERR_ALIGN;
+  // B = W [N][K]; block scale of (n, slice r) = sw[(n/128)*(K/128) + r]
+  return launch_skinny_gemm_splitk(qa, qw, M, N, K, sa, ldsa, sw, K / 128, 1, y, ldy, workspace,
+                                   workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+

@@ -357,9 +357,9 @@ __global__ void __launch_bounds__(256) rowgroup_quant_kernel(Src src, int64_t M,
 
 // ---------------------------------------------------------------------------
 // a3: RMSNorm + 1x128 quantization.
-// Rows of up to kWarpRowChunks*256 elements: one warp per row (the row stays in
-// registers, the sum of squares is a warp reduction), 8 rows per CTA.
-// Longer rows: one CTA (256 threads) per row.
+// Rows of up to kWarpRowChunks*256 elements in batches of more than 1024 rows: one warp
+// per row (the row stays in registers, the sum of squares is a warp reduction), 8 rows
+// per CTA. Longer rows, and small batches: one CTA (256 threads) per row.
 // Thread t of the row owns 8-element chunks t, t+T, ... (T = threads per row), so
 // that each half-warp covers one 128-group.
 // ---------------------------------------------------------------------------
@@ -919,7 +919,9 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t gsm = static_cast<size_t>(H) * 2;  // gamma in shared memory
-  if (H <= 8 * 32 * kWarpRowChunks) {
+  // One warp per row needs many rows to fill the GPU; up to 1024 rows one CTA per row
+  // is faster (measured 3x at 16-256 rows, equal at 8192).
+  if (H <= 8 * 32 * kWarpRowChunks && M > 1024) {
     const int64_t ctas = (M + 7) / 8;  // one warp per row
     if (H <= 8 * 32 * 16) {
       static int occ[64];

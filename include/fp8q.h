@@ -138,6 +138,30 @@ fp8q_status fp8q_linear_fwd(const uint8_t* qa, const float* sa, int64_t ldsa,
                             const uint8_t* qw, const float* sw, int64_t M, int64_t N,
                             int64_t K, uint16_t* y, int64_t ldy, void* stream);
 
+/* a5 at decode sizes with the K dimension split over several CTAs, bit for bit the
+ * same result as fp8q_linear_fwd. With few tokens the forward GEMM is bound by how many
+ * 128-wide K slices one CTA walks per byte of weights; splitting K multiplies the CTAs
+ * per output strip. Each CTA writes the raw FP8 products of its slices (fp32, before
+ * any scale) to `workspace`; the last CTA to finish a strip (an atomic counter in the
+ * workspace) promotes all slices of the strip in increasing kb from +0, exactly as the
+ * other kernels do, and writes Y.
+ *   workspace: device memory owned by the caller, 16-byte aligned, at least
+ *   fp8q_linear_fwd_splitk_workspace(M, N, K) bytes. Its first
+ *   fp8q_linear_fwd_splitk_counter_bytes(M, N) bytes are counters that must be zero
+ *   before the first call (e.g. one cudaMemset) and are zero again when a call has
+ *   completed; the rest needs no initialisation. Two calls that share a workspace
+ *   must not run at the same time (they would race on the counters and partials).
+ * Shapes that already fill the GPU without a split fall back to fp8q_linear_fwd's
+ * kernel and leave the workspace untouched.
+ * Requires 1 <= M <= 128, N % 128 == 0, K % 128 == 0; other arguments as
+ * fp8q_linear_fwd. FP8Q_ERR_SHAPE if workspace_bytes is too small. */
+int64_t fp8q_linear_fwd_splitk_workspace(int64_t M, int64_t N, int64_t K);
+int64_t fp8q_linear_fwd_splitk_counter_bytes(int64_t M, int64_t N);
+fp8q_status fp8q_linear_fwd_splitk(const uint8_t* qa, const float* sa, int64_t ldsa,
+                                   const uint8_t* qw, const float* sw, int64_t M, int64_t N,
+                                   int64_t K, uint16_t* y, int64_t ldy, void* workspace,
+                                   int64_t workspace_bytes, void* stream);
+
 /* a7. DGrad in FP8 ("Esquema de Cuantización", backward GEMMs):
  *   dX[m,k] = sum_nb sdy[nb][m] * sw[nb][k/128] * sum_{n in nb} qdy[m,n] * qw[n,k]
  * with the row-wise dY codes of fp8q_transpose_quant_bf16 and the transposed

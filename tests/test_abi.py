@@ -105,6 +105,28 @@ def test_validation_gemms():
     assert call("fp8q_linear_wgrad", A, B, C, D, 128, 256, 256, ODD, 256, NUL) == 3
 
 
+def test_validation_splitk():
+    f = "fp8q_linear_fwd_splitk"
+    W = ctypes.c_void_p(0x10000)
+    assert call(f, A, B, 16, C, D, 200, 256, 128, E, 256, W, 1 << 20, NUL) == 2    # M > 128
+    assert call(f, A, B, 16, C, D, 16, 200, 128, E, 256, W, 1 << 20, NUL) == 2    # N % 128
+    assert call(f, A, B, 16, C, D, 16, 256, 100, E, 256, W, 1 << 20, NUL) == 2    # K % 128
+    assert call(f, A, B, 16, C, D, 16, 256, 128, E, 260, W, 1 << 20, NUL) == 3    # ldy % 8
+    assert call(f, NUL, B, 16, C, D, 16, 256, 128, E, 256, W, 1 << 20, NUL) == 1
+
+
+def test_splitk_workspace_sizes():
+    import fp8_block_scaled_08_b200 as f
+    # counters: one word per 64-column strip, padded to 256 bytes; partials: one fp32 per
+    # (output column, K slice, token row)
+    assert f._lib.fp8q_linear_fwd_splitk_counter_bytes(16, 4096) == 256
+    assert f._lib.fp8q_linear_fwd_splitk_counter_bytes(16, 24576) == 1536
+    assert f._lib.fp8q_linear_fwd_splitk_workspace(16, 4096, 4096) == 256 + 4096 * 32 * 16 * 4
+    assert f.linear_fwd_splitk_workspace_bytes(1, 128, 256) == 256 + 128 * 2 * 1 * 4
+    assert f._lib.fp8q_linear_fwd_splitk_workspace(129, 4096, 4096) == 0
+    assert f._lib.fp8q_linear_fwd_splitk_workspace(16, 100, 4096) == 0
+
+
 def test_validation_tile_quantizers():
     assert call("fp8q_transpose_quant_bf16", A, 100, 128, 128, B, C, 128, D, E, NUL) == 2
     assert call("fp8q_transpose_quant_bf16", A, 128, 128, 128, B, NUL, 128, D, E, NUL) == 1

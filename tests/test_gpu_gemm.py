@@ -175,3 +175,38 @@ def test_full_size_llama_layer_gemms_sampled(fq, oracle_mod):
     check(dw, lambda rows: oracle_mod.linear_wgrad(qdoT_n, sdo_n, qaT_n, saT_n, rows),
           lambda n: oracle_mod.dequant_cols(qdoT_n, sdo_n, n, 1)[0],
           lambda k: oracle_mod.dequant_cols(qaT_n, saT_n, k, 1)[0], "o wgrad")
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 4096, 4096), (1, 512, 640), (100, 4608, 3584),
+                                   (128, 1024, 2048), (32, 5120, 5120), (16, 256, 27648)])
+def test_splitk_matches_linear_fwd_bitwise(fq, oracle_mod, M, N, K):
+    """The split-K forward writes raw slice products to its workspace and promotes them in
+    order in the last CTA of each strip: the same bits as fp8q_linear_fwd, twice in a row
+    on one workspace (its counters return to zero), and within the oracle's tolerance."""
+    qx, sx, qw, sw, _ = quantized_linear(fq, M, N, K, 1400 + M)
+    ref = fq.linear_fwd_alloc(qx, sx, qw, sw)
+    ws = fq.splitk_workspace(M, N, K, DEV)
+    counters = fq._lib.fp8q_linear_fwd_splitk_counter_bytes(M, N)
+    for _ in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+        fq.linear_fwd_splitk(qx, sx, qw, sw, y, ws)
+        torch.cuda.synchronize()
+        assert fq.device_error() == fq.FP8Q_OK
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+        assert int(ws[:counters].count_nonzero()) == 0
+    if M * N * K <= 2 ** 28:
+        r, ab = oracle_mod.linear_fwd(np_u8(qx), np_f32(sx), np_u8(qw), np_f32(sw))
+        assert_gemm_close(y.float().cpu().numpy(), r, ab, "split-K fwd %dx%dx%d" % (M, N, K))
+
+
+def test_splitk_workspace_errors(fq):
+    qx, sx, qw, sw, _ = quantized_linear(fq, 16, 4096, 4096, 1500)
+    y = torch.empty((16, 4096), dtype=torch.bfloat16, device=DEV)
+    small = torch.zeros(1024, dtype=torch.uint8, device=DEV)
+    with pytest.raises(fq.Fp8qError) as e:
+        fq.linear_fwd_splitk(qx, sx, qw, sw, y, small)
+    assert e.value.status == fq.FP8Q_ERR_SHAPE
+    st = fq._lib.fp8q_linear_fwd_splitk(fq._ptr(qx), fq._ptr(sx), sx.shape[1], fq._ptr(qw),
+                                        fq._ptr(sw), 16, 4096, 4096, fq._ptr(y), 4096, None,
+                                        0, fq._stream())
+    assert st == fq.FP8Q_ERR_NULL
