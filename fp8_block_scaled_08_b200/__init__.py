@@ -53,6 +53,8 @@ _SIGS = {
     "fp8q_linear_fwd_splitk_counter_bytes": ([_I, _I], ctypes.c_int64),
     "fp8q_linear_fwd_splitk": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P],
                                ctypes.c_int),
+    "fp8q_linear_fwd_splitk_noalloc": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P],
+                                       ctypes.c_int),
     "fp8q_linear_dgrad": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_linear_wgrad": ([_P, _P, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_debug_wait_timeout": ([_I, _P], ctypes.c_int),
@@ -248,6 +250,20 @@ def linear_fwd_splitk(qa, sa, qw, sw, y, workspace, stream=None):
                                        K, _ptr(y), _rows_dense(y, "y"), _ptr(workspace),
                                        workspace.numel(), _stream(stream)),
            "fp8q_linear_fwd_splitk")
+
+
+def linear_fwd_splitk_noalloc(qa, sa, qw, sw, y, stream=None):
+    """linear_fwd_splitk on the library's static workspace (no allocation; calls on one
+    device must not overlap)."""
+    for t, n in ((qa, "qa"), (sa, "sa"), (qw, "qw"), (sw, "sw")):
+        _dense(t, n)
+    _want(y, torch.bfloat16, 2, "y")
+    M, K = qa.shape
+    N = qw.shape[0]
+    _check(_lib.fp8q_linear_fwd_splitk_noalloc(_ptr(qa), _ptr(sa), sa.shape[1], _ptr(qw),
+                                               _ptr(sw), M, N, K, _ptr(y), _rows_dense(y, "y"),
+                                               _stream(stream)),
+           "fp8q_linear_fwd_splitk_noalloc")
 
 
 def linear_dgrad(qdy, sdy, qwT, sw, dx, stream=None):

@@ -87,6 +87,8 @@ void set_last_error(const char* where, cudaError_t e) {
            cudaGetErrorName(e));
 }
 
+void set_last_error_text(const char* text) { snprintf(g_last_error, sizeof(g_last_error), "%s", text); }
+
 unsigned* device_error_word() {
   DeviceInfo* d = current_info();
   return d ? d->err : nullptr;

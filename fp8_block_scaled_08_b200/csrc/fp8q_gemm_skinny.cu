@@ -39,6 +39,8 @@
 // Every mbarrier wait is bounded; a wait that gives up records FP8Q_ERR_TIMEOUT in the
 // device error word and the CTA winds down.
 #include <algorithm>
+#include <cstdio>
+#include <mutex>
 
 #include "fp8q_device.cuh"
 #include "fp8q_host.h"
@@ -548,6 +550,51 @@ fp8q_status launch_skinny_gemm_splitk(const uint8_t* A, const uint8_t* B, int64_
   return launch_skinny<kSplitBN, true>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
 }
 
+// The split launch with the counters and the partial products at given addresses
+// (counters zero on entry; left zero).
+fp8q_status launch_skinny_gemm_splitk_into(const uint8_t* A, const uint8_t* B, int64_t Mg,
+                                           int64_t Ng, int64_t Kg, const float* sa, int64_t ldsa,
+                                           const float* sb, int64_t sb_sj, int64_t sb_sr,
+                                           uint16_t* y, int64_t ldy, unsigned* counters,
+                                           float* partials, cudaStream_t stream) {
+  const int sms = sm100_sm_count();
+  if (!sms) return FP8Q_ERR_UNSUPPORTED;
+  if (Mg <= 0 || Mg > 128 || Ng % 128 || Kg % 128 || Ng > 0x7FFFFFFF || Kg > 0x7FFFFFFF)
+    return FP8Q_ERR_SHAPE;
+  const int64_t strips = Ng / kSplitBN;
+  const int64_t kblocks = Kg / kSkBK;
+  const int64_t target = (2 * sms + strips - 1) / strips;
+  int64_t splits = 1;
+  if (target > 1) {
+    splits = kblocks;
+    for (int64_t d = target; d < kblocks; ++d)
+      if (kblocks % d == 0) { splits = d; break; }
+  }
+  if (splits <= 1)  // the strips alone fill the GPU
+    return launch_skinny_gemm(A, B, Mg, Ng, Kg, sa, ldsa, sb, sb_sj, sb_sr, y, ldy, stream);
+  SkinnyParams p;
+  p.M = static_cast<int32_t>(Mg);
+  p.N = static_cast<int32_t>(Ng);
+  p.kblocks = static_cast<int32_t>(kblocks);
+  p.mtiles = 1;
+  p.a_rows = static_cast<uint32_t>((Mg + 7) / 8 * 8);
+  p.a_slice = p.a_rows * kSkBK;
+  p.sa = sa;
+  p.ldsa = ldsa;
+  p.sb = sb;
+  p.sb_sj = sb_sj;
+  p.sb_sr = sb_sr;
+  p.y = y;
+  p.ldy = ldy;
+  p.splits = static_cast<int32_t>(splits);
+  p.ws_counters = counters;
+  p.ws_partials = partials;
+  p.err = device_error_word();
+  p.wait_limit_ns = kWaitLimitNs;
+  if (!p.err) return FP8Q_ERR_CUDA;
+  return launch_skinny<kSplitBN, true>(A, Mg, sa, ldsa, B, Ng, Kg, p, stream);
+}
+
 }  // namespace fp8q
 
 using namespace fp8q;
@@ -578,3 +625,92 @@ extern "C" fp8q_status fp8q_linear_fwd_splitk(const uint8_t* qa, const float* sa
                                    workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------
+// Split-K forward without a caller workspace: the scratch is one static device array
+// per device, laid out as a fixed counter area followed by the partial products (fixed
+// so that the counters never sit where an earlier call of another shape wrote
+// partials). The array is zero when the module loads, the counter area is cleared once
+// more per device before its first use, and every completed call leaves the counters
+// at zero. All calls on a device share the one array, so calls must not overlap.
+// ---------------------------------------------------------------------------
+namespace fp8q {
+namespace {
+
+constexpr int64_t kNoAllocBytes = 64ll << 20;
+constexpr int64_t kNoAllocCounterBytes = 64ll << 10;
+static __device__ __align__(256) uint8_t g_noalloc_workspace[kNoAllocBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_address[64] = {nullptr};
+bool g_noalloc_cleared[64] = {false};
+
+// The array's address on the current device (looked up once per device, with that
+// device current) with its counter area cleared; nullptr on failure (message recorded).
+void* noalloc_workspace(cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) {
+    set_last_error("cudaGetDevice (static split-K workspace)",
+                   e != cudaSuccess ? e : cudaErrorInvalidDevice);
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_address[dev]) {
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, g_noalloc_workspace);
+    if (e != cudaSuccess || !addr) {
+      set_last_error("cudaGetSymbolAddress (static split-K workspace)",
+                     e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_address[dev] = addr;
+  }
+  if (!g_noalloc_cleared[dev]) {
+    e = cudaMemsetAsync(g_noalloc_address[dev], 0, kNoAllocCounterBytes, stream);
+    if (e != cudaSuccess) {
+      set_last_error("cudaMemsetAsync (static split-K workspace counters)", e);
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_cleared[dev] = true;
+  }
+  return g_noalloc_address[dev];
+}
+
+}  // namespace
+}  // namespace fp8q
+
+extern "C" fp8q_status fp8q_linear_fwd_splitk_noalloc(const uint8_t* qa, const float* sa,
+                                                      int64_t ldsa, const uint8_t* qw,
+                                                      const float* sw, int64_t M, int64_t N,
+                                                      int64_t K, uint16_t* y, int64_t ldy,
+                                                      void* stream) {
+  if (!qa || !sa || !qw || !sw || !y) return FP8Q_ERR_NULL;
+  if (M <= 0 || M > 128 || N <= 0 || K <= 0 || N % 128 || K % 128 || ldsa < M || ldy < N)
+    return FP8Q_ERR_SHAPE;
+  if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y) ||
+      ldsa % 4 || ldy % 8)
+    return FP8Q_ERR_ALIGN;
+  const int64_t counters = 4 * (N / kSplitBN);
+  const int64_t partials = N * (K / kSkBK) * M * 4;
+  if (counters > kNoAllocCounterBytes || partials > kNoAllocBytes - kNoAllocCounterBytes) {
+    char msg[200];
+    snprintf(msg, sizeof(msg),
+             "fp8q_linear_fwd_splitk_noalloc: M=%lld N=%lld K=%lld needs %lld bytes of "
+             "partials; the static workspace holds %lld",
+             static_cast<long long>(M), static_cast<long long>(N), static_cast<long long>(K),
+             static_cast<long long>(partials),
+             static_cast<long long>(kNoAllocBytes - kNoAllocCounterBytes));
+    set_last_error_text(msg);
+    return FP8Q_ERR_SHAPE;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(noalloc_workspace(st));
+  if (!ws) return FP8Q_ERR_CUDA;
+  // B = W [N][K]; block scale of (n, slice r) = sw[(n/128)*(K/128) + r]
+  return launch_skinny_gemm_splitk_into(qa, qw, M, N, K, sa, ldsa, sw, K / 128, 1, y, ldy,
+                                        reinterpret_cast<unsigned*>(ws),
+                                        reinterpret_cast<float*>(ws + kNoAllocCounterBytes), st);
+}

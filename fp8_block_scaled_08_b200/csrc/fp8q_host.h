@@ -33,6 +33,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Remembers the text of a failure for fp8q_last_error_message (thread-local).
 void set_last_error(const char* where, cudaError_t e);
+void set_last_error_text(const char* text);
 
 inline fp8q_status launch_status(const char* where = "launch") {
   cudaError_t e = cudaGetLastError();

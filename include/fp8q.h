@@ -162,6 +162,24 @@ fp8q_status fp8q_linear_fwd_splitk(const uint8_t* qa, const float* sa, int64_t l
                                    int64_t K, uint16_t* y, int64_t ldy, void* workspace,
                                    int64_t workspace_bytes, void* stream);
 
+/* fp8q_linear_fwd_splitk without a caller workspace (the paper has no counterpart: this
+ * is an interface convenience of this library). The scratch is one static device array
+ * of 64 MiB per device inside libfp8q: a fixed 64 KiB counter area (zero when the module
+ * loads, cleared once more per device before first use, left zero by every completed
+ * call) followed by the partial products. Nothing is allocated per call.
+ *   Bit for bit the same result as fp8q_linear_fwd and fp8q_linear_fwd_splitk.
+ *   FP8Q_ERR_SHAPE, with a message in fp8q_last_error_message, if the shape's partial
+ *   products (N * K/128 * M * 4 bytes) exceed the array; shapes that need no split run
+ *   fp8q_linear_fwd's kernel and do not touch it.
+ *   All calls on one device share the array: calls that overlap in time (on different
+ *   streams or host threads) race on it and give wrong results; serialise them.
+ * Requires 1 <= M <= 128, N % 128 == 0, K % 128 == 0; other arguments as
+ * fp8q_linear_fwd. */
+fp8q_status fp8q_linear_fwd_splitk_noalloc(const uint8_t* qa, const float* sa, int64_t ldsa,
+                                           const uint8_t* qw, const float* sw, int64_t M,
+                                           int64_t N, int64_t K, uint16_t* y, int64_t ldy,
+                                           void* stream);
+
 /* a7. DGrad in FP8 ("Esquema de Cuantización", backward GEMMs):
  *   dX[m,k] = sum_nb sdy[nb][m] * sw[nb][k/128] * sum_{n in nb} qdy[m,n] * qw[n,k]
  * with the row-wise dY codes of fp8q_transpose_quant_bf16 and the transposed
