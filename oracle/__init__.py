@@ -226,6 +226,27 @@ def transpose_quant_bf16(dy, lds_row: int | None = None, want_row: bool = True):
     return q_row, s_row, q_colT, s_col
 
 
+def rmsnorm_quant_dual(x, gamma, eps: float, lds_row: int | None = None):
+    """Saved activations in both groupings from BF16 (the survey's option B for the RMSNorm
+    producer): y = RMSNorm(x) * gamma rounded to BF16 as in rmsnorm_quant, then y
+    quantized 1x128 along rows (forward) and 128x1 along columns, stored transposed
+    (WGrad), plus the per-row reciprocal RMS r. Returns (q_row, s_row, q_colT, s_col, r)."""
+    x = _bf16(x)
+    q, s, y = rmsnorm_quant(x, gamma, eps, lds_row, want_y=True)
+    _, _, qT, sT = transpose_quant_bf16(y, want_row=False)
+    r = np.array([rmsnorm_rstd(row, eps) for row in x], np.float32)
+    return q, s, qT, sT, r
+
+
+def swiglu_quant_dual(gu, lds_row: int | None = None):
+    """Option B for the SwiGLU producer: h = SwiGLU(gate, up) in BF16 as in swiglu_quant,
+    then h quantized 1x128 along rows and 128x1 along columns (transposed).
+    Returns (q_row, s_row, q_colT, s_col)."""
+    q, s, h = swiglu_quant(gu, lds_row, want_h=True)
+    _, _, qT, sT = transpose_quant_bf16(h, want_row=False)
+    return q, s, qT, sT
+
+
 def transpose_quant_fp8(q, s):
     """a8: saved FP8 activation (q [M,K], s [K/128, lds]) -> 128x1 requantized,
     transposed (qT [K,M], sT [M/128, K])."""

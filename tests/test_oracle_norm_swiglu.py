@@ -108,3 +108,40 @@ def test_swiglu_layout_gate_then_up(oracle_mod):
     u = bits(gu)[0, 128 + 3]
     assert h[0, 3] == oracle_mod.swiglu_one(int(g), int(u))
     assert h[0, 3] != oracle_mod.swiglu_one(int(u), int(g)) or g == u
+
+
+def _bf16_rne_bits(v: np.ndarray) -> np.ndarray:
+    """fp32 values -> BF16 bit patterns, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return r.astype(np.uint16)
+
+
+def test_rmsnorm_dual_emission_pins(oracle_mod):
+    """Option B for the RMSNorm producer: rows are the single-output producer's codes;
+    columns (128x1 along tokens, transposed) equal the 1x128 quantization of y^T, a
+    layout identity against the separately pinned activation quantizer; and the returned
+    r regenerates y as bf16(fl32(fl32(x r) g))."""
+    x = torch.randn(256, 384, generator=torch.Generator().manual_seed(41)).to(torch.bfloat16)
+    x[:, 17] *= 40.0
+    g = (1.0 + 0.1 * torch.randn(384, generator=torch.Generator().manual_seed(42))).to(torch.bfloat16)
+    q, s, qT, sT, r = oracle_mod.rmsnorm_quant_dual(bits(x), bits(g), 1e-5)
+    q1, s1, y = oracle_mod.rmsnorm_quant(bits(x), bits(g), 1e-5, want_y=True)
+    assert np.array_equal(q, q1) and np.array_equal(s.view(np.uint32), s1.view(np.uint32))
+    qa, sa = oracle_mod.quant_act_1x128(np.ascontiguousarray(y.T))
+    assert np.array_equal(qT, qa)
+    assert np.array_equal(sT.view(np.uint32), sa[:, :384].view(np.uint32))
+    xf = f32_of_bits(bits(x)).astype(np.float32)
+    gf = f32_of_bits(bits(g)).astype(np.float32)
+    yy = _bf16_rne_bits((xf * r[:, None].astype(np.float32)).astype(np.float32) * gf)
+    assert np.array_equal(yy, y)
+
+
+def test_swiglu_dual_emission_pins(oracle_mod):
+    gu = (1.5 * torch.randn(128, 512, generator=torch.Generator().manual_seed(43))).to(torch.bfloat16)
+    q, s, qT, sT = oracle_mod.swiglu_quant_dual(bits(gu))
+    q1, s1, h = oracle_mod.swiglu_quant(bits(gu), want_h=True)
+    assert np.array_equal(q, q1) and np.array_equal(s.view(np.uint32), s1.view(np.uint32))
+    qa, sa = oracle_mod.quant_act_1x128(np.ascontiguousarray(h.T))
+    assert np.array_equal(qT, qa)
+    assert np.array_equal(sT.view(np.uint32), sa[:, :256].view(np.uint32))
