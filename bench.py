@@ -55,6 +55,11 @@ BYTES_PER_ELEM = {
     "quant_weight_128x128": 2 + 1 + 1 + 4 / 16384,  # with the transposed copy
     "transpose_quant_bf16": 2 + 2 * (1 + 4 / 128),
     "transpose_quant_fp8": (1 + 4 / 128) * 2,
+    # option B producers: read once, write both groupings (the RMSNorm variant reads x a
+    # second time for its per-row reciprocal RMS; that re-read is not algorithmic)
+    "rmsnorm_quant_dual": 2 + 2 * (1 + 4 / 128),
+    "swiglu_quant_dual": 4 + 2 * (1 + 4 / 128),   # per output element
+    "transpose_quant_bf16_act": 2 + 2 * (1 + 4 / 128),
 }
 
 
@@ -99,8 +104,9 @@ def whole_job_tflops(flops_per_rank: float, world: int, max_ms_per_step: float) 
 class LayerStep:
     """Device buffers of one layer pass and the launch sequence (all through the C ABI)."""
 
-    def __init__(self, fq, wl, device, seed_offset=0, forward_only=False):
+    def __init__(self, fq, wl, device, seed_offset=0, forward_only=False, saved="fp8"):
         self.fq = fq
+        self.saved = saved  # "fp8": requantize the saved FP8 input for WGrad; "dual": option B
         L = wl.layer
         self.M = M = wl.tokens
         self.L = L
@@ -125,6 +131,8 @@ class LayerStep:
                          q_dyT=e(N, M), s_dyc=e(M // 128, N, dt=f32))
             self.lin[lin.name] = d
         self.flops = workloads.layer_gemm_flops(L, M, passes=1 if forward_only else 3)
+        if saved == "dual":
+            self.rstd = {n: e(M, dt=f32) for n in ("qkv", "gate_up")}
         if forward_only:
             # serving: the weights are quantized once (at weight sync), not per step
             for name, d in self.lin.items():
@@ -144,6 +152,7 @@ class LayerStep:
     def run(self, timer=None, stream=None, only=None):
         fq, inp, lin, M = self.fq, self.inp, self.lin, self.M
         self.only = only
+        self.timer = timer
         k = self._k
         # weights: 128x128 quantization of the BF16 masters, with the transposed codes
         for name, d in (() if self.forward_only else lin.items()):
@@ -151,6 +160,8 @@ class LayerStep:
               lambda d=d, name=name: fq.quant_weight_128x128(inp["w"][name], d["qw"], d["sw"],
                                                              d["qwT"], stream), timer)
         q, o, gu, dn = lin["qkv"], lin["o"], lin["gate_up"], lin["down"]
+        if self.saved == "dual":
+            return self._run_dual(k, stream)
         # forward
         k("rmsnorm_quant", lambda: fq.rmsnorm_quant(inp["x_attn"], inp["gamma1"], self.eps,
                                                     q["q_in"], q["s_in"], stream), timer)
@@ -181,9 +192,46 @@ class LayerStep:
             k("gemm_wgrad", lambda d=d: fq.linear_wgrad(d["q_dyT"], d["s_dyc"], d["q_inT"],
                                                         d["s_inT"], d["dw"], stream), timer)
 
+    def _run_dual(self, k, stream):
+        """Option B: every producer emits the 1x128 codes for the forward GEMM and the
+        transposed 128x1 codes for WGrad from its BF16 output; no FP8 requantization."""
+        fq, inp, lin = self.fq, self.inp, self.lin
+        q, o, gu, dn = lin["qkv"], lin["o"], lin["gate_up"], lin["down"]
+        k("rmsnorm_quant_dual", lambda: fq.rmsnorm_quant_dual(
+            inp["x_attn"], inp["gamma1"], self.eps, q["q_in"], q["s_in"], q["q_inT"], q["s_inT"],
+            self.rstd["qkv"], stream), self.timer)
+        k("gemm_fwd", lambda: fq.linear_fwd(q["q_in"], q["s_in"], q["qw"], q["sw"], q["y"], stream),
+          self.timer)
+        k("transpose_quant_bf16_act", lambda: fq.transpose_quant_bf16(
+            inp["attn_out"], o["q_in"], o["s_in"], o["q_inT"], o["s_inT"], stream), self.timer)
+        k("gemm_fwd", lambda: fq.linear_fwd(o["q_in"], o["s_in"], o["qw"], o["sw"], o["y"], stream),
+          self.timer)
+        k("rmsnorm_quant_dual", lambda: fq.rmsnorm_quant_dual(
+            inp["x_mlp"], inp["gamma2"], self.eps, gu["q_in"], gu["s_in"], gu["q_inT"],
+            gu["s_inT"], self.rstd["gate_up"], stream), self.timer)
+        k("gemm_fwd", lambda: fq.linear_fwd(gu["q_in"], gu["s_in"], gu["qw"], gu["sw"], gu["y"],
+                                            stream), self.timer)
+        k("swiglu_quant_dual", lambda: fq.swiglu_quant_dual(
+            gu["y"], dn["q_in"], dn["s_in"], dn["q_inT"], dn["s_inT"], stream), self.timer)
+        k("gemm_fwd", lambda: fq.linear_fwd(dn["q_in"], dn["s_in"], dn["qw"], dn["sw"], dn["y"],
+                                            stream), self.timer)
+        for name in ("down", "gate_up", "o", "qkv"):
+            d = lin[name]
+            k("transpose_quant_bf16",
+              lambda d=d, name=name: fq.transpose_quant_bf16(inp["dy"][name], d["q_dy"], d["s_dy"],
+                                                             d["q_dyT"], d["s_dyc"], stream),
+              self.timer)
+            k("gemm_dgrad", lambda d=d: fq.linear_dgrad(d["q_dy"], d["s_dy"], d["qwT"], d["sw"],
+                                                        d["dx"], stream), self.timer)
+            k("gemm_wgrad", lambda d=d: fq.linear_wgrad(d["q_dyT"], d["s_dyc"], d["q_inT"],
+                                                        d["s_inT"], d["dw"], stream), self.timer)
+
     @property
     def launches_per_step(self):
-        return 8 if self.forward_only else 28
+        if self.forward_only:
+            return 8
+        # option B: no FP8 requantization (-4); each RMSNorm producer runs two kernels (+2)
+        return 26 if self.saved == "dual" else 28
 
     def gemm_flops_by_kind(self):
         M = self.M
@@ -207,6 +255,15 @@ class LayerStep:
         w_elems = sum(d["N"] * d["K"] for d in self.lin.values())
         dy_elems = sum(M * d["N"] for d in self.lin.values())
         in_elems = sum(M * d["K"] for d in self.lin.values())
+        if self.saved == "dual":
+            e = {
+                "quant_weight_128x128": w_elems,
+                "transpose_quant_bf16": dy_elems,
+                "rmsnorm_quant_dual": 2 * M * H,
+                "transpose_quant_bf16_act": M * qo,
+                "swiglu_quant_dual": M * I,
+            }
+            return {k: v * BYTES_PER_ELEM[k] for k, v in e.items()}
         e = {} if self.forward_only else {
             "quant_weight_128x128": w_elems,
             "transpose_quant_bf16": dy_elems,
@@ -638,6 +695,9 @@ def main():
     ap.add_argument("--case-reps", type=int, default=3)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=WORKLOAD.name,
                     help="layer shape (default: the Llama-3.1-8B layer at M = 8192)")
+    ap.add_argument("--saved", choices=("fp8", "dual"), default="fp8",
+                    help="saved activations for WGrad: fp8 = requantize the saved FP8 tensor "
+                         "(the pages' flow, default); dual = producers emit both groupings")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     if args.case:
@@ -663,7 +723,8 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    step = LayerStep(fq, wl, dev, seed_offset=rank_seed_offset(rank), forward_only=is_decode(wl))
+    step = LayerStep(fq, wl, dev, seed_offset=rank_seed_offset(rank), forward_only=is_decode(wl),
+                     saved=args.saved)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
         step.run()
@@ -784,6 +845,9 @@ def main():
                        "hidden": wl.layer.hidden,
                        "intermediate": wl.layer.intermediate,
                        "pass": "forward (serving)" if step.forward_only else "forward+backward",
+                       "saved_activations": ("n/a" if step.forward_only else
+                                             {"fp8": "FP8, requantized 128x1 for WGrad",
+                                              "dual": "both groupings from BF16 (option B)"}[args.saved]),
                        "gemm_tflop_per_step_per_gpu": step.flops / 1e12,
                        "launches_per_step": step.launches_per_step,
                        "l2": "inputs larger than L2: %.1f GB touched per step" % (

@@ -48,6 +48,9 @@ _SIGS = {
     "fp8q_swiglu_quant": ([_P, _I, _I, _I, _P, _P, _I, _P], ctypes.c_int),
     "fp8q_transpose_quant_bf16": ([_P, _I, _I, _I, _P, _P, _I, _P, _P, _P], ctypes.c_int),
     "fp8q_transpose_quant_fp8": ([_P, _P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
+    "fp8q_rmsnorm_quant_dual": ([_P, _P, _I, _I, _I, _F, _P, _P, _I, _P, _P, _P, _P],
+                                ctypes.c_int),
+    "fp8q_swiglu_quant_dual": ([_P, _I, _I, _I, _P, _P, _I, _P, _P, _P], ctypes.c_int),
     "fp8q_linear_fwd": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_linear_fwd_splitk_workspace": ([_I, _I, _I], ctypes.c_int64),
     "fp8q_linear_fwd_splitk_counter_bytes": ([_I, _I], ctypes.c_int64),
@@ -210,6 +213,53 @@ def transpose_quant_fp8(q, s, qT, sT, stream=None):
     M, K = q.shape
     _check(_lib.fp8q_transpose_quant_fp8(_ptr(q), _ptr(s), M, K, s.shape[1], _ptr(qT), _ptr(sT),
                                          _stream(stream)), "fp8q_transpose_quant_fp8")
+
+
+def rmsnorm_quant_dual(x, gamma, eps, q_row, s_row, q_colT, s_col, rstd, stream=None):
+    """Option B: RMSNorm(x)*gamma in BF16, emitted 1x128 (rows) and 128x1 (transposed),
+    plus the per-row reciprocal RMS."""
+    _want(x, torch.bfloat16, 2, "x"); _want(gamma, torch.bfloat16, 1, "gamma")
+    for t, n in ((q_row, "q_row"), (s_row, "s_row"), (q_colT, "q_colT"), (s_col, "s_col"),
+                 (rstd, "rstd")):
+        _dense(t, n)
+    M, H = x.shape
+    _check(_lib.fp8q_rmsnorm_quant_dual(_ptr(x), _ptr(gamma), M, H, _rows_dense(x, "x"),
+                                        float(eps), _ptr(q_row), _ptr(s_row), s_row.shape[1],
+                                        _ptr(q_colT), _ptr(s_col), _ptr(rstd), _stream(stream)),
+           "fp8q_rmsnorm_quant_dual")
+
+
+def rmsnorm_quant_dual_alloc(x, gamma, eps, stream=None):
+    M, H = x.shape
+    q = _empty((M, H), torch.uint8, x.device)
+    s = _empty((H // 128, lds_for(M)), torch.float32, x.device)
+    qT = _empty((H, M), torch.uint8, x.device)
+    sT = _empty((M // 128, H), torch.float32, x.device)
+    r = _empty((M,), torch.float32, x.device)
+    rmsnorm_quant_dual(x, gamma, eps, q, s, qT, sT, r, stream)
+    return q, s, qT, sT, r
+
+
+def swiglu_quant_dual(gu, q_row, s_row, q_colT, s_col, stream=None):
+    """Option B: SwiGLU(gate, up) in BF16, emitted 1x128 (rows) and 128x1 (transposed)."""
+    _want(gu, torch.bfloat16, 2, "gu")
+    for t, n in ((q_row, "q_row"), (s_row, "s_row"), (q_colT, "q_colT"), (s_col, "s_col")):
+        _dense(t, n)
+    M, I2 = gu.shape
+    _check(_lib.fp8q_swiglu_quant_dual(_ptr(gu), M, I2 // 2, _rows_dense(gu, "gu"), _ptr(q_row),
+                                       _ptr(s_row), s_row.shape[1], _ptr(q_colT), _ptr(s_col),
+                                       _stream(stream)), "fp8q_swiglu_quant_dual")
+
+
+def swiglu_quant_dual_alloc(gu, stream=None):
+    M, I2 = gu.shape
+    I = I2 // 2
+    q = _empty((M, I), torch.uint8, gu.device)
+    s = _empty((I // 128, lds_for(M)), torch.float32, gu.device)
+    qT = _empty((I, M), torch.uint8, gu.device)
+    sT = _empty((M // 128, I), torch.float32, gu.device)
+    swiglu_quant_dual(gu, q, s, qT, sT, stream)
+    return q, s, qT, sT
 
 
 def linear_fwd(qa, sa, qw, sw, y, stream=None):

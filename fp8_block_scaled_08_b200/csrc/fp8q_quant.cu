@@ -20,6 +20,8 @@
 // FP8 saved activations produced by the preceding operator, BF16 gradients,
 // 1x128 / 128x1 WGrad grouping) and section "Implementación" (fused
 // activation/RMSNorm and transposition kernels).
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -768,6 +770,137 @@ __global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
 
+// ---------------------------------------------------------------------------
+// Option B for saved activations (the producer emits both groupings from BF16, no FP8
+// requantization): the producer's BF16 output is formed tile by tile in shared memory
+// (thread t forms exactly the chunks its row pass quantizes, from registers), then the
+// column pass reads the staged BF16 tile as in a6.
+// ---------------------------------------------------------------------------
+
+// Per-row reciprocal RMS, r = (float)(1/sqrt(ss/H + eps)) with the fp64 sum of squares
+// of the RMSNorm kernels (eight partial sums per lane, then a warp reduction).
+__global__ void __launch_bounds__(256) rmsnorm_rstd_kernel(const uint16_t* __restrict__ x,
+                                                           int64_t M, int64_t H, int64_t ldx,
+                                                           float eps, float* __restrict__ rstd) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nch = H >> 3;
+  const int64_t wglobal = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t m = wglobal; m < M; m += nw) {
+    const uint16_t* row = x + m * ldx;
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    for (int64_t c = lane; c < nch; c += 32) {
+      float v[8];
+      unpack_bf16x8(ld_nc_v4(row + c * 8), v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const double d = static_cast<double>(v[i]);
+        acc[i] = __fma_rn(d, d, acc[i]);
+      }
+    }
+    double ss = __dadd_rn(__dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3])),
+                          __dadd_rn(__dadd_rn(acc[4], acc[5]), __dadd_rn(acc[6], acc[7])));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, off));
+    if (lane == 0) rstd[m] = rstd_from_ss(ss, H, eps);
+  }
+}
+
+// y = bf16(fl32(fl32(x r) g)) on one staged x tile, r per row, g per column.
+struct RmsDual {
+  const float* rstd;
+  const uint16_t* gamma;
+  static constexpr int kTiles = 1;
+  __device__ __forceinline__ void form(uint16_t* chunk, const uint16_t* /*second*/, int64_t m,
+                                       int64_t c, float (&v)[8]) const {
+    float xv[8], gv[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(chunk), xv);
+    unpack_bf16x8(ld_nc_v4(gamma + c), gv);
+    const float r = __ldg(rstd + m);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float a0, a1, b0, b1;
+      mul2(a0, a1, xv[i], xv[i + 1], r, r);
+      mul2(b0, b1, a0, a1, gv[i], gv[i + 1]);
+      v[i] = round_bf16(b0);
+      v[i + 1] = round_bf16(b1);
+    }
+  }
+};
+
+// h = SwiGLU(gate, up) on two staged tiles (gate columns c, up columns I + c).
+struct SwigluDual {
+  int64_t I;
+  static constexpr int kTiles = 2;
+  __device__ __forceinline__ void form(uint16_t* chunk, const uint16_t* up, int64_t /*m*/,
+                                       int64_t /*c*/, float (&v)[8]) const {
+    float g[8], u[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(chunk), g);
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(up), u);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[i], v[i + 1]);
+  }
+};
+
+// Tile t covers rows (t / NB) * 128 and output columns (t % NB) * 128; the source tile(s)
+// arrive by TMA, the formed BF16 values overwrite the first one in place.
+template <class X>
+__global__ void __launch_bounds__(256) dual_quant_kernel(
+    const __grid_constant__ CUtensorMap tmSrc, X xf, int64_t M, int64_t N,
+    uint8_t* __restrict__ q_row, float* __restrict__ s_row, int64_t lds_row,
+    uint8_t* __restrict__ q_colT, float* __restrict__ s_col, unsigned* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  constexpr uint32_t kBufBytes = X::kTiles * kTileElems * 2;
+  const TileSmem sm = carve_tiles(smem_raw, kBufBytes);
+  __shared__ int abort_flag;
+  const WaitCtl ctl{&abort_flag, err, limit_ns};
+  if (threadIdx.x == 0) abort_flag = 0;
+  const int64_t NB = N >> 7;
+  const int64_t tiles = (M >> 7) * NB;
+  const int tid = threadIdx.x;
+  const int rr = tid >> 4, c8 = (tid & 15) * 8;
+  auto issue = [&](int b, int64_t t) {
+    mbar_arrive_expect_tx(sm.bar + b, kBufBytes);
+    const int32_t col = static_cast<int32_t>((t % NB) * 128), row = static_cast<int32_t>((t / NB) * 128);
+    tma_load_2d(sm.buf[b], &tmSrc, col, row, sm.bar + b);
+    if constexpr (X::kTiles == 2)
+      tma_load_2d(sm.buf[b] + kTileElems * 2, &tmSrc, static_cast<int32_t>(xf.I) + col, row,
+                  sm.bar + b);
+  };
+  tiles_prologue(sm, tiles, issue);
+  const GroupScale unused{1.0f, 1.0f, -1.0f, false};
+  int i = 0;
+  int64_t t = blockIdx.x;
+  for (; t < tiles; t += gridDim.x, ++i) {
+    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    tiles_refill(t, tiles, i, issue);
+    uint16_t* Ts = reinterpret_cast<uint16_t*>(sm.buf[i & 1]);
+    const int64_t mb = t / NB, nb = t % NB;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {  // form this thread's chunks, quantize their rows
+      const int r = rr + 16 * j;
+      uint16_t* chunk = Ts + r * 128 + c8;
+      float v[8];
+      xf.form(chunk, chunk + kTileElems, mb * 128 + r, nb * 128 + c8, v);
+      *reinterpret_cast<uint4*>(chunk) =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]));
+      uint2 codes;
+      const float sc = quant_half_warp(v, codes);
+      const int64_t m = mb * 128 + r;
+      *reinterpret_cast<uint2*>(q_row + m * N + nb * 128 + c8) = codes;
+      if ((tid & 15) == 0) s_row[nb * lds_row + m] = sc;
+    }
+    // the formed values were written by the generic proxy into a buffer the TMA (async
+    // proxy) refills later; order them before that, and let the column pass see them
+    fence_proxy_async_smem();
+    __syncthreads();
+    tile_cols_bf16(Ts, sm.red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
+                   s_col + mb * N + nb * 128);
+  }
+  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
+}
+
 // a8: saved FP8 activation tiles (1x128 groups) -> xhat = fl32(s * dec(q)) -> 128x1
 // groups along M, stored transposed; persistent over the (M/128) x (K/128) tiles.
 // Each buffer holds the 16 KB code tile and its 128 row scales. xhat is an arbitrary
@@ -1011,4 +1144,63 @@ extern "C" fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s
                                static_cast<cudaStream_t>(stream)>>>(tmq, tms, M, K, qT, sT, err,
                                                                     kWaitLimitNs);
   return launch_status("transpose_quant_fp8 launch");
+}
+
+extern "C" fp8q_status fp8q_rmsnorm_quant_dual(const uint16_t* x, const uint16_t* gamma,
+                                               int64_t M, int64_t H, int64_t ldx, float eps,
+                                               uint8_t* q_row, float* s_row, int64_t lds_row,
+                                               uint8_t* q_colT, float* s_col, float* rstd,
+                                               void* stream) {
+  if (!x || !gamma || !q_row || !s_row || !q_colT || !s_col || !rstd) return FP8Q_ERR_NULL;
+  if (M <= 0 || H <= 0 || M % 128 || H % 128 || ldx < H || lds_row < M || lds_row % 4 ||
+      !(eps >= 0.0f))
+    return FP8Q_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(q_row) || !aligned16(s_row) ||
+      !aligned16(q_colT) || !aligned16(s_col) || !aligned16(rstd) || ldx % 8)
+    return FP8Q_ERR_ALIGN;
+  const int sms = sm100_sm_count();
+  if (!sms) return FP8Q_ERR_UNSUPPORTED;
+  CUtensorMap tm;
+  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, ldx * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the reciprocal RMS of every row first (one warp per row), then the tiles
+  const int64_t rstd_ctas = std::min<int64_t>((M + 7) / 8, static_cast<int64_t>(sms) * 8);
+  rmsnorm_rstd_kernel<<<static_cast<int>(rstd_ctas), 256, 0, st>>>(x, M, H, ldx, eps, rstd);
+  const fp8q_status s1 = launch_status("rmsnorm_rstd launch");
+  if (s1 != FP8Q_OK) return s1;
+  static int occ[64];
+  const int per_sm = resident_ctas(dual_quant_kernel<RmsDual>, 256, kTileSmemBF16, occ);
+  dual_quant_kernel<RmsDual><<<grid_for((M / 128) * (H / 128), per_sm), 256, kTileSmemBF16, st>>>(
+      tm, RmsDual{rstd, gamma}, M, H, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
+  return launch_status("rmsnorm_quant_dual launch");
+}
+
+extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int64_t I,
+                                              int64_t ldgu, uint8_t* q_row, float* s_row,
+                                              int64_t lds_row, uint8_t* q_colT, float* s_col,
+                                              void* stream) {
+  if (!gu || !q_row || !s_row || !q_colT || !s_col) return FP8Q_ERR_NULL;
+  if (M <= 0 || I <= 0 || M % 128 || I % 128 || ldgu < 2 * I || lds_row < M || lds_row % 4)
+    return FP8Q_ERR_SHAPE;
+  if (!aligned16(gu) || !aligned16(q_row) || !aligned16(s_row) || !aligned16(q_colT) ||
+      !aligned16(s_col) || ldgu % 8)
+    return FP8Q_ERR_ALIGN;
+  if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
+  CUtensorMap tm;
+  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu, 2 * I, M, ldgu * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  constexpr size_t kSmem = 1024 + 2 * (2 * kTileElems * 2) + 4 * 128 * 4 + 64;
+  static int occ[64];
+  const int per_sm = resident_ctas(dual_quant_kernel<SwigluDual>, 256, kSmem, occ);
+  dual_quant_kernel<SwigluDual><<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem,
+                                  static_cast<cudaStream_t>(stream)>>>(
+      tm, SwigluDual{I}, M, I, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
+  return launch_status("swiglu_quant_dual launch");
 }

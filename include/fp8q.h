@@ -119,6 +119,31 @@ fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, int64_t N,
                                       int64_t lds_row, uint8_t* q_colT, float* s_col,
                                       void* stream);
 
+/* Option B for the saved activations (the survey's next row f2): the producer emits both
+ * groupings from its BF16 output, so WGrad takes 128x1 codes of the BF16 values instead
+ * of re-quantizing the saved FP8 tensor (fp8q_transpose_quant_fp8).
+ * ("Esquema de Cuantización": FP8 saved activations produced by the preceding operator;
+ * "Implementación": fused RMSNorm / activation and transposition kernels.)
+ *
+ * RMSNorm producer: y = bf16(fl32(fl32(x * r) * gamma)) with r the per-row reciprocal RMS
+ * (the same values as fp8q_rmsnorm_quant), then
+ *   q_row [M][H], s_row [H/128][lds_row]: 1x128 groups along rows (forward GEMM),
+ *   q_colT [H][M], s_col [M/128][H]: 128x1 groups along tokens, transposed (WGrad),
+ *   rstd [M]: r (fp32), which the RMSNorm backward also needs.
+ * Requires M % 128 == 0, H % 128 == 0, lds_row >= M, lds_row % 4 == 0. */
+fp8q_status fp8q_rmsnorm_quant_dual(const uint16_t* x, const uint16_t* gamma, int64_t M,
+                                    int64_t H, int64_t ldx, float eps, uint8_t* q_row,
+                                    float* s_row, int64_t lds_row, uint8_t* q_colT,
+                                    float* s_col, float* rstd, void* stream);
+
+/* SwiGLU producer: h = SwiGLU(gate, up) in BF16 (the same values as fp8q_swiglu_quant),
+ * then h in both groupings as above (q_row [M][I], s_row [I/128][lds_row], q_colT [I][M],
+ * s_col [M/128][I]). gu [M][2I] = [gate | up], row stride ldgu.
+ * Requires M % 128 == 0, I % 128 == 0. */
+fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int64_t I, int64_t ldgu,
+                                   uint8_t* q_row, float* s_row, int64_t lds_row,
+                                   uint8_t* q_colT, float* s_col, void* stream);
+
 /* a8. The saved FP8 activation (1x128 groups) re-grouped 128x1 for WGrad:
  * xhat = fl32(s * dec(q)), then 128x1 quantization along M, stored transposed.
  *   q [M][K] codes, s [K/128][lds]  ->  qT [K][M] codes, sT [M/128][K].

@@ -145,3 +145,31 @@ def test_swiglu_dual_emission_pins(oracle_mod):
     qa, sa = oracle_mod.quant_act_1x128(np.ascontiguousarray(h.T))
     assert np.array_equal(qT, qa)
     assert np.array_equal(sT.view(np.uint32), sa[:, :256].view(np.uint32))
+
+
+def test_saved_activation_option_b_accuracy(oracle_mod, capsys):
+    """Saved-activation groupings for WGrad ("Resumen Técnico: Jet-RL", «Esquema de
+    Cuantización»: 1x128 in the forward pass, 128x1 for WGrad). Option A requantizes the
+    saved 1x128 codes into 128x1 groups (two roundings); option B quantizes the BF16
+    value once per grouping. On these seeded inputs B's WGrad error against the exact
+    fp64 product of the BF16 operands is not above A's; the figures are printed."""
+    import workloads
+    cases = ((512, 512, 256, 0.005, 50.0, 3000), (512, 512, 256, 0.0, 1.0, 3010))
+    for M, K, N, frac, scale, seed in cases:
+        x = workloads.activations_bf16((M, K), 0, seed, "cpu", outlier_frac=frac,
+                                       outlier_scale=scale)
+        dy = workloads.gradients_bf16((M, N), 1e-3, 0, seed + 1, "cpu")
+        xb, dyb = bits(x), bits(dy)
+        exact = dy.double().numpy().T @ x.double().numpy()
+        _, _, qdyT, sdyc = oracle_mod.transpose_quant_bf16(dyb, want_row=False)
+        qa, sa = oracle_mod.quant_act_1x128(xb)
+        qaT, saT = oracle_mod.transpose_quant_fp8(qa, sa)
+        _, _, qbT, sbT = oracle_mod.transpose_quant_bf16(xb, want_row=False)
+        ra, _ = oracle_mod.linear_wgrad(qdyT, sdyc, qaT, saT)
+        rb, _ = oracle_mod.linear_wgrad(qdyT, sdyc, qbT, sbT)
+        ea = np.linalg.norm(ra - exact) / np.linalg.norm(exact)
+        eb = np.linalg.norm(rb - exact) / np.linalg.norm(exact)
+        with capsys.disabled():
+            print(f"\n[{M}x{K}x{N} outliers {frac}] WGrad rel. error: option A {ea:.3e}, "
+                  f"option B {eb:.3e}")
+        assert 0.0 < eb <= ea < 0.1
