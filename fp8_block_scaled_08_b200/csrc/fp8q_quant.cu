@@ -538,13 +538,13 @@ __device__ __forceinline__ bool tile_acquire(const TileSmem& sm, int b, uint32_t
   return true;
 }
 
-// Codes of a column pair's 32 values (lo / hi halves of w[]), four per word.
-template <bool kMaybeSmall>
-__device__ __forceinline__ void col_codes(const uint32_t (&w)[32], const GroupScale& g0,
-                                          const GroupScale& g1, uint32_t (&o0)[8],
-                                          uint32_t (&o1)[8]) {
+// Codes of a column pair's kR values (lo / hi halves of w[]), four per word.
+template <bool kMaybeSmall, int kR>
+__device__ __forceinline__ void col_codes(const uint32_t (&w)[kR], const GroupScale& g0,
+                                          const GroupScale& g1, uint32_t (&o0)[kR / 4],
+                                          uint32_t (&o1)[kR / 4]) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < kR / 4; ++k) {
     float t0[4], t1[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -562,45 +562,54 @@ __device__ __forceinline__ void col_codes(const uint32_t (&w)[32], const GroupSc
   }
 }
 
-// Column pass over a staged BF16 tile Ts[128][128] (dense rows). Column scales:
-// computed per column (per_col) or the given block scale. Codes go to
-// dst[c * ldd + r] for tile column c and tile row r; per-column scales to scol[c].
+// Column pass over a staged BF16 tile Ts[128][128] (dense rows) by a CTA of kThreads
+// threads: thread t takes column pair t % 64 over kR = 128 / (kThreads / 64) consecutive
+// rows. Column scales: computed per column (per_col; red holds kThreads / 64 x 128
+// floats) or the given block scale. Codes go to dst[c * ldd + r] for tile column c and
+// tile row r; per-column scales to scol[c].
+template <int kThreads = 256>
 __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, bool per_col,
                                                const GroupScale& blk, uint8_t* __restrict__ dst,
                                                int64_t ldd, float* __restrict__ scol) {
+  constexpr int kQ = kThreads / 64, kR = 128 / kQ;
+  static_assert(kQ * 64 == kThreads && kR % 16 == 0, "column pass: 256 or 512 threads");
   const int tid = threadIdx.x;
   const int cp = tid & 63, rq = tid >> 6;
-  uint32_t w[32];
+  uint32_t w[kR];
 #pragma unroll
-  for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(Ts + (32 * rq + r) * 128 + 2 * cp);
+  for (int r = 0; r < kR; ++r) w[r] = *reinterpret_cast<const uint32_t*>(Ts + (kR * rq + r) * 128 + 2 * cp);
   GroupScale g0 = blk, g1 = blk;
   if (per_col) {
-    // column maxima of the 32 rows on packed pairs (four interleaved chains)
+    // column maxima of the kR rows on packed pairs (four interleaved chains)
     uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int r = 0; r < 32; ++r) m[r & 3] = bf16x2_absmax(m[r & 3], w[r]);
+    for (int r = 0; r < kR; ++r) m[r & 3] = bf16x2_absmax(m[r & 3], w[r]);
     const uint32_t mm = bf16x2_absmax(bf16x2_absmax(m[0], m[1]), bf16x2_absmax(m[2], m[3]));
     red[rq * 128 + 2 * cp] = bf16_lo(mm);
     red[rq * 128 + 2 * cp + 1] = bf16_hi(mm);
     __syncthreads();
-    const float c0 = fmaxf(fmaxf(red[2 * cp], red[128 + 2 * cp]), fmaxf(red[256 + 2 * cp], red[384 + 2 * cp]));
-    const float c1 = fmaxf(fmaxf(red[2 * cp + 1], red[128 + 2 * cp + 1]),
-                           fmaxf(red[256 + 2 * cp + 1], red[384 + 2 * cp + 1]));
+    float c0 = red[2 * cp], c1 = red[2 * cp + 1];
+#pragma unroll
+    for (int q = 1; q < kQ; ++q) {
+      c0 = fmaxf(c0, red[q * 128 + 2 * cp]);
+      c1 = fmaxf(c1, red[q * 128 + 2 * cp + 1]);
+    }
     g0 = group_scale_bf16(c0);
     g1 = group_scale_bf16(c1);
     if (rq == 0 && scol) *reinterpret_cast<float2*>(scol + 2 * cp) = make_float2(g0.s, g1.s);
   }
-  uint32_t o0[8], o1[8];
+  uint32_t o0[kR / 4], o1[kR / 4];
   if (__any_sync(kFull, g0.small || g1.small))
-    col_codes<true>(w, g0, g1, o0, o1);
+    col_codes<true, kR>(w, g0, g1, o0, o1);
   else
-    col_codes<false>(w, g0, g1, o0, o1);
-  uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * ldd + 32 * rq);
-  uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * ldd + 32 * rq);
-  d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-  d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
-  d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-  d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+    col_codes<false, kR>(w, g0, g1, o0, o1);
+  uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * ldd + kR * rq);
+  uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * ldd + kR * rq);
+#pragma unroll
+  for (int k = 0; k < kR / 16; ++k) {
+    d0[k] = make_uint4(o0[4 * k], o0[4 * k + 1], o0[4 * k + 2], o0[4 * k + 3]);
+    d1[k] = make_uint4(o1[4 * k], o1[4 * k + 1], o1[4 * k + 2], o1[4 * k + 3]);
+  }
 }
 
 // Shared memory of the BF16 tile kernels: two 32 KB tiles, the column reduction, bars.
@@ -608,14 +617,15 @@ constexpr size_t kTileSmemBF16 = 1024 + 2 * kTileElems * 2 + 4 * 128 * 4 + 64;
 // ... of the FP8 tile kernel: two (16 KB codes + 512 B row scales) buffers.
 constexpr size_t kTileSmemFP8 = 1024 + 2 * (kTileElems + 512) + 4 * 128 * 4 + 64;
 
-__device__ __forceinline__ TileSmem carve_tiles(uint8_t* raw, int buf_bytes) {
+__device__ __forceinline__ TileSmem carve_tiles(uint8_t* raw, int buf_bytes,
+                                               int red_floats = 4 * 128) {
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
   TileSmem sm;
   sm.buf[0] = base;
   sm.buf[1] = base + buf_bytes;
   sm.red = reinterpret_cast<float*>(base + 2 * buf_bytes);
-  sm.bar = reinterpret_cast<uint64_t*>(base + 2 * buf_bytes + 4 * 128 * 4);
+  sm.bar = reinterpret_cast<uint64_t*>(base + 2 * buf_bytes + red_floats * 4);
   sm.flag = reinterpret_cast<int*>(sm.bar + 2);
   return sm;
 }
@@ -789,7 +799,23 @@ __global__ void __launch_bounds__(256) rmsnorm_rstd_kernel(const uint16_t* __res
   for (int64_t m = wglobal; m < M; m += nw) {
     const uint16_t* row = x + m * ldx;
     double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-    for (int64_t c = lane; c < nch; c += 32) {
+    int64_t c = lane;
+    for (; c + 96 < nch; c += 128) {  // four 16-byte loads in flight per lane
+      uint4 raw[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) raw[u] = ld_nc_v4(row + (c + 32 * u) * 8);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float v[8];
+        unpack_bf16x8(raw[u], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const double d = static_cast<double>(v[i]);
+          acc[i] = __fma_rn(d, d, acc[i]);
+        }
+      }
+    }
+    for (; c < nch; c += 32) {
       float v[8];
       unpack_bf16x8(ld_nc_v4(row + c * 8), v);
 #pragma unroll
@@ -806,16 +832,23 @@ __global__ void __launch_bounds__(256) rmsnorm_rstd_kernel(const uint16_t* __res
   }
 }
 
-// y = bf16(fl32(fl32(x r) g)) on one staged x tile, r per row, g per column.
+// y = bf16(fl32(fl32(x r) g)) on one staged x tile, r per row, g per column. A thread's
+// chunks of a tile share their columns, so g is loaded once per tile (`Col`).
 struct RmsDual {
   const float* rstd;
   const uint16_t* gamma;
-  static constexpr int kTiles = 1;
+  static constexpr int kTiles = 1, kThreads = 256;
+  struct Col { float g[8]; };
+  __device__ __forceinline__ Col column(int64_t c) const {
+    Col k;
+    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + c)), k.g);
+    return k;
+  }
   __device__ __forceinline__ void form(uint16_t* chunk, const uint16_t* /*second*/, int64_t m,
-                                       int64_t c, float (&v)[8]) const {
-    float xv[8], gv[8];
+                                       const Col& k, float (&v)[8]) const {
+    float xv[8];
+    const float(&gv)[8] = k.g;
     unpack_bf16x8(*reinterpret_cast<const uint4*>(chunk), xv);
-    unpack_bf16x8(ld_nc_v4(gamma + c), gv);
     const float r = __ldg(rstd + m);
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
@@ -831,9 +864,12 @@ struct RmsDual {
 // h = SwiGLU(gate, up) on two staged tiles (gate columns c, up columns I + c).
 struct SwigluDual {
   int64_t I;
-  static constexpr int kTiles = 2;
+  // one 131 KB CTA per SM (two stages of a gate tile and an up tile): 16 warps
+  static constexpr int kTiles = 2, kThreads = 512;
+  struct Col {};
+  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
   __device__ __forceinline__ void form(uint16_t* chunk, const uint16_t* up, int64_t /*m*/,
-                                       int64_t /*c*/, float (&v)[8]) const {
+                                       const Col&, float (&v)[8]) const {
     float g[8], u[8];
     unpack_bf16x8(*reinterpret_cast<const uint4*>(chunk), g);
     unpack_bf16x8(*reinterpret_cast<const uint4*>(up), u);
@@ -845,13 +881,14 @@ struct SwigluDual {
 // Tile t covers rows (t / NB) * 128 and output columns (t % NB) * 128; the source tile(s)
 // arrive by TMA, the formed BF16 values overwrite the first one in place.
 template <class X>
-__global__ void __launch_bounds__(256) dual_quant_kernel(
+__global__ void __launch_bounds__(X::kThreads) dual_quant_kernel(
     const __grid_constant__ CUtensorMap tmSrc, X xf, int64_t M, int64_t N,
     uint8_t* __restrict__ q_row, float* __restrict__ s_row, int64_t lds_row,
     uint8_t* __restrict__ q_colT, float* __restrict__ s_col, unsigned* err, uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   constexpr uint32_t kBufBytes = X::kTiles * kTileElems * 2;
-  const TileSmem sm = carve_tiles(smem_raw, kBufBytes);
+  constexpr int kRowStep = X::kThreads / 16;  // tile rows formed per pass of the CTA
+  const TileSmem sm = carve_tiles(smem_raw, kBufBytes, (X::kThreads / 64) * 128);
   __shared__ int abort_flag;
   const WaitCtl ctl{&abort_flag, err, limit_ns};
   if (threadIdx.x == 0) abort_flag = 0;
@@ -876,12 +913,13 @@ __global__ void __launch_bounds__(256) dual_quant_kernel(
     tiles_refill(t, tiles, i, issue);
     uint16_t* Ts = reinterpret_cast<uint16_t*>(sm.buf[i & 1]);
     const int64_t mb = t / NB, nb = t % NB;
+    const typename X::Col col = xf.column(nb * 128 + c8);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {  // form this thread's chunks, quantize their rows
-      const int r = rr + 16 * j;
+    for (int j = 0; j < 128 / kRowStep; ++j) {  // form this thread's chunks, quantize their rows
+      const int r = rr + kRowStep * j;
       uint16_t* chunk = Ts + r * 128 + c8;
       float v[8];
-      xf.form(chunk, chunk + kTileElems, mb * 128 + r, nb * 128 + c8, v);
+      xf.form(chunk, chunk + kTileElems, mb * 128 + r, col, v);
       *reinterpret_cast<uint4*>(chunk) =
           make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                      pack_bf16x2(v[6], v[7]));
@@ -895,7 +933,7 @@ __global__ void __launch_bounds__(256) dual_quant_kernel(
     // proxy) refills later; order them before that, and let the column pass see them
     fence_proxy_async_smem();
     __syncthreads();
-    tile_cols_bf16(Ts, sm.red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
+    tile_cols_bf16<X::kThreads>(Ts, sm.red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
                    s_col + mb * N + nb * 128);
   }
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
@@ -1196,10 +1234,11 @@ extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int
     return FP8Q_ERR_UNSUPPORTED;
   unsigned* err = device_error_word();
   if (!err) return FP8Q_ERR_CUDA;
-  constexpr size_t kSmem = 1024 + 2 * (2 * kTileElems * 2) + 4 * 128 * 4 + 64;
+  constexpr int kThr = SwigluDual::kThreads;
+  constexpr size_t kSmem = 1024 + 2 * (2 * kTileElems * 2) + (kThr / 64) * 128 * 4 + 64;
   static int occ[64];
-  const int per_sm = resident_ctas(dual_quant_kernel<SwigluDual>, 256, kSmem, occ);
-  dual_quant_kernel<SwigluDual><<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem,
+  const int per_sm = resident_ctas(dual_quant_kernel<SwigluDual>, kThr, kSmem, occ);
+  dual_quant_kernel<SwigluDual><<<grid_for((M / 128) * (I / 128), per_sm), kThr, kSmem,
                                   static_cast<cudaStream_t>(stream)>>>(
       tm, SwigluDual{I}, M, I, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
   return launch_status("swiglu_quant_dual launch");
