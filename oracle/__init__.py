@@ -77,6 +77,10 @@ def _load():
     lib.oracle_swiglu_quant.argtypes = [P, I, I, I, P, P, I, P]
     lib.oracle_transpose_quant_bf16.argtypes = [P, I, I, I, P, P, I, P, P]
     lib.oracle_transpose_quant_fp8.argtypes = [P, P, I, I, I, P, P]
+    lib.oracle_swiglu_bwd_one.argtypes = [ctypes.c_uint16, ctypes.c_uint16, ctypes.c_uint16,
+                                          P, P]
+    lib.oracle_swiglu_bwd.argtypes = [P, P, I, I, P]
+    lib.oracle_rmsnorm_bwd.argtypes = [P, P, P, P, I, I, F, P, P, P, P]
     lib.oracle_dequant_rows.argtypes = [P, P, I, I, I, I, I, P]
     lib.oracle_dequant_block.argtypes = [P, P, I, I, I, I, P]
     lib.oracle_dequant_cols.argtypes = [P, P, I, I, I, I, P]
@@ -245,6 +249,62 @@ def swiglu_quant_dual(gu, lds_row: int | None = None):
     q, s, h = swiglu_quant(gu, lds_row, want_h=True)
     _, _, qT, sT = transpose_quant_bf16(h, want_row=False)
     return q, s, qT, sT
+
+
+def swiglu_bwd_one(gate_bits: int, up_bits: int, dh_bits: int) -> tuple[int, int]:
+    """Backward of one SwiGLU element: (d_gate, d_up) BF16 bits."""
+    dg, du = ctypes.c_uint16(0), ctypes.c_uint16(0)
+    _load().oracle_swiglu_bwd_one(int(gate_bits), int(up_bits), int(dh_bits),
+                                  ctypes.byref(dg), ctypes.byref(du))
+    return int(dg.value), int(du.value)
+
+
+def swiglu_bwd(gu, dh) -> np.ndarray:
+    """SwiGLU backward in BF16: gu [M, 2I] (gate | up), dh [M, I] -> dgu [M, 2I]
+    (d_gate | d_up), the rounding sequence of oracle_swiglu_bwd_one."""
+    gu, dh = _bf16(gu), _bf16(dh)
+    M, I2 = gu.shape
+    I = I2 // 2
+    assert I2 % 2 == 0 and dh.shape == (M, I)
+    dgu = np.zeros((M, I2), np.uint16)
+    _load().oracle_swiglu_bwd(_p(gu), _p(dh), M, I, _p(dgu))
+    return dgu
+
+
+def swiglu_bwd_dual(gu, dh, lds_row: int | None = None):
+    """The SwiGLU backward with the gradient quantizer a6 fused behind it: dgu (BF16)
+    quantized 1x128 along rows (DGrad of the gate/up projection) and 128x1 along columns,
+    stored transposed (its WGrad). Returns (q_row, s_row, q_colT, s_col, dgu)."""
+    dgu = swiglu_bwd(gu, dh)
+    q, s, qT, sT = transpose_quant_bf16(dgu, lds_row)
+    return q, s, qT, sT, dgu
+
+
+def rmsnorm_bwd(x, gamma, dy, dres, eps: float):
+    """RMSNorm backward in BF16 plus the residual gradient: x, dy, dres [M, H] BF16
+    (dres may be None), gamma [H]. Returns (out [M, H] BF16 bits, dgamma [H] fp32,
+    r [M] fp32, k [M] fp32) with the rounding sequence of oracle_rmsnorm_bwd."""
+    x, dy, g = _bf16(x), _bf16(dy), _bf16(gamma)
+    M, H = x.shape
+    assert dy.shape == (M, H) and g.shape == (H,)
+    dr = None if dres is None else _bf16(dres)
+    assert dr is None or dr.shape == (M, H)
+    out = np.zeros((M, H), np.uint16)
+    dgamma = np.zeros(H, np.float32)
+    r = np.zeros(M, np.float32)
+    k = np.zeros(M, np.float32)
+    _load().oracle_rmsnorm_bwd(_p(x), _p(g), _p(dy), None if dr is None else _p(dr), M, H,
+                               float(eps), _p(out), _p(dgamma), _p(r), _p(k))
+    return out, dgamma, r, k
+
+
+def rmsnorm_bwd_dual(x, gamma, dy, dres, eps: float, lds_row: int | None = None):
+    """The RMSNorm backward (+ residual gradient) with a6 fused behind it: out (BF16)
+    and its 1x128 row codes and 128x1 transposed column codes. Returns
+    (out, q_row, s_row, q_colT, s_col, dgamma)."""
+    out, dgamma, _, _ = rmsnorm_bwd(x, gamma, dy, dres, eps)
+    q, s, qT, sT = transpose_quant_bf16(out, lds_row)
+    return out, q, s, qT, sT, dgamma
 
 
 def transpose_quant_fp8(q, s):

@@ -30,6 +30,7 @@
  * OpenMP only splits independent rows/blocks; no sum changes order.
  */
 #include <math.h>
+#include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -332,6 +333,119 @@ void oracle_swiglu_quant(const uint16_t* gu, i64 M, i64 I, i64 ldgu,
       for (int i = 0; i < 128; ++i) q[m * I + g * 128 + i] = quant_one(hv[i], sc);
     }
   }
+}
+
+/* ------------------------------------------------------------------ */
+/* Backward of the SwiGLU producer, in BF16 (Jet-RL summary, "Esquema de */
+/* Cuantización": gradients between operators stay BF16). The page       */
+/* gives no formula; this is the derivative of h = silu(g) * u with      */
+/* silu(g) = g * sigma(g), sigma(g) = 1 / (1 + e^-g):                    */
+/*   dL/du = dh * silu(g),  dL/dg = dh * u * sigma(g) * (1 + g*(1 - sigma(g))).
+/* Reading (every step one IEEE fp32 operation, no contraction; the      */
+/* exponential and silu exactly as in the forward producer):             */
+/*   e = E(-g); d = fl32(1 + e); silu = fl32(g / d); sig = fl32(1 / d);   */
+/*   du = bf16(fl32(dh * silu));                                         */
+/*   ds = fl32(sig * fl32(1 + fl32(g * fl32(1 - sig))));                  */
+/*   dg = bf16(fl32(fl32(dh * u) * ds)).                                 */
+/* Layout: gu and dgu [M][2I] with gate / d_gate in columns 0..I-1 and   */
+/* up / d_up in I..2I-1; dh [M][I].                                      */
+/* ------------------------------------------------------------------ */
+void oracle_swiglu_bwd_one(uint16_t gate, uint16_t up, uint16_t dhb, uint16_t* dgate,
+                           uint16_t* dup) {
+  float g = oracle_bf16_to_f32(gate), u = oracle_bf16_to_f32(up);
+  float dh = oracle_bf16_to_f32(dhb);
+  float e = oracle_exp_cw(-g);
+  volatile float d = 1.0f + e;
+  volatile float silu = g / d;
+  volatile float sig = 1.0f / d;
+  volatile float du = dh * silu;
+  volatile float t1 = 1.0f - sig;
+  volatile float t2 = g * t1;
+  volatile float t3 = 1.0f + t2;
+  volatile float ds = sig * t3;
+  volatile float dhu = dh * u;
+  volatile float dg = dhu * ds;
+  *dgate = oracle_f32_to_bf16(dg);
+  *dup = oracle_f32_to_bf16(du);
+}
+
+void oracle_swiglu_bwd(const uint16_t* gu, const uint16_t* dh, i64 M, i64 I,
+                       uint16_t* dgu) {
+#pragma omp parallel for schedule(static)
+  for (i64 m = 0; m < M; ++m)
+    for (i64 c = 0; c < I; ++c)
+      oracle_swiglu_bwd_one(gu[m * 2 * I + c], gu[m * 2 * I + I + c], dh[m * I + c],
+                            &dgu[m * 2 * I + c], &dgu[m * 2 * I + I + c]);
+}
+
+/* ------------------------------------------------------------------ */
+/* Backward of the RMSNorm producer, in BF16, with the residual          */
+/* gradient added (the gradient that flows on along the residual        */
+/* stream). Forward: y_j = x_j * r * gamma_j, r = (mean(x^2) + eps)^-1/2. */
+/* Derivative: dx_j = r * gamma_j * dy_j - x_j * r^3 * c / H with        */
+/* c = sum_j gamma_j * dy_j * x_j; dgamma_j = sum_m dy_mj * x_mj * r_m.  */
+/* Reading (the page gives no formula; rounding as an unfused BF16       */
+/* RMSNorm backward followed by a BF16 residual add):                    */
+/*   r as in the forward producer (oracle_rmsnorm_rstd);                 */
+/*   c = sum_j fl32(fl32(gamma_j * dy_j) * x_j) in fp64 (each product is */
+/*       exact: three 8-bit significands), in index order;               */
+/*   k = (float)((((c * r) * r) * r) / H) in fp64;                        */
+/*   dx_j = bf16(fl32(fl32(r * fl32(gamma_j * dy_j)) - fl32(k * x_j)));   */
+/*   out_j = bf16(fl32(dx_j + dres_j))  (dres NULL: out_j = dx_j);        */
+/*   dgamma_j = (float) sum over m (in order) of fl32(dy_mj * fl32(x_mj * r_m)) in fp64.
+/* r_out (if not NULL) receives r per row, k_out (if not NULL) k.        */
+/* ------------------------------------------------------------------ */
+void oracle_rmsnorm_bwd(const uint16_t* x, const uint16_t* gamma, const uint16_t* dy,
+                        const uint16_t* dres, i64 M, i64 H, float eps, uint16_t* out,
+                        float* dgamma, float* r_out, float* k_out) {
+  float* rr = (float*)malloc(sizeof(float) * (size_t)M);
+#pragma omp parallel for schedule(static)
+  for (i64 m = 0; m < M; ++m) {
+    const uint16_t* xr = x + m * H;
+    const uint16_t* dyr = dy + m * H;
+    float r = oracle_rmsnorm_rstd(xr, H, eps);
+    double c = 0.0;
+    for (i64 j = 0; j < H; ++j) {
+      volatile float gd = oracle_bf16_to_f32(gamma[j]) * oracle_bf16_to_f32(dyr[j]);
+      volatile float t = gd * oracle_bf16_to_f32(xr[j]);
+      c += (double)t;
+    }
+    double kd = c * (double)r;
+    kd = kd * (double)r;
+    kd = kd * (double)r;
+    kd = kd / (double)H;
+    float k = (float)kd;
+    rr[m] = r;
+    if (r_out) r_out[m] = r;
+    if (k_out) k_out[m] = k;
+    for (i64 j = 0; j < H; ++j) {
+      float xv = oracle_bf16_to_f32(xr[j]);
+      volatile float gd = oracle_bf16_to_f32(gamma[j]) * oracle_bf16_to_f32(dyr[j]);
+      volatile float a = r * gd;
+      volatile float b = k * xv;
+      volatile float dx = a - b;
+      uint16_t dxb = oracle_f32_to_bf16(dx);
+      if (dres) {
+        volatile float o = oracle_bf16_to_f32(dxb) + oracle_bf16_to_f32(dres[m * H + j]);
+        out[m * H + j] = oracle_f32_to_bf16(o);
+      } else {
+        out[m * H + j] = dxb;
+      }
+    }
+  }
+  if (dgamma) {
+#pragma omp parallel for schedule(static)
+    for (i64 j = 0; j < H; ++j) {
+      double acc = 0.0;
+      for (i64 m = 0; m < M; ++m) {
+        volatile float xr = oracle_bf16_to_f32(x[m * H + j]) * rr[m];
+        volatile float t = oracle_bf16_to_f32(dy[m * H + j]) * xr;
+        acc += (double)t;
+      }
+      dgamma[j] = (float)acc;
+    }
+  }
+  free(rr);
 }
 
 /* ------------------------------------------------------------------ */
