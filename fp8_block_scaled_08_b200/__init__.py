@@ -51,6 +51,10 @@ _SIGS = {
     "fp8q_rmsnorm_quant_dual": ([_P, _P, _I, _I, _I, _F, _P, _P, _I, _P, _P, _P, _P],
                                 ctypes.c_int),
     "fp8q_swiglu_quant_dual": ([_P, _I, _I, _I, _P, _P, _I, _P, _P, _P], ctypes.c_int),
+    "fp8q_swiglu_bwd_quant_dual": ([_P, _P, _I, _I, _P, _P, _P, _I, _P, _P, _P], ctypes.c_int),
+    "fp8q_rmsnorm_bwd_workspace_bytes": ([_I, _I], ctypes.c_int64),
+    "fp8q_rmsnorm_bwd_quant_dual": ([_P, _P, _P, _P, _I, _I, _F, _P, _P, _P, _I, _P, _P, _P,
+                                     _P, _I, _P], ctypes.c_int),
     "fp8q_linear_fwd": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_linear_fwd_splitk_workspace": ([_I, _I, _I], ctypes.c_int64),
     "fp8q_linear_fwd_splitk_counter_bytes": ([_I, _I], ctypes.c_int64),
@@ -260,6 +264,80 @@ def swiglu_quant_dual_alloc(gu, stream=None):
     sT = _empty((M // 128, I), torch.float32, gu.device)
     swiglu_quant_dual(gu, q, s, qT, sT, stream)
     return q, s, qT, sT
+
+
+def swiglu_bwd_quant_dual(gu, dh, q_row, s_row, q_colT, s_col, dgu=None, stream=None):
+    """SwiGLU backward in BF16 (gu [M, 2I] = [gate | up], dh [M, I]) with the gradient
+    [d_gate | d_up] quantized 1x128 (rows) and 128x1 (transposed); dgu optionally receives
+    the BF16 gradient."""
+    _want(gu, torch.bfloat16, 2, "gu"); _want(dh, torch.bfloat16, 2, "dh")
+    for t, n in ((gu, "gu"), (dh, "dh"), (q_row, "q_row"), (s_row, "s_row"),
+                 (q_colT, "q_colT"), (s_col, "s_col")):
+        _dense(t, n)
+    if dgu is not None:
+        _want(dgu, torch.bfloat16, 2, "dgu"); _dense(dgu, "dgu")
+    M, I2 = gu.shape
+    if dh.shape != (M, I2 // 2):
+        raise ValueError("dh must be [M, I] for gu [M, 2I]")
+    _check(_lib.fp8q_swiglu_bwd_quant_dual(_ptr(gu), _ptr(dh), M, I2 // 2, _ptr(dgu), _ptr(q_row),
+                                           _ptr(s_row), s_row.shape[1], _ptr(q_colT),
+                                           _ptr(s_col), _stream(stream)),
+           "fp8q_swiglu_bwd_quant_dual")
+
+
+def swiglu_bwd_quant_dual_alloc(gu, dh, want_dgu=False, stream=None):
+    M, I2 = gu.shape
+    q = _empty((M, I2), torch.uint8, gu.device)
+    s = _empty((I2 // 128, lds_for(M)), torch.float32, gu.device)
+    qT = _empty((I2, M), torch.uint8, gu.device)
+    sT = _empty((M // 128, I2), torch.float32, gu.device)
+    dgu = _empty((M, I2), torch.bfloat16, gu.device) if want_dgu else None
+    swiglu_bwd_quant_dual(gu, dh, q, s, qT, sT, dgu, stream)
+    return q, s, qT, sT, dgu
+
+
+def rmsnorm_bwd_workspace_bytes(M: int, H: int) -> int:
+    return int(_lib.fp8q_rmsnorm_bwd_workspace_bytes(int(M), int(H)))
+
+
+def rmsnorm_bwd_quant_dual(x, gamma, dy, dres, eps, out, q_row, s_row, q_colT, s_col, dgamma,
+                           workspace, stream=None):
+    """RMSNorm backward in BF16 plus the residual gradient dres (may be None): out [M, H]
+    BF16, its 1x128 and 128x1 (transposed) quantizations, dgamma [H] fp32 (may be None).
+    workspace: a uint8 CUDA tensor of rmsnorm_bwd_workspace_bytes(M, H) bytes."""
+    _want(x, torch.bfloat16, 2, "x"); _want(gamma, torch.bfloat16, 1, "gamma")
+    _want(dy, torch.bfloat16, 2, "dy"); _want(out, torch.bfloat16, 2, "out")
+    if dres is not None:
+        _want(dres, torch.bfloat16, 2, "dres")
+    for t, n in ((x, "x"), (dy, "dy"), (dres, "dres"), (out, "out"), (q_row, "q_row"),
+                 (s_row, "s_row"), (q_colT, "q_colT"), (s_col, "s_col"), (dgamma, "dgamma"),
+                 (workspace, "workspace")):
+        if t is not None:
+            _dense(t, n)
+    M, H = x.shape
+    for t, n in ((dy, "dy"), (dres, "dres"), (out, "out")):
+        if t is not None and t.shape != (M, H):
+            raise ValueError("%s must have the shape of x" % n)
+    _check(_lib.fp8q_rmsnorm_bwd_quant_dual(
+        _ptr(x), _ptr(gamma), _ptr(dy), _ptr(dres), M, H, float(eps), _ptr(out), _ptr(q_row),
+        _ptr(s_row), s_row.shape[1], _ptr(q_colT), _ptr(s_col), _ptr(dgamma), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)),
+        "fp8q_rmsnorm_bwd_quant_dual")
+
+
+def rmsnorm_bwd_quant_dual_alloc(x, gamma, dy, dres, eps, stream=None):
+    M, H = x.shape
+    dev = x.device
+    out = _empty((M, H), torch.bfloat16, dev)
+    q = _empty((M, H), torch.uint8, dev)
+    s = _empty((H // 128, lds_for(M)), torch.float32, dev)
+    qT = _empty((H, M), torch.uint8, dev)
+    sT = _empty((M // 128, H), torch.float32, dev)
+    dg = _empty((H,), torch.float32, dev)
+    nbytes = rmsnorm_bwd_workspace_bytes(M, H)
+    ws = _empty((max(nbytes, 16),), torch.uint8, dev)
+    rmsnorm_bwd_quant_dual(x, gamma, dy, dres, eps, out, q, s, qT, sT, dg, ws, stream)
+    return out, q, s, qT, sT, dg
 
 
 def linear_fwd(qa, sa, qw, sw, y, stream=None):

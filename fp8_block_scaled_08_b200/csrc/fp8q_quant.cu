@@ -939,6 +939,305 @@ __global__ void __launch_bounds__(X::kThreads) dual_quant_kernel(
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
 
+// ---------------------------------------------------------------------------
+// Backward producers in BF16 with the gradient quantizer a6 fused behind them: the
+// gradient handed to the preceding linear layer is formed tile by tile in shared
+// memory and quantized both ways (1x128 rows for its DGrad, 128x1 columns, stored
+// transposed, for its WGrad) without a BF16 round trip through HBM.
+// ---------------------------------------------------------------------------
+
+// SwiGLU backward on three staged tiles (gate, up, dh): forms d_gate and d_up in place
+// of gate and up. Every step one IEEE fp32 operation, the exponential and silu as in
+// the forward producer:
+//   e = E(-g), d = 1 + e, silu = g / d, sig = 1 / d,
+//   d_up = bf16(dh silu), d_gate = bf16((dh u) (sig (1 + g (1 - sig)))).
+struct SwigluBwd {
+  static constexpr int kIn = 3, kOut = 2, kThreads = 512;
+  __device__ __forceinline__ void form(uint16_t* t0, uint16_t* t1, const uint16_t* t2,
+                                       float (&v)[2][8]) const {
+    float g[8], u[8], dh[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(t0), g);
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(t1), u);
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(t2), dh);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float e0, e1;
+      exp_cw2(-g[i], -g[i + 1], e0, e1);
+      const float d0 = __fadd_rn(1.0f, e0), d1 = __fadd_rn(1.0f, e1);
+      const float silu0 = __fdiv_rn(g[i], d0), silu1 = __fdiv_rn(g[i + 1], d1);
+      const float sig0 = __frcp_rn(d0), sig1 = __frcp_rn(d1);
+      float du0, du1, dhu0, dhu1;
+      mul2(du0, du1, dh[i], dh[i + 1], silu0, silu1);
+      mul2(dhu0, dhu1, dh[i], dh[i + 1], u[i], u[i + 1]);
+      const float t10 = __fsub_rn(1.0f, sig0), t11 = __fsub_rn(1.0f, sig1);
+      float t20, t21;
+      mul2(t20, t21, g[i], g[i + 1], t10, t11);
+      const float t30 = __fadd_rn(1.0f, t20), t31 = __fadd_rn(1.0f, t21);
+      float ds0, ds1, dg0, dg1;
+      mul2(ds0, ds1, sig0, sig1, t30, t31);
+      mul2(dg0, dg1, dhu0, dhu1, ds0, ds1);
+      v[0][i] = round_bf16(dg0);
+      v[0][i + 1] = round_bf16(dg1);
+      v[1][i] = round_bf16(du0);
+      v[1][i + 1] = round_bf16(du1);
+    }
+    *reinterpret_cast<uint4*>(t0) =
+        make_uint4(pack_bf16x2(v[0][0], v[0][1]), pack_bf16x2(v[0][2], v[0][3]),
+                   pack_bf16x2(v[0][4], v[0][5]), pack_bf16x2(v[0][6], v[0][7]));
+    *reinterpret_cast<uint4*>(t1) =
+        make_uint4(pack_bf16x2(v[1][0], v[1][1]), pack_bf16x2(v[1][2], v[1][3]),
+                   pack_bf16x2(v[1][4], v[1][5]), pack_bf16x2(v[1][6], v[1][7]));
+  }
+};
+
+// Per-row scalars of the RMSNorm backward: r (as in the forward producer) and
+// k = (float)((((c r) r) r) / H) in fp64, c = sum_j fl32(fl32(gamma_j dy_j) x_j) in fp64
+// (each product exact: three 8-bit significands). One warp per row.
+__global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma,
+    const uint16_t* __restrict__ dy, int64_t M, int64_t H, float eps, float* __restrict__ r_out,
+    float* __restrict__ k_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nch = H >> 3;
+  const int64_t wglobal = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t m = wglobal; m < M; m += nw) {
+    const uint16_t* xr = x + m * H;
+    const uint16_t* dr = dy + m * H;
+    double ss[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    double cc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    int64_t c = lane;
+    for (; c + 32 < nch; c += 64) {  // two chunks of each operand in flight per lane
+      uint4 rx[2], rd[2], rg[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        rx[u] = ld_nc_v4(xr + (c + 32 * u) * 8);
+        rd[u] = ld_nc_v4(dr + (c + 32 * u) * 8);
+        rg[u] = __ldg(reinterpret_cast<const uint4*>(gamma + (c + 32 * u) * 8));
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float xv[8], dv[8], gv[8];
+        unpack_bf16x8(rx[u], xv);
+        unpack_bf16x8(rd[u], dv);
+        unpack_bf16x8(rg[u], gv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const double xd = static_cast<double>(xv[i]);
+          ss[i] = __fma_rn(xd, xd, ss[i]);
+          const float t = __fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]);
+          cc[i] = __dadd_rn(cc[i], static_cast<double>(t));
+        }
+      }
+    }
+    for (; c < nch; c += 32) {
+      float xv[8], dv[8], gv[8];
+      unpack_bf16x8(ld_nc_v4(xr + c * 8), xv);
+      unpack_bf16x8(ld_nc_v4(dr + c * 8), dv);
+      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + c * 8)), gv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const double xd = static_cast<double>(xv[i]);
+        ss[i] = __fma_rn(xd, xd, ss[i]);
+        const float t = __fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]);
+        cc[i] = __dadd_rn(cc[i], static_cast<double>(t));
+      }
+    }
+    double s2 = __dadd_rn(__dadd_rn(__dadd_rn(ss[0], ss[1]), __dadd_rn(ss[2], ss[3])),
+                          __dadd_rn(__dadd_rn(ss[4], ss[5]), __dadd_rn(ss[6], ss[7])));
+    double c2 = __dadd_rn(__dadd_rn(__dadd_rn(cc[0], cc[1]), __dadd_rn(cc[2], cc[3])),
+                          __dadd_rn(__dadd_rn(cc[4], cc[5]), __dadd_rn(cc[6], cc[7])));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      s2 = __dadd_rn(s2, __shfl_xor_sync(kFull, s2, off));
+      c2 = __dadd_rn(c2, __shfl_xor_sync(kFull, c2, off));
+    }
+    if (lane == 0) {
+      const float r = rstd_from_ss(s2, H, eps);
+      const double rd = static_cast<double>(r);
+      double kd = __dmul_rn(c2, rd);
+      kd = __dmul_rn(kd, rd);
+      kd = __dmul_rn(kd, rd);
+      kd = __ddiv_rn(kd, static_cast<double>(H));
+      r_out[m] = r;
+      k_out[m] = __double2float_rn(kd);
+    }
+  }
+}
+
+// RMSNorm backward on staged x, dy (and dres) tiles: out = bf16(bf16(dx) + dres) with
+// dx = fl32(fl32(r fl32(gamma dy)) - fl32(k x)), formed in place of x; the terms
+// fl32(dy fl32(x r)) of dgamma are summed per column in fp64.
+struct RmsBwd {
+  const float* r;
+  const float* k;
+  const uint16_t* gamma;
+  bool has_res;
+  static constexpr int kIn = 3, kOut = 1, kThreads = 512;
+  __device__ __forceinline__ void form(uint16_t* t0, const uint16_t* t1, const uint16_t* t2,
+                                       int64_t m, const float (&gv)[8], double (&dg)[8],
+                                       float (&v)[8]) const {
+    float xv[8], dv[8], rv[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(t0), xv);
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(t1), dv);
+    if (has_res) unpack_bf16x8(*reinterpret_cast<const uint4*>(t2), rv);
+    const float rr = __ldg(r + m), kk = __ldg(k + m);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float gd0, gd1, a0, a1, b0, b1, xr0, xr1, p0, p1;
+      mul2(gd0, gd1, gv[i], gv[i + 1], dv[i], dv[i + 1]);
+      mul2(a0, a1, gd0, gd1, rr, rr);
+      mul2(b0, b1, xv[i], xv[i + 1], kk, kk);
+      float o0 = round_bf16(__fsub_rn(a0, b0)), o1 = round_bf16(__fsub_rn(a1, b1));
+      if (has_res) {
+        o0 = round_bf16(__fadd_rn(o0, rv[i]));
+        o1 = round_bf16(__fadd_rn(o1, rv[i + 1]));
+      }
+      v[i] = o0;
+      v[i + 1] = o1;
+      mul2(xr0, xr1, xv[i], xv[i + 1], rr, rr);
+      mul2(p0, p1, dv[i], dv[i + 1], xr0, xr1);
+      dg[i] = __dadd_rn(dg[i], static_cast<double>(p0));
+      dg[i + 1] = __dadd_rn(dg[i + 1], static_cast<double>(p1));
+    }
+    *reinterpret_cast<uint4*>(t0) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+};
+
+// Shared memory of the backward tile kernels: two stages of three 32 KB tiles, one
+// column reduction per output tile, the dgamma partials (RMSNorm), barriers.
+template <class X>
+constexpr size_t bwd_smem_bytes() {
+  return 1024 + 2 * (X::kIn * kTileElems * 2) + X::kOut * (X::kThreads / 64) * 128 * 4 +
+         (X::kOut == 1 ? (X::kThreads / 32) * 128 * 8 : 0) + 64;
+}
+
+// Persistent over the (M/128) x NB units. Unit t covers rows (t / NB) * 128 and input
+// column block t % NB. Output tile o of the unit is column block ob(o) of the
+// [M, Nout] gradient: nb for the RMSNorm, nb and NB + nb (d_gate, d_up) for the SwiGLU.
+// Inputs (tmA, tmB, tmC), by unit column c = 128 * (t % NB):
+//   SwiGLU:  gate = tmA at c, up = tmA at I + c, dh = tmB at c;
+//   RMSNorm: x = tmA at c, dy = tmB at c, dres = tmC at c (if present).
+// bf16_out (optional for the SwiGLU, required for the RMSNorm) receives the BF16
+// gradient [M, Nout]; dg_part (RMSNorm) the fp64 dgamma partial of each unit.
+template <class X>
+__global__ void __launch_bounds__(X::kThreads) bwd_dual_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const __grid_constant__ CUtensorMap tmC, X xf, int64_t M, int64_t NB,
+    uint16_t* __restrict__ bf16_out, uint8_t* __restrict__ q_row, float* __restrict__ s_row,
+    int64_t lds_row, uint8_t* __restrict__ q_colT, float* __restrict__ s_col,
+    const uint16_t* __restrict__ gamma, double* __restrict__ dg_part, int load_c, unsigned* err,
+    uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  constexpr int kT = X::kThreads, kQ = kT / 64, kRowStep = kT / 16;
+  constexpr uint32_t kTileBytes = kTileElems * 2;
+  constexpr uint32_t kBufBytes = X::kIn * kTileBytes;
+  const TileSmem sm = carve_tiles(smem_raw, kBufBytes, X::kOut * kQ * 128 +
+                                                           (X::kOut == 1 ? kT / 32 * 128 * 2 : 0));
+  double* dgs = reinterpret_cast<double*>(sm.red + X::kOut * kQ * 128);  // [kT/32][128]
+  __shared__ int abort_flag;
+  const WaitCtl ctl{&abort_flag, err, limit_ns};
+  if (threadIdx.x == 0) abort_flag = 0;
+  const int64_t Nout = X::kOut * NB * 128;
+  const int64_t tiles = (M >> 7) * NB;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rr = tid >> 4, c8 = (tid & 15) * 8;
+  const uint32_t in_bytes = (X::kIn - (load_c ? 0 : 1)) * kTileBytes;
+  auto issue = [&](int b, int64_t t) {
+    mbar_arrive_expect_tx(sm.bar + b, in_bytes);
+    const int32_t col = static_cast<int32_t>((t % NB) * 128), row = static_cast<int32_t>((t / NB) * 128);
+    tma_load_2d(sm.buf[b], &tmA, col, row, sm.bar + b);
+    if (X::kOut == 2) {  // SwiGLU: up from the second half of gu, dh from its own map
+      tma_load_2d(sm.buf[b] + kTileBytes, &tmA, static_cast<int32_t>(NB * 128) + col, row, sm.bar + b);
+      tma_load_2d(sm.buf[b] + 2 * kTileBytes, &tmB, col, row, sm.bar + b);
+    } else {
+      tma_load_2d(sm.buf[b] + kTileBytes, &tmB, col, row, sm.bar + b);
+      if (load_c) tma_load_2d(sm.buf[b] + 2 * kTileBytes, &tmC, col, row, sm.bar + b);
+    }
+  };
+  tiles_prologue(sm, tiles, issue);
+  const GroupScale unused{1.0f, 1.0f, -1.0f, false};
+  int i = 0;
+  int64_t t = blockIdx.x;
+  for (; t < tiles; t += gridDim.x, ++i) {
+    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
+    tiles_refill(t, tiles, i, issue);
+    uint16_t* T0 = reinterpret_cast<uint16_t*>(sm.buf[i & 1]);
+    uint16_t* T1 = T0 + kTileElems;
+    uint16_t* T2 = T1 + kTileElems;
+    const int64_t mb = t / NB, nb = t % NB;
+    float gv[8];
+    double dg[8];
+    if constexpr (X::kOut == 1) {
+      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + nb * 128 + c8)), gv);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dg[q] = 0.0;
+    }
+#pragma unroll
+    for (int j = 0; j < 128 / kRowStep; ++j) {  // form this thread's chunks, quantize their rows
+      const int r = rr + kRowStep * j;
+      const int64_t m = mb * 128 + r;
+      const int off = r * 128 + c8;
+      float v[X::kOut][8];
+      if constexpr (X::kOut == 2)
+        xf.form(T0 + off, T1 + off, T2 + off, v);
+      else
+        xf.form(T0 + off, T1 + off, T2 + off, m, gv, dg, v[0]);
+#pragma unroll
+      for (int o = 0; o < X::kOut; ++o) {
+        const int64_t ob = o * NB + nb;
+        if (bf16_out)
+          *reinterpret_cast<uint4*>(bf16_out + m * Nout + ob * 128 + c8) =
+              *reinterpret_cast<const uint4*>((o ? T1 : T0) + off);
+        uint2 codes;
+        const float sc = quant_half_warp(v[o], codes);
+        *reinterpret_cast<uint2*>(q_row + m * Nout + ob * 128 + c8) = codes;
+        if ((tid & 15) == 0) s_row[ob * lds_row + m] = sc;
+      }
+    }
+    if constexpr (X::kOut == 1) {  // dgamma: this warp's two row sets, per column
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dg[q] = __dadd_rn(dg[q], __shfl_xor_sync(kFull, dg[q], 16));
+      if (lane < 16) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dgs[warp * 128 + c8 + q] = dg[q];
+      }
+    }
+    // the formed values were written by the generic proxy into buffers the TMA refills
+    // later; order them before that, and let the column pass see them
+    fence_proxy_async_smem();
+    __syncthreads();
+    if constexpr (X::kOut == 1) {
+      if (tid < 128) {
+        double a = dgs[tid];
+#pragma unroll
+        for (int w = 1; w < kT / 32; ++w) a = __dadd_rn(a, dgs[w * 128 + tid]);
+        dg_part[mb * (NB * 128) + nb * 128 + tid] = a;
+      }
+    }
+#pragma unroll
+    for (int o = 0; o < X::kOut; ++o) {
+      const int64_t ob = o * NB + nb;
+      tile_cols_bf16<kT>(o ? T1 : T0, sm.red + o * kQ * 128, true, unused,
+                         q_colT + (ob * 128) * M + mb * 128, M, s_col + mb * Nout + ob * 128);
+    }
+  }
+  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
+}
+
+// dgamma_j = (float) sum over row blocks (in order) of the fp64 unit partials.
+__global__ void __launch_bounds__(256) dgamma_reduce_kernel(const double* __restrict__ part,
+                                                            int64_t MB, int64_t H,
+                                                            float* __restrict__ dgamma) {
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < H;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    double a = 0.0;
+    for (int64_t b = 0; b < MB; ++b) a = __dadd_rn(a, part[b * H + j]);
+    dgamma[j] = __double2float_rn(a);
+  }
+}
+
 // a8: saved FP8 activation tiles (1x128 groups) -> xhat = fl32(s * dec(q)) -> 128x1
 // groups along M, stored transposed; persistent over the (M/128) x (K/128) tiles.
 // Each buffer holds the 16 KB code tile and its 128 row scales. xhat is an arbitrary
@@ -1242,4 +1541,94 @@ extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int
                                   static_cast<cudaStream_t>(stream)>>>(
       tm, SwigluDual{I}, M, I, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
   return launch_status("swiglu_quant_dual launch");
+}
+
+extern "C" fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint16_t* dh,
+                                                  int64_t M, int64_t I, uint16_t* dgu,
+                                                  uint8_t* q_row, float* s_row, int64_t lds_row,
+                                                  uint8_t* q_colT, float* s_col, void* stream) {
+  if (!gu || !dh || !q_row || !s_row || !q_colT || !s_col) return FP8Q_ERR_NULL;
+  if (M <= 0 || I <= 0 || M % 128 || I % 128 || lds_row < M || lds_row % 4) return FP8Q_ERR_SHAPE;
+  if (!aligned16(gu) || !aligned16(dh) || (dgu && !aligned16(dgu)) || !aligned16(q_row) ||
+      !aligned16(s_row) || !aligned16(q_colT) || !aligned16(s_col))
+    return FP8Q_ERR_ALIGN;
+  if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
+  CUtensorMap tmGU, tmDH;
+  if (!encode_tmap_2d(&tmGU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu, 2 * I, M, 2 * I * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmDH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dh, I, M, I * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  constexpr size_t kSmem = bwd_smem_bytes<SwigluBwd>();
+  static int occ[64];
+  const int per_sm = resident_ctas(bwd_dual_kernel<SwigluBwd>, SwigluBwd::kThreads, kSmem, occ);
+  bwd_dual_kernel<SwigluBwd><<<grid_for((M / 128) * (I / 128), per_sm), SwigluBwd::kThreads, kSmem,
+                               static_cast<cudaStream_t>(stream)>>>(
+      tmGU, tmDH, tmDH, SwigluBwd{}, M, I / 128, dgu, q_row, s_row, lds_row, q_colT, s_col,
+      nullptr, nullptr, 1, err, kWaitLimitNs);
+  return launch_status("swiglu_bwd_quant_dual launch");
+}
+
+namespace {
+int64_t rmsnorm_bwd_ws_scalars(int64_t M) { return (8 * M + 255) / 256 * 256; }
+}  // namespace
+
+extern "C" int64_t fp8q_rmsnorm_bwd_workspace_bytes(int64_t M, int64_t H) {
+  if (M <= 0 || H <= 0 || M % 128 || H % 128) return -1;
+  return rmsnorm_bwd_ws_scalars(M) + (M / 128) * H * 8;
+}
+
+extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
+    const uint16_t* x, const uint16_t* gamma, const uint16_t* dy, const uint16_t* dres, int64_t M,
+    int64_t H, float eps, uint16_t* out, uint8_t* q_row, float* s_row, int64_t lds_row,
+    uint8_t* q_colT, float* s_col, float* dgamma, void* workspace, int64_t workspace_bytes,
+    void* stream) {
+  if (!x || !gamma || !dy || !out || !q_row || !s_row || !q_colT || !s_col || !workspace)
+    return FP8Q_ERR_NULL;
+  if (M <= 0 || H <= 0 || M % 128 || H % 128 || lds_row < M || lds_row % 4 || !(eps >= 0.0f))
+    return FP8Q_ERR_SHAPE;
+  if (workspace_bytes < fp8q_rmsnorm_bwd_workspace_bytes(M, H)) {
+    set_last_error_text("rmsnorm_bwd_quant_dual: workspace smaller than "
+                        "fp8q_rmsnorm_bwd_workspace_bytes(M, H)");
+    return FP8Q_ERR_SHAPE;
+  }
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(dy) || (dres && !aligned16(dres)) ||
+      !aligned16(out) || !aligned16(q_row) || !aligned16(s_row) || !aligned16(q_colT) ||
+      !aligned16(s_col) || (dgamma && !aligned16(dgamma)) || !aligned16(workspace))
+    return FP8Q_ERR_ALIGN;
+  const int sms = sm100_sm_count();
+  if (!sms) return FP8Q_ERR_UNSUPPORTED;
+  CUtensorMap tmX, tmDY, tmR;
+  if (!encode_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, H * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmDY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, H, M, H * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dres ? dres : dy, H, M, H * 2, 128,
+                      128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* r = reinterpret_cast<float*>(ws);
+  float* k = r + M;
+  double* part = reinterpret_cast<double*>(ws + rmsnorm_bwd_ws_scalars(M));
+  // per-row r and k first (one warp per row), then the tiles, then dgamma
+  const int64_t row_ctas = std::min<int64_t>((M + 7) / 8, static_cast<int64_t>(sms) * 8);
+  rmsnorm_bwd_rows_kernel<<<static_cast<int>(row_ctas), 256, 0, st>>>(x, gamma, dy, M, H, eps, r, k);
+  fp8q_status s1 = launch_status("rmsnorm_bwd_rows launch");
+  if (s1 != FP8Q_OK) return s1;
+  constexpr size_t kSmem = bwd_smem_bytes<RmsBwd>();
+  static int occ[64];
+  const int per_sm = resident_ctas(bwd_dual_kernel<RmsBwd>, RmsBwd::kThreads, kSmem, occ);
+  bwd_dual_kernel<RmsBwd><<<grid_for((M / 128) * (H / 128), per_sm), RmsBwd::kThreads, kSmem, st>>>(
+      tmX, tmDY, tmR, RmsBwd{r, k, gamma, dres != nullptr}, M, H / 128, out, q_row, s_row, lds_row,
+      q_colT, s_col, gamma, part, dres ? 1 : 0, err, kWaitLimitNs);
+  s1 = launch_status("rmsnorm_bwd_quant_dual launch");
+  if (s1 != FP8Q_OK || !dgamma) return s1;
+  const int64_t red_ctas = std::min<int64_t>((H + 255) / 256, static_cast<int64_t>(sms) * 4);
+  dgamma_reduce_kernel<<<static_cast<int>(red_ctas), 256, 0, st>>>(part, M / 128, H, dgamma);
+  return launch_status("dgamma_reduce launch");
 }

@@ -144,6 +144,56 @@ fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int64_t I, int
                                    uint8_t* q_row, float* s_row, int64_t lds_row,
                                    uint8_t* q_colT, float* s_col, void* stream);
 
+/* Backward producers in BF16 with the gradient quantizer fused behind them (the
+ * survey's next row f1). "Esquema de Cuantización" keeps gradients between operators
+ * in BF16 and runs DGrad / WGrad in FP8 (1x128 and 128x1 for WGrad); the page gives no
+ * formula for the operators' own backward, so these are their derivatives with the
+ * fp32 rounding sequence stated below. The gradient that the preceding linear layer
+ * consumes is quantized both ways as fp8q_transpose_quant_bf16 would quantize it:
+ *   q_row [M][Nout], s_row [Nout/128][lds_row]   1x128 groups (that layer's DGrad),
+ *   q_colT [Nout][M], s_col [M/128][Nout]        128x1 groups, transposed (its WGrad).
+ * Dense rows everywhere (row stride = columns). Requires M % 128 == 0, lds_row >= M,
+ * lds_row % 4 == 0. Enqueues its kernels on `stream`.
+ *
+ * SwiGLU backward. gu [M][2I] = [gate | up] (the forward producer's input), dh [M][I]
+ * (the gradient of h), Nout = 2I, output columns [d_gate | d_up]. Per element, each
+ * step one IEEE fp32 operation: e = E(-g) (the forward producer's exponential),
+ * d = 1 + e, silu = g / d, sig = 1 / d, d_up = bf16(dh * silu),
+ * d_gate = bf16((dh * u) * (sig * (1 + g * (1 - sig)))). dgu [M][2I] (BF16) receives
+ * the gradient itself if not NULL. Requires I % 128 == 0. */
+fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint16_t* dh, int64_t M,
+                                       int64_t I, uint16_t* dgu, uint8_t* q_row, float* s_row,
+                                       int64_t lds_row, uint8_t* q_colT, float* s_col,
+                                       void* stream);
+
+/* Bytes of device workspace fp8q_rmsnorm_bwd_quant_dual needs for (M, H): per-row
+ * scalars and one fp64 dgamma partial per 128-row block and column. -1 for a shape it
+ * does not accept. */
+int64_t fp8q_rmsnorm_bwd_workspace_bytes(int64_t M, int64_t H);
+
+/* RMSNorm backward plus the residual gradient. x [M][H] (the forward input), gamma [H],
+ * dy [M][H] (the gradient of the normalized output), dres [M][H] (the gradient arriving
+ * along the residual stream; NULL = none), Nout = H. With r the forward producer's
+ * reciprocal RMS of the row (fp64 sum of squares), c = sum_j (gamma_j dy_j) x_j in fp64
+ * (each product exact in fp32) and k = (float)((((c r) r) r) / H) in fp64:
+ *   dx_j  = bf16(fl32(fl32(r * fl32(gamma_j * dy_j)) - fl32(k * x_j))),
+ *   out_j = bf16(fl32(dx_j + dres_j))  (out_j = dx_j without dres),
+ *   dgamma_j = (float) sum over rows of fl32(dy_mj * fl32(x_mj * r_m)), summed in fp64.
+ * out [M][H] (BF16, required: the gradient continues along the residual stream) and
+ * its two quantizations; dgamma [H] fp32 if not NULL. The fp64 sums are blocked, so
+ * their last bits can differ from a sequential sum: out, k and dgamma agree with a
+ * sequential evaluation except where the exact value lies within that difference of
+ * a rounding boundary; the codes always equal the quantization of `out`.
+ * workspace: device memory of fp8q_rmsnorm_bwd_workspace_bytes(M, H) bytes, 16-byte
+ * aligned, used only during the call's kernels (calls sharing one workspace must be
+ * ordered on one stream). Requires H % 128 == 0, eps >= 0. */
+fp8q_status fp8q_rmsnorm_bwd_quant_dual(const uint16_t* x, const uint16_t* gamma,
+                                        const uint16_t* dy, const uint16_t* dres, int64_t M,
+                                        int64_t H, float eps, uint16_t* out, uint8_t* q_row,
+                                        float* s_row, int64_t lds_row, uint8_t* q_colT,
+                                        float* s_col, float* dgamma, void* workspace,
+                                        int64_t workspace_bytes, void* stream);
+
 /* a8. The saved FP8 activation (1x128 groups) re-grouped 128x1 for WGrad:
  * xhat = fl32(s * dec(q)), then 128x1 quantization along M, stored transposed.
  *   q [M][K] codes, s [K/128][lds]  ->  qT [K][M] codes, sT [M/128][K].

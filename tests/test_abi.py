@@ -136,3 +136,25 @@ def test_validation_tile_quantizers():
     assert call("fp8q_rmsnorm_quant", A, B, 4, 32768, 32768, ctypes.c_float(1e-5), C, D, 4, NUL) == 2
     assert call("fp8q_swiglu_quant", A, 4, 128, 200, B, C, 4, NUL) == 2   # ldgu < 2I
     assert call("fp8q_debug_wait_timeout", 0, NUL) == 2
+
+
+def test_validation_backward_producers():
+    W = ctypes.c_void_p(0x10000)
+    F = ctypes.c_float
+    f = "fp8q_swiglu_bwd_quant_dual"
+    assert call(f, A, B, 100, 128, NUL, C, D, 128, E, A, NUL) == 2               # M % 128
+    assert call(f, A, B, 128, 100, NUL, C, D, 128, E, A, NUL) == 2               # I % 128
+    assert call(f, A, B, 128, 128, NUL, C, D, 126, E, A, NUL) == 2               # lds_row < M
+    assert call(f, NUL, B, 128, 128, NUL, C, D, 128, E, A, NUL) == 1
+    assert call(f, A, B, 128, 128, ctypes.c_void_p(0x10008), C, D, 128, E, A, NUL) == 3
+    g = "fp8q_rmsnorm_bwd_quant_dual"
+    need = call("fp8q_rmsnorm_bwd_workspace_bytes", 256, 512)
+    assert need == 2048 + 2 * 512 * 8                                              # r, k, partials
+    assert call("fp8q_rmsnorm_bwd_workspace_bytes", 100, 512) == -1
+    ok = (A, B, C, NUL, 256, 512, F(1e-5), D, E, A, 256, B, C, NUL, W)
+    assert call(g, *ok, need - 1, NUL) == 2                                        # workspace
+    assert call(g, A, B, C, NUL, 256, 512, F(-1.0), D, E, A, 256, B, C, NUL, W, need, NUL) == 2
+    assert call(g, A, B, C, NUL, 256, 500, F(1e-5), D, E, A, 256, B, C, NUL, W, need, NUL) == 2
+    assert call(g, A, B, C, NUL, 256, 512, F(1e-5), NUL, E, A, 256, B, C, NUL, W, need, NUL) == 1
+    assert call(g, A, B, C, ctypes.c_void_p(0x10004), 256, 512, F(1e-5), D, E, A, 256, B, C, NUL,
+                W, need, NUL) == 3                                                 # dres align

@@ -1,0 +1,181 @@
+"""Backward producers with the gradient quantizer fused behind them (the survey's NEXT row
+f1) against the oracle through the C ABI: the SwiGLU backward bit for bit (gradient,
+codes, scales); the RMSNorm backward's BF16 gradient within one BF16 ulp (its fp64 sums
+are blocked on the GPU, sequential in the oracle), its codes and scales bit for bit
+against the oracle's quantization of the kernel's own gradient, dgamma within fp32
+rounding of the fp64 sum; the full-size Llama-3.1-8B shapes on sampled 128-row blocks."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from gpu_util import assert_codes_equal, assert_scales_equal, bits, np_f32
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def fq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import fp8_block_scaled_08_b200 as f
+    return f
+
+
+def _f(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _ulp_bf16(v: np.ndarray) -> np.ndarray:
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def _swiglu_inputs(M, I, seed):
+    gu = workloads.normal_bf16((M, 2 * I), 2.0, 0, seed, DEV)
+    dh = workloads.gradients_bf16((M, I), 1e-3, 0, seed + 1, DEV, small_row_frac=0.02,
+                                  small_row_scale=1e-6)
+    # saturated, vanishing and signed-zero gates, a zero gradient column
+    gu[:, 3] = 40.0
+    gu[:, 4] = -100.0
+    gu[:, 5] = 0.0
+    gu[:, 6] = -0.0
+    gu[:, I + 9] = 0.0
+    dh[:, 11] = 0.0
+    return gu, dh
+
+
+@pytest.mark.parametrize("M,I", [(128, 128), (256, 384), (384, 256), (128, 1024)])
+def test_swiglu_bwd_dual_matches_oracle(fq, oracle_mod, M, I):
+    gu, dh = _swiglu_inputs(M, I, 3000 + M + I)
+    q, s, qT, sT, dgu = fq.swiglu_bwd_quant_dual_alloc(gu, dh, want_dgu=True)
+    torch.cuda.synchronize()
+    rq, rs, rqT, rsT, rdgu = oracle_mod.swiglu_bwd_dual(bits(gu), bits(dh))
+    g = bits(dgu)
+    if not np.array_equal(g, rdgu):
+        bad = np.argwhere(g != rdgu)
+        i = tuple(bad[0])
+        raise AssertionError("dgu: %d mismatches, first at %s: gpu %#x oracle %#x" % (
+            len(bad), i, g[i], rdgu[i]))
+    assert_codes_equal(q, rq, "swiglu bwd rows")
+    assert_scales_equal(s, rs, "swiglu bwd row scales", cols=M)
+    assert_codes_equal(qT, rqT, "swiglu bwd columns")
+    assert_scales_equal(sT, rsT, "swiglu bwd column scales")
+
+
+def test_swiglu_bwd_dual_without_bf16_output(fq, oracle_mod):
+    M, I = 256, 256
+    gu, dh = _swiglu_inputs(M, I, 3100)
+    q, s, qT, sT, dgu = fq.swiglu_bwd_quant_dual_alloc(gu, dh, want_dgu=False)
+    torch.cuda.synchronize()
+    assert dgu is None
+    rq, rs, rqT, rsT, _ = oracle_mod.swiglu_bwd_dual(bits(gu), bits(dh))
+    assert_codes_equal(q, rq, "swiglu bwd rows (no dgu)")
+    assert_codes_equal(qT, rqT, "swiglu bwd columns (no dgu)")
+    assert_scales_equal(sT, rsT, "swiglu bwd column scales (no dgu)")
+
+
+def _rms_inputs(M, H, seed, with_res):
+    x = workloads.activations_bf16((M, H), 0, seed, DEV, outlier_frac=0.005, outlier_scale=50.0)
+    g = workloads.gamma_bf16(H, 0, seed + 1, DEV)
+    dy = workloads.gradients_bf16((M, H), 1e-3, 0, seed + 2, DEV, small_row_frac=0.02,
+                                  small_row_scale=1e-4)
+    dres = workloads.gradients_bf16((M, H), 1e-3, 0, seed + 3, DEV) if with_res else None
+    return x, g, dy, dres
+
+
+def _check_rms(fq, oracle_mod, x, g, dy, dres, eps, out, q, s, qT, sT, dg, what):
+    M, H = x.shape
+    rout, rdg, rr, rk = oracle_mod.rmsnorm_bwd(bits(x), bits(g), bits(dy),
+                                               None if dres is None else bits(dres), eps)
+    got, ref = _f(bits(out)), _f(rout)
+    err = np.abs(got - ref)
+    assert np.all(err <= _ulp_bf16(ref)), "%s: out beyond one BF16 ulp at %s" % (
+        what, np.argwhere(err > _ulp_bf16(ref))[:4].tolist())
+    assert np.mean(err == 0) >= 0.999, "%s: %.5f of out exact" % (what, np.mean(err == 0))
+    # the codes are the quantization of the kernel's own BF16 gradient
+    oq, os_, oqT, osT = oracle_mod.transpose_quant_bf16(bits(out))
+    assert_codes_equal(q, oq, what + " rows")
+    assert_scales_equal(s, os_, what + " row scales", cols=M)
+    assert_codes_equal(qT, oqT, what + " columns")
+    assert_scales_equal(sT, osT, what + " column scales")
+    # dgamma: fp64 sums of the same fp32 terms, in another order
+    xr = _f(bits(x)) * rr.astype(np.float64)[:, None]
+    scale = np.abs(_f(bits(dy)) * xr).sum(axis=0)
+    d = np.abs(np_f32(dg).astype(np.float64) - rdg.astype(np.float64))
+    spacing = np.spacing(np.abs(rdg)).astype(np.float64)
+    assert np.all(d <= spacing + 1e-12 * scale), what + " dgamma"
+
+
+@pytest.mark.parametrize("M,H,eps,with_res", [(128, 128, 1e-5, True), (256, 512, 1e-5, False),
+                                              (384, 640, 1e-6, True), (256, 3584, 0.0, True),
+                                              (128, 6144, 1e-5, True)])
+def test_rmsnorm_bwd_dual_matches_oracle(fq, oracle_mod, M, H, eps, with_res):
+    x, g, dy, dres = _rms_inputs(M, H, 3200 + M + H, with_res)
+    out, q, s, qT, sT, dg = fq.rmsnorm_bwd_quant_dual_alloc(x, g, dy, dres, eps)
+    torch.cuda.synchronize()
+    _check_rms(fq, oracle_mod, x, g, dy, dres, eps, out, q, s, qT, sT, dg,
+               "rmsnorm bwd %dx%d" % (M, H))
+
+
+def test_rmsnorm_bwd_dual_repeatable_and_workspace_reuse(fq):
+    """Two calls on one workspace give bit-identical results (fixed reduction order)."""
+    M, H = 256, 1024
+    x, g, dy, dres = _rms_inputs(M, H, 3300, True)
+    a = fq.rmsnorm_bwd_quant_dual_alloc(x, g, dy, dres, 1e-5)
+    b = fq.rmsnorm_bwd_quant_dual_alloc(x, g, dy, dres, 1e-5)
+    torch.cuda.synchronize()
+    for u, v in zip(a, b):
+        assert torch.equal(u.view(torch.uint8) if u.dtype != torch.uint8 else u,
+                           v.view(torch.uint8) if v.dtype != torch.uint8 else v)
+
+
+def test_rmsnorm_bwd_rejects_small_workspace(fq):
+    M, H = 128, 128
+    x, g, dy, _ = _rms_inputs(M, H, 3400, False)
+    out = torch.empty_like(x)
+    q = torch.empty((M, H), dtype=torch.uint8, device=DEV)
+    s = torch.empty((H // 128, M), dtype=torch.float32, device=DEV)
+    qT = torch.empty((H, M), dtype=torch.uint8, device=DEV)
+    sT = torch.empty((M // 128, H), dtype=torch.float32, device=DEV)
+    ws = torch.empty(fq.rmsnorm_bwd_workspace_bytes(M, H) - 16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(fq.Fp8qError):
+        fq.rmsnorm_bwd_quant_dual(x, g, dy, None, 1e-5, out, q, s, qT, sT, None, ws)
+
+
+def test_full_size_llama_backward_producers_sampled(fq, oracle_mod):
+    """Llama-3.1-8B layer at M = 8192: SwiGLU backward (I = 14336) and RMSNorm backward
+    (H = 4096, with the residual gradient) checked on one random 128-row block each;
+    dgamma over all rows against the oracle's full sum."""
+    wl = workloads.LLAMA_LAYER
+    M, H, I = wl.tokens, wl.layer.hidden, wl.layer.intermediate
+    rng = np.random.default_rng(7)
+    gu, dh = _swiglu_inputs(M, I, 3500)
+    q, s, qT, sT, dgu = fq.swiglu_bwd_quant_dual_alloc(gu, dh, want_dgu=True)
+    torch.cuda.synchronize()
+    mb = int(rng.integers(0, M // 128))
+    blk = slice(mb * 128, mb * 128 + 128)
+    rq, rs, rqT, rsT, rdgu = oracle_mod.swiglu_bwd_dual(bits(gu[blk]), bits(dh[blk]))
+    assert np.array_equal(bits(dgu[blk]), rdgu)
+    assert_codes_equal(q[blk], rq, "full swiglu bwd rows")
+    assert_codes_equal(qT[:, blk], rqT, "full swiglu bwd columns")
+    assert np.array_equal(np_f32(sT[mb:mb + 1]).view(np.uint32), rsT.view(np.uint32))
+    del gu, dh, q, s, qT, sT, dgu
+    x, g, dy, dres = _rms_inputs(M, H, 3600, True)
+    out, q, s, qT, sT, dg = fq.rmsnorm_bwd_quant_dual_alloc(x, g, dy, dres, wl.eps)
+    torch.cuda.synchronize()
+    mb = int(rng.integers(0, M // 128))
+    blk = slice(mb * 128, mb * 128 + 128)
+    rout, _, _, _ = oracle_mod.rmsnorm_bwd(bits(x[blk]), bits(g), bits(dy[blk]), bits(dres[blk]),
+                                           wl.eps)
+    err = np.abs(_f(bits(out[blk])) - _f(rout))
+    assert np.all(err <= _ulp_bf16(_f(rout)))
+    oq, _, oqT, osT = oracle_mod.transpose_quant_bf16(bits(out[blk]))
+    assert_codes_equal(q[blk], oq, "full rmsnorm bwd rows")
+    assert_codes_equal(qT[:, blk], oqT, "full rmsnorm bwd columns")
+    assert np.array_equal(np_f32(sT[mb:mb + 1]).view(np.uint32), osT.view(np.uint32))
+    _, rdg, _, _ = oracle_mod.rmsnorm_bwd(bits(x), bits(g), bits(dy), None, wl.eps)
+    d = np.abs(np_f32(dg).astype(np.float64) - rdg.astype(np.float64))
+    assert np.all(d <= 2 * np.spacing(np.abs(rdg)).astype(np.float64) + 1e-12)
