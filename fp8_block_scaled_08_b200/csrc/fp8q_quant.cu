@@ -733,58 +733,11 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
 
-// a6: BF16 dY tiles -> row-wise 1x128 codes (row pass) + column-wise 128x1 codes
-// (column pass, transposed), persistent over the (M/128) x (N/128) tiles.
-__global__ void __launch_bounds__(256) transpose_quant_bf16_kernel(
-    const __grid_constant__ CUtensorMap tmDY, int64_t M, int64_t N, uint8_t* __restrict__ q_row,
-    float* __restrict__ s_row, int64_t lds_row, uint8_t* __restrict__ q_colT,
-    float* __restrict__ s_col, unsigned* err, uint64_t limit_ns) {
-  extern __shared__ uint8_t smem_raw[];
-  const TileSmem sm = carve_tiles(smem_raw, kTileElems * 2);
-  __shared__ int abort_flag;
-  const WaitCtl ctl{&abort_flag, err, limit_ns};
-  if (threadIdx.x == 0) abort_flag = 0;
-  const int64_t NB = N >> 7;
-  const int64_t tiles = (M >> 7) * NB;
-  const int tid = threadIdx.x;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  auto issue = [&](int b, int64_t t) {
-    mbar_arrive_expect_tx(sm.bar + b, kTileElems * 2);
-    tma_load_2d(sm.buf[b], &tmDY, static_cast<int32_t>((t % NB) * 128),
-                static_cast<int32_t>((t / NB) * 128), sm.bar + b);
-  };
-  tiles_prologue(sm, tiles, issue);
-  const GroupScale unused{1.0f, 1.0f, -1.0f, false};
-  int i = 0;
-  int64_t t = blockIdx.x;
-  for (; t < tiles; t += gridDim.x, ++i) {
-    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
-    tiles_refill(t, tiles, i, issue);
-    const uint16_t* Ts = reinterpret_cast<const uint16_t*>(sm.buf[i & 1]);
-    const int64_t mb = t / NB, nb = t % NB;
-    if (q_row) {  // each tile row is one 1x128 group, held by a half-warp
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float v[8];
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(Ts + (rr + 16 * j) * 128 + c8), v);
-        uint2 codes;
-        const float sc = quant_half_warp(v, codes);
-        const int64_t m = mb * 128 + rr + 16 * j;
-        *reinterpret_cast<uint2*>(q_row + m * N + nb * 128 + c8) = codes;
-        if ((tid & 15) == 0) s_row[nb * lds_row + m] = sc;
-      }
-    }
-    tile_cols_bf16(Ts, sm.red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
-                   s_col + mb * N + nb * 128);
-  }
-  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
-}
-
 // ---------------------------------------------------------------------------
 // Option B for saved activations (the producer emits both groupings from BF16, no FP8
-// requantization): the producer's BF16 output is formed tile by tile in shared memory
-// (thread t forms exactly the chunks its row pass quantizes, from registers), then the
-// column pass reads the staged BF16 tile as in a6.
+// requantization): the producer's BF16 output is formed 128 x 128 tile by tile by
+// direct_dual_kernel below, with RmsDirect / SwigluDirect as the source; the RMSNorm
+// needs its per-row reciprocal RMS first.
 // ---------------------------------------------------------------------------
 
 // Per-row reciprocal RMS, r = (float)(1/sqrt(ss/H + eps)) with the fp64 sum of squares
@@ -832,133 +785,38 @@ __global__ void __launch_bounds__(256) rmsnorm_rstd_kernel(const uint16_t* __res
   }
 }
 
-// y = bf16(fl32(fl32(x r) g)) on one staged x tile, r per row, g per column. A thread's
-// chunks of a tile share their columns, so g is loaded once per tile (`Col`).
-struct RmsDual {
-  const float* rstd;
-  const uint16_t* gamma;
-  static constexpr int kTiles = 1, kThreads = 256;
-  struct Col { float g[8]; };
-  __device__ __forceinline__ Col column(int64_t c) const {
-    Col k;
-    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + c)), k.g);
-    return k;
-  }
-  __device__ __forceinline__ void form(uint16_t* chunk, const uint16_t* /*second*/, int64_t m,
-                                       const Col& k, float (&v)[8]) const {
-    float xv[8];
-    const float(&gv)[8] = k.g;
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(chunk), xv);
-    const float r = __ldg(rstd + m);
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      float a0, a1, b0, b1;
-      mul2(a0, a1, xv[i], xv[i + 1], r, r);
-      mul2(b0, b1, a0, a1, gv[i], gv[i + 1]);
-      v[i] = round_bf16(b0);
-      v[i + 1] = round_bf16(b1);
-    }
-  }
-};
-
-// h = SwiGLU(gate, up) on two staged tiles (gate columns c, up columns I + c).
-struct SwigluDual {
-  int64_t I;
-  // one 131 KB CTA per SM (two stages of a gate tile and an up tile): 16 warps
-  static constexpr int kTiles = 2, kThreads = 512;
-  struct Col {};
-  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
-  __device__ __forceinline__ void form(uint16_t* chunk, const uint16_t* up, int64_t /*m*/,
-                                       const Col&, float (&v)[8]) const {
-    float g[8], u[8];
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(chunk), g);
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(up), u);
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[i], v[i + 1]);
-  }
-};
-
-// Tile t covers rows (t / NB) * 128 and output columns (t % NB) * 128; the source tile(s)
-// arrive by TMA, the formed BF16 values overwrite the first one in place.
-template <class X>
-__global__ void __launch_bounds__(X::kThreads) dual_quant_kernel(
-    const __grid_constant__ CUtensorMap tmSrc, X xf, int64_t M, int64_t N,
-    uint8_t* __restrict__ q_row, float* __restrict__ s_row, int64_t lds_row,
-    uint8_t* __restrict__ q_colT, float* __restrict__ s_col, unsigned* err, uint64_t limit_ns) {
-  extern __shared__ uint8_t smem_raw[];
-  constexpr uint32_t kBufBytes = X::kTiles * kTileElems * 2;
-  constexpr int kRowStep = X::kThreads / 16;  // tile rows formed per pass of the CTA
-  const TileSmem sm = carve_tiles(smem_raw, kBufBytes, (X::kThreads / 64) * 128);
-  __shared__ int abort_flag;
-  const WaitCtl ctl{&abort_flag, err, limit_ns};
-  if (threadIdx.x == 0) abort_flag = 0;
-  const int64_t NB = N >> 7;
-  const int64_t tiles = (M >> 7) * NB;
-  const int tid = threadIdx.x;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  auto issue = [&](int b, int64_t t) {
-    mbar_arrive_expect_tx(sm.bar + b, kBufBytes);
-    const int32_t col = static_cast<int32_t>((t % NB) * 128), row = static_cast<int32_t>((t / NB) * 128);
-    tma_load_2d(sm.buf[b], &tmSrc, col, row, sm.bar + b);
-    if constexpr (X::kTiles == 2)
-      tma_load_2d(sm.buf[b] + kTileElems * 2, &tmSrc, static_cast<int32_t>(xf.I) + col, row,
-                  sm.bar + b);
-  };
-  tiles_prologue(sm, tiles, issue);
-  const GroupScale unused{1.0f, 1.0f, -1.0f, false};
-  int i = 0;
-  int64_t t = blockIdx.x;
-  for (; t < tiles; t += gridDim.x, ++i) {
-    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
-    tiles_refill(t, tiles, i, issue);
-    uint16_t* Ts = reinterpret_cast<uint16_t*>(sm.buf[i & 1]);
-    const int64_t mb = t / NB, nb = t % NB;
-    const typename X::Col col = xf.column(nb * 128 + c8);
-#pragma unroll
-    for (int j = 0; j < 128 / kRowStep; ++j) {  // form this thread's chunks, quantize their rows
-      const int r = rr + kRowStep * j;
-      uint16_t* chunk = Ts + r * 128 + c8;
-      float v[8];
-      xf.form(chunk, chunk + kTileElems, mb * 128 + r, col, v);
-      *reinterpret_cast<uint4*>(chunk) =
-          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                     pack_bf16x2(v[6], v[7]));
-      uint2 codes;
-      const float sc = quant_half_warp(v, codes);
-      const int64_t m = mb * 128 + r;
-      *reinterpret_cast<uint2*>(q_row + m * N + nb * 128 + c8) = codes;
-      if ((tid & 15) == 0) s_row[nb * lds_row + m] = sc;
-    }
-    // the formed values were written by the generic proxy into a buffer the TMA (async
-    // proxy) refills later; order them before that, and let the column pass see them
-    fence_proxy_async_smem();
-    __syncthreads();
-    tile_cols_bf16<X::kThreads>(Ts, sm.red, true, unused, q_colT + (nb * 128) * M + mb * 128, M,
-                   s_col + mb * N + nb * 128);
-  }
-  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
-}
-
 // ---------------------------------------------------------------------------
-// Backward producers in BF16 with the gradient quantizer a6 fused behind them: the
-// gradient handed to the preceding linear layer is formed tile by tile in shared
-// memory and quantized both ways (1x128 rows for its DGrad, 128x1 columns, stored
-// transposed, for its WGrad) without a BF16 round trip through HBM.
+// Tensors quantized both ways from a BF16 value formed on the fly (1x128 rows, and
+// 128x1 columns stored transposed), one 128 x 128 unit at a time: a6 itself (the value
+// is the input), the option-B forward producers, and the backward producers in BF16
+// with a6 fused behind them (the gradient handed to the preceding linear layer never
+// makes a BF16 round trip through HBM).
 // ---------------------------------------------------------------------------
 
-// SwiGLU backward on three staged tiles (gate, up, dh): forms d_gate and d_up in place
-// of gate and up. Every step one IEEE fp32 operation, the exponential and silu as in
-// the forward producer:
+// SwiGLU backward per element, every step one IEEE fp32 operation (the exponential and
+// silu as in the forward producer):
 //   e = E(-g), d = 1 + e, silu = g / d, sig = 1 / d,
 //   d_up = bf16(dh silu), d_gate = bf16((dh u) (sig (1 + g (1 - sig)))).
+// A thread's chunk: 8 consecutive gate, up and dh values of one row.
 struct SwigluBwd {
-  static constexpr int kIn = 3, kOut = 2, kThreads = 512;
-  __device__ __forceinline__ void form(uint16_t* t0, uint16_t* t1, const uint16_t* t2,
+  const uint16_t* gu;
+  const uint16_t* dh;
+  int64_t I;
+  static constexpr int kOut = 2;
+  static constexpr bool kDgamma = false;
+  struct In { uint4 g, u, d; };
+  struct Col {};
+  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
+  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
+    const uint16_t* row = gu + m * 2 * I;
+    return In{ld_nc_v4(row + col), ld_nc_v4(row + I + col), ld_nc_v4(dh + m * I + col)};
+  }
+  __device__ __forceinline__ void form(const In& in, int64_t /*m*/, const Col&, double (&)[8],
                                        float (&v)[2][8]) const {
     float g[8], u[8], dh[8];
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(t0), g);
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(t1), u);
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(t2), dh);
+    unpack_bf16x8(in.g, g);
+    unpack_bf16x8(in.u, u);
+    unpack_bf16x8(in.d, dh);
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       float e0, e1;
@@ -981,12 +839,6 @@ struct SwigluBwd {
       v[1][i] = round_bf16(du0);
       v[1][i + 1] = round_bf16(du1);
     }
-    *reinterpret_cast<uint4*>(t0) =
-        make_uint4(pack_bf16x2(v[0][0], v[0][1]), pack_bf16x2(v[0][2], v[0][3]),
-                   pack_bf16x2(v[0][4], v[0][5]), pack_bf16x2(v[0][6], v[0][7]));
-    *reinterpret_cast<uint4*>(t1) =
-        make_uint4(pack_bf16x2(v[1][0], v[1][1]), pack_bf16x2(v[1][2], v[1][3]),
-                   pack_bf16x2(v[1][4], v[1][5]), pack_bf16x2(v[1][6], v[1][7]));
   }
 };
 
@@ -1065,23 +917,43 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
   }
 }
 
-// RMSNorm backward on staged x, dy (and dres) tiles: out = bf16(bf16(dx) + dres) with
-// dx = fl32(fl32(r fl32(gamma dy)) - fl32(k x)), formed in place of x; the terms
-// fl32(dy fl32(x r)) of dgamma are summed per column in fp64.
+// RMSNorm backward per element: out = bf16(bf16(dx) + dres) with
+// dx = fl32(fl32(r fl32(gamma dy)) - fl32(k x)); the terms fl32(dy fl32(x r)) of dgamma
+// are summed per column in fp64. A thread's chunk: 8 consecutive x, dy (and dres)
+// values of one row.
 struct RmsBwd {
+  const uint16_t* x;
+  const uint16_t* dy;
+  const uint16_t* dres;  // may be NULL
   const float* r;
   const float* k;
   const uint16_t* gamma;
-  bool has_res;
-  static constexpr int kIn = 3, kOut = 1, kThreads = 512;
-  __device__ __forceinline__ void form(uint16_t* t0, const uint16_t* t1, const uint16_t* t2,
-                                       int64_t m, const float (&gv)[8], double (&dg)[8],
-                                       float (&v)[8]) const {
+  int64_t H;
+  static constexpr int kOut = 1;
+  static constexpr bool kDgamma = true;
+  struct In { uint4 x, d, res; };
+  struct Col { float g[8]; };
+  __device__ __forceinline__ Col column(int64_t c) const {
+    Col k;
+    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + c)), k.g);
+    return k;
+  }
+  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
+    In in;
+    in.x = ld_nc_v4(x + m * H + col);
+    in.d = ld_nc_v4(dy + m * H + col);
+    in.res = dres ? ld_nc_v4(dres + m * H + col) : make_uint4(0u, 0u, 0u, 0u);
+    return in;
+  }
+  __device__ __forceinline__ void form(const In& in, int64_t m, const Col& col, double (&dg)[8],
+                                       float (&v)[1][8]) const {
+    const float(&gv)[8] = col.g;
     float xv[8], dv[8], rv[8];
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(t0), xv);
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(t1), dv);
-    if (has_res) unpack_bf16x8(*reinterpret_cast<const uint4*>(t2), rv);
+    unpack_bf16x8(in.x, xv);
+    unpack_bf16x8(in.d, dv);
+    unpack_bf16x8(in.res, rv);
     const float rr = __ldg(r + m), kk = __ldg(k + m);
+    const bool res = dres != nullptr;
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       float gd0, gd1, a0, a1, b0, b1, xr0, xr1, p0, p1;
@@ -1089,114 +961,170 @@ struct RmsBwd {
       mul2(a0, a1, gd0, gd1, rr, rr);
       mul2(b0, b1, xv[i], xv[i + 1], kk, kk);
       float o0 = round_bf16(__fsub_rn(a0, b0)), o1 = round_bf16(__fsub_rn(a1, b1));
-      if (has_res) {
+      if (res) {
         o0 = round_bf16(__fadd_rn(o0, rv[i]));
         o1 = round_bf16(__fadd_rn(o1, rv[i + 1]));
       }
-      v[i] = o0;
-      v[i + 1] = o1;
+      v[0][i] = o0;
+      v[0][i + 1] = o1;
       mul2(xr0, xr1, xv[i], xv[i + 1], rr, rr);
       mul2(p0, p1, dv[i], dv[i + 1], xr0, xr1);
       dg[i] = __dadd_rn(dg[i], static_cast<double>(p0));
       dg[i + 1] = __dadd_rn(dg[i + 1], static_cast<double>(p1));
     }
-    *reinterpret_cast<uint4*>(t0) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
 };
 
-// Shared memory of the backward tile kernels: two stages of three 32 KB tiles, one
-// column reduction per output tile, the dgamma partials (RMSNorm), barriers.
+// a6 through the direct kernel: the BF16 values themselves.
+struct GradDirect {
+  const uint16_t* dy;
+  int64_t ld;
+  static constexpr int kOut = 1;
+  static constexpr bool kDgamma = false;
+  struct In { uint4 a; };
+  struct Col {};
+  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
+  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
+    return In{ld_nc_v4(dy + m * ld + col)};
+  }
+  __device__ __forceinline__ void form(const In& in, int64_t, const Col&, double (&)[8],
+                                       float (&v)[1][8]) const {
+    unpack_bf16x8(in.a, v[0]);
+  }
+};
+
+// Option B RMSNorm producer: y = bf16(fl32(fl32(x r) gamma)), r per row from the pre-pass.
+struct RmsDirect {
+  const uint16_t* x;
+  int64_t ldx;
+  const float* rstd;
+  const uint16_t* gamma;
+  static constexpr int kOut = 1;
+  static constexpr bool kDgamma = false;
+  struct In { uint4 a; };
+  struct Col { float g[8]; };
+  __device__ __forceinline__ Col column(int64_t c) const {
+    Col k;
+    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + c)), k.g);
+    return k;
+  }
+  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
+    return In{ld_nc_v4(x + m * ldx + col)};
+  }
+  __device__ __forceinline__ void form(const In& in, int64_t m, const Col& k, double (&)[8],
+                                       float (&v)[1][8]) const {
+    float xv[8];
+    unpack_bf16x8(in.a, xv);
+    const float r = __ldg(rstd + m);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float a0, a1, b0, b1;
+      mul2(a0, a1, xv[i], xv[i + 1], r, r);
+      mul2(b0, b1, a0, a1, k.g[i], k.g[i + 1]);
+      v[0][i] = round_bf16(b0);
+      v[0][i + 1] = round_bf16(b1);
+    }
+  }
+};
+
+// Option B SwiGLU producer: h = SwiGLU(gate, up) in BF16 (gate columns c, up I + c).
+struct SwigluDirect {
+  const uint16_t* gu;
+  int64_t ldgu, I;
+  static constexpr int kOut = 1;
+  static constexpr bool kDgamma = false;
+  struct In { uint4 g, u; };
+  struct Col {};
+  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
+  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
+    const uint16_t* row = gu + m * ldgu;
+    return In{ld_nc_v4(row + col), ld_nc_v4(row + I + col)};
+  }
+  __device__ __forceinline__ void form(const In& in, int64_t, const Col&, double (&)[8],
+                                       float (&v)[1][8]) const {
+    float g[8], u[8];
+    unpack_bf16x8(in.g, g);
+    unpack_bf16x8(in.u, u);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[0][i], v[0][i + 1]);
+  }
+};
+
+// Rows loaded per batch and the occupancy the backward kernels are compiled for.
+constexpr int kBwdBatch = 2;
+constexpr int kBwdMinBlocks = 3;
+constexpr int kFwdBatch = 4;
+constexpr int kFwdMinBlocks = 4;
+constexpr int kA6Batch = 4;
+constexpr int kA6MinBlocks = 4;
+
+// Shared memory of the backward kernels: the formed BF16 output tile(s), one column
+// reduction per output tile, the dgamma partials of the 8 warps (RMSNorm).
 template <class X>
-constexpr size_t bwd_smem_bytes() {
-  return 1024 + 2 * (X::kIn * kTileElems * 2) + X::kOut * (X::kThreads / 64) * 128 * 4 +
-         (X::kOut == 1 ? (X::kThreads / 32) * 128 * 8 : 0) + 64;
+constexpr size_t direct_smem_bytes() {
+  return X::kOut * (kTileElems * 2 + 4 * 128 * 4) + (X::kDgamma ? 8 * 128 * 8 : 0);
 }
 
-// Persistent over the (M/128) x NB units. Unit t covers rows (t / NB) * 128 and input
-// column block t % NB. Output tile o of the unit is column block ob(o) of the
-// [M, Nout] gradient: nb for the RMSNorm, nb and NB + nb (d_gate, d_up) for the SwiGLU.
-// Inputs (tmA, tmB, tmC), by unit column c = 128 * (t % NB):
-//   SwiGLU:  gate = tmA at c, up = tmA at I + c, dh = tmB at c;
-//   RMSNorm: x = tmA at c, dy = tmB at c, dres = tmC at c (if present).
-// bf16_out (optional for the SwiGLU, required for the RMSNorm) receives the BF16
-// gradient [M, Nout]; dg_part (RMSNorm) the fp64 dgamma partial of each unit.
-template <class X>
-__global__ void __launch_bounds__(X::kThreads) bwd_dual_kernel(
-    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-    const __grid_constant__ CUtensorMap tmC, X xf, int64_t M, int64_t NB,
-    uint16_t* __restrict__ bf16_out, uint8_t* __restrict__ q_row, float* __restrict__ s_row,
-    int64_t lds_row, uint8_t* __restrict__ q_colT, float* __restrict__ s_col,
-    const uint16_t* __restrict__ gamma, double* __restrict__ dg_part, int load_c, unsigned* err,
-    uint64_t limit_ns) {
-  extern __shared__ uint8_t smem_raw[];
-  constexpr int kT = X::kThreads, kQ = kT / 64, kRowStep = kT / 16;
-  constexpr uint32_t kTileBytes = kTileElems * 2;
-  constexpr uint32_t kBufBytes = X::kIn * kTileBytes;
-  const TileSmem sm = carve_tiles(smem_raw, kBufBytes, X::kOut * kQ * 128 +
-                                                           (X::kOut == 1 ? kT / 32 * 128 * 2 : 0));
-  double* dgs = reinterpret_cast<double*>(sm.red + X::kOut * kQ * 128);  // [kT/32][128]
-  __shared__ int abort_flag;
-  const WaitCtl ctl{&abort_flag, err, limit_ns};
-  if (threadIdx.x == 0) abort_flag = 0;
-  const int64_t Nout = X::kOut * NB * 128;
+// Persistent over the (M/128) x NB units; unit t covers rows (t / NB) * 128 and input
+// columns (t % NB) * 128. Each thread loads its chunks (rows rr + 16 j, columns c8..c8+7)
+// straight into registers, kBatch rows at a time, forms the gradient, stores it in the
+// output tile(s) in shared memory (and in bf16_out if given) and quantizes its rows;
+// after one barrier the column pass runs on the staged tile(s). Output tile o is column
+// block o * NB + nb of the [M, Nout] gradient (Nout = kOut * NB * 128): for the SwiGLU
+// d_gate and d_up, for the RMSNorm the gradient itself. dg_part (RMSNorm) receives the
+// fp64 dgamma partial of each unit.
+template <class X, int kBatch, int kMinBlocks>
+__global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
+    X xf, int64_t M, int64_t NB, uint16_t* __restrict__ bf16_out, uint8_t* __restrict__ q_row,
+    float* __restrict__ s_row, int64_t lds_row, uint8_t* __restrict__ q_colT,
+    float* __restrict__ s_col, double* __restrict__ dg_part) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  constexpr int kOut = X::kOut;
+  uint16_t* tile = reinterpret_cast<uint16_t*>(smem_raw);
+  float* red = reinterpret_cast<float*>(smem_raw + kOut * kTileElems * 2);
+  double* dgs = reinterpret_cast<double*>(red + kOut * 4 * 128);  // [8 warps][128]
+  const int64_t Nout = kOut * NB * 128;
   const int64_t tiles = (M >> 7) * NB;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  const uint32_t in_bytes = (X::kIn - (load_c ? 0 : 1)) * kTileBytes;
-  auto issue = [&](int b, int64_t t) {
-    mbar_arrive_expect_tx(sm.bar + b, in_bytes);
-    const int32_t col = static_cast<int32_t>((t % NB) * 128), row = static_cast<int32_t>((t / NB) * 128);
-    tma_load_2d(sm.buf[b], &tmA, col, row, sm.bar + b);
-    if (X::kOut == 2) {  // SwiGLU: up from the second half of gu, dh from its own map
-      tma_load_2d(sm.buf[b] + kTileBytes, &tmA, static_cast<int32_t>(NB * 128) + col, row, sm.bar + b);
-      tma_load_2d(sm.buf[b] + 2 * kTileBytes, &tmB, col, row, sm.bar + b);
-    } else {
-      tma_load_2d(sm.buf[b] + kTileBytes, &tmB, col, row, sm.bar + b);
-      if (load_c) tma_load_2d(sm.buf[b] + 2 * kTileBytes, &tmC, col, row, sm.bar + b);
-    }
-  };
-  tiles_prologue(sm, tiles, issue);
   const GroupScale unused{1.0f, 1.0f, -1.0f, false};
-  int i = 0;
-  int64_t t = blockIdx.x;
-  for (; t < tiles; t += gridDim.x, ++i) {
-    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
-    tiles_refill(t, tiles, i, issue);
-    uint16_t* T0 = reinterpret_cast<uint16_t*>(sm.buf[i & 1]);
-    uint16_t* T1 = T0 + kTileElems;
-    uint16_t* T2 = T1 + kTileElems;
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
     const int64_t mb = t / NB, nb = t % NB;
-    float gv[8];
+    const int64_t col = nb * 128 + c8;
+    const typename X::Col cs = xf.column(col);
     double dg[8];
-    if constexpr (X::kOut == 1) {
-      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + nb * 128 + c8)), gv);
+    if constexpr (X::kDgamma) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) dg[q] = 0.0;
     }
 #pragma unroll
-    for (int j = 0; j < 128 / kRowStep; ++j) {  // form this thread's chunks, quantize their rows
-      const int r = rr + kRowStep * j;
-      const int64_t m = mb * 128 + r;
-      const int off = r * 128 + c8;
-      float v[X::kOut][8];
-      if constexpr (X::kOut == 2)
-        xf.form(T0 + off, T1 + off, T2 + off, v);
-      else
-        xf.form(T0 + off, T1 + off, T2 + off, m, gv, dg, v[0]);
+    for (int h = 0; h < 8 / kBatch; ++h) {
+      typename X::In in[kBatch];
 #pragma unroll
-      for (int o = 0; o < X::kOut; ++o) {
-        const int64_t ob = o * NB + nb;
-        if (bf16_out)
-          *reinterpret_cast<uint4*>(bf16_out + m * Nout + ob * 128 + c8) =
-              *reinterpret_cast<const uint4*>((o ? T1 : T0) + off);
-        uint2 codes;
-        const float sc = quant_half_warp(v[o], codes);
-        *reinterpret_cast<uint2*>(q_row + m * Nout + ob * 128 + c8) = codes;
-        if ((tid & 15) == 0) s_row[ob * lds_row + m] = sc;
+      for (int j = 0; j < kBatch; ++j) in[j] = xf.load(mb * 128 + rr + 16 * (h * kBatch + j), col);
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int r = rr + 16 * (h * kBatch + j);
+        const int64_t m = mb * 128 + r;
+        float v[kOut][8];
+        xf.form(in[j], m, cs, dg, v);
+#pragma unroll
+        for (int o = 0; o < kOut; ++o) {
+          const int64_t ob = o * NB + nb;
+          const uint4 pk = make_uint4(pack_bf16x2(v[o][0], v[o][1]), pack_bf16x2(v[o][2], v[o][3]),
+                                      pack_bf16x2(v[o][4], v[o][5]), pack_bf16x2(v[o][6], v[o][7]));
+          *reinterpret_cast<uint4*>(tile + o * kTileElems + r * 128 + c8) = pk;
+          if (bf16_out) *reinterpret_cast<uint4*>(bf16_out + m * Nout + ob * 128 + c8) = pk;
+          if (q_row) {
+            uint2 codes;
+            const float sc = quant_half_warp(v[o], codes);
+            *reinterpret_cast<uint2*>(q_row + m * Nout + ob * 128 + c8) = codes;
+            if ((tid & 15) == 0) s_row[ob * lds_row + m] = sc;
+          }
+        }
       }
     }
-    if constexpr (X::kOut == 1) {  // dgamma: this warp's two row sets, per column
+    if constexpr (X::kDgamma) {  // dgamma: this warp's two row sets, per column
 #pragma unroll
       for (int q = 0; q < 8; ++q) dg[q] = __dadd_rn(dg[q], __shfl_xor_sync(kFull, dg[q], 16));
       if (lane < 16) {
@@ -1204,26 +1132,24 @@ __global__ void __launch_bounds__(X::kThreads) bwd_dual_kernel(
         for (int q = 0; q < 8; ++q) dgs[warp * 128 + c8 + q] = dg[q];
       }
     }
-    // the formed values were written by the generic proxy into buffers the TMA refills
-    // later; order them before that, and let the column pass see them
-    fence_proxy_async_smem();
     __syncthreads();
-    if constexpr (X::kOut == 1) {
+    if constexpr (X::kDgamma) {
       if (tid < 128) {
         double a = dgs[tid];
 #pragma unroll
-        for (int w = 1; w < kT / 32; ++w) a = __dadd_rn(a, dgs[w * 128 + tid]);
+        for (int w = 1; w < 8; ++w) a = __dadd_rn(a, dgs[w * 128 + tid]);
         dg_part[mb * (NB * 128) + nb * 128 + tid] = a;
       }
     }
+    // Each column pass reads its tile into registers before its own barrier, so once
+    // every thread is past the last one the tiles may be overwritten by the next unit.
 #pragma unroll
-    for (int o = 0; o < X::kOut; ++o) {
+    for (int o = 0; o < kOut; ++o) {
       const int64_t ob = o * NB + nb;
-      tile_cols_bf16<kT>(o ? T1 : T0, sm.red + o * kQ * 128, true, unused,
-                         q_colT + (ob * 128) * M + mb * 128, M, s_col + mb * Nout + ob * 128);
+      tile_cols_bf16<256>(tile + o * kTileElems, red + o * 4 * 128, true, unused,
+                          q_colT + (ob * 128) * M + mb * 128, M, s_col + mb * Nout + ob * 128);
     }
   }
-  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
 
 // dgamma_j = (float) sum over row blocks (in order) of the fp64 unit partials.
@@ -1445,17 +1371,12 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
       (q_row && (!aligned16(q_row) || !aligned16(s_row))))
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  CUtensorMap tm;
-  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, N, M, lddy * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
-    return FP8Q_ERR_UNSUPPORTED;
-  unsigned* err = device_error_word();
-  if (!err) return FP8Q_ERR_CUDA;
+  constexpr size_t kSmem = direct_smem_bytes<GradDirect>();
+  auto kern = direct_dual_kernel<GradDirect, kA6Batch, kA6MinBlocks>;
   static int occ[64];
-  const int per_sm = resident_ctas(transpose_quant_bf16_kernel, 256, kTileSmemBF16, occ);
-  transpose_quant_bf16_kernel<<<grid_for((M / 128) * (N / 128), per_sm), 256, kTileSmemBF16,
-                                static_cast<cudaStream_t>(stream)>>>(
-      tm, M, N, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
+  kern<<<grid_for((M / 128) * (N / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
+      GradDirect{dy, lddy}, M, N / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col, nullptr);
   return launch_status("transpose_quant_bf16 launch");
 }
 
@@ -1497,22 +1418,19 @@ extern "C" fp8q_status fp8q_rmsnorm_quant_dual(const uint16_t* x, const uint16_t
     return FP8Q_ERR_ALIGN;
   const int sms = sm100_sm_count();
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
-  CUtensorMap tm;
-  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, ldx * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
-    return FP8Q_ERR_UNSUPPORTED;
-  unsigned* err = device_error_word();
-  if (!err) return FP8Q_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the reciprocal RMS of every row first (one warp per row), then the tiles
   const int64_t rstd_ctas = std::min<int64_t>((M + 7) / 8, static_cast<int64_t>(sms) * 8);
   rmsnorm_rstd_kernel<<<static_cast<int>(rstd_ctas), 256, 0, st>>>(x, M, H, ldx, eps, rstd);
   const fp8q_status s1 = launch_status("rmsnorm_rstd launch");
   if (s1 != FP8Q_OK) return s1;
+  constexpr size_t kSmem = direct_smem_bytes<RmsDirect>();
+  auto kern = direct_dual_kernel<RmsDirect, kFwdBatch, kFwdMinBlocks>;
   static int occ[64];
-  const int per_sm = resident_ctas(dual_quant_kernel<RmsDual>, 256, kTileSmemBF16, occ);
-  dual_quant_kernel<RmsDual><<<grid_for((M / 128) * (H / 128), per_sm), 256, kTileSmemBF16, st>>>(
-      tm, RmsDual{rstd, gamma}, M, H, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
+  kern<<<grid_for((M / 128) * (H / 128), per_sm), 256, kSmem, st>>>(
+      RmsDirect{x, ldx, rstd, gamma}, M, H / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col,
+      nullptr);
   return launch_status("rmsnorm_quant_dual launch");
 }
 
@@ -1527,19 +1445,12 @@ extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int
       !aligned16(s_col) || ldgu % 8)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  CUtensorMap tm;
-  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu, 2 * I, M, ldgu * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
-    return FP8Q_ERR_UNSUPPORTED;
-  unsigned* err = device_error_word();
-  if (!err) return FP8Q_ERR_CUDA;
-  constexpr int kThr = SwigluDual::kThreads;
-  constexpr size_t kSmem = 1024 + 2 * (2 * kTileElems * 2) + (kThr / 64) * 128 * 4 + 64;
+  constexpr size_t kSmem = direct_smem_bytes<SwigluDirect>();
+  auto kern = direct_dual_kernel<SwigluDirect, kBwdBatch, kBwdMinBlocks>;
   static int occ[64];
-  const int per_sm = resident_ctas(dual_quant_kernel<SwigluDual>, kThr, kSmem, occ);
-  dual_quant_kernel<SwigluDual><<<grid_for((M / 128) * (I / 128), per_sm), kThr, kSmem,
-                                  static_cast<cudaStream_t>(stream)>>>(
-      tm, SwigluDual{I}, M, I, q_row, s_row, lds_row, q_colT, s_col, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
+  kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
+      SwigluDirect{gu, ldgu, I}, M, I / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col, nullptr);
   return launch_status("swiglu_quant_dual launch");
 }
 
@@ -1553,21 +1464,12 @@ extern "C" fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint
       !aligned16(s_row) || !aligned16(q_colT) || !aligned16(s_col))
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  CUtensorMap tmGU, tmDH;
-  if (!encode_tmap_2d(&tmGU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu, 2 * I, M, 2 * I * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_tmap_2d(&tmDH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dh, I, M, I * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
-    return FP8Q_ERR_UNSUPPORTED;
-  unsigned* err = device_error_word();
-  if (!err) return FP8Q_ERR_CUDA;
-  constexpr size_t kSmem = bwd_smem_bytes<SwigluBwd>();
+  constexpr size_t kSmem = direct_smem_bytes<SwigluBwd>();
+  auto kern = direct_dual_kernel<SwigluBwd, kBwdBatch, kBwdMinBlocks>;
   static int occ[64];
-  const int per_sm = resident_ctas(bwd_dual_kernel<SwigluBwd>, SwigluBwd::kThreads, kSmem, occ);
-  bwd_dual_kernel<SwigluBwd><<<grid_for((M / 128) * (I / 128), per_sm), SwigluBwd::kThreads, kSmem,
-                               static_cast<cudaStream_t>(stream)>>>(
-      tmGU, tmDH, tmDH, SwigluBwd{}, M, I / 128, dgu, q_row, s_row, lds_row, q_colT, s_col,
-      nullptr, nullptr, 1, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
+  kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
+      SwigluBwd{gu, dh, I}, M, I / 128, dgu, q_row, s_row, lds_row, q_colT, s_col, nullptr);
   return launch_status("swiglu_bwd_quant_dual launch");
 }
 
@@ -1600,16 +1502,6 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
     return FP8Q_ERR_ALIGN;
   const int sms = sm100_sm_count();
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
-  CUtensorMap tmX, tmDY, tmR;
-  if (!encode_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, H * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_tmap_2d(&tmDY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, H, M, H * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_tmap_2d(&tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dres ? dres : dy, H, M, H * 2, 128,
-                      128, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return FP8Q_ERR_UNSUPPORTED;
-  unsigned* err = device_error_word();
-  if (!err) return FP8Q_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* r = reinterpret_cast<float*>(ws);
@@ -1620,12 +1512,13 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
   rmsnorm_bwd_rows_kernel<<<static_cast<int>(row_ctas), 256, 0, st>>>(x, gamma, dy, M, H, eps, r, k);
   fp8q_status s1 = launch_status("rmsnorm_bwd_rows launch");
   if (s1 != FP8Q_OK) return s1;
-  constexpr size_t kSmem = bwd_smem_bytes<RmsBwd>();
+  constexpr size_t kSmem = direct_smem_bytes<RmsBwd>();
+  auto kern = direct_dual_kernel<RmsBwd, kBwdBatch, kBwdMinBlocks>;
   static int occ[64];
-  const int per_sm = resident_ctas(bwd_dual_kernel<RmsBwd>, RmsBwd::kThreads, kSmem, occ);
-  bwd_dual_kernel<RmsBwd><<<grid_for((M / 128) * (H / 128), per_sm), RmsBwd::kThreads, kSmem, st>>>(
-      tmX, tmDY, tmR, RmsBwd{r, k, gamma, dres != nullptr}, M, H / 128, out, q_row, s_row, lds_row,
-      q_colT, s_col, gamma, part, dres ? 1 : 0, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
+  kern<<<grid_for((M / 128) * (H / 128), per_sm), 256, kSmem, st>>>(
+      RmsBwd{x, dy, dres, r, k, gamma, H}, M, H / 128, out, q_row, s_row, lds_row, q_colT, s_col,
+      part);
   s1 = launch_status("rmsnorm_bwd_quant_dual launch");
   if (s1 != FP8Q_OK || !dgamma) return s1;
   const int64_t red_ctas = std::min<int64_t>((H + 255) / 256, static_cast<int64_t>(sms) * 4);
