@@ -60,7 +60,13 @@ BYTES_PER_ELEM = {
     "rmsnorm_quant_dual": 2 + 2 * (1 + 4 / 128),
     "swiglu_quant_dual": 4 + 2 * (1 + 4 / 128),   # per output element
     "transpose_quant_bf16_act": 2 + 2 * (1 + 4 / 128),
+    # backward producers with the quantizer fused: gate, up, dh in, both groupings of
+    # [d_gate | d_up] out (per (token, i)); x, dy, dres in, BF16 out + both groupings
+    "swiglu_bwd_quant_dual": 6 + 2 * 2 * (1 + 4 / 128),
+    "rmsnorm_bwd_quant_dual": 6 + 2 + 2 * (1 + 4 / 128),
 }
+# kernels one call launches (the rest launch one)
+KERNELS_PER_CALL = {"rmsnorm_quant_dual": 2, "rmsnorm_bwd_quant_dual": 3}
 
 
 def read_peaks():
@@ -104,9 +110,13 @@ def whole_job_tflops(flops_per_rank: float, world: int, max_ms_per_step: float) 
 class LayerStep:
     """Device buffers of one layer pass and the launch sequence (all through the C ABI)."""
 
-    def __init__(self, fq, wl, device, seed_offset=0, forward_only=False, saved="fp8"):
+    def __init__(self, fq, wl, device, seed_offset=0, forward_only=False, saved="fp8",
+                 backward="a6"):
         self.fq = fq
         self.saved = saved  # "fp8": requantize the saved FP8 input for WGrad; "dual": option B
+        # "a6": every linear's BF16 upstream gradient is an input, quantized by a6;
+        # "fused": the SwiGLU and RMSNorm backward producers emit those codes (chained)
+        self.backward = backward
         L = wl.layer
         self.M = M = wl.tokens
         self.L = L
@@ -133,6 +143,19 @@ class LayerStep:
         self.flops = workloads.layer_gemm_flops(L, M, passes=1 if forward_only else 3)
         if saved == "dual":
             self.rstd = {n: e(M, dt=f32) for n in ("qkv", "gate_up")}
+        if backward == "fused" and not forward_only:
+            # a stack of identical layers in steady state: the gradient arriving from the
+            # layer above (dy["down"]) is an input; this layer's RMSNorm1 backward emits
+            # the down projection's dY codes of the layer below, which the next step
+            # consumes as its own (the first step's come from a6 here)
+            self.d_h = e(M, H, dt=bf)
+            self.d_x = e(M, H, dt=bf)
+            self.dgamma = [e(H, dt=f32), e(H, dt=f32)]
+            self.ws = e(fq.rmsnorm_bwd_workspace_bytes(M, H))
+            dn = self.lin["down"]
+            fq.transpose_quant_bf16(inp["dy"]["down"], dn["q_dy"], dn["s_dy"], dn["q_dyT"],
+                                    dn["s_dyc"])
+        self.launch_count = None
         if forward_only:
             # serving: the weights are quantized once (at weight sync), not per step
             for name, d in self.lin.items():
@@ -141,6 +164,7 @@ class LayerStep:
     def _k(self, name, fn, timer):
         if self.only is not None and name not in self.only:
             return
+        self._launched += KERNELS_PER_CALL.get(name, 1)
         if timer is not None:
             timer.start(name)
         fn()
@@ -150,6 +174,12 @@ class LayerStep:
     only = None  # when set: launch only the kernels of these kinds (per-kind graphs)
 
     def run(self, timer=None, stream=None, only=None):
+        self._launched = 0
+        self._run(timer, stream, only)
+        if only is None:
+            self.launch_count = self._launched
+
+    def _run(self, timer, stream, only):
         fq, inp, lin, M = self.fq, self.inp, self.lin, self.M
         self.only = only
         self.timer = timer
@@ -161,7 +191,19 @@ class LayerStep:
                                                              d["qwT"], stream), timer)
         q, o, gu, dn = lin["qkv"], lin["o"], lin["gate_up"], lin["down"]
         if self.saved == "dual":
-            return self._run_dual(k, stream)
+            self._forward_dual(k, stream)
+        else:
+            self._forward_fp8(k, stream)
+        if self.forward_only:
+            return
+        if self.backward == "fused":
+            self._backward_fused(k, stream)
+        else:
+            self._backward_a6(k, stream)
+
+    def _forward_fp8(self, k, stream):
+        fq, inp, lin, timer = self.fq, self.inp, self.lin, self.timer
+        q, o, gu, dn = lin["qkv"], lin["o"], lin["gate_up"], lin["down"]
         # forward
         k("rmsnorm_quant", lambda: fq.rmsnorm_quant(inp["x_attn"], inp["gamma1"], self.eps,
                                                     q["q_in"], q["s_in"], stream), timer)
@@ -178,21 +220,59 @@ class LayerStep:
         k("swiglu_quant", lambda: fq.swiglu_quant(gu["y"], dn["q_in"], dn["s_in"], stream), timer)
         k("gemm_fwd", lambda: fq.linear_fwd(dn["q_in"], dn["s_in"], dn["qw"], dn["sw"], dn["y"],
                                             stream), timer)
-        # backward of each linear (BF16 upstream gradients)
-        for name in (() if self.forward_only else ("down", "gate_up", "o", "qkv")):
+
+    def _wgrad(self, k, d, stream):
+        """WGrad of one linear; with FP8 saved activations their 128x1 codes come from the
+        requantizer a8 first."""
+        fq = self.fq
+        if self.saved == "fp8":
+            k("transpose_quant_fp8", lambda: fq.transpose_quant_fp8(d["q_in"], d["s_in"], d["q_inT"],
+                                                                    d["s_inT"], stream), self.timer)
+        k("gemm_wgrad", lambda: fq.linear_wgrad(d["q_dyT"], d["s_dyc"], d["q_inT"], d["s_inT"],
+                                                d["dw"], stream), self.timer)
+
+    def _backward_a6(self, k, stream):
+        """Backward of each linear from its BF16 upstream gradient (an input), quantized by
+        a6."""
+        fq, inp, lin = self.fq, self.inp, self.lin
+        for name in ("down", "gate_up", "o", "qkv"):
             d = lin[name]
             k("transpose_quant_bf16",
               lambda d=d, name=name: fq.transpose_quant_bf16(inp["dy"][name], d["q_dy"], d["s_dy"],
-                                                             d["q_dyT"], d["s_dyc"], stream), timer)
+                                                             d["q_dyT"], d["s_dyc"], stream),
+              self.timer)
             k("gemm_dgrad", lambda d=d: fq.linear_dgrad(d["q_dy"], d["s_dy"], d["qwT"], d["sw"],
-                                                        d["dx"], stream), timer)
-            k("transpose_quant_fp8", lambda d=d: fq.transpose_quant_fp8(d["q_in"], d["s_in"],
-                                                                        d["q_inT"], d["s_inT"],
-                                                                        stream), timer)
-            k("gemm_wgrad", lambda d=d: fq.linear_wgrad(d["q_dyT"], d["s_dyc"], d["q_inT"],
-                                                        d["s_inT"], d["dw"], stream), timer)
+                                                        d["dx"], stream), self.timer)
+            self._wgrad(k, d, stream)
 
-    def _run_dual(self, k, stream):
+    def _backward_fused(self, k, stream):
+        """Chained backward: each producer's BF16 backward emits the codes of the gradient
+        its preceding linear consumes. The QKV gradient comes from attention's backward
+        (outside this path): an input, quantized by a6."""
+        fq, inp, lin, t, eps = self.fq, self.inp, self.lin, self.timer, self.eps
+        q, o, gu, dn = lin["qkv"], lin["o"], lin["gate_up"], lin["down"]
+        dgrad = lambda d: k("gemm_dgrad", lambda: fq.linear_dgrad(  # noqa: E731
+            d["q_dy"], d["s_dy"], d["qwT"], d["sw"], d["dx"], stream), t)
+        dgrad(dn)                                  # dh = dY_down W_down
+        self._wgrad(k, dn, stream)
+        k("swiglu_bwd_quant_dual", lambda: fq.swiglu_bwd_quant_dual(
+            gu["y"], dn["dx"], gu["q_dy"], gu["s_dy"], gu["q_dyT"], gu["s_dyc"], None, stream), t)
+        dgrad(gu)                                  # gradient of the RMSNorm2 output
+        self._wgrad(k, gu, stream)
+        k("rmsnorm_bwd_quant_dual", lambda: fq.rmsnorm_bwd_quant_dual(
+            inp["x_mlp"], inp["gamma2"], gu["dx"], inp["dy"]["down"], eps, self.d_h, o["q_dy"],
+            o["s_dy"], o["q_dyT"], o["s_dyc"], self.dgamma[1], self.ws, stream), t)
+        dgrad(o)                                   # gradient of the attention output
+        self._wgrad(k, o, stream)
+        k("transpose_quant_bf16", lambda: fq.transpose_quant_bf16(
+            inp["dy"]["qkv"], q["q_dy"], q["s_dy"], q["q_dyT"], q["s_dyc"], stream), t)
+        dgrad(q)                                   # gradient of the RMSNorm1 output
+        self._wgrad(k, q, stream)
+        k("rmsnorm_bwd_quant_dual", lambda: fq.rmsnorm_bwd_quant_dual(
+            inp["x_attn"], inp["gamma1"], q["dx"], self.d_h, eps, self.d_x, dn["q_dy"], dn["s_dy"],
+            dn["q_dyT"], dn["s_dyc"], self.dgamma[0], self.ws, stream), t)
+
+    def _forward_dual(self, k, stream):
         """Option B: every producer emits the 1x128 codes for the forward GEMM and the
         transposed 128x1 codes for WGrad from its BF16 output; no FP8 requantization."""
         fq, inp, lin = self.fq, self.inp, self.lin
@@ -215,23 +295,19 @@ class LayerStep:
             gu["y"], dn["q_in"], dn["s_in"], dn["q_inT"], dn["s_inT"], stream), self.timer)
         k("gemm_fwd", lambda: fq.linear_fwd(dn["q_in"], dn["s_in"], dn["qw"], dn["sw"], dn["y"],
                                             stream), self.timer)
-        for name in ("down", "gate_up", "o", "qkv"):
-            d = lin[name]
-            k("transpose_quant_bf16",
-              lambda d=d, name=name: fq.transpose_quant_bf16(inp["dy"][name], d["q_dy"], d["s_dy"],
-                                                             d["q_dyT"], d["s_dyc"], stream),
-              self.timer)
-            k("gemm_dgrad", lambda d=d: fq.linear_dgrad(d["q_dy"], d["s_dy"], d["qwT"], d["sw"],
-                                                        d["dx"], stream), self.timer)
-            k("gemm_wgrad", lambda d=d: fq.linear_wgrad(d["q_dyT"], d["s_dyc"], d["q_inT"],
-                                                        d["s_inT"], d["dw"], stream), self.timer)
+
+    def grad_inputs(self):
+        """Upstream BF16 gradients that enter a step from outside it."""
+        if self.forward_only:
+            return ()
+        return ("down", "qkv") if self.backward == "fused" else tuple(self.inp["dy"])
 
     @property
     def launches_per_step(self):
-        if self.forward_only:
-            return 8
-        # option B: no FP8 requantization (-4); each RMSNorm producer runs two kernels (+2)
-        return 26 if self.saved == "dual" else 28
+        """Kernels one full step launched (counted during the last full run)."""
+        if self.launch_count is None:
+            raise RuntimeError("run the step once before asking for its launch count")
+        return self.launch_count
 
     def gemm_flops_by_kind(self):
         M = self.M
@@ -257,23 +333,27 @@ class LayerStep:
         in_elems = sum(M * d["K"] for d in self.lin.values())
         if self.saved == "dual":
             e = {
-                "quant_weight_128x128": w_elems,
-                "transpose_quant_bf16": dy_elems,
                 "rmsnorm_quant_dual": 2 * M * H,
                 "transpose_quant_bf16_act": M * qo,
                 "swiglu_quant_dual": M * I,
             }
+        else:
+            e = {
+                "rmsnorm_quant": 2 * M * H,
+                "quant_act_1x128": M * qo,
+                "swiglu_quant": M * I,
+            }
+        if self.forward_only:
             return {k: v * BYTES_PER_ELEM[k] for k, v in e.items()}
-        e = {} if self.forward_only else {
-            "quant_weight_128x128": w_elems,
-            "transpose_quant_bf16": dy_elems,
-            "transpose_quant_fp8": in_elems,
-        }
-        e.update({
-            "rmsnorm_quant": 2 * M * H,
-            "quant_act_1x128": M * qo,
-            "swiglu_quant": M * I,
-        })
+        e["quant_weight_128x128"] = w_elems
+        if self.saved == "fp8":
+            e["transpose_quant_fp8"] = in_elems
+        if self.backward == "fused":
+            e["transpose_quant_bf16"] = M * self.lin["qkv"]["N"]
+            e["swiglu_bwd_quant_dual"] = M * I
+            e["rmsnorm_bwd_quant_dual"] = 2 * M * H
+        else:
+            e["transpose_quant_bf16"] = dy_elems
         return {k: v * BYTES_PER_ELEM[k] for k, v in e.items()}
 
     # end-to-end: the per-step batch comes from pinned host memory, the results go back
@@ -292,7 +372,7 @@ class E2EPipeline:
         self.step = step
         inp = step.inp
         names = ["x_attn", "x_mlp", "attn_out"]
-        self.keys = [(n, None) for n in names] + [("dy", n) for n in inp["dy"]]
+        self.keys = [(n, None) for n in names] + [("dy", n) for n in step.grad_inputs()]
         get = lambda d, k: d[k[0]] if k[1] is None else d[k[0]][k[1]]  # noqa: E731
         self.get = get
         self.host = {}
@@ -695,6 +775,10 @@ def main():
     ap.add_argument("--case-reps", type=int, default=3)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=WORKLOAD.name,
                     help="layer shape (default: the Llama-3.1-8B layer at M = 8192)")
+    ap.add_argument("--backward", choices=("a6", "fused"), default="a6",
+                    help="a6 = every linear's BF16 upstream gradient is an input quantized by "
+                         "a6; fused = the SwiGLU / RMSNorm backward producers emit the codes "
+                         "(chained, steady-state stack of identical layers)")
     ap.add_argument("--saved", choices=("fp8", "dual"), default="fp8",
                     help="saved activations for WGrad: fp8 = requantize the saved FP8 tensor "
                          "(the pages' flow, default); dual = producers emit both groupings")
@@ -724,7 +808,7 @@ def main():
         pg = dist
 
     step = LayerStep(fq, wl, dev, seed_offset=rank_seed_offset(rank), forward_only=is_decode(wl),
-                     saved=args.saved)
+                     saved=args.saved, backward=args.backward)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
         step.run()
@@ -848,6 +932,10 @@ def main():
                        "saved_activations": ("n/a" if step.forward_only else
                                              {"fp8": "FP8, requantized 128x1 for WGrad",
                                               "dual": "both groupings from BF16 (option B)"}[args.saved]),
+                       "backward": ("n/a" if step.forward_only else
+                                    {"a6": "each linear's BF16 gradient quantized by a6",
+                                     "fused": "SwiGLU / RMSNorm backward producers emit the "
+                                              "gradient codes (chained)"}[args.backward]),
                        "gemm_tflop_per_step_per_gpu": step.flops / 1e12,
                        "launches_per_step": step.launches_per_step,
                        "l2": "inputs larger than L2: %.1f GB touched per step" % (

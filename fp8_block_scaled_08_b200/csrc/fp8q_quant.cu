@@ -804,6 +804,7 @@ struct SwigluBwd {
   int64_t I;
   static constexpr int kOut = 2;
   static constexpr bool kDgamma = false;
+  static constexpr bool kHeavy = true;  // long form: keep the row-batch loop rolled
   struct In { uint4 g, u, d; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -822,8 +823,15 @@ struct SwigluBwd {
       float e0, e1;
       exp_cw2(-g[i], -g[i + 1], e0, e1);
       const float d0 = __fadd_rn(1.0f, e0), d1 = __fadd_rn(1.0f, e1);
-      const float silu0 = __fdiv_rn(g[i], d0), silu1 = __fdiv_rn(g[i + 1], d1);
       const float sig0 = __frcp_rn(d0), sig1 = __frcp_rn(d1);
+      // silu = g / d from sig = RN(1/d): q = g sig, t = q d - g, silu = q - t sig. For every
+      // BF16 g (d = fl32(1 + E(-g))) this equals the IEEE quotient, signed zeros included
+      // (exhaustive proof in the CPU tests); it replaces a second division.
+      float q0, q1, t0 = -g[i], t1 = -g[i + 1];
+      mul2(q0, q1, g[i], g[i + 1], sig0, sig1);
+      fma2(t0, t1, q0, q1, d0, d1);
+      float silu0 = q0, silu1 = q1;
+      fma2(silu0, silu1, t0, t1, -sig0, -sig1);
       float du0, du1, dhu0, dhu1;
       mul2(du0, du1, dh[i], dh[i + 1], silu0, silu1);
       mul2(dhu0, dhu1, dh[i], dh[i + 1], u[i], u[i + 1]);
@@ -931,6 +939,7 @@ struct RmsBwd {
   int64_t H;
   static constexpr int kOut = 1;
   static constexpr bool kDgamma = true;
+  static constexpr bool kHeavy = false;
   struct In { uint4 x, d, res; };
   struct Col { float g[8]; };
   __device__ __forceinline__ Col column(int64_t c) const {
@@ -981,6 +990,7 @@ struct GradDirect {
   int64_t ld;
   static constexpr int kOut = 1;
   static constexpr bool kDgamma = false;
+  static constexpr bool kHeavy = false;
   struct In { uint4 a; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1001,6 +1011,7 @@ struct RmsDirect {
   const uint16_t* gamma;
   static constexpr int kOut = 1;
   static constexpr bool kDgamma = false;
+  static constexpr bool kHeavy = false;
   struct In { uint4 a; };
   struct Col { float g[8]; };
   __device__ __forceinline__ Col column(int64_t c) const {
@@ -1033,6 +1044,7 @@ struct SwigluDirect {
   int64_t ldgu, I;
   static constexpr int kOut = 1;
   static constexpr bool kDgamma = false;
+  static constexpr bool kHeavy = true;
   struct In { uint4 g, u; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1097,7 +1109,10 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
 #pragma unroll
       for (int q = 0; q < 8; ++q) dg[q] = 0.0;
     }
-#pragma unroll
+    // unrolled for short forms; a long form (the SwiGLU exponential and divisions) stays
+    // rolled, which keeps the kernel inside the instruction cache (measured faster)
+    constexpr int kOuterUnroll = X::kHeavy ? 1 : 8 / kBatch;
+#pragma unroll kOuterUnroll
     for (int h = 0; h < 8 / kBatch; ++h) {
       typename X::In in[kBatch];
 #pragma unroll
