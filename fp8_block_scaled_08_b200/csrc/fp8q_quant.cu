@@ -359,9 +359,9 @@ __global__ void __launch_bounds__(256) rowgroup_quant_kernel(Src src, int64_t M,
 
 // ---------------------------------------------------------------------------
 // a3: RMSNorm + 1x128 quantization.
-// Rows of up to kWarpRowChunks*256 elements in batches of more than 1024 rows: one warp
-// per row (the row stays in registers, the sum of squares is a warp reduction), 8 rows
-// per CTA. Longer rows, and small batches: one CTA (256 threads) per row.
+// Batches of more than 1024 rows: one warp per row in two passes (the sum of squares,
+// a warp reduction, then the row again from L2 to form and quantize y), 8 rows per CTA.
+// Small batches: one CTA (256 threads) per row, the row held in registers.
 // Thread t of the row owns 8-element chunks t, t+T, ... (T = threads per row), so
 // that each half-warp covers one 128-group.
 // ---------------------------------------------------------------------------
@@ -425,10 +425,12 @@ __device__ __forceinline__ void norm_quant_chunk(const uint4& xr, const uint16_t
   }
 }
 
-constexpr int kWarpRowChunks = 24;  // warp-per-row path: H <= 24 * 256 = 6144
-
-template <int kChunks>
-__global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(
+// One warp per row in two passes: the fp64 sum of squares with four 16-byte loads in
+// flight per lane (the partial sums and their order are those of sum_squares, so r is
+// the same), then the row again (from L2: a warp's row is a few KB, read moments
+// before) to form y and quantize it. Holding no whole row in registers keeps the
+// kernel small enough for several CTAs per SM.
+__global__ void __launch_bounds__(256) rmsnorm_quant_warp2_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma, int64_t M, int64_t H,
     int64_t ldx, float eps, uint8_t* __restrict__ q, float* __restrict__ s, int64_t lds) {
   extern __shared__ uint4 gamma_sm[];  // H BF16 values, shared by every row
@@ -440,22 +442,46 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t m = wglobal; m < M; m += nw) {
     const uint16_t* row = x + m * ldx;
-    uint4 raw[kChunks];
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    for (int64_t c0 = 0; c0 < nch; c0 += 128) {
+      uint4 raw[4];
 #pragma unroll
-    for (int j = 0; j < kChunks; ++j) {
-      const int64_t c = lane + 32 * j;
-      if (c < nch) raw[j] = ld_nc_v4(row + c * 8);
+      for (int u = 0; u < 4; ++u) {
+        const int64_t c = c0 + lane + 32 * u;
+        if (c < nch) raw[u] = ld_nc_v4(row + c * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (c0 + lane + 32 * u < nch) {
+          float v[8];
+          unpack_bf16x8(raw[u], v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const double d = static_cast<double>(v[i]);
+            acc[i] = __fma_rn(d, d, acc[i]);
+          }
+        }
+      }
     }
-    double ss = sum_squares<kChunks>(raw, lane, 32, nch);
+    double ss = __dadd_rn(__dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3])),
+                          __dadd_rn(__dadd_rn(acc[4], acc[5]), __dadd_rn(acc[6], acc[7])));
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, off));
     const float r = rstd_from_ss(ss, H, eps);
+    for (int64_t c0 = 0; c0 < nch; c0 += 128) {
+      uint4 raw[4];
 #pragma unroll
-    for (int j = 0; j < kChunks; ++j) {
-      if (32 * j >= nch) break;  // warp-uniform; nch is a multiple of 16
-      const int64_t c = lane + 32 * j;
-      norm_quant_chunk(raw[j], reinterpret_cast<const uint16_t*>(gamma_sm), c, c < nch, r,
-                       q + m * H, s, lds, m, lane);
+      for (int u = 0; u < 4; ++u) {
+        const int64_t c = c0 + lane + 32 * u;
+        if (c < nch) raw[u] = *reinterpret_cast<const uint4*>(row + c * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (c0 + 32 * u >= nch) break;  // warp-uniform; nch is a multiple of 16
+        const int64_t c = c0 + lane + 32 * u;
+        norm_quant_chunk(raw[u], reinterpret_cast<const uint16_t*>(gamma_sm), c, c < nch, r,
+                         q + m * H, s, lds, m, lane);
+      }
     }
   }
 }
@@ -1332,20 +1358,12 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   const size_t gsm = static_cast<size_t>(H) * 2;  // gamma in shared memory
   // One warp per row needs many rows to fill the GPU; up to 1024 rows one CTA per row
   // is faster (measured 3x at 16-256 rows, equal at 8192).
-  if (H <= 8 * 32 * kWarpRowChunks && M > 1024) {
+  if (M > 1024) {
     const int64_t ctas = (M + 7) / 8;  // one warp per row
-    if (H <= 8 * 32 * 16) {
-      static int occ[64];
-      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<16>, 256, 8 * 32 * 16 * 2, occ);
-      rmsnorm_quant_warp_kernel<16><<<grid_for(ctas, per_sm), 256, gsm, st>>>(x, gamma, M, H, ldx,
-                                                                              eps, q, s, lds);
-    } else {
-      static int occ[64];
-      const int per_sm = resident_ctas(rmsnorm_quant_warp_kernel<kWarpRowChunks>, 256,
-                                       8 * 32 * kWarpRowChunks * 2, occ);
-      rmsnorm_quant_warp_kernel<kWarpRowChunks><<<grid_for(ctas, per_sm), 256, gsm, st>>>(
-          x, gamma, M, H, ldx, eps, q, s, lds);
-    }
+    static int occ[64];
+    const int per_sm = resident_ctas(rmsnorm_quant_warp2_kernel, 256, gsm, occ);
+    rmsnorm_quant_warp2_kernel<<<grid_for(ctas, per_sm), 256, gsm, st>>>(x, gamma, M, H, ldx, eps,
+                                                                         q, s, lds);
   } else {
     const int64_t grid = M < static_cast<int64_t>(sms) * 64 ? M : static_cast<int64_t>(sms) * 64;
     rmsnorm_quant_cta_kernel<<<static_cast<int>(grid), kNormThreads, gsm, st>>>(x, gamma, M, H,

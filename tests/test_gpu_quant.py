@@ -149,11 +149,12 @@ def test_weight_quant_matches_oracle(fq, oracle_mod, N, K):
 
 
 # ---------------------------------------------------------------- a3
-# batches up to 1024 rows take the CTA-per-row kernel; above, rows up to 6144 wide take
-# the warp-per-row kernel (1100 x 640: ragged chunk count per lane; 1030 x 6144: widest)
+# batches up to 1024 rows take the CTA-per-row kernel; above, the two-pass warp-per-row
+# kernel (1100 x 640: ragged chunk count per lane; 1030 x 6144; 1025 x 16384: widest)
 @pytest.mark.parametrize("M,H,eps", [(256, 512, 1e-5), (5, 4096, 1e-6), (130, 3584, 1e-5),
                                      (3, 16384, 0.0), (64, 128, 1e-5), (1100, 640, 1e-5),
-                                     (1030, 6144, 1e-6)])
+                                     (1030, 6144, 1e-6), (1025, 16384, 1e-5),
+                                     (1040, 4224, 0.0)])
 def test_rmsnorm_quant_matches_oracle(fq, oracle_mod, M, H, eps):
     x = workloads.activations_bf16((M, H), 0, 300 + M, DEV, outlier_frac=0.005,
                                    outlier_scale=50.0)
