@@ -688,7 +688,7 @@ def run_reference(args, rank, world):
 # with only the buffers it needs on the device.
 # --------------------------------------------------------------------------
 
-CASES = ("gemm_fwd", "gemm_dgrad", "gemm_wgrad", "quantizers", "gemm_decode")
+CASES = ("gemm_fwd", "gemm_dgrad", "gemm_wgrad", "quantizers", "gemm_decode", "producers")
 
 
 def run_case(name, reps):
@@ -746,6 +746,27 @@ def run_case(name, reps):
             fq.quant_weight_alloc(w)
             fq.transpose_quant_bf16_alloc(dy)
             fq.transpose_quant_fp8_alloc(q, s)
+    elif name == "producers":
+        # the kernels that quantize a value formed on the fly, at sizes above L2 but a
+        # few hundred MB each: a6 on a 4096 x 28672 gradient, the option-B producers and
+        # the backward producers (SwiGLU at 2048 x 14336, RMSNorm at 8192 x 4096)
+        I = wl.layer.intermediate
+        Ms = 2048
+        dy = workloads.gradients_bf16((4096, N), wl.dy_std, wl.seed, workloads.TID_DY[lin.name],
+                                      dev)
+        gu = workloads.normal_bf16((Ms, 2 * I), 1.5, wl.seed, 700, dev)
+        dh = workloads.gradients_bf16((Ms, I), wl.dy_std, wl.seed, 701, dev)
+        x = workloads.activations_bf16((M, K), wl.seed, workloads.TID_X_MLP, dev)
+        g = workloads.gamma_bf16(K, wl.seed, workloads.TID_GAMMA2, dev)
+        dyk = workloads.gradients_bf16((M, K), wl.dy_std, wl.seed, 702, dev)
+        dres = workloads.gradients_bf16((M, K), wl.dy_std, wl.seed, 703, dev)
+
+        def fn():
+            fq.transpose_quant_bf16_alloc(dy)
+            fq.swiglu_quant_dual_alloc(gu)
+            fq.rmsnorm_quant_dual_alloc(x, g, wl.eps)
+            fq.swiglu_bwd_quant_dual_alloc(gu, dh)
+            fq.rmsnorm_bwd_quant_dual_alloc(x, g, dyk, dres, wl.eps)
     else:
         raise SystemExit("unknown case %r (choose from %s)" % (name, ", ".join(CASES)))
     torch.cuda.synchronize()

@@ -1193,16 +1193,28 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   }
 }
 
-// dgamma_j = (float) sum over row blocks (in order) of the fp64 unit partials.
+// dgamma_j = (float) of the fp64 sum of the unit partials over the row blocks: eight
+// lanes per column each sum a contiguous eighth of the row blocks in order, then the
+// eight sums combine in a fixed tree (lane pairs, pairs of pairs, halves); a fixed order,
+// so the result is the same on every run.
 __global__ void __launch_bounds__(256) dgamma_reduce_kernel(const double* __restrict__ part,
                                                             int64_t MB, int64_t H,
                                                             float* __restrict__ dgamma) {
-  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < H;
-       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    double a = 0.0;
-    for (int64_t b = 0; b < MB; ++b) a = __dadd_rn(a, part[b * H + j]);
-    dgamma[j] = __double2float_rn(a);
+  const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t j = gt >> 3;
+  const int sub = threadIdx.x & 7;
+  const int64_t per = (MB + 7) / 8;
+  double a = 0.0;
+  if (j < H) {
+    const int64_t b0 = sub * per;
+    const int64_t b1 = b0 + per < MB ? b0 + per : MB;
+#pragma unroll 4
+    for (int64_t b = b0; b < b1; ++b) a = __dadd_rn(a, part[b * H + j]);
   }
+  a = __dadd_rn(a, __shfl_xor_sync(kFull, a, 1));
+  a = __dadd_rn(a, __shfl_xor_sync(kFull, a, 2));
+  a = __dadd_rn(a, __shfl_xor_sync(kFull, a, 4));
+  if (j < H && sub == 0) dgamma[j] = __double2float_rn(a);
 }
 
 // a8: saved FP8 activation tiles (1x128 groups) -> xhat = fl32(s * dec(q)) -> 128x1
@@ -1554,7 +1566,7 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
       part);
   s1 = launch_status("rmsnorm_bwd_quant_dual launch");
   if (s1 != FP8Q_OK || !dgamma) return s1;
-  const int64_t red_ctas = std::min<int64_t>((H + 255) / 256, static_cast<int64_t>(sms) * 4);
-  dgamma_reduce_kernel<<<static_cast<int>(red_ctas), 256, 0, st>>>(part, M / 128, H, dgamma);
+  dgamma_reduce_kernel<<<static_cast<int>((H * 8 + 255) / 256), 256, 0, st>>>(part, M / 128, H,
+                                                                             dgamma);
   return launch_status("dgamma_reduce launch");
 }
