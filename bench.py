@@ -688,7 +688,8 @@ def run_reference(args, rank, world):
 # with only the buffers it needs on the device.
 # --------------------------------------------------------------------------
 
-CASES = ("gemm_fwd", "gemm_dgrad", "gemm_wgrad", "quantizers", "gemm_decode", "producers")
+CASES = ("gemm_fwd", "gemm_dgrad", "gemm_wgrad", "gemm_wgrad_acc", "quantizers", "gemm_decode",
+         "producers")
 
 
 def run_case(name, reps):
@@ -714,14 +715,18 @@ def run_case(name, reps):
         _, sw, qwT = fq.quant_weight_alloc(w)
         dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.linear_dgrad(qdy, sdy, qwT, sw, dx)  # noqa: E731
-    elif name == "gemm_wgrad":
+    elif name in ("gemm_wgrad", "gemm_wgrad_acc"):
         x = workloads.activations_bf16((M, K), wl.seed, workloads.TID_X_MLP, dev)
         dy = workloads.gradients_bf16((M, N), wl.dy_std, wl.seed, workloads.TID_DY[lin.name], dev)
         qx, sx = fq.quant_act_1x128_alloc(x)
         qxT, sxT = fq.transpose_quant_fp8_alloc(qx, sx)
         _, _, qdyT, sdyc = fq.transpose_quant_bf16_alloc(dy, want_row=False)
-        dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
-        fn = lambda: fq.linear_wgrad(qdyT, sdyc, qxT, sxT, dw)  # noqa: E731
+        if name == "gemm_wgrad":
+            dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+            fn = lambda: fq.linear_wgrad(qdyT, sdyc, qxT, sxT, dw)  # noqa: E731
+        else:  # fp32 dW accumulated into (read and written once per launch)
+            dw = torch.zeros((N, K), dtype=torch.float32, device=dev)
+            fn = lambda: fq.linear_wgrad_acc_f32(qdyT, sdyc, qxT, sxT, dw)  # noqa: E731
     elif name == "gemm_decode":
         # Qwen3-8B gate/up projection at a 16-token decode batch (skinny-M kernel)
         dwl = workloads.QWEN3_DECODE[0]

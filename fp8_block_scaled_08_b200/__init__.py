@@ -64,6 +64,7 @@ _SIGS = {
                                        ctypes.c_int),
     "fp8q_linear_dgrad": ([_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_linear_wgrad": ([_P, _P, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
+    "fp8q_linear_wgrad_acc_f32": ([_P, _P, _P, _P, _I, _I, _I, _P, _I, _P], ctypes.c_int),
     "fp8q_debug_wait_timeout": ([_I, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -418,6 +419,20 @@ def linear_wgrad(qdyT, sdy_c, qxT, sx_c, dw, stream=None):
     _check(_lib.fp8q_linear_wgrad(_ptr(qdyT), _ptr(sdy_c), _ptr(qxT), _ptr(sx_c), M, N, K,
                                   _ptr(dw), _rows_dense(dw, "dw"), _stream(stream)),
            "fp8q_linear_wgrad")
+
+
+def linear_wgrad_acc_f32(qdyT, sdy_c, qxT, sx_c, dw, stream=None):
+    """WGrad accumulated in fp32: dw [N,K] (fp32) += the fp32 accumulator of linear_wgrad."""
+    for t, n in ((qdyT, "qdyT"), (sdy_c, "sdy_c"), (qxT, "qxT"), (sx_c, "sx_c")):
+        _dense(t, n)
+    _want(dw, torch.float32, 2, "dw")
+    N, M = qdyT.shape
+    K = qxT.shape[0]
+    if dw.shape[0] != N or dw.shape[1] != K:
+        raise ValueError("dw must be [N, K]")
+    _check(_lib.fp8q_linear_wgrad_acc_f32(_ptr(qdyT), _ptr(sdy_c), _ptr(qxT), _ptr(sx_c), M, N,
+                                          K, _ptr(dw), _rows_dense(dw, "dw"), _stream(stream)),
+           "fp8q_linear_wgrad_acc_f32")
 
 
 def debug_wait_timeout(limit_ns: int, stream=None) -> int:

@@ -124,7 +124,9 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
-template <bool kColScaleB, bool kSplitN>
+// kAccF32: instead of storing BF16, add the fp32 accumulator into an fp32 output
+// (out += A x B^T) by TMA reduce-add of 32 x 32 boxes.
+template <bool kColScaleB, bool kSplitN, bool kAccF32 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -379,34 +381,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: BF16 rows into this warp's two swizzled 32 x 64 boxes, then TMA stores
+      // (fp32 accumulate: four 32 x 32 boxes, two at a time, added by TMA reduce)
       const int wrow0 = row0 + wq * 32;
       if (wrow0 < p.M && lo_ok) {
-        if (stored) {  // the previous tile's stores must have read the boxes
-          if (lane == 0) tma_store_wait_read();
-          __syncwarp();
-        }
+        if constexpr (kAccF32) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint8_t* box = j ? out1 : out0;
+          for (int hh = 0; hh < 2; ++hh) {  // acc[64 hh + 0..63]: tile columns col_lo / col_hi
+            if (stored) {  // the previous boxes must have been read
+              if (lane == 0) tma_store_wait_read();
+              __syncwarp();
+            }
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float* a = acc + j * 64 + c * 8;
-            uint4 v;
-            v.x = pack_bf16x2(a[0], a[1]);
-            v.y = pack_bf16x2(a[2], a[3]);
-            v.z = pack_bf16x2(a[4], a[5]);
-            v.w = pack_bf16x2(a[6], a[7]);
-            *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
+            for (int j = 0; j < 2; ++j) {
+              uint8_t* box = j ? out1 : out0;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const float* a = acc + hh * 64 + j * 32 + c * 4;
+                *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                    make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                               __float_as_uint(a[3]));
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && (hh == 0 || hi_ok)) {
+              const int cb = hh ? col_hi : col_lo;
+              tma_reduce_add_2d(&tmY, out0, cb, wrow0);
+              tma_reduce_add_2d(&tmY, out1, cb + 32, wrow0);
+              tma_store_commit();
+            }
+            stored = true;
           }
+        } else {
+          if (stored) {  // the previous tile's stores must have read the boxes
+            if (lane == 0) tma_store_wait_read();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            uint8_t* box = j ? out1 : out0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float* a = acc + j * 64 + c * 8;
+              uint4 v;
+              v.x = pack_bf16x2(a[0], a[1]);
+              v.y = pack_bf16x2(a[2], a[3]);
+              v.z = pack_bf16x2(a[4], a[5]);
+              v.w = pack_bf16x2(a[6], a[7]);
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, out0, col_lo, wrow0);
+            if (hi_ok) tma_store_2d(&tmY, out1, col_hi, wrow0);
+            tma_store_commit();
+          }
+          stored = true;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmY, out0, col_lo, wrow0);
-          if (hi_ok) tma_store_2d(&tmY, out1, col_hi, wrow0);
-          tma_store_commit();
-        }
-        stored = true;
       }
     }
     if (stored && lane == 0) tma_store_wait_all();
@@ -425,14 +458,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // budget of the hand-over, and find how many CTA pairs can be resident at once (pairs
 // are placed within one GPC, so this can be below half the SM count). Returns that
 // number, or 0 on failure (the reason is in fp8q_last_error_message).
-template <bool kCol, bool kSplit>
+template <bool kCol, bool kSplit, bool kAcc = false>
 int kernel_setup() {
   static int pairs_for_device[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (pairs_for_device[dev]) return pairs_for_device[dev];
   const cudaError_t e = cudaFuncSetAttribute(
-      gemm_kernel<kCol, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+      gemm_kernel<kCol, kSplit, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) {
     set_last_error("cudaFuncSetAttribute(gemm max dynamic smem)", e);
     cudaGetLastError();
@@ -441,7 +475,7 @@ int kernel_setup() {
   // The register hand-over inside the kernel waits until the block's launch allocation
   // covers the new budgets; refuse to launch a build whose allocation would not.
   cudaFuncAttributes attr;
-  const cudaError_t ea = cudaFuncGetAttributes(&attr, gemm_kernel<kCol, kSplit>);
+  const cudaError_t ea = cudaFuncGetAttributes(&attr, gemm_kernel<kCol, kSplit, kAcc>);
   if (ea != cudaSuccess) {
     set_last_error("cudaFuncGetAttributes(gemm)", ea);
     cudaGetLastError();
@@ -464,7 +498,8 @@ int kernel_setup() {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int clusters = 0;
-  const cudaError_t eo = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<kCol, kSplit>, &cfg);
+  const cudaError_t eo =
+      cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<kCol, kSplit, kAcc>, &cfg);
   if (eo != cudaSuccess || clusters <= 0) {
     set_last_error("cudaOccupancyMaxActiveClusters(gemm)", eo != cudaSuccess ? eo : cudaErrorInvalidConfiguration);
     cudaGetLastError();
@@ -474,11 +509,12 @@ int kernel_setup() {
   return clusters;
 }
 
-// out [Mg][Ng] = A [Mg][Kg] x B [Ng][Kg]^T with the scales described above.
-template <bool kCol, bool kSplit>
+// out [Mg][Ng] = A [Mg][Kg] x B [Ng][Kg]^T with the scales described above; out is BF16
+// (y: uint16_t) or, with kAcc, an fp32 array the product is added to (y: float).
+template <bool kCol, bool kSplit, bool kAcc = false>
 fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t Ng, int64_t Kg,
                         const float* sa, int64_t ldsa, const float* sb, int64_t sb_sj,
-                        int64_t sb_sr, const float* sbcol, uint16_t* y, int64_t ldy,
+                        int64_t sb_sr, const float* sbcol, void* y, int64_t ldy,
                         cudaStream_t stream) {
   const int sms = sm100_sm_count();
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
@@ -488,8 +524,10 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
                            CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, Kg, Ng, Kg, BK, BN / 2,
                            CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, Ng, Mg, ldy * 2, 64, 32,
-                           CU_TENSOR_MAP_SWIZZLE_128B) &&
+            (kAcc ? encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y, Ng, Mg, ldy * 4, 32,
+                                   32, CU_TENSOR_MAP_SWIZZLE_128B)
+                  : encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, Ng, Mg, ldy * 2, 64,
+                                   32, CU_TENSOR_MAP_SWIZZLE_128B)) &&
             encode_tmap_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, Mg, Kg / BK, ldsa * 4, BM,
                            1, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (ok && kCol)
@@ -498,7 +536,7 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   else
     tmSB = tmSA;
   if (!ok) return FP8Q_ERR_UNSUPPORTED;
-  const int max_pairs = kernel_setup<kCol, kSplit>();
+  const int max_pairs = kernel_setup<kCol, kSplit, kAcc>();
   if (max_pairs <= 0) return FP8Q_ERR_CUDA;
 
   GemmParams p;
@@ -512,7 +550,7 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   p.sb = sb;
   p.sb_sj = sb_sj;
   p.sb_sr = sb_sr;
-  p.y = y;
+  p.y = static_cast<uint16_t*>(y);
   p.ldy = ldy;
   p.err = device_error_word();
   p.wait_limit_ns = kWaitLimitNs;
@@ -520,7 +558,8 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   const int64_t tiles = static_cast<int64_t>(p.mblocks) * p.nblocks;
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, max_pairs));
-  gemm_kernel<kCol, kSplit><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmSA, tmSB, tmY, p);
+  gemm_kernel<kCol, kSplit, kAcc><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmSA, tmSB,
+                                                                           tmY, p);
   return launch_status("gemm_kernel launch");
 }
 
@@ -580,4 +619,19 @@ extern "C" fp8q_status fp8q_linear_wgrad(const uint8_t* qdyT, const float* sdy_c
   // Column scale of (k, slice r) = sx_c[r*K + k]
   return launch_gemm<true, false>(qdyT, qxT, N, K, M, sdy_c, N, nullptr, 0, 0, sx_c, dw, lddw,
                            static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_linear_wgrad_acc_f32(const uint8_t* qdyT, const float* sdy_c,
+                                                 const uint8_t* qxT, const float* sx_c, int64_t M,
+                                                 int64_t N, int64_t K, float* dw, int64_t lddw,
+                                                 void* stream) {
+  if (!qdyT || !sdy_c || !qxT || !sx_c || !dw) return FP8Q_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 128 || lddw < K)
+    return FP8Q_ERR_SHAPE;
+  if (!aligned16(qdyT) || !aligned16(sdy_c) || !aligned16(qxT) || !aligned16(sx_c) ||
+      !aligned16(dw) || lddw % 4)
+    return FP8Q_ERR_ALIGN;
+  // as fp8q_linear_wgrad, with dw += the fp32 accumulator instead of dw = bf16(it)
+  return launch_gemm<true, false, true>(qdyT, qxT, N, K, M, sdy_c, N, nullptr, 0, 0, sx_c, dw,
+                                        lddw, static_cast<cudaStream_t>(stream));
 }

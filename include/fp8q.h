@@ -275,6 +275,20 @@ fp8q_status fp8q_linear_wgrad(const uint8_t* qdyT, const float* sdy_c, const uin
                               const float* sx_c, int64_t M, int64_t N, int64_t K,
                               uint16_t* dw, int64_t lddw, void* stream);
 
+/* WGrad accumulated in fp32 (the survey's next row f3: an fp32 accumulate-into-dW
+ * option, for gradient accumulation over micro-batches): as fp8q_linear_wgrad, but
+ *   dw[n,k] = fl32(dw[n,k] + acc[n,k])
+ * where acc is the same fp32 accumulator fp8q_linear_wgrad rounds to BF16; dw [N][K]
+ * fp32 (row stride lddw elements, lddw % 4 == 0) is read and written once per element by
+ * the tensor memory accelerator's reduce-add, so each call adds exactly one product and
+ * the result does not depend on timing. Calls that add into the same dw must be ordered
+ * (one stream). The pages keep master weights in BF16 and say nothing of the gradient
+ * buffer's precision; this entry point has no counterpart on them. */
+fp8q_status fp8q_linear_wgrad_acc_f32(const uint8_t* qdyT, const float* sdy_c,
+                                      const uint8_t* qxT, const float* sx_c, int64_t M,
+                                      int64_t N, int64_t K, float* dw, int64_t lddw,
+                                      void* stream);
+
 /* Diagnostic: launches one CTA that waits on a barrier nothing completes, with a
  * wait limit of `limit_ns` nanoseconds, exactly as the GEMM's bounded waits do.
  * The kernel gives up, records FP8Q_ERR_TIMEOUT in the device error word and

@@ -158,3 +158,12 @@ def test_validation_backward_producers():
     assert call(g, A, B, C, NUL, 256, 512, F(1e-5), NUL, E, A, 256, B, C, NUL, W, need, NUL) == 1
     assert call(g, A, B, C, ctypes.c_void_p(0x10004), 256, 512, F(1e-5), D, E, A, 256, B, C, NUL,
                 W, need, NUL) == 3                                                 # dres align
+
+
+def test_validation_wgrad_acc_f32():
+    f = "fp8q_linear_wgrad_acc_f32"
+    assert call(f, A, B, C, D, 100, 128, 128, E, 128, NUL) == 2       # M % 128
+    assert call(f, A, B, C, D, 128, 128, 100, E, 128, NUL) == 2       # K % 128
+    assert call(f, A, B, C, D, 128, 128, 128, E, 126, NUL) == 2       # lddw < K
+    assert call(f, A, B, C, D, 128, 128, 256, E, 258, NUL) == 3       # lddw % 4
+    assert call(f, A, B, C, NUL, 128, 128, 128, E, 128, NUL) == 1
