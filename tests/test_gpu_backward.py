@@ -179,3 +179,40 @@ def test_full_size_llama_backward_producers_sampled(fq, oracle_mod):
     _, rdg, _, _ = oracle_mod.rmsnorm_bwd(bits(x), bits(g), bits(dy), None, wl.eps)
     d = np.abs(np_f32(dg).astype(np.float64) - rdg.astype(np.float64))
     assert np.all(d <= 2 * np.spacing(np.abs(rdg)).astype(np.float64) + 1e-12)
+
+
+def test_rmsnorm_bwd_degenerate_rows(fq, oracle_mod):
+    """A zero input row (r = 1/sqrt(eps), c = 0: dx = r gamma dy), a zero gradient row
+    (dx = 0, out = dres), a zero residual gradient, one row block (M = 128)."""
+    M, H, eps = 128, 1024, 1e-5
+    x, g, dy, dres = _rms_inputs(M, H, 3700, True)
+    x[3] = 0.0
+    dy[7] = 0.0
+    dy[9] = -0.0
+    dres[11] = 0.0
+    out, q, s, qT, sT, dg = fq.rmsnorm_bwd_quant_dual_alloc(x, g, dy, dres, eps)
+    torch.cuda.synchronize()
+    _check_rms(fq, oracle_mod, x, g, dy, dres, eps, out, q, s, qT, sT, dg, "degenerate rows")
+    assert torch.equal(out[7].float(), dres[7].float())
+
+
+def test_swiglu_bwd_dual_every_bf16_gate(fq, oracle_mod):
+    """Every BF16 bit pattern as a gate (128 x 512 of them) with fixed up and dh values:
+    the gradient and its codes bit for bit. Patterns of magnitude 2^127 and up (and the
+    non-finite ones) are replaced by zero: with dh = -1.5 their products leave fp32's
+    range, and non-finite values are outside the contract."""
+    M, I = 128, 512
+    pats = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    exp = (pats >> 7) & 0xFF
+    pats[exp >= 0xFE] = 0
+    gate = torch.from_numpy(pats.view(np.int16).reshape(M, I)).view(torch.bfloat16).to(DEV)
+    up = torch.full((M, I), 0.75, dtype=torch.bfloat16, device=DEV)
+    gu = torch.cat([gate, up], dim=1).contiguous()
+    dh = torch.full((M, I), -1.5, dtype=torch.bfloat16, device=DEV)
+    q, s, qT, sT, dgu = fq.swiglu_bwd_quant_dual_alloc(gu, dh, want_dgu=True)
+    torch.cuda.synchronize()
+    rq, rs, rqT, rsT, rdgu = oracle_mod.swiglu_bwd_dual(bits(gu), bits(dh))
+    assert np.array_equal(bits(dgu), rdgu)
+    assert_codes_equal(q, rq, "every gate rows")
+    assert_codes_equal(qT, rqT, "every gate columns")
+    assert_scales_equal(sT, rsT, "every gate column scales")
