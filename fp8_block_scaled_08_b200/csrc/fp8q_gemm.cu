@@ -32,13 +32,17 @@
 //               ring.
 //   warp 1      allocates 512 TMEM columns (both CTAs); in the leader, one thread
 //               issues the pair MMAs into TMEM buffer r%2 and commits to barriers in
-//               both CTAs that free the smem stage / publish the slice.
-//   warps 2, 3  idle. Warpgroup 0 (warps 0-3) hands registers to the others.
+//               both CTAs that free the smem stage / publish the slice. With the N
+//               split (forward, DGrad: each slice as two N = 128 halves) one thread of
+//               warp 2 issues every other slice, so two threads share the issuing.
+//   warps 2, 3  otherwise idle. Warpgroup 0 (warps 0-3) hands registers to the others.
 //   warps 4..11 two warpgroups; warpgroup h promotes columns 128h..128h+127 of this
 //               CTA's 128 x 256 part: tcgen05.ld, packed fp32 FMA into 128 registers
 //               per thread, release the TMEM buffer (the peer's warps arrive on the
 //               leader's barrier); after the last slice they round to BF16, stage the
-//               rows in shared memory (128-byte swizzle) and store them with TMA.
+//               rows in shared memory (128-byte swizzle) and store them with TMA (the
+//               fp32-accumulate WGrad stages fp32 boxes and adds them into its output
+//               with TMA reduce-add instead).
 // Registers: the block launches with 168 per thread (168 x 384 = 64512); warpgroup
 // 0 drops to 40 and the promotion warpgroups rise to 232 (40*128 + 232*256 = 64512).
 // Every mbarrier wait is bounded (kWaitLimitNs): a wait that gives up records

@@ -1,7 +1,9 @@
 // Quantizer kernels of libfp8q (sm_100a): the 1x128 activation quantizer, the
 // 128x128 weight quantizer, fused RMSNorm+quantize, fused SwiGLU+quantize, the
-// dual (row 1x128 + transposed column 128x1) quantizer of BF16 gradients and the
-// transposed 128x1 requantizer of saved FP8 activations.
+// dual (row 1x128 + transposed column 128x1) quantizer of BF16 gradients, the
+// transposed 128x1 requantizer of saved FP8 activations, the producers that emit
+// both groupings of their BF16 output (RMSNorm, SwiGLU), and the RMSNorm / SwiGLU
+// backward in BF16 with the dual gradient quantizer fused behind them.
 //
 // All of them are HBM-bound: BF16 is read with 16-byte loads that a warp issues as
 // contiguous runs, group maxima are taken with warp shuffles, and the codes come from
