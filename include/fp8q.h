@@ -27,14 +27,18 @@
  *
  * Conventions
  *   - Every pointer is a DEVICE pointer owned by the caller; the library allocates
- *     no device memory, keeps no per-call state and never synchronises the host.
+ *     no device memory (scratch space is a caller-owned workspace argument, or, for
+ *     fp8q_linear_fwd_splitk_noalloc, a fixed array in the library's own device
+ *     memory), keeps no per-call state and never synchronises the host.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Each call validates
- *     its arguments synchronously, then enqueues one kernel on `stream`.
+ *     its arguments synchronously, then enqueues its kernels on `stream` (one kernel;
+ *     two for fp8q_rmsnorm_quant_dual, up to three for fp8q_rmsnorm_bwd_quant_dual).
  *   - Shapes: K (the grouped / reduction dimension) % 128 == 0 everywhere;
  *     weight N % 128 == 0; M % 128 == 0 on the 128x1 paths; otherwise M >= 1.
  *   - Alignment: every pointer 16-byte aligned; BF16 row strides % 8 == 0.
  *   - No call aborts or throws; each returns an fp8q_status.
- *   - Thread safety: re-entrant; calls on different streams may overlap.
+ *   - Thread safety: re-entrant; calls on different streams may overlap, except
+ *     those sharing a workspace (and fp8q_linear_fwd_splitk_noalloc, see there).
  */
 #ifndef FP8Q_H
 #define FP8Q_H
