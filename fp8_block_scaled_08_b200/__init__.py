@@ -42,6 +42,7 @@ _SIGS = {
     "fp8q_version": ([], ctypes.c_int),
     "fp8q_last_error_message": ([], ctypes.c_char_p),
     "fp8q_device_error": ([_P, ctypes.c_int], ctypes.c_int),
+    "fp8q_last_device_error": ([_P], ctypes.c_int),
     "fp8q_quant_act_1x128": ([_P, _I, _I, _I, _P, _P, _I, _P], ctypes.c_int),
     "fp8q_quant_weight_128x128": ([_P, _I, _I, _I, _P, _P, _P, _P], ctypes.c_int),
     "fp8q_rmsnorm_quant": ([_P, _P, _I, _I, _I, _F, _P, _P, _I, _P], ctypes.c_int),

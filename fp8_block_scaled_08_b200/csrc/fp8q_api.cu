@@ -181,6 +181,10 @@ extern "C" fp8q_status fp8q_device_error(void* stream, int clear) {
   return (v & kErrTimeout) ? FP8Q_ERR_TIMEOUT : FP8Q_OK;
 }
 
+extern "C" fp8q_status fp8q_last_device_error(void* stream) {
+  return fp8q_device_error(stream, 0);
+}
+
 extern "C" fp8q_status fp8q_debug_wait_timeout(int64_t limit_ns, void* stream) {
   if (limit_ns <= 0 || limit_ns > 10000000000ll) return FP8Q_ERR_SHAPE;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;

@@ -74,6 +74,9 @@ int fp8q_version(void);
  * Returns FP8Q_OK when no kernel reported an error. For tests and diagnostics. */
 fp8q_status fp8q_device_error(void* stream, int clear);
 
+/* fp8q_device_error(stream, 0): the same read, without clearing. */
+fp8q_status fp8q_last_device_error(void* stream);
+
 /* a1. Activation quantization per 1x128 group ("Esquema de Cuantización",
  * activations bullet).
  *   x  [M][K] BF16, row stride ldx (>= K, % 8 == 0)
