@@ -1,6 +1,8 @@
 """The failure path on a GPU without faulting it: a bounded wait that nothing completes
 gives up, the host reads FP8Q_ERR_TIMEOUT from the device error word, and the context
 stays usable. Invalid arguments are rejected before any launch."""
+import ctypes
+
 import pytest
 import torch
 
@@ -20,6 +22,8 @@ def fq():
 def test_bounded_wait_reports_timeout_and_context_survives(fq, oracle_mod):
     assert fq.device_error() == fq.FP8Q_OK
     assert fq.debug_wait_timeout(50_000_000) == fq.FP8Q_OK   # 50 ms limit
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert fq._lib.fp8q_last_device_error(stream) == fq.FP8Q_ERR_TIMEOUT  # reads, keeps
     assert fq.device_error(clear=True) == fq.FP8Q_ERR_TIMEOUT
     assert fq.device_error() == fq.FP8Q_OK                    # cleared
     x = workloads.activations_bf16((64, 256), 0, 900, "cuda")
