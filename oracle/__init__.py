@@ -52,8 +52,14 @@ def _load():
     global _lib
     if _lib is not None:
         return _lib
-    build()
-    lib = ctypes.CDLL(_LIB_PATH)
+    # FP8Q_ORACLE_LIB: load another build of fp8q_oracle.c instead (the mutation test
+    # of the pins points it at copies with a deliberately planted mistake)
+    other = os.environ.get("FP8Q_ORACLE_LIB")
+    if other:
+        lib = ctypes.CDLL(other)
+    else:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
     P = ctypes.c_void_p
     I = ctypes.c_int64
     F = ctypes.c_float

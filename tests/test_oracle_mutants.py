@@ -1,0 +1,87 @@
+"""Mutation check of the oracle's pins. Each case copies oracle/fp8q_oracle.c, plants one
+plausible mistake (a dropped term or factor, a wrong constant, sign, index or rounding
+rule, a swapped operand), builds the copy with the oracle's own flags, and runs the pin
+files that cover that function in a subprocess whose oracle loader uses the copy
+(FP8Q_ORACLE_LIB): at least one pin must fail. An unaltered copy, built and run the
+same way, must pass them all — so a failure is the mistake's doing, not the harness's."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "fp8q_oracle.c")
+
+E4M3, QUANT = "tests/test_oracle_e4m3.py", "tests/test_oracle_quant.py"
+NORM, BWD = "tests/test_oracle_norm_swiglu.py", "tests/test_oracle_backward.py"
+
+# (name, exact text in fp8q_oracle.c, replacement, pin files that must catch it)
+MUTANTS = [
+    ("e4m3 ties round up",
+     "else pick = (lo & 1) ? up : lo; /* tie: even mantissa",
+     "else pick = up; /* tie: even mantissa", [E4M3]),
+    ("scale = amax / 240",
+     "volatile float s = amax / 448.0f;", "volatile float s = amax / 240.0f;", [QUANT]),
+    ("rmsnorm without eps",
+     "double r = 1.0 / sqrt(ms + (double)eps);", "double r = 1.0 / sqrt(ms);", [NORM]),
+    ("rmsnorm without gamma",
+     "volatile float t2 = t1 * oracle_bf16_to_f32(gamma[c]);", "volatile float t2 = t1;", [NORM]),
+    ("swiglu gate and up swapped",
+     "oracle_swiglu_one(gu[m * ldgu + c], gu[m * ldgu + I + c])",
+     "oracle_swiglu_one(gu[m * ldgu + I + c], gu[m * ldgu + c])", [NORM]),
+    ("exp: 1/6 coefficient rounded",
+     "const float C3 = 0x1.555556p-3f;", "const float C3 = 0x1.5p-3f;", [NORM]),
+    ("swiglu backward without 1 + g(1 - sig)",
+     "volatile float t3 = 1.0f + t2;", "volatile float t3 = 1.0f;", [BWD]),
+    ("swiglu backward sig = g / d",
+     "volatile float sig = 1.0f / d;", "volatile float sig = g / d;", [BWD]),
+    ("rmsnorm backward k with r^2",
+     "    kd = kd * (double)r;\n    kd = kd * (double)r;\n", "    kd = kd * (double)r;\n", [BWD]),
+    ("rmsnorm backward without the residual",
+     "oracle_bf16_to_f32(dxb) + oracle_bf16_to_f32(dres[m * H + j]);",
+     "oracle_bf16_to_f32(dxb);", [BWD]),
+    ("dgamma without r",
+     "volatile float xr = oracle_bf16_to_f32(x[m * H + j]) * rr[m];",
+     "volatile float xr = oracle_bf16_to_f32(x[m * H + j]);", [BWD]),
+    ("128x1 column group rows mis-indexed",
+     "dy[(mb * 128 + i) * lddy + n]", "dy[(mb + i) * lddy + n]", [QUANT]),
+    ("requantizer drops the row scale",
+     "volatile float v = s[(k / 128) * lds + m] * dec;", "volatile float v = dec;", [QUANT]),
+]
+
+
+def _build_copy(tmp_path, name, text):
+    src = tmp_path / (name + ".c")
+    src.write_text(text)
+    lib = tmp_path / (name + ".so")
+    subprocess.check_call(["gcc", *oracle.GCC_FLAGS, str(src), "-o", str(lib), "-lm"])
+    return str(lib)
+
+
+def _run_pins(lib, files):
+    env = dict(os.environ, FP8Q_ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", *files, "-x", "-q", "-m", "not gpu",
+                        "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=600)
+    return r.returncode, r.stdout[-2000:]
+
+
+def test_unaltered_copy_passes_every_pin_file(tmp_path):
+    with open(SRC) as f:
+        text = f.read()
+    lib = _build_copy(tmp_path, "unaltered", text)
+    code, out = _run_pins(lib, [E4M3, QUANT, NORM, BWD])
+    assert code == 0, out
+
+
+@pytest.mark.parametrize("name,old,new,files", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_fails_a_pin(tmp_path, name, old, new, files):
+    with open(SRC) as f:
+        text = f.read()
+    assert text.count(old) == 1, "mutation site not unique: %r" % old
+    lib = _build_copy(tmp_path, "mutant", text.replace(old, new))
+    code, out = _run_pins(lib, files)
+    assert code != 0, "no pin caught the mistake %r:\n%s" % (name, out)
