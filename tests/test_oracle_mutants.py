@@ -17,6 +17,7 @@ SRC = os.path.join(ROOT, "oracle", "fp8q_oracle.c")
 
 E4M3, QUANT = "tests/test_oracle_e4m3.py", "tests/test_oracle_quant.py"
 NORM, BWD = "tests/test_oracle_norm_swiglu.py", "tests/test_oracle_backward.py"
+GEMM = "tests/test_oracle_gemm.py"
 
 # (name, exact text in fp8q_oracle.c, replacement, pin files that must catch it)
 MUTANTS = [
@@ -50,7 +51,38 @@ MUTANTS = [
      "dy[(mb * 128 + i) * lddy + n]", "dy[(mb + i) * lddy + n]", [QUANT]),
     ("requantizer drops the row scale",
      "volatile float v = s[(k / 128) * lds + m] * dec;", "volatile float v = dec;", [QUANT]),
+    ("weight block scale transposed",
+     "s[((r0 + i) / 128) * KB + k / 128]", "s[(k / 128) * KB + (r0 + i) / 128]", [GEMM]),
 ]
+
+# The same for the GEMM definitions in oracle/__init__.py (numpy): the module's source,
+# with the mistake, is executed again in the module's own namespace before the pins run.
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
+PY_MUTANTS = [
+    ("forward without the activation scale",
+     "A = dequant_rows(qa, sa, r0, nr)", "A = dequant_rows(qa, np.ones_like(sa), r0, nr)", [GEMM]),
+    ("DGrad against the reversed weight rows",
+     "return A @ W, np.abs(A) @ np.abs(W)", "return A @ W[::-1], np.abs(A) @ np.abs(W)", [GEMM]),
+    ("WGrad with the X operand's scales doubled",
+     "B = dequant_cols(qxT, sx_c)                 # [K, M]",
+     "B = dequant_cols(qxT, sx_c * 2)             # [K, M]", [GEMM]),
+    ("GEMM without the transposed operand",
+     "return a @ b.T, np.abs(a) @ np.abs(b).T", "return a @ b[::-1].T, np.abs(a) @ np.abs(b).T",
+     [GEMM]),
+]
+
+_PY_RUNNER = """
+import sys
+sys.path.insert(0, {root!r})
+import numpy as np
+import pytest
+import oracle
+src = open({src!r}).read()
+assert src.count({old!r}) == 1, "mutation site not unique"
+oracle._lib = None
+exec(compile(src.replace({old!r}, {new!r}), {src!r}, "exec"), oracle.__dict__)
+sys.exit(pytest.main({files!r} + ["-x", "-q", "-m", "not gpu", "-p", "no:cacheprovider"]))
+"""
 
 
 def _build_copy(tmp_path, name, text):
@@ -84,4 +116,23 @@ def test_planted_mistake_fails_a_pin(tmp_path, name, old, new, files):
     assert text.count(old) == 1, "mutation site not unique: %r" % old
     lib = _build_copy(tmp_path, "mutant", text.replace(old, new))
     code, out = _run_pins(lib, files)
+    assert code != 0, "no pin caught the mistake %r:\n%s" % (name, out)
+
+
+def _run_py(old, new, files):
+    code = _PY_RUNNER.format(root=ROOT, src=PY_SRC, old=old, new=new, files=files)
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    return r.returncode, r.stdout[-2000:] + r.stderr[-1000:]
+
+
+def test_unaltered_module_passes_the_gemm_pins():
+    # the runner with a no-op replacement: the harness itself does not fail the pins
+    code, out = _run_py("def gemm_nt(", "def gemm_nt(", [GEMM])
+    assert code == 0, out
+
+
+@pytest.mark.parametrize("name,old,new,files", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_planted_gemm_mistake_fails_a_pin(name, old, new, files):
+    code, out = _run_py(old, new, files)
     assert code != 0, "no pin caught the mistake %r:\n%s" % (name, out)
