@@ -167,3 +167,21 @@ def test_validation_wgrad_acc_f32():
     assert call(f, A, B, C, D, 128, 128, 128, E, 126, NUL) == 2       # lddw < K
     assert call(f, A, B, C, D, 128, 128, 256, E, 258, NUL) == 3       # lddw % 4
     assert call(f, A, B, C, NUL, 128, 128, 128, E, 128, NUL) == 1
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """No fallback: a copy of the package without libfp8q.so refuses to import."""
+    import shutil
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "fp8_block_scaled_08_b200")
+    dst = tmp_path / "fp8_block_scaled_08_b200"
+    dst.mkdir()
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            shutil.copy(os.path.join(pkg, name), dst / name)
+    r = subprocess.run([sys.executable, "-c", "import fp8_block_scaled_08_b200"],
+                       cwd=str(tmp_path), capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libfp8q.so is not built" in r.stderr
