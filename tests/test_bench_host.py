@@ -60,3 +60,48 @@ def test_peaks_reader():
     p = bench.read_peaks()
     assert p["hbm_gbs"] > 1000 and p["bf16_tflops"] > 100
     assert p["source"] in ("measured", "fallback")
+
+
+class _StubBinding:
+    """Records the binding calls a layer step makes (no device, no kernels)."""
+
+    def __init__(self):
+        self.calls = []
+
+    def lds_for(self, m):
+        return (m + 3) // 4 * 4
+
+    def rmsnorm_bwd_workspace_bytes(self, M, H):
+        return 16
+
+    def __getattr__(self, name):
+        def record(*args, **kwargs):
+            self.calls.append(name)
+        return record
+
+
+@pytest.mark.parametrize("saved,backward,launches,grads", [
+    ("fp8", "a6", 28, {"qkv", "o", "gate_up", "down"}),
+    ("dual", "a6", 26, {"qkv", "o", "gate_up", "down"}),
+    ("fp8", "fused", 32, {"down", "qkv"}),
+    ("dual", "fused", 30, {"down", "qkv"})])
+def test_layer_step_modes_on_a_stub(saved, backward, launches, grads):
+    """The four step variants: kernel launches per step, which upstream gradients enter
+    from outside, and a byte count for every quantizer kind the step times."""
+    import dataclasses
+    fq = _StubBinding()
+    wl = dataclasses.replace(workloads.LLAMA_LAYER, tokens=256)
+    step = bench.LayerStep(fq, wl, "cpu", saved=saved, backward=backward)
+    fq.calls.clear()
+    step.run()
+    assert step.launches_per_step == launches
+    assert set(step.grad_inputs()) == grads
+    kinds = set(step.quant_bytes_by_kind())
+    called = set(fq.calls) - {"linear_fwd", "linear_dgrad", "linear_wgrad"}
+    # every quantizer entry point the step calls has its bytes accounted for (the
+    # option-B attention-output quantizer is a6 under its own timing name)
+    assert called - {"transpose_quant_bf16"} <= kinds
+    assert ("transpose_quant_fp8" in kinds) == (saved == "fp8")
+    assert ("swiglu_bwd_quant_dual" in kinds) == (backward == "fused")
+    assert fq.calls.count("linear_fwd") == 4 and fq.calls.count("linear_wgrad") == 4
+    assert fq.calls.count("linear_dgrad") == 4
