@@ -11,6 +11,14 @@ head_dim 128, intermediate 14336):
 That is 28 kernel launches and 10.72 TFLOP of FP8 GEMM work per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--saved fp8|dual] [--backward a6|fused]
+                    [--case NAME]
+
+--saved dual: the producers emit both groupings of their BF16 output (no FP8
+requantization). --backward fused: the SwiGLU and RMSNorm backward producers emit the
+gradient codes of the preceding linears (a chained backward; only the QKV gradient,
+from attention, and the gradient from the layer above enter from outside). --case runs
+one kernel family once, for profiling.
 
 With N > 1 (torchrun, one rank per GPU) every rank runs its own token batch: weak
 scaling, no collective on the data path; the step time is the max over ranks.
