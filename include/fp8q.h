@@ -126,7 +126,7 @@ fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, int64_t N,
                                       int64_t lds_row, uint8_t* q_colT, float* s_col,
                                       void* stream);
 
-/* Option B for the saved activations (the survey's next row f2): the producer emits both
+/* "Option B" for the saved activations: the producer emits both
  * groupings from its BF16 output, so WGrad takes 128x1 codes of the BF16 values instead
  * of re-quantizing the saved FP8 tensor (fp8q_transpose_quant_fp8).
  * ("Esquema de Cuantización": FP8 saved activations produced by the preceding operator;
@@ -151,8 +151,8 @@ fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int64_t I, int
                                    uint8_t* q_row, float* s_row, int64_t lds_row,
                                    uint8_t* q_colT, float* s_col, void* stream);
 
-/* Backward producers in BF16 with the gradient quantizer fused behind them (the
- * survey's next row f1). "Esquema de Cuantización" keeps gradients between operators
+/* Backward producers in BF16 with the gradient quantizer fused behind them.
+ * "Esquema de Cuantización" keeps gradients between operators
  * in BF16 and runs DGrad / WGrad in FP8 (1x128 and 128x1 for WGrad); the page gives no
  * formula for the operators' own backward, so these are their derivatives with the
  * fp32 rounding sequence stated below. The gradient that the preceding linear layer
@@ -282,8 +282,8 @@ fp8q_status fp8q_linear_wgrad(const uint8_t* qdyT, const float* sdy_c, const uin
                               const float* sx_c, int64_t M, int64_t N, int64_t K,
                               uint16_t* dw, int64_t lddw, void* stream);
 
-/* WGrad accumulated in fp32 (the survey's next row f3: an fp32 accumulate-into-dW
- * option, for gradient accumulation over micro-batches): as fp8q_linear_wgrad, but
+/* WGrad accumulated in fp32 (an accumulate-into-dW option, for gradient accumulation
+ * over micro-batches): as fp8q_linear_wgrad, but
  *   dw[n,k] = fl32(dw[n,k] + acc[n,k])
  * where acc is the same fp32 accumulator fp8q_linear_wgrad rounds to BF16; dw [N][K]
  * fp32 (row stride lddw elements, lddw % 4 == 0) is read and written once per element by

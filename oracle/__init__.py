@@ -237,8 +237,8 @@ def transpose_quant_bf16(dy, lds_row: int | None = None, want_row: bool = True):
 
 
 def rmsnorm_quant_dual(x, gamma, eps: float, lds_row: int | None = None):
-    """Saved activations in both groupings from BF16 (the survey's option B for the RMSNorm
-    producer): y = RMSNorm(x) * gamma rounded to BF16 as in rmsnorm_quant, then y
+    """Saved activations in both groupings from BF16 ("option B" for the RMSNorm producer:
+    no FP8 requantization): y = RMSNorm(x) * gamma rounded to BF16 as in rmsnorm_quant, then y
     quantized 1x128 along rows (forward) and 128x1 along columns, stored transposed
     (WGrad), plus the per-row reciprocal RMS r. Returns (q_row, s_row, q_colT, s_col, r)."""
     x = _bf16(x)

@@ -1,5 +1,5 @@
-"""Backward producers with the gradient quantizer fused behind them (the survey's NEXT row
-f1) against the oracle through the C ABI: the SwiGLU backward bit for bit (gradient,
+"""Backward producers with the gradient quantizer fused behind them, against the oracle
+through the C ABI: the SwiGLU backward bit for bit (gradient,
 codes, scales); the RMSNorm backward's BF16 gradient within one BF16 ulp (its fp64 sums
 are blocked on the GPU, sequential in the oracle), its codes and scales bit for bit
 against the oracle's quantization of the kernel's own gradient, dgamma within fp32

@@ -1,4 +1,4 @@
-"""WGrad accumulated into an fp32 dW (the survey's NEXT row f3 option): dw += the fp32
+"""WGrad accumulated into an fp32 dW (gradient accumulation): dw += the fp32
 accumulator, against the oracle (dw_in + the fp64 product, within one fp32 ulp of the
 sum + 1e-5 * sum |a b|), two calls summing, the BF16 WGrad equal to the BF16 rounding of
 the accumulator added to zero, an N tail, and the full Llama-3.1-8B gate/up shape on

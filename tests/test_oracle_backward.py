@@ -1,5 +1,5 @@
-"""Pins of the oracle's BF16 backward producers (SwiGLU and RMSNorm, the survey's NEXT
-row f1) against torch fp64 autograd, closed forms, exact scaling identities and the
+"""Pins of the oracle's BF16 backward producers (SwiGLU and RMSNorm) against torch
+fp64 autograd, closed forms, exact scaling identities and the
 independently pinned forward producers. The pages ("Resumen Técnico: Jet-RL",
 «Esquema de Cuantización») fix only that gradients between operators stay BF16; the
 formulas are the operators' derivatives."""

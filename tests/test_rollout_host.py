@@ -1,4 +1,4 @@
-"""Host logic of the rollout weight refresh (the survey's NEXT row f4) without a GPU:
+"""Host logic of the per-step rollout weight refresh without a GPU:
 the packed layout, and the distribution on two gloo ranks — rank 0 fills the buffer with
 the oracle's 128x128 quantization of seeded BF16 masters (standing in for the library's
 quantizer, which needs a GPU), one broadcast, and rank 1 holds exactly those codes and
