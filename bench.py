@@ -133,7 +133,7 @@ class LayerStep:
         wl_seeded = workloads.Workload(**{**wl.__dict__, "seed": wl.seed + seed_offset})
         self.inp = inp = workloads.layer_inputs(wl_seeded, device, with_grads=not forward_only)
         lds = fq.lds_for(M)
-        H, I = L.hidden, L.intermediate
+        H = L.hidden
         e = lambda *s, dt=torch.uint8: torch.empty(s, dtype=dt, device=device)  # noqa: E731
         f32 = torch.float32
         bf = torch.bfloat16
@@ -188,7 +188,7 @@ class LayerStep:
             self.launch_count = self._launched
 
     def _run(self, timer, stream, only):
-        fq, inp, lin, M = self.fq, self.inp, self.lin, self.M
+        fq, inp, lin = self.fq, self.inp, self.lin
         self.only = only
         self.timer = timer
         k = self._k
@@ -197,7 +197,6 @@ class LayerStep:
             k("quant_weight_128x128",
               lambda d=d, name=name: fq.quant_weight_128x128(inp["w"][name], d["qw"], d["sw"],
                                                              d["qwT"], stream), timer)
-        q, o, gu, dn = lin["qkv"], lin["o"], lin["gate_up"], lin["down"]
         if self.saved == "dual":
             self._forward_dual(k, stream)
         else:
@@ -334,7 +333,7 @@ class LayerStep:
     def quant_bytes_by_kind(self):
         M = self.M
         L = self.L
-        H, I = L.hidden, L.intermediate
+        H = L.hidden
         qo = L.q_heads * L.head_dim
         w_elems = sum(d["N"] * d["K"] for d in self.lin.values())
         dy_elems = sum(M * d["N"] for d in self.lin.values())
