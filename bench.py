@@ -333,7 +333,7 @@ class LayerStep:
     def quant_bytes_by_kind(self):
         M = self.M
         L = self.L
-        H = L.hidden
+        H, I = L.hidden, L.intermediate
         qo = L.q_heads * L.head_dim
         w_elems = sum(d["N"] * d["K"] for d in self.lin.values())
         dy_elems = sum(M * d["N"] for d in self.lin.values())
