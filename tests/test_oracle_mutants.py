@@ -55,8 +55,9 @@ MUTANTS = [
      "s[((r0 + i) / 128) * KB + k / 128]", "s[(k / 128) * KB + (r0 + i) / 128]", [GEMM]),
 ]
 
-# The same for the GEMM definitions in oracle/__init__.py (numpy): the module's source,
-# with the mistake, is executed again in the module's own namespace before the pins run.
+# The same for the definitions in oracle/__init__.py (the numpy GEMMs and the dual /
+# backward compositions): the module's source, with the mistake, is executed again in
+# the module's own namespace before the pins run.
 PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
 PY_MUTANTS = [
     ("forward without the activation scale",
@@ -69,6 +70,18 @@ PY_MUTANTS = [
     ("GEMM without the transposed operand",
      "return a @ b.T, np.abs(a) @ np.abs(b).T", "return a @ b[::-1].T, np.abs(a) @ np.abs(b).T",
      [GEMM]),
+    ("RMSNorm dual emission quantizes x instead of y",
+     "_, _, qT, sT = transpose_quant_bf16(y, want_row=False)",
+     "_, _, qT, sT = transpose_quant_bf16(x, want_row=False)", [NORM]),
+    ("SwiGLU dual emission quantizes the gate instead of h",
+     "_, _, qT, sT = transpose_quant_bf16(h, want_row=False)",
+     "_, _, qT, sT = transpose_quant_bf16(_bf16(gu)[:, :h.shape[1]], want_row=False)", [NORM]),
+    ("SwiGLU backward quantizes gu instead of its gradient",
+     "q, s, qT, sT = transpose_quant_bf16(dgu, lds_row)",
+     "q, s, qT, sT = transpose_quant_bf16(_bf16(gu), lds_row)", [BWD]),
+    ("RMSNorm backward quantizes dy instead of its output",
+     "q, s, qT, sT = transpose_quant_bf16(out, lds_row)",
+     "q, s, qT, sT = transpose_quant_bf16(_bf16(dy), lds_row)", [BWD]),
 ]
 
 _PY_RUNNER = """
@@ -126,13 +139,13 @@ def _run_py(old, new, files):
     return r.returncode, r.stdout[-2000:] + r.stderr[-1000:]
 
 
-def test_unaltered_module_passes_the_gemm_pins():
+def test_unaltered_module_passes_the_pins():
     # the runner with a no-op replacement: the harness itself does not fail the pins
-    code, out = _run_py("def gemm_nt(", "def gemm_nt(", [GEMM])
+    code, out = _run_py("def gemm_nt(", "def gemm_nt(", [GEMM, NORM, BWD])
     assert code == 0, out
 
 
 @pytest.mark.parametrize("name,old,new,files", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
-def test_planted_gemm_mistake_fails_a_pin(name, old, new, files):
+def test_planted_python_mistake_fails_a_pin(name, old, new, files):
     code, out = _run_py(old, new, files)
     assert code != 0, "no pin caught the mistake %r:\n%s" % (name, out)
