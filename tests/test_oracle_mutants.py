@@ -98,6 +98,10 @@ sys.exit(pytest.main({files!r} + ["-x", "-q", "-m", "not gpu", "-p", "no:cachepr
 """
 
 
+_JOBS = 8                       # subprocesses at a time
+_ENV = dict(os.environ, OMP_NUM_THREADS="2")
+
+
 def _build_copy(tmp_path, name, text):
     src = tmp_path / (name + ".c")
     src.write_text(text)
@@ -107,45 +111,71 @@ def _build_copy(tmp_path, name, text):
 
 
 def _run_pins(lib, files):
-    env = dict(os.environ, FP8Q_ORACLE_LIB=lib)
+    env = dict(_ENV, FP8Q_ORACLE_LIB=lib)
     r = subprocess.run([sys.executable, "-m", "pytest", *files, "-x", "-q", "-m", "not gpu",
                         "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True,
                        text=True, timeout=600)
     return r.returncode, r.stdout[-2000:]
 
 
-def test_unaltered_copy_passes_every_pin_file(tmp_path):
+@pytest.fixture(scope="module")
+def c_results(tmp_path_factory):
+    """Builds the unaltered copy and every C mutant, runs their pin files concurrently:
+    {name: (return code, output tail)} ("" is the unaltered copy)."""
+    from concurrent.futures import ThreadPoolExecutor
+    tmp = tmp_path_factory.mktemp("c_mutants")
     with open(SRC) as f:
         text = f.read()
-    lib = _build_copy(tmp_path, "unaltered", text)
-    code, out = _run_pins(lib, [E4M3, QUANT, NORM, BWD])
+    jobs = {"": (text, [E4M3, QUANT, NORM, BWD])}
+    for i, (name, old, new, files) in enumerate(MUTANTS):
+        assert text.count(old) == 1, "mutation site not unique: %r" % old
+        jobs[name] = (text.replace(old, new), files)
+
+    def run(item):
+        name, (src, files) = item
+        lib = _build_copy(tmp, "m%d" % abs(hash(name)), src)
+        return name, _run_pins(lib, files)
+
+    with ThreadPoolExecutor(_JOBS) as ex:
+        return dict(ex.map(run, jobs.items()))
+
+
+def test_unaltered_copy_passes_every_pin_file(c_results):
+    code, out = c_results[""]
     assert code == 0, out
 
 
-@pytest.mark.parametrize("name,old,new,files", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_planted_mistake_fails_a_pin(tmp_path, name, old, new, files):
-    with open(SRC) as f:
-        text = f.read()
-    assert text.count(old) == 1, "mutation site not unique: %r" % old
-    lib = _build_copy(tmp_path, "mutant", text.replace(old, new))
-    code, out = _run_pins(lib, files)
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_planted_mistake_fails_a_pin(c_results, name):
+    code, out = c_results[name]
     assert code != 0, "no pin caught the mistake %r:\n%s" % (name, out)
 
 
 def _run_py(old, new, files):
     code = _PY_RUNNER.format(root=ROOT, src=PY_SRC, old=old, new=new, files=files)
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
-                       timeout=600)
+                       timeout=600, env=_ENV)
     return r.returncode, r.stdout[-2000:] + r.stderr[-1000:]
 
 
-def test_unaltered_module_passes_the_pins():
-    # the runner with a no-op replacement: the harness itself does not fail the pins
-    code, out = _run_py("def gemm_nt(", "def gemm_nt(", [GEMM, NORM, BWD])
+@pytest.fixture(scope="module")
+def py_results():
+    """Runs the unaltered module (a no-op replacement) and every Python mutant
+    concurrently: {name: (return code, output tail)}."""
+    from concurrent.futures import ThreadPoolExecutor
+    jobs = {"": ("def gemm_nt(", "def gemm_nt(", [GEMM, NORM, BWD])}
+    for name, old, new, files in PY_MUTANTS:
+        jobs[name] = (old, new, files)
+    with ThreadPoolExecutor(_JOBS) as ex:
+        return dict(ex.map(lambda kv: (kv[0], _run_py(*kv[1])), jobs.items()))
+
+
+def test_unaltered_module_passes_the_pins(py_results):
+    code, out = py_results[""]
     assert code == 0, out
 
 
-@pytest.mark.parametrize("name,old,new,files", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
-def test_planted_python_mistake_fails_a_pin(name, old, new, files):
-    code, out = _run_py(old, new, files)
+@pytest.mark.parametrize("name", [m[0] for m in PY_MUTANTS])
+def test_planted_python_mistake_fails_a_pin(py_results, name):
+    code, out = py_results[name]
     assert code != 0, "no pin caught the mistake %r:\n%s" % (name, out)
