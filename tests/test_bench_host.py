@@ -105,3 +105,26 @@ def test_layer_step_modes_on_a_stub(saved, backward, launches, grads):
     assert ("swiglu_bwd_quant_dual" in kinds) == (backward == "fused")
     assert fq.calls.count("linear_fwd") == 4 and fq.calls.count("linear_wgrad") == 4
     assert fq.calls.count("linear_dgrad") == 4
+
+
+def test_reference_arm_prints_its_line():
+    """`bench.py --impl reference` (the oracle on the host cores, a bounded sample per
+    step) prints one JSON line with the contract's keys; it needs no GPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], cwd=root, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["higher_is_better"]
+    assert line["steps"] == 1 and line["warmup"] == 3
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
