@@ -138,6 +138,31 @@ def _dense(t, name):
         raise ValueError("%s must be contiguous" % name)
 
 
+def _groups(n: int) -> int:
+    """Number of 128-wide groups covering n elements."""
+    return (int(n) + 127) // 128
+
+
+def _shape(t, shape, dtype, name):
+    """Operand `name` must be a `dtype` tensor of exactly `shape` (checked before any
+    pointer reaches the C side, whose tensor maps and stores trust these extents)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dtype != dtype or tuple(t.shape) != tuple(int(d) for d in shape):
+        raise ValueError("%s must be a %s tensor of shape %s, got %s %s" % (
+            name, dtype, tuple(int(d) for d in shape), tuple(t.shape), t.dtype))
+
+
+def _scales_1x128(s, groups, rows, name):
+    """1x128 scale array: fp32 [groups, lds] with lds >= rows (a multiple of 4 is
+    checked by the library)."""
+    if not isinstance(s, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if s.dtype != torch.float32 or s.dim() != 2 or s.shape[0] != groups or s.shape[1] < rows:
+        raise ValueError("%s must be a float32 tensor [%d, >=%d], got %s %s" % (
+            name, groups, rows, tuple(s.shape), s.dtype))
+
+
 def lds_for(m: int) -> int:
     """Smallest legal leading dimension of a 1x128 scale array for M rows."""
     return (max(m, 1) + 3) // 4 * 4
@@ -157,6 +182,8 @@ def quant_act_1x128(x, q, s, stream=None):
     _want(x, torch.bfloat16, 2, "x"); _want(q, torch.uint8, 2, "q"); _want(s, torch.float32, 2, "s")
     _dense(q, "q"); _dense(s, "s")
     M, K = x.shape
+    _shape(q, (M, K), torch.uint8, "q")
+    _scales_1x128(s, _groups(K), M, "s")
     _check(_lib.fp8q_quant_act_1x128(_ptr(x), M, K, _rows_dense(x, "x"), _ptr(q), _ptr(s),
                                      s.shape[1], _stream(stream)), "fp8q_quant_act_1x128")
 
@@ -168,6 +195,10 @@ def quant_weight_128x128(w, q, s, qT=None, stream=None):
     if qT is not None:
         _want(qT, torch.uint8, 2, "qT"); _dense(qT, "qT")
     N, K = w.shape
+    _shape(q, (N, K), torch.uint8, "q")
+    _shape(s, (_groups(N), _groups(K)), torch.float32, "s")
+    if qT is not None:
+        _shape(qT, (K, N), torch.uint8, "qT")
     _check(_lib.fp8q_quant_weight_128x128(_ptr(w), N, K, _rows_dense(w, "w"), _ptr(q), _ptr(s),
                                           _ptr(qT), _stream(stream)), "fp8q_quant_weight_128x128")
 
@@ -178,6 +209,9 @@ def rmsnorm_quant(x, gamma, eps, q, s, stream=None):
     _want(q, torch.uint8, 2, "q"); _want(s, torch.float32, 2, "s")
     _dense(gamma, "gamma"); _dense(q, "q"); _dense(s, "s")
     M, H = x.shape
+    _shape(gamma, (H,), torch.bfloat16, "gamma")
+    _shape(q, (M, H), torch.uint8, "q")
+    _scales_1x128(s, _groups(H), M, "s")
     _check(_lib.fp8q_rmsnorm_quant(_ptr(x), _ptr(gamma), M, H, _rows_dense(x, "x"), float(eps),
                                    _ptr(q), _ptr(s), s.shape[1], _stream(stream)),
            "fp8q_rmsnorm_quant")
@@ -188,6 +222,10 @@ def swiglu_quant(gu, q, s, stream=None):
     _want(gu, torch.bfloat16, 2, "gu"); _want(q, torch.uint8, 2, "q"); _want(s, torch.float32, 2, "s")
     _dense(q, "q"); _dense(s, "s")
     M, I2 = gu.shape
+    if I2 % 2:
+        raise ValueError("gu must be [M, 2I] (gate | up), got %s" % (tuple(gu.shape),))
+    _shape(q, (M, I2 // 2), torch.uint8, "q")
+    _scales_1x128(s, _groups(I2 // 2), M, "s")
     _check(_lib.fp8q_swiglu_quant(_ptr(gu), M, I2 // 2, _rows_dense(gu, "gu"), _ptr(q), _ptr(s),
                                   s.shape[1], _stream(stream)), "fp8q_swiglu_quant")
 
@@ -204,6 +242,11 @@ def transpose_quant_bf16(dy, q_row, s_row, q_colT, s_col, stream=None):
         _dense(q_row, "q_row"); _dense(s_row, "s_row")
         lds_row = s_row.shape[1]
     M, N = dy.shape
+    if q_row is not None:
+        _shape(q_row, (M, N), torch.uint8, "q_row")
+        _scales_1x128(s_row, _groups(N), M, "s_row")
+    _shape(q_colT, (N, M), torch.uint8, "q_colT")
+    _shape(s_col, (_groups(M), N), torch.float32, "s_col")
     _check(_lib.fp8q_transpose_quant_bf16(_ptr(dy), M, N, _rows_dense(dy, "dy"), _ptr(q_row),
                                           _ptr(s_row), lds_row, _ptr(q_colT), _ptr(s_col),
                                           _stream(stream)), "fp8q_transpose_quant_bf16")
@@ -217,6 +260,9 @@ def transpose_quant_fp8(q, s, qT, sT, stream=None):
     for t, n in ((q, "q"), (s, "s"), (qT, "qT"), (sT, "sT")):
         _dense(t, n)
     M, K = q.shape
+    _scales_1x128(s, _groups(K), M, "s")
+    _shape(qT, (K, M), torch.uint8, "qT")
+    _shape(sT, (_groups(M), K), torch.float32, "sT")
     _check(_lib.fp8q_transpose_quant_fp8(_ptr(q), _ptr(s), M, K, s.shape[1], _ptr(qT), _ptr(sT),
                                          _stream(stream)), "fp8q_transpose_quant_fp8")
 
@@ -229,6 +275,12 @@ def rmsnorm_quant_dual(x, gamma, eps, q_row, s_row, q_colT, s_col, rstd, stream=
                  (rstd, "rstd")):
         _dense(t, n)
     M, H = x.shape
+    _shape(gamma, (H,), torch.bfloat16, "gamma")
+    _shape(q_row, (M, H), torch.uint8, "q_row")
+    _scales_1x128(s_row, _groups(H), M, "s_row")
+    _shape(q_colT, (H, M), torch.uint8, "q_colT")
+    _shape(s_col, (_groups(M), H), torch.float32, "s_col")
+    _shape(rstd, (M,), torch.float32, "rstd")
     _check(_lib.fp8q_rmsnorm_quant_dual(_ptr(x), _ptr(gamma), M, H, _rows_dense(x, "x"),
                                         float(eps), _ptr(q_row), _ptr(s_row), s_row.shape[1],
                                         _ptr(q_colT), _ptr(s_col), _ptr(rstd), _stream(stream)),
@@ -252,6 +304,13 @@ def swiglu_quant_dual(gu, q_row, s_row, q_colT, s_col, stream=None):
     for t, n in ((q_row, "q_row"), (s_row, "s_row"), (q_colT, "q_colT"), (s_col, "s_col")):
         _dense(t, n)
     M, I2 = gu.shape
+    if I2 % 2:
+        raise ValueError("gu must be [M, 2I] (gate | up), got %s" % (tuple(gu.shape),))
+    I = I2 // 2
+    _shape(q_row, (M, I), torch.uint8, "q_row")
+    _scales_1x128(s_row, _groups(I), M, "s_row")
+    _shape(q_colT, (I, M), torch.uint8, "q_colT")
+    _shape(s_col, (_groups(M), I), torch.float32, "s_col")
     _check(_lib.fp8q_swiglu_quant_dual(_ptr(gu), M, I2 // 2, _rows_dense(gu, "gu"), _ptr(q_row),
                                        _ptr(s_row), s_row.shape[1], _ptr(q_colT), _ptr(s_col),
                                        _stream(stream)), "fp8q_swiglu_quant_dual")
@@ -281,6 +340,12 @@ def swiglu_bwd_quant_dual(gu, dh, q_row, s_row, q_colT, s_col, dgu=None, stream=
     M, I2 = gu.shape
     if dh.shape != (M, I2 // 2):
         raise ValueError("dh must be [M, I] for gu [M, 2I]")
+    _shape(q_row, (M, I2), torch.uint8, "q_row")
+    _scales_1x128(s_row, _groups(I2), M, "s_row")
+    _shape(q_colT, (I2, M), torch.uint8, "q_colT")
+    _shape(s_col, (_groups(M), I2), torch.float32, "s_col")
+    if dgu is not None:
+        _shape(dgu, (M, I2), torch.bfloat16, "dgu")
     _check(_lib.fp8q_swiglu_bwd_quant_dual(_ptr(gu), _ptr(dh), M, I2 // 2, _ptr(dgu), _ptr(q_row),
                                            _ptr(s_row), s_row.shape[1], _ptr(q_colT),
                                            _ptr(s_col), _stream(stream)),
@@ -320,6 +385,15 @@ def rmsnorm_bwd_quant_dual(x, gamma, dy, dres, eps, out, q_row, s_row, q_colT, s
     for t, n in ((dy, "dy"), (dres, "dres"), (out, "out")):
         if t is not None and t.shape != (M, H):
             raise ValueError("%s must have the shape of x" % n)
+    _shape(gamma, (H,), torch.bfloat16, "gamma")
+    _shape(q_row, (M, H), torch.uint8, "q_row")
+    _scales_1x128(s_row, _groups(H), M, "s_row")
+    _shape(q_colT, (H, M), torch.uint8, "q_colT")
+    _shape(s_col, (_groups(M), H), torch.float32, "s_col")
+    if dgamma is not None:
+        _shape(dgamma, (H,), torch.float32, "dgamma")
+    if workspace.dtype != torch.uint8:
+        raise ValueError("workspace must be a uint8 tensor")
     _check(_lib.fp8q_rmsnorm_bwd_quant_dual(
         _ptr(x), _ptr(gamma), _ptr(dy), _ptr(dres), M, H, float(eps), _ptr(out), _ptr(q_row),
         _ptr(s_row), s_row.shape[1], _ptr(q_colT), _ptr(s_col), _ptr(dgamma), _ptr(workspace),
@@ -342,13 +416,28 @@ def rmsnorm_bwd_quant_dual_alloc(x, gamma, dy, dres, eps, stream=None):
     return out, q, s, qT, sT, dg
 
 
+def _gemm_operands(qa, sa, qw, name_a, name_sa, name_w):
+    """Extents of a block-scaled product [M, N] = qa [M, K] x qw [N, K]^T: checks the
+    two code operands and the 1x128 row scales sa [K/128, >= M]; returns (M, N, K) for
+    the caller to check the block scales and the output against."""
+    if not isinstance(qa, torch.Tensor) or qa.dim() != 2 or qa.dtype != torch.uint8:
+        raise ValueError("%s must be a 2-D uint8 tensor" % name_a)
+    if not isinstance(qw, torch.Tensor) or qw.dim() != 2 or qw.dtype != torch.uint8:
+        raise ValueError("%s must be a 2-D uint8 tensor" % name_w)
+    M, K = qa.shape
+    N = qw.shape[0]
+    _shape(qw, (N, K), torch.uint8, name_w)
+    _scales_1x128(sa, _groups(K), M, name_sa)
+    return M, N, K
+
+
 def linear_fwd(qa, sa, qw, sw, y, stream=None):
     """a5: y BF16 [M,N] = block-scaled qa [M,K] x qw [N,K]^T."""
     for t, n in ((qa, "qa"), (sa, "sa"), (qw, "qw"), (sw, "sw")):
         _dense(t, n)
-    _want(y, torch.bfloat16, 2, "y")
-    M, K = qa.shape
-    N = qw.shape[0]
+    M, N, K = _gemm_operands(qa, sa, qw, "qa", "sa", "qw")
+    _shape(sw, (_groups(N), _groups(K)), torch.float32, "sw")
+    _shape(y, (M, N), torch.bfloat16, "y")
     _check(_lib.fp8q_linear_fwd(_ptr(qa), _ptr(sa), sa.shape[1], _ptr(qw), _ptr(sw), M, N, K,
                                 _ptr(y), _rows_dense(y, "y"), _stream(stream)), "fp8q_linear_fwd")
 
@@ -372,10 +461,10 @@ def linear_fwd_splitk(qa, sa, qw, sw, y, workspace, stream=None):
     is a uint8 device tensor from splitk_workspace (not shared by concurrent calls)."""
     for t, n in ((qa, "qa"), (sa, "sa"), (qw, "qw"), (sw, "sw")):
         _dense(t, n)
-    _want(y, torch.bfloat16, 2, "y")
+    M, N, K = _gemm_operands(qa, sa, qw, "qa", "sa", "qw")
+    _shape(sw, (_groups(N), _groups(K)), torch.float32, "sw")
+    _shape(y, (M, N), torch.bfloat16, "y")
     _want(workspace, torch.uint8, 1, "workspace")
-    M, K = qa.shape
-    N = qw.shape[0]
     _check(_lib.fp8q_linear_fwd_splitk(_ptr(qa), _ptr(sa), sa.shape[1], _ptr(qw), _ptr(sw), M, N,
                                        K, _ptr(y), _rows_dense(y, "y"), _ptr(workspace),
                                        workspace.numel(), _stream(stream)),
@@ -387,9 +476,9 @@ def linear_fwd_splitk_noalloc(qa, sa, qw, sw, y, stream=None):
     device must not overlap)."""
     for t, n in ((qa, "qa"), (sa, "sa"), (qw, "qw"), (sw, "sw")):
         _dense(t, n)
-    _want(y, torch.bfloat16, 2, "y")
-    M, K = qa.shape
-    N = qw.shape[0]
+    M, N, K = _gemm_operands(qa, sa, qw, "qa", "sa", "qw")
+    _shape(sw, (_groups(N), _groups(K)), torch.float32, "sw")
+    _shape(y, (M, N), torch.bfloat16, "y")
     _check(_lib.fp8q_linear_fwd_splitk_noalloc(_ptr(qa), _ptr(sa), sa.shape[1], _ptr(qw),
                                                _ptr(sw), M, N, K, _ptr(y), _rows_dense(y, "y"),
                                                _stream(stream)),
@@ -401,12 +490,27 @@ def linear_dgrad(qdy, sdy, qwT, sw, dx, stream=None):
     qwT [K,N])."""
     for t, n in ((qdy, "qdy"), (sdy, "sdy"), (qwT, "qwT"), (sw, "sw")):
         _dense(t, n)
-    _want(dx, torch.bfloat16, 2, "dx")
-    M, N = qdy.shape
-    K = qwT.shape[0]
+    # dx [M, K] = qdy [M, N] x qwT [K, N]^T: the product's reduction runs over N
+    M, K, N = _gemm_operands(qdy, sdy, qwT, "qdy", "sdy", "qwT")
+    _shape(sw, (_groups(N), _groups(K)), torch.float32, "sw")
+    _shape(dx, (M, K), torch.bfloat16, "dx")
     _check(_lib.fp8q_linear_dgrad(_ptr(qdy), _ptr(sdy), sdy.shape[1], _ptr(qwT), _ptr(sw), M, N,
                                   K, _ptr(dx), _rows_dense(dx, "dx"), _stream(stream)),
            "fp8q_linear_dgrad")
+
+
+def _wgrad_operands(qdyT, sdy_c, qxT, sx_c):
+    """Shapes of WGrad: qdyT [N, M] and qxT [K, M] (128x1 codes, transposed) with their
+    scales sdy_c [M/128, N] and sx_c [M/128, K]. Returns (N, M, K)."""
+    for t, n in ((qdyT, "qdyT"), (qxT, "qxT")):
+        if not isinstance(t, torch.Tensor) or t.dim() != 2 or t.dtype != torch.uint8:
+            raise ValueError("%s must be a 2-D uint8 tensor" % n)
+    N, M = qdyT.shape
+    K = qxT.shape[0]
+    _shape(qxT, (K, M), torch.uint8, "qxT")
+    _shape(sdy_c, (_groups(M), N), torch.float32, "sdy_c")
+    _shape(sx_c, (_groups(M), K), torch.float32, "sx_c")
+    return N, M, K
 
 
 def linear_wgrad(qdyT, sdy_c, qxT, sx_c, dw, stream=None):
@@ -414,9 +518,8 @@ def linear_wgrad(qdyT, sdy_c, qxT, sx_c, dw, stream=None):
     the 128x1 scales sdy_c [M/128,N] and sx_c [M/128,K]."""
     for t, n in ((qdyT, "qdyT"), (sdy_c, "sdy_c"), (qxT, "qxT"), (sx_c, "sx_c")):
         _dense(t, n)
-    _want(dw, torch.bfloat16, 2, "dw")
-    N, M = qdyT.shape
-    K = qxT.shape[0]
+    N, M, K = _wgrad_operands(qdyT, sdy_c, qxT, sx_c)
+    _shape(dw, (N, K), torch.bfloat16, "dw")
     _check(_lib.fp8q_linear_wgrad(_ptr(qdyT), _ptr(sdy_c), _ptr(qxT), _ptr(sx_c), M, N, K,
                                   _ptr(dw), _rows_dense(dw, "dw"), _stream(stream)),
            "fp8q_linear_wgrad")
@@ -426,11 +529,8 @@ def linear_wgrad_acc_f32(qdyT, sdy_c, qxT, sx_c, dw, stream=None):
     """WGrad accumulated in fp32: dw [N,K] (fp32) += the fp32 accumulator of linear_wgrad."""
     for t, n in ((qdyT, "qdyT"), (sdy_c, "sdy_c"), (qxT, "qxT"), (sx_c, "sx_c")):
         _dense(t, n)
-    _want(dw, torch.float32, 2, "dw")
-    N, M = qdyT.shape
-    K = qxT.shape[0]
-    if dw.shape[0] != N or dw.shape[1] != K:
-        raise ValueError("dw must be [N, K]")
+    N, M, K = _wgrad_operands(qdyT, sdy_c, qxT, sx_c)
+    _shape(dw, (N, K), torch.float32, "dw")
     _check(_lib.fp8q_linear_wgrad_acc_f32(_ptr(qdyT), _ptr(sdy_c), _ptr(qxT), _ptr(sx_c), M, N,
                                           K, _ptr(dw), _rows_dense(dw, "dw"), _stream(stream)),
            "fp8q_linear_wgrad_acc_f32")

@@ -48,6 +48,8 @@
 // Every mbarrier wait is bounded (kWaitLimitNs): a wait that gives up records
 // FP8Q_ERR_TIMEOUT in the device error word and both CTAs wind down.
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 
 #include "fp8q_device.cuh"
 #include "fp8q_host.h"
@@ -464,10 +466,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // number, or 0 on failure (the reason is in fp8q_last_error_message).
 template <bool kCol, bool kSplit, bool kAcc = false>
 int kernel_setup() {
-  static int pairs_for_device[64] = {0};
+  // written once per device under the lock; host threads may launch concurrently
+  static std::atomic<int> pairs_for_device[64];
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (pairs_for_device[dev]) return pairs_for_device[dev];
+  if (const int known = pairs_for_device[dev].load(std::memory_order_acquire)) return known;
+  std::lock_guard<std::mutex> lock(mu);
+  if (const int known = pairs_for_device[dev].load(std::memory_order_relaxed)) return known;
   const cudaError_t e = cudaFuncSetAttribute(
       gemm_kernel<kCol, kSplit, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
       static_cast<int>(kSmemBytes));
@@ -509,7 +515,7 @@ int kernel_setup() {
     cudaGetLastError();
     return 0;
   }
-  pairs_for_device[dev] = clusters;
+  pairs_for_device[dev].store(clusters, std::memory_order_release);
   return clusters;
 }
 

@@ -40,6 +40,7 @@
 // device error word and the CTA winds down.
 #include <algorithm>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 
 #include "fp8q_device.cuh"
@@ -367,12 +368,17 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(
 }
 
 // Per device and kernel variant: opt in to the shared memory the launch asks for.
+// Per device and kernel variant: the dynamic shared memory opted in so far (host threads
+// launching on different streams may get here at once: reads are atomic, updates locked).
 template <int kBN, bool kSplit>
 bool skinny_setup(size_t smem_bytes) {
-  static size_t opted[64] = {0};
+  static std::atomic<size_t> opted[64];
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (opted[dev] >= smem_bytes) return true;
+  if (opted[dev].load(std::memory_order_acquire) >= smem_bytes) return true;
+  std::lock_guard<std::mutex> lock(mu);
+  if (opted[dev].load(std::memory_order_relaxed) >= smem_bytes) return true;
   const cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel<kBN, kSplit>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem_bytes));
@@ -381,7 +387,7 @@ bool skinny_setup(size_t smem_bytes) {
     cudaGetLastError();
     return false;
   }
-  opted[dev] = smem_bytes;
+  opted[dev].store(smem_bytes, std::memory_order_release);
   return true;
 }
 

@@ -23,6 +23,7 @@
 // 1x128 / 128x1 WGrad grouping) and section "Implementación" (fused
 // activation/RMSNorm and transposition kernels).
 #include <algorithm>
+#include <atomic>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -1300,17 +1301,19 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
 
 // Resident CTAs per SM of a kernel (cached per device), for grid-stride/persistent grids.
 template <class Kernel>
-int resident_ctas(Kernel k, int threads, size_t dyn_smem, int* cache) {
+// `cache` is a per-device table owned by the caller; host threads may race to fill an
+// entry (with the same value), so entries are atomics.
+int resident_ctas(Kernel k, int threads, size_t dyn_smem, std::atomic<int>* cache) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
-  if (cache[dev]) return cache[dev];
+  if (const int known = cache[dev].load(std::memory_order_acquire)) return known;
   if (dyn_smem > 48 * 1024)
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn_smem));
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, dyn_smem) != cudaSuccess || n < 1)
     n = 1;
   cudaGetLastError();
-  cache[dev] = n;
+  cache[dev].store(n, std::memory_order_release);
   return n;
 }
 
@@ -1333,7 +1336,7 @@ extern "C" fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   const int64_t G = K / 128;
   const int64_t units = M * ((G + 1) / 2);
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(rowgroup_quant_kernel<ActSrc, 4>, 256, 0, occ);
   rowgroup_quant_kernel<ActSrc, 4><<<grid_for((units + 31) / 32, per_sm), 256, 0,
                                      static_cast<cudaStream_t>(stream)>>>(ActSrc{x, ldx}, M, G, q,
@@ -1349,7 +1352,7 @@ extern "C" fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t 
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   const int64_t G = I / 128;
   const int64_t units = M * ((G + 1) / 2);
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(rowgroup_quant_kernel<SwigluSrc, 2>, 256, 0, occ);
   rowgroup_quant_kernel<SwigluSrc, 2><<<grid_for((units + 15) / 16, per_sm), 256, 0,
                                         static_cast<cudaStream_t>(stream)>>>(
@@ -1374,7 +1377,7 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   // is faster (measured 3x at 16-256 rows, equal at 8192).
   if (M > 1024) {
     const int64_t ctas = (M + 7) / 8;  // one warp per row
-    static int occ[64];
+    static std::atomic<int> occ[64];
     const int per_sm = resident_ctas(rmsnorm_quant_warp2_kernel, 256, gsm, occ);
     rmsnorm_quant_warp2_kernel<<<grid_for(ctas, per_sm), 256, gsm, st>>>(x, gamma, M, H, ldx, eps,
                                                                          q, s, lds);
@@ -1400,7 +1403,7 @@ extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, i
     return FP8Q_ERR_UNSUPPORTED;
   unsigned* err = device_error_word();
   if (!err) return FP8Q_ERR_CUDA;
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(quant_weight_kernel, 256, kTileSmemBF16, occ);
   quant_weight_kernel<<<grid_for((N / 128) * (K / 128), per_sm), 256, kTileSmemBF16,
                         static_cast<cudaStream_t>(stream)>>>(tm, N, K, q, s, qT, err, kWaitLimitNs);
@@ -1420,7 +1423,7 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   constexpr size_t kSmem = direct_smem_bytes<GradDirect>();
   auto kern = direct_dual_kernel<GradDirect, kA6Batch, kA6MinBlocks>;
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (N / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
       GradDirect{dy, lddy}, M, N / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col, nullptr);
@@ -1443,7 +1446,7 @@ extern "C" fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s
     return FP8Q_ERR_UNSUPPORTED;
   unsigned* err = device_error_word();
   if (!err) return FP8Q_ERR_CUDA;
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(transpose_quant_fp8_kernel, 256, kTileSmemFP8, occ);
   transpose_quant_fp8_kernel<<<grid_for((M / 128) * (K / 128), per_sm), 256, kTileSmemFP8,
                                static_cast<cudaStream_t>(stream)>>>(tmq, tms, M, K, qT, sT, err,
@@ -1473,7 +1476,7 @@ extern "C" fp8q_status fp8q_rmsnorm_quant_dual(const uint16_t* x, const uint16_t
   if (s1 != FP8Q_OK) return s1;
   constexpr size_t kSmem = direct_smem_bytes<RmsDirect>();
   auto kern = direct_dual_kernel<RmsDirect, kFwdBatch, kFwdMinBlocks>;
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (H / 128), per_sm), 256, kSmem, st>>>(
       RmsDirect{x, ldx, rstd, gamma}, M, H / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col,
@@ -1494,7 +1497,7 @@ extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   constexpr size_t kSmem = direct_smem_bytes<SwigluDirect>();
   auto kern = direct_dual_kernel<SwigluDirect, kBwdBatch, kBwdMinBlocks>;
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
       SwigluDirect{gu, ldgu, I}, M, I / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col, nullptr);
@@ -1513,7 +1516,7 @@ extern "C" fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   constexpr size_t kSmem = direct_smem_bytes<SwigluBwd>();
   auto kern = direct_dual_kernel<SwigluBwd, kBwdBatch, kBwdMinBlocks>;
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
       SwigluBwd{gu, dh, I}, M, I / 128, dgu, q_row, s_row, lds_row, q_colT, s_col, nullptr);
@@ -1561,7 +1564,7 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
   if (s1 != FP8Q_OK) return s1;
   constexpr size_t kSmem = direct_smem_bytes<RmsBwd>();
   auto kern = direct_dual_kernel<RmsBwd, kBwdBatch, kBwdMinBlocks>;
-  static int occ[64];
+  static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (H / 128), per_sm), 256, kSmem, st>>>(
       RmsBwd{x, dy, dres, r, k, gamma, H}, M, H / 128, out, q_row, s_row, lds_row, q_colT, s_col,
