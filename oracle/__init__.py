@@ -87,6 +87,8 @@ def _load():
                                           P, P]
     lib.oracle_swiglu_bwd.argtypes = [P, P, I, I, P]
     lib.oracle_rmsnorm_bwd.argtypes = [P, P, P, P, I, I, F, P, P, P, P]
+    lib.oracle_exact_sum_f32.argtypes = [P, I, ctypes.c_int]
+    lib.oracle_exact_sum_f32.restype = ctypes.c_double
     lib.oracle_dequant_rows.argtypes = [P, P, I, I, I, I, I, P]
     lib.oracle_dequant_block.argtypes = [P, P, I, I, I, I, P]
     lib.oracle_dequant_cols.argtypes = [P, P, I, I, I, I, P]
@@ -284,6 +286,13 @@ def swiglu_bwd_dual(gu, dh, lds_row: int | None = None):
     dgu = swiglu_bwd(gu, dh)
     q, s, qT, sT = transpose_quant_bf16(dgu, lds_row)
     return q, s, qT, sT, dgu
+
+
+def exact_sum_f32(t, to_f32: bool = False) -> float:
+    """The exact sum of the fp32 values t, rounded once: to the nearest double, or (to_f32)
+    to the nearest fp32 (returned as a Python float). The reductions of rmsnorm_bwd."""
+    a = np.ascontiguousarray(np.asarray(t, dtype=np.float32))
+    return float(_load().oracle_exact_sum_f32(_p(a), a.size, 1 if to_f32 else 0))
 
 
 def rmsnorm_bwd(x, gamma, dy, dres, eps: float):

@@ -340,7 +340,7 @@ void oracle_swiglu_quant(const uint16_t* gu, i64 M, i64 I, i64 ldgu,
 /* Cuantización": gradients between operators stay BF16). The page       */
 /* gives no formula; this is the derivative of h = silu(g) * u with      */
 /* silu(g) = g * sigma(g), sigma(g) = 1 / (1 + e^-g):                    */
-/*   dL/du = dh * silu(g),  dL/dg = dh * u * sigma(g) * (1 + g*(1 - sigma(g))).
+/*   dL/du = dh * silu(g),  dL/dg = dh * u * sigma(g) * (1 + g*(1 - sigma(g))). */
 /* Reading (every step one IEEE fp32 operation, no contraction; the      */
 /* exponential and silu exactly as in the forward producer):             */
 /*   e = E(-g); d = fl32(1 + e); silu = fl32(g / d); sig = fl32(1 / d);   */
@@ -379,20 +379,117 @@ void oracle_swiglu_bwd(const uint16_t* gu, const uint16_t* dh, i64 M, i64 I,
 }
 
 /* ------------------------------------------------------------------ */
+/* Exact sum of fp32 numbers, rounded once (the reductions of the         */
+/* RMSNorm backward). Every finite fp32 value is an integer multiple of   */
+/* 2^-149 (the smallest subnormal), so a sum of them is that integer      */
+/* times 2^-149. The integer is kept in two's complement over ten         */
+/* little-endian 32-bit words (320 bits: room for 2^42 terms of the       */
+/* largest magnitude), every addition carried through all the words (a    */
+/* Kulisch accumulator). No term is ever rounded, so the result does not  */
+/* depend on the order of the additions.                                  */
+/* ------------------------------------------------------------------ */
+#define XACC_WORDS 10
+typedef struct { uint32_t w[XACC_WORDS]; } xacc;
+
+static void xacc_zero(xacc* a) { memset(a, 0, sizeof(*a)); }
+
+static void xacc_add_f32(xacc* a, float t) {
+  uint32_t u;
+  memcpy(&u, &t, 4);
+  uint32_t E = (u >> 23) & 0xFFu, f = u & 0x7FFFFFu;
+  /* |t| = m * 2^(sh - 149): normal numbers carry the implicit bit */
+  uint64_t m = E ? (uint64_t)(f | 0x800000u) : (uint64_t)f;
+  int sh = E ? (int)E - 1 : 0;
+  uint32_t term[XACC_WORDS];
+  memset(term, 0, sizeof(term));
+  uint64_t x = m << (sh % 32); /* < 2^55: two words */
+  term[sh / 32] = (uint32_t)x;
+  term[sh / 32 + 1] = (uint32_t)(x >> 32);
+  if (u >> 31) { /* negative: two's complement of the term */
+    uint64_t c = 1;
+    for (int i = 0; i < XACC_WORDS; ++i) {
+      uint64_t v = (uint64_t)(uint32_t)~term[i] + c;
+      term[i] = (uint32_t)v;
+      c = v >> 32;
+    }
+  }
+  uint64_t c = 0;
+  for (int i = 0; i < XACC_WORDS; ++i) {
+    uint64_t v = (uint64_t)a->w[i] + term[i] + c;
+    a->w[i] = (uint32_t)v;
+    c = v >> 32;
+  }
+}
+
+static int xacc_bit(const uint32_t* w, int i) { return i >= 0 ? (int)((w[i / 32] >> (i % 32)) & 1u) : 0; }
+
+/* The accumulated value rounded to a double: to nearest, ties to even; or,
+ * with odd != 0, to odd (the last mantissa bit forced to 1 when any lower
+ * bit is dropped). A double rounded to odd and then rounded to fp32 (to
+ * nearest even) is the fp32 nearest to the exact value, since 53 >= 24 + 2
+ * (S. Boldo, G. Melquiond, "Emulation of FMA and correctly rounded sums:
+ * proved algorithms using rounding to odd", IEEE Trans. Computers 2008).
+ * An exact zero gives +0. */
+static double xacc_round(const xacc* a, int odd) {
+  uint32_t mag[XACC_WORDS];
+  memcpy(mag, a->w, sizeof(mag));
+  int neg = (int)(mag[XACC_WORDS - 1] >> 31);
+  if (neg) {
+    uint64_t c = 1;
+    for (int i = 0; i < XACC_WORDS; ++i) {
+      uint64_t v = (uint64_t)(uint32_t)~mag[i] + c;
+      mag[i] = (uint32_t)v;
+      c = v >> 32;
+    }
+  }
+  int p = -1; /* highest set bit of the magnitude */
+  for (int i = XACC_WORDS * 32 - 1; i >= 0; --i)
+    if (xacc_bit(mag, i)) { p = i; break; }
+  if (p < 0) return 0.0;
+  uint64_t mant = 0; /* bits p .. p-52 */
+  for (int i = p; i > p - 53; --i) mant = (mant << 1) | (uint64_t)xacc_bit(mag, i);
+  int round = xacc_bit(mag, p - 53), sticky = 0;
+  for (int i = p - 54; i >= 0; --i) sticky |= xacc_bit(mag, i);
+  if (odd) {
+    if (round || sticky) mant |= 1u;
+  } else if (round && (sticky || (mant & 1u))) {
+    mant += 1u; /* may reach 2^53, still exact as a double */
+  }
+  double v = ldexp((double)mant, p - 52 - 149);
+  return neg ? -v : v;
+}
+
+/* The accumulated value rounded once to the nearest fp32 (ties to even). */
+static float xacc_round_f32(const xacc* a) { return (float)xacc_round(a, 1); }
+
+/* Exported for the tests: the exact sum of t[0..n) rounded once, to the
+ * nearest double (to_f32 == 0) or to the nearest fp32 (to_f32 != 0, returned
+ * as a double). */
+double oracle_exact_sum_f32(const float* t, i64 n, int to_f32) {
+  xacc a;
+  xacc_zero(&a);
+  for (i64 i = 0; i < n; ++i) xacc_add_f32(&a, t[i]);
+  if (to_f32) return (double)xacc_round_f32(&a);
+  return xacc_round(&a, 0);
+}
+
+/* ------------------------------------------------------------------ */
 /* Backward of the RMSNorm producer, in BF16, with the residual          */
 /* gradient added (the gradient that flows on along the residual        */
 /* stream). Forward: y_j = x_j * r * gamma_j, r = (mean(x^2) + eps)^-1/2. */
 /* Derivative: dx_j = r * gamma_j * dy_j - x_j * r^3 * c / H with        */
 /* c = sum_j gamma_j * dy_j * x_j; dgamma_j = sum_m dy_mj * x_mj * r_m.  */
 /* Reading (the page gives no formula; rounding as an unfused BF16       */
-/* RMSNorm backward followed by a BF16 residual add):                    */
+/* RMSNorm backward followed by a BF16 residual add; the two reductions  */
+/* are exact sums rounded once, so no summation order enters them):      */
 /*   r as in the forward producer (oracle_rmsnorm_rstd);                 */
-/*   c = sum_j fl32(fl32(gamma_j * dy_j) * x_j) in fp64 (each product is */
-/*       exact: three 8-bit significands), in index order;               */
+/*   c = the exact sum over j of fl32(fl32(gamma_j * dy_j) * x_j),        */
+/*       rounded to the nearest double;                                   */
 /*   k = (float)((((c * r) * r) * r) / H) in fp64;                        */
 /*   dx_j = bf16(fl32(fl32(r * fl32(gamma_j * dy_j)) - fl32(k * x_j)));   */
 /*   out_j = bf16(fl32(dx_j + dres_j))  (dres NULL: out_j = dx_j);        */
-/*   dgamma_j = (float) sum over m (in order) of fl32(dy_mj * fl32(x_mj * r_m)) in fp64.
+/*   dgamma_j = the exact sum over m of fl32(dy_mj * fl32(x_mj * r_m)),   */
+/*       rounded to the nearest fp32.                                     */
 /* r_out (if not NULL) receives r per row, k_out (if not NULL) k.        */
 /* ------------------------------------------------------------------ */
 void oracle_rmsnorm_bwd(const uint16_t* x, const uint16_t* gamma, const uint16_t* dy,
@@ -404,12 +501,14 @@ void oracle_rmsnorm_bwd(const uint16_t* x, const uint16_t* gamma, const uint16_t
     const uint16_t* xr = x + m * H;
     const uint16_t* dyr = dy + m * H;
     float r = oracle_rmsnorm_rstd(xr, H, eps);
-    double c = 0.0;
+    xacc cs;
+    xacc_zero(&cs);
     for (i64 j = 0; j < H; ++j) {
       volatile float gd = oracle_bf16_to_f32(gamma[j]) * oracle_bf16_to_f32(dyr[j]);
       volatile float t = gd * oracle_bf16_to_f32(xr[j]);
-      c += (double)t;
+      xacc_add_f32(&cs, t);
     }
+    double c = xacc_round(&cs, 0);
     double kd = c * (double)r;
     kd = kd * (double)r;
     kd = kd * (double)r;
@@ -436,13 +535,14 @@ void oracle_rmsnorm_bwd(const uint16_t* x, const uint16_t* gamma, const uint16_t
   if (dgamma) {
 #pragma omp parallel for schedule(static)
     for (i64 j = 0; j < H; ++j) {
-      double acc = 0.0;
+      xacc acc;
+      xacc_zero(&acc);
       for (i64 m = 0; m < M; ++m) {
         volatile float xr = oracle_bf16_to_f32(x[m * H + j]) * rr[m];
         volatile float t = oracle_bf16_to_f32(dy[m * H + j]) * xr;
-        acc += (double)t;
+        xacc_add_f32(&acc, t);
       }
-      dgamma[j] = (float)acc;
+      dgamma[j] = xacc_round_f32(&acc);
     }
   }
   free(rr);

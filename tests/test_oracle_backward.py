@@ -205,3 +205,106 @@ def test_rmsnorm_bwd_dual_is_a6_of_the_output(oracle_mod):
     assert np.array_equal(q, q2) and np.array_equal(qT, qT2)
     assert np.array_equal(s, s2) and np.array_equal(sT, sT2)
     assert dgamma.shape == (H,)
+
+
+# ------------------------------------------------- exact reductions of the RMSNorm backward
+# The two reductions (c per row, dgamma per column) are exact sums of fp32 terms rounded
+# once, so no summation order enters them. Pinned against math.fsum (the correctly
+# rounded double of an exact sum) and exact rational arithmetic.
+import math  # noqa: E402
+from fractions import Fraction  # noqa: E402
+
+
+def _hard_sums():
+    """fp32 term sets that break naive summation: cancellation, wide exponent spread,
+    subnormals, ties of the final rounding, long runs."""
+    rng = np.random.default_rng(1234)
+    f = np.float32
+    sets = [
+        np.array([1.0, 2.0 ** -24], f),                      # exactly halfway in fp32
+        np.array([1.0, 2.0 ** -24, 2.0 ** -60], f),          # just above halfway
+        np.array([1.0, -2.0 ** -24, -2.0 ** -70], f),        # just below halfway, negative
+        np.array([2.0 ** 100, 1.0, -2.0 ** 100], f),         # total cancellation of the big part
+        np.array([3.0, -3.0], f),                            # exact zero
+        np.array([2.0 ** -149, 2.0 ** -149, 3 * 2.0 ** -149], f),   # subnormals
+        np.array([2.0 ** 127, 2.0 ** 127, -2.0 ** 127], f),  # beyond fp32 range midway
+        np.array([1.0 + 2.0 ** -23] * 7 + [-7.0], f),
+    ]
+    for k in range(12):
+        n = int(rng.integers(2, 3000))
+        v = rng.standard_normal(n).astype(np.float64)
+        e = rng.integers(-140, 100, n) if k % 3 == 0 else rng.integers(-40, 10, n)
+        t = (v * 2.0 ** e).astype(f)
+        if k % 4 == 1:  # a large pair that cancels, so the small terms decide
+            t = np.concatenate([t, np.array([2.0 ** 90, -2.0 ** 90], f)])
+        rng.shuffle(t)
+        sets.append(t)
+    return sets
+
+
+def _nearest_f32(S: Fraction) -> float:
+    """The fp32 nearest to the rational S (ties to even), from exact comparisons."""
+    guess = np.float32(float(S))
+    cands = {float(guess), float(np.nextafter(guess, np.float32(np.inf))),
+             float(np.nextafter(guess, np.float32(-np.inf)))}
+    best = min(cands, key=lambda c: (abs(Fraction(c) - S),
+                                     int(np.float32(c).view(np.uint32)) & 1))
+    return best
+
+
+def test_exact_sum_equals_fsum(oracle_mod):
+    for t in _hard_sums():
+        got = oracle_mod.exact_sum_f32(t)
+        ref = math.fsum(float(v) for v in t)
+        assert got == ref, (t[:4], got, ref)
+
+
+def test_exact_sum_rounds_once_to_fp32(oracle_mod):
+    for t in _hard_sums():
+        S = sum((Fraction(float(v)) for v in t), Fraction(0))
+        got = oracle_mod.exact_sum_f32(t, to_f32=True)
+        assert got == _nearest_f32(S), (t[:4], got)
+    # the double-rounding trap: 1 + 2^-24 + 2^-60 rounds up in one step (to 1 + 2^-23),
+    # while rounding to a double first would land on the tie and go down to 1
+    t = np.array([1.0, 2.0 ** -24, 2.0 ** -60], np.float32)
+    assert oracle_mod.exact_sum_f32(t, to_f32=True) == 1.0 + 2.0 ** -23
+
+
+def test_exact_sum_is_order_free_and_zero_is_positive(oracle_mod):
+    rng = np.random.default_rng(7)
+    for t in _hard_sums():
+        a = oracle_mod.exact_sum_f32(t)
+        b = oracle_mod.exact_sum_f32(t[rng.permutation(t.size)])
+        assert a == b
+    z = oracle_mod.exact_sum_f32(np.array([5.0, -2.5, -2.5], np.float32))
+    assert z == 0.0 and math.copysign(1.0, z) == 1.0
+
+
+def _rms_bwd_case(M=48, H=384, seed=0):
+    x = workloads.activations_bf16((M, H), seed, 61, "cpu", outlier_frac=0.02, outlier_scale=50)
+    dy = workloads.gradients_bf16((M, H), 1e-3, seed, 62, "cpu")
+    g = workloads.gamma_bf16(H, seed, 63, "cpu")
+    return bits(x), bits(dy), bits(g)
+
+
+def test_rmsnorm_bwd_k_uses_the_exact_row_sum(oracle_mod):
+    xb, dyb, gb = _rms_bwd_case()
+    M, H = xb.shape
+    _, _, r, k = oracle_mod.rmsnorm_bwd(xb, gb, dyb, None, 1e-5)
+    x32, dy32, g32 = (f32_of_bits(b).astype(np.float32) for b in (xb, dyb, gb))
+    for m in range(M):
+        terms = (g32 * dy32[m]) * x32[m]          # fp32 products, IEEE, as the reading says
+        c = math.fsum(float(t) for t in terms)
+        rd = float(r[m])
+        kd = ((c * rd) * rd) * rd / H
+        assert np.float32(kd) == k[m], m
+
+
+def test_rmsnorm_bwd_dgamma_is_the_exact_column_sum(oracle_mod):
+    xb, dyb, gb = _rms_bwd_case(M=64, H=256, seed=1)
+    _, dgamma, r, _ = oracle_mod.rmsnorm_bwd(xb, gb, dyb, None, 1e-5)
+    x32, dy32 = (f32_of_bits(b).astype(np.float32) for b in (xb, dyb))
+    terms = dy32 * (x32 * r[:, None].astype(np.float32))   # fl32(dy * fl32(x * r))
+    for j in range(0, 256, 5):
+        S = sum((Fraction(float(v)) for v in terms[:, j]), Fraction(0))
+        assert float(dgamma[j]) == _nearest_f32(S), j

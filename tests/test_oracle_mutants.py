@@ -47,6 +47,14 @@ MUTANTS = [
     ("dgamma without r",
      "volatile float xr = oracle_bf16_to_f32(x[m * H + j]) * rr[m];",
      "volatile float xr = oracle_bf16_to_f32(x[m * H + j]);", [BWD]),
+    ("exact sum without the carry between words",
+     "uint64_t v = (uint64_t)a->w[i] + term[i] + c;", "uint64_t v = (uint64_t)a->w[i] + term[i];",
+     [BWD]),
+    ("exact sum loses its sticky bits",
+     "for (int i = p - 54; i >= 0; --i) sticky |= xacc_bit(mag, i);",
+     "for (int i = p - 54; i >= 0 && 0; --i) sticky |= xacc_bit(mag, i);", [BWD]),
+    ("fp32 reduction rounded through a double",
+     "{ return (float)xacc_round(a, 1); }", "{ return (float)xacc_round(a, 0); }", [BWD]),
     ("128x1 column group rows mis-indexed",
      "dy[(mb * 128 + i) * lddy + n]", "dy[(mb + i) * lddy + n]", [QUANT]),
     ("requantizer drops the row scale",
