@@ -15,11 +15,16 @@ activations, BF16 inter-operator gradients, FP8 DGrad/WGrad with 1x128 and 128x1
 grouping for WGrad) and section "Implementación" (fused quantize / transpose /
 activation / RMSNorm kernels next to FP8 GEMMs).
 
-Layouts (all row-major):
+Layouts (all row-major; G(n) = ceil(n / 128) groups along a dimension of n elements,
+the last one partial when n is not a multiple of 128):
   codes          uint8 [rows][cols]
-  1x128 scales   float32 [cols/128][lds]   scale of (row m, group g) at s[g, m]
-  weight scales  float32 [N/128][K/128]
-  128x1 scales   float32 [rows/128][cols]  scale of (group mb, column c) at s[mb, c]
+  1x128 scales   float32 [G(cols)][lds]    scale of (row m, group g) at s[g, m]
+  weight scales  float32 [G(N)][G(K)]
+  128x1 scales   float32 [G(rows)][cols]   scale of (group mb, column c) at s[mb, c]
+
+Partial groups (dimensions that are not multiples of 128): the group is the full group
+with zeros in the missing places; its scale comes from its valid elements alone and
+only the codes of the valid places exist.
 """
 from __future__ import annotations
 
@@ -162,6 +167,12 @@ def rmsnorm_rstd(xrow_bits: np.ndarray, eps: float) -> float:
 # Quantizers (all outputs are fresh numpy arrays)
 # --------------------------------------------------------------------------
 
+def groups(n: int) -> int:
+    """Number of 128-element groups along a dimension of n elements (the last one
+    partial when n is not a multiple of 128)."""
+    return (int(n) + 127) // 128
+
+
 def _lds_for(M: int) -> int:
     return (M + 3) // 4 * 4
 
@@ -170,10 +181,9 @@ def quant_act_1x128(x, lds: int | None = None):
     """a1: x BF16 [M,K] -> (q uint8 [M,K], s float32 [K/128, lds])."""
     x = _bf16(x)
     M, K = x.shape
-    assert K % 128 == 0
     lds = _lds_for(M) if lds is None else lds
     q = np.zeros((M, K), np.uint8)
-    s = np.zeros((K // 128, lds), np.float32)
+    s = np.zeros((groups(K), lds), np.float32)
     _load().oracle_quant_act_1x128(_p(x), M, K, K, _p(q), _p(s), lds)
     return q, s
 
@@ -182,9 +192,8 @@ def quant_weight_128x128(w, want_t: bool = True):
     """a2: w BF16 [N,K] -> (q [N,K], s [N/128,K/128], qT [K,N] or None)."""
     w = _bf16(w)
     N, K = w.shape
-    assert N % 128 == 0 and K % 128 == 0
     q = np.zeros((N, K), np.uint8)
-    s = np.zeros((N // 128, K // 128), np.float32)
+    s = np.zeros((groups(N), groups(K)), np.float32)
     qT = np.zeros((K, N), np.uint8) if want_t else None
     _load().oracle_quant_weight_128x128(_p(w), N, K, K, _p(q), _p(s),
                                         _p(qT) if want_t else None)
@@ -196,10 +205,10 @@ def rmsnorm_quant(x, gamma, eps: float, lds: int | None = None, want_y: bool = F
     x = _bf16(x)
     g = _bf16(gamma)
     M, H = x.shape
-    assert H % 128 == 0 and g.shape == (H,)
+    assert g.shape == (H,)
     lds = _lds_for(M) if lds is None else lds
     q = np.zeros((M, H), np.uint8)
-    s = np.zeros((H // 128, lds), np.float32)
+    s = np.zeros((groups(H), lds), np.float32)
     y = np.zeros((M, H), np.uint16) if want_y else None
     _load().oracle_rmsnorm_quant(_p(x), _p(g), M, H, H, float(eps), _p(q), _p(s), lds,
                                  _p(y) if want_y else None)
@@ -211,10 +220,10 @@ def swiglu_quant(gu, lds: int | None = None, want_h: bool = False):
     gu = _bf16(gu)
     M, I2 = gu.shape
     I = I2 // 2
-    assert I2 % 2 == 0 and I % 128 == 0
+    assert I2 % 2 == 0
     lds = _lds_for(M) if lds is None else lds
     q = np.zeros((M, I), np.uint8)
-    s = np.zeros((I // 128, lds), np.float32)
+    s = np.zeros((groups(I), lds), np.float32)
     h = np.zeros((M, I), np.uint16) if want_h else None
     _load().oracle_swiglu_quant(_p(gu), M, I, I2, _p(q), _p(s), lds,
                                 _p(h) if want_h else None)
@@ -226,12 +235,11 @@ def transpose_quant_bf16(dy, lds_row: int | None = None, want_row: bool = True):
     column-wise 128x1 transposed (q_colT [N,M], s_col [M/128, N])."""
     dy = _bf16(dy)
     M, N = dy.shape
-    assert M % 128 == 0 and N % 128 == 0
     lds_row = _lds_for(M) if lds_row is None else lds_row
     q_row = np.zeros((M, N), np.uint8) if want_row else None
-    s_row = np.zeros((N // 128, lds_row), np.float32) if want_row else None
+    s_row = np.zeros((groups(N), lds_row), np.float32) if want_row else None
     q_colT = np.zeros((N, M), np.uint8)
-    s_col = np.zeros((M // 128, N), np.float32)
+    s_col = np.zeros((groups(M), N), np.float32)
     _load().oracle_transpose_quant_bf16(
         _p(dy), M, N, N, _p(q_row) if want_row else None,
         _p(s_row) if want_row else None, lds_row, _p(q_colT), _p(s_col))
@@ -328,9 +336,9 @@ def transpose_quant_fp8(q, s):
     q = np.ascontiguousarray(q, dtype=np.uint8)
     s = np.ascontiguousarray(s, dtype=np.float32)
     M, K = q.shape
-    assert M % 128 == 0 and K % 128 == 0 and s.shape[0] == K // 128
+    assert s.shape[0] == groups(K)
     qT = np.zeros((K, M), np.uint8)
-    sT = np.zeros((M // 128, K), np.float32)
+    sT = np.zeros((groups(M), K), np.float32)
     _load().oracle_transpose_quant_fp8(_p(q), _p(s), M, K, s.shape[1], _p(qT), _p(sT))
     return qT, sT
 

@@ -149,6 +149,15 @@ static uint8_t quant_one(float x, float s) {
   return oracle_e4m3_encode(t);
 }
 
+/* Groups along a dimension of n elements, and the width of group g: every group
+ * has 128 elements except, when n is not a multiple of 128, the last one, which has
+ * the n % 128 remaining elements. Reading (the page fixes only the 1x128 / 128x128
+ * grouping): a partial group is the full group with zeros in the missing places;
+ * zeros raise no maximum, so its scale comes from its valid elements alone, and the
+ * codes of the missing places, which would all be 0, are not stored. */
+static i64 ngroups(i64 n) { return (n + 127) / 128; }
+static int gwidth(i64 n, i64 g) { return n - g * 128 < 128 ? (int)(n - g * 128) : 128; }
+
 /* ------------------------------------------------------------------ */
 /* a1: activation quantization per 1x128 group.                         */
 /* x [M][K] BF16 (row stride ldx) -> q [M][K] (row stride K),            */
@@ -158,18 +167,19 @@ static uint8_t quant_one(float x, float s) {
 void oracle_quant_act_1x128(const uint16_t* x, i64 M, i64 K, i64 ldx,
                             uint8_t* q, float* s, i64 lds) {
   init_mag();
-  i64 G = K / 128;
+  i64 G = ngroups(K);
 #pragma omp parallel for schedule(static)
   for (i64 m = 0; m < M; ++m) {
     for (i64 g = 0; g < G; ++g) {
+      int w = gwidth(K, g);
       float amax = 0.0f;
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < w; ++i) {
         float v = fabsf(oracle_bf16_to_f32(x[m * ldx + g * 128 + i]));
         if (v > amax) amax = v;
       }
       float sc = group_scale(amax);
       s[g * lds + m] = sc;
-      for (int i = 0; i < 128; ++i)
+      for (int i = 0; i < w; ++i)
         q[m * K + g * 128 + i] = quant_one(oracle_bf16_to_f32(x[m * ldx + g * 128 + i]), sc);
     }
   }
@@ -184,20 +194,21 @@ void oracle_quant_act_1x128(const uint16_t* x, i64 M, i64 K, i64 ldx,
 void oracle_quant_weight_128x128(const uint16_t* w, i64 N, i64 K, i64 ldw,
                                  uint8_t* q, float* s, uint8_t* qT) {
   init_mag();
-  i64 NB = N / 128, KB = K / 128;
+  i64 NB = ngroups(N), KB = ngroups(K);
 #pragma omp parallel for schedule(static)
   for (i64 blk = 0; blk < NB * KB; ++blk) {
     i64 nb = blk / KB, kb = blk % KB;
+    int hr = gwidth(N, nb), wc = gwidth(K, kb);
     float amax = 0.0f;
-    for (i64 r = 0; r < 128; ++r)
-      for (i64 c = 0; c < 128; ++c) {
+    for (i64 r = 0; r < hr; ++r)
+      for (i64 c = 0; c < wc; ++c) {
         float v = fabsf(oracle_bf16_to_f32(w[(nb * 128 + r) * ldw + kb * 128 + c]));
         if (v > amax) amax = v;
       }
     float sc = group_scale(amax);
     s[nb * KB + kb] = sc;
-    for (i64 r = 0; r < 128; ++r)
-      for (i64 c = 0; c < 128; ++c) {
+    for (i64 r = 0; r < hr; ++r)
+      for (i64 c = 0; c < wc; ++c) {
         i64 n = nb * 128 + r, k = kb * 128 + c;
         uint8_t code = quant_one(oracle_bf16_to_f32(w[n * ldw + k]), sc);
         q[n * K + k] = code;
@@ -232,15 +243,16 @@ void oracle_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, i64 M, i64 H
                           i64 ldx, float eps, uint8_t* q, float* s, i64 lds,
                           uint16_t* y) {
   init_mag();
-  i64 G = H / 128;
+  i64 G = ngroups(H);
 #pragma omp parallel for schedule(static)
   for (i64 m = 0; m < M; ++m) {
     const uint16_t* xr = x + m * ldx;
     float r = oracle_rmsnorm_rstd(xr, H, eps);
     for (i64 g = 0; g < G; ++g) {
+      int w = gwidth(H, g);
       float yv[128];
       float amax = 0.0f;
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < w; ++i) {
         i64 c = g * 128 + i;
         volatile float t1 = oracle_bf16_to_f32(xr[c]) * r;
         volatile float t2 = t1 * oracle_bf16_to_f32(gamma[c]);
@@ -252,7 +264,7 @@ void oracle_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, i64 M, i64 H
       }
       float sc = group_scale(amax);
       s[g * lds + m] = sc;
-      for (int i = 0; i < 128; ++i) q[m * H + g * 128 + i] = quant_one(yv[i], sc);
+      for (int i = 0; i < w; ++i) q[m * H + g * 128 + i] = quant_one(yv[i], sc);
     }
   }
 }
@@ -314,13 +326,14 @@ uint16_t oracle_swiglu_one(uint16_t gate, uint16_t up) {
 void oracle_swiglu_quant(const uint16_t* gu, i64 M, i64 I, i64 ldgu,
                          uint8_t* q, float* s, i64 lds, uint16_t* h) {
   init_mag();
-  i64 G = I / 128;
+  i64 G = ngroups(I);
 #pragma omp parallel for schedule(static)
   for (i64 m = 0; m < M; ++m) {
     for (i64 g = 0; g < G; ++g) {
+      int w = gwidth(I, g);
       float hv[128];
       float amax = 0.0f;
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < w; ++i) {
         i64 c = g * 128 + i;
         uint16_t hb = oracle_swiglu_one(gu[m * ldgu + c], gu[m * ldgu + I + c]);
         if (h) h[m * I + c] = hb;
@@ -330,7 +343,7 @@ void oracle_swiglu_quant(const uint16_t* gu, i64 M, i64 I, i64 ldgu,
       }
       float sc = group_scale(amax);
       s[g * lds + m] = sc;
-      for (int i = 0; i < 128; ++i) q[m * I + g * 128 + i] = quant_one(hv[i], sc);
+      for (int i = 0; i < w; ++i) q[m * I + g * 128 + i] = quant_one(hv[i], sc);
     }
   }
 }
@@ -563,18 +576,19 @@ void oracle_transpose_quant_bf16(const uint16_t* dy, i64 M, i64 N, i64 lddy,
                                  uint8_t* q_colT, float* s_col) {
   init_mag();
   if (q_row && s_row) oracle_quant_act_1x128(dy, M, N, lddy, q_row, s_row, lds_row);
-  i64 MB = M / 128;
+  i64 MB = ngroups(M);
 #pragma omp parallel for schedule(static)
   for (i64 n = 0; n < N; ++n) {
     for (i64 mb = 0; mb < MB; ++mb) {
+      int w = gwidth(M, mb);
       float amax = 0.0f;
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < w; ++i) {
         float v = fabsf(oracle_bf16_to_f32(dy[(mb * 128 + i) * lddy + n]));
         if (v > amax) amax = v;
       }
       float sc = group_scale(amax);
       s_col[mb * N + n] = sc;
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < w; ++i) {
         i64 m = mb * 128 + i;
         q_colT[n * M + m] = quant_one(oracle_bf16_to_f32(dy[m * lddy + n]), sc);
       }
@@ -593,13 +607,14 @@ void oracle_transpose_quant_bf16(const uint16_t* dy, i64 M, i64 N, i64 lddy,
 void oracle_transpose_quant_fp8(const uint8_t* q, const float* s, i64 M, i64 K,
                                 i64 lds, uint8_t* qT, float* sT) {
   init_mag();
-  i64 MB = M / 128;
+  i64 MB = ngroups(M);
 #pragma omp parallel for schedule(static)
   for (i64 k = 0; k < K; ++k) {
     for (i64 mb = 0; mb < MB; ++mb) {
+      int w = gwidth(M, mb);
       float xh[128];
       float amax = 0.0f;
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < w; ++i) {
         i64 m = mb * 128 + i;
         float dec = (float)oracle_e4m3_decode(q[m * K + k]); /* exact */
         volatile float v = s[(k / 128) * lds + m] * dec;
@@ -609,7 +624,7 @@ void oracle_transpose_quant_fp8(const uint8_t* q, const float* s, i64 M, i64 K,
       }
       float sc = group_scale(amax);
       sT[mb * K + k] = sc;
-      for (int i = 0; i < 128; ++i) qT[k * M + mb * 128 + i] = quant_one(xh[i], sc);
+      for (int i = 0; i < w; ++i) qT[k * M + mb * 128 + i] = quant_one(xh[i], sc);
     }
   }
 }
@@ -637,7 +652,7 @@ void oracle_dequant_rows(const uint8_t* q, const float* s, i64 R, i64 K, i64 lds
 void oracle_dequant_block(const uint8_t* q, const float* s, i64 N, i64 K,
                           i64 r0, i64 nr, double* out) {
   init_mag();
-  i64 KB = K / 128;
+  i64 KB = ngroups(K);
 #pragma omp parallel for schedule(static)
   for (i64 i = 0; i < nr; ++i)
     for (i64 k = 0; k < K; ++k)

@@ -18,6 +18,7 @@ SRC = os.path.join(ROOT, "oracle", "fp8q_oracle.c")
 E4M3, QUANT = "tests/test_oracle_e4m3.py", "tests/test_oracle_quant.py"
 NORM, BWD = "tests/test_oracle_norm_swiglu.py", "tests/test_oracle_backward.py"
 GEMM = "tests/test_oracle_gemm.py"
+TAILS = "tests/test_oracle_tails.py"
 
 # (name, exact text in fp8q_oracle.c, replacement, pin files that must catch it)
 MUTANTS = [
@@ -55,6 +56,13 @@ MUTANTS = [
      "for (int i = p - 54; i >= 0 && 0; --i) sticky |= xacc_bit(mag, i);", [BWD]),
     ("fp32 reduction rounded through a double",
      "{ return (float)xacc_round(a, 1); }", "{ return (float)xacc_round(a, 0); }", [BWD]),
+    ("partial group drops its last element",
+     "static int gwidth(i64 n, i64 g) { return n - g * 128 < 128 ? (int)(n - g * 128) : 128; }",
+     "static int gwidth(i64 n, i64 g) { return n - g * 128 < 128 ? (int)(n - g * 128) - 1 : 128; }",
+     [TAILS]),
+    ("partial group count rounded down",
+     "static i64 ngroups(i64 n) { return (n + 127) / 128; }",
+     "static i64 ngroups(i64 n) { return n / 128; }", [TAILS]),
     ("128x1 column group rows mis-indexed",
      "dy[(mb * 128 + i) * lddy + n]", "dy[(mb + i) * lddy + n]", [QUANT]),
     ("requantizer drops the row scale",
