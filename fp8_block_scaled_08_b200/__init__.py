@@ -290,9 +290,9 @@ def rmsnorm_quant_dual(x, gamma, eps, q_row, s_row, q_colT, s_col, rstd, stream=
 def rmsnorm_quant_dual_alloc(x, gamma, eps, stream=None):
     M, H = x.shape
     q = _empty((M, H), torch.uint8, x.device)
-    s = _empty((H // 128, lds_for(M)), torch.float32, x.device)
+    s = _empty((_groups(H), lds_for(M)), torch.float32, x.device)
     qT = _empty((H, M), torch.uint8, x.device)
-    sT = _empty((M // 128, H), torch.float32, x.device)
+    sT = _empty((_groups(M), H), torch.float32, x.device)
     r = _empty((M,), torch.float32, x.device)
     rmsnorm_quant_dual(x, gamma, eps, q, s, qT, sT, r, stream)
     return q, s, qT, sT, r
@@ -320,9 +320,9 @@ def swiglu_quant_dual_alloc(gu, stream=None):
     M, I2 = gu.shape
     I = I2 // 2
     q = _empty((M, I), torch.uint8, gu.device)
-    s = _empty((I // 128, lds_for(M)), torch.float32, gu.device)
+    s = _empty((_groups(I), lds_for(M)), torch.float32, gu.device)
     qT = _empty((I, M), torch.uint8, gu.device)
-    sT = _empty((M // 128, I), torch.float32, gu.device)
+    sT = _empty((_groups(M), I), torch.float32, gu.device)
     swiglu_quant_dual(gu, q, s, qT, sT, stream)
     return q, s, qT, sT
 
@@ -355,9 +355,9 @@ def swiglu_bwd_quant_dual(gu, dh, q_row, s_row, q_colT, s_col, dgu=None, stream=
 def swiglu_bwd_quant_dual_alloc(gu, dh, want_dgu=False, stream=None):
     M, I2 = gu.shape
     q = _empty((M, I2), torch.uint8, gu.device)
-    s = _empty((I2 // 128, lds_for(M)), torch.float32, gu.device)
+    s = _empty((_groups(I2), lds_for(M)), torch.float32, gu.device)
     qT = _empty((I2, M), torch.uint8, gu.device)
-    sT = _empty((M // 128, I2), torch.float32, gu.device)
+    sT = _empty((_groups(M), I2), torch.float32, gu.device)
     dgu = _empty((M, I2), torch.bfloat16, gu.device) if want_dgu else None
     swiglu_bwd_quant_dual(gu, dh, q, s, qT, sT, dgu, stream)
     return q, s, qT, sT, dgu
@@ -406,9 +406,9 @@ def rmsnorm_bwd_quant_dual_alloc(x, gamma, dy, dres, eps, stream=None):
     dev = x.device
     out = _empty((M, H), torch.bfloat16, dev)
     q = _empty((M, H), torch.uint8, dev)
-    s = _empty((H // 128, lds_for(M)), torch.float32, dev)
+    s = _empty((_groups(H), lds_for(M)), torch.float32, dev)
     qT = _empty((H, M), torch.uint8, dev)
-    sT = _empty((M // 128, H), torch.float32, dev)
+    sT = _empty((_groups(M), H), torch.float32, dev)
     dg = _empty((H,), torch.float32, dev)
     nbytes = rmsnorm_bwd_workspace_bytes(M, H)
     ws = _empty((max(nbytes, 16),), torch.uint8, dev)
@@ -552,7 +552,7 @@ def _empty(shape, dtype, device):
 def quant_act_1x128_alloc(x, stream=None):
     M, K = x.shape
     q = _empty((M, K), torch.uint8, x.device)
-    s = _empty((K // 128, lds_for(M)), torch.float32, x.device)
+    s = _empty((_groups(K), lds_for(M)), torch.float32, x.device)
     quant_act_1x128(x, q, s, stream)
     return q, s
 
@@ -560,7 +560,7 @@ def quant_act_1x128_alloc(x, stream=None):
 def quant_weight_alloc(w, want_t=True, stream=None):
     N, K = w.shape
     q = _empty((N, K), torch.uint8, w.device)
-    s = _empty((N // 128, K // 128), torch.float32, w.device)
+    s = _empty((_groups(N), _groups(K)), torch.float32, w.device)
     qT = _empty((K, N), torch.uint8, w.device) if want_t else None
     quant_weight_128x128(w, q, s, qT, stream)
     return q, s, qT
@@ -569,7 +569,7 @@ def quant_weight_alloc(w, want_t=True, stream=None):
 def rmsnorm_quant_alloc(x, gamma, eps, stream=None):
     M, H = x.shape
     q = _empty((M, H), torch.uint8, x.device)
-    s = _empty((H // 128, lds_for(M)), torch.float32, x.device)
+    s = _empty((_groups(H), lds_for(M)), torch.float32, x.device)
     rmsnorm_quant(x, gamma, eps, q, s, stream)
     return q, s
 
@@ -577,7 +577,7 @@ def rmsnorm_quant_alloc(x, gamma, eps, stream=None):
 def swiglu_quant_alloc(gu, stream=None):
     M, I2 = gu.shape
     q = _empty((M, I2 // 2), torch.uint8, gu.device)
-    s = _empty((I2 // 2 // 128, lds_for(M)), torch.float32, gu.device)
+    s = _empty((_groups(I2 // 2), lds_for(M)), torch.float32, gu.device)
     swiglu_quant(gu, q, s, stream)
     return q, s
 
@@ -585,9 +585,9 @@ def swiglu_quant_alloc(gu, stream=None):
 def transpose_quant_bf16_alloc(dy, want_row=True, stream=None):
     M, N = dy.shape
     q_row = _empty((M, N), torch.uint8, dy.device) if want_row else None
-    s_row = _empty((N // 128, lds_for(M)), torch.float32, dy.device) if want_row else None
+    s_row = _empty((_groups(N), lds_for(M)), torch.float32, dy.device) if want_row else None
     q_colT = _empty((N, M), torch.uint8, dy.device)
-    s_col = _empty((M // 128, N), torch.float32, dy.device)
+    s_col = _empty((_groups(M), N), torch.float32, dy.device)
     transpose_quant_bf16(dy, q_row, s_row, q_colT, s_col, stream)
     return q_row, s_row, q_colT, s_col
 
@@ -595,7 +595,7 @@ def transpose_quant_bf16_alloc(dy, want_row=True, stream=None):
 def transpose_quant_fp8_alloc(q, s, stream=None):
     M, K = q.shape
     qT = _empty((K, M), torch.uint8, q.device)
-    sT = _empty((M // 128, K), torch.float32, q.device)
+    sT = _empty((_groups(M), K), torch.float32, q.device)
     transpose_quant_fp8(q, s, qT, sT, stream)
     return qT, sT
 

@@ -322,7 +322,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row0 = mb * kPairM + static_cast<int>(rank) * BM;
       const int col_lo = nb * BN + (kSplitN ? 64 : 128) * half;  // tile columns of acc[0..63]
       const int col_hi = kSplitN ? nb * BN + 128 + 64 * half : col_lo + 64;  // of acc[64..127]
-      const bool lo_ok = col_lo < p.N;  // the N tail is a multiple of 128
+      // a ragged N (a multiple of 16) ends inside a box: the tensor store clips it
+      const bool lo_ok = col_lo < p.N;
       const bool hi_ok = col_hi < p.N;
       const float* sbp_lo = kColScaleB ? nullptr : p.sb + static_cast<int64_t>(col_lo / 128) * p.sb_sj;
       const float* sbp_hi = kColScaleB ? nullptr : p.sb + static_cast<int64_t>(col_hi / 128) * p.sb_sj;
@@ -413,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0 && (hh == 0 || hi_ok)) {
               const int cb = hh ? col_hi : col_lo;
               tma_reduce_add_2d(&tmY, out0, cb, wrow0);
-              tma_reduce_add_2d(&tmY, out1, cb + 32, wrow0);
+              if (cb + 32 < p.N) tma_reduce_add_2d(&tmY, out1, cb + 32, wrow0);  // ragged N
               tma_store_commit();
             }
             stored = true;
@@ -529,6 +530,9 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   const int sms = sm100_sm_count();
   if (!sms) return FP8Q_ERR_UNSUPPORTED;
   if (Mg > 0x7FFFFFFF || Ng > 0x7FFFFFFF || Kg > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  // 128-wide K slices; a partial last slice (Kg not a multiple of 128) is zero-filled
+  // by the tensor copies, which adds nothing to any dot product
+  const int64_t kslices = (Kg + BK - 1) / BK;
   CUtensorMap tmA, tmB, tmSA, tmSB, tmY;
   bool ok = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, Kg, Mg, Kg, BK, BM,
                            CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -538,10 +542,10 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
                                    32, CU_TENSOR_MAP_SWIZZLE_128B)
                   : encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, Ng, Mg, ldy * 2, 64,
                                    32, CU_TENSOR_MAP_SWIZZLE_128B)) &&
-            encode_tmap_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, Mg, Kg / BK, ldsa * 4, BM,
+            encode_tmap_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, Mg, kslices, ldsa * 4, BM,
                            1, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (ok && kCol)
-    ok = encode_tmap_2d(&tmSB, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sbcol, Ng, Kg / BK, Ng * 4, BN, 1,
+    ok = encode_tmap_2d(&tmSB, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sbcol, Ng, kslices, Ng * 4, BN, 1,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
   else
     tmSB = tmSA;
@@ -555,7 +559,7 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   p.K = static_cast<int32_t>(Kg);
   p.mblocks = static_cast<int32_t>((Mg + kPairM - 1) / kPairM);
   p.nblocks = static_cast<int32_t>((Ng + BN - 1) / BN);
-  p.kblocks = static_cast<int32_t>(Kg / BK);
+  p.kblocks = static_cast<int32_t>(kslices);
   p.n_fastest = Ng <= Mg ? 1 : 0;
   p.sb = sb;
   p.sb_sj = sb_sj;
@@ -582,16 +586,19 @@ extern "C" fp8q_status fp8q_linear_fwd(const uint8_t* qa, const float* sa, int64
                                        const uint8_t* qw, const float* sw, int64_t M, int64_t N,
                                        int64_t K, uint16_t* y, int64_t ldy, void* stream) {
   if (!qa || !sa || !qw || !sw || !y) return FP8Q_ERR_NULL;
-  if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % 128 || ldsa < M || ldy < N)
+  if (M <= 0 || N <= 0 || K <= 0 || N % 16 || K % 16 || ldsa < M || ldy < N)
     return FP8Q_ERR_SHAPE;
   if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y) ||
       ldsa % 4 || ldy % 8)
     return FP8Q_ERR_ALIGN;
-  // B = W [N][K]; block scale of (n, slice r) = sw[(n/128)*(K/128) + r]
-  if (M <= kSkinnyMaxM)
-    return launch_skinny_gemm(qa, qw, M, N, K, sa, ldsa, sw, K / 128, 1, y, ldy,
+  // B = W [N][K]; block scale of (n, slice r) = sw[(n/128)*KB + r], KB = ceil(K/128).
+  // The skinny kernel reads whole 128-wide slices and strips: ragged shapes take the
+  // pair kernel at any M (the same arithmetic in the same order).
+  const int64_t KB = (K + 127) / 128;
+  if (M <= kSkinnyMaxM && K % 128 == 0 && N % 128 == 0)
+    return launch_skinny_gemm(qa, qw, M, N, K, sa, ldsa, sw, KB, 1, y, ldy,
                               static_cast<cudaStream_t>(stream));
-  return launch_gemm<false, true>(qa, qw, M, N, K, sa, ldsa, sw, K / 128, 1, nullptr, y, ldy,
+  return launch_gemm<false, true>(qa, qw, M, N, K, sa, ldsa, sw, KB, 1, nullptr, y, ldy,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -600,17 +607,18 @@ extern "C" fp8q_status fp8q_linear_dgrad(const uint8_t* qdy, const float* sdy, i
                                          int64_t N, int64_t K, uint16_t* dx, int64_t lddx,
                                          void* stream) {
   if (!qdy || !sdy || !qwT || !sw || !dx) return FP8Q_ERR_NULL;
-  if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % 128 || ldsdy < M || lddx < K)
+  if (M <= 0 || N <= 0 || K <= 0 || N % 16 || K % 16 || ldsdy < M || lddx < K)
     return FP8Q_ERR_SHAPE;
   if (!aligned16(qdy) || !aligned16(sdy) || !aligned16(qwT) || !aligned16(sw) ||
       !aligned16(dx) || ldsdy % 4 || lddx % 8)
     return FP8Q_ERR_ALIGN;
   // GEMM rows = M, columns = K, reduction = N. B = W^T [K][N];
-  // block scale of (k, slice r over n) = sw[r*(K/128) + k/128]
-  if (M <= kSkinnyMaxM)
-    return launch_skinny_gemm(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, K / 128, dx, lddx,
+  // block scale of (k, slice r over n) = sw[r*KB + k/128], KB = ceil(K/128)
+  const int64_t KB = (K + 127) / 128;
+  if (M <= kSkinnyMaxM && K % 128 == 0 && N % 128 == 0)
+    return launch_skinny_gemm(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, KB, dx, lddx,
                               static_cast<cudaStream_t>(stream));
-  return launch_gemm<false, true>(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, K / 128, nullptr, dx, lddx,
+  return launch_gemm<false, true>(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, KB, nullptr, dx, lddx,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -619,7 +627,7 @@ extern "C" fp8q_status fp8q_linear_wgrad(const uint8_t* qdyT, const float* sdy_c
                                          int64_t N, int64_t K, uint16_t* dw, int64_t lddw,
                                          void* stream) {
   if (!qdyT || !sdy_c || !qxT || !sx_c || !dw) return FP8Q_ERR_NULL;
-  if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 128 || lddw < K)
+  if (M <= 0 || N <= 0 || K <= 0 || M % 16 || N % 16 || K % 16 || lddw < K)
     return FP8Q_ERR_SHAPE;
   if (!aligned16(qdyT) || !aligned16(sdy_c) || !aligned16(qxT) || !aligned16(sx_c) ||
       !aligned16(dw) || lddw % 8)
@@ -636,7 +644,7 @@ extern "C" fp8q_status fp8q_linear_wgrad_acc_f32(const uint8_t* qdyT, const floa
                                                  int64_t N, int64_t K, float* dw, int64_t lddw,
                                                  void* stream) {
   if (!qdyT || !sdy_c || !qxT || !sx_c || !dw) return FP8Q_ERR_NULL;
-  if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 128 || lddw < K)
+  if (M <= 0 || N <= 0 || K <= 0 || M % 16 || N % 16 || K % 16 || lddw < K)
     return FP8Q_ERR_SHAPE;
   if (!aligned16(qdyT) || !aligned16(sdy_c) || !aligned16(qxT) || !aligned16(sx_c) ||
       !aligned16(dw) || lddw % 4)

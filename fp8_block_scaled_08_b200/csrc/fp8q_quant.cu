@@ -143,6 +143,20 @@ __device__ __forceinline__ float quot(float x, const GroupScale& g) {
   return __fmaf_rn(en, -g.rs, q);
 }
 
+// quot on two values (of groups g0 and g1) with packed fp32 pair instructions: each
+// lane of a pair is the same IEEE operation as in quot, so the results are quot's bit
+// for bit.
+__device__ __forceinline__ void quot2(float x0, float x1, const GroupScale& g0,
+                                      const GroupScale& g1, float& t0, float& t1) {
+  float q0, q1;
+  mul2(q0, q1, x0, x1, g0.rs, g1.rs);
+  float e0 = -x0, e1 = -x1;
+  fma2(e0, e1, q0, q1, g0.s, g1.s);      // q*s - x
+  fma2(q0, q1, e0, e1, -g0.rs, -g1.rs);  // q - (q*s - x)*r
+  t0 = q0;
+  t1 = q1;
+}
+
 // Eight codes of BF16-valued x (packed little-endian into two words). Groups with a
 // tiny scale divide; the branch is per warp and only taken when a lane needs it.
 __device__ __forceinline__ uint2 codes8(const float (&v)[8], const GroupScale& g) {
@@ -152,7 +166,7 @@ __device__ __forceinline__ uint2 codes8(const float (&v)[8], const GroupScale& g
     for (int i = 0; i < 8; ++i) t[i] = g.small ? __fdiv_rn(v[i], g.s) : quot(v[i], g);
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) t[i] = quot(v[i], g);
+    for (int i = 0; i < 8; i += 2) quot2(v[i], v[i + 1], g, g, t[i], t[i + 1]);
   }
   return make_uint2(cvt_e4m3x4(t[0], t[1], t[2], t[3]), cvt_e4m3x4(t[4], t[5], t[6], t[7]));
 }
@@ -327,7 +341,8 @@ __global__ void __launch_bounds__(256) rowgroup_quant_kernel(Src src, int64_t M,
 #pragma unroll
     for (int j = 0; j < kUnroll; ++j) {
       const int64_t g = 2 * pp[j] + half;
-      act[j] = (mm[j] < M) && (g < G);
+      // columns past ldq (a partial last group) are zeros that are not stored
+      act[j] = (mm[j] < M) && (g < G) && (g * 128 + sub * 8 < ldq);
       if (act[j]) raw[j] = src.fetch(mm[j], g * 128 + sub * 8);
     }
 #pragma unroll
@@ -480,7 +495,7 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_warp2_kernel(
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        if (c0 + 32 * u >= nch) break;  // warp-uniform; nch is a multiple of 16
+        if (c0 + 32 * u >= nch) break;  // warp-uniform; lanes past nch hold zeros
         const int64_t c = c0 + lane + 32 * u;
         norm_quant_chunk(raw[u], reinterpret_cast<const uint16_t*>(gamma_sm), c, c < nch, r,
                          q + m * H, s, lds, m, lane);
@@ -526,7 +541,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_cta_kernel(
 #pragma unroll
     for (int j = 0; j < kNormMaxChunks; ++j) {
       const int64_t c0 = static_cast<int64_t>(j) * kNormThreads + (tid & ~31);
-      if (c0 >= nch) break;  // warp-uniform: nch is a multiple of 16
+      if (c0 >= nch) break;  // warp-uniform; lanes past nch (a partial group) hold zeros
       const int64_t c = tid + j * kNormThreads;
       norm_quant_chunk(raw[j], reinterpret_cast<const uint16_t*>(gamma_sm), c, c < nch, r,
                        q + m * H, s, lds, m, lane);
@@ -582,8 +597,7 @@ __device__ __forceinline__ void col_codes(const uint32_t (&w)[kR], const GroupSc
         t0[i] = g0.small ? __fdiv_rn(x0, g0.s) : quot(x0, g0);
         t1[i] = g1.small ? __fdiv_rn(x1, g1.s) : quot(x1, g1);
       } else {
-        t0[i] = quot(x0, g0);
-        t1[i] = quot(x1, g1);
+        quot2(x0, x1, g0, g1, t0[i], t1[i]);
       }
     }
     o0[k] = cvt_e4m3x4(t0[0], t0[1], t0[2], t0[3]);
@@ -595,11 +609,14 @@ __device__ __forceinline__ void col_codes(const uint32_t (&w)[kR], const GroupSc
 // threads: thread t takes column pair t % 64 over kR = 128 / (kThreads / 64) consecutive
 // rows. Column scales: computed per column (per_col; red holds kThreads / 64 x 128
 // floats) or the given block scale. Codes go to dst[c * ldd + r] for tile column c and
-// tile row r; per-column scales to scol[c].
+// tile row r; per-column scales to scol[c]. Only the first `rows` rows and `cols`
+// columns exist (a partial tile at the end of a ragged tensor, both multiples of 16;
+// the staged tile holds zeros beyond them); nothing is stored outside them.
 template <int kThreads = 256>
 __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, bool per_col,
                                                const GroupScale& blk, uint8_t* __restrict__ dst,
-                                               int64_t ldd, float* __restrict__ scol) {
+                                               int64_t ldd, float* __restrict__ scol,
+                                               int rows = 128, int cols = 128) {
   constexpr int kQ = kThreads / 64, kR = 128 / kQ;
   static_assert(kQ * 64 == kThreads && kR % 16 == 0, "column pass: 256 or 512 threads");
   const int tid = threadIdx.x;
@@ -625,17 +642,20 @@ __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, b
     }
     g0 = group_scale_bf16(c0);
     g1 = group_scale_bf16(c1);
-    if (rq == 0 && scol) *reinterpret_cast<float2*>(scol + 2 * cp) = make_float2(g0.s, g1.s);
+    if (rq == 0 && scol && 2 * cp < cols)
+      *reinterpret_cast<float2*>(scol + 2 * cp) = make_float2(g0.s, g1.s);
   }
   uint32_t o0[kR / 4], o1[kR / 4];
   if (__any_sync(kFull, g0.small || g1.small))
     col_codes<true, kR>(w, g0, g1, o0, o1);
   else
     col_codes<false, kR>(w, g0, g1, o0, o1);
+  if (2 * cp >= cols) return;  // cols is even: the pair is in or out together
   uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * ldd + kR * rq);
   uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * ldd + kR * rq);
 #pragma unroll
   for (int k = 0; k < kR / 16; ++k) {
+    if (kR * rq + 16 * k >= rows) break;  // rows is a multiple of 16
     d0[k] = make_uint4(o0[4 * k], o0[4 * k + 1], o0[4 * k + 2], o0[4 * k + 3]);
     d1[k] = make_uint4(o1[4 * k], o1[4 * k + 1], o1[4 * k + 2], o1[4 * k + 3]);
   }
@@ -706,7 +726,9 @@ __device__ __forceinline__ void tiles_drain(const TileSmem& sm, int64_t t_stop, 
   }
 }
 
-// a2: 128x128 weight blocks, persistent over the (N/128) x (K/128) tiles.
+// a2: 128x128 weight blocks, persistent over the ceil(N/128) x ceil(K/128) tiles. A
+// partial block at the end of a ragged N or K arrives zero-filled by the tensor copy
+// (zeros raise no maximum) and only its valid codes are stored.
 __global__ void __launch_bounds__(256) quant_weight_kernel(
     const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t K, uint8_t* __restrict__ q,
     float* __restrict__ s, uint8_t* __restrict__ qT, unsigned* err, uint64_t limit_ns) {
@@ -715,8 +737,8 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(
   __shared__ int abort_flag;
   const WaitCtl ctl{&abort_flag, err, limit_ns};
   if (threadIdx.x == 0) abort_flag = 0;
-  const int64_t KB = K >> 7;
-  const int64_t tiles = (N >> 7) * KB;
+  const int64_t KB = (K + 127) >> 7;
+  const int64_t tiles = ((N + 127) >> 7) * KB;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int rr = tid >> 4, c8 = (tid & 15) * 8;
   auto issue = [&](int b, int64_t t) {
@@ -750,14 +772,18 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(
     for (int k = 1; k < 8; ++k) amax = fmaxf(amax, sm.red[k]);
     const GroupScale g = group_scale_bf16(amax);
     if (tid == 0) s[nb * KB + kb] = g.s;
+    const int rows = N - nb * 128 < 128 ? static_cast<int>(N - nb * 128) : 128;
+    const int cols = K - kb * 128 < 128 ? static_cast<int>(K - kb * 128) : 128;
     uint8_t* qb = q + (nb * 128) * K + kb * 128 + c8;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float v[8];
       unpack_bf16x8(raw[j], v);
-      *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes8(v, g);
+      const uint2 codes = codes8(v, g);  // every lane: the scale branch is warp-collective
+      if (rr + 16 * j < rows && c8 < cols) *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes;
     }
-    if (qT) tile_cols_bf16(Ts, nullptr, false, g, qT + (kb * 128) * N + nb * 128, N, nullptr);
+    if (qT)
+      tile_cols_bf16(Ts, nullptr, false, g, qT + (kb * 128) * N + nb * 128, N, nullptr, rows, cols);
   }
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
@@ -832,7 +858,6 @@ struct SwigluBwd {
   const uint16_t* dh;
   int64_t I;
   static constexpr int kOut = 2;
-  static constexpr bool kDgamma = false;
   static constexpr bool kHeavy = true;  // long form: keep the row-batch loop rolled
   struct In { uint4 g, u, d; };
   struct Col {};
@@ -841,7 +866,7 @@ struct SwigluBwd {
     const uint16_t* row = gu + m * 2 * I;
     return In{ld_nc_v4(row + col), ld_nc_v4(row + I + col), ld_nc_v4(dh + m * I + col)};
   }
-  __device__ __forceinline__ void form(const In& in, int64_t /*m*/, const Col&, double (&)[8],
+  __device__ __forceinline__ void form(const In& in, int64_t /*m*/, const Col&,
                                        float (&v)[2][8]) const {
     float g[8], u[8], dh[8];
     unpack_bf16x8(in.g, g);
@@ -879,9 +904,152 @@ struct SwigluBwd {
   }
 };
 
+// ---------------------------------------------------------------------------
+// Exact sums of fp32 terms (the two reductions of the RMSNorm backward). A finite fp32
+// value is m * 2^(e - 149) with an integer m < 2^24 and e in [0, 253] (subnormals:
+// e = 0, no implicit bit). Bin b = e / 16 holds integers in units of 2^(16 b - 149); a
+// term adds m << (e % 16) (< 2^39) to its bin. Integer additions are exact, so the
+// bins' total is the exact sum of the terms, whatever order the additions take (with
+// fewer than 2^24 terms no bin can overflow). The total is rounded once at the end.
+// ---------------------------------------------------------------------------
+constexpr int kXBins = 16;
+
+struct XTerm {
+  int bin;
+  long long v;
+};
+
+__device__ __forceinline__ XTerm xterm(float t) {
+  const uint32_t u = __float_as_uint(t);
+  const uint32_t E = (u >> 23) & 0xFFu;
+  const uint32_t m = E ? ((u & 0x7FFFFFu) | 0x800000u) : (u & 0x7FFFFFu);
+  const int e = E ? static_cast<int>(E) - 1 : 0;
+  const long long v = static_cast<long long>(m) << (e & 15);
+  return XTerm{e >> 4, (u >> 31) ? -v : v};
+}
+
+// One exact sum per thread: the two bins last added to are cached in registers (the
+// terms of one sum usually span one or two bins); the others live in a separate array
+// `bins` (dynamically indexed, so in local memory), which takes a cached bin when a
+// third one is needed. `mask` has bit b set once bin b may be non-zero in either.
+struct XCache {
+  long long a0, a1;
+  int b0, b1;
+  uint32_t mask;
+  __device__ __forceinline__ void init(long long (&bins)[kXBins]) {
+#pragma unroll
+    for (int i = 0; i < kXBins; ++i) bins[i] = 0;
+    a0 = a1 = 0;
+    b0 = b1 = -1;
+    mask = 0;
+  }
+  __device__ __forceinline__ void add(float t, long long (&bins)[kXBins]) {
+    const XTerm x = xterm(t);
+    if (x.v == 0) return;
+    if (x.bin == b0) {
+      a0 += x.v;
+    } else if (x.bin == b1) {
+      a1 += x.v;
+    } else {
+      if (b1 >= 0) bins[b1] += a1;
+      b1 = b0;
+      a1 = a0;
+      b0 = x.bin;
+      a0 = x.v;
+      mask |= 1u << x.bin;
+    }
+  }
+  // Moves the cached bins into the array (once, after the last add).
+  __device__ __forceinline__ void flush(long long (&bins)[kXBins]) {
+    if (b0 >= 0) bins[b0] += a0;
+    if (b1 >= 0) bins[b1] += a1;
+    b0 = b1 = -1;
+  }
+};
+
+// The value sum_b A[b] * 2^(16 b - 149) rounded once to a double: to nearest, ties to
+// even, or, with `odd`, to odd (the last mantissa bit set when a lower bit is dropped;
+// a double rounded to odd and then rounded to nearest fp32 is the fp32 nearest to the
+// exact value, as 53 >= 24 + 2). An exact zero gives +0. Needs |A[b]| < 2^62.
+__device__ double xbins_round(const long long (&A)[kXBins], bool odd) {
+  // base-2^16 digits D[0..18] of the magnitude: the low 15 from a carry pass, the top bin
+  // (with its carry, < 2^63) split into four more
+  uint32_t D[kXBins + 3];
+  long long carry = 0;
+#pragma unroll
+  for (int b = 0; b < kXBins - 1; ++b) carry = (carry + A[b]) >> 16;
+  const bool neg = A[kXBins - 1] + carry < 0;
+  carry = 0;
+#pragma unroll
+  for (int b = 0; b < kXBins - 1; ++b) {
+    const long long t = (neg ? -A[b] : A[b]) + carry;
+    D[b] = static_cast<uint32_t>(t & 0xFFFF);
+    carry = t >> 16;  // arithmetic: the low digit stays in [0, 2^16)
+  }
+  unsigned long long top =
+      static_cast<unsigned long long>((neg ? -A[kXBins - 1] : A[kXBins - 1]) + carry);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) D[kXBins - 1 + i] = static_cast<uint32_t>((top >> (16 * i)) & 0xFFFF);
+  int h = -1;
+#pragma unroll
+  for (int i = 0; i < kXBins + 3; ++i)
+    if (D[i]) h = i;
+  if (h < 0) return 0.0;
+  // 64-bit window of digits h .. h-3 (missing digits are 0), left-aligned with bits of
+  // digit h-4; everything below is the sticky bit
+  unsigned long long w = 0;
+  for (int i = h; i > h - 4; --i) w = (w << 16) | (i >= 0 ? D[i] : 0u);
+  const uint32_t nxt = h - 4 >= 0 ? D[h - 4] : 0u;
+  bool sticky = false;
+  for (int i = h - 5; i >= 0; --i) sticky |= D[i] != 0;
+  const int lz = __clzll(static_cast<long long>(w));  // 0..15: digit h is non-zero
+  if (lz) {
+    w = (w << lz) | (nxt >> (16 - lz));
+    sticky |= (nxt & ((1u << (16 - lz)) - 1u)) != 0;
+  } else {
+    sticky |= nxt != 0;
+  }
+  // bit 63 of w has weight 2^e_top
+  int e_top = 16 * (h - 3) - lz - 149 + 63;
+  unsigned long long mant = w >> 11;  // 53 bits
+  const uint32_t rem = static_cast<uint32_t>(w & 0x7FF);
+  if (odd) {
+    if (rem || sticky) mant |= 1ull;
+  } else if (rem > 0x400u || (rem == 0x400u && (sticky || (mant & 1ull)))) {
+    ++mant;
+    if (mant >> 53) {
+      mant >>= 1;
+      ++e_top;
+    }
+  }
+  // normal double (e_top >= -149): sign, biased exponent, 52 fraction bits
+  const unsigned long long bits = (static_cast<unsigned long long>(neg) << 63) |
+                                  (static_cast<unsigned long long>(e_top + 1023) << 52) |
+                                  (mant & ((1ull << 52) - 1));
+  return __longlong_as_double(static_cast<long long>(bits));
+}
+
+// Sum over the warp of one exact sum per lane, rounded once to a double (the result is
+// returned to every lane).
+__device__ double warp_exact_sum(XCache& acc, long long (&bins)[kXBins], bool odd) {
+  acc.flush(bins);
+  const uint32_t used = __reduce_or_sync(kFull, acc.mask);
+  long long A[kXBins];
+#pragma unroll
+  for (int b = 0; b < kXBins; ++b) A[b] = 0;
+  for (uint32_t m = used; m; m &= m - 1) {
+    const int b = __ffs(m) - 1;
+    long long v = bins[b];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    A[b] = v;
+  }
+  return xbins_round(A, odd);
+}
+
 // Per-row scalars of the RMSNorm backward: r (as in the forward producer) and
-// k = (float)((((c r) r) r) / H) in fp64, c = sum_j fl32(fl32(gamma_j dy_j) x_j) in fp64
-// (each product exact: three 8-bit significands). One warp per row.
+// k = (float)((((c r) r) r) / H) in fp64, c = the exact sum of the fp32 products
+// fl32(fl32(gamma_j dy_j) x_j) rounded once to a double. One warp per row.
 __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma,
     const uint16_t* __restrict__ dy, int64_t M, int64_t H, float eps, float* __restrict__ r_out,
@@ -894,7 +1062,9 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
     const uint16_t* xr = x + m * H;
     const uint16_t* dr = dy + m * H;
     double ss[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-    double cc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    XCache cc;
+    long long cbins[kXBins];
+    cc.init(cbins);
     int64_t c = lane;
     for (; c + 32 < nch; c += 64) {  // two chunks of each operand in flight per lane
       uint4 rx[2], rd[2], rg[2];
@@ -914,8 +1084,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
         for (int i = 0; i < 8; ++i) {
           const double xd = static_cast<double>(xv[i]);
           ss[i] = __fma_rn(xd, xd, ss[i]);
-          const float t = __fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]);
-          cc[i] = __dadd_rn(cc[i], static_cast<double>(t));
+          cc.add(__fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]), cbins);
         }
       }
     }
@@ -928,19 +1097,14 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
       for (int i = 0; i < 8; ++i) {
         const double xd = static_cast<double>(xv[i]);
         ss[i] = __fma_rn(xd, xd, ss[i]);
-        const float t = __fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]);
-        cc[i] = __dadd_rn(cc[i], static_cast<double>(t));
+        cc.add(__fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]), cbins);
       }
     }
     double s2 = __dadd_rn(__dadd_rn(__dadd_rn(ss[0], ss[1]), __dadd_rn(ss[2], ss[3])),
                           __dadd_rn(__dadd_rn(ss[4], ss[5]), __dadd_rn(ss[6], ss[7])));
-    double c2 = __dadd_rn(__dadd_rn(__dadd_rn(cc[0], cc[1]), __dadd_rn(cc[2], cc[3])),
-                          __dadd_rn(__dadd_rn(cc[4], cc[5]), __dadd_rn(cc[6], cc[7])));
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      s2 = __dadd_rn(s2, __shfl_xor_sync(kFull, s2, off));
-      c2 = __dadd_rn(c2, __shfl_xor_sync(kFull, c2, off));
-    }
+    for (int off = 16; off >= 1; off >>= 1) s2 = __dadd_rn(s2, __shfl_xor_sync(kFull, s2, off));
+    const double c2 = warp_exact_sum(cc, cbins, false);
     if (lane == 0) {
       const float r = rstd_from_ss(s2, H, eps);
       const double rd = static_cast<double>(r);
@@ -955,9 +1119,8 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
 }
 
 // RMSNorm backward per element: out = bf16(bf16(dx) + dres) with
-// dx = fl32(fl32(r fl32(gamma dy)) - fl32(k x)); the terms fl32(dy fl32(x r)) of dgamma
-// are summed per column in fp64. A thread's chunk: 8 consecutive x, dy (and dres)
-// values of one row.
+// dx = fl32(fl32(r fl32(gamma dy)) - fl32(k x)) (dgamma has a kernel of its own). A
+// thread's chunk: 8 consecutive x, dy (and dres) values of one row.
 struct RmsBwd {
   const uint16_t* x;
   const uint16_t* dy;
@@ -967,7 +1130,6 @@ struct RmsBwd {
   const uint16_t* gamma;
   int64_t H;
   static constexpr int kOut = 1;
-  static constexpr bool kDgamma = true;
   static constexpr bool kHeavy = false;
   struct In { uint4 x, d, res; };
   struct Col { float g[8]; };
@@ -983,7 +1145,7 @@ struct RmsBwd {
     in.res = dres ? ld_nc_v4(dres + m * H + col) : make_uint4(0u, 0u, 0u, 0u);
     return in;
   }
-  __device__ __forceinline__ void form(const In& in, int64_t m, const Col& col, double (&dg)[8],
+  __device__ __forceinline__ void form(const In& in, int64_t m, const Col& col,
                                        float (&v)[1][8]) const {
     const float(&gv)[8] = col.g;
     float xv[8], dv[8], rv[8];
@@ -994,7 +1156,7 @@ struct RmsBwd {
     const bool res = dres != nullptr;
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-      float gd0, gd1, a0, a1, b0, b1, xr0, xr1, p0, p1;
+      float gd0, gd1, a0, a1, b0, b1;
       mul2(gd0, gd1, gv[i], gv[i + 1], dv[i], dv[i + 1]);
       mul2(a0, a1, gd0, gd1, rr, rr);
       mul2(b0, b1, xv[i], xv[i + 1], kk, kk);
@@ -1005,10 +1167,6 @@ struct RmsBwd {
       }
       v[0][i] = o0;
       v[0][i + 1] = o1;
-      mul2(xr0, xr1, xv[i], xv[i + 1], rr, rr);
-      mul2(p0, p1, dv[i], dv[i + 1], xr0, xr1);
-      dg[i] = __dadd_rn(dg[i], static_cast<double>(p0));
-      dg[i + 1] = __dadd_rn(dg[i + 1], static_cast<double>(p1));
     }
   }
 };
@@ -1018,7 +1176,6 @@ struct GradDirect {
   const uint16_t* dy;
   int64_t ld;
   static constexpr int kOut = 1;
-  static constexpr bool kDgamma = false;
   static constexpr bool kHeavy = false;
   struct In { uint4 a; };
   struct Col {};
@@ -1026,7 +1183,7 @@ struct GradDirect {
   __device__ __forceinline__ In load(int64_t m, int64_t col) const {
     return In{ld_nc_v4(dy + m * ld + col)};
   }
-  __device__ __forceinline__ void form(const In& in, int64_t, const Col&, double (&)[8],
+  __device__ __forceinline__ void form(const In& in, int64_t, const Col&,
                                        float (&v)[1][8]) const {
     unpack_bf16x8(in.a, v[0]);
   }
@@ -1039,7 +1196,6 @@ struct RmsDirect {
   const float* rstd;
   const uint16_t* gamma;
   static constexpr int kOut = 1;
-  static constexpr bool kDgamma = false;
   static constexpr bool kHeavy = false;
   struct In { uint4 a; };
   struct Col { float g[8]; };
@@ -1051,7 +1207,7 @@ struct RmsDirect {
   __device__ __forceinline__ In load(int64_t m, int64_t col) const {
     return In{ld_nc_v4(x + m * ldx + col)};
   }
-  __device__ __forceinline__ void form(const In& in, int64_t m, const Col& k, double (&)[8],
+  __device__ __forceinline__ void form(const In& in, int64_t m, const Col& k,
                                        float (&v)[1][8]) const {
     float xv[8];
     unpack_bf16x8(in.a, xv);
@@ -1072,7 +1228,6 @@ struct SwigluDirect {
   const uint16_t* gu;
   int64_t ldgu, I;
   static constexpr int kOut = 1;
-  static constexpr bool kDgamma = false;
   static constexpr bool kHeavy = true;
   struct In { uint4 g, u; };
   struct Col {};
@@ -1081,7 +1236,7 @@ struct SwigluDirect {
     const uint16_t* row = gu + m * ldgu;
     return In{ld_nc_v4(row + col), ld_nc_v4(row + I + col)};
   }
-  __device__ __forceinline__ void form(const In& in, int64_t, const Col&, double (&)[8],
+  __device__ __forceinline__ void form(const In& in, int64_t, const Col&,
                                        float (&v)[1][8]) const {
     float g[8], u[8];
     unpack_bf16x8(in.g, g);
@@ -1099,45 +1254,42 @@ constexpr int kFwdMinBlocks = 4;
 constexpr int kA6Batch = 4;
 constexpr int kA6MinBlocks = 4;
 
-// Shared memory of the backward kernels: the formed BF16 output tile(s), one column
-// reduction per output tile, the dgamma partials of the 8 warps (RMSNorm).
+// Shared memory of the unit kernels: the formed BF16 output tile(s) and one column
+// reduction per output tile.
 template <class X>
 constexpr size_t direct_smem_bytes() {
-  return X::kOut * (kTileElems * 2 + 4 * 128 * 4) + (X::kDgamma ? 8 * 128 * 8 : 0);
+  return X::kOut * (kTileElems * 2 + 4 * 128 * 4);
 }
 
-// Persistent over the (M/128) x NB units; unit t covers rows (t / NB) * 128 and input
-// columns (t % NB) * 128. Each thread loads its chunks (rows rr + 16 j, columns c8..c8+7)
-// straight into registers, kBatch rows at a time, forms the gradient, stores it in the
-// output tile(s) in shared memory (and in bf16_out if given) and quantizes its rows;
-// after one barrier the column pass runs on the staged tile(s). Output tile o is column
-// block o * NB + nb of the [M, Nout] gradient (Nout = kOut * NB * 128): for the SwiGLU
-// d_gate and d_up, for the RMSNorm the gradient itself. dg_part (RMSNorm) receives the
-// fp64 dgamma partial of each unit.
+// Persistent over the ceil(M/128) x NB units (NB = ceil(N/128)); unit t covers rows
+// (t / NB) * 128 and input columns (t % NB) * 128. Each thread loads its chunks (rows
+// rr + 16 j, columns c8..c8+7) straight into registers, kBatch rows at a time, forms the
+// gradient, stores it in the output tile(s) in shared memory (and in bf16_out if given)
+// and quantizes its rows; after one barrier the column pass runs on the staged tile(s).
+// Output tile o covers columns o * N + nb * 128 of the [M, Nout] output (Nout = kOut *
+// N): for the SwiGLU d_gate and d_up, for the RMSNorm the gradient itself. M and N must
+// be multiples of 16; the chunks of a partial unit past them are zeros (they raise no
+// group maximum) and are not stored.
 template <class X, int kBatch, int kMinBlocks>
 __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
-    X xf, int64_t M, int64_t NB, uint16_t* __restrict__ bf16_out, uint8_t* __restrict__ q_row,
+    X xf, int64_t M, int64_t N, uint16_t* __restrict__ bf16_out, uint8_t* __restrict__ q_row,
     float* __restrict__ s_row, int64_t lds_row, uint8_t* __restrict__ q_colT,
-    float* __restrict__ s_col, double* __restrict__ dg_part) {
+    float* __restrict__ s_col) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   constexpr int kOut = X::kOut;
   uint16_t* tile = reinterpret_cast<uint16_t*>(smem_raw);
   float* red = reinterpret_cast<float*>(smem_raw + kOut * kTileElems * 2);
-  double* dgs = reinterpret_cast<double*>(red + kOut * 4 * 128);  // [8 warps][128]
-  const int64_t Nout = kOut * NB * 128;
-  const int64_t tiles = (M >> 7) * NB;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t NB = (N + 127) >> 7;
+  const int64_t Nout = kOut * N;
+  const int64_t tiles = ((M + 127) >> 7) * NB;
+  const int tid = threadIdx.x;
   const int rr = tid >> 4, c8 = (tid & 15) * 8;
   const GroupScale unused{1.0f, 1.0f, -1.0f, false};
   for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
     const int64_t mb = t / NB, nb = t % NB;
     const int64_t col = nb * 128 + c8;
-    const typename X::Col cs = xf.column(col);
-    double dg[8];
-    if constexpr (X::kDgamma) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) dg[q] = 0.0;
-    }
+    const bool col_ok = col < N;  // N is a multiple of 8: a chunk is in or out
+    const typename X::Col cs = xf.column(col_ok ? col : 0);
     // unrolled for short forms; a long form (the SwiGLU exponential and divisions) stays
     // rolled, which keeps the kernel inside the instruction cache (measured faster)
     constexpr int kOuterUnroll = X::kHeavy ? 1 : 8 / kBatch;
@@ -1145,79 +1297,102 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
     for (int h = 0; h < 8 / kBatch; ++h) {
       typename X::In in[kBatch];
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) in[j] = xf.load(mb * 128 + rr + 16 * (h * kBatch + j), col);
+      for (int j = 0; j < kBatch; ++j) {
+        const int64_t m = mb * 128 + rr + 16 * (h * kBatch + j);
+        if (m < M && col_ok) in[j] = xf.load(m, col);
+        else in[j] = typename X::In{};
+      }
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int r = rr + 16 * (h * kBatch + j);
         const int64_t m = mb * 128 + r;
+        const bool ok = m < M && col_ok;
         float v[kOut][8];
-        xf.form(in[j], m, cs, dg, v);
+        xf.form(in[j], ok ? m : 0, cs, v);
 #pragma unroll
         for (int o = 0; o < kOut; ++o) {
-          const int64_t ob = o * NB + nb;
+          const int64_t oc = o * N + nb * 128 + c8;  // output column of this chunk
           const uint4 pk = make_uint4(pack_bf16x2(v[o][0], v[o][1]), pack_bf16x2(v[o][2], v[o][3]),
                                       pack_bf16x2(v[o][4], v[o][5]), pack_bf16x2(v[o][6], v[o][7]));
           *reinterpret_cast<uint4*>(tile + o * kTileElems + r * 128 + c8) = pk;
-          if (bf16_out) *reinterpret_cast<uint4*>(bf16_out + m * Nout + ob * 128 + c8) = pk;
+          if (bf16_out && ok) *reinterpret_cast<uint4*>(bf16_out + m * Nout + oc) = pk;
           if (q_row) {
             uint2 codes;
-            const float sc = quant_half_warp(v[o], codes);
-            *reinterpret_cast<uint2*>(q_row + m * Nout + ob * 128 + c8) = codes;
-            if ((tid & 15) == 0) s_row[ob * lds_row + m] = sc;
+            const float sc = quant_half_warp(v[o], codes);  // every lane takes part
+            if (ok) *reinterpret_cast<uint2*>(q_row + m * Nout + oc) = codes;
+            if ((tid & 15) == 0 && m < M) s_row[((o * N) / 128 + nb) * lds_row + m] = sc;
           }
         }
       }
     }
-    if constexpr (X::kDgamma) {  // dgamma: this warp's two row sets, per column
-#pragma unroll
-      for (int q = 0; q < 8; ++q) dg[q] = __dadd_rn(dg[q], __shfl_xor_sync(kFull, dg[q], 16));
-      if (lane < 16) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) dgs[warp * 128 + c8 + q] = dg[q];
-      }
-    }
     __syncthreads();
-    if constexpr (X::kDgamma) {
-      if (tid < 128) {
-        double a = dgs[tid];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) a = __dadd_rn(a, dgs[w * 128 + tid]);
-        dg_part[mb * (NB * 128) + nb * 128 + tid] = a;
-      }
-    }
     // Each column pass reads its tile into registers before its own barrier, so once
     // every thread is past the last one the tiles may be overwritten by the next unit.
+    const int rows = M - mb * 128 < 128 ? static_cast<int>(M - mb * 128) : 128;
+    const int cols = N - nb * 128 < 128 ? static_cast<int>(N - nb * 128) : 128;
 #pragma unroll
     for (int o = 0; o < kOut; ++o) {
-      const int64_t ob = o * NB + nb;
+      const int64_t oc0 = o * N + nb * 128;
       tile_cols_bf16<256>(tile + o * kTileElems, red + o * 4 * 128, true, unused,
-                          q_colT + (ob * 128) * M + mb * 128, M, s_col + mb * Nout + ob * 128);
+                          q_colT + oc0 * M + mb * 128, M, s_col + mb * Nout + oc0, rows, cols);
     }
   }
 }
 
-// dgamma_j = (float) of the fp64 sum of the unit partials over the row blocks: eight
-// lanes per column each sum a contiguous eighth of the row blocks in order, then the
-// eight sums combine in a fixed tree (lane pairs, pairs of pairs, halves); a fixed order,
-// so the result is the same on every run.
-__global__ void __launch_bounds__(256) dgamma_reduce_kernel(const double* __restrict__ part,
-                                                            int64_t MB, int64_t H,
-                                                            float* __restrict__ dgamma) {
-  const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t j = gt >> 3;
-  const int sub = threadIdx.x & 7;
-  const int64_t per = (MB + 7) / 8;
-  double a = 0.0;
-  if (j < H) {
-    const int64_t b0 = sub * per;
-    const int64_t b1 = b0 + per < MB ? b0 + per : MB;
-#pragma unroll 4
-    for (int64_t b = b0; b < b1; ++b) a = __dadd_rn(a, part[b * H + j]);
+// dgamma_j = the exact sum over rows of fl32(dy_mj * fl32(x_mj * r_m)), rounded once to
+// fp32. A warp takes a strip of 32 8-column chunks (one per lane) over kDgRows rows, keeps
+// each of its 8 columns as an exact sum, and adds each column's bins into the global
+// bins [H][kXBins] with 64-bit integer atomics: integer additions, so the order in which
+// the warps land does not matter.
+constexpr int kDgRows = 64;
+
+__global__ void __launch_bounds__(256) dgamma_exact_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ dy, const float* __restrict__ r,
+    int64_t M, int64_t H, unsigned long long* __restrict__ bins) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nch = H >> 3;
+  const int64_t strips = (nch + 31) / 32;
+  const int64_t rblocks = (M + kDgRows - 1) / kDgRows;
+  const int64_t wglobal = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t u = wglobal; u < strips * rblocks; u += nw) {
+    const int64_t ch = (u % strips) * 32 + lane;
+    const int64_t m0 = (u / strips) * kDgRows;
+    const int64_t m1 = m0 + kDgRows < M ? m0 + kDgRows : M;
+    if (ch >= nch) continue;  // lanes past the last chunk (H not a multiple of 256)
+    XCache acc[8];
+    long long cbins[8][kXBins];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q].init(cbins[q]);
+    for (int64_t m = m0; m < m1; ++m) {
+      float xv[8], dv[8];
+      unpack_bf16x8(ld_nc_v4(x + m * H + ch * 8), xv);
+      unpack_bf16x8(ld_nc_v4(dy + m * H + ch * 8), dv);
+      const float rm = __ldg(r + m);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q].add(__fmul_rn(dv[q], __fmul_rn(xv[q], rm)), cbins[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      acc[q].flush(cbins[q]);
+      unsigned long long* col = bins + (ch * 8 + q) * kXBins;
+      for (uint32_t mk = acc[q].mask; mk; mk &= mk - 1) {
+        const int b = __ffs(mk) - 1;
+        if (cbins[q][b]) atomicAdd(col + b, static_cast<unsigned long long>(cbins[q][b]));
+      }
+    }
   }
-  a = __dadd_rn(a, __shfl_xor_sync(kFull, a, 1));
-  a = __dadd_rn(a, __shfl_xor_sync(kFull, a, 2));
-  a = __dadd_rn(a, __shfl_xor_sync(kFull, a, 4));
-  if (j < H && sub == 0) dgamma[j] = __double2float_rn(a);
+}
+
+// dgamma from the bins (two's complement in the unsigned words), one thread per column.
+__global__ void __launch_bounds__(256) dgamma_round_kernel(const unsigned long long* __restrict__ bins,
+                                                           int64_t H, float* __restrict__ dgamma) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= H) return;
+  long long A[kXBins];
+#pragma unroll
+  for (int b = 0; b < kXBins; ++b) A[b] = static_cast<long long>(bins[j * kXBins + b]);
+  dgamma[j] = __double2float_rn(xbins_round(A, true));
 }
 
 // a8: saved FP8 activation tiles (1x128 groups) -> xhat = fl32(s * dec(q)) -> 128x1
@@ -1233,8 +1408,8 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
   __shared__ int abort_flag;
   const WaitCtl ctl{&abort_flag, err, limit_ns};
   if (threadIdx.x == 0) abort_flag = 0;
-  const int64_t KB = K >> 7;
-  const int64_t tiles = (M >> 7) * KB;
+  const int64_t KB = (K + 127) >> 7;
+  const int64_t tiles = ((M + 127) >> 7) * KB;
   const int tid = threadIdx.x;
   auto issue = [&](int b, int64_t t) {
     const int32_t mx = static_cast<int32_t>((t / KB) * 128), kx = static_cast<int32_t>(t % KB);
@@ -1279,7 +1454,11 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
                fmaxf(sm.red[256 + 2 * cp + 1], sm.red[384 + 2 * cp + 1]));
     const float s0 = (a0 == 0.0f) ? 1.0f : __fdiv_rn(a0, 448.0f);
     const float s1 = (a1 == 0.0f) ? 1.0f : __fdiv_rn(a1, 448.0f);
-    if (rq == 0) *reinterpret_cast<float2*>(sT + mb * K + kb * 128 + 2 * cp) = make_float2(s0, s1);
+    // a partial tile (ragged M or K) arrived zero-filled; store only its valid part
+    const int rows = M - mb * 128 < 128 ? static_cast<int>(M - mb * 128) : 128;
+    const bool col_ok = kb * 128 + 2 * cp < K;  // K is even: the pair is in or out
+    if (rq == 0 && col_ok)
+      *reinterpret_cast<float2*>(sT + mb * K + kb * 128 + 2 * cp) = make_float2(s0, s1);
     uint32_t o0[8], o1[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -1291,10 +1470,14 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
     uint8_t* dst = qT + (kb * 128) * M + mb * 128;
     uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * M + 32 * rq);
     uint4* d1 = reinterpret_cast<uint4*>(dst + (2 * cp + 1) * M + 32 * rq);
-    d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-    d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
-    d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-    d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+    if (col_ok && 32 * rq < rows) {  // rows is a multiple of 16
+      d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+      d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+    }
+    if (col_ok && 32 * rq + 16 < rows) {
+      d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
+      d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+    }
   }
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
@@ -1331,10 +1514,10 @@ using namespace fp8q;
 extern "C" fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                                             uint8_t* q, float* s, int64_t lds, void* stream) {
   if (!x || !q || !s) return FP8Q_ERR_NULL;
-  if (M <= 0 || K <= 0 || K % 128 || ldx < K || lds < M || lds % 4) return FP8Q_ERR_SHAPE;
+  if (M <= 0 || K <= 0 || K % 16 || ldx < K || lds < M || lds % 4) return FP8Q_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(q) || !aligned16(s) || ldx % 8) return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  const int64_t G = K / 128;
+  const int64_t G = (K + 127) / 128;
   const int64_t units = M * ((G + 1) / 2);
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(rowgroup_quant_kernel<ActSrc, 4>, 256, 0, occ);
@@ -1347,10 +1530,10 @@ extern "C" fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_
 extern "C" fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t I, int64_t ldgu,
                                          uint8_t* q, float* s, int64_t lds, void* stream) {
   if (!gu || !q || !s) return FP8Q_ERR_NULL;
-  if (M <= 0 || I <= 0 || I % 128 || ldgu < 2 * I || lds < M || lds % 4) return FP8Q_ERR_SHAPE;
+  if (M <= 0 || I <= 0 || I % 16 || ldgu < 2 * I || lds < M || lds % 4) return FP8Q_ERR_SHAPE;
   if (!aligned16(gu) || !aligned16(q) || !aligned16(s) || ldgu % 8) return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  const int64_t G = I / 128;
+  const int64_t G = (I + 127) / 128;
   const int64_t units = M * ((G + 1) / 2);
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(rowgroup_quant_kernel<SwigluSrc, 2>, 256, 0, occ);
@@ -1364,7 +1547,7 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
                                           int64_t H, int64_t ldx, float eps, uint8_t* q, float* s,
                                           int64_t lds, void* stream) {
   if (!x || !gamma || !q || !s) return FP8Q_ERR_NULL;
-  if (M <= 0 || H <= 0 || H % 128 || H > 8 * kNormMaxChunks * kNormThreads || ldx < H ||
+  if (M <= 0 || H <= 0 || H % 16 || H > 8 * kNormMaxChunks * kNormThreads || ldx < H ||
       lds < M || lds % 4 || !(eps >= 0.0f))
     return FP8Q_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(q) || !aligned16(s) || ldx % 8)
@@ -1393,7 +1576,7 @@ extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, i
                                                  int64_t ldw, uint8_t* q, float* s, uint8_t* qT,
                                                  void* stream) {
   if (!w || !q || !s) return FP8Q_ERR_NULL;
-  if (N <= 0 || K <= 0 || N % 128 || K % 128 || ldw < K) return FP8Q_ERR_SHAPE;
+  if (N <= 0 || K <= 0 || N % 16 || K % 16 || ldw < K) return FP8Q_ERR_SHAPE;
   if (!aligned16(w) || !aligned16(q) || !aligned16(s) || (qT && !aligned16(qT)) || ldw % 8)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
@@ -1405,7 +1588,7 @@ extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, i
   if (!err) return FP8Q_ERR_CUDA;
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(quant_weight_kernel, 256, kTileSmemBF16, occ);
-  quant_weight_kernel<<<grid_for((N / 128) * (K / 128), per_sm), 256, kTileSmemBF16,
+  quant_weight_kernel<<<grid_for(((N + 127) / 128) * ((K + 127) / 128), per_sm), 256, kTileSmemBF16,
                         static_cast<cudaStream_t>(stream)>>>(tm, N, K, q, s, qT, err, kWaitLimitNs);
   return launch_status("quant_weight_128x128 launch");
 }
@@ -1415,7 +1598,7 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
                                                  int64_t lds_row, uint8_t* q_colT, float* s_col,
                                                  void* stream) {
   if (!dy || !q_colT || !s_col || (q_row != nullptr) != (s_row != nullptr)) return FP8Q_ERR_NULL;
-  if (M <= 0 || N <= 0 || M % 128 || N % 128 || lddy < N || (q_row && (lds_row < M || lds_row % 4)))
+  if (M <= 0 || N <= 0 || M % 16 || N % 16 || lddy < N || (q_row && (lds_row < M || lds_row % 4)))
     return FP8Q_ERR_SHAPE;
   if (!aligned16(dy) || !aligned16(q_colT) || !aligned16(s_col) || lddy % 8 ||
       (q_row && (!aligned16(q_row) || !aligned16(s_row))))
@@ -1425,8 +1608,9 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
   auto kern = direct_dual_kernel<GradDirect, kA6Batch, kA6MinBlocks>;
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
-  kern<<<grid_for((M / 128) * (N / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      GradDirect{dy, lddy}, M, N / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col, nullptr);
+  kern<<<grid_for(((M + 127) / 128) * ((N + 127) / 128), per_sm), 256, kSmem,
+         static_cast<cudaStream_t>(stream)>>>(
+      GradDirect{dy, lddy}, M, N, nullptr, q_row, s_row, lds_row, q_colT, s_col);
   return launch_status("transpose_quant_bf16 launch");
 }
 
@@ -1434,21 +1618,22 @@ extern "C" fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s
                                                 int64_t K, int64_t lds, uint8_t* qT, float* sT,
                                                 void* stream) {
   if (!q || !s || !qT || !sT) return FP8Q_ERR_NULL;
-  if (M <= 0 || K <= 0 || M % 128 || K % 128 || lds < M) return FP8Q_ERR_SHAPE;
+  if (M <= 0 || K <= 0 || M % 16 || K % 16 || lds < M) return FP8Q_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(s) || !aligned16(qT) || !aligned16(sT) || lds % 4)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
+  const int64_t KB = (K + 127) / 128;
   CUtensorMap tmq, tms;
   if (!encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, M, K, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_tmap_2d(&tms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, s, M, K / 128, lds * 4, 128, 1,
+      !encode_tmap_2d(&tms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, s, M, KB, lds * 4, 128, 1,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
     return FP8Q_ERR_UNSUPPORTED;
   unsigned* err = device_error_word();
   if (!err) return FP8Q_ERR_CUDA;
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(transpose_quant_fp8_kernel, 256, kTileSmemFP8, occ);
-  transpose_quant_fp8_kernel<<<grid_for((M / 128) * (K / 128), per_sm), 256, kTileSmemFP8,
+  transpose_quant_fp8_kernel<<<grid_for(((M + 127) / 128) * KB, per_sm), 256, kTileSmemFP8,
                                static_cast<cudaStream_t>(stream)>>>(tmq, tms, M, K, qT, sT, err,
                                                                     kWaitLimitNs);
   return launch_status("transpose_quant_fp8 launch");
@@ -1479,8 +1664,7 @@ extern "C" fp8q_status fp8q_rmsnorm_quant_dual(const uint16_t* x, const uint16_t
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (H / 128), per_sm), 256, kSmem, st>>>(
-      RmsDirect{x, ldx, rstd, gamma}, M, H / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col,
-      nullptr);
+      RmsDirect{x, ldx, rstd, gamma}, M, H, nullptr, q_row, s_row, lds_row, q_colT, s_col);
   return launch_status("rmsnorm_quant_dual launch");
 }
 
@@ -1500,7 +1684,7 @@ extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      SwigluDirect{gu, ldgu, I}, M, I / 128, nullptr, q_row, s_row, lds_row, q_colT, s_col, nullptr);
+      SwigluDirect{gu, ldgu, I}, M, I, nullptr, q_row, s_row, lds_row, q_colT, s_col);
   return launch_status("swiglu_quant_dual launch");
 }
 
@@ -1519,17 +1703,19 @@ extern "C" fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      SwigluBwd{gu, dh, I}, M, I / 128, dgu, q_row, s_row, lds_row, q_colT, s_col, nullptr);
+      SwigluBwd{gu, dh, I}, M, I, dgu, q_row, s_row, lds_row, q_colT, s_col);
   return launch_status("swiglu_bwd_quant_dual launch");
 }
 
 namespace {
 int64_t rmsnorm_bwd_ws_scalars(int64_t M) { return (8 * M + 255) / 256 * 256; }
+// dgamma's exact bins hold fewer than 2^23 terms of < 2^39 each: no int64 overflow
+constexpr int64_t kRmsBwdMaxRows = int64_t{1} << 23;
 }  // namespace
 
 extern "C" int64_t fp8q_rmsnorm_bwd_workspace_bytes(int64_t M, int64_t H) {
-  if (M <= 0 || H <= 0 || M % 128 || H % 128) return -1;
-  return rmsnorm_bwd_ws_scalars(M) + (M / 128) * H * 8;
+  if (M <= 0 || H <= 0 || M % 128 || H % 128 || M > kRmsBwdMaxRows) return -1;
+  return rmsnorm_bwd_ws_scalars(M) + H * kXBins * 8;
 }
 
 extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
@@ -1539,7 +1725,8 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
     void* stream) {
   if (!x || !gamma || !dy || !out || !q_row || !s_row || !q_colT || !s_col || !workspace)
     return FP8Q_ERR_NULL;
-  if (M <= 0 || H <= 0 || M % 128 || H % 128 || lds_row < M || lds_row % 4 || !(eps >= 0.0f))
+  if (M <= 0 || H <= 0 || M % 128 || H % 128 || lds_row < M || lds_row % 4 || !(eps >= 0.0f) ||
+      M > kRmsBwdMaxRows)
     return FP8Q_ERR_SHAPE;
   if (workspace_bytes < fp8q_rmsnorm_bwd_workspace_bytes(M, H)) {
     set_last_error_text("rmsnorm_bwd_quant_dual: workspace smaller than "
@@ -1556,7 +1743,7 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* r = reinterpret_cast<float*>(ws);
   float* k = r + M;
-  double* part = reinterpret_cast<double*>(ws + rmsnorm_bwd_ws_scalars(M));
+  unsigned long long* bins = reinterpret_cast<unsigned long long*>(ws + rmsnorm_bwd_ws_scalars(M));
   // per-row r and k first (one warp per row), then the tiles, then dgamma
   const int64_t row_ctas = std::min<int64_t>((M + 7) / 8, static_cast<int64_t>(sms) * 8);
   rmsnorm_bwd_rows_kernel<<<static_cast<int>(row_ctas), 256, 0, st>>>(x, gamma, dy, M, H, eps, r, k);
@@ -1567,11 +1754,18 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
   static std::atomic<int> occ[64];
   const int per_sm = resident_ctas(kern, 256, kSmem, occ);
   kern<<<grid_for((M / 128) * (H / 128), per_sm), 256, kSmem, st>>>(
-      RmsBwd{x, dy, dres, r, k, gamma, H}, M, H / 128, out, q_row, s_row, lds_row, q_colT, s_col,
-      part);
+      RmsBwd{x, dy, dres, r, k, gamma, H}, M, H, out, q_row, s_row, lds_row, q_colT, s_col);
   s1 = launch_status("rmsnorm_bwd_quant_dual launch");
   if (s1 != FP8Q_OK || !dgamma) return s1;
-  dgamma_reduce_kernel<<<static_cast<int>((H * 8 + 255) / 256), 256, 0, st>>>(part, M / 128, H,
-                                                                             dgamma);
-  return launch_status("dgamma_reduce launch");
+  // exact dgamma: the bins start at zero, the warps add into them, one thread per
+  // column rounds
+  if (cudaMemsetAsync(bins, 0, static_cast<size_t>(H) * kXBins * 8, st) != cudaSuccess)
+    return launch_status("dgamma bins clear");
+  const int64_t dg_warps = ((H / 8 + 31) / 32) * ((M + kDgRows - 1) / kDgRows);
+  const int64_t dg_ctas = std::min<int64_t>((dg_warps + 7) / 8, static_cast<int64_t>(sms) * 8);
+  dgamma_exact_kernel<<<static_cast<int>(dg_ctas), 256, 0, st>>>(x, dy, r, M, H, bins);
+  s1 = launch_status("dgamma_exact launch");
+  if (s1 != FP8Q_OK) return s1;
+  dgamma_round_kernel<<<static_cast<int>((H + 255) / 256), 256, 0, st>>>(bins, H, dgamma);
+  return launch_status("dgamma_round launch");
 }

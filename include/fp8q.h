@@ -16,14 +16,21 @@
  *          ties to even, saturating at +-448, sign kept (so -0 encodes as 0x80).
  *   BF16   passed as uint16_t bit patterns.
  *
- * Layouts (row-major; "ld" is a row stride in elements)
+ * Layouts (row-major; "ld" is a row stride in elements; G(n) = ceil(n / 128) is the
+ * number of groups along a dimension of n elements)
  *   codes         uint8_t [rows][cols], dense (row stride = cols).
- *   1x128 scales  float [cols/128][lds]: scale of (row m, group g) at s[g*lds + m].
+ *   1x128 scales  float [G(cols)][lds]: scale of (row m, group g) at s[g*lds + m].
  *                 lds >= rows, lds % 4 == 0 (the GEMMs load 128 row scales of one
  *                 group as one contiguous 512-byte run).
- *   128x128       float [N/128][K/128].
- *   128x1 scales  float [rows/128][cols]: scale of (row group mb, column c) at
+ *   128x128       float [G(N)][G(K)].
+ *   128x1 scales  float [G(rows)][cols]: scale of (row group mb, column c) at
  *                 s[mb*cols + c]; the codes of such groups are stored transposed.
+ *
+ * Partial groups. A dimension that is not a multiple of 128 ends in a partial group
+ * (the scheme fixes the 1x128 / 128x128 groupings, not what happens at a ragged edge;
+ * this library's reading): the group is the full group with zeros in the missing
+ * places, so its scale comes from its valid elements alone, and only the valid codes
+ * are stored. The GEMMs' last K slice is likewise partial (zeros add nothing).
  *
  * Conventions
  *   - Every pointer is a DEVICE pointer owned by the caller; the library allocates
@@ -33,8 +40,11 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Each call validates
  *     its arguments synchronously, then enqueues its kernels on `stream` (one kernel;
  *     two for fp8q_rmsnorm_quant_dual, up to three for fp8q_rmsnorm_bwd_quant_dual).
- *   - Shapes: K (the grouped / reduction dimension) % 128 == 0 everywhere;
- *     weight N % 128 == 0; M % 128 == 0 on the 128x1 paths; otherwise M >= 1.
+ *   - Shapes: a grouped or reduction dimension is a multiple of 16 (the tensor
+ *     copies need 16-byte rows of codes); a token dimension M that no group runs
+ *     along is any M >= 1. The fused producers with both groupings and the backward
+ *     producers (fp8q_*_quant_dual, fp8q_*_bwd_*) and the split-K forward still need
+ *     multiples of 128 where their groups run.
  *   - Alignment: every pointer 16-byte aligned; BF16 row strides % 8 == 0.
  *   - No call aborts or throws; each returns an fp8q_status.
  *   - Thread safety: re-entrant; calls on different streams may overlap, except
@@ -52,8 +62,8 @@ extern "C" {
 typedef int fp8q_status;
 #define FP8Q_OK 0
 #define FP8Q_ERR_NULL 1        /* a required pointer is NULL                        */
-#define FP8Q_ERR_SHAPE 2       /* a size is <= 0, not a multiple of 128 where
-                                  required, or a leading dimension is too small      */
+#define FP8Q_ERR_SHAPE 2       /* a size is <= 0, not a multiple of 16 (or 128)
+                                  where required, or a leading dimension too small   */
 #define FP8Q_ERR_ALIGN 3       /* a pointer or row stride breaks 16-byte alignment   */
 #define FP8Q_ERR_CUDA 4        /* the launch failed (cudaGetLastError)               */
 #define FP8Q_ERR_TIMEOUT 5     /* a kernel gave up a bounded wait (device error word) */
@@ -80,17 +90,17 @@ fp8q_status fp8q_last_device_error(void* stream);
 /* a1. Activation quantization per 1x128 group ("Esquema de Cuantización",
  * activations bullet).
  *   x  [M][K] BF16, row stride ldx (>= K, % 8 == 0)
- *   q  [M][K] FP8 codes (dense)        s [K/128][lds] fp32 (1x128 layout)
- * Requires M >= 1, K % 128 == 0. */
+ *   q  [M][K] FP8 codes (dense)        s [G(K)][lds] fp32 (1x128 layout)
+ * Requires M >= 1, K % 16 == 0. */
 fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                                  uint8_t* q, float* s, int64_t lds, void* stream);
 
 /* a2. Weight quantization per 128x128 block ("Esquema de Cuantización", weights
  * bullet). Run once per optimizer step from the BF16 master weights
  * ("Arquitectura Central", master weights bullet).
- *   w  [N][K] BF16, row stride ldw     q [N][K] codes   s [N/128][K/128] fp32
+ *   w  [N][K] BF16, row stride ldw     q [N][K] codes   s [G(N)][G(K)] fp32
  *   qT [K][N] codes: the same codes transposed (the DGrad operand); may be NULL.
- * Requires N % 128 == 0, K % 128 == 0. */
+ * Requires N % 16 == 0, K % 16 == 0. */
 fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
                                       uint8_t* q, float* s, uint8_t* qT, void* stream);
 
@@ -100,8 +110,8 @@ fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, int64_t K, i
  *   y_i = bf16( fl32( fl32(x_i * r) * gamma_i ) ),
  *   r   = (float)(1 / sqrt(sum_i x_i^2 / H + eps)) computed in fp64,
  * then the 1x128 quantization of y.
- *   x [M][H] BF16 (row stride ldx), gamma [H] BF16, q [M][H], s [H/128][lds].
- * Requires H % 128 == 0 and H <= 16384. */
+ *   x [M][H] BF16 (row stride ldx), gamma [H] BF16, q [M][H], s [G(H)][lds].
+ * The mean runs over the H elements of the row. Requires H % 16 == 0, H <= 16384. */
 fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, int64_t M,
                                int64_t H, int64_t ldx, float eps, uint8_t* q, float* s,
                                int64_t lds, void* stream);
@@ -112,15 +122,15 @@ fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, int64_t
  *   h = bf16( fl32( fl32(g / fl32(1 + E(-g))) * u ) ),
  * with E the library's fixed fp32 exponential (Cody-Waite range reduction and a
  * degree-7 Taylor polynomial, argument clamped to [-80, 88]), then the 1x128
- * quantization of h:  q [M][I], s [I/128][lds].   Requires I % 128 == 0. */
+ * quantization of h:  q [M][I], s [G(I)][lds].   Requires I % 16 == 0. */
 fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t I, int64_t ldgu,
                               uint8_t* q, float* s, int64_t lds, void* stream);
 
 /* a6. The BF16 gradient dY quantized for both backward GEMMs in one pass
  * ("Esquema de Cuantización", backward bullets; "Implementación", transposition):
- *   row-wise 1x128 for DGrad:  q_row [M][N], s_row [N/128][lds_row]  (may be NULL)
- *   column-wise 128x1 for WGrad, stored transposed: q_colT [N][M], s_col [M/128][N].
- *   dy [M][N] BF16, row stride lddy.  Requires M % 128 == 0, N % 128 == 0. */
+ *   row-wise 1x128 for DGrad:  q_row [M][N], s_row [G(N)][lds_row]  (may be NULL)
+ *   column-wise 128x1 for WGrad, stored transposed: q_colT [N][M], s_col [G(M)][N].
+ *   dy [M][N] BF16, row stride lddy.  Requires M % 16 == 0, N % 16 == 0. */
 fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, int64_t N,
                                       int64_t lddy, uint8_t* q_row, float* s_row,
                                       int64_t lds_row, uint8_t* q_colT, float* s_col,
@@ -174,26 +184,28 @@ fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint16_t* dh, i
                                        void* stream);
 
 /* Bytes of device workspace fp8q_rmsnorm_bwd_quant_dual needs for (M, H): per-row
- * scalars and one fp64 dgamma partial per 128-row block and column. -1 for a shape it
+ * scalars and, per column, the 16 integer words of dgamma's exact sum. -1 for a shape it
  * does not accept. */
 int64_t fp8q_rmsnorm_bwd_workspace_bytes(int64_t M, int64_t H);
 
-/* RMSNorm backward plus the residual gradient. x [M][H] (the forward input), gamma [H],
- * dy [M][H] (the gradient of the normalized output), dres [M][H] (the gradient arriving
- * along the residual stream; NULL = none), Nout = H. With r the forward producer's
- * reciprocal RMS of the row (fp64 sum of squares), c = sum_j (gamma_j dy_j) x_j in fp64
- * (each product exact in fp32) and k = (float)((((c r) r) r) / H) in fp64:
+/* RMSNorm backward plus the residual gradient (Jet-RL summary, "Esquema de
+ * Cuantización": gradients between operators stay BF16; the formulas are the operator's
+ * derivative). x [M][H] (the forward input), gamma [H], dy [M][H] (the gradient of the
+ * normalized output), dres [M][H] (the gradient arriving along the residual stream;
+ * NULL = none), Nout = H. With r the forward producer's reciprocal RMS of the row (fp64
+ * sum of squares), c = the exact sum over j of fl32(fl32(gamma_j dy_j) x_j) rounded once
+ * to a double, and k = (float)((((c r) r) r) / H) in fp64:
  *   dx_j  = bf16(fl32(fl32(r * fl32(gamma_j * dy_j)) - fl32(k * x_j))),
  *   out_j = bf16(fl32(dx_j + dres_j))  (out_j = dx_j without dres),
- *   dgamma_j = (float) sum over rows of fl32(dy_mj * fl32(x_mj * r_m)), summed in fp64.
+ *   dgamma_j = the exact sum over rows of fl32(dy_mj * fl32(x_mj * r_m)), rounded once
+ *              to fp32.
+ * The two sums are exact (integer bins), so no summation order enters the results.
  * out [M][H] (BF16, required: the gradient continues along the residual stream) and
- * its two quantizations; dgamma [H] fp32 if not NULL. The fp64 sums are blocked, so
- * their last bits can differ from a sequential sum: out, k and dgamma agree with a
- * sequential evaluation except where the exact value lies within that difference of
- * a rounding boundary; the codes always equal the quantization of `out`.
+ * its two quantizations; dgamma [H] fp32 if not NULL.
  * workspace: device memory of fp8q_rmsnorm_bwd_workspace_bytes(M, H) bytes, 16-byte
  * aligned, used only during the call's kernels (calls sharing one workspace must be
- * ordered on one stream). Requires H % 128 == 0, eps >= 0. */
+ * ordered on one stream; it needs no initialisation). Requires H % 128 == 0, eps >= 0,
+ * M <= 2^23 (FP8Q_ERR_SHAPE otherwise). */
 fp8q_status fp8q_rmsnorm_bwd_quant_dual(const uint16_t* x, const uint16_t* gamma,
                                         const uint16_t* dy, const uint16_t* dres, int64_t M,
                                         int64_t H, float eps, uint16_t* out, uint8_t* q_row,
@@ -203,8 +215,8 @@ fp8q_status fp8q_rmsnorm_bwd_quant_dual(const uint16_t* x, const uint16_t* gamma
 
 /* a8. The saved FP8 activation (1x128 groups) re-grouped 128x1 for WGrad:
  * xhat = fl32(s * dec(q)), then 128x1 quantization along M, stored transposed.
- *   q [M][K] codes, s [K/128][lds]  ->  qT [K][M] codes, sT [M/128][K].
- * Requires M % 128 == 0, K % 128 == 0. */
+ *   q [M][K] codes, s [G(K)][lds]  ->  qT [K][M] codes, sT [G(M)][K].
+ * Requires M % 16 == 0, K % 16 == 0. */
 fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s, int64_t M,
                                      int64_t K, int64_t lds, uint8_t* qT, float* sT,
                                      void* stream);
@@ -214,8 +226,9 @@ fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s, int64_t M
  *   Y[m,n] = sum_kb  sa[kb][m] * sw[n/128][kb] * sum_{k in kb} qa[m,k] * qw[n,k]
  * accumulated in fp32 one 128-wide K slice at a time, in increasing kb, then
  * rounded to BF16. Row m of Y does not depend on M (batch invariant).
- *   qa [M][K], sa [K/128][ldsa], qw [N][K], sw [N/128][K/128], y [M][N] BF16 (ldy).
- * Requires N % 128 == 0, K % 128 == 0, M >= 1. */
+ *   qa [M][K], sa [G(K)][ldsa], qw [N][K], sw [G(N)][G(K)], y [M][N] BF16 (ldy).
+ * Requires N % 16 == 0, K % 16 == 0, M >= 1. A ragged K or N at M <= 256 runs on the
+ * large-tile kernel (the same arithmetic in the same order as the decode kernel). */
 fp8q_status fp8q_linear_fwd(const uint8_t* qa, const float* sa, int64_t ldsa,
                             const uint8_t* qw, const float* sw, int64_t M, int64_t N,
                             int64_t K, uint16_t* y, int64_t ldy, void* stream);
@@ -266,8 +279,8 @@ fp8q_status fp8q_linear_fwd_splitk_noalloc(const uint8_t* qa, const float* sa, i
  *   dX[m,k] = sum_nb sdy[nb][m] * sw[nb][k/128] * sum_{n in nb} qdy[m,n] * qw[n,k]
  * with the row-wise dY codes of fp8q_transpose_quant_bf16 and the transposed
  * weight codes qwT [K][N] of fp8q_quant_weight_128x128.
- *   qdy [M][N], sdy [N/128][ldsdy], qwT [K][N], sw [N/128][K/128], dx [M][K] (lddx).
- * Requires N % 128 == 0, K % 128 == 0, M >= 1. */
+ *   qdy [M][N], sdy [G(N)][ldsdy], qwT [K][N], sw [G(N)][G(K)], dx [M][K] (lddx).
+ * Requires N % 16 == 0, K % 16 == 0, M >= 1. */
 fp8q_status fp8q_linear_dgrad(const uint8_t* qdy, const float* sdy, int64_t ldsdy,
                               const uint8_t* qwT, const float* sw, int64_t M, int64_t N,
                               int64_t K, uint16_t* dx, int64_t lddx, void* stream);
@@ -275,9 +288,9 @@ fp8q_status fp8q_linear_dgrad(const uint8_t* qdy, const float* sdy, int64_t ldsd
 /* a9. WGrad in FP8 with 1x128 / 128x1 grouping ("Esquema de Cuantización"): both
  * operands grouped along the reduction dimension M (tokens):
  *   dW[n,k] = sum_mb sdy_c[mb][n] * sx_c[mb][k] * sum_{m in mb} qdyT[n,m] * qxT[k,m]
- *   qdyT [N][M], sdy_c [M/128][N] (from fp8q_transpose_quant_bf16),
- *   qxT [K][M], sx_c [M/128][K] (from fp8q_transpose_quant_fp8), dw [N][K] BF16 (lddw).
- * Requires M % 128 == 0, N % 128 == 0, K % 128 == 0. */
+ *   qdyT [N][M], sdy_c [G(M)][N] (from fp8q_transpose_quant_bf16),
+ *   qxT [K][M], sx_c [G(M)][K] (from fp8q_transpose_quant_fp8), dw [N][K] BF16 (lddw).
+ * Requires M % 16 == 0, N % 16 == 0, K % 16 == 0. */
 fp8q_status fp8q_linear_wgrad(const uint8_t* qdyT, const float* sdy_c, const uint8_t* qxT,
                               const float* sx_c, int64_t M, int64_t N, int64_t K,
                               uint16_t* dw, int64_t lddw, void* stream);

@@ -84,7 +84,7 @@ def call(name, *args):
 def test_validation_act_quant():
     f = "fp8q_quant_act_1x128"
     assert call(f, NUL, 8, 128, 128, B, C, 8, NUL) == 1
-    assert call(f, A, 8, 100, 128, B, C, 8, NUL) == 2        # K % 128
+    assert call(f, A, 8, 100, 128, B, C, 8, NUL) == 2        # K % 16
     assert call(f, A, 0, 128, 128, B, C, 8, NUL) == 2        # M <= 0
     assert call(f, A, 8, 128, 128, B, C, 6, NUL) == 2        # lds % 4
     assert call(f, A, 8, 128, 128, B, C, 4, NUL) == 2        # lds < M
@@ -94,14 +94,14 @@ def test_validation_act_quant():
 
 
 def test_validation_gemms():
-    assert call("fp8q_linear_fwd", A, B, 16, C, D, 16, 200, 128, E, 256, NUL) == 2   # N % 128
-    assert call("fp8q_linear_fwd", A, B, 16, C, D, 16, 256, 100, E, 256, NUL) == 2   # K % 128
+    assert call("fp8q_linear_fwd", A, B, 16, C, D, 16, 200, 128, E, 256, NUL) == 2   # N % 16
+    assert call("fp8q_linear_fwd", A, B, 16, C, D, 16, 256, 100, E, 256, NUL) == 2   # K % 16
     assert call("fp8q_linear_fwd", A, B, 8, C, D, 16, 256, 128, E, 256, NUL) == 2    # ldsa < M
     assert call("fp8q_linear_fwd", A, B, 16, C, D, 16, 256, 128, E, 250, NUL) == 2   # ldy < N
     assert call("fp8q_linear_fwd", A, B, 16, C, D, 16, 256, 128, E, 260, NUL) == 3   # ldy % 8
     assert call("fp8q_linear_fwd", A, NUL, 16, C, D, 16, 256, 128, E, 256, NUL) == 1
     assert call("fp8q_linear_dgrad", A, B, 16, C, D, 16, 256, 200, E, 256, NUL) == 2
-    assert call("fp8q_linear_wgrad", A, B, C, D, 100, 256, 256, E, 256, NUL) == 2    # M % 128
+    assert call("fp8q_linear_wgrad", A, B, C, D, 100, 256, 256, E, 256, NUL) == 2    # M % 16
     assert call("fp8q_linear_wgrad", A, B, C, D, 128, 256, 256, ODD, 256, NUL) == 3
 
 
@@ -149,8 +149,9 @@ def test_validation_backward_producers():
     assert call(f, A, B, 128, 128, ctypes.c_void_p(0x10008), C, D, 128, E, A, NUL) == 3
     g = "fp8q_rmsnorm_bwd_quant_dual"
     need = call("fp8q_rmsnorm_bwd_workspace_bytes", 256, 512)
-    assert need == 2048 + 2 * 512 * 8                                              # r, k, partials
+    assert need == 2048 + 512 * 16 * 8                                  # r, k, dgamma's bins
     assert call("fp8q_rmsnorm_bwd_workspace_bytes", 100, 512) == -1
+    assert call("fp8q_rmsnorm_bwd_workspace_bytes", (1 << 23) + 128, 512) == -1   # M too large
     ok = (A, B, C, NUL, 256, 512, F(1e-5), D, E, A, 256, B, C, NUL, W)
     assert call(g, *ok, need - 1, NUL) == 2                                        # workspace
     assert call(g, A, B, C, NUL, 256, 512, F(-1.0), D, E, A, 256, B, C, NUL, W, need, NUL) == 2
@@ -162,8 +163,8 @@ def test_validation_backward_producers():
 
 def test_validation_wgrad_acc_f32():
     f = "fp8q_linear_wgrad_acc_f32"
-    assert call(f, A, B, C, D, 100, 128, 128, E, 128, NUL) == 2       # M % 128
-    assert call(f, A, B, C, D, 128, 128, 100, E, 128, NUL) == 2       # K % 128
+    assert call(f, A, B, C, D, 100, 128, 128, E, 128, NUL) == 2       # M % 16
+    assert call(f, A, B, C, D, 128, 128, 100, E, 128, NUL) == 2       # K % 16
     assert call(f, A, B, C, D, 128, 128, 128, E, 126, NUL) == 2       # lddw < K
     assert call(f, A, B, C, D, 128, 128, 256, E, 258, NUL) == 3       # lddw % 4
     assert call(f, A, B, C, NUL, 128, 128, 128, E, 128, NUL) == 1

@@ -1,9 +1,8 @@
 """Backward producers with the gradient quantizer fused behind them, against the oracle
-through the C ABI: the SwiGLU backward bit for bit (gradient,
-codes, scales); the RMSNorm backward's BF16 gradient within one BF16 ulp (its fp64 sums
-are blocked on the GPU, sequential in the oracle), its codes and scales bit for bit
-against the oracle's quantization of the kernel's own gradient, dgamma within fp32
-rounding of the fp64 sum; the full-size Llama-3.1-8B shapes on sampled 128-row blocks."""
+through the C ABI, bit for bit: the SwiGLU backward (gradient, codes, scales) and the
+RMSNorm backward (BF16 gradient, its codes and scales both ways, dgamma: the reductions
+are exact sums rounded once on both sides); the full-size Llama-3.1-8B shapes on sampled
+128-row blocks and dgamma over all rows."""
 import numpy as np
 import pytest
 import torch
@@ -21,16 +20,6 @@ def fq():
         pytest.skip("needs a CUDA device")
     import fp8_block_scaled_08_b200 as f
     return f
-
-
-def _f(b: np.ndarray) -> np.ndarray:
-    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-
-
-def _ulp_bf16(v: np.ndarray) -> np.ndarray:
-    a = np.abs(v)
-    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
-    return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
 
 
 def _swiglu_inputs(M, I, seed):
@@ -87,26 +76,26 @@ def _rms_inputs(M, H, seed, with_res):
 
 
 def _check_rms(fq, oracle_mod, x, g, dy, dres, eps, out, q, s, qT, sT, dg, what):
+    """Bit for bit against the oracle chain: the BF16 gradient, its codes and scales both
+    ways (the oracle quantizing its own gradient), and dgamma (exact sums on both sides)."""
     M, H = x.shape
-    rout, rdg, rr, rk = oracle_mod.rmsnorm_bwd(bits(x), bits(g), bits(dy),
-                                               None if dres is None else bits(dres), eps)
-    got, ref = _f(bits(out)), _f(rout)
-    err = np.abs(got - ref)
-    assert np.all(err <= _ulp_bf16(ref)), "%s: out beyond one BF16 ulp at %s" % (
-        what, np.argwhere(err > _ulp_bf16(ref))[:4].tolist())
-    assert np.mean(err == 0) >= 0.999, "%s: %.5f of out exact" % (what, np.mean(err == 0))
-    # the codes are the quantization of the kernel's own BF16 gradient
-    oq, os_, oqT, osT = oracle_mod.transpose_quant_bf16(bits(out))
-    assert_codes_equal(q, oq, what + " rows")
-    assert_scales_equal(s, os_, what + " row scales", cols=M)
-    assert_codes_equal(qT, oqT, what + " columns")
-    assert_scales_equal(sT, osT, what + " column scales")
-    # dgamma: fp64 sums of the same fp32 terms, in another order
-    xr = _f(bits(x)) * rr.astype(np.float64)[:, None]
-    scale = np.abs(_f(bits(dy)) * xr).sum(axis=0)
-    d = np.abs(np_f32(dg).astype(np.float64) - rdg.astype(np.float64))
-    spacing = np.spacing(np.abs(rdg)).astype(np.float64)
-    assert np.all(d <= spacing + 1e-12 * scale), what + " dgamma"
+    rout, rq, rs, rqT, rsT, rdg = oracle_mod.rmsnorm_bwd_dual(
+        bits(x), bits(g), bits(dy), None if dres is None else bits(dres), eps)
+    got = bits(out)
+    if not np.array_equal(got, rout):
+        bad = np.argwhere(got != rout)
+        i = tuple(bad[0])
+        raise AssertionError("%s: %d gradient mismatches, first at %s: gpu %#x oracle %#x" % (
+            what, len(bad), i, got[i], rout[i]))
+    assert_codes_equal(q, rq, what + " rows")
+    assert_scales_equal(s, rs, what + " row scales", cols=M)
+    assert_codes_equal(qT, rqT, what + " columns")
+    assert_scales_equal(sT, rsT, what + " column scales")
+    gd = np_f32(dg)
+    if not np.array_equal(gd.view(np.uint32), rdg.view(np.uint32)):
+        bad = np.flatnonzero(gd.view(np.uint32) != rdg.view(np.uint32))
+        raise AssertionError("%s: %d dgamma mismatches, first at %d: gpu %r oracle %r" % (
+            what, len(bad), bad[0], gd[bad[0]], rdg[bad[0]]))
 
 
 @pytest.mark.parametrize("M,H,eps,with_res", [(128, 128, 1e-5, True), (256, 512, 1e-5, False),
@@ -121,7 +110,7 @@ def test_rmsnorm_bwd_dual_matches_oracle(fq, oracle_mod, M, H, eps, with_res):
 
 
 def test_rmsnorm_bwd_dual_repeatable_and_workspace_reuse(fq):
-    """Two calls on one workspace give bit-identical results (fixed reduction order)."""
+    """Two calls on one workspace give bit-identical results (exact reductions)."""
     M, H = 256, 1024
     x, g, dy, dres = _rms_inputs(M, H, 3300, True)
     a = fq.rmsnorm_bwd_quant_dual_alloc(x, g, dy, dres, 1e-5)
@@ -168,17 +157,15 @@ def test_full_size_llama_backward_producers_sampled(fq, oracle_mod):
     torch.cuda.synchronize()
     mb = int(rng.integers(0, M // 128))
     blk = slice(mb * 128, mb * 128 + 128)
-    rout, _, _, _ = oracle_mod.rmsnorm_bwd(bits(x[blk]), bits(g), bits(dy[blk]), bits(dres[blk]),
-                                           wl.eps)
-    err = np.abs(_f(bits(out[blk])) - _f(rout))
-    assert np.all(err <= _ulp_bf16(_f(rout)))
-    oq, _, oqT, osT = oracle_mod.transpose_quant_bf16(bits(out[blk]))
+    rout, oq, _, oqT, osT, _ = oracle_mod.rmsnorm_bwd_dual(
+        bits(x[blk]), bits(g), bits(dy[blk]), bits(dres[blk]), wl.eps)
+    assert np.array_equal(bits(out[blk]), rout)
     assert_codes_equal(q[blk], oq, "full rmsnorm bwd rows")
     assert_codes_equal(qT[:, blk], oqT, "full rmsnorm bwd columns")
     assert np.array_equal(np_f32(sT[mb:mb + 1]).view(np.uint32), osT.view(np.uint32))
+    # dgamma sums over all 8192 rows: the oracle's exact sums, bit for bit
     _, rdg, _, _ = oracle_mod.rmsnorm_bwd(bits(x), bits(g), bits(dy), None, wl.eps)
-    d = np.abs(np_f32(dg).astype(np.float64) - rdg.astype(np.float64))
-    assert np.all(d <= 2 * np.spacing(np.abs(rdg)).astype(np.float64) + 1e-12)
+    assert np.array_equal(np_f32(dg).view(np.uint32), rdg.view(np.uint32))
 
 
 def test_rmsnorm_bwd_degenerate_rows(fq, oracle_mod):

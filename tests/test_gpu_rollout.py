@@ -1,10 +1,12 @@
-"""The rollout weight refresh on one GPU: the packed views hold exactly what separate
-calls of the weight quantizer produce, and the forward GEMM reading them gives the same
+"""The rollout weight refresh on one GPU: the packed views hold exactly the oracle's
+128x128 quantization of each BF16 master (codes and scales bit for bit), the same as
+separate calls of the weight quantizer, and the forward GEMM reading them gives the same
 output bit for bit."""
 import pytest
 import torch
 
 import workloads
+from gpu_util import assert_codes_equal, assert_scales_equal, bits
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -18,7 +20,7 @@ def fq():
     return f
 
 
-def test_refresh_views_equal_separate_quantization(fq):
+def test_refresh_views_equal_separate_quantization(fq, oracle_mod):
     from fp8_block_scaled_08_b200.rollout import PackedFp8Weights, refresh
     L = workloads.LLAMA31_8B
     shapes = {lin.name: (lin.n, lin.k) for lin in L.linears}
@@ -32,6 +34,10 @@ def test_refresh_views_equal_separate_quantization(fq):
                                    outlier_scale=50.0)
     qx, sx = fq.quant_act_1x128_alloc(x)
     for name, w in masters.items():
+        # the oracle's quantization of the master, in full
+        rq, rs, _ = oracle_mod.quant_weight_128x128(bits(w), want_t=False)
+        assert_codes_equal(views[name][0], rq, "packed codes " + name)
+        assert_scales_equal(views[name][1], rs, "packed scales " + name)
         q, s, _ = fq.quant_weight_alloc(w, want_t=False)
         torch.cuda.synchronize()
         assert torch.equal(views[name][0], q), name
