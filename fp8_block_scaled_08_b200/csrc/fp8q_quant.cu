@@ -859,6 +859,7 @@ struct SwigluBwd {
   int64_t I;
   static constexpr int kOut = 2;
   static constexpr bool kHeavy = true;  // long form: keep the row-batch loop rolled
+  static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
   struct In { uint4 g, u, d; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1131,6 +1132,7 @@ struct RmsBwd {
   int64_t H;
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = false;
+  static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
   struct In { uint4 x, d, res; };
   struct Col { float g[8]; };
   __device__ __forceinline__ Col column(int64_t c) const {
@@ -1177,6 +1179,7 @@ struct GradDirect {
   int64_t ld;
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = false;
+  static constexpr bool kTails = true;  // ragged M / N accepted by its entry point
   struct In { uint4 a; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1197,6 +1200,7 @@ struct RmsDirect {
   const uint16_t* gamma;
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = false;
+  static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
   struct In { uint4 a; };
   struct Col { float g[8]; };
   __device__ __forceinline__ Col column(int64_t c) const {
@@ -1229,6 +1233,7 @@ struct SwigluDirect {
   int64_t ldgu, I;
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = true;
+  static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
   struct In { uint4 g, u; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1261,6 +1266,83 @@ constexpr size_t direct_smem_bytes() {
   return X::kOut * (kTileElems * 2 + 4 * 128 * 4);
 }
 
+// One 128 x 128 unit of direct_dual_kernel (described there). kEdge: the unit may reach
+// past a ragged M or N; loads past them read zeros and nothing past them is stored.
+template <class X, int kBatch, bool kEdge>
+__device__ __forceinline__ void dual_unit(const X& xf, int64_t mb, int64_t nb, int64_t M, int64_t N,
+                                          uint16_t* __restrict__ bf16_out,
+                                          uint8_t* __restrict__ q_row, float* __restrict__ s_row,
+                                          int64_t lds_row, uint8_t* __restrict__ q_colT,
+                                          float* __restrict__ s_col, uint16_t* tile, float* red) {
+  constexpr int kOut = X::kOut;
+  const int64_t Nout = kOut * N;
+  const int tid = threadIdx.x;
+  const int rr = tid >> 4, c8 = (tid & 15) * 8;
+  const GroupScale unused{1.0f, 1.0f, -1.0f, false};
+  {
+    const int64_t col = nb * 128 + c8;
+    const bool col_ok = !kEdge || col < N;  // N is a multiple of 8: a chunk is in or out
+    const typename X::Col cs = xf.column(col_ok ? col : 0);
+    // unrolled for short forms; a long form (the SwiGLU exponential and divisions) stays
+    // rolled, which keeps the kernel inside the instruction cache (measured faster)
+    constexpr int kOuterUnroll = X::kHeavy ? 1 : 8 / kBatch;
+#pragma unroll kOuterUnroll
+    for (int h = 0; h < 8 / kBatch; ++h) {
+      typename X::In in[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int64_t m = mb * 128 + rr + 16 * (h * kBatch + j);
+        if (!kEdge || (m < M && col_ok)) in[j] = xf.load(m, col);
+        else in[j] = typename X::In{};
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int r = rr + 16 * (h * kBatch + j);
+        const int64_t m = mb * 128 + r;
+        const bool ok = !kEdge || (m < M && col_ok);
+        float v[kOut][8];
+        xf.form(in[j], ok ? m : 0, cs, v);
+#pragma unroll
+        for (int o = 0; o < kOut; ++o) {
+          const int64_t oc = o * N + nb * 128 + c8;  // output column of this chunk
+          const uint4 pk = make_uint4(pack_bf16x2(v[o][0], v[o][1]), pack_bf16x2(v[o][2], v[o][3]),
+                                      pack_bf16x2(v[o][4], v[o][5]), pack_bf16x2(v[o][6], v[o][7]));
+          *reinterpret_cast<uint4*>(tile + o * kTileElems + r * 128 + c8) = pk;
+          if (bf16_out && ok) *reinterpret_cast<uint4*>(bf16_out + m * Nout + oc) = pk;
+          if (q_row) {
+            uint2 codes;
+            const float sc = quant_half_warp(v[o], codes);  // every lane takes part
+            if (ok) *reinterpret_cast<uint2*>(q_row + m * Nout + oc) = codes;
+            if ((tid & 15) == 0 && (!kEdge || m < M)) s_row[((o * N) / 128 + nb) * lds_row + m] = sc;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // Each column pass reads its tile into registers before its own barrier, so once
+    // every thread is past the last one the tiles may be overwritten by the next unit.
+    const int rows = kEdge && M - mb * 128 < 128 ? static_cast<int>(M - mb * 128) : 128;
+    const int cols = kEdge && N - nb * 128 < 128 ? static_cast<int>(N - nb * 128) : 128;
+#pragma unroll
+    for (int o = 0; o < kOut; ++o) {
+      const int64_t oc0 = o * N + nb * 128;
+      tile_cols_bf16<256>(tile + o * kTileElems, red + o * 4 * 128, true, unused,
+                          q_colT + oc0 * M + mb * 128, M, s_col + mb * Nout + oc0, rows, cols);
+    }
+  }
+}
+
+// The checked unit out of line, so that the rare edge path does not take registers from
+// the common one.
+template <class X, int kBatch>
+__device__ __noinline__ void dual_unit_edge(const X& xf, int64_t mb, int64_t nb, int64_t M,
+                                            int64_t N, uint16_t* bf16_out, uint8_t* q_row,
+                                            float* s_row, int64_t lds_row, uint8_t* q_colT,
+                                            float* s_col, uint16_t* tile, float* red) {
+  dual_unit<X, kBatch, true>(xf, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT, s_col,
+                             tile, red);
+}
+
 // Persistent over the ceil(M/128) x NB units (NB = ceil(N/128)); unit t covers rows
 // (t / NB) * 128 and input columns (t % NB) * 128. Each thread loads its chunks (rows
 // rr + 16 j, columns c8..c8+7) straight into registers, kBatch rows at a time, forms the
@@ -1280,62 +1362,17 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   uint16_t* tile = reinterpret_cast<uint16_t*>(smem_raw);
   float* red = reinterpret_cast<float*>(smem_raw + kOut * kTileElems * 2);
   const int64_t NB = (N + 127) >> 7;
-  const int64_t Nout = kOut * N;
   const int64_t tiles = ((M + 127) >> 7) * NB;
-  const int tid = threadIdx.x;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  const GroupScale unused{1.0f, 1.0f, -1.0f, false};
   for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
     const int64_t mb = t / NB, nb = t % NB;
-    const int64_t col = nb * 128 + c8;
-    const bool col_ok = col < N;  // N is a multiple of 8: a chunk is in or out
-    const typename X::Col cs = xf.column(col_ok ? col : 0);
-    // unrolled for short forms; a long form (the SwiGLU exponential and divisions) stays
-    // rolled, which keeps the kernel inside the instruction cache (measured faster)
-    constexpr int kOuterUnroll = X::kHeavy ? 1 : 8 / kBatch;
-#pragma unroll kOuterUnroll
-    for (int h = 0; h < 8 / kBatch; ++h) {
-      typename X::In in[kBatch];
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int64_t m = mb * 128 + rr + 16 * (h * kBatch + j);
-        if (m < M && col_ok) in[j] = xf.load(m, col);
-        else in[j] = typename X::In{};
-      }
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int r = rr + 16 * (h * kBatch + j);
-        const int64_t m = mb * 128 + r;
-        const bool ok = m < M && col_ok;
-        float v[kOut][8];
-        xf.form(in[j], ok ? m : 0, cs, v);
-#pragma unroll
-        for (int o = 0; o < kOut; ++o) {
-          const int64_t oc = o * N + nb * 128 + c8;  // output column of this chunk
-          const uint4 pk = make_uint4(pack_bf16x2(v[o][0], v[o][1]), pack_bf16x2(v[o][2], v[o][3]),
-                                      pack_bf16x2(v[o][4], v[o][5]), pack_bf16x2(v[o][6], v[o][7]));
-          *reinterpret_cast<uint4*>(tile + o * kTileElems + r * 128 + c8) = pk;
-          if (bf16_out && ok) *reinterpret_cast<uint4*>(bf16_out + m * Nout + oc) = pk;
-          if (q_row) {
-            uint2 codes;
-            const float sc = quant_half_warp(v[o], codes);  // every lane takes part
-            if (ok) *reinterpret_cast<uint2*>(q_row + m * Nout + oc) = codes;
-            if ((tid & 15) == 0 && m < M) s_row[((o * N) / 128 + nb) * lds_row + m] = sc;
-          }
-        }
-      }
-    }
-    __syncthreads();
-    // Each column pass reads its tile into registers before its own barrier, so once
-    // every thread is past the last one the tiles may be overwritten by the next unit.
-    const int rows = M - mb * 128 < 128 ? static_cast<int>(M - mb * 128) : 128;
-    const int cols = N - nb * 128 < 128 ? static_cast<int>(N - nb * 128) : 128;
-#pragma unroll
-    for (int o = 0; o < kOut; ++o) {
-      const int64_t oc0 = o * N + nb * 128;
-      tile_cols_bf16<256>(tile + o * kTileElems, red + o * 4 * 128, true, unused,
-                          q_colT + oc0 * M + mb * 128, M, s_col + mb * Nout + oc0, rows, cols);
-    }
+    // a unit past the end of a ragged M or N (only sources that accept one) takes the
+    // checked path; whole units take the unchecked one
+    if (X::kTails && (mb * 128 + 128 > M || nb * 128 + 128 > N))
+      dual_unit_edge<X, kBatch>(xf, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT, s_col,
+                                tile, red);
+    else
+      dual_unit<X, kBatch, false>(xf, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT,
+                                  s_col, tile, red);
   }
 }
 
@@ -1398,7 +1435,8 @@ __global__ void __launch_bounds__(256) dgamma_round_kernel(const unsigned long l
 // a8: saved FP8 activation tiles (1x128 groups) -> xhat = fl32(s * dec(q)) -> 128x1
 // groups along M, stored transposed; persistent over the (M/128) x (K/128) tiles.
 // Each buffer holds the 16 KB code tile and its 128 row scales. xhat is an arbitrary
-// fp32 value here, so the quotients use IEEE division.
+// fp32 value here (not a BF16 one), so the quotients are the IEEE quotient itself, formed
+// through an fp64 reciprocal (exact, see the column loop).
 __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS, int64_t M,
     int64_t K, uint8_t* __restrict__ qT, float* __restrict__ sT, unsigned* err,
@@ -1459,13 +1497,21 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
     const bool col_ok = kb * 128 + 2 * cp < K;  // K is even: the pair is in or out
     if (rq == 0 && col_ok)
       *reinterpret_cast<float2*>(sT + mb * K + kb * 128 + 2 * cp) = make_float2(s0, s1);
+    // fl32(x / s) as fl32(x * fl64(1 / s)), the product in fp64: the IEEE quotient for
+    // every finite fp32 x and s (an exact quotient of fp32 values stays ~2^-49 away from
+    // any fp32 rounding midpoint, the fp64 product within ~2^-52 of it)
+    const double r0 = __ddiv_rn(1.0, static_cast<double>(s0));
+    const double r1 = __ddiv_rn(1.0, static_cast<double>(s1));
+    auto qd = [](float x, double r) {
+      return __double2float_rn(__dmul_rn(static_cast<double>(x), r));
+    };
     uint32_t o0[8], o1[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      o0[k] = cvt_e4m3x4(__fdiv_rn(x0[4 * k], s0), __fdiv_rn(x0[4 * k + 1], s0),
-                         __fdiv_rn(x0[4 * k + 2], s0), __fdiv_rn(x0[4 * k + 3], s0));
-      o1[k] = cvt_e4m3x4(__fdiv_rn(x1[4 * k], s1), __fdiv_rn(x1[4 * k + 1], s1),
-                         __fdiv_rn(x1[4 * k + 2], s1), __fdiv_rn(x1[4 * k + 3], s1));
+      o0[k] = cvt_e4m3x4(qd(x0[4 * k], r0), qd(x0[4 * k + 1], r0), qd(x0[4 * k + 2], r0),
+                         qd(x0[4 * k + 3], r0));
+      o1[k] = cvt_e4m3x4(qd(x1[4 * k], r1), qd(x1[4 * k + 1], r1), qd(x1[4 * k + 2], r1),
+                         qd(x1[4 * k + 3], r1));
     }
     uint8_t* dst = qT + (kb * 128) * M + mb * 128;
     uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * M + 32 * rq);
