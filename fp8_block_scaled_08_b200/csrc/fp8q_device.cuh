@@ -100,6 +100,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
                                                const WaitCtl& ctl) {
   const uint32_t a = smem_u32(bar);
+  // first try before reading the clock (the common case in the GEMM's promotion)
+  if (__all_sync(0xFFFFFFFFu, mbar_try_wait(a, parity))) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
     const bool done = mbar_try_wait(a, parity);

@@ -28,13 +28,16 @@
 // KB with single-CTA 128x256 tiles, which keeps shared-memory bandwidth below the
 // tensor core's demand. 384 threads per CTA:
 //   warp 0      TMA producer: its A/B halves into a 4-stage ring (128-byte swizzle),
-//               completing on the leader's barrier; its scale vectors into an 8-slot
-//               ring.
+//               completing on the leader's barrier; the row scales (and WGrad's column
+//               scales) into a small ring of slots, 8 slices per slot for the
+//               block-scaled kernels, so their promotion waits for scales once per 8
+//               slices (a barrier wait costs ~100-200 cycles even when it is already
+//               complete: measured).
 //   warp 1      allocates 512 TMEM columns (both CTAs); in the leader, one thread
 //               issues the pair MMAs into TMEM buffer r%2 and commits to barriers in
-//               both CTAs that free the smem stage / publish the slice. With the N
-//               split (forward, DGrad: each slice as two N = 128 halves) one thread of
-//               warp 2 issues every other slice, so two threads share the issuing.
+//               both CTAs that free the smem stage / publish the slice. For the
+//               block-scaled B (forward, DGrad) one thread of warp 2 issues every other
+//               slice, so two threads share the issuing.
 //   warps 2, 3  otherwise idle. Warpgroup 0 (warps 0-3) hands registers to the others.
 //   warps 4..11 two warpgroups; warpgroup h promotes columns 128h..128h+127 of this
 //               CTA's 128 x 256 part: tcgen05.ld, packed fp32 FMA into 128 registers
@@ -44,7 +47,8 @@
 //               fp32-accumulate WGrad stages fp32 boxes and adds them into its output
 //               with TMA reduce-add instead).
 // Registers: the block launches with 168 per thread (168 x 384 = 64512); warpgroup
-// 0 drops to 40 and the promotion warpgroups rise to 232 (40*128 + 232*256 = 64512).
+// 0 drops to 56 and the promotion warpgroups rise to 224 (56*128 + 224*256 = 64512),
+// 40 and 232 for the column-scaled WGrad.
 // Every mbarrier wait is bounded (kWaitLimitNs): a wait that gives up records
 // FP8Q_ERR_TIMEOUT in the device error word and both CTAs wind down.
 #include <algorithm>
@@ -62,37 +66,62 @@ constexpr int BN = 256;        // columns of the tile (each CTA loads 128 rows o
 constexpr int BK = 128;        // one scale slice
 constexpr int kPairM = 2 * BM;
 constexpr int kStages = 4;
-constexpr int kScStages = 8;
+// Scales: the row scales (and the column-scaled WGrad's column scales) of sc_batch
+// consecutive slices arrive together in one of sc_slots slots. The block-scaled kernels
+// take 8 slices per barrier wait (measured 13-19 % faster than one); the WGrad measured
+// ~7 % slower that way than with one slice per slot and 8 slots.
+template <bool kCol>
+__host__ __device__ constexpr int sc_batch() { return kCol ? 1 : 8; }
+template <bool kCol>
+__host__ __device__ constexpr int sc_slots() { return kCol ? 8 : 2; }
+constexpr int kScSlotsMax = 8;
 constexpr int kThreads = 384;
-// Leader threads issuing MMAs (alternate slices, warps 1 and 2) when each slice is 8 MMAs
-// (N split in two halves); one for 4 MMAs a slice, where a second issuer measured slower.
-template <bool kSplitN>
-__host__ __device__ constexpr int issuers() { return kSplitN ? 2 : 1; }
+// Leader threads issuing MMAs, taking alternate slices (warps 1 and 2): one thread needs
+// about 90 cycles per MMA plus ~100-200 per barrier wait (measured), close to the 512
+// cycles of tensor work per slice. The column-scaled WGrad measured ~2 % slower with two.
+template <bool kColScaleB>
+__host__ __device__ constexpr int issuers() { return kColScaleB ? 1 : 2; }
 static_assert(kStages % 2 == 0, "each ring stage is always used by the same issuer");
 constexpr uint32_t kRegsLaunch = 168;   // what ptxas allots under __launch_bounds__(384, 1)
-constexpr uint32_t kRegsControl = 40;   // warpgroup 0 after the hand-over
-constexpr uint32_t kRegsPromote = 232;  // warpgroups 1 and 2 after the hand-over
-static_assert(kRegsControl * 128 + kRegsPromote * 256 <= kRegsLaunch * kThreads,
+// Warpgroup 0 after the hand-over: with two MMA issuers 40 registers made the compiler
+// spill in the issue loop, so the block-scaled kernels give it 56.
+template <bool kCol>
+__host__ __device__ constexpr uint32_t regs_control() { return kCol ? 40 : 56; }
+// Warpgroups 1 and 2 after the hand-over.
+template <bool kCol>
+__host__ __device__ constexpr uint32_t regs_promote() { return kCol ? 232 : 224; }
+static_assert(regs_control<true>() * 128 + regs_promote<true>() * 256 <= kRegsLaunch * kThreads &&
+                  regs_control<false>() * 128 + regs_promote<false>() * 256 <= kRegsLaunch * kThreads,
               "register hand-over exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;  // two 128x256 fp32 accumulators
 constexpr uint32_t kABytes = BM * BK;
 constexpr uint32_t kBBytes = (BN / 2) * BK;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;  // per CTA
-constexpr uint32_t kScABytes = BM * 4;
-constexpr uint32_t kScBBytes = BN * 4;
-constexpr uint32_t kScSlot = kScABytes + kScBBytes;
+template <bool kCol>  // [sc_batch][BM] row scales
+__host__ __device__ constexpr uint32_t sc_a_bytes() { return BM * 4 * sc_batch<kCol>(); }
+template <bool kCol>  // [sc_batch][BN] column scales (WGrad)
+__host__ __device__ constexpr uint32_t sc_b_bytes() { return kCol ? BN * 4 * sc_batch<kCol>() : 0; }
+constexpr uint32_t kScRegion = 24576;  // scale slots of either variant
+static_assert(sc_slots<true>() * (sc_a_bytes<true>() + sc_b_bytes<true>()) <= kScRegion &&
+                  sc_slots<false>() * (sc_a_bytes<false>() + sc_b_bytes<false>()) <= kScRegion &&
+                  sc_slots<true>() <= kScSlotsMax && sc_slots<false>() <= kScSlotsMax,
+              "scale slots exceed their region");
 constexpr uint32_t kStageOutBytes = 32 * 64 * 2;  // one 32-row x 64-column BF16 box
 
 __host__ __device__ constexpr uint32_t kOffA(int s) { return s * kStageBytes; }
 __host__ __device__ constexpr uint32_t kOffB(int s) { return s * kStageBytes + kABytes; }
-__host__ __device__ constexpr uint32_t kOffScA(int i) { return kStages * kStageBytes + i * kScSlot; }
-__host__ __device__ constexpr uint32_t kOffScB(int i) { return kOffScA(i) + kScABytes; }
-constexpr uint32_t kOffOut = kStages * kStageBytes + kScStages * kScSlot;  // 8 warps x 2 boxes
+template <bool kCol>
+__host__ __device__ constexpr uint32_t off_sc_a(int i) {
+  return kStages * kStageBytes + i * (sc_a_bytes<kCol>() + sc_b_bytes<kCol>());
+}
+template <bool kCol>
+__host__ __device__ constexpr uint32_t off_sc_b(int i) { return off_sc_a<kCol>(i) + sc_a_bytes<kCol>(); }
+constexpr uint32_t kOffOut = kStages * kStageBytes + kScRegion;  // 8 warps x 2 boxes
 __host__ __device__ constexpr uint32_t kOffOutBox(int w, int j) {
   return kOffOut + (2 * w + j) * kStageOutBytes;
 }
 constexpr uint32_t kOffBars = kOffOut + 16 * kStageOutBytes;
-constexpr uint32_t kNumBars = 2 * kStages + 8 + 2 * kScStages + 1;
+constexpr uint32_t kNumBars = 2 * kStages + 4 + 2 * kScSlotsMax + 1;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
@@ -132,7 +161,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 
 // kAccF32: instead of storing BF16, add the fp32 accumulator into an fp32 output
 // (out += A x B^T) by TMA reduce-add of 32 x 32 boxes.
-template <bool kColScaleB, bool kSplitN, bool kAccF32 = false>
+template <bool kColScaleB, bool kAccF32 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -143,11 +172,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint64_t* full = bars;              // leader: both CTAs' A/B bytes of a stage
   uint64_t* empty = full + kStages;   // both: stage consumed by the pair MMAs
-  uint64_t* tfull = empty + kStages;  // both: half-slice accumulator [buf*2 + half] ready
-  uint64_t* tempty = tfull + 4;       // leader: both CTAs' warpgroup `half` done with it
-  uint64_t* sfull = tempty + 4;       // local scale ring
-  uint64_t* sempty = sfull + kScStages;
-  uint64_t* done = sempty + kScStages;
+  uint64_t* tfull = empty + kStages;  // both: slice accumulator in TMEM buffer b ready
+  uint64_t* tempty = tfull + 2;       // leader: both CTAs' promotion done with buffer b
+  uint64_t* sfull = tempty + 2;       // local scale batches
+  uint64_t* sempty = sfull + kScSlotsMax;
+  uint64_t* done = sempty + kScSlotsMax;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -162,20 +191,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    // Split slices: one barrier per half-buffer, released by every thread of one
-    // promotion warpgroup in each CTA. Whole slices: one barrier per buffer (index
-    // buf*2), released by every thread of both promotion warpgroups of each CTA. (Every
-    // thread arrives, with no warp-level gather first: measured 5-6 % faster for all
-    // three GEMMs than one arrival per warp after a __syncwarp.)
-    for (int b = 0; b < 4; ++b) {
+    // A TMEM buffer is released by every thread of both promotion warpgroups of each
+    // CTA (every thread arrives, with no warp-level gather first: measured 5-6 % faster
+    // for all three GEMMs than one arrival per warp after a __syncwarp).
+    for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, kSplitN ? 2 * 128 : 2 * 256);
+      mbar_init(tempty + b, 2 * 256);
     }
-    for (int i = 0; i < kScStages; ++i) {
+    for (int i = 0; i < sc_slots<kColScaleB>(); ++i) {
       mbar_init(sfull + i, 1);
       mbar_init(sempty + i, 256);
     }
-    mbar_init(done, issuers<kSplitN>());
+    mbar_init(done, issuers<kColScaleB>());
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -197,7 +224,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp < 4) {
    // Each role's code sits inside the branch of its register budget, so that the
    // compiler allocates it under that budget.
-   regs_decrease<kRegsControl>();
+   regs_decrease<regs_control<kColScaleB>()>();
    if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -218,46 +245,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tma_load_2d_pair(smem + kOffB(stage), &tmB, kb * BK, brow0, leader_full);
           issued |= 1u << stage;
           par = (par & ~(1u << stage)) | (phase << stage);
-          if (!mbar_wait(sempty + sci, scph ^ 1, ctl)) { ok = false; break; }
-          mbar_arrive_expect_tx(sfull + sci, kScABytes + (kColScaleB ? kScBBytes : 0u));
-          tma_load_2d(smem + kOffScA(sci), &tmSA, row0, kb, sfull + sci);
-          if (kColScaleB) tma_load_2d(smem + kOffScB(sci), &tmSB, nb * BN, kb, sfull + sci);
-          sc_issued |= 1u << sci;
-          sc_par = (sc_par & ~(1u << sci)) | (scph << sci);
+          if (kb % sc_batch<kColScaleB>() == 0) {  // the scales of slices kb .. kb + batch - 1
+            if (!mbar_wait(sempty + sci, scph ^ 1, ctl)) { ok = false; break; }
+            mbar_arrive_expect_tx(sfull + sci, sc_a_bytes<kColScaleB>() + sc_b_bytes<kColScaleB>());
+            tma_load_2d(smem + off_sc_a<kColScaleB>(sci), &tmSA, row0, kb, sfull + sci);
+            if (kColScaleB) tma_load_2d(smem + off_sc_b<kColScaleB>(sci), &tmSB, nb * BN, kb, sfull + sci);
+            sc_issued |= 1u << sci;
+            sc_par = (sc_par & ~(1u << sci)) | (scph << sci);
+            if (++sci == sc_slots<kColScaleB>()) { sci = 0; scph ^= 1; }
+          }
           if (++stage == kStages) { stage = 0; phase ^= 1; }
-          if (++sci == kScStages) { sci = 0; scph ^= 1; }
         }
       }
       if (!ok) {  // let every copy already issued land before the CTA exits
         if (rank == 0)
           for (int s = 0; s < kStages; ++s)
             if ((issued >> s) & 1u) mbar_wait_drain(full + s, (par >> s) & 1u, p.wait_limit_ns);
-        for (int i = 0; i < kScStages; ++i)
+        for (int i = 0; i < sc_slots<kColScaleB>(); ++i)
           if ((sc_issued >> i) & 1u) mbar_wait_drain(sfull + i, (sc_par >> i) & 1u, p.wait_limit_ns);
       }
     }
     __syncwarp();
-   } else if (warp <= issuers<kSplitN>()) {
+   } else if (warp <= issuers<kColScaleB>()) {
     // ------------------------------------------------------------ MMA issuers (leader)
     // With two issuers, issuer i = warp - 1 takes the slices that use TMEM buffer i (slice
-    // parity): each slice is an independent group of MMAs into its own buffer, and one
-    // thread needs ~70 cycles to issue each MMA (measured), which for 8 MMAs a slice
-    // approaches the tensor core's own time per slice.
+    // parity); each slice is 4 MMAs of N = 256 into its buffer and one commit.
     if (lane == 0 && rank == 0) {
       const uint32_t issuer = static_cast<uint32_t>(warp - 1);
-      // kSplitN: each slice is issued as two N = 128 halves into separate TMEM
-      // half-buffers with their own barriers, so a promotion warpgroup starts on its half
-      // as soon as that half is done and the MMAs can run half a slice further ahead.
-      // Otherwise one N = 256 group per slice on one barrier per buffer. (Measured in
-      // one process on one B200: the split is ~20 % faster for the long-K DGrad, equal
-      // for the forward, ~5 % slower for the column-scaled WGrad.)
-      const uint32_t idesc = idesc_e4m3_f32(kPairM, kSplitN ? BN / 2 : BN);
+      const uint32_t idesc = idesc_e4m3_f32(kPairM, BN);
       uint32_t stage = 0, phase = 0, it = 0;
       bool ok = true;
       for (int t = pair; ok && t < num_tiles; t += npairs) {
         for (int kb = 0; ok && kb < p.kblocks; ++kb) {
           const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
-          if (issuers<kSplitN>() == 2 && buf != issuer) {  // the other issuer's slice
+          if (issuers<kColScaleB>() == 2 && buf != issuer) {  // the other issuer's slice
             if (++stage == kStages) { stage = 0; phase ^= 1; }
             ++it;
             continue;
@@ -265,31 +286,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!mbar_wait(full + stage, phase, ctl)) { ok = false; break; }
           const uint32_t a0 = smem_u32(smem + kOffA(stage));
           const uint32_t b0 = smem_u32(smem + kOffB(stage));
-          if (kSplitN) {
+          if (!mbar_wait(tempty + buf, tph ^ 1u, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + buf * BN;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!mbar_wait(tempty + buf * 2 + h, tph ^ 1u, ctl)) { ok = false; break; }
-              tc_fence_after();
-              // half h: B rows [64h, 64h + 64) of each CTA's B half (8 swizzle atoms in)
-              const uint32_t bh = b0 + h * (BN / 4) * BK;
-              const uint32_t d = tmem_base + buf * BN + h * (BN / 2);
-#pragma unroll
-              for (int k = 0; k < BK / 32; ++k)
-                mma_f8f6f4_pair(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(bh + 32 * k),
-                                idesc, k > 0 ? 1u : 0u);
-              mma_commit_pair_multicast(tfull + buf * 2 + h, 0x3);
-            }
-          } else {
-            if (!mbar_wait(tempty + buf * 2, tph ^ 1u, ctl)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t d = tmem_base + buf * BN;
-#pragma unroll
-            for (int k = 0; k < BK / 32; ++k)
-              mma_f8f6f4_pair(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k),
-                              idesc, k > 0 ? 1u : 0u);
-            mma_commit_pair_multicast(tfull + buf * 2, 0x3);
-          }
-          if (!ok) break;
+          for (int k = 0; k < BK / 32; ++k)
+            mma_f8f6f4_pair(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k),
+                            idesc, k > 0 ? 1u : 0u);
+          mma_commit_pair_multicast(tfull + buf, 0x3);
           mma_commit_pair_multicast(empty + stage, 0x3);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
           ++it;
@@ -303,13 +307,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
    }
   } else {
-    regs_increase<kRegsPromote>();
+    regs_increase<regs_promote<kColScaleB>()>();
     // ------------------------------------------------------------ promotion + epilogue
-    // Warpgroup `half` owns TMEM columns [128*half, +128) of each slice buffer. A pair
-    // MMA of width N takes its first N/2 columns from the leader's B rows and the next
-    // N/2 from the peer's. With N = 256 the warpgroup's accumulator columns are tile
-    // columns 128*half + [0,128); with the split (two N = 128 halves) its columns [0,64)
-    // are tile columns 64*half + [0,64) and [64,128) are 128 + 64*half + [0,64).
+    // Warpgroup `half` owns TMEM columns [128*half, +128) of each slice buffer, which are
+    // tile columns 128*half + [0,128) (a pair MMA of width 256 takes its first 128
+    // columns from the leader's B rows and the next 128 from the peer's): one 128-wide
+    // block of B, so one block scale per slice when B is block-scaled.
     const int wq = warp & 3;           // TMEM lane quarter this warp may access
     const int half = (warp - 4) >> 2;  // TMEM half-buffer of this warpgroup
     const int row = wq * 32 + lane;
@@ -322,31 +325,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int mb, nb;
       tile_coords(t, p, mb, nb);
       const int row0 = mb * kPairM + static_cast<int>(rank) * BM;
-      const int col_lo = nb * BN + (kSplitN ? 64 : 128) * half;  // tile columns of acc[0..63]
-      const int col_hi = kSplitN ? nb * BN + 128 + 64 * half : col_lo + 64;  // of acc[64..127]
+      const int col_lo = nb * BN + 128 * half;  // tile columns of acc[0..63]
+      const int col_hi = col_lo + 64;           // of acc[64..127]
       // a ragged N (a multiple of 16) ends inside a box: the tensor store clips it
       const bool lo_ok = col_lo < p.N;
       const bool hi_ok = col_hi < p.N;
-      const float* sbp_lo = kColScaleB ? nullptr : p.sb + static_cast<int64_t>(col_lo / 128) * p.sb_sj;
-      const float* sbp_hi = kColScaleB ? nullptr : p.sb + static_cast<int64_t>(col_hi / 128) * p.sb_sj;
+      const float* sbp = kColScaleB ? nullptr : p.sb + static_cast<int64_t>(col_lo / 128) * p.sb_sj;
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-      // block scales of the next slice, loaded one slice ahead
-      float sbn_lo = (!kColScaleB && lo_ok) ? __ldg(sbp_lo) : 0.0f;
-      float sbn_hi = (!kColScaleB && hi_ok) ? __ldg(sbp_hi) : 0.0f;
+      // block scales of B, 32 slices at a time: lane l holds slice 32*(kb/32) + l; the
+      // next 32 are fetched 16 slices ahead (a global load per slice, even prefetched one
+      // slice ahead, measured ~10 % slower)
+      auto sb_fetch = [&](int kk) -> float {
+        return (!kColScaleB && lo_ok && kk < p.kblocks) ? __ldg(sbp + static_cast<int64_t>(kk) * p.sb_sr)
+                                                        : 0.0f;
+      };
+      float sbv = sb_fetch(lane), sbx = 0.0f;
       for (int kb = 0; kb < p.kblocks; ++kb) {
-        const float sb_lo = sbn_lo, sb_hi = sbn_hi;
-        if (!kColScaleB && kb + 1 < p.kblocks) {
-          if (lo_ok) sbn_lo = __ldg(sbp_lo + (kb + 1) * p.sb_sr);
-          if (hi_ok) sbn_hi = __ldg(sbp_hi + (kb + 1) * p.sb_sr);
+        const int j = kb % sc_batch<kColScaleB>();  // slice within its scale batch
+        if (!kColScaleB) {
+          if ((kb & 31) == 16) sbx = sb_fetch(kb + 16 + lane);
+          if ((kb & 31) == 0 && kb > 0) sbv = sbx;
         }
-        if (!mbar_wait_warp(sfull + sci, scph, ctl)) { ok = false; break; }
-        const float sa = reinterpret_cast<const float*>(smem + kOffScA(sci))[row];
-        const float* scb = reinterpret_cast<const float*>(smem + kOffScB(sci));
+        const float sb = kColScaleB ? 0.0f : __shfl_sync(0xFFFFFFFFu, sbv, kb & 31);
+        if (j == 0 && !mbar_wait_warp(sfull + sci, scph, ctl)) { ok = false; break; }
+        const float sa = reinterpret_cast<const float*>(smem + off_sc_a<kColScaleB>(sci))[j * BM + row];
+        const float* scb = reinterpret_cast<const float*>(smem + off_sc_b<kColScaleB>(sci)) + j * BN;
         const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
-        const uint32_t bar_idx = buf * 2 + (kSplitN ? half : 0);
-        if (!mbar_wait_warp(tfull + bar_idx, tph, ctl)) { ok = false; break; }
+        if (!mbar_wait_warp(tfull + buf, tph, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr =
             tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + buf * BN + half * (BN / 2);
@@ -357,7 +364,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
           if (!kColScaleB) {
-            const float s = __fmul_rn(sa, c ? sb_hi : sb_lo);
+            const float s = __fmul_rn(sa, sb);
 #pragma unroll
             for (int i = 0; i < 64; i += 2)
               fma2(acc[c * 64 + i], acc[c * 64 + i + 1], __uint_as_float(r[i]),
@@ -377,14 +384,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // hand the TMEM half-buffer and the scale slot back: every thread arrives once its
-        // own TMEM loads are complete and its scale reads consumed
+        // hand the TMEM buffer back: every thread arrives once its own TMEM loads are
+        // complete; the scale batch likewise after its last slice
         tc_fence_before();
-        if (rank == 0) mbar_arrive(tempty + bar_idx);
-        else mbar_arrive_cluster(tempty_leader0 + bar_idx * 8);
-        mbar_arrive(sempty + sci);
+        if (rank == 0) mbar_arrive(tempty + buf);
+        else mbar_arrive_cluster(tempty_leader0 + buf * 8);
+        if (j == sc_batch<kColScaleB>() - 1 || kb == p.kblocks - 1) {
+          mbar_arrive(sempty + sci);
+          if (++sci == sc_slots<kColScaleB>()) { sci = 0; scph ^= 1; }
+        }
         ++it;
-        if (++sci == kScStages) { sci = 0; scph ^= 1; }
       }
       if (!ok) break;
       // epilogue: BF16 rows into this warp's two swizzled 32 x 64 boxes, then TMA stores
@@ -465,7 +474,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // budget of the hand-over, and find how many CTA pairs can be resident at once (pairs
 // are placed within one GPC, so this can be below half the SM count). Returns that
 // number, or 0 on failure (the reason is in fp8q_last_error_message).
-template <bool kCol, bool kSplit, bool kAcc = false>
+template <bool kCol, bool kAcc = false>
 int kernel_setup() {
   // written once per device under the lock; host threads may launch concurrently
   static std::atomic<int> pairs_for_device[64];
@@ -476,7 +485,7 @@ int kernel_setup() {
   std::lock_guard<std::mutex> lock(mu);
   if (const int known = pairs_for_device[dev].load(std::memory_order_relaxed)) return known;
   const cudaError_t e = cudaFuncSetAttribute(
-      gemm_kernel<kCol, kSplit, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      gemm_kernel<kCol, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
       static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) {
     set_last_error("cudaFuncSetAttribute(gemm max dynamic smem)", e);
@@ -486,13 +495,14 @@ int kernel_setup() {
   // The register hand-over inside the kernel waits until the block's launch allocation
   // covers the new budgets; refuse to launch a build whose allocation would not.
   cudaFuncAttributes attr;
-  const cudaError_t ea = cudaFuncGetAttributes(&attr, gemm_kernel<kCol, kSplit, kAcc>);
+  const cudaError_t ea = cudaFuncGetAttributes(&attr, gemm_kernel<kCol, kAcc>);
   if (ea != cudaSuccess) {
     set_last_error("cudaFuncGetAttributes(gemm)", ea);
     cudaGetLastError();
     return 0;
   }
-  if (static_cast<uint32_t>(attr.numRegs) * kThreads < kRegsControl * 128 + kRegsPromote * 256 ||
+  if (static_cast<uint32_t>(attr.numRegs) * kThreads <
+          regs_control<kCol>() * 128 + regs_promote<kCol>() * 256 ||
       attr.maxThreadsPerBlock < kThreads) {
     set_last_error("gemm register budget check", cudaErrorLaunchOutOfResources);
     return 0;
@@ -510,7 +520,7 @@ int kernel_setup() {
   cfg.numAttrs = 1;
   int clusters = 0;
   const cudaError_t eo =
-      cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<kCol, kSplit, kAcc>, &cfg);
+      cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<kCol, kAcc>, &cfg);
   if (eo != cudaSuccess || clusters <= 0) {
     set_last_error("cudaOccupancyMaxActiveClusters(gemm)", eo != cudaSuccess ? eo : cudaErrorInvalidConfiguration);
     cudaGetLastError();
@@ -522,7 +532,7 @@ int kernel_setup() {
 
 // out [Mg][Ng] = A [Mg][Kg] x B [Ng][Kg]^T with the scales described above; out is BF16
 // (y: uint16_t) or, with kAcc, an fp32 array the product is added to (y: float).
-template <bool kCol, bool kSplit, bool kAcc = false>
+template <bool kCol, bool kAcc = false>
 fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t Ng, int64_t Kg,
                         const float* sa, int64_t ldsa, const float* sb, int64_t sb_sj,
                         int64_t sb_sr, const float* sbcol, void* y, int64_t ldy,
@@ -543,14 +553,15 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
                   : encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, Ng, Mg, ldy * 2, 64,
                                    32, CU_TENSOR_MAP_SWIZZLE_128B)) &&
             encode_tmap_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, Mg, kslices, ldsa * 4, BM,
-                           1, CU_TENSOR_MAP_SWIZZLE_NONE);
+                           sc_batch<kCol>(), CU_TENSOR_MAP_SWIZZLE_NONE);
+  // (scale batches past the last slice read the copies' zero fill)
   if (ok && kCol)
-    ok = encode_tmap_2d(&tmSB, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sbcol, Ng, kslices, Ng * 4, BN, 1,
-                        CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = encode_tmap_2d(&tmSB, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sbcol, Ng, kslices, Ng * 4, BN,
+                        sc_batch<kCol>(), CU_TENSOR_MAP_SWIZZLE_NONE);
   else
     tmSB = tmSA;
   if (!ok) return FP8Q_ERR_UNSUPPORTED;
-  const int max_pairs = kernel_setup<kCol, kSplit, kAcc>();
+  const int max_pairs = kernel_setup<kCol, kAcc>();
   if (max_pairs <= 0) return FP8Q_ERR_CUDA;
 
   GemmParams p;
@@ -572,7 +583,7 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   const int64_t tiles = static_cast<int64_t>(p.mblocks) * p.nblocks;
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, max_pairs));
-  gemm_kernel<kCol, kSplit, kAcc><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmSA, tmSB,
+  gemm_kernel<kCol, kAcc><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmSA, tmSB,
                                                                            tmY, p);
   return launch_status("gemm_kernel launch");
 }
@@ -598,7 +609,7 @@ extern "C" fp8q_status fp8q_linear_fwd(const uint8_t* qa, const float* sa, int64
   if (M <= kSkinnyMaxM && K % 128 == 0 && N % 128 == 0)
     return launch_skinny_gemm(qa, qw, M, N, K, sa, ldsa, sw, KB, 1, y, ldy,
                               static_cast<cudaStream_t>(stream));
-  return launch_gemm<false, true>(qa, qw, M, N, K, sa, ldsa, sw, KB, 1, nullptr, y, ldy,
+  return launch_gemm<false>(qa, qw, M, N, K, sa, ldsa, sw, KB, 1, nullptr, y, ldy,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -618,7 +629,7 @@ extern "C" fp8q_status fp8q_linear_dgrad(const uint8_t* qdy, const float* sdy, i
   if (M <= kSkinnyMaxM && K % 128 == 0 && N % 128 == 0)
     return launch_skinny_gemm(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, KB, dx, lddx,
                               static_cast<cudaStream_t>(stream));
-  return launch_gemm<false, true>(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, KB, nullptr, dx, lddx,
+  return launch_gemm<false>(qdy, qwT, M, K, N, sdy, ldsdy, sw, 1, KB, nullptr, dx, lddx,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -635,7 +646,7 @@ extern "C" fp8q_status fp8q_linear_wgrad(const uint8_t* qdyT, const float* sdy_c
   // GEMM rows = N, columns = K, reduction = M (tokens).
   // Row scale of (n, slice r) = sdy_c[r*N + n]  (a [M/128][N] array: ldsa = N)
   // Column scale of (k, slice r) = sx_c[r*K + k]
-  return launch_gemm<true, false>(qdyT, qxT, N, K, M, sdy_c, N, nullptr, 0, 0, sx_c, dw, lddw,
+  return launch_gemm<true>(qdyT, qxT, N, K, M, sdy_c, N, nullptr, 0, 0, sx_c, dw, lddw,
                            static_cast<cudaStream_t>(stream));
 }
 
@@ -650,6 +661,6 @@ extern "C" fp8q_status fp8q_linear_wgrad_acc_f32(const uint8_t* qdyT, const floa
       !aligned16(dw) || lddw % 4)
     return FP8Q_ERR_ALIGN;
   // as fp8q_linear_wgrad, with dw += the fp32 accumulator instead of dw = bf16(it)
-  return launch_gemm<true, false, true>(qdyT, qxT, N, K, M, sdy_c, N, nullptr, 0, 0, sx_c, dw,
+  return launch_gemm<true, true>(qdyT, qxT, N, K, M, sdy_c, N, nullptr, 0, 0, sx_c, dw,
                                         lddw, static_cast<cudaStream_t>(stream));
 }
