@@ -353,6 +353,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float sa = reinterpret_cast<const float*>(smem + off_sc_a<kColScaleB>(sci))[j * BM + row];
         const float* scb = reinterpret_cast<const float*>(smem + off_sc_b<kColScaleB>(sci)) + j * BN;
         const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
+        // the scale reads complete before the wait, not after it on the critical path
+        // (measured ~16 % faster for the column-scaled WGrad)
+        float s_h = kColScaleB ? sa : __fmul_rn(sa, sb);
+        asm volatile("" : "+f"(s_h));
         if (!mbar_wait_warp(tfull + buf, tph, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr =
@@ -360,11 +364,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {  // acc columns [64c, 64c + 64), two loads in flight
           uint32_t r[64];
-          tmem_ld32(taddr + c * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(taddr + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          if (kColScaleB) {  // (the wide load makes the block-scaled kernels spill)
+            tmem_ld64(taddr + c * 64, r);
+          } else {
+            tmem_ld32(taddr + c * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            tmem_ld32(taddr + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          }
           tmem_wait_ld();
+          if (kColScaleB && c == 1) {
+            // column-scaled B: the buffer goes back before the last FMAs (measured ~6 %
+            // faster there, ~7 % slower for the block-scaled kernels)
+            tc_fence_before();
+            if (rank == 0) mbar_arrive(tempty + buf);
+            else mbar_arrive_cluster(tempty_leader0 + buf * 8);
+          }
           if (!kColScaleB) {
-            const float s = __fmul_rn(sa, sb);
+            const float s = s_h;
 #pragma unroll
             for (int i = 0; i < 64; i += 2)
               fma2(acc[c * 64 + i], acc[c * 64 + i + 1], __uint_as_float(r[i]),
@@ -386,9 +401,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         // hand the TMEM buffer back: every thread arrives once its own TMEM loads are
         // complete; the scale batch likewise after its last slice
-        tc_fence_before();
-        if (rank == 0) mbar_arrive(tempty + buf);
-        else mbar_arrive_cluster(tempty_leader0 + buf * 8);
+        if (!kColScaleB) {
+          tc_fence_before();
+          if (rank == 0) mbar_arrive(tempty + buf);
+          else mbar_arrive_cluster(tempty_leader0 + buf * 8);
+        }
         if (j == sc_batch<kColScaleB>() - 1 || kb == p.kblocks - 1) {
           mbar_arrive(sempty + sci);
           if (++sci == sc_slots<kColScaleB>()) { sci = 0; scph ^= 1; }
