@@ -131,7 +131,8 @@ static_assert(kOffOut % 1024 == 0, "TMA store boxes need 1024-byte alignment");
 struct GemmParams {
   int32_t M, N, K;
   int32_t mblocks, nblocks, kblocks;
-  int32_t n_fastest;
+  int32_t group;  // panels per raster group (column panels; row panels with `swap`)
+  int32_t swap;
   const float* sb;  // per-block B scales: sb[(j/128)*sb_sj + r*sb_sr]
   int64_t sb_sj, sb_sr;
   uint16_t* y;
@@ -140,14 +141,27 @@ struct GemmParams {
   uint64_t wait_limit_ns;
 };
 
+// Tile order. Within a group of `group` consecutive column panels (row panels with
+// `swap`) the tiles walk that group fastest and the other dimension's panels slower.
+// The host picks one of two orders from the operand sizes:
+//  - the smaller operand fits in half of L2: one group spans all of its panels, so they
+//    stay in L2 while each panel of the larger operand streams through once;
+//  - otherwise groups of 8 column panels, so that the 74 tiles of one wave of CTA pairs
+//    cover about 9 row panels x 8 column panels (17 distinct operand panels). Every wave
+//    re-reads its panels from DRAM (the K loop restarts), so the distinct panels per wave
+//    set the traffic (measured 17 % less DRAM traffic for the down-projection forward
+//    and 10 % less for the gate/up DGrad than a walk over all 16 column panels).
 __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& mb, int& nb) {
-  if (p.n_fastest) {
-    nb = t % p.nblocks;
-    mb = t / p.nblocks;
-  } else {
-    mb = t % p.mblocks;
-    nb = t / p.mblocks;
-  }
+  const int slow = p.swap ? p.nblocks : p.mblocks;
+  const int fast = p.swap ? p.mblocks : p.nblocks;
+  const int span = p.group * slow;
+  const int g = t / span;
+  const int w = t - g * span;
+  const int width = min(p.group, fast - g * p.group);
+  const int x = g * p.group + w % width;
+  const int y = w / width;
+  mb = p.swap ? x : y;
+  nb = p.swap ? y : x;
 }
 
 // Wait used while winding down after a give-up: ignores the abort flag, still bounded.
@@ -350,52 +364,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         const float sb = kColScaleB ? 0.0f : __shfl_sync(0xFFFFFFFFu, sbv, kb & 31);
         if (j == 0 && !mbar_wait_warp(sfull + sci, scph, ctl)) { ok = false; break; }
-        const float sa = reinterpret_cast<const float*>(smem + off_sc_a<kColScaleB>(sci))[j * BM + row];
+        const float* sa_slot = reinterpret_cast<const float*>(smem + off_sc_a<kColScaleB>(sci)) + j * BM;
         const float* scb = reinterpret_cast<const float*>(smem + off_sc_b<kColScaleB>(sci)) + j * BN;
         const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
-        // the scale reads complete before the wait, not after it on the critical path
-        // (measured ~16 % faster for the column-scaled WGrad)
-        float s_h = kColScaleB ? sa : __fmul_rn(sa, sb);
-        asm volatile("" : "+f"(s_h));
+        // block-scaled B: one scale product per slice; column-scaled B: the row scales of
+        // this thread's four rows (lanes 8e + lane/4 of the warp's quarter, the 16x256b
+        // layout below). Both are read before the wait, not after it on the critical path
+        // (measured ~16 % faster for the column-scaled WGrad).
+        float s_h = kColScaleB ? 0.0f : __fmul_rn(sa_slot[row], sb);
+        float sa4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (kColScaleB) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sa4[e] = sa_slot[wq * 32 + 8 * e + (lane >> 2)];
+        }
+        asm volatile("" : "+f"(s_h), "+f"(sa4[0]), "+f"(sa4[1]), "+f"(sa4[2]), "+f"(sa4[3]));
         if (!mbar_wait_warp(tfull + buf, tph, ctl)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t taddr =
-            tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + buf * BN + half * (BN / 2);
+        if constexpr (!kColScaleB) {
+          const uint32_t taddr =
+              tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + buf * BN + half * (BN / 2);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {  // acc columns [64c, 64c + 64), two loads in flight
-          uint32_t r[64];
-          if (kColScaleB) {  // (the wide load makes the block-scaled kernels spill)
-            tmem_ld64(taddr + c * 64, r);
-          } else {
+          for (int c = 0; c < 2; ++c) {  // acc columns [64c, 64c + 64), two loads in flight
+            uint32_t r[64];
             tmem_ld32(taddr + c * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
             tmem_ld32(taddr + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          }
-          tmem_wait_ld();
-          if (kColScaleB && c == 1) {
-            // column-scaled B: the buffer goes back before the last FMAs (measured ~6 %
-            // faster there, ~7 % slower for the block-scaled kernels)
-            tc_fence_before();
-            if (rank == 0) mbar_arrive(tempty + buf);
-            else mbar_arrive_cluster(tempty_leader0 + buf * 8);
-          }
-          if (!kColScaleB) {
-            const float s = s_h;
+            tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 64; i += 2)
               fma2(acc[c * 64 + i], acc[c * 64 + i + 1], __uint_as_float(r[i]),
-                   __uint_as_float(r[i + 1]), s, s);
-          } else {
-            const float4* scb4 = reinterpret_cast<const float4*>(scb + (c ? col_hi : col_lo) - nb * BN);
+                   __uint_as_float(r[i + 1]), s_h, s_h);
+          }
+        } else {
+          // Column-scaled B: every element needs its own column's scale. With one row per
+          // thread (the 32x32b shape) each thread would hold all 128 column scales of its
+          // columns in registers every slice, and filling them from shared memory took
+          // 70 % of the shared-memory pipe (measured): that bound the kernel. In the
+          // 16x256b shape a thread holds 4 rows x 32 columns, so it needs a quarter of the
+          // column scales. acc[((2b + cc) * 8 + k) * 4 + 2hi + {0,1}] is row
+          // 16b + 8hi + lane/4 of the warp's quarter, columns 64cc + 8k + 2(lane%4) + {0,1}
+          // of the warpgroup's 128.
 #pragma unroll
-            for (int i = 0; i < 64; i += 4) {
-              const float4 sb4 = scb4[i / 4];
-              float s0, s1, s2, s3;
-              mul2(s0, s1, sa, sa, sb4.x, sb4.y);
-              mul2(s2, s3, sa, sa, sb4.z, sb4.w);
-              fma2(acc[c * 64 + i], acc[c * 64 + i + 1], __uint_as_float(r[i]),
-                   __uint_as_float(r[i + 1]), s0, s1);
-              fma2(acc[c * 64 + i + 2], acc[c * 64 + i + 3], __uint_as_float(r[i + 2]),
-                   __uint_as_float(r[i + 3]), s2, s3);
+          for (int cc = 0; cc < 2; ++cc) {
+            float2 sb2[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              sb2[k] = *reinterpret_cast<const float2*>(scb + 128 * half + 64 * cc + 8 * k + 2 * (lane & 3));
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              uint32_t r[32];
+              tmem_ld_16x256b_x8(tmem_base + (static_cast<uint32_t>(wq * 32 + 16 * b) << 16) + buf * BN +
+                                     half * (BN / 2) + 64 * cc,
+                                 r);
+              tmem_wait_ld();
+              if (cc == 1 && b == 1) {
+                // the buffer goes back before the last FMAs (measured ~6 % faster here,
+                // ~7 % slower for the block-scaled kernels)
+                tc_fence_before();
+                if (rank == 0) mbar_arrive(tempty + buf);
+                else mbar_arrive_cluster(tempty_leader0 + buf * 8);
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                float* a = acc + ((2 * b + cc) * 8 + k) * 4;
+                float s0, s1, s2, s3;
+                mul2(s0, s1, sa4[2 * b], sa4[2 * b], sb2[k].x, sb2[k].y);
+                mul2(s2, s3, sa4[2 * b + 1], sa4[2 * b + 1], sb2[k].x, sb2[k].y);
+                fma2(a[0], a[1], __uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]), s0, s1);
+                fma2(a[2], a[3], __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]), s2, s3);
+              }
             }
           }
         }
@@ -419,20 +455,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (wrow0 < p.M && lo_ok) {
         if constexpr (kAccF32) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {  // acc[64 hh + 0..63]: tile columns col_lo / col_hi
+          for (int hh = 0; hh < 2; ++hh) {  // tile columns col_lo (hh = 0) / col_hi, 64 each
             if (stored) {  // the previous boxes must have been read
               if (lane == 0) tma_store_wait_read();
               __syncwarp();
             }
+            if constexpr (kColScaleB) {  // the 16x256b layout (see the promotion)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              uint8_t* box = j ? out1 : out0;
+              for (int b = 0; b < 2; ++b)
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const float* a = acc + hh * 64 + j * 32 + c * 4;
-                *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                    make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
-                               __float_as_uint(a[3]));
+                for (int hi = 0; hi < 2; ++hi)
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) {
+                    const int rr = 16 * b + 8 * hi + (lane >> 2);
+                    const float* a = acc + ((2 * b + hh) * 8 + k) * 4 + 2 * hi;
+                    const int chunk = 2 * (k & 3) + ((lane & 3) >> 1);
+                    uint8_t* box = (k >> 2) ? out1 : out0;
+                    *reinterpret_cast<uint2*>(box + rr * 128 + ((chunk ^ (rr & 7)) << 4) + 8 * (lane & 1)) =
+                        make_uint2(__float_as_uint(a[0]), __float_as_uint(a[1]));
+                  }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                uint8_t* box = j ? out1 : out0;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const float* a = acc + hh * 64 + j * 32 + c * 4;
+                  *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                      make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                                 __float_as_uint(a[3]));
+                }
               }
             }
             fence_proxy_async_smem();
@@ -450,18 +502,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) tma_store_wait_read();
             __syncwarp();
           }
+          if constexpr (kColScaleB) {  // the 16x256b layout (see the promotion)
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            uint8_t* box = j ? out1 : out0;
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float* a = acc + j * 64 + c * 8;
-              uint4 v;
-              v.x = pack_bf16x2(a[0], a[1]);
-              v.y = pack_bf16x2(a[2], a[3]);
-              v.z = pack_bf16x2(a[4], a[5]);
-              v.w = pack_bf16x2(a[6], a[7]);
-              *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
+              for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi)
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) {
+                    const int rr = 16 * b + 8 * hi + (lane >> 2);
+                    const float* a = acc + ((2 * b + cc) * 8 + k) * 4 + 2 * hi;
+                    uint8_t* box = cc ? out1 : out0;
+                    *reinterpret_cast<uint32_t*>(box + rr * 128 + ((k ^ (rr & 7)) << 4) + 4 * (lane & 3)) =
+                        pack_bf16x2(a[0], a[1]);
+                  }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              uint8_t* box = j ? out1 : out0;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const float* a = acc + j * 64 + c * 8;
+                uint4 v;
+                v.x = pack_bf16x2(a[0], a[1]);
+                v.y = pack_bf16x2(a[2], a[3]);
+                v.z = pack_bf16x2(a[4], a[5]);
+                v.w = pack_bf16x2(a[6], a[7]);
+                *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
+              }
             }
           }
           fence_proxy_async_smem();
@@ -588,7 +657,16 @@ fp8q_status launch_gemm(const uint8_t* A, const uint8_t* B, int64_t Mg, int64_t 
   p.mblocks = static_cast<int32_t>((Mg + kPairM - 1) / kPairM);
   p.nblocks = static_cast<int32_t>((Ng + BN - 1) / BN);
   p.kblocks = static_cast<int32_t>(kslices);
-  p.n_fastest = Ng <= Mg ? 1 : 0;
+  {
+    const double a_bytes = static_cast<double>(Mg) * Kg, b_bytes = static_cast<double>(Ng) * Kg;
+    if (std::min(a_bytes, b_bytes) <= 48e6) {  // the smaller operand stays in L2
+      p.swap = b_bytes <= a_bytes ? 0 : 1;
+      p.group = p.swap ? p.mblocks : p.nblocks;
+    } else {
+      p.swap = 0;
+      p.group = std::min<int32_t>(8, p.nblocks);
+    }
+  }
   p.sb = sb;
   p.sb_sj = sb_sj;
   p.sb_sr = sb_sr;
