@@ -91,7 +91,7 @@ fp8q_status fp8q_last_device_error(void* stream);
  * activations bullet).
  *   x  [M][K] BF16, row stride ldx (>= K, % 8 == 0)
  *   q  [M][K] FP8 codes (dense)        s [G(K)][lds] fp32 (1x128 layout)
- * Requires M >= 1, K % 16 == 0. */
+ * Requires M >= 1, K % 16 == 0, ceil(M/64) * G(K) < 2^31. */
 fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                                  uint8_t* q, float* s, int64_t lds, void* stream);
 
@@ -122,7 +122,8 @@ fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, int64_t
  *   h = bf16( fl32( fl32(g / fl32(1 + E(-g))) * u ) ),
  * with E the library's fixed fp32 exponential (Cody-Waite range reduction and a
  * degree-7 Taylor polynomial, argument clamped to [-80, 88]), then the 1x128
- * quantization of h:  q [M][I], s [G(I)][lds].   Requires I % 16 == 0. */
+ * quantization of h:  q [M][I], s [G(I)][lds].
+ * Requires I % 16 == 0, ceil(M/64) * G(I) < 2^31. */
 fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t I, int64_t ldgu,
                               uint8_t* q, float* s, int64_t lds, void* stream);
 
