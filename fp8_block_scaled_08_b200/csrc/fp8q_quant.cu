@@ -279,19 +279,17 @@ __device__ __forceinline__ void swiglu2(float g0, float g1, float u0, float u1, 
 }
 
 // ---------------------------------------------------------------------------
-// Row-group quantizers (a1, a4), fed by tensor copies. A unit is a box of kRgRows rows x
-// one 128-column group (16 KB of BF16; a4 takes two, the gate and the up columns). A
-// persistent CTA has one producer warp that keeps up to kStages boxes in flight through
-// a ring in shared memory, and 8 consumer warps: warp w quantizes rows 8w .. 8w+7 of a
-// box, two rows per step (a half-warp per row, lane l owning columns 8*(l%16) .. +7).
-// Loads through registers kept too few bytes in flight per SM to reach HBM bandwidth
-// (0.39 of it measured for a1); the ring keeps 96 KB per CTA in flight.
-// A box past a ragged M or K arrives zero-filled (zeros raise no group maximum) and only
-// its valid rows and columns are stored.
+// Row-group quantizer of SwiGLU (a4), fed by tensor copies. A unit is a box of kRgRows
+// rows x one 128-column group of the gate and the same of the up half (2 x 16 KB of
+// BF16). A persistent CTA has one producer warp that keeps up to kStages units in flight
+// through a ring in shared memory, and kConsumers consumer warps, each quantizing its
+// share of the box's rows two at a time (a half-warp per row, lane l owning columns
+// 8*(l%16) .. +7), so that many warps hide the latency of the exponential and the
+// divisions (one lane per whole group, as in a1, measured 1.5x slower here). A box past
+// a ragged M or K arrives zero-filled (zeros raise no group maximum) and only its valid
+// rows and columns are stored.
 // ---------------------------------------------------------------------------
-#ifndef A1_STAGES
-#define A1_STAGES 4
-#define A1_CONS 16
+#ifndef A4_STAGES
 #define A4_STAGES 2
 #define A4_CONS 16
 #endif
@@ -300,13 +298,6 @@ constexpr uint32_t kRgBoxBytes = kRgRows * 128 * 2;
 template <int kConsumers>
 constexpr int rg_threads() { return 32 * (kConsumers + 1); }
 
-struct ActBoxes {  // a1: the values themselves
-  static constexpr int kBoxes = 1;
-  __device__ __forceinline__ static void values(const uint16_t* b0, const uint16_t*, int off,
-                                                float (&v)[8]) {
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(b0 + off), v);
-  }
-};
 
 struct SwigluBoxes {  // a4: h = SwiGLU(gate, up) from the gate box and the up box
   static constexpr int kBoxes = 2;
@@ -413,6 +404,197 @@ __global__ void __launch_bounds__(rg_threads<kConsumers>()) rowgroup_tma_kernel(
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + st);  // this warp is done with the stage
   }
+}
+
+// ---------------------------------------------------------------------------
+// Lane-per-group row quantizer (a1). A unit is kLgRows = 32 rows x one 128-column group;
+// each lane of a consumer warp owns one row of it, i.e. one whole 1x128 group, so the
+// group maximum needs no shuffles and the scale is formed once per 128 values. A
+// producer warp streams units through tensor-copy stages; consumer warp w takes units w,
+// w + kConsumers, ... and owns kPer stages of its own (its units rotate through them), so
+// that a warp only ever waits on a stage whose previous phase it consumed itself (an
+// mbarrier parity wait cannot tell phase k from phase k - 2). The codes go through a per-warp staging box in
+// shared memory and leave by a tensor store (which also clips a ragged M or K); the
+// scales (one per lane) are one coalesced 128-byte store per unit.
+// Rows of a staged unit are 256 bytes apart, so lane r reads its 16-byte chunks in the
+// rotated order c = (j + r) mod 16: the 32 lanes of one load then cover 16 distinct chunk
+// positions (8 bank groups), 4 wavefronts for 512 bytes, the least possible. Codes are
+// staged in the same rotated order (8-byte pieces, 2 wavefronts per 256 bytes).
+// ---------------------------------------------------------------------------
+#ifndef LG1_PER
+#define LG1_PER 2
+#define LG1_CONS 10
+#endif
+#ifndef RL_CONS
+#define RL_CONS 8
+#define RL_PER 2
+#endif
+constexpr int kLgRows = 32;
+constexpr uint32_t kLgBoxBytes = kLgRows * 128 * 2;  // one BF16 box
+constexpr uint32_t kLgOutBytes = kLgRows * 128;      // its codes
+template <int kConsumers>
+constexpr int lg_threads() { return 32 * (kConsumers + 1); }
+
+template <class B, int kPer, int kConsumers>
+constexpr size_t lanegroup_smem() {
+  return 1024 + static_cast<size_t>(kPer * kConsumers) * B::kBoxes * kLgBoxBytes +
+         static_cast<size_t>(kConsumers) * kLgOutBytes + 2 * kPer * kConsumers * 8 + 16;
+}
+
+// Lane-wise max(|a|, |b|) of two packed BF16 pairs; the sign bits of the result are the
+// XOR of the operands' (max.xorsign.abs), so only the magnitudes are meaningful.
+__device__ __forceinline__ uint32_t bf16x2_maxabs_xs(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Magnitude of the larger half of a packed pair from bf16x2_maxabs_xs.
+__device__ __forceinline__ float bf16x2_hmax_abs(uint32_t m) {
+  return fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
+}
+
+// Codes of 8 BF16 values (four packed words) of one group; kSmall: some lane of the warp
+// has a tiny scale (the division path).
+template <bool kSmall>
+__device__ __forceinline__ uint2 codes8_words(const uint4& w, const GroupScale& g) {
+  float v[8];
+  unpack_bf16x8(w, v);
+  float t[8];
+  if (kSmall) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = g.small ? __fdiv_rn(v[i], g.s) : quot(v[i], g);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) quot2(v[i], v[i + 1], g, g, t[i], t[i + 1]);
+  }
+  return make_uint2(cvt_e4m3x4(t[0], t[1], t[2], t[3]), cvt_e4m3x4(t[4], t[5], t[6], t[7]));
+}
+
+struct ActLane {  // a1: the staged values themselves
+  static constexpr int kBoxes = 1;
+  __device__ __forceinline__ static uint4 chunk(const uint16_t* b0, const uint16_t*, int off) {
+    return *reinterpret_cast<const uint4*>(b0 + off);
+  }
+};
+
+
+// M rows, G = ceil(K / 128) groups of K valid columns. tm0 (and tm1) map the [M][K]
+// source(s) with 128 x kLgRows boxes; tmQ maps the [M][K] codes (same box); scales go to
+// s[g * lds + m]. The host keeps the unit count below 2^31.
+template <class B, int kPer, int kConsumers>
+__global__ void __launch_bounds__(lg_threads<kConsumers>(), 1) lanegroup_kernel(
+    const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+    const __grid_constant__ CUtensorMap tmQ, int64_t M, int64_t G, float* __restrict__ s,
+    int64_t lds, unsigned* err, uint64_t limit_ns) {
+  constexpr int kStages = kPer * kConsumers;
+  static_assert(kStages <= 32, "stage flags are one word");
+  constexpr uint32_t kStageBytes = B::kBoxes * kLgBoxBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* outs = base + kStages * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(outs + kConsumers * kLgOutBytes);
+  uint64_t* empty = full + kStages;
+  int* abort_flag = reinterpret_cast<int*>(empty + kStages);
+  const WaitCtl ctl{abort_flag, err, limit_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(full + st, 1);
+      mbar_init(empty + st, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const uint32_t units = static_cast<uint32_t>(((M + kLgRows - 1) / kLgRows) * G);
+  const uint32_t G32 = static_cast<uint32_t>(G);
+  if (warp == kConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0, par = 0;  // bit st: stage st has a copy issued / its parity
+      bool ok = true;
+      int i = 0;
+      for (uint32_t t = blockIdx.x; t < units; t += gridDim.x, ++i) {
+        const int li = i / kConsumers;  // the unit's index among its warp's units
+        const int st = (i % kConsumers) * kPer + li % kPer;
+        const uint32_t ph = static_cast<uint32_t>(li / kPer) & 1u;
+        if (li >= kPer && !mbar_wait(empty + st, ph ^ 1u, ctl)) { ok = false; break; }
+        const uint32_t tb = t / G32;
+        const int32_t x0 = static_cast<int32_t>((t - tb * G32) * 128);
+        const int32_t y0 = static_cast<int32_t>(tb * kLgRows);
+        mbar_arrive_expect_tx(full + st, kStageBytes);
+        tma_load_2d(base + st * kStageBytes, &tm0, x0, y0, full + st);
+        if (B::kBoxes == 2) tma_load_2d(base + st * kStageBytes + kLgBoxBytes, &tm1, x0, y0, full + st);
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (ph << st);
+      }
+      if (!ok) {  // let every copy already issued land before the CTA exits
+        for (int st = 0; st < kStages; ++st) {
+          if (!((issued >> st) & 1u)) continue;
+          const uint32_t a = smem_u32(full + st);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, (par >> st) & 1u))
+            if (global_timer_ns() - t0 > limit_ns) break;
+        }
+      }
+    }
+    return;
+  }
+  // -------------------------------------------------------------- consumers
+  uint8_t* out = outs + warp * kLgOutBytes;
+  bool stored = false;
+  int li = 0;
+  for (uint32_t t = blockIdx.x + warp * gridDim.x; t < units; t += kConsumers * gridDim.x, ++li) {
+    const int st = warp * kPer + li % kPer;
+    if (!mbar_wait_warp(full + st, static_cast<uint32_t>(li / kPer) & 1u, ctl)) break;
+    const uint16_t* row0 = reinterpret_cast<const uint16_t*>(base + st * kStageBytes) + lane * 128;
+    const uint16_t* row1 = row0 + kLgRows * 128;
+    uint4 w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = B::chunk(row0, row1, ((j + lane) & 15) * 8);
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      m[0] = bf16x2_maxabs_xs(m[0], w[j].x);
+      m[1] = bf16x2_maxabs_xs(m[1], w[j].y);
+      m[2] = bf16x2_maxabs_xs(m[2], w[j].z);
+      m[3] = bf16x2_maxabs_xs(m[3], w[j].w);
+    }
+    const float amax =
+        bf16x2_hmax_abs(bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3])));
+    __syncwarp();  // every lane's reads of the stage are complete (their values are used)
+    if (lane == 0) mbar_arrive(empty + st);
+    const GroupScale g = group_scale_bf16(amax);
+    const uint32_t tb = t / G32;
+    const int32_t x0 = static_cast<int32_t>((t - tb * G32) * 128);
+    const int32_t y0 = static_cast<int32_t>(tb * kLgRows);
+    if (stored) {  // the previous unit's store must have read the staging box
+      if (lane == 0) tma_store_wait_read();
+      __syncwarp();
+    }
+    uint8_t* orow = out + lane * 128;
+    if (__any_sync(kFull, g.small)) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = codes8_words<true>(w[j], g);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = codes8_words<false>(w[j], g);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&tmQ, out, x0, y0);
+      tma_store_commit();
+    }
+    stored = true;
+    const int64_t mrow = static_cast<int64_t>(y0) + lane;
+    if (mrow < M) s[static_cast<int64_t>(x0 / 128) * lds + mrow] = g.s;
+  }
+  if (stored && lane == 0) tma_store_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -588,6 +770,167 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_quant_cta_kernel(
     }
     __syncthreads();  // red / r_sh are reused by the next row
   }
+}
+
+// Lane-per-group RMSNorm + quantization (H a multiple of 128, at most 64 groups): a unit
+// is one row, staged whole by one tensor copy (a [M][G][128] view); consumer warp w takes
+// rows w, w + kConsumers, ... of the CTA's share. Lane l owns groups l, l + 32, ...: it
+// adds its groups' squares in fp64 (eight partial sums, one per position in a chunk), a
+// butterfly over the warp gives the row's sum, and from r each lane forms y = bf16(fl32(
+// fl32(x r) g)) of its group as packed BF16 words, takes their maximum, and writes the
+// codes into the warp's staging row, which leaves by a tensor store. Each consumer warp
+// owns `per` row stages (set by the host from the shared-memory budget; stages are per
+// warp for the reason given at lanegroup_kernel). Groups are 256 bytes apart
+// in a staged row, so lanes read their chunks in the rotated order of lanegroup_kernel.
+template <int kConsumers>
+__global__ void __launch_bounds__(32 * (kConsumers + 1), 1) rmsnorm_lane_kernel(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
+    const uint16_t* __restrict__ gamma, int64_t M, int G, int per, float eps,
+    float* __restrict__ s, int64_t lds, unsigned* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  const int nst = per * kConsumers;
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t row_bytes = static_cast<uint32_t>(G) * 256;
+  const uint16_t* gam = reinterpret_cast<const uint16_t*>(base);
+  uint8_t* ring = base + row_bytes;
+  uint8_t* outs = ring + static_cast<uint32_t>(nst) * row_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(outs + kConsumers * (row_bytes / 2));
+  uint64_t* empty = full + nst;
+  int* abort_flag = reinterpret_cast<int*>(empty + nst);
+  const WaitCtl ctl{abort_flag, err, limit_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t H = static_cast<int64_t>(G) * 128;
+  for (int i = threadIdx.x; i < G * 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(base)[i] = ld_nc_v4(gamma + i * 8);
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < nst; ++st) {
+      mbar_init(full + st, 1);
+      mbar_init(empty + st, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == kConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint64_t issued = 0, par = 0;  // bit st: stage st has a copy issued / its parity
+      bool ok = true;
+      int i = 0;
+      for (int64_t t = blockIdx.x; t < M; t += gridDim.x, ++i) {
+        const int li = i / kConsumers;  // the row's index among its warp's rows
+        const int st = (i % kConsumers) * per + li % per;
+        const uint32_t ph = static_cast<uint32_t>(li / per) & 1u;
+        if (li >= per && !mbar_wait(empty + st, ph ^ 1u, ctl)) { ok = false; break; }
+        mbar_arrive_expect_tx(full + st, row_bytes);
+        tma_load_3d(ring + st * row_bytes, &tmX, 0, 0, static_cast<int32_t>(t), full + st);
+        issued |= uint64_t{1} << st;
+        par = (par & ~(uint64_t{1} << st)) | (static_cast<uint64_t>(ph) << st);
+      }
+      if (!ok) {  // let every copy already issued land before the CTA exits
+        for (int st = 0; st < nst; ++st) {
+          if (!((issued >> st) & 1u)) continue;
+          const uint32_t a = smem_u32(full + st);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, static_cast<uint32_t>(par >> st) & 1u))
+            if (global_timer_ns() - t0 > limit_ns) break;
+        }
+      }
+    }
+    return;
+  }
+  // -------------------------------------------------------------- consumers
+  uint8_t* out = outs + warp * (row_bytes / 2);
+  const int rounds = (G + 31) >> 5;
+  bool stored = false;
+  int li = 0;
+  for (int64_t t = blockIdx.x + static_cast<int64_t>(warp) * gridDim.x; t < M;
+       t += static_cast<int64_t>(kConsumers) * gridDim.x, ++li) {
+    const int st = warp * per + li % per;
+    if (!mbar_wait_warp(full + st, static_cast<uint32_t>(li / per) & 1u, ctl)) break;
+    const uint16_t* xr = reinterpret_cast<const uint16_t*>(ring + st * row_bytes);
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    for (int k = 0; k < rounds; ++k) {
+      const int g = lane + 32 * k;
+      if (g < G) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float v[8];
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(xr + g * 128 + ((j + lane) & 15) * 8), v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const double d = static_cast<double>(v[e]);
+            acc[e] = __fma_rn(d, d, acc[e]);
+          }
+        }
+      }
+    }
+    double ss = __dadd_rn(__dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3])),
+                          __dadd_rn(__dadd_rn(acc[4], acc[5]), __dadd_rn(acc[6], acc[7])));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, off));
+    const float r = rstd_from_ss(ss, H, eps);
+    if (stored) {  // the previous row's store must have read the staging row
+      if (lane == 0) tma_store_wait_read();
+      __syncwarp();
+    }
+    for (int k = 0; k < rounds; ++k) {
+      const int g = lane + 32 * k;
+      const bool act = g < G;
+      const int gg = act ? g : 0;
+      uint4 y[16];
+      uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int off = gg * 128 + ((j + lane) & 15) * 8;
+        float xv[8], gv[8], b[8];
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(xr + off), xv);
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(gam + off), gv);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          float a0, a1;
+          mul2(a0, a1, xv[e], xv[e + 1], r, r);
+          mul2(b[e], b[e + 1], a0, a1, gv[e], gv[e + 1]);
+        }
+        y[j] = act ? make_uint4(pack_bf16x2(b[0], b[1]), pack_bf16x2(b[2], b[3]),
+                                pack_bf16x2(b[4], b[5]), pack_bf16x2(b[6], b[7]))
+                   : make_uint4(0u, 0u, 0u, 0u);
+        m[0] = bf16x2_maxabs_xs(m[0], y[j].x);
+        m[1] = bf16x2_maxabs_xs(m[1], y[j].y);
+        m[2] = bf16x2_maxabs_xs(m[2], y[j].z);
+        m[3] = bf16x2_maxabs_xs(m[3], y[j].w);
+      }
+      const float amax =
+          bf16x2_hmax_abs(bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3])));
+      const GroupScale gs = group_scale_bf16(amax);
+      uint8_t* orow = out + gg * 128;
+      if (__any_sync(kFull, gs.small)) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint2 c = codes8_words<true>(y[j], gs);
+          if (act) *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = c;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint2 c = codes8_words<false>(y[j], gs);
+          if (act) *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = c;
+        }
+      }
+      if (act) s[static_cast<int64_t>(g) * lds + t] = gs.s;
+    }
+    __syncwarp();  // every lane is done with the stage and has staged its codes
+    if (lane == 0) mbar_arrive(empty + st);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(&tmQ, out, 0, 0, static_cast<int32_t>(t));
+      tma_store_commit();
+    }
+    stored = true;
+  }
+  if (stored && lane == 0) tma_store_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -1586,6 +1929,25 @@ int resident_ctas(Kernel k, int threads, size_t dyn_smem, std::atomic<int>* cach
   return n;
 }
 
+// Opt a kernel in to the largest dynamic shared memory of an sm_100 CTA (once per device).
+constexpr size_t kMaxDynSmem = 232448;
+template <class Kernel>
+bool allow_max_smem(Kernel k) {
+  static std::atomic<int> done[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (done[dev].load(std::memory_order_acquire)) return true;
+  const cudaError_t e =
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kMaxDynSmem));
+  if (e != cudaSuccess) {
+    set_last_error("cudaFuncSetAttribute(max dynamic smem)", e);
+    cudaGetLastError();
+    return false;
+  }
+  done[dev].store(1, std::memory_order_release);
+  return true;
+}
+
 int grid_for(int64_t ctas_needed, int per_sm) {
   const int64_t cap = static_cast<int64_t>(sm100_sm_count()) * per_sm;
   const int64_t g = ctas_needed < cap ? ctas_needed : cap;
@@ -1604,20 +1966,23 @@ extern "C" fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_
   if (!aligned16(x) || !aligned16(q) || !aligned16(s) || ldx % 8) return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   const int64_t G = (K + 127) / 128;
-  if (((M + kRgRows - 1) / kRgRows) * G >= (int64_t{1} << 31)) return FP8Q_ERR_SHAPE;
-  CUtensorMap tm;
-  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, ldx * 2, 128, kRgRows,
+  const int64_t units = ((M + kLgRows - 1) / kLgRows) * G;
+  if (units >= (int64_t{1} << 31)) return FP8Q_ERR_SHAPE;
+  CUtensorMap tm, tmq;
+  if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, ldx * 2, 128, kLgRows,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, M, K, 128, kLgRows,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
     return FP8Q_ERR_UNSUPPORTED;
   unsigned* err = device_error_word();
   if (!err) return FP8Q_ERR_CUDA;
-  constexpr int kStages = A1_STAGES, kConsumers = A1_CONS;
-  auto kern = rowgroup_tma_kernel<ActBoxes, kStages, kConsumers>;
-  constexpr size_t smem = rowgroup_tma_smem<ActBoxes, kStages>();
+  constexpr int kPer = LG1_PER, kConsumers = LG1_CONS;
+  auto kern = lanegroup_kernel<ActLane, kPer, kConsumers>;
+  constexpr size_t smem = lanegroup_smem<ActLane, kPer, kConsumers>();
   static std::atomic<int> occ[64];
-  const int per_sm = resident_ctas(kern, rg_threads<kConsumers>(), smem, occ);
-  kern<<<grid_for(((M + kRgRows - 1) / kRgRows) * G, per_sm), rg_threads<kConsumers>(), smem,
-         static_cast<cudaStream_t>(stream)>>>(tm, tm, M, G, K, q, K, s, lds, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(kern, lg_threads<kConsumers>(), smem, occ);
+  kern<<<grid_for((units + kConsumers - 1) / kConsumers, per_sm), lg_threads<kConsumers>(), smem,
+         static_cast<cudaStream_t>(stream)>>>(tm, tm, tmq, M, G, s, lds, err, kWaitLimitNs);
   return launch_status("quant_act_1x128 launch");
 }
 
@@ -1664,6 +2029,36 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   const size_t gsm = static_cast<size_t>(H) * 2;  // gamma in shared memory
   // One warp per row needs many rows to fill the GPU; up to 1024 rows one CTA per row
   // is faster (measured 3x at 16-256 rows, equal at 8192).
+  if (M > 1024 && H % 128 == 0 && H <= 64 * 128) {
+    constexpr int kConsumers = RL_CONS;
+    const int G = static_cast<int>(H / 128);
+    const size_t row_bytes = static_cast<size_t>(G) * 256;
+    const size_t fixed = 1024 + row_bytes + kConsumers * (row_bytes / 2) + 16;
+    const int per = static_cast<int>(
+        std::min<size_t>(RL_PER, (kMaxDynSmem - fixed) / (kConsumers * (row_bytes + 16))));
+    const int nst = per * kConsumers;
+    if (per >= 1) {
+      const uint64_t dx[3] = {128, static_cast<uint64_t>(G), static_cast<uint64_t>(M)};
+      const uint64_t sx[2] = {256, static_cast<uint64_t>(ldx) * 2};
+      const uint64_t sq[2] = {128, static_cast<uint64_t>(H)};
+      const uint32_t box[3] = {128, static_cast<uint32_t>(G), 1};
+      CUtensorMap tmx, tmq;
+      if (!encode_tmap_3d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, dx, sx, box,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) ||
+          !encode_tmap_3d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, dx, sq, box,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+        return FP8Q_ERR_UNSUPPORTED;
+      unsigned* err = device_error_word();
+      if (!err) return FP8Q_ERR_CUDA;
+      auto kern = rmsnorm_lane_kernel<kConsumers>;
+      if (!allow_max_smem(kern)) return FP8Q_ERR_CUDA;
+      const size_t smem = fixed + static_cast<size_t>(nst) * (row_bytes + 16);
+      const int64_t ctas = (M + kConsumers - 1) / kConsumers;
+      kern<<<static_cast<int>(ctas < sms ? ctas : sms), 32 * (kConsumers + 1), smem, st>>>(
+          tmx, tmq, gamma, M, G, per, eps, s, lds, err, kWaitLimitNs);
+      return launch_status("rmsnorm_quant launch");
+    }
+  }
   if (M > 1024) {
     const int64_t ctas = (M + 7) / 8;  // one warp per row
     static std::atomic<int> occ[64];

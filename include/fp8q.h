@@ -91,7 +91,7 @@ fp8q_status fp8q_last_device_error(void* stream);
  * activations bullet).
  *   x  [M][K] BF16, row stride ldx (>= K, % 8 == 0)
  *   q  [M][K] FP8 codes (dense)        s [G(K)][lds] fp32 (1x128 layout)
- * Requires M >= 1, K % 16 == 0, ceil(M/64) * G(K) < 2^31. */
+ * Requires M >= 1, K % 16 == 0, ceil(M/32) * G(K) < 2^31. */
 fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                                  uint8_t* q, float* s, int64_t lds, void* stream);
 

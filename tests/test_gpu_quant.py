@@ -149,12 +149,14 @@ def test_weight_quant_matches_oracle(fq, oracle_mod, N, K):
 
 
 # ---------------------------------------------------------------- a3
-# batches up to 1024 rows take the CTA-per-row kernel; above, the two-pass warp-per-row
-# kernel (1100 x 640: ragged chunk count per lane; 1030 x 6144; 1025 x 16384: widest)
+# batches up to 1024 rows take the CTA-per-row kernel; above, H a multiple of 128 with at
+# most 64 groups takes the lane-per-group kernel (1100 x 640: 5 groups; 2050 x 4096: one
+# group per lane; 1040 x 4224 and 1030 x 6144: lanes with a second group), otherwise the
+# two-pass warp-per-row kernel (1025 x 16384: widest; 1060 x 4112: H not a multiple of 128)
 @pytest.mark.parametrize("M,H,eps", [(256, 512, 1e-5), (5, 4096, 1e-6), (130, 3584, 1e-5),
                                      (3, 16384, 0.0), (64, 128, 1e-5), (1100, 640, 1e-5),
                                      (1030, 6144, 1e-6), (1025, 16384, 1e-5),
-                                     (1040, 4224, 0.0)])
+                                     (1040, 4224, 0.0), (2050, 4096, 1e-5), (1060, 4112, 1e-5)])
 def test_rmsnorm_quant_matches_oracle(fq, oracle_mod, M, H, eps):
     x = workloads.activations_bf16((M, H), 0, 300 + M, DEV, outlier_frac=0.005,
                                    outlier_scale=50.0)
