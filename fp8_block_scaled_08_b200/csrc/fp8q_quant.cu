@@ -1759,6 +1759,265 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   }
 }
 
+// a6 for a BF16 gradient that is already formed (GradDirect): both groupings from one
+// 128 x 128 tile staged by a tensor copy, with every group owned by one lane.
+//   warps 0-3  1x128 rows: lane l of warp w owns row 32w + l of the tile (one group),
+//              exactly as lanegroup_kernel: codes through a per-warp staging box and a
+//              tensor store, one coalesced scale store per warp.
+//   warps 4-7  128x1 columns: warp 4 + q reads rows 32q .. 32q+31; lane l the column
+//              pairs (2l, 2l+1) and (64+2l, 65+2l) (one 4-byte word each per row, 128
+//              consecutive bytes per warp load). Partial maxima of the four row quarters
+//              meet in shared memory; warp 4 + q then forms the scales of columns 32q ..
+//              32q+31 (one per lane, also a coalesced store), and every lane quantizes its
+//              4 columns x 32 rows into a transposed [128 columns][128 rows] staging tile
+//              (128-byte swizzle, 2-way bank conflicts at most), which one tensor store
+//              writes to q_colT.
+//   warp 8     producer: tiles into a ring of kA6Stages buffers (one CTA per SM keeps
+//              up to 3 tiles = 96 KB in flight while it works on the fourth).
+// The scale tables sit in shared memory here: the column scales look up 32 different
+// entries per warp load, which the constant cache would serve one at a time.
+#ifndef A6_STAGES
+#define A6_STAGES 4
+#endif
+constexpr int kA6Stages = A6_STAGES;
+constexpr uint32_t kA6Tile = 128 * 128 * 2;
+constexpr uint32_t kA6OffCol = kA6Stages * kA6Tile;      // transposed codes, 16 KB
+constexpr uint32_t kA6OffRow = kA6OffCol + 128 * 128;    // 4 x (32 x 128) row codes
+constexpr uint32_t kA6OffRed = kA6OffRow + 128 * 128;    // [4][64] partial maxima
+constexpr uint32_t kA6OffSc = kA6OffRed + 4 * 64 * 4;    // [128] (s, rs) of the columns
+constexpr uint32_t kA6OffTab = kA6OffSc + 128 * 8;       // scale and reciprocal tables
+constexpr uint32_t kA6OffBar = kA6OffTab + 256 * 4;      // full[], empty[], csync
+constexpr size_t kA6Smem = 1024 + kA6OffBar + (2 * kA6Stages + 1) * 8 + 16;
+constexpr int kA6Threads = 9 * 32;
+
+// group_scale_bf16 with its tables in shared memory (tab[0..127] the scale mantissas,
+// tab[128..255] their reciprocals); same result.
+__device__ __forceinline__ GroupScale group_scale_bf16_sm(float amax, const float* tab) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ebias = static_cast<int>(b >> 23);
+  const bool tiny = ebias < 127 - 71 || ebias == 255;
+  const int e = ebias - 127;
+  const uint32_t i = (b >> 16) & 0x7Fu;
+  GroupScale g;
+  g.s = __uint_as_float(__float_as_uint(tab[i]) + static_cast<uint32_t>((e - 6) << 23));
+  g.rs = __uint_as_float(__float_as_uint(tab[128 + i]) + static_cast<uint32_t>((6 - e) << 23));
+  g.small = false;
+  if (__any_sync(kFull, tiny)) {
+    if (tiny) {
+      g = group_scale(amax);
+      g.small = true;
+    }
+  }
+  g.ns = -g.s;
+  return g;
+}
+
+template <bool kRows>
+__global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
+    const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmQ,
+    const __grid_constant__ CUtensorMap tmQT, int64_t M, int64_t N, float* __restrict__ s_row,
+    int64_t lds_row, float* __restrict__ s_col, unsigned* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float* tab = reinterpret_cast<float*>(base + kA6OffTab);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kA6OffBar);
+  uint64_t* empty = full + kA6Stages;
+  uint64_t* csync = empty + kA6Stages;  // the column warps' rendezvous (bounded, unlike bar.sync)
+  int* abort_flag = reinterpret_cast<int*>(csync + 1);
+  const WaitCtl ctl{abort_flag, err, limit_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < 128) {
+    tab[threadIdx.x] = kScaleMant[threadIdx.x];
+    tab[128 + threadIdx.x] = kRecipMant[threadIdx.x];
+  }
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < kA6Stages; ++b) {
+      mbar_init(full + b, 1);
+      mbar_init(empty + b, 8);
+    }
+    mbar_init(csync, 4);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int64_t NB = (N + 127) >> 7;
+  const int64_t tiles = ((M + 127) >> 7) * NB;
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0, par = 0;
+      bool ok = true;
+      int i = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int b = i % kA6Stages;
+        const uint32_t ph = static_cast<uint32_t>(i / kA6Stages) & 1u;
+        if (i >= kA6Stages && !mbar_wait(empty + b, ph ^ 1u, ctl)) { ok = false; break; }
+        const int64_t mb = t / NB, nb = t - mb * NB;
+        mbar_arrive_expect_tx(full + b, kA6Tile);
+        tma_load_2d(base + b * kA6Tile, &tmD, static_cast<int32_t>(nb * 128),
+                    static_cast<int32_t>(mb * 128), full + b);
+        issued |= 1u << b;
+        par = (par & ~(1u << b)) | (ph << b);
+      }
+      if (!ok) {  // let every copy already issued land before the CTA exits
+        for (int b = 0; b < kA6Stages; ++b) {
+          if (!((issued >> b) & 1u)) continue;
+          const uint32_t a = smem_u32(full + b);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, (par >> b) & 1u))
+            if (global_timer_ns() - t0 > limit_ns) break;
+        }
+      }
+    }
+    return;
+  }
+  bool stored = false;
+  if (warp < 4) {
+    // ------------------------------------------------------------ 1x128 rows
+    uint8_t* out = base + kA6OffRow + warp * (32 * 128);
+    int i = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int b = i % kA6Stages;
+      if (!mbar_wait_warp(full + b, static_cast<uint32_t>(i / kA6Stages) & 1u, ctl)) break;
+      if (!kRows) {
+        if (lane == 0) mbar_arrive(empty + b);
+        continue;
+      }
+      const uint16_t* row = reinterpret_cast<const uint16_t*>(base + b * kA6Tile) + (warp * 32 + lane) * 128;
+      uint4 w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) w[j] = *reinterpret_cast<const uint4*>(row + ((j + lane) & 15) * 8);
+      uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        m[0] = bf16x2_maxabs_xs(m[0], w[j].x);
+        m[1] = bf16x2_maxabs_xs(m[1], w[j].y);
+        m[2] = bf16x2_maxabs_xs(m[2], w[j].z);
+        m[3] = bf16x2_maxabs_xs(m[3], w[j].w);
+      }
+      const float amax =
+          bf16x2_hmax_abs(bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3])));
+      __syncwarp();  // every lane's reads of the tile are complete (their values are used)
+      if (lane == 0) mbar_arrive(empty + b);
+      const GroupScale g = group_scale_bf16_sm(amax, tab);
+      const int64_t mb = t / NB, nb = t - mb * NB;
+      if (stored) {
+        if (lane == 0) tma_store_wait_read();
+        __syncwarp();
+      }
+      uint8_t* orow = out + lane * 128;
+      if (__any_sync(kFull, g.small)) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = codes8_words<true>(w[j], g);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = codes8_words<false>(w[j], g);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int64_t m0 = mb * 128 + warp * 32;
+      if (lane == 0) {
+        tma_store_2d(&tmQ, out, static_cast<int32_t>(nb * 128), static_cast<int32_t>(m0));
+        tma_store_commit();
+      }
+      stored = true;
+      if (m0 + lane < M) s_row[nb * lds_row + m0 + lane] = g.s;
+    }
+  } else {
+    // ------------------------------------------------------------ 128x1 columns
+    const int q4 = warp - 4;  // row quarter
+    uint32_t* red = reinterpret_cast<uint32_t*>(base + kA6OffRed);
+    float2* sc = reinterpret_cast<float2*>(base + kA6OffSc);
+    uint8_t* colst = base + kA6OffCol;
+    // All four column warps meet here three times a tile: each warp's lanes finish their
+    // shared-memory writes, lane 0 arrives, and the warp waits (bounded) for the phase.
+    uint32_t nsync = 0;
+    auto col_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(csync);
+      return mbar_wait_warp(csync, (nsync++) & 1u, ctl);
+    };
+    int i = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int b = i % kA6Stages;
+      if (!mbar_wait_warp(full + b, static_cast<uint32_t>(i / kA6Stages) & 1u, ctl)) break;
+      const uint32_t* tw = reinterpret_cast<const uint32_t*>(base + b * kA6Tile) + q4 * 32 * 64;
+      uint32_t w0[32], w1[32];  // pair (2l, 2l+1) and (64+2l, 65+2l), rows 32q4 + k
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        w0[k] = tw[k * 64 + lane];
+        w1[k] = tw[k * 64 + 32 + lane];
+      }
+      uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        m0 = bf16x2_maxabs_xs(m0, w0[k]);
+        m1 = bf16x2_maxabs_xs(m1, w0[k + 1]);
+        m2 = bf16x2_maxabs_xs(m2, w1[k]);
+        m3 = bf16x2_maxabs_xs(m3, w1[k + 1]);
+      }
+      __syncwarp();  // every lane's reads of the tile are complete (their values are used)
+      if (lane == 0) mbar_arrive(empty + b);
+      red[q4 * 64 + lane] = bf16x2_maxabs_xs(m0, m1);       // columns 2l, 2l+1
+      red[q4 * 64 + 32 + lane] = bf16x2_maxabs_xs(m2, m3);  // columns 64+2l, 65+2l
+      if (stored && q4 == 0 && lane == 0) tma_store_wait_read();  // the staging tile is free
+      if (!col_sync()) break;
+      const int64_t mb = t / NB, nb = t - mb * NB;
+      {  // the scale of column c = 32 q4 + lane
+        const int c = q4 * 32 + lane;
+        const int wi = (c & 63) >> 1, hi = c & 1;
+        uint32_t mm = 0u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) mm = bf16x2_maxabs_xs(mm, red[q * 64 + (c >> 6) * 32 + wi]);
+        const float amax = fabsf(hi ? bf16_hi(mm) : bf16_lo(mm));
+        const GroupScale g = group_scale_bf16_sm(amax, tab);
+        sc[c] = make_float2(g.s, g.rs);
+        if (nb * 128 + c < N) s_col[mb * N + nb * 128 + c] = g.s;
+      }
+      if (!col_sync()) break;
+      // codes of columns 2l, 2l+1 (w0) and 64+2l, 65+2l (w1), rows 32 q4 .. +31
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t* wv = h ? w1 : w0;
+        const int c0 = 64 * h + 2 * lane;
+        const float2 sr0 = sc[c0], sr1 = sc[c0 + 1];
+        GroupScale g0, g1;
+        g0.s = sr0.x; g0.rs = sr0.y; g0.ns = -sr0.x; g0.small = sr0.x < kSmallScale;
+        g1.s = sr1.x; g1.rs = sr1.y; g1.ns = -sr1.x; g1.small = sr1.x < kSmallScale;
+        uint32_t o0[8], o1[8];
+        if (__any_sync(kFull, g0.small || g1.small))
+          col_codes<true, 32>(*reinterpret_cast<const uint32_t(*)[32]>(wv), g0, g1, o0, o1);
+        else
+          col_codes<false, 32>(*reinterpret_cast<const uint32_t(*)[32]>(wv), g0, g1, o0, o1);
+        // staging row c holds column c's 128 codes; 16-byte chunk k of the row (rows 16k ..
+        // 16k+15 of the tile) sits at position k ^ (c & 7) (the 128-byte swizzle)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = c0 + e;
+          const uint32_t* o = e ? o1 : o0;
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int k = 2 * q4 + k2;
+            *reinterpret_cast<uint4*>(colst + c * 128 + ((k ^ (c & 7)) << 4)) =
+                make_uint4(o[4 * k2], o[4 * k2 + 1], o[4 * k2 + 2], o[4 * k2 + 3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      if (!col_sync()) break;
+      if (q4 == 0 && lane == 0) {
+        tma_store_2d(&tmQT, colst, static_cast<int32_t>(mb * 128), static_cast<int32_t>(nb * 128));
+        tma_store_commit();
+      }
+      stored = true;
+    }
+  }
+  if (stored && lane == 0) tma_store_wait_all();
+}
+
 // dgamma_j = the exact sum over rows of fl32(dy_mj * fl32(x_mj * r_m)), rounded once to
 // fp32. A warp takes a strip of 32 8-column chunks (one per lane) over kDgRows rows, keeps
 // each of its 8 columns as an exact sum, and adds each column's bins into the global
@@ -2105,13 +2364,31 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
       (q_row && (!aligned16(q_row) || !aligned16(s_row))))
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  constexpr size_t kSmem = direct_smem_bytes<GradDirect>();
-  auto kern = direct_dual_kernel<GradDirect, kA6Batch, kA6MinBlocks>;
-  static std::atomic<int> occ[64];
-  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
-  kern<<<grid_for(((M + 127) / 128) * ((N + 127) / 128), per_sm), 256, kSmem,
-         static_cast<cudaStream_t>(stream)>>>(
-      GradDirect{dy, lddy}, M, N, nullptr, q_row, s_row, lds_row, q_colT, s_col);
+  CUtensorMap tmd, tmq, tmqt;
+  if (!encode_tmap_2d(&tmd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, N, M, lddy * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_colT, M, N, M, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8Q_ERR_UNSUPPORTED;
+  if (q_row && !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_row, N, M, N, 128, 32,
+                               CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  if (!q_row) tmq = tmqt;  // unused
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  const int64_t tiles = ((M + 127) / 128) * ((N + 127) / 128);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (q_row) {
+    static std::atomic<int> occ[64];
+    const int per_sm = resident_ctas(a6_tile_kernel<true>, kA6Threads, kA6Smem, occ);
+    a6_tile_kernel<true><<<grid_for(tiles, per_sm), kA6Threads, kA6Smem, st>>>(
+        tmd, tmq, tmqt, M, N, s_row, lds_row, s_col, err, kWaitLimitNs);
+  } else {
+    static std::atomic<int> occ[64];
+    const int per_sm = resident_ctas(a6_tile_kernel<false>, kA6Threads, kA6Smem, occ);
+    a6_tile_kernel<false><<<grid_for(tiles, per_sm), kA6Threads, kA6Smem, st>>>(
+        tmd, tmq, tmqt, M, N, s_row, lds_row, s_col, err, kWaitLimitNs);
+  }
   return launch_status("transpose_quant_bf16 launch");
 }
 
