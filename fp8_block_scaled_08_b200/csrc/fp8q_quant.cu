@@ -1764,15 +1764,14 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
 //   warps 0-3  1x128 rows: lane l of warp w owns row 32w + l of the tile (one group),
 //              exactly as lanegroup_kernel: codes through a per-warp staging box and a
 //              tensor store, one coalesced scale store per warp.
-//   warps 4-7  128x1 columns: warp 4 + q reads rows 32q .. 32q+31; lane l the column
-//              pairs (2l, 2l+1) and (64+2l, 65+2l) (one 4-byte word each per row, 128
+//   warps 4-11 128x1 columns: warp 4 + 4h + q reads rows 32q .. 32q+31 of the column
+//              pairs 64h + (2l, 2l+1), l the lane (one 4-byte word per row and lane, 128
 //              consecutive bytes per warp load). Partial maxima of the four row quarters
-//              meet in shared memory; warp 4 + q then forms the scales of columns 32q ..
-//              32q+31 (one per lane, also a coalesced store), and every lane quantizes its
-//              4 columns x 32 rows into a transposed [128 columns][128 rows] staging tile
-//              (128-byte swizzle, 2-way bank conflicts at most), which one tensor store
-//              writes to q_colT.
-//   warp 8     producer: tiles into a ring of kA6Stages buffers (one CTA per SM keeps
+//              meet in shared memory; every lane then forms the scales of its two columns
+//              and quantizes its 2 columns x 32 rows into a transposed [128 columns][128
+//              rows] staging tile (128-byte swizzle, 2-way bank conflicts at most), which
+//              one tensor store writes to q_colT.
+//   warp 12    producer: tiles into a ring of kA6Stages buffers (one CTA per SM keeps
 //              up to 3 tiles = 96 KB in flight while it works on the fourth).
 // The scale tables sit in shared memory here: the column scales look up 32 different
 // entries per warp load, which the constant cache would serve one at a time.
@@ -1784,11 +1783,10 @@ constexpr uint32_t kA6Tile = 128 * 128 * 2;
 constexpr uint32_t kA6OffCol = kA6Stages * kA6Tile;      // transposed codes, 16 KB
 constexpr uint32_t kA6OffRow = kA6OffCol + 128 * 128;    // 4 x (32 x 128) row codes
 constexpr uint32_t kA6OffRed = kA6OffRow + 128 * 128;    // [4][64] partial maxima
-constexpr uint32_t kA6OffSc = kA6OffRed + 4 * 64 * 4;    // [128] (s, rs) of the columns
-constexpr uint32_t kA6OffTab = kA6OffSc + 128 * 8;       // scale and reciprocal tables
+constexpr uint32_t kA6OffTab = kA6OffRed + 4 * 64 * 4;   // scale and reciprocal tables
 constexpr uint32_t kA6OffBar = kA6OffTab + 256 * 4;      // full[], empty[], csync
 constexpr size_t kA6Smem = 1024 + kA6OffBar + (2 * kA6Stages + 1) * 8 + 16;
-constexpr int kA6Threads = 9 * 32;
+constexpr int kA6Threads = 13 * 32;
 
 // group_scale_bf16 with its tables in shared memory (tab[0..127] the scale mantissas,
 // tab[128..255] their reciprocals); same result.
@@ -1834,16 +1832,16 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
   if (threadIdx.x == 0) {
     for (int b = 0; b < kA6Stages; ++b) {
       mbar_init(full + b, 1);
-      mbar_init(empty + b, 8);
+      mbar_init(empty + b, 12);
     }
-    mbar_init(csync, 4);
+    mbar_init(csync, 8);
     *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
   const int64_t NB = (N + 127) >> 7;
   const int64_t tiles = ((M + 127) >> 7) * NB;
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t issued = 0, par = 0;
@@ -1928,12 +1926,13 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
     }
   } else {
     // ------------------------------------------------------------ 128x1 columns
-    const int q4 = warp - 4;  // row quarter
+    const int cw = warp - 4;
+    const int q4 = cw & 3;                // row quarter: rows 32 q4 .. 32 q4 + 31
+    const int c0 = 64 * (cw >> 2) + 2 * lane;  // this lane's column pair c0, c0 + 1
     uint32_t* red = reinterpret_cast<uint32_t*>(base + kA6OffRed);
-    float2* sc = reinterpret_cast<float2*>(base + kA6OffSc);
     uint8_t* colst = base + kA6OffCol;
-    // All four column warps meet here three times a tile: each warp's lanes finish their
-    // shared-memory writes, lane 0 arrives, and the warp waits (bounded) for the phase.
+    // The eight column warps meet twice a tile: each warp's lanes finish their shared-
+    // memory writes, lane 0 arrives, and the warp waits (bounded) for the phase.
     uint32_t nsync = 0;
     auto col_sync = [&]() -> bool {
       __syncwarp();
@@ -1944,71 +1943,50 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int b = i % kA6Stages;
       if (!mbar_wait_warp(full + b, static_cast<uint32_t>(i / kA6Stages) & 1u, ctl)) break;
-      const uint32_t* tw = reinterpret_cast<const uint32_t*>(base + b * kA6Tile) + q4 * 32 * 64;
-      uint32_t w0[32], w1[32];  // pair (2l, 2l+1) and (64+2l, 65+2l), rows 32q4 + k
+      const uint32_t* tw = reinterpret_cast<const uint32_t*>(base + b * kA6Tile) + q4 * 32 * 64 + (c0 >> 1);
+      uint32_t w[32];  // columns c0, c0 + 1 of rows 32 q4 + k
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        w0[k] = tw[k * 64 + lane];
-        w1[k] = tw[k * 64 + 32 + lane];
-      }
-      uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
+      for (int k = 0; k < 32; ++k) w[k] = tw[k * 64];
+      uint32_t m0 = 0u, m1 = 0u;
 #pragma unroll
       for (int k = 0; k < 32; k += 2) {
-        m0 = bf16x2_maxabs_xs(m0, w0[k]);
-        m1 = bf16x2_maxabs_xs(m1, w0[k + 1]);
-        m2 = bf16x2_maxabs_xs(m2, w1[k]);
-        m3 = bf16x2_maxabs_xs(m3, w1[k + 1]);
+        m0 = bf16x2_maxabs_xs(m0, w[k]);
+        m1 = bf16x2_maxabs_xs(m1, w[k + 1]);
       }
       __syncwarp();  // every lane's reads of the tile are complete (their values are used)
       if (lane == 0) mbar_arrive(empty + b);
-      red[q4 * 64 + lane] = bf16x2_maxabs_xs(m0, m1);       // columns 2l, 2l+1
-      red[q4 * 64 + 32 + lane] = bf16x2_maxabs_xs(m2, m3);  // columns 64+2l, 65+2l
-      if (stored && q4 == 0 && lane == 0) tma_store_wait_read();  // the staging tile is free
+      red[q4 * 64 + (c0 >> 1)] = bf16x2_maxabs_xs(m0, m1);
+      if (stored && cw == 0 && lane == 0) tma_store_wait_read();  // the staging tile is free
       if (!col_sync()) break;
       const int64_t mb = t / NB, nb = t - mb * NB;
-      {  // the scale of column c = 32 q4 + lane
-        const int c = q4 * 32 + lane;
-        const int wi = (c & 63) >> 1, hi = c & 1;
-        uint32_t mm = 0u;
+      uint32_t mm = 0u;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) mm = bf16x2_maxabs_xs(mm, red[q * 64 + (c >> 6) * 32 + wi]);
-        const float amax = fabsf(hi ? bf16_hi(mm) : bf16_lo(mm));
-        const GroupScale g = group_scale_bf16_sm(amax, tab);
-        sc[c] = make_float2(g.s, g.rs);
-        if (nb * 128 + c < N) s_col[mb * N + nb * 128 + c] = g.s;
-      }
-      if (!col_sync()) break;
-      // codes of columns 2l, 2l+1 (w0) and 64+2l, 65+2l (w1), rows 32 q4 .. +31
+      for (int q = 0; q < 4; ++q) mm = bf16x2_maxabs_xs(mm, red[q * 64 + (c0 >> 1)]);
+      const GroupScale g0 = group_scale_bf16_sm(fabsf(bf16_lo(mm)), tab);
+      const GroupScale g1 = group_scale_bf16_sm(fabsf(bf16_hi(mm)), tab);
+      if (q4 == 0 && nb * 128 + c0 < N)
+        *reinterpret_cast<float2*>(s_col + mb * N + nb * 128 + c0) = make_float2(g0.s, g1.s);
+      uint32_t o0[8], o1[8];
+      if (__any_sync(kFull, g0.small || g1.small))
+        col_codes<true, 32>(w, g0, g1, o0, o1);
+      else
+        col_codes<false, 32>(w, g0, g1, o0, o1);
+      // staging row c holds column c's 128 codes; 16-byte chunk k of the row (rows 16k ..
+      // 16k+15 of the tile) sits at position k ^ (c & 7) (the 128-byte swizzle)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t* wv = h ? w1 : w0;
-        const int c0 = 64 * h + 2 * lane;
-        const float2 sr0 = sc[c0], sr1 = sc[c0 + 1];
-        GroupScale g0, g1;
-        g0.s = sr0.x; g0.rs = sr0.y; g0.ns = -sr0.x; g0.small = sr0.x < kSmallScale;
-        g1.s = sr1.x; g1.rs = sr1.y; g1.ns = -sr1.x; g1.small = sr1.x < kSmallScale;
-        uint32_t o0[8], o1[8];
-        if (__any_sync(kFull, g0.small || g1.small))
-          col_codes<true, 32>(*reinterpret_cast<const uint32_t(*)[32]>(wv), g0, g1, o0, o1);
-        else
-          col_codes<false, 32>(*reinterpret_cast<const uint32_t(*)[32]>(wv), g0, g1, o0, o1);
-        // staging row c holds column c's 128 codes; 16-byte chunk k of the row (rows 16k ..
-        // 16k+15 of the tile) sits at position k ^ (c & 7) (the 128-byte swizzle)
+      for (int e = 0; e < 2; ++e) {
+        const int c = c0 + e;
+        const uint32_t* o = e ? o1 : o0;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = c0 + e;
-          const uint32_t* o = e ? o1 : o0;
-#pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const int k = 2 * q4 + k2;
-            *reinterpret_cast<uint4*>(colst + c * 128 + ((k ^ (c & 7)) << 4)) =
-                make_uint4(o[4 * k2], o[4 * k2 + 1], o[4 * k2 + 2], o[4 * k2 + 3]);
-          }
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int k = 2 * q4 + k2;
+          *reinterpret_cast<uint4*>(colst + c * 128 + ((k ^ (c & 7)) << 4)) =
+              make_uint4(o[4 * k2], o[4 * k2 + 1], o[4 * k2 + 2], o[4 * k2 + 3]);
         }
       }
       fence_proxy_async_smem();
       if (!col_sync()) break;
-      if (q4 == 0 && lane == 0) {
+      if (cw == 0 && lane == 0) {
         tma_store_2d(&tmQT, colst, static_cast<int32_t>(mb * 128), static_cast<int32_t>(nb * 128));
         tma_store_commit();
       }
