@@ -1786,7 +1786,7 @@ constexpr uint32_t kA6OffRed = kA6OffRow + 128 * 128;    // [4][64] partial maxi
 constexpr uint32_t kA6OffTab = kA6OffRed + 4 * 64 * 4;   // scale and reciprocal tables
 constexpr uint32_t kA6OffBar = kA6OffTab + 256 * 4;      // full[], empty[], csync
 constexpr size_t kA6Smem = 1024 + kA6OffBar + (2 * kA6Stages + 1) * 8 + 16;
-constexpr int kA6Threads = 13 * 32;
+constexpr int kA6Threads = 17 * 32;
 
 // group_scale_bf16 with its tables in shared memory (tab[0..127] the scale mantissas,
 // tab[128..255] their reciprocals); same result.
@@ -1832,7 +1832,7 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
   if (threadIdx.x == 0) {
     for (int b = 0; b < kA6Stages; ++b) {
       mbar_init(full + b, 1);
-      mbar_init(empty + b, 12);
+      mbar_init(empty + b, 16);
     }
     mbar_init(csync, 8);
     *abort_flag = 0;
@@ -1841,7 +1841,7 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
   __syncthreads();
   const int64_t NB = (N + 127) >> 7;
   const int64_t tiles = ((M + 127) >> 7) * NB;
-  if (warp == 12) {
+  if (warp == 16) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t issued = 0, par = 0;
@@ -1871,9 +1871,11 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
     return;
   }
   bool stored = false;
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------------------ 1x128 rows
-    uint8_t* out = base + kA6OffRow + warp * (32 * 128);
+    // lane l of warp w: row 16w + (l % 16) of the tile, chunks 8 (l / 16) .. + 7 of it
+    uint8_t* out = base + kA6OffRow + warp * (16 * 128);
+    const int rl = lane & 15, hh = lane >> 4;
     int i = 0;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int b = i % kA6Stages;
@@ -1882,20 +1884,21 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
         if (lane == 0) mbar_arrive(empty + b);
         continue;
       }
-      const uint16_t* row = reinterpret_cast<const uint16_t*>(base + b * kA6Tile) + (warp * 32 + lane) * 128;
-      uint4 w[16];
+      const uint16_t* row = reinterpret_cast<const uint16_t*>(base + b * kA6Tile) + (warp * 16 + rl) * 128 + hh * 64;
+      uint4 w[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) w[j] = *reinterpret_cast<const uint4*>(row + ((j + lane) & 15) * 8);
+      for (int j = 0; j < 8; ++j) w[j] = *reinterpret_cast<const uint4*>(row + ((j + lane) & 7) * 8);
       uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 8; ++j) {
         m[0] = bf16x2_maxabs_xs(m[0], w[j].x);
         m[1] = bf16x2_maxabs_xs(m[1], w[j].y);
         m[2] = bf16x2_maxabs_xs(m[2], w[j].z);
         m[3] = bf16x2_maxabs_xs(m[3], w[j].w);
       }
-      const float amax =
-          bf16x2_hmax_abs(bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3])));
+      uint32_t mh = bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3]));
+      mh = bf16x2_maxabs_xs(mh, __shfl_xor_sync(kFull, mh, 16));  // the row's other half
+      const float amax = bf16x2_hmax_abs(mh);
       __syncwarp();  // every lane's reads of the tile are complete (their values are used)
       if (lane == 0) mbar_arrive(empty + b);
       const GroupScale g = group_scale_bf16_sm(amax, tab);
@@ -1904,29 +1907,29 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
         if (lane == 0) tma_store_wait_read();
         __syncwarp();
       }
-      uint8_t* orow = out + lane * 128;
+      uint8_t* orow = out + rl * 128 + hh * 64;
       if (__any_sync(kFull, g.small)) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = codes8_words<true>(w[j], g);
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint2*>(orow + ((j + lane) & 7) * 8) = codes8_words<true>(w[j], g);
       } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = codes8_words<false>(w[j], g);
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint2*>(orow + ((j + lane) & 7) * 8) = codes8_words<false>(w[j], g);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      const int64_t m0 = mb * 128 + warp * 32;
+      const int64_t m0 = mb * 128 + warp * 16;
       if (lane == 0) {
         tma_store_2d(&tmQ, out, static_cast<int32_t>(nb * 128), static_cast<int32_t>(m0));
         tma_store_commit();
       }
       stored = true;
-      if (m0 + lane < M) s_row[nb * lds_row + m0 + lane] = g.s;
+      if (hh == 0 && m0 + rl < M) s_row[nb * lds_row + m0 + rl] = g.s;
     }
   } else {
     // ------------------------------------------------------------ 128x1 columns
-    const int cw = warp - 4;
+    const int cw = warp - 8;
     const int q4 = cw & 3;                // row quarter: rows 32 q4 .. 32 q4 + 31
     const int c0 = 64 * (cw >> 2) + 2 * lane;  // this lane's column pair c0, c0 + 1
     uint32_t* red = reinterpret_cast<uint32_t*>(base + kA6OffRed);
@@ -2348,7 +2351,7 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
       !encode_tmap_2d(&tmqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_colT, M, N, M, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_UNSUPPORTED;
-  if (q_row && !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_row, N, M, N, 128, 32,
+  if (q_row && !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_row, N, M, N, 128, 16,
                                CU_TENSOR_MAP_SWIZZLE_NONE))
     return FP8Q_ERR_UNSUPPORTED;
   if (!q_row) tmq = tmqt;  // unused
