@@ -2058,8 +2058,10 @@ __global__ void __launch_bounds__(256) dgamma_round_kernel(const unsigned long l
 // a8: saved FP8 activation tiles (1x128 groups) -> xhat = fl32(s * dec(q)) -> 128x1
 // groups along M, stored transposed; persistent over the (M/128) x (K/128) tiles.
 // Each buffer holds the 16 KB code tile and its 128 row scales. xhat is an arbitrary
-// fp32 value here (not a BF16 one), so the quotients are the IEEE quotient itself, formed
-// through an fp64 reciprocal (exact, see the column loop).
+// fp32 value here (not a BF16 one), so the quotient must be the IEEE quotient itself:
+// quot's q + (x - q s) y with y = fl32(1/s) and q = fl32(x y) is fl32(x / s) for every
+// x and s of fp32 without underflow (Markstein's theorem: y within half an ulp of 1/s,
+// q within one ulp of x/s, the residual exact by the FMA). Scales below 2^-80 divide.
 __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS, int64_t M,
     int64_t K, uint8_t* __restrict__ qT, float* __restrict__ sT, unsigned* err,
@@ -2113,28 +2115,35 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
                fmaxf(sm.red[256 + 2 * cp], sm.red[384 + 2 * cp]));
     a1 = fmaxf(fmaxf(sm.red[2 * cp + 1], sm.red[128 + 2 * cp + 1]),
                fmaxf(sm.red[256 + 2 * cp + 1], sm.red[384 + 2 * cp + 1]));
-    const float s0 = (a0 == 0.0f) ? 1.0f : __fdiv_rn(a0, 448.0f);
-    const float s1 = (a1 == 0.0f) ? 1.0f : __fdiv_rn(a1, 448.0f);
+    const GroupScale g0 = group_scale(a0), g1 = group_scale(a1);
+    const float s0 = g0.s, s1 = g1.s;
     // a partial tile (ragged M or K) arrived zero-filled; store only its valid part
     const int rows = M - mb * 128 < 128 ? static_cast<int>(M - mb * 128) : 128;
     const bool col_ok = kb * 128 + 2 * cp < K;  // K is even: the pair is in or out
     if (rq == 0 && col_ok)
       *reinterpret_cast<float2*>(sT + mb * K + kb * 128 + 2 * cp) = make_float2(s0, s1);
-    // fl32(x / s) as fl32(x * fl64(1 / s)), the product in fp64: the IEEE quotient for
-    // every finite fp32 x and s (an exact quotient of fp32 values stays ~2^-49 away from
-    // any fp32 rounding midpoint, the fp64 product within ~2^-52 of it)
-    const double r0 = __ddiv_rn(1.0, static_cast<double>(s0));
-    const double r1 = __ddiv_rn(1.0, static_cast<double>(s1));
-    auto qd = [](float x, double r) {
-      return __double2float_rn(__dmul_rn(static_cast<double>(x), r));
-    };
     uint32_t o0[8], o1[8];
+    if (__any_sync(kFull, g0.small || g1.small)) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      o0[k] = cvt_e4m3x4(qd(x0[4 * k], r0), qd(x0[4 * k + 1], r0), qd(x0[4 * k + 2], r0),
-                         qd(x0[4 * k + 3], r0));
-      o1[k] = cvt_e4m3x4(qd(x1[4 * k], r1), qd(x1[4 * k + 1], r1), qd(x1[4 * k + 2], r1),
-                         qd(x1[4 * k + 3], r1));
+      for (int k = 0; k < 8; ++k) {
+        float t0[4], t1[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          t0[e] = g0.small ? __fdiv_rn(x0[4 * k + e], g0.s) : quot(x0[4 * k + e], g0);
+          t1[e] = g1.small ? __fdiv_rn(x1[4 * k + e], g1.s) : quot(x1[4 * k + e], g1);
+        }
+        o0[k] = cvt_e4m3x4(t0[0], t0[1], t0[2], t0[3]);
+        o1[k] = cvt_e4m3x4(t1[0], t1[1], t1[2], t1[3]);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float t0[4], t1[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) quot2(x0[4 * k + e], x1[4 * k + e], g0, g1, t0[e], t1[e]);
+        o0[k] = cvt_e4m3x4(t0[0], t0[1], t0[2], t0[3]);
+        o1[k] = cvt_e4m3x4(t1[0], t1[1], t1[2], t1[3]);
+      }
     }
     uint8_t* dst = qT + (kb * 128) * M + mb * 128;
     uint4* d0 = reinterpret_cast<uint4*>(dst + (2 * cp) * M + 32 * rq);
