@@ -934,16 +934,16 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1) rmsnorm_lane_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// 128x128 tile kernels (a2, a6, a8): persistent CTAs of 256 threads. Tiles arrive in
-// shared memory by TMA into a double buffer, so the next tile loads while this one is
-// processed; a tile's arrival is an mbarrier that thread 0 waits on with the bounded
-// wait (the CTA stops if it gives up, after letting issued copies land).
-// Row pass: thread t owns rows t/16 + 16j (j = 0..7) and the 8 columns 8*(t%16) .. +7
-// of the staged tile (a half-warp reads one 256-byte row), so each row is one 1x128
-// group. Column pass: thread t owns the column pair 2*(t%64), +1 and the 32 rows
-// 32*(t/64) .. +31; a warp reads 32 consecutive column pairs of one row per load (no
-// bank conflicts) and each thread writes 2 x 32 consecutive codes of the transposed
-// output as two 32-byte runs.
+// 128x128 tile helpers of the FP8 requantizer (a8) and of the fused dual producers:
+// persistent CTAs of 256 threads. Tiles arrive in shared memory by TMA into a double
+// buffer, so the next tile loads while this one is processed; a tile's arrival is an
+// mbarrier that thread 0 waits on with the bounded wait (the CTA stops if it gives up,
+// after letting issued copies land). Row pass: thread t owns rows t/16 + 16j (j = 0..7)
+// and the 8 columns 8*(t%16) .. +7 of the staged tile (a half-warp reads one 256-byte
+// row), so each row is one 1x128 group. Column pass: thread t owns the column pair
+// 2*(t%64), +1 and the 32 rows 32*(t/64) .. +31; a warp reads 32 consecutive column pairs
+// of one row per load (no bank conflicts) and each thread writes 2 x 32 consecutive codes
+// of the transposed output as two 32-byte runs. (a2 and a6 have kernels of their own.)
 // ---------------------------------------------------------------------------
 constexpr int kTileElems = 128 * 128;
 
@@ -1044,9 +1044,7 @@ __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, b
   }
 }
 
-// Shared memory of the BF16 tile kernels: two 32 KB tiles, the column reduction, bars.
-constexpr size_t kTileSmemBF16 = 1024 + 2 * kTileElems * 2 + 4 * 128 * 4 + 64;
-// ... of the FP8 tile kernel: two (16 KB codes + 512 B row scales) buffers.
+// Shared memory of the FP8 tile kernel (a8): two (16 KB codes + 512 B row scales) buffers.
 constexpr size_t kTileSmemFP8 = 1024 + 2 * (kTileElems + 512) + 4 * 128 * 4 + 64;
 
 __device__ __forceinline__ TileSmem carve_tiles(uint8_t* raw, int buf_bytes,
@@ -1109,67 +1107,6 @@ __device__ __forceinline__ void tiles_drain(const TileSmem& sm, int64_t t_stop, 
   }
 }
 
-// a2: 128x128 weight blocks, persistent over the ceil(N/128) x ceil(K/128) tiles. A
-// partial block at the end of a ragged N or K arrives zero-filled by the tensor copy
-// (zeros raise no maximum) and only its valid codes are stored.
-__global__ void __launch_bounds__(256) quant_weight_kernel(
-    const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t K, uint8_t* __restrict__ q,
-    float* __restrict__ s, uint8_t* __restrict__ qT, unsigned* err, uint64_t limit_ns) {
-  extern __shared__ uint8_t smem_raw[];
-  const TileSmem sm = carve_tiles(smem_raw, kTileElems * 2);
-  __shared__ int abort_flag;
-  const WaitCtl ctl{&abort_flag, err, limit_ns};
-  if (threadIdx.x == 0) abort_flag = 0;
-  const int64_t KB = (K + 127) >> 7;
-  const int64_t tiles = ((N + 127) >> 7) * KB;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int rr = tid >> 4, c8 = (tid & 15) * 8;
-  auto issue = [&](int b, int64_t t) {
-    mbar_arrive_expect_tx(sm.bar + b, kTileElems * 2);
-    tma_load_2d(sm.buf[b], &tmW, static_cast<int32_t>((t % KB) * 128),
-                static_cast<int32_t>((t / KB) * 128), sm.bar + b);
-  };
-  tiles_prologue(sm, tiles, issue);
-  int i = 0;
-  int64_t t = blockIdx.x;
-  for (; t < tiles; t += gridDim.x, ++i) {
-    if (!tile_acquire(sm, i & 1, (i >> 1) & 1, ctl)) break;
-    tiles_refill(t, tiles, i, issue);
-    const uint16_t* Ts = reinterpret_cast<const uint16_t*>(sm.buf[i & 1]);
-    const int64_t nb = t / KB, kb = t % KB;
-    uint4 raw[8];
-    float a = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      raw[j] = *reinterpret_cast<const uint4*>(Ts + (rr + 16 * j) * 128 + c8);
-      float v[8];
-      unpack_bf16x8(raw[j], v);
-      a = fmaxf(a, absmax8(v));
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
-    if (lane == 0) sm.red[wid] = a;
-    __syncthreads();
-    float amax = sm.red[0];
-#pragma unroll
-    for (int k = 1; k < 8; ++k) amax = fmaxf(amax, sm.red[k]);
-    const GroupScale g = group_scale_bf16(amax);
-    if (tid == 0) s[nb * KB + kb] = g.s;
-    const int rows = N - nb * 128 < 128 ? static_cast<int>(N - nb * 128) : 128;
-    const int cols = K - kb * 128 < 128 ? static_cast<int>(K - kb * 128) : 128;
-    uint8_t* qb = q + (nb * 128) * K + kb * 128 + c8;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float v[8];
-      unpack_bf16x8(raw[j], v);
-      const uint2 codes = codes8(v, g);  // every lane: the scale branch is warp-collective
-      if (rr + 16 * j < rows && c8 < cols) *reinterpret_cast<uint2*>(qb + (rr + 16 * j) * K) = codes;
-    }
-    if (qT)
-      tile_cols_bf16(Ts, nullptr, false, g, qT + (kb * 128) * N + nb * 128, N, nullptr, rows, cols);
-  }
-  if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
-}
 
 // ---------------------------------------------------------------------------
 // Option B for saved activations (the producer emits both groupings from BF16, no FP8
@@ -1556,25 +1493,6 @@ struct RmsBwd {
   }
 };
 
-// a6 through the direct kernel: the BF16 values themselves.
-struct GradDirect {
-  const uint16_t* dy;
-  int64_t ld;
-  static constexpr int kOut = 1;
-  static constexpr bool kHeavy = false;
-  static constexpr bool kTails = true;  // ragged M / N accepted by its entry point
-  struct In { uint4 a; };
-  struct Col {};
-  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
-  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
-    return In{ld_nc_v4(dy + m * ld + col)};
-  }
-  __device__ __forceinline__ void form(const In& in, int64_t, const Col&,
-                                       float (&v)[1][8]) const {
-    unpack_bf16x8(in.a, v[0]);
-  }
-};
-
 // Option B RMSNorm producer: y = bf16(fl32(fl32(x r) gamma)), r per row from the pre-pass.
 struct RmsDirect {
   const uint16_t* x;
@@ -1639,8 +1557,6 @@ constexpr int kBwdBatch = 2;
 constexpr int kBwdMinBlocks = 3;
 constexpr int kFwdBatch = 4;
 constexpr int kFwdMinBlocks = 4;
-constexpr int kA6Batch = 4;
-constexpr int kA6MinBlocks = 4;
 
 // Shared memory of the unit kernels: the formed BF16 output tile(s) and one column
 // reduction per output tile.
@@ -1759,7 +1675,7 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   }
 }
 
-// a6 for a BF16 gradient that is already formed (GradDirect): both groupings from one
+// a6 for a BF16 gradient that is already formed: both groupings from one
 // 128 x 128 tile staged by a tensor copy, with every group owned by one lane.
 //   warps 0-3  1x128 rows: lane l of warp w owns row 32w + l of the tile (one group),
 //              exactly as lanegroup_kernel: codes through a per-warp staging box and a
@@ -2160,6 +2076,195 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
   if (t < tiles) tiles_drain(sm, t, tiles, i, limit_ns);
 }
 
+// a2 on a tile ring. The block scale is shared by a block and its transpose, so qT is the
+// byte transpose of q: the codes are formed once, staged in shared memory, and leave twice
+// by tensor stores, the second time after an in-register 8x8 byte transpose.
+//   warps 0-7  thread t: rows t/16 + 16j (j < 8), columns 8(t%16) .. +7 of the tile (a
+//              half-warp reads one 256-byte row); the warps' maxima meet in shared memory
+//              (bounded rendezvous), every thread forms the block scale and its codes and
+//              stores them in the q staging tile; then thread t transposes the 8x8 code
+//              block (row block t%16, column block (t%16 + t/16) % 16) into the qT staging
+//              tile. Both staging tiles use the 128-byte swizzle, which with this diagonal
+//              assignment keeps the 8-byte reads and writes free of bank conflicts.
+//   warp 8     producer: tiles into a ring of kA2Stages buffers.
+// A partial block at the end of a ragged N or K arrives zero-filled (zeros raise no
+// maximum) and the tensor stores write only its valid part.
+#ifndef A2_STAGES
+#define A2_STAGES 4
+#endif
+constexpr int kA2Stages = A2_STAGES;
+constexpr uint32_t kA2Tile = 128 * 128 * 2;
+constexpr uint32_t kA2OffQ = kA2Stages * kA2Tile;     // q staging, 16 KB
+constexpr uint32_t kA2OffQT = kA2OffQ + 128 * 128;    // qT staging, 16 KB
+constexpr uint32_t kA2OffRed = kA2OffQT + 128 * 128;  // [8] warp maxima
+constexpr uint32_t kA2OffTab = kA2OffRed + 64;        // scale and reciprocal tables
+constexpr uint32_t kA2OffBar = kA2OffTab + 256 * 4;   // full[], empty[], csync
+constexpr size_t kA2Smem = 1024 + kA2OffBar + (2 * kA2Stages + 1) * 8 + 16;
+constexpr int kA2Threads = 9 * 32;
+
+// 4x4 byte transpose: word i holds row i (byte k = column k); returns word k = column k.
+__device__ __forceinline__ void transpose_4x4_bytes(uint32_t& a, uint32_t& b, uint32_t& c,
+                                                    uint32_t& d) {
+  const uint32_t t0 = __byte_perm(a, b, 0x5140), t1 = __byte_perm(a, b, 0x7362);
+  const uint32_t t2 = __byte_perm(c, d, 0x5140), t3 = __byte_perm(c, d, 0x7362);
+  a = __byte_perm(t0, t2, 0x5410);
+  b = __byte_perm(t0, t2, 0x7632);
+  c = __byte_perm(t1, t3, 0x5410);
+  d = __byte_perm(t1, t3, 0x7632);
+}
+
+// Byte offset of (row r, byte column c) in a [128][128]-byte tile with the 128-byte
+// swizzle (16-byte chunk index XOR row % 8), the layout a swizzled tensor store reads.
+__device__ __forceinline__ uint32_t sw128(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((((c >> 4) ^ r) & 7) << 4) + (c & 15));
+}
+
+__global__ void __launch_bounds__(kA2Threads, 1) a2_tile_kernel(
+    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmQ,
+    const __grid_constant__ CUtensorMap tmQT, int64_t N, int64_t K, float* __restrict__ s,
+    bool want_t, unsigned* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float* red = reinterpret_cast<float*>(base + kA2OffRed);
+  float* tab = reinterpret_cast<float*>(base + kA2OffTab);
+  uint8_t* qs = base + kA2OffQ;
+  uint8_t* qts = base + kA2OffQT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kA2OffBar);
+  uint64_t* empty = full + kA2Stages;
+  uint64_t* csync = empty + kA2Stages;  // the compute warps' rendezvous (bounded)
+  int* abort_flag = reinterpret_cast<int*>(csync + 1);
+  const WaitCtl ctl{abort_flag, err, limit_ns};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid < 128) {
+    tab[tid] = kScaleMant[tid];
+    tab[128 + tid] = kRecipMant[tid];
+  }
+  if (tid == 0) {
+    for (int b = 0; b < kA2Stages; ++b) {
+      mbar_init(full + b, 1);
+      mbar_init(empty + b, 8);
+    }
+    mbar_init(csync, 8);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int64_t KB = (K + 127) >> 7;
+  const int64_t tiles = ((N + 127) >> 7) * KB;
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0, par = 0;
+      bool ok = true;
+      int i = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int b = i % kA2Stages;
+        const uint32_t ph = static_cast<uint32_t>(i / kA2Stages) & 1u;
+        if (i >= kA2Stages && !mbar_wait(empty + b, ph ^ 1u, ctl)) { ok = false; break; }
+        const int64_t nb = t / KB, kb = t - nb * KB;
+        mbar_arrive_expect_tx(full + b, kA2Tile);
+        tma_load_2d(base + b * kA2Tile, &tmW, static_cast<int32_t>(kb * 128),
+                    static_cast<int32_t>(nb * 128), full + b);
+        issued |= 1u << b;
+        par = (par & ~(1u << b)) | (ph << b);
+      }
+      if (!ok) {  // let every copy already issued land before the CTA exits
+        for (int b = 0; b < kA2Stages; ++b) {
+          if (!((issued >> b) & 1u)) continue;
+          const uint32_t a = smem_u32(full + b);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, (par >> b) & 1u))
+            if (global_timer_ns() - t0 > limit_ns) break;
+        }
+      }
+    }
+    return;
+  }
+  uint32_t nsync = 0;
+  auto sync8 = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(csync);
+    return mbar_wait_warp(csync, (nsync++) & 1u, ctl);
+  };
+  const int rr = tid >> 4, c8 = (tid & 15) * 8;
+  const int tbr = tid & 15, tbc = ((tid & 15) + (tid >> 4)) & 15;  // transposed 8x8 block
+  bool stored = false;
+  int i = 0;
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+    const int b = i % kA2Stages;
+    if (!mbar_wait_warp(full + b, static_cast<uint32_t>(i / kA2Stages) & 1u, ctl)) break;
+    const uint16_t* Ts = reinterpret_cast<const uint16_t*>(base + b * kA2Tile);
+    uint4 raw[8];
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      raw[j] = *reinterpret_cast<const uint4*>(Ts + (rr + 16 * j) * 128 + c8);
+      m[0] = bf16x2_maxabs_xs(m[0], raw[j].x);
+      m[1] = bf16x2_maxabs_xs(m[1], raw[j].y);
+      m[2] = bf16x2_maxabs_xs(m[2], raw[j].z);
+      m[3] = bf16x2_maxabs_xs(m[3], raw[j].w);
+    }
+    float a = bf16x2_hmax_abs(bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3])));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, off));
+    if (lane == 0) {
+      red[warp] = a;
+      mbar_arrive(empty + b);  // the lanes' reads of the tile are complete (values used)
+    }
+    if (stored && tid == 0) tma_store_wait_read();  // both staging tiles are free
+    if (!sync8()) break;
+    float amax = red[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) amax = fmaxf(amax, red[k]);
+    const GroupScale g = group_scale_bf16_sm(amax, tab);
+    const int64_t nb = t / KB, kb = t - nb * KB;
+    if (tid == 0) s[nb * KB + kb] = g.s;
+    if (g.small) {  // uniform over the CTA
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint2*>(qs + sw128(rr + 16 * j, c8)) = codes8_words<true>(raw[j], g);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint2*>(qs + sw128(rr + 16 * j, c8)) = codes8_words<false>(raw[j], g);
+    }
+    fence_proxy_async_smem();
+    if (!sync8()) break;
+    if (tid == 0) {
+      tma_store_2d(&tmQ, qs, static_cast<int32_t>(kb * 128), static_cast<int32_t>(nb * 128));
+      tma_store_commit();
+    }
+    if (want_t) {
+      // rows 8 tbr .. +7, bytes 8 tbc .. +7 of q  ->  rows 8 tbc .. +7, bytes 8 tbr .. +7 of qT
+      uint32_t lo[8], hi[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const uint2 v = *reinterpret_cast<const uint2*>(qs + sw128(8 * tbr + r, 8 * tbc));
+        lo[r] = v.x;
+        hi[r] = v.y;
+      }
+      transpose_4x4_bytes(lo[0], lo[1], lo[2], lo[3]);
+      transpose_4x4_bytes(lo[4], lo[5], lo[6], lo[7]);
+      transpose_4x4_bytes(hi[0], hi[1], hi[2], hi[3]);
+      transpose_4x4_bytes(hi[4], hi[5], hi[6], hi[7]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        *reinterpret_cast<uint2*>(qts + sw128(8 * tbc + c, 8 * tbr)) = make_uint2(lo[c], lo[4 + c]);
+        *reinterpret_cast<uint2*>(qts + sw128(8 * tbc + 4 + c, 8 * tbr)) = make_uint2(hi[c], hi[4 + c]);
+      }
+      fence_proxy_async_smem();
+      if (!sync8()) break;
+      if (tid == 0) {
+        tma_store_2d(&tmQT, qts, static_cast<int32_t>(nb * 128), static_cast<int32_t>(kb * 128));
+        tma_store_commit();
+      }
+    }
+    stored = true;
+  }
+  if (stored && tid == 0) tma_store_wait_all();
+}
+
 // Resident CTAs per SM of a kernel (cached per device), for grid-stride/persistent grids.
 template <class Kernel>
 // `cache` is a per-device table owned by the caller; host threads may race to fill an
@@ -2330,16 +2435,23 @@ extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, i
   if (!aligned16(w) || !aligned16(q) || !aligned16(s) || (qT && !aligned16(qT)) || ldw % 8)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  CUtensorMap tm;
+  CUtensorMap tm, tmq, tmqt;
   if (!encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, ldw * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, K, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_UNSUPPORTED;
+  if (qT && !encode_tmap_2d(&tmqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, qT, N, K, N, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8Q_ERR_UNSUPPORTED;
+  if (!qT) tmqt = tmq;  // unused
   unsigned* err = device_error_word();
   if (!err) return FP8Q_ERR_CUDA;
   static std::atomic<int> occ[64];
-  const int per_sm = resident_ctas(quant_weight_kernel, 256, kTileSmemBF16, occ);
-  quant_weight_kernel<<<grid_for(((N + 127) / 128) * ((K + 127) / 128), per_sm), 256, kTileSmemBF16,
-                        static_cast<cudaStream_t>(stream)>>>(tm, N, K, q, s, qT, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(a2_tile_kernel, kA2Threads, kA2Smem, occ);
+  a2_tile_kernel<<<grid_for(((N + 127) / 128) * ((K + 127) / 128), per_sm), kA2Threads, kA2Smem,
+                   static_cast<cudaStream_t>(stream)>>>(tm, tmq, tmqt, N, K, s, qT != nullptr, err,
+                                                        kWaitLimitNs);
   return launch_status("quant_weight_128x128 launch");
 }
 
