@@ -284,8 +284,7 @@ __device__ __forceinline__ void swiglu2(float g0, float g1, float u0, float u1, 
 // BF16). A persistent CTA has one producer warp that keeps up to kStages units in flight
 // through a ring in shared memory, and kConsumers consumer warps, each quantizing its
 // share of the box's rows two at a time (a half-warp per row, lane l owning columns
-// 8*(l%16) .. +7), so that many warps hide the latency of the exponential and the
-// divisions (one lane per whole group, as in a1, measured 1.5x slower here). A box past
+// 8*(l%16) .. +7). The gate factor comes from a per-CTA table (see sg_index). A box past
 // a ragged M or K arrives zero-filled (zeros raise no group maximum) and only its valid
 // rows and columns are stored.
 // ---------------------------------------------------------------------------
@@ -299,21 +298,77 @@ template <int kConsumers>
 constexpr int rg_threads() { return 32 * (kConsumers + 1); }
 
 
+// The gate factor sg(g) = fl32(g / fl32(1 + E(-g))) of SwiGLU depends on the BF16 gate
+// alone, so each CTA tabulates it, with the same device arithmetic, for every BF16 g with
+// 2^-24 <= |g| < 2^7 (biased exponents 103 .. 133, both signs: 7936 values, 31 KB of
+// shared memory); a chunk with a gate outside that range computes sg directly.
+constexpr uint32_t kSgLoExp = 127 - 24;
+constexpr uint32_t kSgExps = 31;
+constexpr uint32_t kSgHalf = kSgExps * 128;  // entries per sign
+constexpr uint32_t kSgEntries = 2 * kSgHalf;
+
+// Table index of the BF16 gate with bit pattern gb, or kSgEntries when outside the table.
+__device__ __forceinline__ uint32_t sg_index(uint32_t gb) {
+  const uint32_t rel = (gb & 0x7FFFu) - (kSgLoExp << 7);  // wraps below the range
+  return rel < kSgHalf ? rel + (gb >> 15) * kSgHalf : kSgEntries;
+}
+
+// sg of two gates, the arithmetic of swiglu2 up to the product with the up value.
+__device__ __forceinline__ void sg2(float g0, float g1, float& s0, float& s1) {
+  float e0, e1;
+  exp_cw2(-g0, -g1, e0, e1);
+  s0 = __fdiv_rn(g0, __fadd_rn(1.0f, e0));
+  s1 = __fdiv_rn(g1, __fadd_rn(1.0f, e1));
+}
+
+__device__ __forceinline__ void sg_table_fill(float* tab) {
+  for (uint32_t i = threadIdx.x; i < kSgEntries / 2; i += blockDim.x) {
+    const uint32_t e0 = 2 * i, e1 = 2 * i + 1;  // entries with the same sign
+    const uint32_t sign = e0 / kSgHalf;
+    const float g0 = __uint_as_float(((sign << 15) | ((e0 - sign * kSgHalf) + (kSgLoExp << 7))) << 16);
+    const float g1 = __uint_as_float(((sign << 15) | ((e1 - sign * kSgHalf) + (kSgLoExp << 7))) << 16);
+    sg2(g0, g1, tab[e0], tab[e1]);
+  }
+}
+
 struct SwigluBoxes {  // a4: h = SwiGLU(gate, up) from the gate box and the up box
   static constexpr int kBoxes = 2;
   __device__ __forceinline__ static void values(const uint16_t* b0, const uint16_t* b1, int off,
-                                                float (&v)[8]) {
-    float g[8], u[8];
-    unpack_bf16x8(*reinterpret_cast<const uint4*>(b0 + off), g);
+                                                const float* tab, float (&v)[8]) {
+    const uint4 gw = *reinterpret_cast<const uint4*>(b0 + off);
+    float g[8], u[8], sg[8];
+    unpack_bf16x8(gw, g);
     unpack_bf16x8(*reinterpret_cast<const uint4*>(b1 + off), u);
+    const uint32_t w[4] = {gw.x, gw.y, gw.z, gw.w};
+    uint32_t idx[8];
+    bool in = true;
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[i], v[i + 1]);
+    for (int i = 0; i < 4; ++i) {
+      idx[2 * i] = sg_index(w[i] & 0xFFFFu);
+      idx[2 * i + 1] = sg_index(w[i] >> 16);
+      in = in && idx[2 * i] < kSgEntries && idx[2 * i + 1] < kSgEntries;
+    }
+    if (__all_sync(kFull, in)) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sg[i] = tab[idx[i]];
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) sg2(g[i], g[i + 1], sg[i], sg[i + 1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float m0, m1;
+      mul2(m0, m1, sg[i], sg[i + 1], u[i], u[i + 1]);
+      v[i] = round_bf16(m0);
+      v[i + 1] = round_bf16(m1);
+    }
   }
 };
 
 template <class B, int kStages>
 constexpr size_t rowgroup_tma_smem() {
-  return 1024 + static_cast<size_t>(kStages) * B::kBoxes * kRgBoxBytes + 2 * kStages * 8 + 16;
+  return 1024 + static_cast<size_t>(kStages) * B::kBoxes * kRgBoxBytes + 2 * kStages * 8 + 16 +
+         kSgEntries * 4;
 }
 
 // M rows, G = ceil(K / 128) groups of K valid columns; codes q[m * ldq + k], scales
@@ -331,6 +386,7 @@ __global__ void __launch_bounds__(rg_threads<kConsumers>()) rowgroup_tma_kernel(
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
   uint64_t* empty = full + kStages;
   int* abort_flag = reinterpret_cast<int*>(empty + kStages);
+  float* tab = reinterpret_cast<float*>(empty + kStages + 2);
   const WaitCtl ctl{abort_flag, err, limit_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -341,6 +397,7 @@ __global__ void __launch_bounds__(rg_threads<kConsumers>()) rowgroup_tma_kernel(
     *abort_flag = 0;
     fence_barrier_init();
   }
+  sg_table_fill(tab);
   __syncthreads();
   // unit u = (row box) * G + group; the host keeps the unit count below 2^31
   const uint32_t units = static_cast<uint32_t>(((M + kRgRows - 1) / kRgRows) * G);
@@ -392,7 +449,7 @@ __global__ void __launch_bounds__(rg_threads<kConsumers>()) rowgroup_tma_kernel(
     for (int step = 0; step < kRgRows / kConsumers / 2; ++step) {
       const int r = warp * (kRgRows / kConsumers) + 2 * step + half;
       float v[8];
-      B::values(b0, b1, r * 128 + sub * 8, v);
+      B::values(b0, b1, r * 128 + sub * 8, tab, v);
       uint2 codes;
       const float sc = quant_half_warp(v, codes);  // every lane takes part
       const int64_t m = m0 + r;

@@ -206,6 +206,27 @@ def test_swiglu_extreme_gates(fq, oracle_mod):
     assert_scales_equal(s, rs, "a4 extremes scales", cols=4)
 
 
+def test_swiglu_every_bf16_gate(fq, oracle_mod):
+    """Every BF16 gate value below 2^61 in magnitude (the kernel tabulates the gate factor
+    for 2^-24 <= |g| < 2^7 and computes it directly elsewhere; larger gates would make h
+    overflow), each with an up value drawn from N(0, 1); 512 rows of 128 gates, so some
+    groups mix table and direct gates and some hold only one kind."""
+    pats = np.arange(65536, dtype=np.uint32)
+    pats = pats[((pats >> 7) & 0xFF) < 127 + 61].astype(np.uint16)
+    pats = np.resize(pats, 512 * 128)  # repeats the start to fill the rows
+    rng = np.random.default_rng(5)
+    order = rng.permutation(pats.size)
+    order[: pats.size // 2] = np.sort(order[: pats.size // 2])  # half the rows in order
+    g = torch.from_numpy(pats[order].view(np.int16).reshape(512, 128).copy()).view(torch.bfloat16)
+    u = workloads.normal_bf16((512, 128), 1.0, 0, 77, "cpu")
+    gu = torch.cat([g, u], 1).contiguous()
+    q, s = fq.swiglu_quant_alloc(gu.to(DEV))
+    torch.cuda.synchronize()
+    rq, rs = oracle_mod.swiglu_quant(bits(gu))
+    assert_codes_equal(q, rq, "a4 every gate")
+    assert_scales_equal(s, rs, "a4 every gate scales", cols=512)
+
+
 # ---------------------------------------------------------------- a6
 @pytest.mark.parametrize("M,N", [(256, 512), (128, 128), (384, 256)])
 def test_transpose_quant_bf16_matches_oracle(fq, oracle_mod, M, N):
