@@ -482,10 +482,6 @@ __global__ void __launch_bounds__(rg_threads<kConsumers>()) rowgroup_tma_kernel(
 #define LG1_PER 2
 #define LG1_CONS 10
 #endif
-#ifndef RL_CONS
-#define RL_CONS 8
-#define RL_PER 2
-#endif
 constexpr int kLgRows = 32;
 constexpr uint32_t kLgBoxBytes = kLgRows * 128 * 2;  // one BF16 box
 constexpr uint32_t kLgOutBytes = kLgRows * 128;      // its codes
@@ -899,7 +895,10 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1) rmsnorm_lane_kernel(
   }
   // -------------------------------------------------------------- consumers
   uint8_t* out = outs + warp * (row_bytes / 2);
-  const int rounds = (G + 31) >> 5;
+  // lane l takes half h = l % 2 (64 values) of groups l/2, l/2 + 16, ...; chunk j of the
+  // half is read in the rotated order h*8 + (j + l/2) % 8
+  const int gl = lane >> 1, hh = lane & 1;
+  const int rounds = (G + 15) >> 4;
   bool stored = false;
   int li = 0;
   for (int64_t t = blockIdx.x + static_cast<int64_t>(warp) * gridDim.x; t < M;
@@ -909,12 +908,12 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1) rmsnorm_lane_kernel(
     const uint16_t* xr = reinterpret_cast<const uint16_t*>(ring + st * row_bytes);
     double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
     for (int k = 0; k < rounds; ++k) {
-      const int g = lane + 32 * k;
+      const int g = gl + 16 * k;
       if (g < G) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           float v[8];
-          unpack_bf16x8(*reinterpret_cast<const uint4*>(xr + g * 128 + ((j + lane) & 15) * 8), v);
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(xr + g * 128 + (hh * 8 + ((j + gl) & 7)) * 8), v);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const double d = static_cast<double>(v[e]);
@@ -933,14 +932,14 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1) rmsnorm_lane_kernel(
       __syncwarp();
     }
     for (int k = 0; k < rounds; ++k) {
-      const int g = lane + 32 * k;
+      const int g = gl + 16 * k;
       const bool act = g < G;
       const int gg = act ? g : 0;
-      uint4 y[16];
+      uint4 y[8];
       uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int off = gg * 128 + ((j + lane) & 15) * 8;
+      for (int j = 0; j < 8; ++j) {
+        const int off = gg * 128 + (hh * 8 + ((j + gl) & 7)) * 8;
         float xv[8], gv[8], b[8];
         unpack_bf16x8(*reinterpret_cast<const uint4*>(xr + off), xv);
         unpack_bf16x8(*reinterpret_cast<const uint4*>(gam + off), gv);
@@ -958,24 +957,24 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1) rmsnorm_lane_kernel(
         m[2] = bf16x2_maxabs_xs(m[2], y[j].z);
         m[3] = bf16x2_maxabs_xs(m[3], y[j].w);
       }
-      const float amax =
-          bf16x2_hmax_abs(bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3])));
-      const GroupScale gs = group_scale_bf16(amax);
+      uint32_t mh = bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3]));
+      mh = bf16x2_maxabs_xs(mh, __shfl_xor_sync(kFull, mh, 1));  // the group's other half
+      const GroupScale gs = group_scale_bf16(bf16x2_hmax_abs(mh));
       uint8_t* orow = out + gg * 128;
       if (__any_sync(kFull, gs.small)) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const uint2 c = codes8_words<true>(y[j], gs);
-          if (act) *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = c;
+          if (act) *reinterpret_cast<uint2*>(orow + (hh * 8 + ((j + gl) & 7)) * 8) = c;
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const uint2 c = codes8_words<false>(y[j], gs);
-          if (act) *reinterpret_cast<uint2*>(orow + ((j + lane) & 15) * 8) = c;
+          if (act) *reinterpret_cast<uint2*>(orow + (hh * 8 + ((j + gl) & 7)) * 8) = c;
         }
       }
-      if (act) s[static_cast<int64_t>(g) * lds + t] = gs.s;
+      if (act && hh == 0) s[static_cast<int64_t>(g) * lds + t] = gs.s;
     }
     __syncwarp();  // every lane is done with the stage and has staged its codes
     if (lane == 0) mbar_arrive(empty + st);
@@ -2340,11 +2339,13 @@ int resident_ctas(Kernel k, int threads, size_t dyn_smem, std::atomic<int>* cach
   return n;
 }
 
-// Opt a kernel in to the largest dynamic shared memory of an sm_100 CTA (once per device).
+// Opt a kernel in to the largest dynamic shared memory of an sm_100 CTA, once per device.
+// `done` is a per-device table owned by the caller, one per kernel (kernels of the same
+// signature share a function-pointer type, so a table inside this template would be
+// shared between them).
 constexpr size_t kMaxDynSmem = 232448;
 template <class Kernel>
-bool allow_max_smem(Kernel k) {
-  static std::atomic<int> done[64];
+bool allow_max_smem(Kernel k, std::atomic<int>* done) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (done[dev].load(std::memory_order_acquire)) return true;
@@ -2425,6 +2426,46 @@ extern "C" fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t 
   return launch_status("swiglu_quant launch");
 }
 
+namespace fp8q {
+namespace {
+// a3 through rmsnorm_lane_kernel<kConsumers> with `per` row stages per warp as the shared
+// memory allows; FP8Q_ERR_SHAPE (nothing launched) when not even one stage per warp fits.
+template <int kConsumers>
+fp8q_status launch_rmsnorm_lane(const uint16_t* x, const uint16_t* gamma, int64_t M, int64_t H,
+                                int64_t ldx, float eps, uint8_t* q, float* s, int64_t lds,
+                                int sms, cudaStream_t st) {
+  const int G = static_cast<int>(H / 128);
+  const size_t row_bytes = static_cast<size_t>(G) * 256;
+  const size_t fixed = 1024 + row_bytes + kConsumers * (row_bytes / 2) + 16;
+  if (fixed >= kMaxDynSmem) return FP8Q_ERR_SHAPE;
+  const int per = static_cast<int>(
+      std::min<size_t>(2, (kMaxDynSmem - fixed) / (kConsumers * (row_bytes + 16))));
+  if (per < 1) return FP8Q_ERR_SHAPE;
+  const int nst = per * kConsumers;
+  const uint64_t dx[3] = {128, static_cast<uint64_t>(G), static_cast<uint64_t>(M)};
+  const uint64_t sx[2] = {256, static_cast<uint64_t>(ldx) * 2};
+  const uint64_t sq[2] = {128, static_cast<uint64_t>(H)};
+  const uint32_t box[3] = {128, static_cast<uint32_t>(G), 1};
+  CUtensorMap tmx, tmq;
+  if (!encode_tmap_3d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, dx, sx, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_3d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, dx, sq, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  auto kern = rmsnorm_lane_kernel<kConsumers>;
+  static std::atomic<int> smem_ok[64];  // per instantiation, so per kernel
+  if (!allow_max_smem(kern, smem_ok)) return FP8Q_ERR_CUDA;
+  const size_t smem = fixed + static_cast<size_t>(nst) * (row_bytes + 16);
+  const int64_t ctas = (M + kConsumers - 1) / kConsumers;
+  kern<<<static_cast<int>(ctas < sms ? ctas : sms), 32 * (kConsumers + 1), smem, st>>>(
+      tmx, tmq, gamma, M, G, per, eps, s, lds, err, kWaitLimitNs);
+  return launch_status("rmsnorm_quant launch");
+}
+}  // namespace
+}  // namespace fp8q
+
 extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, int64_t M,
                                           int64_t H, int64_t ldx, float eps, uint8_t* q, float* s,
                                           int64_t lds, void* stream) {
@@ -2441,34 +2482,11 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   // One warp per row needs many rows to fill the GPU; up to 1024 rows one CTA per row
   // is faster (measured 3x at 16-256 rows, equal at 8192).
   if (M > 1024 && H % 128 == 0 && H <= 64 * 128) {
-    constexpr int kConsumers = RL_CONS;
-    const int G = static_cast<int>(H / 128);
-    const size_t row_bytes = static_cast<size_t>(G) * 256;
-    const size_t fixed = 1024 + row_bytes + kConsumers * (row_bytes / 2) + 16;
-    const int per = static_cast<int>(
-        std::min<size_t>(RL_PER, (kMaxDynSmem - fixed) / (kConsumers * (row_bytes + 16))));
-    const int nst = per * kConsumers;
-    if (per >= 1) {
-      const uint64_t dx[3] = {128, static_cast<uint64_t>(G), static_cast<uint64_t>(M)};
-      const uint64_t sx[2] = {256, static_cast<uint64_t>(ldx) * 2};
-      const uint64_t sq[2] = {128, static_cast<uint64_t>(H)};
-      const uint32_t box[3] = {128, static_cast<uint32_t>(G), 1};
-      CUtensorMap tmx, tmq;
-      if (!encode_tmap_3d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, dx, sx, box,
-                          CU_TENSOR_MAP_SWIZZLE_NONE) ||
-          !encode_tmap_3d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, dx, sq, box,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-        return FP8Q_ERR_UNSUPPORTED;
-      unsigned* err = device_error_word();
-      if (!err) return FP8Q_ERR_CUDA;
-      auto kern = rmsnorm_lane_kernel<kConsumers>;
-      if (!allow_max_smem(kern)) return FP8Q_ERR_CUDA;
-      const size_t smem = fixed + static_cast<size_t>(nst) * (row_bytes + 16);
-      const int64_t ctas = (M + kConsumers - 1) / kConsumers;
-      kern<<<static_cast<int>(ctas < sms ? ctas : sms), 32 * (kConsumers + 1), smem, st>>>(
-          tmx, tmq, gamma, M, G, per, eps, s, lds, err, kWaitLimitNs);
-      return launch_status("rmsnorm_quant launch");
-    }
+    // 16 consumer warps where their row stages fit in shared memory, else 8
+    const fp8q_status r16 = launch_rmsnorm_lane<16>(x, gamma, M, H, ldx, eps, q, s, lds, sms, st);
+    if (r16 != FP8Q_ERR_SHAPE) return r16;
+    const fp8q_status r8 = launch_rmsnorm_lane<8>(x, gamma, M, H, ldx, eps, q, s, lds, sms, st);
+    if (r8 != FP8Q_ERR_SHAPE) return r8;
   }
   if (M > 1024) {
     const int64_t ctas = (M + 7) / 8;  // one warp per row
