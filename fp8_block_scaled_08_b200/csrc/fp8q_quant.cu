@@ -110,6 +110,22 @@ __constant__ float kRecipMant[128] = {
     0x1.c3870ep+1f, 0x1.c1c1c4p+1f,
 };
 
+// group_scale for an arbitrary fp32 amax, with amax/448 formed as quot does (y =
+// fl32(1/448), q = fl32(amax y), q + (amax - q 448) y): the correctly rounded quotient
+// (Markstein's theorem) for amax >= 2^-60; below that, and for amax = 0, group_scale.
+__device__ __forceinline__ GroupScale group_scale_fma(float amax) {
+  if (amax < 0x1p-60f) return group_scale(amax);
+  constexpr float kY = 1.0f / 448.0f;  // fl32(1/448), rounded once by the compiler
+  const float q = __fmul_rn(amax, kY);
+  const float e = __fmaf_rn(-q, 448.0f, amax);
+  GroupScale g;
+  g.s = __fmaf_rn(e, kY, q);
+  g.rs = __frcp_rn(g.s);
+  g.ns = -g.s;
+  g.small = g.s < kSmallScale;
+  return g;
+}
+
 // Same result as group_scale for every amax that is a BF16 value (the maximum of BF16
 // values is one). amax < 2^-71 (s below about 2^-80), and non-finite amax (outside the
 // contract), take the division path; the branch is taken per warp, only when one of its
@@ -2064,13 +2080,17 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
     const int64_t mb = t / KB, kb = t % KB;
     float x0[32], x1[32];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const int row = 32 * rq + r;
-      const uint16_t two = *reinterpret_cast<const uint16_t*>(Tq + row * 128 + 2 * cp);
-      const float2 d = e4m3x2_to_f32(two);
-      const float sr = rsc[row];
-      x0[r] = __fmul_rn(sr, d.x);
-      x1[r] = __fmul_rn(sr, d.y);
+    for (int r4 = 0; r4 < 32; r4 += 4) {
+      const float4 sr4 = *reinterpret_cast<const float4*>(rsc + 32 * rq + r4);  // broadcast
+      const float sr[4] = {sr4.x, sr4.y, sr4.z, sr4.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = r4 + k;
+        const uint16_t two = *reinterpret_cast<const uint16_t*>(Tq + (32 * rq + r) * 128 + 2 * cp);
+        const float2 d = e4m3x2_to_f32(two);
+        x0[r] = __fmul_rn(sr[k], d.x);
+        x1[r] = __fmul_rn(sr[k], d.y);
+      }
     }
     float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -2087,7 +2107,7 @@ __global__ void __launch_bounds__(256) transpose_quant_fp8_kernel(
                fmaxf(sm.red[256 + 2 * cp], sm.red[384 + 2 * cp]));
     a1 = fmaxf(fmaxf(sm.red[2 * cp + 1], sm.red[128 + 2 * cp + 1]),
                fmaxf(sm.red[256 + 2 * cp + 1], sm.red[384 + 2 * cp + 1]));
-    const GroupScale g0 = group_scale(a0), g1 = group_scale(a1);
+    const GroupScale g0 = group_scale_fma(a0), g1 = group_scale_fma(a1);
     const float s0 = g0.s, s1 = g1.s;
     // a partial tile (ragged M or K) arrived zero-filled; store only its valid part
     const int rows = M - mb * 128 < 128 ? static_cast<int>(M - mb * 128) : 128;

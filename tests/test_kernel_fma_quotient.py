@@ -1,7 +1,7 @@
 """The FP8 requantizer (a8) divides arbitrary fp32 values x (a dequantized code times its
-row scale) by a column scale s >= 2^-80 with the same residual correction as the other
-quantizers: y = fl32(1/s), q = fl32(x y), t = q - fl32(q s - x) y, both steps fused
-multiply-adds. Markstein's theorem (y within half an ulp of 1/s, q within one ulp of
+row scale) by a column scale s >= 2^-80, and forms that scale s = amax / 448 for
+amax >= 2^-60, with the same residual correction as the other quantizers: y = fl32(1/s),
+q = fl32(x y), t = q - fl32(q s - x) y, both steps fused multiply-adds. Markstein's theorem (y within half an ulp of 1/s, q within one ulp of
 x/s, the residual exact) makes t the correctly rounded quotient fl32(x/s) whenever
 nothing underflows; below that the E4M3 code is a signed zero either way.
 
@@ -68,6 +68,11 @@ int main(void) {
     check(nextafterf(x, -INFINITY), s);
     check(-x, s);
   }
+  for (int i = 0; i < 4000000; ++i) {  /* the column scale amax / 448, amax >= 2^-60 */
+    float amax = (float)ldexp(1.0 + unif(), (int)(next() % 187) - 60);
+    check(amax, 448.0f);
+    check(f_of(u_of(amax) & 0xFFFF0000u), 448.0f);  /* BF16-valued amax */
+  }
   for (int k = -40; k <= 40; ++k) {  /* tiny quotients, signed zeros */
     check((float)ldexp(1.0, k - 100), 0x1p-80f);
     check(-(float)ldexp(1.0, k - 100), 0x1p-79f);
@@ -89,5 +94,5 @@ def test_fma_quotient_is_the_ieee_quotient():
                                "-lm"])
         out = subprocess.run([exe], capture_output=True, text=True, timeout=900)
         total, bad = map(int, out.stdout.split())
-        assert total > 2 * 10 ** 7
+        assert total > 3 * 10 ** 7
         assert bad == 0 and out.returncode == 0
