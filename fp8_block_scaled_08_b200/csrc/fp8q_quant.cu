@@ -114,7 +114,11 @@ __constant__ float kRecipMant[128] = {
 // fl32(1/448), q = fl32(amax y), q + (amax - q 448) y): the correctly rounded quotient
 // (Markstein's theorem) for amax >= 2^-60; below that, and for amax = 0, group_scale.
 __device__ __forceinline__ GroupScale group_scale_fma(float amax) {
-  if (amax < 0x1p-60f) return group_scale(amax);
+  if (amax < 0x1p-60f) {
+    GroupScale g = group_scale(amax);
+    g.small = g.small && amax != 0.0f;  // 0 / 1 is exact on the fast path
+    return g;
+  }
   constexpr float kY = 1.0f / 448.0f;  // fl32(1/448), rounded once by the compiler
   const float q = __fmul_rn(amax, kY);
   const float e = __fmaf_rn(-q, 448.0f, amax);
@@ -127,18 +131,21 @@ __device__ __forceinline__ GroupScale group_scale_fma(float amax) {
 }
 
 // Same result as group_scale for every amax that is a BF16 value (the maximum of BF16
-// values is one). amax < 2^-71 (s below about 2^-80), and non-finite amax (outside the
-// contract), take the division path; the branch is taken per warp, only when one of its
-// lanes needs it.
+// values is one). amax = 0 gives s = 1 directly (its codes are those of 0 / 1 = 0 on
+// the fast path too, so an all-zero group, or a lane with no group, does not send its
+// warp down the division path); 0 < amax < 2^-71 (s below about 2^-80) and non-finite
+// amax (outside the contract) take the division path; the branch is taken per warp,
+// only when one of its lanes needs it.
 __device__ __forceinline__ GroupScale group_scale_bf16(float amax) {
   const uint32_t b = __float_as_uint(amax);
   const int ebias = static_cast<int>(b >> 23);  // biased exponent (amax >= 0)
-  const bool tiny = ebias < 127 - 71 || ebias == 255;
+  const bool tiny = (ebias < 127 - 71 && b != 0) || ebias == 255;
   const int e = ebias - 127;
   const uint32_t i = (b >> 16) & 0x7Fu;
   GroupScale g;
   g.s = __uint_as_float(__float_as_uint(kScaleMant[i]) + static_cast<uint32_t>((e - 6) << 23));
   g.rs = __uint_as_float(__float_as_uint(kRecipMant[i]) + static_cast<uint32_t>((6 - e) << 23));
+  if (b == 0) g.s = g.rs = 1.0f;  // an all-zero group: s = 1, and 0 / 1 is exact either way
   g.small = false;
   if (__any_sync(kFull, tiny)) {
     if (tiny) {
@@ -1781,12 +1788,13 @@ constexpr int kA6Threads = 17 * 32;
 __device__ __forceinline__ GroupScale group_scale_bf16_sm(float amax, const float* tab) {
   const uint32_t b = __float_as_uint(amax);
   const int ebias = static_cast<int>(b >> 23);
-  const bool tiny = ebias < 127 - 71 || ebias == 255;
+  const bool tiny = (ebias < 127 - 71 && b != 0) || ebias == 255;
   const int e = ebias - 127;
   const uint32_t i = (b >> 16) & 0x7Fu;
   GroupScale g;
   g.s = __uint_as_float(__float_as_uint(tab[i]) + static_cast<uint32_t>((e - 6) << 23));
   g.rs = __uint_as_float(__float_as_uint(tab[128 + i]) + static_cast<uint32_t>((6 - e) << 23));
+  if (b == 0) g.s = g.rs = 1.0f;  // an all-zero group (see group_scale_bf16)
   g.small = false;
   if (__any_sync(kFull, tiny)) {
     if (tiny) {

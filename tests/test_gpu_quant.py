@@ -91,6 +91,41 @@ def test_special_groups(fq, oracle_mod):
     assert_scales_equal(s, rs, "special scales", cols=6)
 
 
+def test_zero_groups_in_tile_and_row_kernels(fq, oracle_mod):
+    """All-zero groups and blocks next to ordinary ones (s = 1; codes of +0 and -0) through
+    a6 (rows, columns), a2 (a zero 128x128 block) and a3 on the lane-per-group path with a
+    partial last round of groups (H = 3584: 28 groups) and a zero row."""
+    dy = workloads.gradients_bf16((256, 384), 1e-3, 0, 901, "cpu")
+    dy[:, 128:256] = 0.0                 # zero column groups and row groups
+    dy[130:140] = 0.0                    # zero rows
+    dyv = dy.view(torch.int16)
+    dyv[131, 200] = -32768               # -0.0 inside zero groups
+    dyv[5, 150] = -32768
+    q_row, s_row, q_colT, s_col = fq.transpose_quant_bf16_alloc(dy.to(DEV))
+    w = workloads.normal_bf16((256, 384), 0.02, 0, 902, "cpu")
+    w[128:, 128:256] = 0.0               # one zero block
+    w.view(torch.int16)[200, 130] = -32768
+    qw, sw, qwT = fq.quant_weight_alloc(w.to(DEV))
+    x = workloads.activations_bf16((1100, 3584), 0, 903, "cpu", outlier_frac=0.005,
+                                   outlier_scale=50.0)
+    x[17] = 0.0
+    g = workloads.gamma_bf16(3584, 0, 904, "cpu")
+    qn, sn = fq.rmsnorm_quant_alloc(x.to(DEV), g.to(DEV), 1e-5)
+    torch.cuda.synchronize()
+    rqr, rsr, rqc, rsc = oracle_mod.transpose_quant_bf16(bits(dy))
+    assert_codes_equal(q_row, rqr, "a6 row codes, zero groups")
+    assert_scales_equal(s_row, rsr, "a6 row scales, zero groups", cols=256)
+    assert_codes_equal(q_colT, rqc, "a6 column codes, zero groups")
+    assert_scales_equal(s_col, rsc, "a6 column scales, zero groups")
+    rq, rs, rqT = oracle_mod.quant_weight_128x128(bits(w))
+    assert_codes_equal(qw, rq, "a2 codes, zero block")
+    assert_codes_equal(qwT, rqT, "a2 transposed codes, zero block")
+    assert_scales_equal(sw, rs, "a2 scales, zero block")
+    rqn, rsn = oracle_mod.rmsnorm_quant(bits(x), bits(g), 1e-5)
+    assert_codes_equal(qn, rqn, "a3 codes, 28 groups")
+    assert_scales_equal(sn, rsn, "a3 scales, 28 groups", cols=1100)
+
+
 def test_quotient_dense_sweep(fq, oracle_mod):
     """Groups whose amax is a chosen BF16 value and whose other 127 elements sweep the
     BF16 values below it: the kernel's quotient path against the oracle's IEEE
