@@ -1259,6 +1259,9 @@ struct SwigluBwd {
   static constexpr int kOut = 2;
   static constexpr bool kHeavy = true;  // long form: keep the row-batch loop rolled
   static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
+  // No gate table here: its (silu, ds) pairs (36 KB) next to the two output tiles leave two CTAs
+  // per SM instead of three, which measured slower (0.50 -> 0.55 ms in the layer step).
+  static constexpr int kTab = 0;
   struct In { uint4 g, u, d; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1532,6 +1535,7 @@ struct RmsBwd {
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = false;
   static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
+  static constexpr int kTab = 0;         // floats per entry of a per-CTA gate table
   struct In { uint4 x, d, res; };
   struct Col { float g[8]; };
   __device__ __forceinline__ Col column(int64_t c) const {
@@ -1581,6 +1585,7 @@ struct RmsDirect {
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = false;
   static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
+  static constexpr int kTab = 0;         // floats per entry of a per-CTA gate table
   struct In { uint4 a; };
   struct Col { float g[8]; };
   __device__ __forceinline__ Col column(int64_t c) const {
@@ -1611,9 +1616,11 @@ struct RmsDirect {
 struct SwigluDirect {
   const uint16_t* gu;
   int64_t ldgu, I;
+  const float* tab = nullptr;  // the gate-factor table (sg_index), in shared memory
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = true;
   static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
+  static constexpr int kTab = 1;         // floats per entry of a per-CTA gate table
   struct In { uint4 g, u; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1626,8 +1633,27 @@ struct SwigluDirect {
     float g[8], u[8];
     unpack_bf16x8(in.g, g);
     unpack_bf16x8(in.u, u);
+    const uint32_t w[4] = {in.g.x, in.g.y, in.g.z, in.g.w};
+    uint32_t idx[8];
+    bool inr = true;
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[0][i], v[0][i + 1]);
+    for (int i = 0; i < 4; ++i) {
+      idx[2 * i] = sg_index(w[i] & 0xFFFFu);
+      idx[2 * i + 1] = sg_index(w[i] >> 16);
+      inr = inr && idx[2 * i] < kSgEntries && idx[2 * i + 1] < kSgEntries;
+    }
+    if (__all_sync(kFull, inr)) {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        float m0, m1;
+        mul2(m0, m1, tab[idx[i]], tab[idx[i + 1]], u[i], u[i + 1]);
+        v[0][i] = round_bf16(m0);
+        v[0][i + 1] = round_bf16(m1);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[0][i], v[0][i + 1]);
+    }
   }
 };
 
@@ -1640,8 +1666,12 @@ constexpr int kFwdMinBlocks = 4;
 // Shared memory of the unit kernels: the formed BF16 output tile(s) and one column
 // reduction per output tile.
 template <class X>
+constexpr size_t direct_table_bytes() {
+  return X::kTab == 1 ? kSgEntries * 4 : 0;
+}
+template <class X>
 constexpr size_t direct_smem_bytes() {
-  return X::kOut * (kTileElems * 2 + 4 * 128 * 4);
+  return X::kOut * (kTileElems * 2 + 4 * 128 * 4) + direct_table_bytes<X>();
 }
 
 // One 128 x 128 unit of direct_dual_kernel (described there). kEdge: the unit may reach
@@ -1739,6 +1769,13 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   constexpr int kOut = X::kOut;
   uint16_t* tile = reinterpret_cast<uint16_t*>(smem_raw);
   float* red = reinterpret_cast<float*>(smem_raw + kOut * kTileElems * 2);
+  X xs = xf;
+  if constexpr (X::kTab != 0) {  // the source's gate table, after the tiles
+    float* tab = reinterpret_cast<float*>(smem_raw + kOut * (kTileElems * 2 + 4 * 128 * 4));
+    sg_table_fill(tab);
+    xs.tab = tab;
+    __syncthreads();
+  }
   const int64_t NB = (N + 127) >> 7;
   const int64_t tiles = ((M + 127) >> 7) * NB;
   for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
@@ -1746,10 +1783,10 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
     // a unit past the end of a ragged M or N (only sources that accept one) takes the
     // checked path; whole units take the unchecked one
     if (X::kTails && (mb * 128 + 128 > M || nb * 128 + 128 > N))
-      dual_unit_edge<X, kBatch>(xf, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT, s_col,
+      dual_unit_edge<X, kBatch>(xs, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT, s_col,
                                 tile, red);
     else
-      dual_unit<X, kBatch, false>(xf, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT,
+      dual_unit<X, kBatch, false>(xs, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT,
                                   s_col, tile, red);
   }
 }

@@ -99,3 +99,22 @@ def test_wgrad_from_dual_codes(fq, oracle_mod):
     torch.cuda.synchronize()
     ref, ab = oracle_mod.linear_wgrad(np_u8(qdyT), np_f32(sdyc), np_u8(qT), np_f32(sT))
     assert_gemm_close(dw.float().cpu().numpy(), ref, ab, "wgrad from dual codes")
+
+
+def test_swiglu_dual_every_bf16_gate(fq, oracle_mod):
+    """Every BF16 gate below 2^61 in magnitude once (the kernel tabulates the gate factor
+    for 2^-24 <= |g| < 2^7 and computes it directly elsewhere), up values from N(0, 1):
+    both groupings bit for bit."""
+    pats = np.arange(65536, dtype=np.uint32)
+    pats = pats[((pats >> 7) & 0xFF) < 127 + 61].astype(np.uint16)
+    pats = np.resize(pats, 512 * 128)
+    g = torch.from_numpy(pats.view(np.int16).reshape(512, 128).copy()).view(torch.bfloat16)
+    u = workloads.normal_bf16((512, 128), 1.0, 0, 78, "cpu")
+    gu = torch.cat([g, u], 1).contiguous()
+    q, s, qT, sT = fq.swiglu_quant_dual_alloc(gu.to(DEV))
+    torch.cuda.synchronize()
+    rq, rs, rqT, rsT = oracle_mod.swiglu_quant_dual(bits(gu))
+    assert_codes_equal(q, rq, "dual every gate rows")
+    assert_scales_equal(s, rs, "dual every gate row scales", cols=512)
+    assert_codes_equal(qT, rqT, "dual every gate columns")
+    assert_scales_equal(sT, rsT, "dual every gate column scales")
