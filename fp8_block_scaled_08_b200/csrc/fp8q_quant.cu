@@ -2409,6 +2409,8 @@ int resident_ctas(Kernel k, int threads, size_t dyn_smem, std::atomic<int>* cach
 // signature share a function-pointer type, so a table inside this template would be
 // shared between them).
 constexpr size_t kMaxDynSmem = 232448;
+// Tensor-copy coordinates are signed 32-bit: the kernels fed by them take extents below this.
+constexpr int64_t kMaxTmaCoord = int64_t{1} << 31;
 template <class Kernel>
 bool allow_max_smem(Kernel k, std::atomic<int>* done) {
   int dev = 0;
@@ -2440,6 +2442,7 @@ extern "C" fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_
                                             uint8_t* q, float* s, int64_t lds, void* stream) {
   if (!x || !q || !s) return FP8Q_ERR_NULL;
   if (M <= 0 || K <= 0 || K % 16 || ldx < K || lds < M || lds % 4) return FP8Q_ERR_SHAPE;
+  if (M >= kMaxTmaCoord || K >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit tensor coordinates
   if (!aligned16(x) || !aligned16(q) || !aligned16(s) || ldx % 8) return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   const int64_t G = (K + 127) / 128;
@@ -2546,7 +2549,7 @@ extern "C" fp8q_status fp8q_rmsnorm_quant(const uint16_t* x, const uint16_t* gam
   const size_t gsm = static_cast<size_t>(H) * 2;  // gamma in shared memory
   // One warp per row needs many rows to fill the GPU; up to 1024 rows one CTA per row
   // is faster (measured 3x at 16-256 rows, equal at 8192).
-  if (M > 1024 && H % 128 == 0 && H <= 64 * 128) {
+  if (M > 1024 && M < kMaxTmaCoord && H % 128 == 0 && H <= 64 * 128) {
     // 16 consumer warps where their row stages fit in shared memory, else 8
     const fp8q_status r16 = launch_rmsnorm_lane<16>(x, gamma, M, H, ldx, eps, q, s, lds, sms, st);
     if (r16 != FP8Q_ERR_SHAPE) return r16;
@@ -2572,6 +2575,7 @@ extern "C" fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, i
                                                  void* stream) {
   if (!w || !q || !s) return FP8Q_ERR_NULL;
   if (N <= 0 || K <= 0 || N % 16 || K % 16 || ldw < K) return FP8Q_ERR_SHAPE;
+  if (N >= kMaxTmaCoord || K >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit tensor coordinates
   if (!aligned16(w) || !aligned16(q) || !aligned16(s) || (qT && !aligned16(qT)) || ldw % 8)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
@@ -2602,6 +2606,7 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
   if (!dy || !q_colT || !s_col || (q_row != nullptr) != (s_row != nullptr)) return FP8Q_ERR_NULL;
   if (M <= 0 || N <= 0 || M % 16 || N % 16 || lddy < N || (q_row && (lds_row < M || lds_row % 4)))
     return FP8Q_ERR_SHAPE;
+  if (M >= kMaxTmaCoord || N >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit tensor coordinates
   if (!aligned16(dy) || !aligned16(q_colT) || !aligned16(s_col) || lddy % 8 ||
       (q_row && (!aligned16(q_row) || !aligned16(s_row))))
     return FP8Q_ERR_ALIGN;
@@ -2639,6 +2644,7 @@ extern "C" fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s
                                                 void* stream) {
   if (!q || !s || !qT || !sT) return FP8Q_ERR_NULL;
   if (M <= 0 || K <= 0 || M % 16 || K % 16 || lds < M) return FP8Q_ERR_SHAPE;
+  if (M >= kMaxTmaCoord || K >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit tensor coordinates
   if (!aligned16(q) || !aligned16(s) || !aligned16(qT) || !aligned16(sT) || lds % 4)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;

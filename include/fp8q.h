@@ -91,7 +91,7 @@ fp8q_status fp8q_last_device_error(void* stream);
  * activations bullet).
  *   x  [M][K] BF16, row stride ldx (>= K, % 8 == 0)
  *   q  [M][K] FP8 codes (dense)        s [G(K)][lds] fp32 (1x128 layout)
- * Requires M >= 1, K % 16 == 0, ceil(M/32) * G(K) < 2^31. */
+ * Requires M >= 1, K % 16 == 0, M < 2^31, K < 2^31. */
 fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                                  uint8_t* q, float* s, int64_t lds, void* stream);
 
@@ -100,7 +100,7 @@ fp8q_status fp8q_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_
  * ("Arquitectura Central", master weights bullet).
  *   w  [N][K] BF16, row stride ldw     q [N][K] codes   s [G(N)][G(K)] fp32
  *   qT [K][N] codes: the same codes transposed (the DGrad operand); may be NULL.
- * Requires N % 16 == 0, K % 16 == 0. */
+ * Requires N % 16 == 0, K % 16 == 0, N < 2^31, K < 2^31. */
 fp8q_status fp8q_quant_weight_128x128(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
                                       uint8_t* q, float* s, uint8_t* qT, void* stream);
 
@@ -131,7 +131,7 @@ fp8q_status fp8q_swiglu_quant(const uint16_t* gu, int64_t M, int64_t I, int64_t 
  * ("Esquema de Cuantización", backward bullets; "Implementación", transposition):
  *   row-wise 1x128 for DGrad:  q_row [M][N], s_row [G(N)][lds_row]  (may be NULL)
  *   column-wise 128x1 for WGrad, stored transposed: q_colT [N][M], s_col [G(M)][N].
- *   dy [M][N] BF16, row stride lddy.  Requires M % 16 == 0, N % 16 == 0. */
+ *   dy [M][N] BF16, row stride lddy.  Requires M % 16 == 0, N % 16 == 0, M and N < 2^31. */
 fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, int64_t N,
                                       int64_t lddy, uint8_t* q_row, float* s_row,
                                       int64_t lds_row, uint8_t* q_colT, float* s_col,
@@ -217,7 +217,7 @@ fp8q_status fp8q_rmsnorm_bwd_quant_dual(const uint16_t* x, const uint16_t* gamma
 /* a8. The saved FP8 activation (1x128 groups) re-grouped 128x1 for WGrad:
  * xhat = fl32(s * dec(q)), then 128x1 quantization along M, stored transposed.
  *   q [M][K] codes, s [G(K)][lds]  ->  qT [K][M] codes, sT [G(M)][K].
- * Requires M % 16 == 0, K % 16 == 0. */
+ * Requires M % 16 == 0, K % 16 == 0, M < 2^31, K < 2^31. */
 fp8q_status fp8q_transpose_quant_fp8(const uint8_t* q, const float* s, int64_t M,
                                      int64_t K, int64_t lds, uint8_t* qT, float* sT,
                                      void* stream);
