@@ -157,6 +157,37 @@ __device__ __forceinline__ GroupScale group_scale_bf16(float amax) {
   return g;
 }
 
+// group_scale_bf16 with its tables in shared memory (tab[0..127] the scale mantissas,
+// tab[128..255] their reciprocals); same result.
+__device__ __forceinline__ GroupScale group_scale_bf16_sm(float amax, const float* tab) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ebias = static_cast<int>(b >> 23);
+  const bool tiny = (ebias < 127 - 71 && b != 0) || ebias == 255;
+  const int e = ebias - 127;
+  const uint32_t i = (b >> 16) & 0x7Fu;
+  GroupScale g;
+  g.s = __uint_as_float(__float_as_uint(tab[i]) + static_cast<uint32_t>((e - 6) << 23));
+  g.rs = __uint_as_float(__float_as_uint(tab[128 + i]) + static_cast<uint32_t>((6 - e) << 23));
+  if (b == 0) g.s = g.rs = 1.0f;  // an all-zero group (see group_scale_bf16)
+  g.small = false;
+  if (__any_sync(kFull, tiny)) {
+    if (tiny) {
+      g = group_scale(amax);
+      g.small = true;
+    }
+  }
+  g.ns = -g.s;
+  return g;
+}
+
+// Copies the two scale tables into shared memory (256 floats), for group_scale_bf16_sm.
+__device__ __forceinline__ void scale_tables_fill(float* tab) {
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    tab[i] = kScaleMant[i];
+    tab[128 + i] = kRecipMant[i];
+  }
+}
+
 // x/s for a BF16-valued x (see the file header for why this has the IEEE quotient's
 // code): q = x*r, then q - (q*s - x)*r. Written this way the sign of x = -0 survives
 // without a separate copy-sign (q*s - x is +0 and q - (+0)*r is -0 + -0).
@@ -1078,7 +1109,8 @@ template <int kThreads = 256>
 __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, bool per_col,
                                                const GroupScale& blk, uint8_t* __restrict__ dst,
                                                int64_t ldd, float* __restrict__ scol,
-                                               int rows = 128, int cols = 128) {
+                                               const float* tab, int rows = 128,
+                                               int cols = 128) {
   constexpr int kQ = kThreads / 64, kR = 128 / kQ;
   static_assert(kQ * 64 == kThreads && kR % 16 == 0, "column pass: 256 or 512 threads");
   const int tid = threadIdx.x;
@@ -1102,8 +1134,8 @@ __device__ __forceinline__ void tile_cols_bf16(const uint16_t* Ts, float* red, b
       c0 = fmaxf(c0, red[q * 128 + 2 * cp]);
       c1 = fmaxf(c1, red[q * 128 + 2 * cp + 1]);
     }
-    g0 = group_scale_bf16(c0);
-    g1 = group_scale_bf16(c1);
+    g0 = group_scale_bf16_sm(c0, tab);  // 32 different entries per warp: shared memory
+    g1 = group_scale_bf16_sm(c1, tab);
     if (rq == 0 && scol && 2 * cp < cols)
       *reinterpret_cast<float2*>(scol + 2 * cp) = make_float2(g0.s, g1.s);
   }
@@ -1671,7 +1703,7 @@ constexpr size_t direct_table_bytes() {
 }
 template <class X>
 constexpr size_t direct_smem_bytes() {
-  return X::kOut * (kTileElems * 2 + 4 * 128 * 4) + direct_table_bytes<X>();
+  return X::kOut * (kTileElems * 2 + 4 * 128 * 4) + 256 * 4 + direct_table_bytes<X>();
 }
 
 // One 128 x 128 unit of direct_dual_kernel (described there). kEdge: the unit may reach
@@ -1681,7 +1713,8 @@ __device__ __forceinline__ void dual_unit(const X& xf, int64_t mb, int64_t nb, i
                                           uint16_t* __restrict__ bf16_out,
                                           uint8_t* __restrict__ q_row, float* __restrict__ s_row,
                                           int64_t lds_row, uint8_t* __restrict__ q_colT,
-                                          float* __restrict__ s_col, uint16_t* tile, float* red) {
+                                          float* __restrict__ s_col, uint16_t* tile, float* red,
+                                          const float* stab) {
   constexpr int kOut = X::kOut;
   const int64_t Nout = kOut * N;
   const int tid = threadIdx.x;
@@ -1735,7 +1768,8 @@ __device__ __forceinline__ void dual_unit(const X& xf, int64_t mb, int64_t nb, i
     for (int o = 0; o < kOut; ++o) {
       const int64_t oc0 = o * N + nb * 128;
       tile_cols_bf16<256>(tile + o * kTileElems, red + o * 4 * 128, true, unused,
-                          q_colT + oc0 * M + mb * 128, M, s_col + mb * Nout + oc0, rows, cols);
+                          q_colT + oc0 * M + mb * 128, M, s_col + mb * Nout + oc0, stab, rows,
+                          cols);
     }
   }
 }
@@ -1746,9 +1780,10 @@ template <class X, int kBatch>
 __device__ __noinline__ void dual_unit_edge(const X& xf, int64_t mb, int64_t nb, int64_t M,
                                             int64_t N, uint16_t* bf16_out, uint8_t* q_row,
                                             float* s_row, int64_t lds_row, uint8_t* q_colT,
-                                            float* s_col, uint16_t* tile, float* red) {
+                                            float* s_col, uint16_t* tile, float* red,
+                                            const float* stab) {
   dual_unit<X, kBatch, true>(xf, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT, s_col,
-                             tile, red);
+                             tile, red, stab);
 }
 
 // Persistent over the ceil(M/128) x NB units (NB = ceil(N/128)); unit t covers rows
@@ -1769,13 +1804,16 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   constexpr int kOut = X::kOut;
   uint16_t* tile = reinterpret_cast<uint16_t*>(smem_raw);
   float* red = reinterpret_cast<float*>(smem_raw + kOut * kTileElems * 2);
+  // the scale tables, then the source's gate table, after the tiles
+  float* stab = reinterpret_cast<float*>(smem_raw + kOut * (kTileElems * 2 + 4 * 128 * 4));
+  scale_tables_fill(stab);
   X xs = xf;
-  if constexpr (X::kTab != 0) {  // the source's gate table, after the tiles
-    float* tab = reinterpret_cast<float*>(smem_raw + kOut * (kTileElems * 2 + 4 * 128 * 4));
+  if constexpr (X::kTab != 0) {
+    float* tab = stab + 256;
     sg_table_fill(tab);
     xs.tab = tab;
-    __syncthreads();
   }
+  __syncthreads();
   const int64_t NB = (N + 127) >> 7;
   const int64_t tiles = ((M + 127) >> 7) * NB;
   for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
@@ -1784,10 +1822,10 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
     // checked path; whole units take the unchecked one
     if (X::kTails && (mb * 128 + 128 > M || nb * 128 + 128 > N))
       dual_unit_edge<X, kBatch>(xs, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT, s_col,
-                                tile, red);
+                                tile, red, stab);
     else
       dual_unit<X, kBatch, false>(xs, mb, nb, M, N, bf16_out, q_row, s_row, lds_row, q_colT,
-                                  s_col, tile, red);
+                                  s_col, tile, red, stab);
   }
 }
 
@@ -1819,29 +1857,6 @@ constexpr uint32_t kA6OffTab = kA6OffRed + 4 * 64 * 4;   // scale and reciprocal
 constexpr uint32_t kA6OffBar = kA6OffTab + 256 * 4;      // full[], empty[], csync
 constexpr size_t kA6Smem = 1024 + kA6OffBar + (2 * kA6Stages + 1) * 8 + 16;
 constexpr int kA6Threads = 17 * 32;
-
-// group_scale_bf16 with its tables in shared memory (tab[0..127] the scale mantissas,
-// tab[128..255] their reciprocals); same result.
-__device__ __forceinline__ GroupScale group_scale_bf16_sm(float amax, const float* tab) {
-  const uint32_t b = __float_as_uint(amax);
-  const int ebias = static_cast<int>(b >> 23);
-  const bool tiny = (ebias < 127 - 71 && b != 0) || ebias == 255;
-  const int e = ebias - 127;
-  const uint32_t i = (b >> 16) & 0x7Fu;
-  GroupScale g;
-  g.s = __uint_as_float(__float_as_uint(tab[i]) + static_cast<uint32_t>((e - 6) << 23));
-  g.rs = __uint_as_float(__float_as_uint(tab[128 + i]) + static_cast<uint32_t>((6 - e) << 23));
-  if (b == 0) g.s = g.rs = 1.0f;  // an all-zero group (see group_scale_bf16)
-  g.small = false;
-  if (__any_sync(kFull, tiny)) {
-    if (tiny) {
-      g = group_scale(amax);
-      g.small = true;
-    }
-  }
-  g.ns = -g.s;
-  return g;
-}
 
 template <bool kRows>
 __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
