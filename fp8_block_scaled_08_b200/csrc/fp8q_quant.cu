@@ -319,19 +319,6 @@ __device__ __forceinline__ void exp_cw2(float x0, float x1, float& e0, float& e1
   mul2(e0, e1, c0, c1, s0, s1);
 }
 
-// h = bf16( fl32( fl32(g / fl32(1 + E(-g))) * u ) ), two at a time.
-__device__ __forceinline__ void swiglu2(float g0, float g1, float u0, float u1, float& h0,
-                                        float& h1) {
-  float e0, e1;
-  exp_cw2(-g0, -g1, e0, e1);
-  const float d0 = __fadd_rn(1.0f, e0), d1 = __fadd_rn(1.0f, e1);
-  const float s0 = __fdiv_rn(g0, d0), s1 = __fdiv_rn(g1, d1);
-  float m0, m1;
-  mul2(m0, m1, s0, s1, u0, u1);
-  h0 = round_bf16(m0);
-  h1 = round_bf16(m1);
-}
-
 // ---------------------------------------------------------------------------
 // Row-group quantizer of SwiGLU (a4), fed by tensor copies. A unit is a box of kRgRows
 // rows x one 128-column group of the gate and the same of the up half (2 x 16 KB of
@@ -367,7 +354,7 @@ __device__ __forceinline__ uint32_t sg_index(uint32_t gb) {
   return rel < kSgHalf ? rel + (gb >> 15) * kSgHalf : kSgEntries;
 }
 
-// sg of two gates, the arithmetic of swiglu2 up to the product with the up value.
+// sg(g) = fl32(g / fl32(1 + E(-g))) of two gates; h = bf16(fl32(sg(g) u)) then follows.
 __device__ __forceinline__ void sg2(float g0, float g1, float& s0, float& s1) {
   float e0, e1;
   exp_cw2(-g0, -g1, e0, e1);
@@ -1221,9 +1208,10 @@ __device__ __forceinline__ void tiles_drain(const TileSmem& sm, int64_t t_stop, 
 
 // ---------------------------------------------------------------------------
 // Option B for saved activations (the producer emits both groupings from BF16, no FP8
-// requantization): the producer's BF16 output is formed 128 x 128 tile by tile by
-// direct_dual_kernel below, with RmsDirect / SwigluDirect as the source; the RMSNorm
-// needs its per-row reciprocal RMS first.
+// requantization): the producer's BF16 output is formed 128 x 128 tile by tile inside
+// a6_tile_kernel, with TileRms / TileSwiglu as the source (the row warps form the tile in
+// shared memory, then both groupings are quantized from it); the RMSNorm needs its
+// per-row reciprocal RMS first.
 // ---------------------------------------------------------------------------
 
 // Per-row reciprocal RMS, r = (float)(1/sqrt(ss/H + eps)) with the fp64 sum of squares
@@ -1293,7 +1281,6 @@ struct SwigluBwd {
   static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
   // No gate table here: its (silu, ds) pairs (36 KB) next to the two output tiles leave two CTAs
   // per SM instead of three, which measured slower (0.50 -> 0.55 ms in the layer step).
-  static constexpr int kTab = 0;
   struct In { uint4 g, u, d; };
   struct Col {};
   __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
@@ -1567,7 +1554,6 @@ struct RmsBwd {
   static constexpr int kOut = 1;
   static constexpr bool kHeavy = false;
   static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
-  static constexpr int kTab = 0;         // floats per entry of a per-CTA gate table
   struct In { uint4 x, d, res; };
   struct Col { float g[8]; };
   __device__ __forceinline__ Col column(int64_t c) const {
@@ -1608,102 +1594,15 @@ struct RmsBwd {
   }
 };
 
-// Option B RMSNorm producer: y = bf16(fl32(fl32(x r) gamma)), r per row from the pre-pass.
-struct RmsDirect {
-  const uint16_t* x;
-  int64_t ldx;
-  const float* rstd;
-  const uint16_t* gamma;
-  static constexpr int kOut = 1;
-  static constexpr bool kHeavy = false;
-  static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
-  static constexpr int kTab = 0;         // floats per entry of a per-CTA gate table
-  struct In { uint4 a; };
-  struct Col { float g[8]; };
-  __device__ __forceinline__ Col column(int64_t c) const {
-    Col k;
-    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + c)), k.g);
-    return k;
-  }
-  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
-    return In{ld_nc_v4(x + m * ldx + col)};
-  }
-  __device__ __forceinline__ void form(const In& in, int64_t m, const Col& k,
-                                       float (&v)[1][8]) const {
-    float xv[8];
-    unpack_bf16x8(in.a, xv);
-    const float r = __ldg(rstd + m);
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      float a0, a1, b0, b1;
-      mul2(a0, a1, xv[i], xv[i + 1], r, r);
-      mul2(b0, b1, a0, a1, k.g[i], k.g[i + 1]);
-      v[0][i] = round_bf16(b0);
-      v[0][i + 1] = round_bf16(b1);
-    }
-  }
-};
-
-// Option B SwiGLU producer: h = SwiGLU(gate, up) in BF16 (gate columns c, up I + c).
-struct SwigluDirect {
-  const uint16_t* gu;
-  int64_t ldgu, I;
-  const float* tab = nullptr;  // the gate-factor table (sg_index), in shared memory
-  static constexpr int kOut = 1;
-  static constexpr bool kHeavy = true;
-  static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
-  static constexpr int kTab = 1;         // floats per entry of a per-CTA gate table
-  struct In { uint4 g, u; };
-  struct Col {};
-  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
-  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
-    const uint16_t* row = gu + m * ldgu;
-    return In{ld_nc_v4(row + col), ld_nc_v4(row + I + col)};
-  }
-  __device__ __forceinline__ void form(const In& in, int64_t, const Col&,
-                                       float (&v)[1][8]) const {
-    float g[8], u[8];
-    unpack_bf16x8(in.g, g);
-    unpack_bf16x8(in.u, u);
-    const uint32_t w[4] = {in.g.x, in.g.y, in.g.z, in.g.w};
-    uint32_t idx[8];
-    bool inr = true;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      idx[2 * i] = sg_index(w[i] & 0xFFFFu);
-      idx[2 * i + 1] = sg_index(w[i] >> 16);
-      inr = inr && idx[2 * i] < kSgEntries && idx[2 * i + 1] < kSgEntries;
-    }
-    if (__all_sync(kFull, inr)) {
-#pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        float m0, m1;
-        mul2(m0, m1, tab[idx[i]], tab[idx[i + 1]], u[i], u[i + 1]);
-        v[0][i] = round_bf16(m0);
-        v[0][i + 1] = round_bf16(m1);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; i += 2) swiglu2(g[i], g[i + 1], u[i], u[i + 1], v[0][i], v[0][i + 1]);
-    }
-  }
-};
-
 // Rows loaded per batch and the occupancy the backward kernels are compiled for.
 constexpr int kBwdBatch = 2;
 constexpr int kBwdMinBlocks = 3;
-constexpr int kFwdBatch = 4;
-constexpr int kFwdMinBlocks = 4;
 
 // Shared memory of the unit kernels: the formed BF16 output tile(s) and one column
 // reduction per output tile.
 template <class X>
-constexpr size_t direct_table_bytes() {
-  return X::kTab == 1 ? kSgEntries * 4 : 0;
-}
-template <class X>
 constexpr size_t direct_smem_bytes() {
-  return X::kOut * (kTileElems * 2 + 4 * 128 * 4) + 256 * 4 + direct_table_bytes<X>();
+  return X::kOut * (kTileElems * 2 + 4 * 128 * 4) + 256 * 4;
 }
 
 // One 128 x 128 unit of direct_dual_kernel (described there). kEdge: the unit may reach
@@ -1804,15 +1703,10 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   constexpr int kOut = X::kOut;
   uint16_t* tile = reinterpret_cast<uint16_t*>(smem_raw);
   float* red = reinterpret_cast<float*>(smem_raw + kOut * kTileElems * 2);
-  // the scale tables, then the source's gate table, after the tiles
+  // the scale tables, after the tiles
   float* stab = reinterpret_cast<float*>(smem_raw + kOut * (kTileElems * 2 + 4 * 128 * 4));
   scale_tables_fill(stab);
-  X xs = xf;
-  if constexpr (X::kTab != 0) {
-    float* tab = stab + 256;
-    sg_table_fill(tab);
-    xs.tab = tab;
-  }
+  const X& xs = xf;
   __syncthreads();
   const int64_t NB = (N + 127) >> 7;
   const int64_t tiles = ((M + 127) >> 7) * NB;
@@ -1854,33 +1748,91 @@ constexpr uint32_t kA6OffCol = kA6Stages * kA6Tile;      // transposed codes, 16
 constexpr uint32_t kA6OffRow = kA6OffCol + 128 * 128;    // 4 x (32 x 128) row codes
 constexpr uint32_t kA6OffRed = kA6OffRow + 128 * 128;    // [4][64] partial maxima
 constexpr uint32_t kA6OffTab = kA6OffRed + 4 * 64 * 4;   // scale and reciprocal tables
-constexpr uint32_t kA6OffBar = kA6OffTab + 256 * 4;      // full[], empty[], csync
-constexpr size_t kA6Smem = 1024 + kA6OffBar + (2 * kA6Stages + 1) * 8 + 16;
+constexpr uint32_t kA6OffBar = kA6OffTab + 256 * 4;      // full[], empty[], formed[], csync
+constexpr uint32_t kA6OffGateTab = kA6OffBar + (3 * kA6Stages + 1) * 8 + 16;  // SwiGLU gate table
+template <class Src>
+constexpr size_t a6_smem() {
+  return 1024 + kA6OffGateTab + (Src::kTable ? kSgEntries * 4 : 0);
+}
 constexpr int kA6Threads = 17 * 32;
 
-template <bool kRows>
+// Sources of the tile kernel. kBoxes tensor copies per tile (the ring then holds
+// kA6Stages / kBoxes tiles); with kForm the row warps form the BF16 value from them and
+// write it over box 0, where the column warps read it once all eight row warps are done.
+struct TileGrad {  // a6: the BF16 gradient itself (no forming step)
+  static constexpr int kBoxes = 1;
+  static constexpr bool kForm = false;
+  static constexpr bool kTable = false;
+};
+
+struct TileRms {  // option B, RMSNorm: y = bf16(fl32(fl32(x r) g)), r from the pre-pass
+  const float* rstd;
+  const uint16_t* gamma;
+  static constexpr int kBoxes = 1;
+  static constexpr bool kForm = true;
+  static constexpr bool kTable = false;
+  __device__ __forceinline__ float row_factor(int64_t m) const { return __ldg(rstd + m); }
+  // 8 values at x0 (staged), output columns col .. col + 7
+  __device__ __forceinline__ uint4 form(const uint16_t* x0, const uint16_t*, int64_t col, float r,
+                                        const float*) const {
+    float xv[8], gv[8], b[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(x0), xv);
+    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + col)), gv);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float a0, a1;
+      mul2(a0, a1, xv[i], xv[i + 1], r, r);
+      mul2(b[i], b[i + 1], a0, a1, gv[i], gv[i + 1]);
+    }
+    return make_uint4(pack_bf16x2(b[0], b[1]), pack_bf16x2(b[2], b[3]), pack_bf16x2(b[4], b[5]),
+                      pack_bf16x2(b[6], b[7]));
+  }
+};
+
+struct TileSwiglu {  // option B, SwiGLU: h = bf16(fl32(sg(g) u)), gate and up staged
+  static constexpr int kBoxes = 2;
+  static constexpr bool kForm = true;
+  static constexpr bool kTable = true;
+  __device__ __forceinline__ float row_factor(int64_t) const { return 0.0f; }
+  __device__ __forceinline__ uint4 form(const uint16_t* g0, const uint16_t* u0, int64_t, float,
+                                        const float* tab) const {
+    float v[8];
+    SwigluBoxes::values(g0, u0, 0, tab, v);
+    return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                      pack_bf16x2(v[6], v[7]));
+  }
+};
+
+template <class Src, bool kRows>
 __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
-    const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmQ,
-    const __grid_constant__ CUtensorMap tmQT, int64_t M, int64_t N, float* __restrict__ s_row,
-    int64_t lds_row, float* __restrict__ s_col, unsigned* err, uint64_t limit_ns) {
+    const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD1,
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQT, Src src,
+    int64_t M, int64_t N, float* __restrict__ s_row, int64_t lds_row, float* __restrict__ s_col,
+    unsigned* err, uint64_t limit_ns) {
+  constexpr int kStages = kA6Stages / Src::kBoxes;
+  constexpr uint32_t kStageBytes = Src::kBoxes * kA6Tile;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   float* tab = reinterpret_cast<float*>(base + kA6OffTab);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kA6OffBar);
   uint64_t* empty = full + kA6Stages;
-  uint64_t* csync = empty + kA6Stages;  // the column warps' rendezvous (bounded, unlike bar.sync)
+  uint64_t* formed = empty + kA6Stages;  // kForm: the eight row warps have written the tile
+  uint64_t* csync = formed + kA6Stages;  // the column warps' rendezvous (bounded, unlike bar.sync)
   int* abort_flag = reinterpret_cast<int*>(csync + 1);
+  float* gtab = reinterpret_cast<float*>(base + kA6OffGateTab);  // Src::kTable
   const WaitCtl ctl{abort_flag, err, limit_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < 128) {
     tab[threadIdx.x] = kScaleMant[threadIdx.x];
     tab[128 + threadIdx.x] = kRecipMant[threadIdx.x];
   }
+  if (Src::kTable) sg_table_fill(gtab);
   if (threadIdx.x == 0) {
-    for (int b = 0; b < kA6Stages; ++b) {
+    for (int b = 0; b < kStages; ++b) {
       mbar_init(full + b, 1);
       mbar_init(empty + b, 16);
+      mbar_init(formed + b, 8);
     }
     mbar_init(csync, 8);
     *abort_flag = 0;
@@ -1896,18 +1848,21 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
       bool ok = true;
       int i = 0;
       for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
-        const int b = i % kA6Stages;
-        const uint32_t ph = static_cast<uint32_t>(i / kA6Stages) & 1u;
-        if (i >= kA6Stages && !mbar_wait(empty + b, ph ^ 1u, ctl)) { ok = false; break; }
+        const int b = i % kStages;
+        const uint32_t ph = static_cast<uint32_t>(i / kStages) & 1u;
+        if (i >= kStages && !mbar_wait(empty + b, ph ^ 1u, ctl)) { ok = false; break; }
         const int64_t mb = t / NB, nb = t - mb * NB;
-        mbar_arrive_expect_tx(full + b, kA6Tile);
-        tma_load_2d(base + b * kA6Tile, &tmD, static_cast<int32_t>(nb * 128),
+        mbar_arrive_expect_tx(full + b, kStageBytes);
+        tma_load_2d(base + b * kStageBytes, &tmD, static_cast<int32_t>(nb * 128),
                     static_cast<int32_t>(mb * 128), full + b);
+        if (Src::kBoxes == 2)
+          tma_load_2d(base + b * kStageBytes + kA6Tile, &tmD1, static_cast<int32_t>(nb * 128),
+                      static_cast<int32_t>(mb * 128), full + b);
         issued |= 1u << b;
         par = (par & ~(1u << b)) | (ph << b);
       }
       if (!ok) {  // let every copy already issued land before the CTA exits
-        for (int b = 0; b < kA6Stages; ++b) {
+        for (int b = 0; b < kStages; ++b) {
           if (!((issued >> b) & 1u)) continue;
           const uint32_t a = smem_u32(full + b);
           const uint64_t t0 = global_timer_ns();
@@ -1926,16 +1881,34 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
     const int rl = lane & 15, hh = lane >> 4;
     int i = 0;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
-      const int b = i % kA6Stages;
-      if (!mbar_wait_warp(full + b, static_cast<uint32_t>(i / kA6Stages) & 1u, ctl)) break;
-      if (!kRows) {
+      const int b = i % kStages;
+      if (!mbar_wait_warp(full + b, static_cast<uint32_t>(i / kStages) & 1u, ctl)) break;
+      if (!kRows && !Src::kForm) {
         if (lane == 0) mbar_arrive(empty + b);
         continue;
       }
-      const uint16_t* row = reinterpret_cast<const uint16_t*>(base + b * kA6Tile) + (warp * 16 + rl) * 128 + hh * 64;
+      const int64_t mb = t / NB, nb = t - mb * NB;
+      const int roff = (warp * 16 + rl) * 128 + hh * 64;
+      uint16_t* row = reinterpret_cast<uint16_t*>(base + b * kStageBytes) + roff;
       uint4 w[8];
+      if constexpr (Src::kForm) {
+        // form the value from the staged inputs and write it over box 0 (same rotated
+        // order as the reads: no bank conflicts)
+        const uint16_t* row1 = reinterpret_cast<const uint16_t*>(base + b * kStageBytes + kA6Tile) + roff;
+        const float rf = src.row_factor(mb * 128 + warp * 16 + rl);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) w[j] = *reinterpret_cast<const uint4*>(row + ((j + lane) & 7) * 8);
+        for (int j = 0; j < 8; ++j) {
+          const int off = ((j + lane) & 7) * 8;
+          w[j] = src.form(row + off, row1 + off, nb * 128 + hh * 64 + off, rf, gtab);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(row + ((j + lane) & 7) * 8) = w[j];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(formed + b);  // release: the column warps may read it
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = *reinterpret_cast<const uint4*>(row + ((j + lane) & 7) * 8);
+      }
       uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -1949,8 +1922,8 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
       const float amax = bf16x2_hmax_abs(mh);
       __syncwarp();  // every lane's reads of the tile are complete (their values are used)
       if (lane == 0) mbar_arrive(empty + b);
+      if (!kRows) continue;
       const GroupScale g = group_scale_bf16_sm(amax, tab);
-      const int64_t mb = t / NB, nb = t - mb * NB;
       if (stored) {
         if (lane == 0) tma_store_wait_read();
         __syncwarp();
@@ -1992,9 +1965,11 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
     };
     int i = 0;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
-      const int b = i % kA6Stages;
-      if (!mbar_wait_warp(full + b, static_cast<uint32_t>(i / kA6Stages) & 1u, ctl)) break;
-      const uint32_t* tw = reinterpret_cast<const uint32_t*>(base + b * kA6Tile) + q4 * 32 * 64 + (c0 >> 1);
+      const int b = i % kStages;
+      if (!mbar_wait_warp(Src::kForm ? formed + b : full + b,
+                          static_cast<uint32_t>(i / kStages) & 1u, ctl))
+        break;
+      const uint32_t* tw = reinterpret_cast<const uint32_t*>(base + b * kStageBytes) + q4 * 32 * 64 + (c0 >> 1);
       uint32_t w[32];  // columns c0, c0 + 1 of rows 32 q4 + k
 #pragma unroll
       for (int k = 0; k < 32; ++k) w[k] = tw[k * 64];
@@ -2640,16 +2615,17 @@ extern "C" fp8q_status fp8q_transpose_quant_bf16(const uint16_t* dy, int64_t M, 
   if (!err) return FP8Q_ERR_CUDA;
   const int64_t tiles = ((M + 127) / 128) * ((N + 127) / 128);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  constexpr size_t kSmem = a6_smem<TileGrad>();
   if (q_row) {
     static std::atomic<int> occ[64];
-    const int per_sm = resident_ctas(a6_tile_kernel<true>, kA6Threads, kA6Smem, occ);
-    a6_tile_kernel<true><<<grid_for(tiles, per_sm), kA6Threads, kA6Smem, st>>>(
-        tmd, tmq, tmqt, M, N, s_row, lds_row, s_col, err, kWaitLimitNs);
+    const int per_sm = resident_ctas(a6_tile_kernel<TileGrad, true>, kA6Threads, kSmem, occ);
+    a6_tile_kernel<TileGrad, true><<<grid_for(tiles, per_sm), kA6Threads, kSmem, st>>>(
+        tmd, tmd, tmq, tmqt, TileGrad{}, M, N, s_row, lds_row, s_col, err, kWaitLimitNs);
   } else {
     static std::atomic<int> occ[64];
-    const int per_sm = resident_ctas(a6_tile_kernel<false>, kA6Threads, kA6Smem, occ);
-    a6_tile_kernel<false><<<grid_for(tiles, per_sm), kA6Threads, kA6Smem, st>>>(
-        tmd, tmq, tmqt, M, N, s_row, lds_row, s_col, err, kWaitLimitNs);
+    const int per_sm = resident_ctas(a6_tile_kernel<TileGrad, false>, kA6Threads, kSmem, occ);
+    a6_tile_kernel<TileGrad, false><<<grid_for(tiles, per_sm), kA6Threads, kSmem, st>>>(
+        tmd, tmd, tmq, tmqt, TileGrad{}, M, N, s_row, lds_row, s_col, err, kWaitLimitNs);
   }
   return launch_status("transpose_quant_bf16 launch");
 }
@@ -2697,15 +2673,26 @@ extern "C" fp8q_status fp8q_rmsnorm_quant_dual(const uint16_t* x, const uint16_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the reciprocal RMS of every row first (one warp per row), then the tiles
   const int64_t rstd_ctas = std::min<int64_t>((M + 7) / 8, static_cast<int64_t>(sms) * 8);
+  if (M >= kMaxTmaCoord || H >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit coordinates
+  CUtensorMap tmx, tmq, tmqt;
+  if (!encode_tmap_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, ldx * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_row, H, M, H, 128, 16,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_colT, M, H, M, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
   rmsnorm_rstd_kernel<<<static_cast<int>(rstd_ctas), 256, 0, st>>>(x, M, H, ldx, eps, rstd);
   const fp8q_status s1 = launch_status("rmsnorm_rstd launch");
   if (s1 != FP8Q_OK) return s1;
-  constexpr size_t kSmem = direct_smem_bytes<RmsDirect>();
-  auto kern = direct_dual_kernel<RmsDirect, kFwdBatch, kFwdMinBlocks>;
+  constexpr size_t kSmem = a6_smem<TileRms>();
+  auto kern = a6_tile_kernel<TileRms, true>;
   static std::atomic<int> occ[64];
-  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
-  kern<<<grid_for((M / 128) * (H / 128), per_sm), 256, kSmem, st>>>(
-      RmsDirect{x, ldx, rstd, gamma}, M, H, nullptr, q_row, s_row, lds_row, q_colT, s_col);
+  const int per_sm = resident_ctas(kern, kA6Threads, kSmem, occ);
+  kern<<<grid_for((M / 128) * (H / 128), per_sm), kA6Threads, kSmem, st>>>(
+      tmx, tmx, tmq, tmqt, TileRms{rstd, gamma}, M, H, s_row, lds_row, s_col, err, kWaitLimitNs);
   return launch_status("rmsnorm_quant_dual launch");
 }
 
@@ -2720,12 +2707,26 @@ extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int
       !aligned16(s_col) || ldgu % 8)
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  constexpr size_t kSmem = direct_smem_bytes<SwigluDirect>();
-  auto kern = direct_dual_kernel<SwigluDirect, kBwdBatch, kBwdMinBlocks>;
+  if (M >= kMaxTmaCoord || I >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit coordinates
+  // the gate and the up halves as two [M][I] tensors
+  CUtensorMap tmg, tmu, tmq, tmqt;
+  if (!encode_tmap_2d(&tmg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu, I, M, ldgu * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu + I, I, M, ldgu * 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_row, I, M, I, 128, 16,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_colT, M, I, M, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  constexpr size_t kSmem = a6_smem<TileSwiglu>();
+  auto kern = a6_tile_kernel<TileSwiglu, true>;
   static std::atomic<int> occ[64];
-  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
-  kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      SwigluDirect{gu, ldgu, I}, M, I, nullptr, q_row, s_row, lds_row, q_colT, s_col);
+  const int per_sm = resident_ctas(kern, kA6Threads, kSmem, occ);
+  kern<<<grid_for((M / 128) * (I / 128), per_sm), kA6Threads, kSmem, static_cast<cudaStream_t>(stream)>>>(
+      tmg, tmu, tmq, tmqt, TileSwiglu{}, M, I, s_row, lds_row, s_col, err, kWaitLimitNs);
   return launch_status("swiglu_quant_dual launch");
 }
 
