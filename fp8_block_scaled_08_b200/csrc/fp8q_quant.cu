@@ -1271,60 +1271,103 @@ __global__ void __launch_bounds__(256) rmsnorm_rstd_kernel(const uint16_t* __res
 // silu as in the forward producer):
 //   e = E(-g), d = 1 + e, silu = g / d, sig = 1 / d,
 //   d_up = bf16(dh silu), d_gate = bf16((dh u) (sig (1 + g (1 - sig)))).
-// A thread's chunk: 8 consecutive gate, up and dh values of one row.
-struct SwigluBwd {
-  const uint16_t* gu;
-  const uint16_t* dh;
-  int64_t I;
-  static constexpr int kOut = 2;
-  static constexpr bool kHeavy = true;  // long form: keep the row-batch loop rolled
-  static constexpr bool kTails = false;  // ragged M / N accepted by its entry point
-  // No gate table here: its (silu, ds) pairs (36 KB) next to the two output tiles leave two CTAs
-  // per SM instead of three, which measured slower (0.50 -> 0.55 ms in the layer step).
-  struct In { uint4 g, u, d; };
-  struct Col {};
-  __device__ __forceinline__ Col column(int64_t) const { return Col{}; }
-  __device__ __forceinline__ In load(int64_t m, int64_t col) const {
-    const uint16_t* row = gu + m * 2 * I;
-    return In{ld_nc_v4(row + col), ld_nc_v4(row + I + col), ld_nc_v4(dh + m * I + col)};
+// silu and ds = sig (1 + g (1 - sig)) depend on the gate alone; sgb2 computes them for
+// two gates.
+__device__ __forceinline__ void sgb2(float g0, float g1, float& silu0, float& silu1, float& ds0,
+                                     float& ds1) {
+  float e0, e1;
+  exp_cw2(-g0, -g1, e0, e1);
+  const float d0 = __fadd_rn(1.0f, e0), d1 = __fadd_rn(1.0f, e1);
+  const float sig0 = __frcp_rn(d0), sig1 = __frcp_rn(d1);
+  // silu = g / d from sig = RN(1/d): q = g sig, t = q d - g, silu = q - t sig. For every
+  // BF16 g (d = fl32(1 + E(-g))) this equals the IEEE quotient, signed zeros included
+  // (exhaustive proof in the CPU tests); it replaces a second division.
+  float q0, q1, t0 = -g0, t1 = -g1;
+  mul2(q0, q1, g0, g1, sig0, sig1);
+  fma2(t0, t1, q0, q1, d0, d1);
+  silu0 = q0;
+  silu1 = q1;
+  fma2(silu0, silu1, t0, t1, -sig0, -sig1);
+  const float t10 = __fsub_rn(1.0f, sig0), t11 = __fsub_rn(1.0f, sig1);
+  float t20, t21;
+  mul2(t20, t21, g0, g1, t10, t11);
+  const float t30 = __fadd_rn(1.0f, t20), t31 = __fadd_rn(1.0f, t21);
+  mul2(ds0, ds1, sig0, sig1, t30, t31);
+}
+
+// The products with dh and u for two columns, rounded to BF16.
+__device__ __forceinline__ void swiglu_bwd_out2(float dh0, float dh1, float u0, float u1,
+                                                float silu0, float silu1, float ds0, float ds1,
+                                                float& dg0, float& dg1, float& du0, float& du1) {
+  float a0, a1, b0, b1, c0, c1;
+  mul2(a0, a1, dh0, dh1, silu0, silu1);
+  mul2(b0, b1, dh0, dh1, u0, u1);
+  mul2(c0, c1, b0, b1, ds0, ds1);
+  dg0 = round_bf16(c0);
+  dg1 = round_bf16(c1);
+  du0 = round_bf16(a0);
+  du1 = round_bf16(a1);
+}
+
+// A chunk: 8 consecutive gate, up and dh values of one row; v[0] receives d_gate, v[1]
+// d_up.
+__device__ __forceinline__ void swiglu_bwd8(const uint4& gw, const uint4& uw, const uint4& dw,
+                                            float (&v)[2][8]) {
+  float g[8], u[8], dh[8];
+  unpack_bf16x8(gw, g);
+  unpack_bf16x8(uw, u);
+  unpack_bf16x8(dw, dh);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    float s0, s1, d0, d1;
+    sgb2(g[i], g[i + 1], s0, s1, d0, d1);
+    swiglu_bwd_out2(dh[i], dh[i + 1], u[i], u[i + 1], s0, s1, d0, d1, v[0][i], v[0][i + 1],
+                    v[1][i], v[1][i + 1]);
   }
-  __device__ __forceinline__ void form(const In& in, int64_t /*m*/, const Col&,
-                                       float (&v)[2][8]) const {
-    float g[8], u[8], dh[8];
-    unpack_bf16x8(in.g, g);
-    unpack_bf16x8(in.u, u);
-    unpack_bf16x8(in.d, dh);
+}
+
+// The (silu, ds) pair of every BF16 gate in the table range of sg_index (62 KB), with
+// the arithmetic of sgb2.
+__device__ __forceinline__ void sgb_table_fill(float2* tab) {
+  for (uint32_t i = threadIdx.x; i < kSgEntries / 2; i += blockDim.x) {
+    const uint32_t e0 = 2 * i, e1 = 2 * i + 1;  // entries with the same sign
+    const uint32_t sign = e0 / kSgHalf;
+    const float g0 = __uint_as_float(((sign << 15) | ((e0 - sign * kSgHalf) + (kSgLoExp << 7))) << 16);
+    const float g1 = __uint_as_float(((sign << 15) | ((e1 - sign * kSgHalf) + (kSgLoExp << 7))) << 16);
+    float s0, s1, d0, d1;
+    sgb2(g0, g1, s0, s1, d0, d1);
+    tab[e0] = make_float2(s0, d0);
+    tab[e1] = make_float2(s1, d1);
+  }
+}
+
+// swiglu_bwd8 with silu and ds looked up in the table when every gate of the warp's
+// chunks lies in its range (computed otherwise).
+__device__ __forceinline__ void swiglu_bwd8_tab(const uint4& gw, const uint4& uw, const uint4& dw,
+                                                const float2* tab, float (&v)[2][8]) {
+  const uint32_t w[4] = {gw.x, gw.y, gw.z, gw.w};
+  uint32_t idx[8];
+  bool in = true;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    idx[2 * i] = sg_index(w[i] & 0xFFFFu);
+    idx[2 * i + 1] = sg_index(w[i] >> 16);
+    in = in && idx[2 * i] < kSgEntries && idx[2 * i + 1] < kSgEntries;
+  }
+  if (__all_sync(kFull, in)) {
+    float u[8], dh[8];
+    unpack_bf16x8(uw, u);
+    unpack_bf16x8(dw, dh);
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-      float e0, e1;
-      exp_cw2(-g[i], -g[i + 1], e0, e1);
-      const float d0 = __fadd_rn(1.0f, e0), d1 = __fadd_rn(1.0f, e1);
-      const float sig0 = __frcp_rn(d0), sig1 = __frcp_rn(d1);
-      // silu = g / d from sig = RN(1/d): q = g sig, t = q d - g, silu = q - t sig. For every
-      // BF16 g (d = fl32(1 + E(-g))) this equals the IEEE quotient, signed zeros included
-      // (exhaustive proof in the CPU tests); it replaces a second division.
-      float q0, q1, t0 = -g[i], t1 = -g[i + 1];
-      mul2(q0, q1, g[i], g[i + 1], sig0, sig1);
-      fma2(t0, t1, q0, q1, d0, d1);
-      float silu0 = q0, silu1 = q1;
-      fma2(silu0, silu1, t0, t1, -sig0, -sig1);
-      float du0, du1, dhu0, dhu1;
-      mul2(du0, du1, dh[i], dh[i + 1], silu0, silu1);
-      mul2(dhu0, dhu1, dh[i], dh[i + 1], u[i], u[i + 1]);
-      const float t10 = __fsub_rn(1.0f, sig0), t11 = __fsub_rn(1.0f, sig1);
-      float t20, t21;
-      mul2(t20, t21, g[i], g[i + 1], t10, t11);
-      const float t30 = __fadd_rn(1.0f, t20), t31 = __fadd_rn(1.0f, t21);
-      float ds0, ds1, dg0, dg1;
-      mul2(ds0, ds1, sig0, sig1, t30, t31);
-      mul2(dg0, dg1, dhu0, dhu1, ds0, ds1);
-      v[0][i] = round_bf16(dg0);
-      v[0][i + 1] = round_bf16(dg1);
-      v[1][i] = round_bf16(du0);
-      v[1][i + 1] = round_bf16(du1);
+      const float2 t0 = tab[idx[i]], t1 = tab[idx[i + 1]];
+      swiglu_bwd_out2(dh[i], dh[i + 1], u[i], u[i + 1], t0.x, t1.x, t0.y, t1.y, v[0][i],
+                      v[0][i + 1], v[1][i], v[1][i + 1]);
     }
+  } else {
+    swiglu_bwd8(gw, uw, dw, v);
   }
-};
+}
 
 // ---------------------------------------------------------------------------
 // Exact sums of fp32 terms (the two reductions of the RMSNorm backward). A finite fp32
@@ -1723,38 +1766,46 @@ __global__ void __launch_bounds__(256, kMinBlocks) direct_dual_kernel(
   }
 }
 
-// a6 for a BF16 gradient that is already formed: both groupings from one
-// 128 x 128 tile staged by a tensor copy, with every group owned by one lane.
-//   warps 0-3  1x128 rows: lane l of warp w owns row 32w + l of the tile (one group),
-//              exactly as lanegroup_kernel: codes through a per-warp staging box and a
-//              tensor store, one coalesced scale store per warp.
-//   warps 4-11 128x1 columns: warp 4 + 4h + q reads rows 32q .. 32q+31 of the column
+// a6 for a BF16 gradient that is already formed, and the producers that form their BF16
+// value from staged inputs (option B's RMSNorm and SwiGLU, the SwiGLU backward): both
+// groupings from one 128 x 128 tile staged by tensor copies, persistent CTAs of 17 warps.
+//   warps 0-7  1x128 rows: lane l of warp w holds half of row 16w + (l % 16) of the tile
+//              (columns 64 (l / 16) .. +63; the halves meet by one shuffle). A forming
+//              source has these warps form their rows from the staged inputs first and
+//              write them over the first box(es). Codes leave through a per-warp staging
+//              box and a tensor store, one scale store per row.
+//   warps 8-15 128x1 columns: warp 8 + 4h + q reads rows 32q .. 32q+31 of the column
 //              pairs 64h + (2l, 2l+1), l the lane (one 4-byte word per row and lane, 128
 //              consecutive bytes per warp load). Partial maxima of the four row quarters
 //              meet in shared memory; every lane then forms the scales of its two columns
 //              and quantizes its 2 columns x 32 rows into a transposed [128 columns][128
 //              rows] staging tile (128-byte swizzle, 2-way bank conflicts at most), which
 //              one tensor store writes to q_colT.
-//   warp 12    producer: tiles into a ring of kA6Stages buffers (one CTA per SM keeps
-//              up to 3 tiles = 96 KB in flight while it works on the fourth).
+//   warp 16    producer: tiles into a ring of stages of kBoxes boxes each.
 // The scale tables sit in shared memory here: the column scales look up 32 different
 // entries per warp load, which the constant cache would serve one at a time.
 #ifndef A6_STAGES
 #define A6_STAGES 4
 #endif
-constexpr int kA6Stages = A6_STAGES;
+constexpr int kA6Stages = A6_STAGES;  // boxes in the ring of a one- or two-box source
 constexpr uint32_t kA6Tile = 128 * 128 * 2;
-constexpr uint32_t kA6OffCol = kA6Stages * kA6Tile;      // transposed codes, 16 KB
-constexpr uint32_t kA6OffRow = kA6OffCol + 128 * 128;    // 4 x (32 x 128) row codes
-constexpr uint32_t kA6OffRed = kA6OffRow + 128 * 128;    // [4][64] partial maxima
-constexpr uint32_t kA6OffTab = kA6OffRed + 4 * 64 * 4;   // scale and reciprocal tables
-constexpr uint32_t kA6OffBar = kA6OffTab + 256 * 4;      // full[], empty[], formed[], csync
-constexpr uint32_t kA6OffGateTab = kA6OffBar + (3 * kA6Stages + 1) * 8 + 16;  // SwiGLU gate table
+constexpr int kA6Threads = 17 * 32;
+template <class Src>
+struct A6Layout {
+  static constexpr int kStages = kA6Stages / Src::kBoxes;
+  static constexpr uint32_t kStageBytes = Src::kBoxes * kA6Tile;
+  static constexpr uint32_t kOffCol = kStages * kStageBytes;  // transposed codes, 16 KB
+  static constexpr uint32_t kOffRow = kOffCol + 128 * 128;    // 8 x (16 x 128) row codes
+  static constexpr uint32_t kOffRed = kOffRow + 128 * 128;    // [4][64] partial maxima
+  static constexpr uint32_t kOffTab = kOffRed + 4 * 64 * 4;  // scale and reciprocal tables
+  static constexpr uint32_t kOffBar = kOffTab + 256 * 4;     // full, empty, formed, csync
+  static constexpr uint32_t kOffGateTab = kOffBar + (3 * kStages + 1) * 8 + 16;
+  static constexpr size_t kSmem = 1024 + kOffGateTab + (Src::kTable ? kSgEntries * 4 : 0);
+};
 template <class Src>
 constexpr size_t a6_smem() {
-  return 1024 + kA6OffGateTab + (Src::kTable ? kSgEntries * 4 : 0);
+  return A6Layout<Src>::kSmem;
 }
-constexpr int kA6Threads = 17 * 32;
 
 // Sources of the tile kernel. kBoxes tensor copies per tile (the ring then holds
 // kA6Stages / kBoxes tiles); with kForm the row warps form the BF16 value from them and
@@ -1803,24 +1854,59 @@ struct TileSwiglu {  // option B, SwiGLU: h = bf16(fl32(sg(g) u)), gate and up s
   }
 };
 
+// Group maximum from a lane's four running bf16x2 maxima and its partner's (lane ^ 16).
+__device__ __forceinline__ float half_row_amax_finish(const uint32_t (&m)[4]) {
+  uint32_t mh = bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3]));
+  mh = bf16x2_maxabs_xs(mh, __shfl_xor_sync(kFull, mh, 16));
+  return bf16x2_hmax_abs(mh);
+}
+
+// Group maximum of a lane's 64 values w and its partner's.
+__device__ __forceinline__ float half_row_amax(const uint4 (&w)[8]) {
+  uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    m[0] = bf16x2_maxabs_xs(m[0], w[j].x);
+    m[1] = bf16x2_maxabs_xs(m[1], w[j].y);
+    m[2] = bf16x2_maxabs_xs(m[2], w[j].z);
+    m[3] = bf16x2_maxabs_xs(m[3], w[j].w);
+  }
+  return half_row_amax_finish(m);
+}
+
+// A lane's 64 codes of w (scale g) at orow, chunk j at position (j + lane) % 8.
+__device__ __forceinline__ void half_row_codes(const uint4 (&w)[8], const GroupScale& g,
+                                               uint8_t* orow, int lane) {
+  if (__any_sync(kFull, g.small)) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint2*>(orow + ((j + lane) & 7) * 8) = codes8_words<true>(w[j], g);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint2*>(orow + ((j + lane) & 7) * 8) = codes8_words<false>(w[j], g);
+  }
+}
+
 template <class Src, bool kRows>
 __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
     const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD1,
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQT, Src src,
     int64_t M, int64_t N, float* __restrict__ s_row, int64_t lds_row, float* __restrict__ s_col,
     unsigned* err, uint64_t limit_ns) {
-  constexpr int kStages = kA6Stages / Src::kBoxes;
-  constexpr uint32_t kStageBytes = Src::kBoxes * kA6Tile;
+  using L = A6Layout<Src>;
+  constexpr int kStages = L::kStages;
+  constexpr uint32_t kStageBytes = L::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* tab = reinterpret_cast<float*>(base + kA6OffTab);
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + kA6OffBar);
-  uint64_t* empty = full + kA6Stages;
-  uint64_t* formed = empty + kA6Stages;  // kForm: the eight row warps have written the tile
-  uint64_t* csync = formed + kA6Stages;  // the column warps' rendezvous (bounded, unlike bar.sync)
+  float* tab = reinterpret_cast<float*>(base + L::kOffTab);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + L::kOffBar);
+  uint64_t* empty = full + kStages;
+  uint64_t* formed = empty + kStages;  // kForm: the eight row warps have written the tile
+  uint64_t* csync = formed + kStages;  // the column warps' rendezvous (bounded, unlike bar.sync)
   int* abort_flag = reinterpret_cast<int*>(csync + 1);
-  float* gtab = reinterpret_cast<float*>(base + kA6OffGateTab);  // Src::kTable
+  float* gtab = reinterpret_cast<float*>(base + L::kOffGateTab);  // Src::kTable
   const WaitCtl ctl{abort_flag, err, limit_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < 128) {
@@ -1877,7 +1963,7 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
   if (warp < 8) {
     // ------------------------------------------------------------ 1x128 rows
     // lane l of warp w: row 16w + (l % 16) of the tile, chunks 8 (l / 16) .. + 7 of it
-    uint8_t* out = base + kA6OffRow + warp * (16 * 128);
+    uint8_t* out = base + L::kOffRow + warp * (16 * 128);
     const int rl = lane & 15, hh = lane >> 4;
     int i = 0;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
@@ -1909,17 +1995,7 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
 #pragma unroll
         for (int j = 0; j < 8; ++j) w[j] = *reinterpret_cast<const uint4*>(row + ((j + lane) & 7) * 8);
       }
-      uint32_t m[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        m[0] = bf16x2_maxabs_xs(m[0], w[j].x);
-        m[1] = bf16x2_maxabs_xs(m[1], w[j].y);
-        m[2] = bf16x2_maxabs_xs(m[2], w[j].z);
-        m[3] = bf16x2_maxabs_xs(m[3], w[j].w);
-      }
-      uint32_t mh = bf16x2_maxabs_xs(bf16x2_maxabs_xs(m[0], m[1]), bf16x2_maxabs_xs(m[2], m[3]));
-      mh = bf16x2_maxabs_xs(mh, __shfl_xor_sync(kFull, mh, 16));  // the row's other half
-      const float amax = bf16x2_hmax_abs(mh);
+      const float amax = half_row_amax(w);
       __syncwarp();  // every lane's reads of the tile are complete (their values are used)
       if (lane == 0) mbar_arrive(empty + b);
       if (!kRows) continue;
@@ -1928,16 +2004,7 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
         if (lane == 0) tma_store_wait_read();
         __syncwarp();
       }
-      uint8_t* orow = out + rl * 128 + hh * 64;
-      if (__any_sync(kFull, g.small)) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint2*>(orow + ((j + lane) & 7) * 8) = codes8_words<true>(w[j], g);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint2*>(orow + ((j + lane) & 7) * 8) = codes8_words<false>(w[j], g);
-      }
+      half_row_codes(w, g, out + rl * 128 + hh * 64, lane);
       fence_proxy_async_smem();
       __syncwarp();
       const int64_t m0 = mb * 128 + warp * 16;
@@ -1953,8 +2020,8 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
     const int cw = warp - 8;
     const int q4 = cw & 3;                // row quarter: rows 32 q4 .. 32 q4 + 31
     const int c0 = 64 * (cw >> 2) + 2 * lane;  // this lane's column pair c0, c0 + 1
-    uint32_t* red = reinterpret_cast<uint32_t*>(base + kA6OffRed);
-    uint8_t* colst = base + kA6OffCol;
+    uint32_t* red = reinterpret_cast<uint32_t*>(base + L::kOffRed);
+    uint8_t* colst = base + L::kOffCol;
     // The eight column warps meet twice a tile: each warp's lanes finish their shared-
     // memory writes, lane 0 arrives, and the warp waits (bounded) for the phase.
     uint32_t nsync = 0;
@@ -2017,6 +2084,259 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
         tma_store_commit();
       }
       stored = true;
+    }
+  }
+  if (stored && lane == 0) tma_store_wait_all();
+}
+
+// ---------------------------------------------------------------------------
+// SwiGLU backward with both groupings of [d_gate | d_up] (f1), on the tile layout: a
+// stage holds the 128 x 128 gate and up boxes of one tile (64 KB, two stages); dh comes
+// straight from HBM into registers, the next tile's while this one is quantized. All
+// sixteen consumer warps first form eight rows each (lane l: row 8w + l / 4, the four
+// 8-column chunks (l % 4) + 4k, rotated by the row so that no two lanes of a shared-
+// memory phase meet in a bank), with silu and ds from a per-CTA table of every BF16
+// gate in range, write d_gate over the gate box and d_up over the up box, take the row
+// maxima by two shuffles and store their rows' codes (and the BF16 gradient) from
+// registers: four lanes cover a row's 128 codes, so every store fills whole sectors.
+// Once all rows are formed, warps 0-7 quantize d_gate's columns and warps 8-15 d_up's,
+// as the column warps of a6_tile_kernel do, staging the transposed codes over the first
+// half of the box they read (each group meets on its own bounded barrier after its
+// reads). Warp 16 is the producer.
+// ---------------------------------------------------------------------------
+constexpr int kSbStages = 2;
+constexpr uint32_t kSbStageBytes = 2 * kA6Tile;                // gate and up boxes
+constexpr uint32_t kSbOffGate = kSbStages * kSbStageBytes;     // (silu, ds) per gate
+constexpr uint32_t kSbOffRed = kSbOffGate + kSgEntries * 8;    // [2 outputs][4][64] maxima
+constexpr uint32_t kSbOffTab = kSbOffRed + 2 * 4 * 64 * 4;     // scale and reciprocal tables
+constexpr uint32_t kSbOffBar = kSbOffTab + 256 * 4;            // full, empty, formed, csync[2]
+constexpr size_t kSbSmem = 1024 + kSbOffBar + (3 * kSbStages + 2) * 8 + 16;
+
+__global__ void __launch_bounds__(kA6Threads, 1) swiglu_bwd_tile_kernel(
+    const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmU,
+    const __grid_constant__ CUtensorMap tmQT, const uint16_t* __restrict__ dh,
+    uint16_t* __restrict__ dgu, uint8_t* __restrict__ q_row, int64_t M, int64_t I,
+    float* __restrict__ s_row, int64_t lds_row, float* __restrict__ s_col, unsigned* err,
+    uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const float2* gtab = reinterpret_cast<const float2*>(base + kSbOffGate);
+  float* tab = reinterpret_cast<float*>(base + kSbOffTab);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kSbOffBar);
+  uint64_t* empty = full + kSbStages;
+  uint64_t* formed = empty + kSbStages;  // all sixteen warps have formed their rows
+  uint64_t* csync = formed + kSbStages;  // [2]: each column group's rendezvous
+  int* abort_flag = reinterpret_cast<int*>(csync + 2);
+  const WaitCtl ctl{abort_flag, err, limit_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < 128) {
+    tab[threadIdx.x] = kScaleMant[threadIdx.x];
+    tab[128 + threadIdx.x] = kRecipMant[threadIdx.x];
+  }
+  sgb_table_fill(reinterpret_cast<float2*>(base + kSbOffGate));
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < kSbStages; ++b) {
+      mbar_init(full + b, 1);
+      mbar_init(empty + b, 16);
+      mbar_init(formed + b, 16);
+    }
+    mbar_init(csync, 8);
+    mbar_init(csync + 1, 8);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int64_t NB = I >> 7;
+  const int64_t tiles = (M >> 7) * NB;
+  if (warp == 16) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0, par = 0;
+      bool ok = true;
+      int i = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int b = i % kSbStages;
+        const uint32_t ph = static_cast<uint32_t>(i / kSbStages) & 1u;
+        if (i >= kSbStages && !mbar_wait(empty + b, ph ^ 1u, ctl)) { ok = false; break; }
+        const int64_t mb = t / NB, nb = t - mb * NB;
+        const int32_t x = static_cast<int32_t>(nb * 128), y = static_cast<int32_t>(mb * 128);
+        uint8_t* st = base + b * kSbStageBytes;
+        mbar_arrive_expect_tx(full + b, kSbStageBytes);
+        tma_load_2d(st, &tmG, x, y, full + b);
+        tma_load_2d(st + kA6Tile, &tmU, x, y, full + b);
+        issued |= 1u << b;
+        par = (par & ~(1u << b)) | (ph << b);
+      }
+      if (!ok) {  // let every copy already issued land before the CTA exits
+        for (int b = 0; b < kSbStages; ++b) {
+          if (!((issued >> b) & 1u)) continue;
+          const uint32_t a = smem_u32(full + b);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, (par >> b) & 1u))
+            if (global_timer_ns() - t0 > limit_ns) break;
+        }
+      }
+    }
+    return;
+  }
+  // row phase: tile row r = 8 warp + lr, chunks (a + 4k + 4 (lr % 4)) % 16, k = 0 .. 3
+  const int lr = lane >> 2, a = lane & 3;
+  const int r = warp * 8 + lr;
+  // column phase: output grp, row quarter q4, column pair c0, c0 + 1
+  const int grp = warp >> 3, cw = warp & 7, q4 = cw & 3;
+  const int c0 = 64 * (cw >> 2) + 2 * lane;
+  uint32_t* red = reinterpret_cast<uint32_t*>(base + kSbOffRed) + grp * 256;
+  uint32_t nsync = 0;
+  auto col_sync = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(csync + grp);
+    return mbar_wait_warp(csync + grp, (nsync++) & 1u, ctl);
+  };
+  auto chunk = [&](int k) { return (a + 4 * k + 4 * (lr & 3)) & 15; };
+  // this lane's dh chunks of tile t
+  uint4 dcur[4];
+  auto load_dh = [&](int64_t t) {
+    const int64_t mb = t / NB, nb = t - mb * NB;
+    const uint16_t* row = dh + (mb * 128 + r) * I + nb * 128;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dcur[k] = ld_nc_v4(row + chunk(k) * 8);
+  };
+  if (static_cast<int64_t>(blockIdx.x) < tiles) load_dh(blockIdx.x);
+  bool stored = false;
+  int i = 0;
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+    const int b = i % kSbStages;
+    const uint32_t ph = static_cast<uint32_t>(i / kSbStages) & 1u;
+    if (!mbar_wait_warp(full + b, ph, ctl)) break;
+    const int64_t mb = t / NB, nb = t - mb * NB;
+    uint8_t* st = base + b * kSbStageBytes;
+    // ---------------------------------------------------------------- rows
+    {
+      uint16_t* rg = reinterpret_cast<uint16_t*>(st) + r * 128;
+      uint16_t* ru = reinterpret_cast<uint16_t*>(st + kA6Tile) + r * 128;
+      uint32_t ma[4] = {0u, 0u, 0u, 0u}, mu[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int off = chunk(k) * 8;
+        float v[2][8];
+        swiglu_bwd8_tab(*reinterpret_cast<const uint4*>(rg + off),
+                        *reinterpret_cast<const uint4*>(ru + off), dcur[k], gtab, v);
+        const uint4 dg = make_uint4(pack_bf16x2(v[0][0], v[0][1]), pack_bf16x2(v[0][2], v[0][3]),
+                                    pack_bf16x2(v[0][4], v[0][5]), pack_bf16x2(v[0][6], v[0][7]));
+        const uint4 du = make_uint4(pack_bf16x2(v[1][0], v[1][1]), pack_bf16x2(v[1][2], v[1][3]),
+                                    pack_bf16x2(v[1][4], v[1][5]), pack_bf16x2(v[1][6], v[1][7]));
+        *reinterpret_cast<uint4*>(rg + off) = dg;
+        *reinterpret_cast<uint4*>(ru + off) = du;
+        ma[0] = bf16x2_maxabs_xs(ma[0], dg.x);
+        ma[1] = bf16x2_maxabs_xs(ma[1], dg.y);
+        ma[2] = bf16x2_maxabs_xs(ma[2], dg.z);
+        ma[3] = bf16x2_maxabs_xs(ma[3], dg.w);
+        mu[0] = bf16x2_maxabs_xs(mu[0], du.x);
+        mu[1] = bf16x2_maxabs_xs(mu[1], du.y);
+        mu[2] = bf16x2_maxabs_xs(mu[2], du.z);
+        mu[3] = bf16x2_maxabs_xs(mu[3], du.w);
+      }
+      // the next tile's dh while this one is quantized
+      if (t + gridDim.x < tiles) load_dh(t + gridDim.x);
+      // the row's four lanes are adjacent: two shuffles give its maximum
+      uint32_t hg = bf16x2_maxabs_xs(bf16x2_maxabs_xs(ma[0], ma[1]), bf16x2_maxabs_xs(ma[2], ma[3]));
+      uint32_t hu = bf16x2_maxabs_xs(bf16x2_maxabs_xs(mu[0], mu[1]), bf16x2_maxabs_xs(mu[2], mu[3]));
+      hg = bf16x2_maxabs_xs(hg, __shfl_xor_sync(kFull, hg, 1));
+      hu = bf16x2_maxabs_xs(hu, __shfl_xor_sync(kFull, hu, 1));
+      hg = bf16x2_maxabs_xs(hg, __shfl_xor_sync(kFull, hg, 2));
+      hu = bf16x2_maxabs_xs(hu, __shfl_xor_sync(kFull, hu, 2));
+      const GroupScale g0 = group_scale_bf16_sm(bf16x2_hmax_abs(hg), tab);
+      const GroupScale g1 = group_scale_bf16_sm(bf16x2_hmax_abs(hu), tab);
+      const int64_t m = mb * 128 + r;
+      uint8_t* qr = q_row + m * 2 * I + nb * 128;
+      uint16_t* br = dgu ? dgu + m * 2 * I + nb * 128 : nullptr;
+      const bool small = __any_sync(kFull, g0.small || g1.small);
+      // the codes from the formed values (this lane's own writes) before the rows are
+      // released: the column groups stage their codes over these boxes afterwards
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = chunk(k) * 8;
+        const uint4 dg = *reinterpret_cast<const uint4*>(rg + c);
+        const uint4 du = *reinterpret_cast<const uint4*>(ru + c);
+        uint2 q0, q1;
+        if (small) {
+          q0 = codes8_words<true>(dg, g0);
+          q1 = codes8_words<true>(du, g1);
+        } else {
+          q0 = codes8_words<false>(dg, g0);
+          q1 = codes8_words<false>(du, g1);
+        }
+        *reinterpret_cast<uint2*>(qr + c) = q0;
+        *reinterpret_cast<uint2*>(qr + I + c) = q1;
+        if (br) {
+          *reinterpret_cast<uint4*>(br + c) = dg;
+          *reinterpret_cast<uint4*>(br + I + c) = du;
+        }
+      }
+      if (a == 0) {
+        s_row[nb * lds_row + m] = g0.s;
+        s_row[(NB + nb) * lds_row + m] = g1.s;
+      }
+      fence_proxy_async_smem();  // the stage is refilled by tensor copies later
+      __syncwarp();
+      if (lane == 0) mbar_arrive(formed + b);  // release: the column warps may read the rows
+    }
+    if (!mbar_wait_warp(formed + b, ph, ctl)) break;
+    // ---------------------------------------------------------------- columns of output grp
+    {
+      uint8_t* box = st + grp * kA6Tile;
+      const uint32_t* tw = reinterpret_cast<const uint32_t*>(box) + q4 * 32 * 64 + (c0 >> 1);
+      uint32_t w[32];  // columns c0, c0 + 1 of rows 32 q4 + k
+#pragma unroll
+      for (int k = 0; k < 32; ++k) w[k] = tw[k * 64];
+      uint32_t m0 = 0u, m1 = 0u;
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        m0 = bf16x2_maxabs_xs(m0, w[k]);
+        m1 = bf16x2_maxabs_xs(m1, w[k + 1]);
+      }
+      red[q4 * 64 + (c0 >> 1)] = bf16x2_maxabs_xs(m0, m1);
+      if (stored && cw == 0 && lane == 0) tma_store_wait_read();  // (earlier stages' stores)
+      if (!col_sync()) break;  // the group's reads of the box are done: it may be overwritten
+      uint32_t mm = 0u;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mm = bf16x2_maxabs_xs(mm, red[q * 64 + (c0 >> 1)]);
+      const GroupScale g0 = group_scale_bf16_sm(fabsf(bf16_lo(mm)), tab);
+      const GroupScale g1 = group_scale_bf16_sm(fabsf(bf16_hi(mm)), tab);
+      if (q4 == 0)
+        *reinterpret_cast<float2*>(s_col + mb * 2 * I + grp * I + nb * 128 + c0) =
+            make_float2(g0.s, g1.s);
+      uint32_t o0[8], o1[8];
+      if (__any_sync(kFull, g0.small || g1.small))
+        col_codes<true, 32>(w, g0, g1, o0, o1);
+      else
+        col_codes<false, 32>(w, g0, g1, o0, o1);
+      // staging (first 16 KB of the box): row c holds column c's 128 codes, 16-byte chunk
+      // k at position k ^ (c & 7) (the 128-byte swizzle)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = c0 + e;
+        const uint32_t* oc = e ? o1 : o0;
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int k = 2 * q4 + k2;
+          *reinterpret_cast<uint4*>(box + c * 128 + ((k ^ (c & 7)) << 4)) =
+              make_uint4(oc[4 * k2], oc[4 * k2 + 1], oc[4 * k2 + 2], oc[4 * k2 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      if (!col_sync()) break;
+      if (lane == 0) {
+        if (cw == 0) {
+          tma_store_2d(&tmQT, box, static_cast<int32_t>(mb * 128),
+                       static_cast<int32_t>(grp * I + nb * 128));
+          tma_store_commit();
+          tma_store_wait_read();  // the stage may be refilled once the store has read it
+          stored = true;
+        }
+        mbar_arrive(empty + b);
+      }
     }
   }
   if (stored && lane == 0) tma_store_wait_all();
@@ -2740,12 +3060,23 @@ extern "C" fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint
       !aligned16(s_row) || !aligned16(q_colT) || !aligned16(s_col))
     return FP8Q_ERR_ALIGN;
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
-  constexpr size_t kSmem = direct_smem_bytes<SwigluBwd>();
-  auto kern = direct_dual_kernel<SwigluBwd, kBwdBatch, kBwdMinBlocks>;
+  if (M >= kMaxTmaCoord || 2 * I >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit coordinates
+  // the gate and the up halves as two [M][I] tensors; the column codes [2I][M]
+  CUtensorMap tmg, tmu, tmqt;
+  if (!encode_tmap_2d(&tmg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu, I, M, I * 4, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu + I, I, M, I * 4, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tmap_2d(&tmqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_colT, M, 2 * I, M, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8Q_ERR_UNSUPPORTED;
+  unsigned* err = device_error_word();
+  if (!err) return FP8Q_ERR_CUDA;
+  auto kern = swiglu_bwd_tile_kernel;
   static std::atomic<int> occ[64];
-  const int per_sm = resident_ctas(kern, 256, kSmem, occ);
-  kern<<<grid_for((M / 128) * (I / 128), per_sm), 256, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      SwigluBwd{gu, dh, I}, M, I, dgu, q_row, s_row, lds_row, q_colT, s_col);
+  const int per_sm = resident_ctas(kern, kA6Threads, kSbSmem, occ);
+  kern<<<grid_for((M / 128) * (I / 128), per_sm), kA6Threads, kSbSmem, static_cast<cudaStream_t>(stream)>>>(
+      tmg, tmu, tmqt, dh, dgu, q_row, M, I, s_row, lds_row, s_col, err, kWaitLimitNs);
   return launch_status("swiglu_bwd_quant_dual launch");
 }
 

@@ -178,7 +178,8 @@ fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int64_t I, int
  * step one IEEE fp32 operation: e = E(-g) (the forward producer's exponential),
  * d = 1 + e, silu = g / d, sig = 1 / d, d_up = bf16(dh * silu),
  * d_gate = bf16((dh * u) * (sig * (1 + g * (1 - sig)))). dgu [M][2I] (BF16) receives
- * the gradient itself if not NULL. Requires I % 128 == 0. */
+ * the gradient itself if not NULL. Requires I % 128 == 0, M < 2^31, 2I < 2^31 (tensor-copy
+ * coordinates; FP8Q_ERR_SHAPE otherwise). */
 fp8q_status fp8q_swiglu_bwd_quant_dual(const uint16_t* gu, const uint16_t* dh, int64_t M,
                                        int64_t I, uint16_t* dgu, uint8_t* q_row, float* s_row,
                                        int64_t lds_row, uint8_t* q_colT, float* s_col,
