@@ -1394,21 +1394,13 @@ __device__ __forceinline__ XTerm xterm(float t) {
 }
 
 // One exact sum per thread: the two bins last added to are cached in registers (the
-// terms of one sum usually span one or two bins); the others live in a separate array
-// `bins` (dynamically indexed, so in local memory), which takes a cached bin when a
-// third one is needed. `mask` has bit b set once bin b may be non-zero in either.
-struct XCache {
-  long long a0, a1;
-  int b0, b1;
-  uint32_t mask;
-  __device__ __forceinline__ void init(long long (&bins)[kXBins]) {
-#pragma unroll
-    for (int i = 0; i < kXBins; ++i) bins[i] = 0;
-    a0 = a1 = 0;
-    b0 = b1 = -1;
-    mask = 0;
-  }
-  __device__ __forceinline__ void add(float t, long long (&bins)[kXBins]) {
+// terms of one sum usually span one or two bins); a bin that leaves the cache goes to
+// spill(bin, value), an atomic add into bins in shared or global memory (rare).
+struct XPair {
+  long long a0 = 0, a1 = 0;
+  int b0 = -1, b1 = -1;
+  template <class Spill>
+  __device__ __forceinline__ void add(float t, Spill&& spill) {
     const XTerm x = xterm(t);
     if (x.v == 0) return;
     if (x.bin == b0) {
@@ -1416,19 +1408,19 @@ struct XCache {
     } else if (x.bin == b1) {
       a1 += x.v;
     } else {
-      if (b1 >= 0) bins[b1] += a1;
+      if (b1 >= 0 && a1 != 0) spill(b1, a1);
       b1 = b0;
       a1 = a0;
       b0 = x.bin;
       a0 = x.v;
-      mask |= 1u << x.bin;
     }
   }
-  // Moves the cached bins into the array (once, after the last add).
-  __device__ __forceinline__ void flush(long long (&bins)[kXBins]) {
-    if (b0 >= 0) bins[b0] += a0;
-    if (b1 >= 0) bins[b1] += a1;
-    b0 = b1 = -1;
+  // bit b set where this lane's cache holds bin b
+  __device__ __forceinline__ uint32_t mask() const {
+    return (b0 >= 0 ? 1u << b0 : 0u) | (b1 >= 0 ? 1u << b1 : 0u);
+  }
+  __device__ __forceinline__ long long value(int b) const {
+    return (b0 == b ? a0 : 0) + (b1 == b ? a1 : 0);
   }
 };
 
@@ -1494,24 +1486,6 @@ __device__ double xbins_round(const long long (&A)[kXBins], bool odd) {
   return __longlong_as_double(static_cast<long long>(bits));
 }
 
-// Sum over the warp of one exact sum per lane, rounded once to a double (the result is
-// returned to every lane).
-__device__ double warp_exact_sum(XCache& acc, long long (&bins)[kXBins], bool odd) {
-  acc.flush(bins);
-  const uint32_t used = __reduce_or_sync(kFull, acc.mask);
-  long long A[kXBins];
-#pragma unroll
-  for (int b = 0; b < kXBins; ++b) A[b] = 0;
-  for (uint32_t m = used; m; m &= m - 1) {
-    const int b = __ffs(m) - 1;
-    long long v = bins[b];
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-    A[b] = v;
-  }
-  return xbins_round(A, odd);
-}
-
 // Per-row scalars of the RMSNorm backward: r (as in the forward producer) and
 // k = (float)((((c r) r) r) / H) in fp64, c = the exact sum of the fp32 products
 // fl32(fl32(gamma_j dy_j) x_j) rounded once to a double. One warp per row.
@@ -1523,13 +1497,17 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
   const int64_t nch = H >> 3;
   const int64_t wglobal = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  // bins evicted from the lanes' register caches, one set per warp
+  __shared__ unsigned long long wbins[8][kXBins];
+  unsigned long long* wb = wbins[threadIdx.x >> 5];
+  auto spill = [&](int b, long long v) { atomicAdd(wb + b, static_cast<unsigned long long>(v)); };
   for (int64_t m = wglobal; m < M; m += nw) {
     const uint16_t* xr = x + m * H;
     const uint16_t* dr = dy + m * H;
     double ss[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-    XCache cc;
-    long long cbins[kXBins];
-    cc.init(cbins);
+    if (lane < kXBins) wb[lane] = 0ull;
+    __syncwarp();
+    XPair cc;
     int64_t c = lane;
     for (; c + 32 < nch; c += 64) {  // two chunks of each operand in flight per lane
       uint4 rx[2], rd[2], rg[2];
@@ -1549,7 +1527,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
         for (int i = 0; i < 8; ++i) {
           const double xd = static_cast<double>(xv[i]);
           ss[i] = __fma_rn(xd, xd, ss[i]);
-          cc.add(__fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]), cbins);
+          cc.add(__fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]), spill);
         }
       }
     }
@@ -1562,14 +1540,27 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
       for (int i = 0; i < 8; ++i) {
         const double xd = static_cast<double>(xv[i]);
         ss[i] = __fma_rn(xd, xd, ss[i]);
-        cc.add(__fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]), cbins);
+        cc.add(__fmul_rn(__fmul_rn(gv[i], dv[i]), xv[i]), spill);
       }
     }
     double s2 = __dadd_rn(__dadd_rn(__dadd_rn(ss[0], ss[1]), __dadd_rn(ss[2], ss[3])),
                           __dadd_rn(__dadd_rn(ss[4], ss[5]), __dadd_rn(ss[6], ss[7])));
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) s2 = __dadd_rn(s2, __shfl_xor_sync(kFull, s2, off));
-    const double c2 = warp_exact_sum(cc, cbins, false);
+    // the cached bins summed over the warp, bin by bin, plus the evicted ones
+    __syncwarp();  // every eviction is in wb
+    long long A[kXBins];
+#pragma unroll
+    for (int b = 0; b < kXBins; ++b) A[b] = static_cast<long long>(wb[b]);
+    for (uint32_t used = __reduce_or_sync(kFull, cc.mask()); used; used &= used - 1) {
+      const int b = __ffs(used) - 1;
+      long long v = cc.value(b);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+      A[b] += v;
+    }
+    __syncwarp();  // wb is read before the next row clears it
+    const double c2 = xbins_round(A, false);
     if (lane == 0) {
       const float r = rstd_from_ss(s2, H, eps);
       const double rd = static_cast<double>(r);
@@ -2348,8 +2339,9 @@ __global__ void __launch_bounds__(kA6Threads, 1) swiglu_bwd_tile_kernel(
 // bins [H][kXBins] with 64-bit integer atomics: integer additions, so the order in which
 // the warps land does not matter.
 constexpr int kDgRows = 64;
+constexpr int kDgBatch = 4;  // rows whose loads are in flight together
 
-__global__ void __launch_bounds__(256) dgamma_exact_kernel(
+__global__ void __launch_bounds__(256, 2) dgamma_exact_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ dy, const float* __restrict__ r,
     int64_t M, int64_t H, unsigned long long* __restrict__ bins) {
   const int lane = threadIdx.x & 31;
@@ -2363,26 +2355,48 @@ __global__ void __launch_bounds__(256) dgamma_exact_kernel(
     const int64_t m0 = (u / strips) * kDgRows;
     const int64_t m1 = m0 + kDgRows < M ? m0 + kDgRows : M;
     if (ch >= nch) continue;  // lanes past the last chunk (H not a multiple of 256)
-    XCache acc[8];
-    long long cbins[8][kXBins];
+    unsigned long long* col = bins + ch * 8 * kXBins;  // this lane's 8 columns' bins
+    XPair acc[8];
+    int64_t m = m0;
+    // kDgBatch rows' loads in flight before their terms are added
+    for (; m + kDgBatch <= m1; m += kDgBatch) {
+      uint4 xr[kDgBatch], dr[kDgBatch];
+      float rm[kDgBatch];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc[q].init(cbins[q]);
-    for (int64_t m = m0; m < m1; ++m) {
+      for (int e = 0; e < kDgBatch; ++e) {
+        xr[e] = ld_nc_v4(x + (m + e) * H + ch * 8);
+        dr[e] = ld_nc_v4(dy + (m + e) * H + ch * 8);
+        rm[e] = __ldg(r + m + e);
+      }
+#pragma unroll
+      for (int e = 0; e < kDgBatch; ++e) {
+        float xv[8], dv[8];
+        unpack_bf16x8(xr[e], xv);
+        unpack_bf16x8(dr[e], dv);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          acc[q].add(__fmul_rn(dv[q], __fmul_rn(xv[q], rm[e])), [&](int b, long long v) {
+            atomicAdd(col + q * kXBins + b, static_cast<unsigned long long>(v));
+          });
+      }
+    }
+    for (; m < m1; ++m) {
       float xv[8], dv[8];
       unpack_bf16x8(ld_nc_v4(x + m * H + ch * 8), xv);
       unpack_bf16x8(ld_nc_v4(dy + m * H + ch * 8), dv);
       const float rm = __ldg(r + m);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q].add(__fmul_rn(dv[q], __fmul_rn(xv[q], rm)), cbins[q]);
+      for (int q = 0; q < 8; ++q)
+        acc[q].add(__fmul_rn(dv[q], __fmul_rn(xv[q], rm)), [&](int b, long long v) {
+          atomicAdd(col + q * kXBins + b, static_cast<unsigned long long>(v));
+        });
     }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      acc[q].flush(cbins[q]);
-      unsigned long long* col = bins + (ch * 8 + q) * kXBins;
-      for (uint32_t mk = acc[q].mask; mk; mk &= mk - 1) {
-        const int b = __ffs(mk) - 1;
-        if (cbins[q][b]) atomicAdd(col + b, static_cast<unsigned long long>(cbins[q][b]));
-      }
+      if (acc[q].b0 >= 0 && acc[q].a0 != 0)
+        atomicAdd(col + q * kXBins + acc[q].b0, static_cast<unsigned long long>(acc[q].a0));
+      if (acc[q].b1 >= 0 && acc[q].a1 != 0)
+        atomicAdd(col + q * kXBins + acc[q].b1, static_cast<unsigned long long>(acc[q].a1));
     }
   }
 }
