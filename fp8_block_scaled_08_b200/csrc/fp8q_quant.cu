@@ -1373,46 +1373,44 @@ __device__ __forceinline__ void swiglu_bwd8_tab(const uint4& gw, const uint4& uw
 // Exact sums of fp32 terms (the two reductions of the RMSNorm backward). A finite fp32
 // value is m * 2^(e - 149) with an integer m < 2^24 and e in [0, 253] (subnormals:
 // e = 0, no implicit bit). Bin b = e / 16 holds integers in units of 2^(16 b - 149); a
-// term adds m << (e % 16) (< 2^39) to its bin. Integer additions are exact, so the
-// bins' total is the exact sum of the terms, whatever order the additions take (with
-// fewer than 2^24 terms no bin can overflow). The total is rounded once at the end.
+// term is m << (e % 16) (< 2^39) of them. Integer additions are exact, so the bins'
+// total is the exact sum of the terms, whatever order the additions take (with fewer
+// than 2^24 terms no bin can overflow). The total is rounded once at the end.
 // ---------------------------------------------------------------------------
 constexpr int kXBins = 16;
 
-struct XTerm {
-  int bin;
-  long long v;
-};
-
-__device__ __forceinline__ XTerm xterm(float t) {
-  const uint32_t u = __float_as_uint(t);
-  const uint32_t E = (u >> 23) & 0xFFu;
-  const uint32_t m = E ? ((u & 0x7FFFFFu) | 0x800000u) : (u & 0x7FFFFFu);
-  const int e = E ? static_cast<int>(E) - 1 : 0;
-  const long long v = static_cast<long long>(m) << (e & 15);
-  return XTerm{e >> 4, (u >> 31) ? -v : v};
-}
-
 // One exact sum per thread: the two bins last added to are cached in registers (the
 // terms of one sum usually span one or two bins); a bin that leaves the cache goes to
-// spill(bin, value), an atomic add into bins in shared or global memory (rare).
+// spill(bin, units), an atomic add into integer bins in shared or global memory (rare).
+// A cached bin is a double: the terms of bin b are integer multiples of its unit
+// 2^(16 b - 149) below 2^39 units, and a double holds every such integer below 2^53
+// exactly, so the fp64 additions of up to 2^14 terms are exact (no rounding) and
+// cheaper than splitting each term into a bin and a 64-bit integer. The integer is
+// formed once, when the bin leaves the cache.
 struct XPair {
-  long long a0 = 0, a1 = 0;
+  double a0 = 0.0, a1 = 0.0;
   int b0 = -1, b1 = -1;
+  // bin b's cached sum in units of 2^(16 b - 149) (an exact scaling by a power of two)
+  static __device__ __forceinline__ long long units(double a, int b) {
+    const double scale = __longlong_as_double(static_cast<long long>(1023 + 149 - 16 * b) << 52);
+    return __double2ll_rn(__dmul_rn(a, scale));
+  }
   template <class Spill>
   __device__ __forceinline__ void add(float t, Spill&& spill) {
-    const XTerm x = xterm(t);
-    if (x.v == 0) return;
-    if (x.bin == b0) {
-      a0 += x.v;
-    } else if (x.bin == b1) {
-      a1 += x.v;
+    if (t == 0.0f) return;
+    const uint32_t E = (__float_as_uint(t) >> 23) & 0xFFu;
+    const int bin = (E ? static_cast<int>(E) - 1 : 0) >> 4;
+    const double d = static_cast<double>(t);
+    if (bin == b0) {
+      a0 = __dadd_rn(a0, d);
+    } else if (bin == b1) {
+      a1 = __dadd_rn(a1, d);
     } else {
-      if (b1 >= 0 && a1 != 0) spill(b1, a1);
+      if (b1 >= 0 && a1 != 0.0) spill(b1, units(a1, b1));
       b1 = b0;
       a1 = a0;
-      b0 = x.bin;
-      a0 = x.v;
+      b0 = bin;
+      a0 = d;
     }
   }
   // bit b set where this lane's cache holds bin b
@@ -1420,7 +1418,7 @@ struct XPair {
     return (b0 >= 0 ? 1u << b0 : 0u) | (b1 >= 0 ? 1u << b1 : 0u);
   }
   __device__ __forceinline__ long long value(int b) const {
-    return (b0 == b ? a0 : 0) + (b1 == b ? a1 : 0);
+    return (b0 == b ? units(a0, b0) : 0) + (b1 == b ? units(a1, b1) : 0);
   }
 };
 
@@ -2338,8 +2336,12 @@ __global__ void __launch_bounds__(kA6Threads, 1) swiglu_bwd_tile_kernel(
 // each of its 8 columns as an exact sum, and adds each column's bins into the global
 // bins [H][kXBins] with 64-bit integer atomics: integer additions, so the order in which
 // the warps land does not matter.
-constexpr int kDgRows = 64;
-constexpr int kDgBatch = 4;  // rows whose loads are in flight together
+#ifndef DG_ROWS
+#define DG_ROWS 64
+#define DG_BATCH 4
+#endif
+constexpr int kDgRows = DG_ROWS;
+constexpr int kDgBatch = DG_BATCH;  // rows whose loads are in flight together
 
 __global__ void __launch_bounds__(256, 2) dgamma_exact_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ dy, const float* __restrict__ r,
@@ -2393,10 +2395,12 @@ __global__ void __launch_bounds__(256, 2) dgamma_exact_kernel(
     }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      if (acc[q].b0 >= 0 && acc[q].a0 != 0)
-        atomicAdd(col + q * kXBins + acc[q].b0, static_cast<unsigned long long>(acc[q].a0));
-      if (acc[q].b1 >= 0 && acc[q].a1 != 0)
-        atomicAdd(col + q * kXBins + acc[q].b1, static_cast<unsigned long long>(acc[q].a1));
+      if (acc[q].b0 >= 0 && acc[q].a0 != 0.0)
+        atomicAdd(col + q * kXBins + acc[q].b0,
+                  static_cast<unsigned long long>(XPair::units(acc[q].a0, acc[q].b0)));
+      if (acc[q].b1 >= 0 && acc[q].a1 != 0.0)
+        atomicAdd(col + q * kXBins + acc[q].b1,
+                  static_cast<unsigned long long>(XPair::units(acc[q].a1, acc[q].b1)));
     }
   }
 }
@@ -3098,10 +3102,13 @@ namespace {
 int64_t rmsnorm_bwd_ws_scalars(int64_t M) { return (8 * M + 255) / 256 * 256; }
 // dgamma's exact bins hold fewer than 2^23 terms of < 2^39 each: no int64 overflow
 constexpr int64_t kRmsBwdMaxRows = int64_t{1} << 23;
+// a lane's cached fp64 bin of a row's sum takes at most H / 32 terms: exact up to 2^14
+constexpr int64_t kRmsBwdMaxCols = int64_t{1} << 19;
 }  // namespace
 
 extern "C" int64_t fp8q_rmsnorm_bwd_workspace_bytes(int64_t M, int64_t H) {
-  if (M <= 0 || H <= 0 || M % 128 || H % 128 || M > kRmsBwdMaxRows) return -1;
+  if (M <= 0 || H <= 0 || M % 128 || H % 128 || M > kRmsBwdMaxRows || H > kRmsBwdMaxCols)
+    return -1;
   return rmsnorm_bwd_ws_scalars(M) + H * kXBins * 8;
 }
 
@@ -3113,7 +3120,7 @@ extern "C" fp8q_status fp8q_rmsnorm_bwd_quant_dual(
   if (!x || !gamma || !dy || !out || !q_row || !s_row || !q_colT || !s_col || !workspace)
     return FP8Q_ERR_NULL;
   if (M <= 0 || H <= 0 || M % 128 || H % 128 || lds_row < M || lds_row % 4 || !(eps >= 0.0f) ||
-      M > kRmsBwdMaxRows)
+      M > kRmsBwdMaxRows || H > kRmsBwdMaxCols)
     return FP8Q_ERR_SHAPE;
   if (workspace_bytes < fp8q_rmsnorm_bwd_workspace_bytes(M, H)) {
     set_last_error_text("rmsnorm_bwd_quant_dual: workspace smaller than "

@@ -207,7 +207,7 @@ int64_t fp8q_rmsnorm_bwd_workspace_bytes(int64_t M, int64_t H);
  * workspace: device memory of fp8q_rmsnorm_bwd_workspace_bytes(M, H) bytes, 16-byte
  * aligned, used only during the call's kernels (calls sharing one workspace must be
  * ordered on one stream; it needs no initialisation). Requires H % 128 == 0, eps >= 0,
- * M <= 2^23 (FP8Q_ERR_SHAPE otherwise). */
+ * M <= 2^23, H <= 2^19 (FP8Q_ERR_SHAPE otherwise). */
 fp8q_status fp8q_rmsnorm_bwd_quant_dual(const uint16_t* x, const uint16_t* gamma,
                                         const uint16_t* dy, const uint16_t* dres, int64_t M,
                                         int64_t H, float eps, uint16_t* out, uint8_t* q_row,

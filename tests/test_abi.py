@@ -152,6 +152,8 @@ def test_validation_backward_producers():
     assert need == 2048 + 512 * 16 * 8                                  # r, k, dgamma's bins
     assert call("fp8q_rmsnorm_bwd_workspace_bytes", 100, 512) == -1
     assert call("fp8q_rmsnorm_bwd_workspace_bytes", (1 << 23) + 128, 512) == -1   # M too large
+    assert call("fp8q_rmsnorm_bwd_workspace_bytes", 256, (1 << 19) + 128) == -1   # H too large
+    assert call("fp8q_rmsnorm_bwd_workspace_bytes", 256, 1 << 19) > 0
     ok = (A, B, C, NUL, 256, 512, F(1e-5), D, E, A, 256, B, C, NUL, W)
     assert call(g, *ok, need - 1, NUL) == 2                                        # workspace
     assert call(g, A, B, C, NUL, 256, 512, F(-1.0), D, E, A, 256, B, C, NUL, W, need, NUL) == 2
