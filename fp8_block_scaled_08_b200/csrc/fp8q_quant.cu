@@ -1208,10 +1208,10 @@ __device__ __forceinline__ void tiles_drain(const TileSmem& sm, int64_t t_stop, 
 
 // ---------------------------------------------------------------------------
 // Option B for saved activations (the producer emits both groupings from BF16, no FP8
-// requantization): the producer's BF16 output is formed 128 x 128 tile by tile inside
-// a6_tile_kernel, with TileRms / TileSwiglu as the source (the row warps form the tile in
-// shared memory, then both groupings are quantized from it); the RMSNorm needs its
-// per-row reciprocal RMS first.
+// requantization): the producer's BF16 output is formed 128 x 128 tile by tile in shared
+// memory and both groupings are quantized from it: the RMSNorm inside a6_tile_kernel
+// with the TileRms source (after its per-row reciprocal RMS), the SwiGLU by
+// swiglu_dual_tile_kernel.
 // ---------------------------------------------------------------------------
 
 // Per-row reciprocal RMS, r = (float)(1/sqrt(ss/H + eps)) with the fp64 sum of squares
@@ -1788,8 +1788,7 @@ struct A6Layout {
   static constexpr uint32_t kOffRed = kOffRow + 128 * 128;    // [4][64] partial maxima
   static constexpr uint32_t kOffTab = kOffRed + 4 * 64 * 4;  // scale and reciprocal tables
   static constexpr uint32_t kOffBar = kOffTab + 256 * 4;     // full, empty, formed, csync
-  static constexpr uint32_t kOffGateTab = kOffBar + (3 * kStages + 1) * 8 + 16;
-  static constexpr size_t kSmem = 1024 + kOffGateTab + (Src::kTable ? kSgEntries * 4 : 0);
+  static constexpr size_t kSmem = 1024 + kOffBar + (3 * kStages + 1) * 8 + 16;
 };
 template <class Src>
 constexpr size_t a6_smem() {
@@ -1802,7 +1801,6 @@ constexpr size_t a6_smem() {
 struct TileGrad {  // a6: the BF16 gradient itself (no forming step)
   static constexpr int kBoxes = 1;
   static constexpr bool kForm = false;
-  static constexpr bool kTable = false;
 };
 
 struct TileRms {  // option B, RMSNorm: y = bf16(fl32(fl32(x r) g)), r from the pre-pass
@@ -1810,11 +1808,10 @@ struct TileRms {  // option B, RMSNorm: y = bf16(fl32(fl32(x r) g)), r from the 
   const uint16_t* gamma;
   static constexpr int kBoxes = 1;
   static constexpr bool kForm = true;
-  static constexpr bool kTable = false;
   __device__ __forceinline__ float row_factor(int64_t m) const { return __ldg(rstd + m); }
   // 8 values at x0 (staged), output columns col .. col + 7
-  __device__ __forceinline__ uint4 form(const uint16_t* x0, const uint16_t*, int64_t col, float r,
-                                        const float*) const {
+  __device__ __forceinline__ uint4 form(const uint16_t* x0, const uint16_t*, int64_t col,
+                                        float r) const {
     float xv[8], gv[8], b[8];
     unpack_bf16x8(*reinterpret_cast<const uint4*>(x0), xv);
     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(gamma + col)), gv);
@@ -1829,19 +1826,6 @@ struct TileRms {  // option B, RMSNorm: y = bf16(fl32(fl32(x r) g)), r from the 
   }
 };
 
-struct TileSwiglu {  // option B, SwiGLU: h = bf16(fl32(sg(g) u)), gate and up staged
-  static constexpr int kBoxes = 2;
-  static constexpr bool kForm = true;
-  static constexpr bool kTable = true;
-  __device__ __forceinline__ float row_factor(int64_t) const { return 0.0f; }
-  __device__ __forceinline__ uint4 form(const uint16_t* g0, const uint16_t* u0, int64_t, float,
-                                        const float* tab) const {
-    float v[8];
-    SwigluBoxes::values(g0, u0, 0, tab, v);
-    return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                      pack_bf16x2(v[6], v[7]));
-  }
-};
 
 // Group maximum from a lane's four running bf16x2 maxima and its partner's (lane ^ 16).
 __device__ __forceinline__ float half_row_amax_finish(const uint32_t (&m)[4]) {
@@ -1895,14 +1879,12 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
   uint64_t* formed = empty + kStages;  // kForm: the eight row warps have written the tile
   uint64_t* csync = formed + kStages;  // the column warps' rendezvous (bounded, unlike bar.sync)
   int* abort_flag = reinterpret_cast<int*>(csync + 1);
-  float* gtab = reinterpret_cast<float*>(base + L::kOffGateTab);  // Src::kTable
   const WaitCtl ctl{abort_flag, err, limit_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < 128) {
     tab[threadIdx.x] = kScaleMant[threadIdx.x];
     tab[128 + threadIdx.x] = kRecipMant[threadIdx.x];
   }
-  if (Src::kTable) sg_table_fill(gtab);
   if (threadIdx.x == 0) {
     for (int b = 0; b < kStages; ++b) {
       mbar_init(full + b, 1);
@@ -1974,7 +1956,7 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int off = ((j + lane) & 7) * 8;
-          w[j] = src.form(row + off, row1 + off, nb * 128 + hh * 64 + off, rf, gtab);
+          w[j] = src.form(row + off, row1 + off, nb * 128 + hh * 64 + off, rf);
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(row + ((j + lane) & 7) * 8) = w[j];
@@ -2073,6 +2055,202 @@ __global__ void __launch_bounds__(kA6Threads, 1) a6_tile_kernel(
         tma_store_commit();
       }
       stored = true;
+    }
+  }
+  if (stored && lane == 0) tma_store_wait_all();
+}
+
+// ---------------------------------------------------------------------------
+// Option B's SwiGLU producer (f2): h = bf16(fl32(sg(g) u)) in both groupings, on the
+// layout of the SwiGLU backward's kernel below: a stage holds the gate and up boxes of a
+// 128 x 128 tile (two stages), sg comes from a4's per-CTA table, and all sixteen
+// consumer warps form eight rows each (four lanes per row, chunks rotated by the row),
+// write h over the gate box, store their rows' codes from registers and arrive on
+// `formed`; then every warp quantizes 16 rows x 2 columns of the tile (warp w: rows
+// 16 (w % 8) .. +15, column pairs 64 (w / 8) + 2 lane), the eight partial maxima of a
+// column meet in shared memory, and the transposed codes are staged over the first half
+// of the gate box for one tensor store.
+// ---------------------------------------------------------------------------
+constexpr int kSfStages = 2;
+constexpr uint32_t kSfStageBytes = 2 * kA6Tile;               // gate and up boxes
+constexpr uint32_t kSfOffGate = kSfStages * kSfStageBytes;    // sg per gate
+constexpr uint32_t kSfOffRed = kSfOffGate + kSgEntries * 4;   // [8][64] partial maxima
+constexpr uint32_t kSfOffTab = kSfOffRed + 8 * 64 * 4;        // scale and reciprocal tables
+constexpr uint32_t kSfOffBar = kSfOffTab + 256 * 4;           // full, empty, formed, csync
+constexpr size_t kSfSmem = 1024 + kSfOffBar + (3 * kSfStages + 1) * 8 + 16;
+
+__global__ void __launch_bounds__(kA6Threads, 1) swiglu_dual_tile_kernel(
+    const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmU,
+    const __grid_constant__ CUtensorMap tmQT, uint8_t* __restrict__ q_row, int64_t M, int64_t I,
+    float* __restrict__ s_row, int64_t lds_row, float* __restrict__ s_col, unsigned* err,
+    uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float* gtab = reinterpret_cast<float*>(base + kSfOffGate);
+  float* tab = reinterpret_cast<float*>(base + kSfOffTab);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kSfOffBar);
+  uint64_t* empty = full + kSfStages;
+  uint64_t* formed = empty + kSfStages;  // all sixteen warps have formed their rows
+  uint64_t* csync = formed + kSfStages;  // the sixteen warps' column rendezvous
+  int* abort_flag = reinterpret_cast<int*>(csync + 1);
+  const WaitCtl ctl{abort_flag, err, limit_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < 128) {
+    tab[threadIdx.x] = kScaleMant[threadIdx.x];
+    tab[128 + threadIdx.x] = kRecipMant[threadIdx.x];
+  }
+  sg_table_fill(gtab);
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < kSfStages; ++b) {
+      mbar_init(full + b, 1);
+      mbar_init(empty + b, 16);
+      mbar_init(formed + b, 16);
+    }
+    mbar_init(csync, 16);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int64_t NB = I >> 7;
+  const int64_t tiles = (M >> 7) * NB;
+  if (warp == 16) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0, par = 0;
+      bool ok = true;
+      int i = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int b = i % kSfStages;
+        const uint32_t ph = static_cast<uint32_t>(i / kSfStages) & 1u;
+        if (i >= kSfStages && !mbar_wait(empty + b, ph ^ 1u, ctl)) { ok = false; break; }
+        const int64_t mb = t / NB, nb = t - mb * NB;
+        const int32_t x = static_cast<int32_t>(nb * 128), y = static_cast<int32_t>(mb * 128);
+        uint8_t* st = base + b * kSfStageBytes;
+        mbar_arrive_expect_tx(full + b, kSfStageBytes);
+        tma_load_2d(st, &tmG, x, y, full + b);
+        tma_load_2d(st + kA6Tile, &tmU, x, y, full + b);
+        issued |= 1u << b;
+        par = (par & ~(1u << b)) | (ph << b);
+      }
+      if (!ok) {  // let every copy already issued land before the CTA exits
+        for (int b = 0; b < kSfStages; ++b) {
+          if (!((issued >> b) & 1u)) continue;
+          const uint32_t a = smem_u32(full + b);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, (par >> b) & 1u))
+            if (global_timer_ns() - t0 > limit_ns) break;
+        }
+      }
+    }
+    return;
+  }
+  // row phase: tile row r = 8 warp + lr, chunks (a + 4k + 4 (lr % 4)) % 16, k = 0 .. 3
+  const int lr = lane >> 2, a = lane & 3;
+  const int r = warp * 8 + lr;
+  auto chunk = [&](int k) { return (a + 4 * k + 4 * (lr & 3)) & 15; };
+  // column phase: rows 16 q8 .. +15, column pair c0, c0 + 1
+  const int q8 = warp & 7;
+  const int c0 = 64 * (warp >> 3) + 2 * lane;
+  uint32_t* red = reinterpret_cast<uint32_t*>(base + kSfOffRed);
+  uint32_t nsync = 0;
+  auto col_sync = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(csync);
+    return mbar_wait_warp(csync, (nsync++) & 1u, ctl);
+  };
+  bool stored = false;
+  int i = 0;
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+    const int b = i % kSfStages;
+    const uint32_t ph = static_cast<uint32_t>(i / kSfStages) & 1u;
+    if (!mbar_wait_warp(full + b, ph, ctl)) break;
+    const int64_t mb = t / NB, nb = t - mb * NB;
+    uint8_t* st = base + b * kSfStageBytes;
+    // ---------------------------------------------------------------- rows
+    {
+      uint16_t* rg = reinterpret_cast<uint16_t*>(st) + r * 128;
+      const uint16_t* ru = reinterpret_cast<const uint16_t*>(st + kA6Tile) + r * 128;
+      uint4 h[4];
+      uint32_t mh[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int off = chunk(k) * 8;
+        float v[8];
+        SwigluBoxes::values(rg, ru, off, gtab, v);
+        h[k] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+        *reinterpret_cast<uint4*>(rg + off) = h[k];
+        mh[0] = bf16x2_maxabs_xs(mh[0], h[k].x);
+        mh[1] = bf16x2_maxabs_xs(mh[1], h[k].y);
+        mh[2] = bf16x2_maxabs_xs(mh[2], h[k].z);
+        mh[3] = bf16x2_maxabs_xs(mh[3], h[k].w);
+      }
+      fence_proxy_async_smem();  // the stage is written by tensor copies and read by a store later
+      __syncwarp();
+      if (lane == 0) mbar_arrive(formed + b);  // release: the column pass may read the rows
+      // the row's four lanes are adjacent: two shuffles give its maximum
+      uint32_t hm = bf16x2_maxabs_xs(bf16x2_maxabs_xs(mh[0], mh[1]), bf16x2_maxabs_xs(mh[2], mh[3]));
+      hm = bf16x2_maxabs_xs(hm, __shfl_xor_sync(kFull, hm, 1));
+      hm = bf16x2_maxabs_xs(hm, __shfl_xor_sync(kFull, hm, 2));
+      const GroupScale g = group_scale_bf16_sm(bf16x2_hmax_abs(hm), tab);
+      const int64_t m = mb * 128 + r;
+      uint8_t* qr = q_row + m * I + nb * 128;
+      if (__any_sync(kFull, g.small)) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint2*>(qr + chunk(k) * 8) = codes8_words<true>(h[k], g);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint2*>(qr + chunk(k) * 8) = codes8_words<false>(h[k], g);
+      }
+      if (a == 0) s_row[nb * lds_row + m] = g.s;
+    }
+    if (!mbar_wait_warp(formed + b, ph, ctl)) break;
+    // ---------------------------------------------------------------- columns
+    {
+      const uint32_t* tw = reinterpret_cast<const uint32_t*>(st) + q8 * 16 * 64 + (c0 >> 1);
+      uint32_t w[16];  // columns c0, c0 + 1 of rows 16 q8 + k
+#pragma unroll
+      for (int k = 0; k < 16; ++k) w[k] = tw[k * 64];
+      uint32_t m0 = 0u, m1 = 0u;
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        m0 = bf16x2_maxabs_xs(m0, w[k]);
+        m1 = bf16x2_maxabs_xs(m1, w[k + 1]);
+      }
+      red[q8 * 64 + (c0 >> 1)] = bf16x2_maxabs_xs(m0, m1);
+      if (!col_sync()) break;  // every warp's reads of the tile are done: it may be overwritten
+      uint32_t mm = 0u;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mm = bf16x2_maxabs_xs(mm, red[q * 64 + (c0 >> 1)]);
+      const GroupScale g0 = group_scale_bf16_sm(fabsf(bf16_lo(mm)), tab);
+      const GroupScale g1 = group_scale_bf16_sm(fabsf(bf16_hi(mm)), tab);
+      if (q8 == 0)
+        *reinterpret_cast<float2*>(s_col + mb * I + nb * 128 + c0) = make_float2(g0.s, g1.s);
+      uint32_t o0[4], o1[4];
+      if (__any_sync(kFull, g0.small || g1.small))
+        col_codes<true, 16>(w, g0, g1, o0, o1);
+      else
+        col_codes<false, 16>(w, g0, g1, o0, o1);
+      // staging (first 16 KB of the gate box): row c holds column c's 128 codes, 16-byte
+      // chunk q8 at position q8 ^ (c & 7) (the 128-byte swizzle)
+      *reinterpret_cast<uint4*>(st + c0 * 128 + ((q8 ^ (c0 & 7)) << 4)) =
+          make_uint4(o0[0], o0[1], o0[2], o0[3]);
+      *reinterpret_cast<uint4*>(st + (c0 + 1) * 128 + ((q8 ^ ((c0 + 1) & 7)) << 4)) =
+          make_uint4(o1[0], o1[1], o1[2], o1[3]);
+      fence_proxy_async_smem();
+      if (!col_sync()) break;  // (red is free again too)
+      if (lane == 0) {
+        if (warp == 0) {
+          tma_store_2d(&tmQT, st, static_cast<int32_t>(mb * 128), static_cast<int32_t>(nb * 128));
+          tma_store_commit();
+          tma_store_wait_read();  // the stage may be refilled once the store has read it
+          stored = true;
+        }
+        mbar_arrive(empty + b);
+      }
     }
   }
   if (stored && lane == 0) tma_store_wait_all();
@@ -3047,24 +3225,21 @@ extern "C" fp8q_status fp8q_swiglu_quant_dual(const uint16_t* gu, int64_t M, int
   if (!sm100_sm_count()) return FP8Q_ERR_UNSUPPORTED;
   if (M >= kMaxTmaCoord || I >= kMaxTmaCoord) return FP8Q_ERR_SHAPE;  // 32-bit coordinates
   // the gate and the up halves as two [M][I] tensors
-  CUtensorMap tmg, tmu, tmq, tmqt;
+  CUtensorMap tmg, tmu, tmqt;
   if (!encode_tmap_2d(&tmg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu, I, M, ldgu * 2, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_tmap_2d(&tmu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gu + I, I, M, ldgu * 2, 128, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_tmap_2d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_row, I, M, I, 128, 16,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_tmap_2d(&tmqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_colT, M, I, M, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_UNSUPPORTED;
   unsigned* err = device_error_word();
   if (!err) return FP8Q_ERR_CUDA;
-  constexpr size_t kSmem = a6_smem<TileSwiglu>();
-  auto kern = a6_tile_kernel<TileSwiglu, true>;
+  auto kern = swiglu_dual_tile_kernel;
   static std::atomic<int> occ[64];
-  const int per_sm = resident_ctas(kern, kA6Threads, kSmem, occ);
-  kern<<<grid_for((M / 128) * (I / 128), per_sm), kA6Threads, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      tmg, tmu, tmq, tmqt, TileSwiglu{}, M, I, s_row, lds_row, s_col, err, kWaitLimitNs);
+  const int per_sm = resident_ctas(kern, kA6Threads, kSfSmem, occ);
+  kern<<<grid_for((M / 128) * (I / 128), per_sm), kA6Threads, kSfSmem, static_cast<cudaStream_t>(stream)>>>(
+      tmg, tmu, tmqt, q_row, M, I, s_row, lds_row, s_col, err, kWaitLimitNs);
   return launch_status("swiglu_quant_dual launch");
 }
 
