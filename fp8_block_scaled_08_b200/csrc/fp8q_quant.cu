@@ -321,19 +321,20 @@ __device__ __forceinline__ void exp_cw2(float x0, float x1, float& e0, float& e1
 
 // ---------------------------------------------------------------------------
 // Row-group quantizer of SwiGLU (a4), fed by tensor copies. A unit is a box of kRgRows
-// rows x one 128-column group of the gate and the same of the up half (2 x 16 KB of
+// rows x one 128-column group of the gate and the same of the up half (2 x 32 KB of
 // BF16). A persistent CTA has one producer warp that keeps up to kStages units in flight
-// through a ring in shared memory, and kConsumers consumer warps, each quantizing its
-// share of the box's rows two at a time (a half-warp per row, lane l owning columns
-// 8*(l%16) .. +7). The gate factor comes from a per-CTA table (see sg_index). A box past
-// a ragged M or K arrives zero-filled (zeros raise no group maximum) and only its valid
+// through a ring in shared memory, and kConsumers consumer warps, each quantizing eight
+// rows of the box (four lanes per row, 32 values a lane: the row maximum takes two
+// shuffles and the scale is formed once per 32 values; a half-warp per row measured 3 %
+// slower). The gate factor comes from a per-CTA table (see sg_index). A box past a
+// ragged M or K arrives zero-filled (zeros raise no group maximum) and only its valid
 // rows and columns are stored.
 // ---------------------------------------------------------------------------
 #ifndef A4_STAGES
 #define A4_STAGES 2
 #define A4_CONS 16
 #endif
-constexpr int kRgRows = 64;
+constexpr int kRgRows = 8 * A4_CONS;  // eight rows per consumer warp
 constexpr uint32_t kRgBoxBytes = kRgRows * 128 * 2;
 template <int kConsumers>
 constexpr int rg_threads() { return 32 * (kConsumers + 1); }
@@ -406,10 +407,16 @@ struct SwigluBoxes {  // a4: h = SwiGLU(gate, up) from the gate box and the up b
   }
 };
 
+// (defined with the lane-per-group quantizers below)
+__device__ __forceinline__ uint32_t bf16x2_maxabs_xs(uint32_t a, uint32_t b);
+__device__ __forceinline__ float bf16x2_hmax_abs(uint32_t m);
+template <bool kSmall>
+__device__ __forceinline__ uint2 codes8_words(const uint4& w, const GroupScale& g);
+
 template <class B, int kStages>
 constexpr size_t rowgroup_tma_smem() {
   return 1024 + static_cast<size_t>(kStages) * B::kBoxes * kRgBoxBytes + 2 * kStages * 8 + 16 +
-         kSgEntries * 4;
+         kSgEntries * 4 + 256 * 4;
 }
 
 // M rows, G = ceil(K / 128) groups of K valid columns; codes q[m * ldq + k], scales
@@ -438,7 +445,9 @@ __global__ void __launch_bounds__(rg_threads<kConsumers>()) rowgroup_tma_kernel(
     *abort_flag = 0;
     fence_barrier_init();
   }
+  float* stab = tab + kSgEntries;  // scale and reciprocal tables
   sg_table_fill(tab);
+  scale_tables_fill(stab);
   __syncthreads();
   // unit u = (row box) * G + group; the host keeps the unit count below 2^31
   const uint32_t units = static_cast<uint32_t>(((M + kRgRows - 1) / kRgRows) * G);
@@ -475,32 +484,52 @@ __global__ void __launch_bounds__(rg_threads<kConsumers>()) rowgroup_tma_kernel(
     return;
   }
   // -------------------------------------------------------------- consumers
-  const int half = lane >> 4, sub = lane & 15;
+  // lane l of consumer warp w: row 8w + l / 4 of the unit, the four 8-column chunks
+  // (l % 4) + 4k rotated by the row (no two lanes of a shared-memory phase in one bank)
+  static_assert(kRgRows == 8 * kConsumers, "eight rows per consumer warp");
+  const int lr = lane >> 2, a = lane & 3;
+  const int r = warp * 8 + lr;
   int i = 0;
   for (uint32_t t = blockIdx.x; t < units; t += gridDim.x, ++i) {
     const int st = i % kStages;
     if (!mbar_wait_warp(full + st, static_cast<uint32_t>(i / kStages) & 1u, ctl)) break;
-    const uint16_t* b0 = reinterpret_cast<const uint16_t*>(base + st * kStageBytes);
+    const uint16_t* b0 = reinterpret_cast<const uint16_t*>(base + st * kStageBytes) + r * 128;
     const uint16_t* b1 = b0 + kRgRows * 128;
     const uint32_t tb = t / G32;
     const int64_t g = t - tb * G32;
-    const int64_t m0 = static_cast<int64_t>(tb) * kRgRows;
-    const bool col_ok = g * 128 + sub * 8 < K;
+    const int64_t m = static_cast<int64_t>(tb) * kRgRows + r;
+    uint4 h[4];
+    uint32_t mh[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int step = 0; step < kRgRows / kConsumers / 2; ++step) {
-      const int r = warp * (kRgRows / kConsumers) + 2 * step + half;
+    for (int k = 0; k < 4; ++k) {
       float v[8];
-      B::values(b0, b1, r * 128 + sub * 8, tab, v);
-      uint2 codes;
-      const float sc = quant_half_warp(v, codes);  // every lane takes part
-      const int64_t m = m0 + r;
-      if (m < M) {
-        if (col_ok) *reinterpret_cast<uint2*>(q + m * ldq + g * 128 + sub * 8) = codes;
-        if (sub == 0) s[g * lds + m] = sc;
-      }
+      B::values(b0, b1, ((a + 4 * k + 4 * (lr & 3)) & 15) * 8, tab, v);
+      h[k] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                        pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+      mh[0] = bf16x2_maxabs_xs(mh[0], h[k].x);
+      mh[1] = bf16x2_maxabs_xs(mh[1], h[k].y);
+      mh[2] = bf16x2_maxabs_xs(mh[2], h[k].z);
+      mh[3] = bf16x2_maxabs_xs(mh[3], h[k].w);
     }
-    __syncwarp();
+    __syncwarp();  // every lane's reads of the stage are complete (their values are used)
     if (lane == 0) mbar_arrive(empty + st);  // this warp is done with the stage
+    // the row's four lanes are adjacent: two shuffles give its maximum
+    uint32_t hm = bf16x2_maxabs_xs(bf16x2_maxabs_xs(mh[0], mh[1]), bf16x2_maxabs_xs(mh[2], mh[3]));
+    hm = bf16x2_maxabs_xs(hm, __shfl_xor_sync(kFull, hm, 1));
+    hm = bf16x2_maxabs_xs(hm, __shfl_xor_sync(kFull, hm, 2));
+    const GroupScale gs = group_scale_bf16_sm(bf16x2_hmax_abs(hm), stab);
+    const bool small = __any_sync(kFull, gs.small);
+    if (m < M) {
+      uint8_t* qr = q + m * ldq + g * 128;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = ((a + 4 * k + 4 * (lr & 3)) & 15) * 8;
+        if (g * 128 + c < K)  // K is a multiple of 16: a chunk is in or out
+          *reinterpret_cast<uint2*>(qr + c) =
+              small ? codes8_words<true>(h[k], gs) : codes8_words<false>(h[k], gs);
+      }
+      if (a == 0) s[g * lds + m] = gs.s;
+    }
   }
 }
 
